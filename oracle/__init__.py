@@ -1,0 +1,346 @@
+"""Plain CPU oracle of the HyperQuant quantize / dequantize path (test infrastructure).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` import this package.  The product library
+(``lattice_entropy_coded_b200``) never imports it and shares no code with it.
+
+The arithmetic lives in ``hqref.c`` (plain C99, strict IEEE fp32, no FMA
+contraction); this module compiles it with gcc on first use and marshals numpy
+arrays through ctypes.  Every function here is argument marshalling only.
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes as C
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hqref.c")
+_HDR = os.path.join(_HERE, "hqref.h")
+_LIB = os.path.join(_HERE, "libhqref.so")
+CFLAGS = ["-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fno-builtin", "-shared", "-fPIC"]
+
+Z, A2, D4, E8 = 0, 1, 2, 3
+LATTICES = {"Z": Z, "A2": A2, "D4": D4, "E8": E8}
+DIM = {Z: 1, A2: 2, D4: 4, E8: 8}
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile hqref.c into libhqref.so (gcc, strict fp32); returns the path."""
+    stale = (not os.path.exists(_LIB)) or any(
+        os.path.getmtime(p) > os.path.getmtime(_LIB) for p in (_SRC, _HDR))
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = _bind(C.CDLL(build()))
+    return _lib
+
+
+@contextlib.contextmanager
+def using_library(path: str):
+    """Temporarily route every oracle call through another build of hqref.c
+    (used by the tests that plant a mistake in a copy of the oracle)."""
+    global _lib
+    lib()
+    old = _lib
+    _lib = _bind(C.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = old
+
+
+def build_variant(src_text: str, out_path: str) -> str:
+    """Compile a modified copy of hqref.c (same flags) to out_path."""
+    d = os.path.dirname(out_path)
+    src = os.path.join(d, "hqref_variant.c")
+    with open(src, "w") as f:
+        f.write(src_text)
+    subprocess.run(["gcc", *CFLAGS, "-I", _HERE, "-o", out_path, src, "-lm"], check=True)
+    return out_path
+
+
+def source() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+_p = C.c_void_p
+_i32, _i64, _u32, _u64, _f32 = C.c_int, C.c_int64, C.c_uint32, C.c_uint64, C.c_float
+
+
+def _bind(L):
+    sig = {
+        "hqref_splitmix64": (_u64, [_u64, _u64]),
+        "hqref_sign": (_i32, [_u64, _u64]),
+        "hqref_bf16_to_f32": (_f32, [C.c_uint16]),
+        "hqref_f32_to_bf16": (C.c_uint16, [_f32]),
+        "hqref_fwht128": (None, [_p]),
+        "hqref_scale_fwd": (_f32, [_f32]),
+        "hqref_scale_inv": (_f32, [_f32]),
+        "hqref_lattice_dim": (_i32, [_i32]),
+        "hqref_decode": (None, [_i32, _p, _p]),
+        "hqref_point": (None, [_i32, _p, _p]),
+        "hqref_is_member": (_i32, [_i32, _p]),
+        "hqref_dither_uniform": (_f32, [_u64, _u64]),
+        "hqref_dither_block": (None, [_i32, _u64, _u64, _p]),
+        "hqref_strip": (None, [_i32, _p, _p, _p]),
+        "hqref_reinsert": (None, [_i32, _p, _u32, _p]),
+        "hqref_zigzag": (_u32, [C.c_int32]),
+        "hqref_unzigzag": (C.c_int32, [_u32]),
+        "hqref_rice_concat": (_u64, [_p, _i64, _i32, _p, _u64]),
+        "hqref_rice_concat_decode": (_i32, [_p, _u64, _i64, _i32, _p]),
+        "hqref_encode_chunk": (_u64, [_i32, _i32, _p, _i32, _p, _u64, _p]),
+        "hqref_decode_chunk": (_i32, [_i32, _i32, _p, _u64, _i32, _p]),
+        "hqref_quantize_tile": (None, [_p, _i32, _f32, _u64, _u64, _i32, _u64, _p]),
+        "hqref_dequantize_tile": (None, [_p, _i32, _f32, _u64, _u64, _i32, _u64, _p]),
+        "hqref_n_chunks": (_i64, [_i64, _i64]),
+        "hqref_quantize": (_i64, [_p, _i64, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _i64, _i64, _p, _u64,
+                                  _p, _p]),
+        "hqref_dequantize": (_i32, [_p, _p, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _i64, _i64, _i32, _p,
+                                    _i64]),
+        "hqref_kv_append": (_i64, [_p, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _p, _u64,
+                                   _u64, _p, _p]),
+        "hqref_kv_read_append": (_i32, [_p, _p, _i64, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _i32, _p,
+                                        _i64, _i64, _i64]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"] or a.ndim == 0
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def _as_u16(x) -> np.ndarray:
+    """bf16 data as a uint16 numpy array (accepts a torch bf16 tensor or uint16 array)."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch
+    assert x.dtype == torch.bfloat16
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+# ---------------------------------------------------------------- scalar pieces
+def splitmix64(s: int, i: int) -> int:
+    return int(lib().hqref_splitmix64(s & (2**64 - 1), i & (2**64 - 1)))
+
+
+def sign(seed: int, j: int) -> int:
+    return int(lib().hqref_sign(seed, j))
+
+
+def bf16_to_f32(b: int) -> float:
+    return float(lib().hqref_bf16_to_f32(b))
+
+
+def f32_to_bf16(f: float) -> int:
+    return int(lib().hqref_f32_to_bf16(f))
+
+
+def fwht128(v) -> np.ndarray:
+    a = np.array(v, dtype=np.float32).copy()
+    assert a.shape == (128,)
+    lib().hqref_fwht128(_ptr(a))
+    return a
+
+
+def scale_fwd(alpha: float) -> float:
+    return float(lib().hqref_scale_fwd(alpha))
+
+
+def scale_inv(alpha: float) -> float:
+    return float(lib().hqref_scale_inv(alpha))
+
+
+def decode(lat: int, v) -> np.ndarray:
+    a = np.ascontiguousarray(v, dtype=np.float32)
+    assert a.shape == (DIM[lat],)
+    q = np.zeros(DIM[lat], dtype=np.int32)
+    lib().hqref_decode(lat, _ptr(a), _ptr(q))
+    return q
+
+
+def point(lat: int, q) -> np.ndarray:
+    a = np.ascontiguousarray(q, dtype=np.int32)
+    p = np.zeros(DIM[lat], dtype=np.float32)
+    lib().hqref_point(lat, _ptr(a), _ptr(p))
+    return p
+
+
+def is_member(lat: int, q) -> bool:
+    a = np.ascontiguousarray(q, dtype=np.int32)
+    return bool(lib().hqref_is_member(lat, _ptr(a)))
+
+
+def dither_uniform(seed: int, e: int) -> float:
+    return float(lib().hqref_dither_uniform(seed, e))
+
+
+def dither_block(lat: int, seed: int, e0: int) -> np.ndarray:
+    d = np.zeros(DIM[lat], dtype=np.float32)
+    lib().hqref_dither_block(lat, seed, e0, _ptr(d))
+    return d
+
+
+def strip(lat: int, q):
+    a = np.ascontiguousarray(q, dtype=np.int32)
+    m = np.zeros(DIM[lat], dtype=np.int32)
+    c = np.zeros(1, dtype=np.uint32)
+    lib().hqref_strip(lat, _ptr(a), _ptr(m), _ptr(c))
+    return m, int(c[0])
+
+
+def reinsert(lat: int, m, coset: int) -> np.ndarray:
+    a = np.ascontiguousarray(m, dtype=np.int32)
+    q = np.zeros(DIM[lat], dtype=np.int32)
+    lib().hqref_reinsert(lat, _ptr(a), coset, _ptr(q))
+    return q
+
+
+def zigzag(m: int) -> int:
+    return int(lib().hqref_zigzag(m))
+
+
+def unzigzag(z: int) -> int:
+    return int(lib().hqref_unzigzag(z))
+
+
+def rice_concat(z, k: int):
+    zz = np.ascontiguousarray(z, dtype=np.uint32)
+    nbits = int(lib().hqref_rice_concat(_ptr(zz), zz.size, k, None, 0))
+    out = np.zeros((nbits + 31) // 32, dtype=np.uint32)
+    lib().hqref_rice_concat(_ptr(zz), zz.size, k, _ptr(out), out.size)
+    return out, nbits
+
+
+def rice_concat_decode(words, nbits: int, n: int, k: int) -> np.ndarray:
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    z = np.zeros(n, dtype=np.uint32)
+    rc = lib().hqref_rice_concat_decode(_ptr(w), nbits, n, k, _ptr(z))
+    if rc != 0:
+        raise ValueError("corrupt Rice stream")
+    return z
+
+
+def encode_chunk(lat: int, k: int, codes):
+    q = np.ascontiguousarray(codes, dtype=np.int32)
+    assert q.size % 128 == 0
+    nt = q.size // 128
+    pb = np.zeros(1, dtype=np.uint64)
+    n = int(lib().hqref_encode_chunk(lat, k, _ptr(q), nt, None, 0, _ptr(pb)))
+    out = np.zeros(n, dtype=np.uint32)
+    lib().hqref_encode_chunk(lat, k, _ptr(q), nt, _ptr(out), n, _ptr(pb))
+    return out, int(pb[0])
+
+
+def decode_chunk(lat: int, k: int, words, ntiles: int) -> np.ndarray:
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    q = np.zeros(ntiles * 128, dtype=np.int32)
+    if lib().hqref_decode_chunk(lat, k, _ptr(w), w.size, ntiles, _ptr(q)) != 0:
+        raise ValueError("corrupt chunk")
+    return q
+
+
+def quantize_tile(x_u16, lat, alpha, seed, sign_col0=0, dither=0, e0=0) -> np.ndarray:
+    x = np.ascontiguousarray(x_u16, dtype=np.uint16)
+    q = np.zeros(128, dtype=np.int32)
+    lib().hqref_quantize_tile(_ptr(x), lat, alpha, seed, sign_col0, dither, e0, _ptr(q))
+    return q
+
+
+def dequantize_tile(q, lat, alpha, seed, sign_col0=0, dither=0, e0=0) -> np.ndarray:
+    a = np.ascontiguousarray(q, dtype=np.int32)
+    out = np.zeros(128, dtype=np.float32)
+    lib().hqref_dequantize_tile(_ptr(a), lat, alpha, seed, sign_col0, dither, e0, _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------- whole tensors
+def n_chunks(rows: int, cols: int) -> int:
+    return int(lib().hqref_n_chunks(rows, cols))
+
+
+def quantize(x, lat: int, alpha: float, k: int, seed: int, dither: int = 0, chunk_lo: int = 0,
+             chunk_hi: int | None = None):
+    """Weights path: bf16 [R, C] -> (stream words, offsets (n+1, relative), payload bits)."""
+    xu = _as_u16(x)
+    R, Cc = xu.shape
+    if chunk_hi is None:
+        chunk_hi = n_chunks(R, Cc)
+    L = lib()
+    off = np.zeros(chunk_hi - chunk_lo + 1, dtype=np.uint64)
+    pb = np.zeros(1, dtype=np.uint64)
+    total = int(L.hqref_quantize(_ptr(xu), R, Cc, Cc, lat, alpha, k, seed, dither, chunk_lo, chunk_hi, None, 0,
+                                 _ptr(off), _ptr(pb)))
+    total = abs(total)
+    stream = np.zeros(max(total, 1), dtype=np.uint32)
+    rc = int(L.hqref_quantize(_ptr(xu), R, Cc, Cc, lat, alpha, k, seed, dither, chunk_lo, chunk_hi,
+                              _ptr(stream), stream.size, _ptr(off), _ptr(pb)))
+    assert rc == total
+    return stream[:total], off, int(pb[0])
+
+
+def dequantize(stream, offsets, rows: int, cols: int, lat: int, alpha: float, k: int, seed: int, dither: int = 0,
+               out_fp32: bool = False, chunk_lo: int = 0, chunk_hi: int | None = None) -> np.ndarray:
+    """Weights path inverse: returns float32 [R, C] (fp32 mode) or uint16 bf16 bits [R, C]."""
+    if chunk_hi is None:
+        chunk_hi = n_chunks(rows, cols)
+    s = np.ascontiguousarray(stream, dtype=np.uint32)
+    o = np.ascontiguousarray(offsets, dtype=np.uint64)
+    out = np.zeros((rows, cols), dtype=np.float32 if out_fp32 else np.uint16)
+    rc = lib().hqref_dequantize(_ptr(s), _ptr(o), rows, cols, lat, alpha, k, seed, dither, chunk_lo, chunk_hi,
+                                int(out_fp32), _ptr(out), cols)
+    if rc != 0:
+        raise ValueError("corrupt stream")
+    return out
+
+
+def kv_append(kv, tok0: int, lat: int, alpha: float, k: int, seed: int, dither: int = 1, base_word: int = 0):
+    """One KV append: bf16 [H, T, 128] -> (stream words, absolute offsets (n+1), payload bits)."""
+    x = _as_u16(kv)
+    H, T, D = x.shape
+    assert D == 128
+    L = lib()
+    nch = H * ((T + 31) // 32)
+    off = np.zeros(nch + 1, dtype=np.uint64)
+    pb = np.zeros(1, dtype=np.uint64)
+    end = abs(int(L.hqref_kv_append(_ptr(x), H, T, 128, T * 128, tok0, lat, alpha, k, seed, dither, None,
+                                    base_word, 0, _ptr(off), _ptr(pb))))
+    total = end - base_word
+    stream = np.zeros(max(end, 1), dtype=np.uint32)
+    L.hqref_kv_append(_ptr(x), H, T, 128, T * 128, tok0, lat, alpha, k, seed, dither, _ptr(stream), base_word,
+                      stream.size, _ptr(off), _ptr(pb))
+    return stream[base_word:end].copy(), off, int(pb[0])
+
+
+def kv_read_append(stream_abs, offsets_abs, H: int, T: int, tok0: int, lat: int, alpha: float, k: int, seed: int,
+                   dither: int, out: np.ndarray, length: int):
+    """Decode one append into out [H, len, 128] (float32 or uint16 bf16 bits)."""
+    s = np.ascontiguousarray(stream_abs, dtype=np.uint32)
+    o = np.ascontiguousarray(offsets_abs, dtype=np.uint64)
+    assert out.flags["C_CONTIGUOUS"] and out.shape[2] == 128
+    rc = lib().hqref_kv_read_append(_ptr(s), _ptr(o), H, T, tok0, lat, alpha, k, seed, dither,
+                                    int(out.dtype == np.float32), _ptr(out), 128, out.shape[1] * 128, length)
+    if rc != 0:
+        raise ValueError("corrupt stream")

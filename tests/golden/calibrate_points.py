@@ -1,0 +1,168 @@
+"""Choose alpha and the Rice parameter k for every operating point of the five
+synthetic workloads, using only the CPU oracle, and write rate_points.json.
+
+The pages say alpha is calibrated and that the realized rate lands within
+~0.01 bits per scalar of any target ("Bit-stripping and Rice coding").  Here,
+per point: for each k in a small range, alpha is bisected (in log space) until
+the oracle's payload rate on a sample of the workload is within 0.002 bps of the
+target; the k whose alpha is largest (finest lattice, lowest distortion at that
+rate) is kept.  Weight points are then refined on the full matrix.
+
+Run:  python tests/golden/calibrate_points.py      (several minutes on 8 cores)
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+import sys
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+sys.path.insert(0, ROOT)
+import oracle as O  # noqa: E402
+import synth  # noqa: E402
+
+OUT = os.path.join(os.path.dirname(os.path.abspath(__file__)), "rate_points.json")
+THREADS = os.cpu_count() or 4
+POOL = ThreadPoolExecutor(THREADS)
+
+
+def weight_bits(x_u16: np.ndarray, lat: int, alpha: float, k: int, seed: int) -> int:
+    """Payload bits of the whole matrix, chunk ranges encoded on THREADS threads."""
+    R, Cc = x_u16.shape
+    nch = O.n_chunks(R, Cc)
+    step = max(1, (nch + THREADS - 1) // THREADS)
+    ranges = [(a, min(nch, a + step)) for a in range(0, nch, step)]
+    res = POOL.map(lambda r: O.quantize(x_u16, lat, alpha, k, seed, 0, r[0], r[1])[2], ranges)
+    return sum(res)
+
+
+def kv_bits(kv_u16: np.ndarray, lat: int, alpha: float, k: int, seed: int) -> int:
+    H, T, _ = kv_u16.shape
+    step = 256
+    jobs = [(t0, kv_u16[:, t0:t0 + step]) for t0 in range(0, T, step)]
+    res = POOL.map(lambda j: O.kv_append(np.ascontiguousarray(j[1]), j[0], lat, alpha, k, seed, 1)[2], jobs)
+    return sum(res)
+
+
+def bisect_alpha(rate, target: float, tol: float = 0.002, lo: float = 1.0, hi: float = 4096.0):
+    rlo, rhi = rate(lo), rate(hi)
+    if not (rlo <= target <= rhi):
+        return None
+    for _ in range(60):
+        mid = math.sqrt(lo * hi)
+        r = rate(mid)
+        if abs(r - target) <= tol:
+            return mid, r
+        if r < target:
+            lo = mid
+        else:
+            hi = mid
+    return math.sqrt(lo * hi), rate(math.sqrt(lo * hi))
+
+
+def calibrate(rate_of, target: float, ks, refine=None):
+    """rate_of(alpha, k) -> bps on the sample; refine(alpha, k) -> bps on the full data."""
+    best = None
+    for k in ks:
+        r = bisect_alpha(lambda a: rate_of(a, k), target)
+        if r is None:
+            continue
+        if best is None or r[0] > best[1]:
+            best = (k, r[0], r[1])
+    k, alpha, r = best
+    full = None
+    if refine is not None:
+        rr = bisect_alpha(lambda a: refine(a, k), target, tol=0.002, lo=alpha * 0.97, hi=alpha * 1.03)
+        if rr is not None:
+            alpha, full = rr
+    return {"k": int(k), "alpha": float(np.float32(alpha)), "bps_payload_sample": float(r),
+            "bps_payload_full": None if full is None else float(full)}
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return np.ascontiguousarray(t.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def main():
+    out = {"note": "alpha and Rice k per operating point; written by tests/golden/calibrate_points.py "
+                   "from the CPU oracle only (payload bits per scalar on the named sample)",
+           "workloads": {}}
+
+    # 1. 1024x1024, E8, k = 2 fixed, alpha for 4 bps (full matrix).
+    w = synth.WORKLOADS["weight_1024x1024_e8_4bps"]
+    x = u16(synth.weight(w["rows"], w["cols"], w["seed"]))
+    n = x.size
+    r = bisect_alpha(lambda a: weight_bits(x, O.E8, a, 2, w["seed"]) / n, 4.0)
+    out["workloads"]["weight_1024x1024_e8_4bps"] = {
+        "sample": "full matrix", "points": [{"lattice": "E8", "bps": 4.0, "k": 2, "alpha": float(np.float32(r[0])),
+                                             "bps_payload_sample": r[1], "bps_payload_full": r[1]}]}
+    print("cfg1", out["workloads"]["weight_1024x1024_e8_4bps"], flush=True)
+
+    # 2. 4096x4096 rate sweep: sample = first 256 rows for k selection, full matrix to refine alpha.
+    w = synth.WORKLOADS["weight_4096x4096_rate_sweep"]
+    xf = u16(synth.weight(w["rows"], w["cols"], w["seed"]))
+    xs = np.ascontiguousarray(xf[:256])
+    pts = []
+    for lat_name in ("E8", "D4", "A2", "Z"):
+        lat = O.LATTICES[lat_name]
+        for bps in (3.0, 4.0, 5.0):
+            p = calibrate(lambda a, k: weight_bits(xs, lat, a, k, w["seed"]) / xs.size, bps, range(0, 7),
+                          refine=lambda a, k: weight_bits(xf, lat, a, k, w["seed"]) / xf.size)
+            p.update(lattice=lat_name, bps=bps)
+            pts.append(p)
+            print("cfg2", p, flush=True)
+    out["workloads"]["weight_4096x4096_rate_sweep"] = {"sample": "rows 0..255 (k), full matrix (alpha)",
+                                                       "points": pts}
+
+    # 3. KV: K and V separately, E8 with dither, 2.0 and 1.7 bps; sample = first 2048 tokens of every head.
+    w = synth.WORKLOADS["kv_8h_32768tok_e8_dither"]
+    K, V = synth.kv(w["heads"], w["tokens"], w["seed"])
+    pts = []
+    for name, t in (("K", K), ("V", V)):
+        s = u16(t[:, :2048])
+        for bps in (2.0, 1.7):
+            p = calibrate(lambda a, k: kv_bits(s, O.E8, a, k, w["seed"]) / s.size, bps, range(0, 4))
+            p.update(tensor=name, lattice="E8", bps=bps)
+            pts.append(p)
+            print("cfg3", p, flush=True)
+    out["workloads"]["kv_8h_32768tok_e8_dither"] = {"sample": "tokens 0..2047 of every head", "points": pts}
+
+    # 4. 8-layer weight set, E8 4 bps, one alpha: sample = 64 rows of each matrix of layer 0.
+    w = synth.WORKLOADS["weights_8b_8layers_e8_4bps"]
+    mats = []
+    for i, (name, m) in enumerate(synth.weight_set(w["seed"])):
+        if i >= len(synth.LAYER_SHAPES):
+            break
+        mats.append(u16(m[:64]))
+    s = np.ascontiguousarray(np.concatenate(mats, axis=0))
+    p = calibrate(lambda a, k: weight_bits(s, O.E8, a, k, w["seed"]) / s.size, 4.0, range(0, 7))
+    p.update(lattice="E8", bps=4.0)
+    print("cfg4", p, flush=True)
+    out["workloads"]["weights_8b_8layers_e8_4bps"] = {"sample": "rows 0..63 of each layer-0 matrix",
+                                                      "points": [p]}
+
+    # 5. Student-t set, E8 at 3 and 4 bps: sample = 512 rows of the first matrix.
+    w = synth.WORKLOADS["student_t_64x8192x8192_e8"]
+    m0 = next(synth.student_t(1, 512, 8192, w["seed"]))
+    s = u16(m0)
+    pts = []
+    for bps in (3.0, 4.0):
+        p = calibrate(lambda a, k: weight_bits(s, O.E8, a, k, w["seed"]) / s.size, bps, range(0, 7))
+        p.update(lattice="E8", bps=bps)
+        pts.append(p)
+        print("cfg5", p, flush=True)
+    out["workloads"]["student_t_64x8192x8192_e8"] = {"sample": "512x8192 Student-t matrix (CPU generator)",
+                                                     "points": pts}
+
+    with open(OUT, "w") as f:
+        json.dump(out, f, indent=1)
+    print("wrote", OUT)
+
+
+if __name__ == "__main__":
+    main()
