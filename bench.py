@@ -1,0 +1,429 @@
+"""Benchmark of the HyperQuant quantize+encode / decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Default workload: the 4096 x 4096 bf16 lattice / rate sweep (N(0, 0.02^2) with
+0.1 % x20 outliers, seed 1): 12 operating points {E8, D4, A2, Z} x {3, 4, 5}
+bits per scalar, alpha and Rice k per point from tests/golden/rate_points.json.
+One step = for every point, hq_quantize (quantize + encode) of the matrix and
+hq_dequantize of the stream back to bf16: the whole weights path.  The 32 MiB
+input fits in the 126 MB L2, so L2 is flushed (a 256 MiB write) before every
+timed kernel and each kernel is timed alone with CUDA events on the stream it
+runs on; the step time is the sum.
+
+metric: GB/s of bf16 input through quantize+encode and decode (the value is the
+round trip: input bytes / (encode time + decode time); each direction is also
+reported), with MSE and bits per scalar per point.
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU (the
+path shards into independent tensors; no collective in the data path): weak
+scaling, value = all ranks' bytes / the slowest rank's time.
+
+--impl reference times the CPU oracle (plain C, tests' reference) on a bounded
+sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "weight_4096x4096_rate_sweep"
+L2_FLUSH_BYTES = 256 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "encode_kernel_weight_4096x4096.md")
+
+
+def rate_points():
+    with open(os.path.join(ROOT, "tests", "golden", "rate_points.json")) as f:
+        return json.load(f)["workloads"]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("hq_encode.cu", "hq_device.cuh", "hq_internal.h"):
+        with open(os.path.join(ROOT, "lattice_entropy_coded_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """(bytes per launch of the encode kernel at the E8 4 bps point, from an ncu
+    capture) if the capture was taken with the current kernel source, else None."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    src_hash, traffic = None, None
+    with open(PROFILE_TRAFFIC) as f:
+        for line in f:
+            if line.startswith("kernel_source_hash:"):
+                src_hash = line.split(":", 1)[1].strip()
+            if line.startswith("traffic_bytes_per_launch:"):
+                traffic = float(line.split(":", 1)[1].strip())
+    return traffic if src_hash == kernel_source_hash() else None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------ workload
+def make_points(workload: str):
+    pts = rate_points()[workload]["points"]
+    return pts
+
+
+def run_ours(args, rank: int, world: int, device: torch.device):
+    import lattice_entropy_coded_b200 as hq
+    assert hq.hq_device_check() == hq.HQ_OK, "needs an sm_100 (B200) device"
+    w = synth.WORKLOADS[args.workload]
+    assert w["kind"] == "weight", "the default bench workload is a single weight matrix"
+    rows, cols, seed = w["rows"], w["cols"], w["seed"]
+    x = synth.weight(rows, cols, seed=seed, device=device)
+    n = x.numel()
+    pts = make_points(args.workload)
+    stream = torch.cuda.current_stream(device)
+
+    codecs = []
+    for p in pts:
+        params = hq.make_params(p["lattice"], p["alpha"], p["k"], seed, 0)
+        cap = int(n * (p["bps"] + 3.0) / 32) + 8192
+        codecs.append(hq.Codec(rows, cols, params, cap_words=cap, device=device))
+    outs = [torch.empty(rows, cols, dtype=torch.bfloat16, device=device) for _ in pts]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def one_step(record):
+        for i, c in enumerate(codecs):
+            flush.fill_(float(i))
+            e0, e1 = record()
+            e0.record(stream)
+            comp = c.quantize(x)
+            e1.record(stream)
+            flush.fill_(float(i) + 0.5)
+            d0, d1 = record()
+            d0.record(stream)
+            c.dequantize(comp, outs[i])
+            d1.record(stream)
+
+    events = []
+
+    def rec():
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        events.append((a, b))
+        return a, b
+
+    for _ in range(args.warmup):
+        one_step(rec)
+    torch.cuda.synchronize(device)
+    events.clear()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            one_step(rec)
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    wall_ms = t0.elapsed_time(t1)
+    ms = np.array([a.elapsed_time(b) for a, b in events]).reshape(args.steps, len(pts), 2)
+    enc_ms = ms[:, :, 0].sum(1)      # per step
+    dec_ms = ms[:, :, 1].sum(1)
+    step_ms = enc_ms + dec_ms
+
+    # per-point results (outside the timed region): rate and MSE of the bf16 reconstruction
+    per_point = []
+    xf = x.double()
+    for i, (p, c) in enumerate(zip(pts, codecs)):
+        st = hq.read_stats(c.stats)
+        assert st["status"] == 0, (p, st)
+        mse = float(((outs[i].double() - xf) ** 2).mean())
+        words = int(c.offsets[-1].item())
+        per_point.append(dict(lattice=p["lattice"], bps_target=p["bps"], k=p["k"], alpha=p["alpha"],
+                              bps_payload=st["payload_bits"] / n, bps_stream=words * 32.0 / n,
+                              bps_total=(words * 32.0 + 64.0 * (c.n_chunks + 1)) / n, mse=mse,
+                              d_over_sigma2=mse / float(xf.var()),
+                              enc_us=float(np.median(ms[:, i, 0]) * 1e3), dec_us=float(np.median(ms[:, i, 1]) * 1e3),
+                              enc_gbs=2.0 * n / (np.median(ms[:, i, 0]) * 1e6),
+                              dec_gbs=2.0 * n / (np.median(ms[:, i, 1]) * 1e6),
+                              stream_words=words))
+
+    # max over ranks of the summed kernel time
+    tot = torch.tensor([float(step_ms.sum()), float(enc_ms.sum()), float(dec_ms.sum()), wall_ms], device=device,
+                       dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.MAX)
+    step_sum, enc_sum, dec_sum, wall_max = [float(v) for v in tot.cpu()]
+    in_bytes = 2.0 * n * len(pts)               # bf16 input bytes per step, per rank
+    value = world * in_bytes * args.steps / (step_sum * 1e6)
+    enc_gbs = world * in_bytes * args.steps / (enc_sum * 1e6)
+    dec_gbs = world * in_bytes * args.steps / (dec_sum * 1e6)
+
+    # roofline of the dominant kernel (the encoder): algorithmic bytes per launch = bf16 in + stream + offsets
+    peak, peak_kind = measured_peaks()
+    alg = [2.0 * n + 4.0 * pp["stream_words"] + 8.0 * (c.n_chunks + 1) for pp, c in zip(per_point, codecs)]
+    enc_launch_ms = ms[:, :, 0].mean(0)
+    dec_launch_ms = ms[:, :, 1].mean(0)
+    achieved = float(np.sum(alg) / (np.sum(enc_launch_ms) * 1e6))
+    achieved_dec = float(np.sum(alg) / (np.sum(dec_launch_ms) * 1e6))
+    dominant = "encode" if enc_sum >= dec_sum else "decode"
+    e4 = [i for i, p in enumerate(per_point) if p["lattice"] == "E8" and p["bps_target"] == 4.0][0]
+    tr = profiled_traffic()
+    roofline = {"kernel": "hq::encode_kernel (all 12 points, averaged)" if dominant == "encode"
+                else "hq::decode_kernel (all 12 points, averaged)",
+                "bound": "hbm", "achieved": round(achieved if dominant == "encode" else achieved_dec, 1),
+                "peak": peak, "unit": "GB/s",
+                "frac": round((achieved if dominant == "encode" else achieved_dec) / peak, 4),
+                "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, burst copy)" if peak_kind == "measured"
+                else "fallback",
+                "traffic": tr, "traffic_launch": "E8 4 bps point" if tr else None,
+                "algorithmic_bytes_e8_4bps": alg[e4],
+                "decode_achieved": round(achieved_dec, 1), "decode_frac": round(achieved_dec / peak, 4),
+                "encode_achieved": round(achieved, 1), "encode_frac": round(achieved / peak, 4)}
+
+    # end to end through the C ABI with host buffers: H2D of the input, quantize+decode per point,
+    # D2H of every reconstruction and stats block
+    e2e = run_e2e(args, hq, codecs, pts, rows, cols, device, stream, world)
+
+    return dict(value=value, enc_gbs=enc_gbs, dec_gbs=dec_gbs, ms_per_step=step_sum / args.steps,
+                wall_ms_per_step=wall_max / args.steps, per_point=per_point, roofline=roofline,
+                clocks=clk.summary(), e2e=e2e, launches=2 * len(pts) * args.steps, n=n, in_bytes=in_bytes)
+
+
+def run_e2e(args, hq, codecs, pts, rows, cols, device, stream, world):
+    n = rows * cols
+    host_x = synth.weight(rows, cols, seed=synth.WORKLOADS[args.workload]["seed"]).pin_memory()
+    host_out = [torch.empty(rows, cols, dtype=torch.bfloat16).pin_memory() for _ in pts]
+    host_stats = [torch.empty(32, dtype=torch.uint8).pin_memory() for _ in pts]
+    dev_x = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
+    dev_out = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
+
+    def step():
+        dev_x.copy_(host_x, non_blocking=True)
+        for i, c in enumerate(codecs):
+            comp = c.quantize(dev_x)
+            c.dequantize(comp, dev_out)
+            host_out[i].copy_(dev_out, non_blocking=True)
+            host_stats[i].copy_(c.stats, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    steps = max(1, min(args.steps, 5))
+    if world > 1:
+        torch.distributed.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = torch.tensor([t0.elapsed_time(t1)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
+    ms = float(ms.item())
+    for i in range(len(pts)):
+        assert hq.read_stats(host_stats[i])["status"] == 0
+    in_bytes = 2.0 * n * len(pts)
+    return {"value": round(world * in_bytes * steps / (ms * 1e6), 3), "unit": "GB/s",
+            "h2d_bytes_per_step": 2 * n, "d2h_bytes_per_step": len(pts) * (2 * n + 32),
+            "steps": steps, "ms_per_step": round(ms / steps, 3)}
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+def oracle_sample_rate(workload: str, rows_sample: int, threads: int, repeat: int = 1):
+    """Oracle quantize+decode of the first rows_sample rows at every point, chunk ranges on
+    `threads` host threads (ctypes releases the GIL).  -> (GB/s of bf16 input, seconds, elems)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle as O
+    w = synth.WORKLOADS[workload]
+    x = synth.weight(w["rows"], w["cols"], seed=w["seed"])[:rows_sample].contiguous()
+    xu = np.ascontiguousarray(x.view(torch.int16).numpy().view(np.uint16))
+    R, Cc = xu.shape
+    nch = O.n_chunks(R, Cc)
+    step = max(1, -(-nch // threads))
+    ranges = [(a, min(nch, a + step)) for a in range(0, nch, step)]
+    pts = make_points(workload)
+    O.lib()
+
+    def job(r, p):
+        lat = O.LATTICES[p["lattice"]]
+        s, off, _ = O.quantize(xu, lat, p["alpha"], p["k"], w["seed"], 0, r[0], r[1])
+        O.dequantize(s, off, R, Cc, lat, p["alpha"], p["k"], w["seed"], 0, False, r[0], r[1])
+
+    t = time.perf_counter()
+    with ThreadPoolExecutor(threads) as ex:
+        for _ in range(repeat):
+            list(ex.map(lambda a: job(*a), [(r, p) for p in pts for r in ranges]))
+    dt = time.perf_counter() - t
+    elems = R * Cc * len(pts) * repeat
+    return 2.0 * elems / dt / 1e9, dt, elems
+
+
+def host_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(workload: str):
+    threads = host_threads()
+    rows = min(4096, max(256, 128 * threads))
+    gbs, dt, elems = oracle_sample_rate(workload, rows, threads)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"rows 0..{rows - 1} of the 4096x4096 matrix at all 12 points, quantize+encode and "
+                      f"decode ({elems} elements per direction, {dt:.1f} s wall on {threads} threads)"}
+
+
+def run_reference(args):
+    threads = host_threads()
+    rows = max(32, min(1024, 32 * threads))
+    for _ in range(args.warmup):
+        oracle_sample_rate(args.workload, rows, threads)
+    gbs, dt, elems = oracle_sample_rate(args.workload, rows, threads, repeat=args.steps)
+    base = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"rows 0..{rows - 1} of the 4096x4096 matrix at all 12 points per step, quantize+encode and "
+                      f"decode, {args.steps} steps ({dt:.1f} s wall on {threads} threads)"}
+    return {"metric": "quantize+encode / decode GB/s of bf16 input vs B200 HBM peak; MSE at bps",
+            "value": base["value"], "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "rows": 4096, "cols": 4096, "points": 12,
+                       "sample_rows": rows, "parallelism": "host threads"},
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    try:
+        r = run_ours(args, rank, world, device)
+        if rank == 0:
+            line = {
+                "metric": "quantize+encode / decode GB/s of bf16 input vs B200 HBM peak; MSE at bps",
+                "value": round(r["value"], 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": args.workload, "rows": 4096, "cols": 4096, "dtype_in": "bf16",
+                           "points": "E8,D4,A2,Z x 3,4,5 bps", "step": "12 x (hq_quantize + hq_dequantize bf16)",
+                           "l2": "flushed (256 MiB write) before every timed kernel; kernels timed alone",
+                           "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU"},
+                "quantize_encode_gbs": round(r["enc_gbs"], 2), "decode_gbs": round(r["dec_gbs"], 2),
+                "roofline": r["roofline"], "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": r["launches"],
+                "points": r["per_point"],
+            }
+            if not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(args.workload)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

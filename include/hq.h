@@ -1,0 +1,229 @@
+/*
+ * hq.h -- C ABI of the B200 (sm_100a) HyperQuant codec library, libhq.so.
+ *
+ * The method: HyperQuant ("Hadamard, optimallY Packing, Entropy Rice-coding"),
+ * as summarised on the gist.science explainer pages of paper 2606.23406
+ * ("Methodology": 1 per-tile RHT, 2 lattice quantization, 3 bit-stripping and
+ * Rice coding, 4 KV-cache bias correction) and its arXiv abstract (steps
+ * (i)-(iv)).  Per 128-element tile: x -> D x (seeded random signs) -> H_128
+ * (Walsh-Hadamard) -> scale by alpha / sqrt(128) -> [+ dither d] -> nearest
+ * point of the lattice (Z, A2, D4 or E8 in an integer embedding) -> strip the
+ * membership-implied bits -> zigzag -> Rice code with parameter k into a
+ * chunked bitstream.  The inverse undoes every step.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer named d_* or documented as "device" is device memory of the
+ *    current CUDA device; host pointers are named h_* or documented as host.
+ *  - The caller owns all memory.  The library allocates nothing and never
+ *    synchronises; every call is asynchronous on the CUDA stream it is given
+ *    (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *  - A negative return value is a synchronous argument or launch error
+ *    (HQ_EINVAL, HQ_EUNSUPPORTED, HQ_ECUDA); nothing was enqueued.  Errors that
+ *    depend on the data are reported on the device in hq_stats.status, which
+ *    the caller reads after its own synchronisation.
+ *  - bf16 tensors are little-endian IEEE bfloat16, 16-byte aligned, with
+ *    element strides that are multiples of 8 elements (16 bytes).
+ *  - A tile is 128 consecutive elements of a row; a chunk is 32 consecutive
+ *    tiles (4096 elements).  Weights: tiles in row-major order of an R x C
+ *    matrix (C % 128 == 0), chunk c = tiles [32c, 32c+32).  KV cache: per
+ *    append of T tokens and H heads, ceil(T/32) chunks per head, head-major;
+ *    one tile = one token's 128-dim head vector.
+ *
+ * Bitstream (all planes LSB-first in little-endian uint32 words, each plane
+ * starting on a word boundary), per chunk of n tiles (N = 128 n symbols):
+ *   [coset plane, E8 only: one bit per 8-element block, ceil(16 n / 32) words]
+ *   [remainder plane: k bits per symbol at bit i*k, 4 k n words]
+ *   [unary plane: per symbol floor(z / 2^k) zeros then a one, zero padded]
+ * offsets[c] is the index of chunk c's first word; offsets[n_chunks] is the
+ * total.  The codewords are exactly the concatenated Rice codewords of the
+ * symbols; the plane split lets a decoder work on all tiles of a chunk at once.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported entry points keep default visibility (the library is built with
+ * hidden visibility for everything else). */
+#if defined(__GNUC__)
+#define HQ_API __attribute__((visibility("default")))
+#else
+#define HQ_API
+#endif
+
+/* Lattices (page section "lattice quantization": E8, D4, A2 or scalar Z) in
+ * their integer embeddings:
+ *   HQ_Z  : Z, code q stands for q.
+ *   HQ_A2 : code (a, b), a = b (mod 2), stands for (a/2, b*sqrt(3)/2)
+ *           (A2 at unit minimum distance).
+ *   HQ_D4 : {q in Z^4 : sum q even}.
+ *   HQ_E8 : 2E8 = 2D8 u (2D8 + 1) in Z^8 (all coordinates of one parity, and
+ *           (q - parity)/2 has an even sum). */
+enum hq_lattice { HQ_Z = 0, HQ_A2 = 1, HQ_D4 = 2, HQ_E8 = 3 };
+
+/* Synchronous return codes. */
+#define HQ_OK 0
+#define HQ_EINVAL (-1)       /* bad argument: null pointer, size, stride, alignment, parameter */
+#define HQ_EUNSUPPORTED (-2) /* valid request outside what this build supports (tile != 128, ...) */
+#define HQ_ECUDA (-3)        /* a CUDA launch or runtime call failed */
+
+/* Device-side status bits (hq_stats.status). */
+#define HQ_ST_CAPACITY 0x1u /* the stream needs more than cap_words words: words at or past the cap
+                               were not written; stats.stream_words holds the size needed */
+#define HQ_ST_CORRUPT 0x2u  /* a chunk failed a consistency check while decoding (offsets out of range
+                               or not monotone, wrong number of unary terminators); its tiles are zero */
+#define HQ_ST_TIMEOUT 0x4u  /* the chunk-offset look-back gave up after its spin limit */
+#define HQ_ST_RANGE 0x8u    /* a scaled coordinate was at or beyond 2^21 in magnitude (or not finite):
+                               codes of that call are outside the supported range and unspecified */
+
+/* Parameters of one call (page sections 1-4).  tile and chunk_tiles are
+ * fixed by this build; the others select the operating point. */
+typedef struct hq_params {
+    int32_t tile;        /* elements per RHT tile; must be 128 */
+    int32_t lattice;     /* enum hq_lattice */
+    float alpha;         /* scale: u = H_128 D x * alpha / sqrt(128); finite, > 0 */
+    int32_t rice_k;      /* Rice parameter, 0..15 */
+    uint64_t seed;       /* seeds the sign diagonal D and the dither */
+    int32_t dither;      /* 0: none; 1: subtractive dither (page section 4; the KV path) */
+    int32_t chunk_tiles; /* tiles per chunk; must be 32 */
+} hq_params;
+
+/* Device-resident statistics written by the kernels (zeroed by each call
+ * that takes it).  32 bytes, 8-byte aligned. */
+typedef struct hq_stats {
+    uint32_t status;       /* HQ_ST_* bits */
+    uint32_t max_symbol;   /* bitwise OR of all zigzag symbols coded: its bit length bounds them */
+    uint64_t payload_bits; /* sum of Rice codeword lengths plus E8 coset bits */
+    uint64_t stream_words; /* words the stream needs (= offsets[n_chunks] when it fit) */
+    uint64_t reserved;
+} hq_stats;
+
+/* One row of a KV cache's append table (device memory; written by
+ * hq_kv_append's kernel).  32 bytes. */
+typedef struct hq_kv_append_row {
+    uint64_t first_chunk; /* global index of the append's first chunk */
+    int64_t token0;       /* first token of the append */
+    int32_t tokens;       /* T */
+    float alpha;          /* alpha used for this append */
+    float scale_fwd;      /* fp32(alpha / sqrt(128)) */
+    float scale_inv;      /* fp32(1 / (alpha * sqrt(128))) */
+} hq_kv_append_row;
+
+/* A compressed KV cache for one of K or V of one layer (page section 4: KV
+ * bias correction with a +-1 sign rotation and subtractive dither).  Plain
+ * data: device buffers owned by the caller, and host-side counters that
+ * hq_kv_append advances.  One K and one V cache are two of these. */
+typedef struct hq_kv_cache {
+    uint32_t *d_words;          /* stream, cap_words words */
+    uint64_t cap_words;
+    uint64_t *d_offsets;        /* chunk offsets, offsets_cap entries (>= total chunks + 1) */
+    uint64_t offsets_cap;
+    hq_kv_append_row *d_table;  /* one row per append, table_cap rows */
+    uint64_t table_cap;
+    uint64_t *d_tail;           /* two words: the append numbered a reads the next free stream word from
+                                   d_tail[a & 1] and writes the new end to d_tail[(a + 1) & 1] */
+    hq_stats *d_stats;          /* accumulated over appends (not zeroed by hq_kv_append) */
+    int32_t heads;              /* H */
+    int32_t head_dim;           /* must be 128 */
+    hq_params params;           /* lattice, k, seed, dither for every append */
+    int64_t tokens;             /* host: tokens appended so far */
+    uint64_t chunks;            /* host: chunks appended so far */
+    uint64_t appends;           /* host: appends so far */
+} hq_kv_cache;
+
+/* --------------------------------------------------------------------- sizes */
+
+/* Number of chunks of an R x C weight matrix and an upper bound on its stream
+ * size in words for symbols of magnitude at most max_abs_symbol (pass 0 for
+ * 255): per chunk, coset + remainder words plus one unary bit per symbol plus
+ * (2 max_abs_symbol + 1) >> k zeros per symbol, rounded up to words.  A call
+ * whose symbols exceed the assumption reports HQ_ST_CAPACITY instead of
+ * overrunning.  Host only; returns HQ_OK or HQ_EINVAL. */
+HQ_API int hq_stream_bound(int64_t rows, int64_t cols, const hq_params *p, uint32_t max_abs_symbol,
+                    uint64_t *max_words, uint64_t *n_chunks);
+
+/* Bytes of device workspace hq_quantize / hq_kv_append need for n_chunks
+ * chunks (chunk look-back state and a chunk ticket).  Host only. */
+HQ_API int hq_workspace_bytes(uint64_t n_chunks, size_t *bytes);
+
+/* ------------------------------------------------------------ weights path */
+
+/* Quantize and encode an R x C bf16 matrix (page sections 1-3; section 4's
+ * dither too if p->dither).
+ *   x         device, bf16, element (r, c) at x[r * ld + c]; ld >= cols, ld % 8 == 0.
+ *   d_stream  device, cap_words uint32 words, written [0, stream_words).
+ *   d_offsets device, n_chunks + 1 uint64 entries, all written.
+ *   d_stats   device hq_stats or NULL; zeroed then filled.
+ *   workspace device, >= hq_workspace_bytes(n_chunks); overwritten (contents
+ *             need no initialisation; the call clears what it uses).
+ * Sign index of element (r, c) is c; dither counter (if any) is r * cols + c.
+ * Rows * cols may be 0 (then only offsets[0] = 0 and stats are written). */
+HQ_API int hq_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p, uint32_t *d_stream,
+                uint64_t cap_words, uint64_t *d_offsets, hq_stats *d_stats, void *workspace, size_t ws_bytes,
+                void *cuda_stream);
+
+/* Decode and dequantize a stream made by hq_quantize with the same rows,
+ * cols and params (page sections 1-3 inverted).
+ *   d_stream   device, stream_words words (offsets are checked against it).
+ *   d_offsets  device, n_chunks + 1 entries.
+ *   out        device; out_dtype 0: bf16 (round to nearest even), 1: fp32
+ *              (the value before bf16 rounding); element (r, c) at out[r * ld + c],
+ *              ld >= cols, ld % 8 == 0 (bf16) or ld % 4 == 0 (fp32).
+ *   d_stats    device or NULL; zeroed, then HQ_ST_CORRUPT is set for a bad chunk
+ *              (whose tiles are written as zeros). */
+HQ_API int hq_dequantize(const uint32_t *d_stream, uint64_t stream_words, const uint64_t *d_offsets, int64_t rows,
+                  int64_t cols, const hq_params *p, void *out, int out_dtype, int64_t ld, hq_stats *d_stats,
+                  void *cuda_stream);
+
+/* ----------------------------------------------------------------- KV path */
+
+/* Fill a hq_kv_cache with the caller's buffers and zero its two tail words
+ * and its stats (two small cudaMemsetAsync on cuda_stream).  p->dither is
+ * normally 1; p->alpha is unused (each append gives its own). */
+HQ_API int hq_kv_init(hq_kv_cache *cache, int32_t heads, int32_t head_dim, const hq_params *p, uint32_t *d_words,
+               uint64_t cap_words, uint64_t *d_offsets, uint64_t offsets_cap, hq_kv_append_row *d_table,
+               uint64_t table_cap, uint64_t *d_tail, hq_stats *d_stats, void *cuda_stream);
+
+/* Append T tokens: kv is device bf16 [H, T, 128], element (h, t, d) at
+ * kv[h * ld_head + t * ld_token + d] (both strides % 8 == 0).  The chunks are
+ * written from the cache's device-resident tail on, so appends queue without a
+ * host sync.  Dither counter of (token, head, dim) is (token * H + head) * 128
+ * + dim, token counted from the cache start; sign index is dim.  alpha is this
+ * append's scale (stored in its table row).  Advances cache->tokens, chunks,
+ * appends on the host.  workspace: >= hq_workspace_bytes(H * ceil(T / 32)). */
+HQ_API int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t ld_token, int64_t ld_head, float alpha,
+                 void *workspace, size_t ws_bytes, void *cuda_stream);
+
+/* Decode the first len tokens of every head: out [H, len, 128], element
+ * (h, t, d) at out[h * out_ld_head + t * out_ld_token + d]; out_dtype as in
+ * hq_dequantize.  len <= cache->tokens. */
+HQ_API int hq_kv_read(const hq_kv_cache *cache, void *out, int out_dtype, int64_t len, int64_t out_ld_token,
+               int64_t out_ld_head, void *cuda_stream);
+
+/* ---------------------------------------------------------------- misc */
+
+/* Human-readable text for a return code (negative) or status bit mask (>= 0). */
+HQ_API const char *hq_status_string(int code);
+
+/* HQ_OK if the current CUDA device is sm_100 (B200-class) and the library's
+ * kernels can run on it; HQ_EUNSUPPORTED or HQ_ECUDA otherwise. */
+HQ_API int hq_device_check(void);
+
+/* Testing aid: the number of polls a chunk's look-back makes on a
+ * predecessor that has not published before it gives up and sets
+ * HQ_ST_TIMEOUT (0 restores the default, 2^22).  Process-wide; affects calls
+ * made after it.  A timed-out call's stream is unspecified but every write
+ * stays inside [0, cap_words). */
+HQ_API void hq_debug_set_spin_limit(uint32_t polls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

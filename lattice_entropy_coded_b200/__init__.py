@@ -1,0 +1,265 @@
+"""Python binding of libhq.so, the B200 (sm_100a) HyperQuant codec library.
+
+Argument marshalling only: every step of the quantize / encode / decode path
+runs in the library's CUDA kernels.  PyTorch supplies device memory and the
+current CUDA stream.  The functions carry the C entry points' names (see
+include/hq.h for the contract of each); the small classes at the end allocate
+buffers with torch and call them.
+
+There is no fallback: if libhq.so is missing or cannot be loaded, importing
+the binding raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhq.so")
+
+HQ_Z, HQ_A2, HQ_D4, HQ_E8 = 0, 1, 2, 3
+LATTICES = {"Z": HQ_Z, "A2": HQ_A2, "D4": HQ_D4, "E8": HQ_E8}
+HQ_OK, HQ_EINVAL, HQ_EUNSUPPORTED, HQ_ECUDA = 0, -1, -2, -3
+HQ_ST_CAPACITY, HQ_ST_CORRUPT, HQ_ST_TIMEOUT, HQ_ST_RANGE = 1, 2, 4, 8
+
+
+class hq_params(C.Structure):
+    _fields_ = [("tile", C.c_int32), ("lattice", C.c_int32), ("alpha", C.c_float), ("rice_k", C.c_int32),
+                ("seed", C.c_uint64), ("dither", C.c_int32), ("chunk_tiles", C.c_int32)]
+
+
+class hq_stats(C.Structure):
+    _fields_ = [("status", C.c_uint32), ("max_symbol", C.c_uint32), ("payload_bits", C.c_uint64),
+                ("stream_words", C.c_uint64), ("reserved", C.c_uint64)]
+
+
+class hq_kv_append_row(C.Structure):
+    _fields_ = [("first_chunk", C.c_uint64), ("token0", C.c_int64), ("tokens", C.c_int32), ("alpha", C.c_float),
+                ("scale_fwd", C.c_float), ("scale_inv", C.c_float)]
+
+
+class hq_kv_cache(C.Structure):
+    _fields_ = [("d_words", C.c_void_p), ("cap_words", C.c_uint64), ("d_offsets", C.c_void_p),
+                ("offsets_cap", C.c_uint64), ("d_table", C.c_void_p), ("table_cap", C.c_uint64),
+                ("d_tail", C.c_void_p), ("d_stats", C.c_void_p), ("heads", C.c_int32), ("head_dim", C.c_int32),
+                ("params", hq_params), ("tokens", C.c_int64), ("chunks", C.c_uint64), ("appends", C.c_uint64)]
+
+
+assert C.sizeof(hq_params) == 32 and C.sizeof(hq_stats) == 32 and C.sizeof(hq_kv_append_row) == 32
+assert C.sizeof(hq_kv_cache) == 128
+
+# C entry points: name -> (restype, argtypes)
+EXPORTS = {
+    "hq_stream_bound": (C.c_int, [C.c_int64, C.c_int64, C.POINTER(hq_params), C.c_uint32, C.POINTER(C.c_uint64),
+                                  C.POINTER(C.c_uint64)]),
+    "hq_workspace_bytes": (C.c_int, [C.c_uint64, C.POINTER(C.c_size_t)]),
+    "hq_quantize": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.POINTER(hq_params), C.c_void_p,
+                              C.c_uint64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "hq_dequantize": (C.c_int, [C.c_void_p, C.c_uint64, C.c_void_p, C.c_int64, C.c_int64, C.POINTER(hq_params),
+                                C.c_void_p, C.c_int, C.c_int64, C.c_void_p, C.c_void_p]),
+    "hq_kv_init": (C.c_int, [C.POINTER(hq_kv_cache), C.c_int32, C.c_int32, C.POINTER(hq_params), C.c_void_p,
+                             C.c_uint64, C.c_void_p, C.c_uint64, C.c_void_p, C.c_uint64, C.c_void_p, C.c_void_p,
+                             C.c_void_p]),
+    "hq_kv_append": (C.c_int, [C.POINTER(hq_kv_cache), C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.c_float,
+                               C.c_void_p, C.c_size_t, C.c_void_p]),
+    "hq_kv_read": (C.c_int, [C.POINTER(hq_kv_cache), C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64,
+                             C.c_void_p]),
+    "hq_status_string": (C.c_char_p, [C.c_int]),
+    "hq_device_check": (C.c_int, []),
+    "hq_debug_set_spin_limit": (None, [C.c_uint32]),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m lattice_entropy_coded_b200.build`")
+    lib = C.CDLL(LIB_PATH)
+    for name, (res, args) in EXPORTS.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+class HQError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str) -> int:
+    if rc < 0:
+        raise HQError(f"{what}: {hq_status_string(rc)} ({rc})")
+    return rc
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    assert isinstance(t, torch.Tensor)
+    return t.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, torch.cuda.Stream):
+        return s.cuda_stream
+    return int(s)
+
+
+def make_params(lattice="E8", alpha=1.0, rice_k=2, seed=0, dither=0) -> hq_params:
+    lat = LATTICES[lattice] if isinstance(lattice, str) else int(lattice)
+    return hq_params(128, lat, float(alpha), int(rice_k), int(seed) & (2**64 - 1), int(dither), 32)
+
+
+# ------------------------------------------------------------------ C entry points
+def hq_status_string(code: int) -> str:
+    return _lib.hq_status_string(int(code)).decode()
+
+
+def hq_device_check() -> int:
+    return int(_lib.hq_device_check())
+
+
+def hq_debug_set_spin_limit(polls: int) -> None:
+    _lib.hq_debug_set_spin_limit(int(polls))
+
+
+def hq_stream_bound(rows: int, cols: int, params: hq_params, max_abs_symbol: int = 0):
+    w, n = C.c_uint64(), C.c_uint64()
+    _check(_lib.hq_stream_bound(rows, cols, C.byref(params), max_abs_symbol, C.byref(w), C.byref(n)),
+           "hq_stream_bound")
+    return int(w.value), int(n.value)
+
+
+def hq_workspace_bytes(n_chunks: int) -> int:
+    b = C.c_size_t()
+    _check(_lib.hq_workspace_bytes(n_chunks, C.byref(b)), "hq_workspace_bytes")
+    return int(b.value)
+
+
+def hq_quantize(x: torch.Tensor, params: hq_params, stream: torch.Tensor, offsets: torch.Tensor,
+                stats: torch.Tensor | None, workspace: torch.Tensor, cuda_stream=None, ld: int | None = None) -> int:
+    """x: bf16 [rows, cols] (row stride ld, default x.stride(0)); stream: int32/uint32 words;
+    offsets: int64 [n_chunks + 1]; stats: uint8 [32] or None; workspace: uint8."""
+    rows, cols = x.shape
+    ld = x.stride(0) if ld is None else ld
+    return _check(_lib.hq_quantize(_ptr(x), rows, cols, ld, C.byref(params), _ptr(stream), stream.numel(),
+                                   _ptr(offsets), _ptr(stats), _ptr(workspace), workspace.numel(),
+                                   _stream(cuda_stream)), "hq_quantize")
+
+
+def hq_dequantize(stream: torch.Tensor, stream_words: int, offsets: torch.Tensor, rows: int, cols: int,
+                  params: hq_params, out: torch.Tensor, stats: torch.Tensor | None = None, cuda_stream=None) -> int:
+    """out: bf16 or fp32 [rows, cols] (row stride out.stride(0))."""
+    dt = 1 if out.dtype == torch.float32 else 0
+    assert out.dtype in (torch.float32, torch.bfloat16)
+    return _check(_lib.hq_dequantize(_ptr(stream), stream_words, _ptr(offsets), rows, cols, C.byref(params),
+                                     _ptr(out), dt, out.stride(0), _ptr(stats), _stream(cuda_stream)),
+                  "hq_dequantize")
+
+
+def hq_kv_init(cache: hq_kv_cache, heads: int, head_dim: int, params: hq_params, words: torch.Tensor,
+               offsets: torch.Tensor, table: torch.Tensor, tail: torch.Tensor, stats: torch.Tensor,
+               cuda_stream=None) -> int:
+    return _check(_lib.hq_kv_init(C.byref(cache), heads, head_dim, C.byref(params), _ptr(words), words.numel(),
+                                  _ptr(offsets), offsets.numel(), _ptr(table), table.numel() // 32, _ptr(tail),
+                                  _ptr(stats), _stream(cuda_stream)), "hq_kv_init")
+
+
+def hq_kv_append(cache: hq_kv_cache, kv: torch.Tensor, alpha: float, workspace: torch.Tensor,
+                 cuda_stream=None) -> int:
+    """kv: bf16 [heads, T, 128] with unit stride in the last dimension."""
+    H, T, D = kv.shape
+    assert D == 128 and kv.stride(2) == 1
+    return _check(_lib.hq_kv_append(C.byref(cache), _ptr(kv), T, kv.stride(1), kv.stride(0), float(alpha),
+                                    _ptr(workspace), workspace.numel(), _stream(cuda_stream)), "hq_kv_append")
+
+
+def hq_kv_read(cache: hq_kv_cache, out: torch.Tensor, length: int, cuda_stream=None) -> int:
+    """out: bf16 or fp32 [heads, >= length, 128]."""
+    dt = 1 if out.dtype == torch.float32 else 0
+    return _check(_lib.hq_kv_read(C.byref(cache), _ptr(out), dt, length, out.stride(1), out.stride(0),
+                                  _stream(cuda_stream)), "hq_kv_read")
+
+
+# ------------------------------------------------------------------ torch-allocated wrappers
+def stats_tensor(device="cuda") -> torch.Tensor:
+    return torch.zeros(32, dtype=torch.uint8, device=device)
+
+
+def read_stats(t: torch.Tensor) -> dict:
+    b = bytes(t.cpu().numpy().tobytes())
+    s = hq_stats.from_buffer_copy(b)
+    return {"status": s.status, "max_symbol": s.max_symbol, "payload_bits": s.payload_bits,
+            "stream_words": s.stream_words}
+
+
+@dataclass
+class Compressed:
+    """A quantized matrix: its stream words, chunk offsets and the parameters."""
+    words: torch.Tensor      # int32, >= n_words
+    offsets: torch.Tensor    # int64 [n_chunks + 1]
+    rows: int
+    cols: int
+    params: hq_params
+    stats: torch.Tensor      # uint8 [32] hq_stats
+
+
+class Codec:
+    """Owns the device buffers of repeated quantize / dequantize calls of one shape."""
+
+    def __init__(self, rows: int, cols: int, params: hq_params, max_abs_symbol: int = 0, device="cuda",
+                 cap_words: int | None = None):
+        self.rows, self.cols, self.params = rows, cols, params
+        bound, self.n_chunks = hq_stream_bound(rows, cols, params, max_abs_symbol)
+        self.cap_words = bound if cap_words is None else cap_words
+        self.words = torch.empty(max(self.cap_words, 1), dtype=torch.int32, device=device)
+        self.offsets = torch.empty(self.n_chunks + 1, dtype=torch.int64, device=device)
+        self.stats = stats_tensor(device)
+        self.workspace = torch.empty(hq_workspace_bytes(self.n_chunks), dtype=torch.uint8, device=device)
+
+    def quantize(self, x: torch.Tensor, cuda_stream=None) -> Compressed:
+        hq_quantize(x, self.params, self.words[:self.cap_words], self.offsets, self.stats, self.workspace,
+                    cuda_stream)
+        return Compressed(self.words, self.offsets, self.rows, self.cols, self.params, self.stats)
+
+    def dequantize(self, c: Compressed, out: torch.Tensor, stats: torch.Tensor | None = None,
+                   cuda_stream=None) -> torch.Tensor:
+        hq_dequantize(c.words, self.cap_words, c.offsets, c.rows, c.cols, c.params, out, stats, cuda_stream)
+        return out
+
+
+class KVCache:
+    """A compressed K or V cache (one layer) with torch-allocated device buffers."""
+
+    def __init__(self, heads: int, max_tokens: int, params: hq_params, words_per_token_head: float = 2.0,
+                 max_appends: int = 4096, max_append_tokens: int = 4096, device="cuda"):
+        max_chunks = heads * ((max_tokens + 31) // 32 + max_appends)
+        cap = int(heads * max_tokens * 128 * words_per_token_head / 32) + max_chunks * 64 + 1024
+        self.words = torch.empty(cap, dtype=torch.int32, device=device)
+        self.offsets = torch.empty(max_chunks + 1, dtype=torch.int64, device=device)
+        self.table = torch.zeros(max_appends * 32, dtype=torch.uint8, device=device)
+        self.tail = torch.zeros(2, dtype=torch.int64, device=device)
+        self.stats = stats_tensor(device)
+        self.workspace = torch.empty(hq_workspace_bytes(heads * ((max_append_tokens + 31) // 32)),
+                                     dtype=torch.uint8, device=device)
+        self.heads = heads
+        self.cache = hq_kv_cache()
+        hq_kv_init(self.cache, heads, 128, params, self.words, self.offsets, self.table, self.tail, self.stats)
+
+    @property
+    def tokens(self) -> int:
+        return int(self.cache.tokens)
+
+    def append(self, kv: torch.Tensor, alpha: float, cuda_stream=None):
+        hq_kv_append(self.cache, kv, alpha, self.workspace, cuda_stream)
+
+    def read(self, out: torch.Tensor, length: int | None = None, cuda_stream=None) -> torch.Tensor:
+        hq_kv_read(self.cache, out, self.tokens if length is None else length, cuda_stream)
+        return out

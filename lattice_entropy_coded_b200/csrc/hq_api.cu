@@ -1,0 +1,309 @@
+// hq_api.cu -- the extern "C" entry points of libhq.so (declared in hq.h):
+// argument validation, workspace clearing and kernel launches.  Host code only;
+// every step of the codec runs in the kernels of hq_encode.cu / hq_decode.cu.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "hq_internal.h"
+
+using namespace hq;
+
+namespace {
+
+constexpr int64_t kMaxCols = 65536;  // the shared sign table holds cols / 128 columns
+uint32_t g_spin_limit = kSpinLimit;
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int check_params(const hq_params *p) {
+    if (!p) return HQ_EINVAL;
+    if (p->lattice < HQ_Z || p->lattice > HQ_E8) return HQ_EINVAL;
+    if (!(p->alpha > 0.0f) || !isfinite(p->alpha)) return HQ_EINVAL;
+    if (p->rice_k < 0 || p->rice_k > 15) return HQ_EINVAL;
+    if (p->dither != 0 && p->dither != 1) return HQ_EINVAL;
+    if (p->tile != kTile || p->chunk_tiles != kChunkTiles) return HQ_EUNSUPPORTED;
+    return HQ_OK;
+}
+
+int check_matrix(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0 || cols % kTile) return HQ_EINVAL;
+    if (cols > kMaxCols) return HQ_EUNSUPPORTED;
+    if (rows > 0 && cols > 0 && rows > (INT64_C(1) << 40) / cols) return HQ_EUNSUPPORTED;
+    return HQ_OK;
+}
+
+uint64_t chunks_of(int64_t rows, int64_t cols) {
+    uint64_t tiles = (uint64_t)rows * (uint64_t)(cols / kTile);
+    return (tiles + kChunkTiles - 1) / kChunkTiles;
+}
+
+float scale_fwd(float alpha) { return (float)((double)alpha / sqrt(128.0)); }
+float scale_inv(float alpha) { return (float)(1.0 / ((double)alpha * sqrt(128.0))); }
+
+size_t ws_bytes_for(uint64_t n_chunks) {
+    size_t b = (size_t)n_chunks * 8 + 8;
+    return (b + 255) & ~(size_t)255;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ECUDA; }
+
+// Per-chunk word bound for ntiles tiles with symbols <= zmax.
+uint64_t chunk_bound(int lattice, int k, uint64_t ntiles, uint64_t zmax) {
+    uint64_t nsym = ntiles * kTile;
+    uint64_t nc = (lattice == HQ_E8) ? (16 * ntiles + 31) / 32 : 0;
+    uint64_t nr = 4 * (uint64_t)k * ntiles;
+    uint64_t ubits = nsym * (1 + (zmax >> k));
+    return nc + nr + (ubits + 31) / 32;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hq_stream_bound(int64_t rows, int64_t cols, const hq_params *p, uint32_t max_abs_symbol, uint64_t *max_words,
+                    uint64_t *n_chunks) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if ((rc = check_matrix(rows, cols))) return rc;
+    if (!max_words || !n_chunks) return HQ_EINVAL;
+    uint64_t m = max_abs_symbol ? max_abs_symbol : 255u;
+    uint64_t zmax = 2 * m + 1;
+    uint64_t tiles = (uint64_t)rows * (uint64_t)(cols / kTile);
+    uint64_t nch = chunks_of(rows, cols);
+    uint64_t full = tiles / kChunkTiles, rest = tiles % kChunkTiles;
+    uint64_t words = full * chunk_bound(p->lattice, p->rice_k, kChunkTiles, zmax);
+    if (rest) words += chunk_bound(p->lattice, p->rice_k, rest, zmax);
+    *max_words = words;
+    *n_chunks = nch;
+    return HQ_OK;
+}
+
+int hq_workspace_bytes(uint64_t n_chunks, size_t *bytes) {
+    if (!bytes) return HQ_EINVAL;
+    *bytes = ws_bytes_for(n_chunks);
+    return HQ_OK;
+}
+
+int hq_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p, uint32_t *d_stream,
+                uint64_t cap_words, uint64_t *d_offsets, hq_stats *d_stats, void *workspace, size_t ws_bytes,
+                void *cuda_stream) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if ((rc = check_matrix(rows, cols))) return rc;
+    const uint64_t nch = chunks_of(rows, cols);
+    if (!d_offsets || !aligned(d_offsets, 8)) return HQ_EINVAL;
+    if (d_stats && !aligned(d_stats, 8)) return HQ_EINVAL;
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    if (d_stats && cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
+    if (nch == 0) return cuda_rc(cudaMemsetAsync(d_offsets, 0, sizeof(uint64_t), s));
+    if (!x || !aligned(x, 16) || ld < cols || ld % 8) return HQ_EINVAL;
+    if (!d_stream || !aligned(d_stream, 4)) return HQ_EINVAL;
+    if (!workspace || !aligned(workspace, 8) || ws_bytes < ws_bytes_for(nch)) return HQ_EINVAL;
+    if (cudaMemsetAsync(workspace, 0, (size_t)nch * 8 + 8, s) != cudaSuccess) return HQ_ECUDA;
+
+    EncodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = (const uint16_t *)x;
+    a.map.kv = 0;
+    a.map.rows = rows;
+    a.map.cols = cols;
+    a.map.ld = ld;
+    a.n_chunks = nch;
+    a.chunk_base = 0;
+    a.c_scale = scale_fwd(p->alpha);
+    a.k = p->rice_k;
+    a.seed = p->seed;
+    a.stream = d_stream;
+    a.cap_words = cap_words;
+    a.offsets = d_offsets;
+    a.stats = d_stats;
+    a.lookback = (unsigned long long *)workspace;
+    a.ticket = (unsigned int *)((char *)workspace + nch * 8);
+    a.tcols = (int)(cols / kTile);
+    a.spin_limit = g_spin_limit;
+    return cuda_rc(launch_encode(p->lattice, p->dither, a, s));
+}
+
+int hq_dequantize(const uint32_t *d_stream, uint64_t stream_words, const uint64_t *d_offsets, int64_t rows,
+                  int64_t cols, const hq_params *p, void *out, int out_dtype, int64_t ld, hq_stats *d_stats,
+                  void *cuda_stream) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if ((rc = check_matrix(rows, cols))) return rc;
+    if (out_dtype != 0 && out_dtype != 1) return HQ_EINVAL;
+    if (d_stats && !aligned(d_stats, 8)) return HQ_EINVAL;
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    if (d_stats && cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
+    const uint64_t nch = chunks_of(rows, cols);
+    if (nch == 0) return HQ_OK;
+    if (!d_stream || !aligned(d_stream, 4) || !d_offsets || !aligned(d_offsets, 8)) return HQ_EINVAL;
+    if (!out || !aligned(out, 16) || ld < cols || ld % (out_dtype ? 4 : 8)) return HQ_EINVAL;
+
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.stream = d_stream;
+    a.stream_words = stream_words;
+    a.offsets = d_offsets;
+    a.map.kv = 0;
+    a.map.rows = rows;
+    a.map.cols = cols;
+    a.n_chunks = nch;
+    a.e_scale = scale_inv(p->alpha);
+    a.k = p->rice_k;
+    a.seed = p->seed;
+    a.out = out;
+    a.out_fp32 = out_dtype;
+    a.out_ld = ld;
+    a.stats = d_stats;
+    a.tcols = (int)(cols / kTile);
+    return cuda_rc(launch_decode(p->lattice, p->dither, a, s));
+}
+
+int hq_kv_init(hq_kv_cache *cache, int32_t heads, int32_t head_dim, const hq_params *p, uint32_t *d_words,
+               uint64_t cap_words, uint64_t *d_offsets, uint64_t offsets_cap, hq_kv_append_row *d_table,
+               uint64_t table_cap, uint64_t *d_tail, hq_stats *d_stats, void *cuda_stream) {
+    if (!cache || !p) return HQ_EINVAL;
+    if (p->lattice < HQ_Z || p->lattice > HQ_E8 || p->rice_k < 0 || p->rice_k > 15) return HQ_EINVAL;
+    if (p->dither != 0 && p->dither != 1) return HQ_EINVAL;
+    if (p->tile != kTile || p->chunk_tiles != kChunkTiles) return HQ_EUNSUPPORTED;
+    if (head_dim != kTile) return HQ_EUNSUPPORTED;
+    if (heads <= 0) return HQ_EINVAL;
+    if (!d_words || !aligned(d_words, 4) || !d_offsets || !aligned(d_offsets, 8) || offsets_cap < 1) return HQ_EINVAL;
+    if (!d_table || !aligned(d_table, 8) || table_cap < 1 || !d_tail || !aligned(d_tail, 8)) return HQ_EINVAL;
+    if (!d_stats || !aligned(d_stats, 8)) return HQ_EINVAL;
+    memset(cache, 0, sizeof(*cache));
+    cache->d_words = d_words;
+    cache->cap_words = cap_words;
+    cache->d_offsets = d_offsets;
+    cache->offsets_cap = offsets_cap;
+    cache->d_table = d_table;
+    cache->table_cap = table_cap;
+    cache->d_tail = d_tail;
+    cache->d_stats = d_stats;
+    cache->heads = heads;
+    cache->head_dim = head_dim;
+    cache->params = *p;
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    if (cudaMemsetAsync(d_tail, 0, 2 * sizeof(uint64_t), s) != cudaSuccess) return HQ_ECUDA;
+    if (cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
+    if (cudaMemsetAsync(d_offsets, 0, sizeof(uint64_t), s) != cudaSuccess) return HQ_ECUDA;
+    return HQ_OK;
+}
+
+int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t ld_token, int64_t ld_head, float alpha,
+                 void *workspace, size_t ws_bytes, void *cuda_stream) {
+    if (!cache || !cache->d_words) return HQ_EINVAL;
+    hq_params p = cache->params;
+    p.alpha = alpha;
+    int rc = check_params(&p);
+    if (rc) return rc;
+    if (T < 0) return HQ_EINVAL;
+    if (T == 0) return HQ_OK;
+    if (!kv || !aligned(kv, 16) || ld_token < kTile || ld_token % 8 || ld_head % 8 || ld_head < 0) return HQ_EINVAL;
+    const uint64_t H = (uint64_t)cache->heads;
+    const uint64_t nch = H * (uint64_t)((T + 31) / 32);
+    if (cache->chunks + nch + 1 > cache->offsets_cap || cache->appends + 1 > cache->table_cap) return HQ_EINVAL;
+    if (!workspace || !aligned(workspace, 8) || ws_bytes < ws_bytes_for(nch)) return HQ_EINVAL;
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    if (cudaMemsetAsync(workspace, 0, (size_t)nch * 8 + 8, s) != cudaSuccess) return HQ_ECUDA;
+
+    EncodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = (const uint16_t *)kv;
+    a.map.kv = 1;
+    a.map.heads = (int64_t)H;
+    a.map.tokens = T;
+    a.map.ld_tok = ld_token;
+    a.map.ld_head = ld_head;
+    a.map.tok0 = cache->tokens;
+    a.n_chunks = nch;
+    a.chunk_base = cache->chunks;
+    a.c_scale = scale_fwd(alpha);
+    a.k = p.rice_k;
+    a.seed = p.seed;
+    a.stream = cache->d_words;
+    a.cap_words = cache->cap_words;
+    a.offsets = cache->d_offsets;
+    a.base_ptr = cache->d_tail + (cache->appends & 1);
+    a.tail_out = cache->d_tail + ((cache->appends + 1) & 1);
+    a.row = cache->d_table + cache->appends;
+    a.row_val.first_chunk = cache->chunks;
+    a.row_val.token0 = cache->tokens;
+    a.row_val.tokens = (int32_t)T;
+    a.row_val.alpha = alpha;
+    a.row_val.scale_fwd = a.c_scale;
+    a.row_val.scale_inv = scale_inv(alpha);
+    a.stats = cache->d_stats;
+    a.lookback = (unsigned long long *)workspace;
+    a.ticket = (unsigned int *)((char *)workspace + nch * 8);
+    a.tcols = 1;
+    a.spin_limit = g_spin_limit;
+    rc = cuda_rc(launch_encode(p.lattice, p.dither, a, s));
+    if (rc) return rc;
+    cache->tokens += T;
+    cache->chunks += nch;
+    cache->appends += 1;
+    return HQ_OK;
+}
+
+int hq_kv_read(const hq_kv_cache *cache, void *out, int out_dtype, int64_t len, int64_t out_ld_token,
+               int64_t out_ld_head, void *cuda_stream) {
+    if (!cache || !cache->d_words) return HQ_EINVAL;
+    if (out_dtype != 0 && out_dtype != 1) return HQ_EINVAL;
+    if (len < 0 || len > cache->tokens) return HQ_EINVAL;
+    if (len == 0 || cache->chunks == 0) return HQ_OK;
+    const int m = out_dtype ? 4 : 8;
+    if (!out || !aligned(out, 16) || out_ld_token < kTile || out_ld_token % m || out_ld_head % m || out_ld_head < 0)
+        return HQ_EINVAL;
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.stream = cache->d_words;
+    a.stream_words = cache->cap_words;
+    a.offsets = cache->d_offsets;
+    a.map.kv = 1;
+    a.map.heads = cache->heads;
+    a.n_chunks = cache->chunks;
+    a.k = cache->params.rice_k;
+    a.seed = cache->params.seed;
+    a.out = out;
+    a.out_fp32 = out_dtype;
+    a.out_ld = out_ld_token;
+    a.out_ld_head = out_ld_head;
+    a.len = len;
+    a.table = cache->d_table;
+    a.n_appends = cache->appends;
+    a.stats = cache->d_stats;
+    a.tcols = 1;
+    return cuda_rc(launch_decode(cache->params.lattice, cache->params.dither, a, (cudaStream_t)cuda_stream));
+}
+
+const char *hq_status_string(int code) {
+    switch (code) {
+    case HQ_OK: return "ok";
+    case HQ_EINVAL: return "invalid argument";
+    case HQ_EUNSUPPORTED: return "unsupported by this build";
+    case HQ_ECUDA: return "CUDA error";
+    }
+    if (code > 0) {
+        if (code & HQ_ST_TIMEOUT) return "look-back timed out";
+        if (code & HQ_ST_CORRUPT) return "corrupt stream";
+        if (code & HQ_ST_CAPACITY) return "stream capacity exceeded";
+        if (code & HQ_ST_RANGE) return "value outside the supported range";
+    }
+    return "unknown";
+}
+
+int hq_device_check(void) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ECUDA;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return HQ_ECUDA;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return HQ_ECUDA;
+    return (major == 10 && minor == 0) ? HQ_OK : HQ_EUNSUPPORTED;
+}
+
+void hq_debug_set_spin_limit(uint32_t polls) { g_spin_limit = polls ? polls : kSpinLimit; }
+
+}  // extern "C"

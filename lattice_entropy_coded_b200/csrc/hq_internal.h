@@ -1,0 +1,80 @@
+// hq_internal.h -- launch arguments shared by the host entry points (hq_api.cu)
+// and the kernels (hq_encode.cu, hq_decode.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hq.h"
+
+namespace hq {
+
+constexpr int kTile = 128;          // elements per RHT tile
+constexpr int kChunkTiles = 32;     // tiles per chunk = lanes per warp (one tile per lane)
+constexpr int kSignStride = 68;     // words per tile column in the shared sign table (64 used, padded)
+constexpr int kWarpsPerCta = 4;     // warps per CTA in both kernels
+constexpr int kStageWords = 2048;   // per-warp shared staging for one chunk's words (encode and decode);
+                                    // holds the coset and remainder planes for every k (16 + 128*15 words)
+constexpr uint32_t kSpinLimit = 1u << 22;   // look-back polls before giving up (HQ_ST_TIMEOUT)
+constexpr uint32_t kMaxUnaryBits = 1u << 31; // chunks with more unary bits are outside the supported range
+
+// Salts xor-ed into the seed: "SIGN" for the sign diagonal, "DITH" for the dither.
+constexpr uint64_t kSignSalt = 0x5349474Eull;
+constexpr uint64_t kDitherSalt = 0x44495448ull;
+
+// How a chunk index maps to tiles.
+//  weights: chunk c = tiles [32c, 32c+32) of the row-major tile order of an R x C matrix.
+//  kv     : chunk c of an append = head c / cph, tokens [32 (c % cph), ...), cph = ceil(T/32).
+struct TileMap {
+    int kv;
+    int64_t rows, cols, ld;           // weights
+    int64_t heads, tokens, ld_tok, ld_head, tok0;  // kv
+};
+
+struct EncodeArgs {
+    const uint16_t *x;
+    TileMap map;
+    uint64_t n_chunks;        // chunks of this call
+    uint64_t chunk_base;      // global index of this call's first chunk (offset array position)
+    float c_scale;            // alpha / sqrt(128), rounded to fp32 on the host
+    int k;                    // Rice parameter
+    uint64_t seed;
+    uint32_t *stream;
+    uint64_t cap_words;
+    uint64_t *offsets;        // offsets[chunk_base + c] written for c in [0, n_chunks]
+    const uint64_t *base_ptr; // device word index where this call's stream starts (KV tail) or null (0)
+    uint64_t *tail_out;       // device word updated with the end of this call's stream, or null
+    hq_kv_append_row *row;    // KV: table row written by the warp of chunk 0, or null
+    hq_kv_append_row row_val;
+    hq_stats *stats;          // may be null
+    unsigned long long *lookback;  // n_chunks words, zeroed
+    unsigned int *ticket;          // one word, zeroed
+    int tcols;                // tile columns in the sign table (cols / 128, or 1 for KV)
+    uint32_t spin_limit;
+};
+
+struct DecodeArgs {
+    const uint32_t *stream;
+    uint64_t stream_words;
+    const uint64_t *offsets;
+    TileMap map;              // for KV the per-append fields come from the table
+    uint64_t n_chunks;
+    float e_scale;            // 1 / (alpha sqrt(128)), weights path
+    int k;
+    uint64_t seed;
+    void *out;
+    int out_fp32;
+    int64_t out_ld;           // weights: row stride; kv: token stride
+    int64_t out_ld_head;      // kv: head stride
+    int64_t len;              // kv: tokens to write
+    const hq_kv_append_row *table;  // kv: append table
+    uint64_t n_appends;
+    hq_stats *stats;
+    int tcols;
+};
+
+// Launchers (defined in hq_encode.cu / hq_decode.cu).  Return cudaSuccess or the launch error.
+cudaError_t launch_encode(int lattice, int dither, const EncodeArgs &a, cudaStream_t s);
+cudaError_t launch_decode(int lattice, int dither, const DecodeArgs &a, cudaStream_t s);
+
+}  // namespace hq

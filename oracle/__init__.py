@@ -302,13 +302,18 @@ def quantize(x, lat: int, alpha: float, k: int, seed: int, dither: int = 0, chun
 
 
 def dequantize(stream, offsets, rows: int, cols: int, lat: int, alpha: float, k: int, seed: int, dither: int = 0,
-               out_fp32: bool = False, chunk_lo: int = 0, chunk_hi: int | None = None) -> np.ndarray:
-    """Weights path inverse: returns float32 [R, C] (fp32 mode) or uint16 bf16 bits [R, C]."""
+               out_fp32: bool = False, chunk_lo: int = 0, chunk_hi: int | None = None,
+               out: np.ndarray | None = None) -> np.ndarray:
+    """Weights path inverse: float32 [R, C] (fp32 mode) or uint16 bf16 bits [R, C].
+    offsets[0] belongs to chunk chunk_lo; only that range's tiles of `out` are written."""
     if chunk_hi is None:
         chunk_hi = n_chunks(rows, cols)
     s = np.ascontiguousarray(stream, dtype=np.uint32)
     o = np.ascontiguousarray(offsets, dtype=np.uint64)
-    out = np.zeros((rows, cols), dtype=np.float32 if out_fp32 else np.uint16)
+    if out is None:
+        out = np.zeros((rows, cols), dtype=np.float32 if out_fp32 else np.uint16)
+    assert out.shape == (rows, cols) and out.flags["C_CONTIGUOUS"]
+    assert out.dtype == (np.float32 if out_fp32 else np.uint16)
     rc = lib().hqref_dequantize(_ptr(s), _ptr(o), rows, cols, lat, alpha, k, seed, dither, chunk_lo, chunk_hi,
                                 int(out_fp32), _ptr(out), cols)
     if rc != 0:

@@ -49,7 +49,7 @@ def kv_bits(kv_u16: np.ndarray, lat: int, alpha: float, k: int, seed: int) -> in
     return sum(res)
 
 
-def bisect_alpha(rate, target: float, tol: float = 0.002, lo: float = 1.0, hi: float = 4096.0):
+def bisect_alpha(rate, target: float, tol: float = 0.002, lo: float = 1e-3, hi: float = 1e4):
     rlo, rhi = rate(lo), rate(hi)
     if not (rlo <= target <= rhi):
         return None
@@ -92,8 +92,34 @@ def main():
     out = {"note": "alpha and Rice k per operating point; written by tests/golden/calibrate_points.py "
                    "from the CPU oracle only (payload bits per scalar on the named sample)",
            "workloads": {}}
+    if os.path.exists(OUT) and "--fresh" not in sys.argv:   # resume: keep finished workloads
+        with open(OUT) as f:
+            out["workloads"].update(json.load(f)["workloads"])
+
+    def save():
+        with open(OUT, "w") as f:
+            json.dump(out, f, indent=1)
 
     # 1. 1024x1024, E8, k = 2 fixed, alpha for 4 bps (full matrix).
+    if "weight_1024x1024_e8_4bps" not in out["workloads"]:
+        calib_1(out)
+        save()
+    if "weight_4096x4096_rate_sweep" not in out["workloads"]:
+        calib_2(out)
+        save()
+    if "kv_8h_32768tok_e8_dither" not in out["workloads"]:
+        calib_3(out)
+        save()
+    if "weights_8b_8layers_e8_4bps" not in out["workloads"]:
+        calib_4(out)
+        save()
+    if "student_t_64x8192x8192_e8" not in out["workloads"]:
+        calib_5(out)
+        save()
+    print("wrote", OUT)
+
+
+def calib_1(out):
     w = synth.WORKLOADS["weight_1024x1024_e8_4bps"]
     x = u16(synth.weight(w["rows"], w["cols"], w["seed"]))
     n = x.size
@@ -103,6 +129,9 @@ def main():
                                              "bps_payload_sample": r[1], "bps_payload_full": r[1]}]}
     print("cfg1", out["workloads"]["weight_1024x1024_e8_4bps"], flush=True)
 
+
+
+def calib_2(out):
     # 2. 4096x4096 rate sweep: sample = first 256 rows for k selection, full matrix to refine alpha.
     w = synth.WORKLOADS["weight_4096x4096_rate_sweep"]
     xf = u16(synth.weight(w["rows"], w["cols"], w["seed"]))
@@ -119,6 +148,9 @@ def main():
     out["workloads"]["weight_4096x4096_rate_sweep"] = {"sample": "rows 0..255 (k), full matrix (alpha)",
                                                        "points": pts}
 
+
+
+def calib_3(out):
     # 3. KV: K and V separately, E8 with dither, 2.0 and 1.7 bps; sample = first 2048 tokens of every head.
     w = synth.WORKLOADS["kv_8h_32768tok_e8_dither"]
     K, V = synth.kv(w["heads"], w["tokens"], w["seed"])
@@ -132,6 +164,9 @@ def main():
             print("cfg3", p, flush=True)
     out["workloads"]["kv_8h_32768tok_e8_dither"] = {"sample": "tokens 0..2047 of every head", "points": pts}
 
+
+
+def calib_4(out):
     # 4. 8-layer weight set, E8 4 bps, one alpha: sample = 64 rows of each matrix of layer 0.
     w = synth.WORKLOADS["weights_8b_8layers_e8_4bps"]
     mats = []
@@ -146,6 +181,9 @@ def main():
     out["workloads"]["weights_8b_8layers_e8_4bps"] = {"sample": "rows 0..63 of each layer-0 matrix",
                                                       "points": [p]}
 
+
+
+def calib_5(out):
     # 5. Student-t set, E8 at 3 and 4 bps: sample = 512 rows of the first matrix.
     w = synth.WORKLOADS["student_t_64x8192x8192_e8"]
     m0 = next(synth.student_t(1, 512, 8192, w["seed"]))
@@ -158,10 +196,6 @@ def main():
         print("cfg5", p, flush=True)
     out["workloads"]["student_t_64x8192x8192_e8"] = {"sample": "512x8192 Student-t matrix (CPU generator)",
                                                      "points": pts}
-
-    with open(OUT, "w") as f:
-        json.dump(out, f, indent=1)
-    print("wrote", OUT)
 
 
 if __name__ == "__main__":

@@ -1,0 +1,116 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry point
+include/hq.h declares, and its host-side logic (sizes, argument checks) is
+right.  No compute call is made here."""
+import ctypes as C
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "hq.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"HQ_API\s+(?:const\s+)?\w+\s*\*?\s*(hq_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("hq_quantize", "hq_dequantize", "hq_kv_append", "hq_kv_read", "hq_stream_bound",
+              "hq_workspace_bytes", "hq_kv_init", "hq_status_string", "hq_device_check"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import lattice_entropy_coded_b200 as hq
+    lib = C.CDLL(hq.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert name in hq.EXPORTS, f"binding misses {name}"
+
+
+def test_struct_layouts_match_header():
+    import lattice_entropy_coded_b200 as hq
+    assert C.sizeof(hq.hq_params) == 32
+    assert hq.hq_params.seed.offset == 16 and hq.hq_params.chunk_tiles.offset == 28
+    assert C.sizeof(hq.hq_stats) == 32 and hq.hq_stats.payload_bits.offset == 8
+    assert C.sizeof(hq.hq_kv_append_row) == 32
+    assert C.sizeof(hq.hq_kv_cache) == 128 and hq.hq_kv_cache.params.offset == 72
+
+
+def test_stream_bound_and_workspace():
+    import lattice_entropy_coded_b200 as hq
+    p = hq.make_params("E8", 300.0, 2)
+    w, n = hq.hq_stream_bound(1024, 1024, p, 255)
+    assert n == 256
+    # per chunk: 16 coset words + 4*2*32 remainder words + 4096 * (1 + 511 >> 2) bits
+    assert w == 256 * (16 + 256 + 4096 * (1 + (511 >> 2)) // 32)
+    w2, n2 = hq.hq_stream_bound(3, 384, p, 7)      # 9 tiles: one partial chunk
+    assert n2 == 1
+    assert w2 == math.ceil(16 * 9 / 32) + 4 * 2 * 9 + math.ceil(9 * 128 * (1 + (15 >> 2)) / 32)
+    assert hq.hq_stream_bound(0, 4096, p) == (0, 0)
+    assert hq.hq_workspace_bytes(1000) >= 1000 * 8 + 8
+    assert hq.hq_workspace_bytes(1000) % 256 == 0
+
+
+@pytest.mark.parametrize("bad", [
+    dict(lattice=7), dict(alpha=0.0), dict(alpha=float("nan")), dict(alpha=-1.0), dict(rice_k=16),
+    dict(rice_k=-1), dict(dither=2)])
+def test_invalid_params_rejected(bad):
+    import lattice_entropy_coded_b200 as hq
+    kw = dict(lattice=3, alpha=1.0, rice_k=2, seed=0, dither=0)
+    kw.update(bad)
+    p = hq.hq_params(128, kw["lattice"], kw["alpha"], kw["rice_k"], 0, kw["dither"], 32)
+    with pytest.raises(hq.HQError, match="invalid"):
+        hq.hq_stream_bound(32, 128, p)
+
+
+def test_unsupported_shapes_rejected():
+    import lattice_entropy_coded_b200 as hq
+    p = hq.make_params()
+    p.tile = 64
+    with pytest.raises(hq.HQError, match="unsupported"):
+        hq.hq_stream_bound(32, 128, p)
+    p = hq.make_params()
+    p.chunk_tiles = 16
+    with pytest.raises(hq.HQError, match="unsupported"):
+        hq.hq_stream_bound(32, 128, p)
+    p = hq.make_params()
+    with pytest.raises(hq.HQError, match="invalid"):
+        hq.hq_stream_bound(32, 100, p)          # cols not a multiple of 128
+    with pytest.raises(hq.HQError, match="unsupported"):
+        hq.hq_stream_bound(1, 128 * 1024, p)    # sign table too wide
+
+
+def test_entry_points_validate_before_touching_the_device():
+    """Null or misaligned pointers come back as HQ_EINVAL with no CUDA call made."""
+    import lattice_entropy_coded_b200 as hq
+    lib = hq._lib
+    p = hq.make_params()
+    off = C.c_uint64()
+    # misaligned offsets
+    assert lib.hq_quantize(None, 32, 128, 128, C.byref(p), None, 0, 3, None, None, 0, None) == hq.HQ_EINVAL
+    assert lib.hq_dequantize(None, 0, None, 32, 128, C.byref(p), None, 0, 128, None, None) == hq.HQ_EINVAL
+    assert lib.hq_dequantize(None, 0, None, 32, 128, C.byref(p), None, 2, 128, None, None) == hq.HQ_EINVAL
+    cache = hq.hq_kv_cache()
+    assert lib.hq_kv_init(C.byref(cache), 8, 64, C.byref(p), None, 0, None, 0, None, 0, None, None,
+                          None) == hq.HQ_EUNSUPPORTED
+    assert lib.hq_kv_append(C.byref(cache), None, 16, 128, 2048, C.c_float(1.0), None, 0, None) == hq.HQ_EINVAL
+    assert lib.hq_kv_read(C.byref(cache), None, 0, 1, 128, 2048, None) == hq.HQ_EINVAL
+    assert hq.hq_status_string(hq.HQ_ST_TIMEOUT) == "look-back timed out"
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """The binding has no fallback: a missing libhq.so is an import error."""
+    import subprocess
+    import sys
+    pkg = tmp_path / "lattice_entropy_coded_b200"
+    pkg.mkdir()
+    with open(os.path.join(ROOT, "lattice_entropy_coded_b200", "__init__.py")) as f:
+        (pkg / "__init__.py").write_text(f.read())
+    r = subprocess.run([sys.executable, "-c", "import lattice_entropy_coded_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libhq.so is missing" in r.stderr
