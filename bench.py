@@ -375,6 +375,44 @@ def run_reference(args):
             "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------ single-matrix case (profiling)
+def run_case(args):
+    """Quantize + decode one R x C synthetic weight matrix (seed 1) at one operating point of
+    the rate sweep, back to back, no L2 flush: the small case the ncu captures run on."""
+    import lattice_entropy_coded_b200 as hq
+    rows, cols = (int(v) for v in args.case.lower().split("x"))
+    p = [q for q in rate_points()[DEFAULT_WORKLOAD]["points"]
+         if q["lattice"] == args.lattice and q["bps"] == args.bps][0]
+    device = torch.device("cuda", 0)
+    x = synth.weight(rows, cols, seed=1, device=device)
+    params = hq.make_params(p["lattice"], p["alpha"], p["k"], 1, args.dither)
+    codec = hq.Codec(rows, cols, params, cap_words=int(x.numel() * (p["bps"] + 3.0) / 32) + 8192, device=device)
+    out = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
+    ev = []
+    for i in range(args.warmup + args.steps):
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record()
+        comp = codec.quantize(x)
+        b.record()
+        codec.dequantize(comp, out)
+        c.record()
+        if i >= args.warmup:
+            ev.append((a, b, c))
+    torch.cuda.synchronize()
+    st = hq.read_stats(codec.stats)
+    enc = float(np.median([a.elapsed_time(b) for a, b, _ in ev]))
+    dec = float(np.median([b.elapsed_time(c) for _, b, c in ev]))
+    n = x.numel()
+    words = int(codec.offsets[-1].item())
+    alg = 2.0 * n + 4.0 * words + 8.0 * (codec.n_chunks + 1)
+    peak, _ = measured_peaks()
+    print(json.dumps({"case": args.case, "lattice": p["lattice"], "bps": p["bps"], "dither": args.dither,
+                      "status": st["status"], "bps_payload": st["payload_bits"] / n,
+                      "enc_ms": enc, "dec_ms": dec, "enc_gbs_in": 2.0 * n / enc / 1e6, "dec_gbs_in": 2.0 * n / dec / 1e6,
+                      "enc_frac": alg / enc / 1e6 / peak, "dec_frac": alg / dec / 1e6 / peak,
+                      "alg_bytes": alg}), flush=True)
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -384,8 +422,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None, help="RxC: time one matrix (profiling case)")
+    ap.add_argument("--lattice", default="E8")
+    ap.add_argument("--bps", type=float, default=4.0)
+    ap.add_argument("--dither", type=int, default=0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.case:
+        run_case(args)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -155,14 +155,16 @@ __device__ __forceinline__ void tile_out(const DecodeArgs &a, unsigned long long
 }
 
 template <int LAT, bool DITHER, bool KV>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kWarpsPerCta * 32, 1) decode_kernel(const DecodeArgs a) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
-    extern __shared__ uint32_t smem[];
+    extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *sign_tab = smem;
-    uint32_t *stage_all = smem + a.tcols * kSignStride;
+    uint32_t *rows_all = smem + a.tcols * kSignStride;
+    uint32_t *stage_all = rows_all + kWarpsPerCta * 32 * kRowStride;
     uint32_t *start_all = stage_all + kWarpsPerCta * kStageWords;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float *row = reinterpret_cast<float *>(rows_all + (warp * 32 + lane) * kRowStride);
     uint32_t *stage = stage_all + warp * kStageWords;
     uint32_t *startbit = start_all + warp * 32;
 
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
         ok = ok && ones == nsym;
         if (ok) {
             const uint32_t before = incl - cnt;
-            // targets: terminator index j = 128 t - 1 for t = 1..ntiles-1 that falls in [before, incl)
+            // terminator index j = 128 t - 1 of tile t = 1..ntiles-1 inside [before, incl)
             uint32_t tt = (before + 1u + 127u) / 128u;
             if (tt == 0) tt = 1;
             uint32_t i = s0, seen = before;
@@ -224,27 +226,26 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
                     w = un[i];
                     pc = __popc(w);
                 }
-                // (j - seen)-th set bit of w
-                for (uint32_t r = j - seen; r; r--) w &= w - 1u;
+                for (uint32_t r = j - seen; r; r--) w &= w - 1u;   // drop the lower set bits
                 startbit[tt] = i * 32u + (uint32_t)(__ffs(w) - 1) + 1u;
             }
             if (lane == 0) startbit[0] = 0;
         }
         __syncwarp();
 
-        float v[kTile];
+        // ---- symbols -> lattice points -> scaled coordinates, group by group into the row
         bool lane_ok = ok;
         if (ok && t.valid) {
             UnaryReader ur;
             ur.init(un, nu, startbit[lane]);
             const uint32_t *rw = src + nc + 4ull * k * lane;
-            uint32_t coset = 0;
-            if (LAT == HQ_E8) coset = (src[lane >> 1] >> (16 * (lane & 1))) & 0xFFFFu;
-#pragma unroll
+            const uint32_t coset = (LAT == HQ_E8) ? (src[lane >> 1] >> (16 * (lane & 1))) & 0xFFFFu : 0u;
+#pragma unroll 1
             for (int g = 0; g < kTile / 8; g++) {
                 uint32_t qv[8], rv[8];
                 ur.group(qv);
                 rem_group(rw, k, g, rv);
+                float u[8];
 #pragma unroll
                 for (int bb = 0; bb < 8 / N; bb++) {
                     const int b = g * (8 / N) + bb;
@@ -256,49 +257,58 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
                     L::point(q, p);
                     if (DITHER) {
                         float d[N];
-                        dither_block<LAT>(a.seed, t.e0 + (unsigned long long)(b * N), d);
+                        dither_block<LAT>(a.seed, t.e0 + (unsigned long long)(8 * g + bb * N), d);
 #pragma unroll
                         for (int i = 0; i < N; i++) p[i] = __fsub_rn(p[i], d[i]);
                     }
 #pragma unroll
-                    for (int i = 0; i < N; i++) v[b * N + i] = __fmul_rn(p[i], t.e_scale);
+                    for (int i = 0; i < N; i++) u[bb * N + i] = p[i];
                 }
+                const float2 e2 = make_float2(t.e_scale, t.e_scale);
+                float2 s0v = f2_mul(make_float2(u[0], u[1]), e2), s1v = f2_mul(make_float2(u[2], u[3]), e2);
+                float2 s2v = f2_mul(make_float2(u[4], u[5]), e2), s3v = f2_mul(make_float2(u[6], u[7]), e2);
+                *reinterpret_cast<float4 *>(row + 8 * g) = make_float4(s0v.x, s0v.y, s1v.x, s1v.y);
+                *reinterpret_cast<float4 *>(row + 8 * g + 4) = make_float4(s2v.x, s2v.y, s3v.x, s3v.y);
             }
             lane_ok = ur.ok;
-            fwht128(v);
         }
         if (__any_sync(0xffffffffu, t.valid && !(ok && lane_ok))) status |= HQ_ST_CORRUPT;
-        if (!(ok && lane_ok)) {
-#pragma unroll
-            for (int i = 0; i < kTile; i++) v[i] = 0.0f;
-        }
 
-        // ---- sign, round, store
+        // ---- FWHT, sign, round, store
         if (t.dst) {
+            const bool good = ok && lane_ok;
+            float2 v[kTile / 2];
+#pragma unroll
+            for (int j = 0; j < kTile / 4; j++) {
+                float4 f = good ? *reinterpret_cast<const float4 *>(row + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[2 * j] = make_float2(f.x, f.y);
+                v[2 * j + 1] = make_float2(f.z, f.w);
+            }
+            fwht128(v);
             const uint32_t *sg = sign_tab + t.tcol * kSignStride;
             if (a.out_fp32) {
                 uint4 *o = reinterpret_cast<uint4 *>(t.dst);
 #pragma unroll
                 for (int j = 0; j < kTile / 4; j++) {
-                    uint32_t s0w = sg[2 * j], s1w = sg[2 * j + 1];
+                    const uint32_t s0w = sg[2 * j], s1w = sg[2 * j + 1];
                     uint4 w;
-                    w.x = __float_as_uint(v[4 * j]) ^ (s0w << 16);
-                    w.y = __float_as_uint(v[4 * j + 1]) ^ (s0w & 0x80000000u);
-                    w.z = __float_as_uint(v[4 * j + 2]) ^ (s1w << 16);
-                    w.w = __float_as_uint(v[4 * j + 3]) ^ (s1w & 0x80000000u);
+                    w.x = __float_as_uint(v[2 * j].x) ^ (s0w << 16);
+                    w.y = __float_as_uint(v[2 * j].y) ^ (s0w & 0x80000000u);
+                    w.z = __float_as_uint(v[2 * j + 1].x) ^ (s1w << 16);
+                    w.w = __float_as_uint(v[2 * j + 1].y) ^ (s1w & 0x80000000u);
                     o[j] = w;
                 }
             } else {
                 uint4 *o = reinterpret_cast<uint4 *>(t.dst);
 #pragma unroll
                 for (int j = 0; j < kTile / 8; j++) {
-                    uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
-                    uint32_t sw[4] = {s.x, s.y, s.z, s.w};
+                    const uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
+                    const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
                     uint32_t pk[4];
 #pragma unroll
-                    for (int u = 0; u < 4; u++) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * j + 2 * u], v[8 * j + 2 * u + 1]);
-                        pk[u] = *reinterpret_cast<uint32_t *>(&h) ^ sw[u];
+                    for (int u2 = 0; u2 < 4; u2++) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(v[4 * j + u2].x, v[4 * j + u2].y);
+                        pk[u2] = *reinterpret_cast<uint32_t *>(&h) ^ sw[u2];
                     }
                     o[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
@@ -314,8 +324,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
 
 template <int LAT, bool DITHER, bool KV>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
-    const size_t smem =
-        (size_t)(a.tcols * kSignStride + kWarpsPerCta * kStageWords + kWarpsPerCta * 32) * sizeof(uint32_t);
+    const size_t smem = (size_t)(a.tcols * kSignStride + kWarpsPerCta * 32 * kRowStride + kWarpsPerCta * kStageWords +
+                                 kWarpsPerCta * 32) *
+                        sizeof(uint32_t);
     auto kern = decode_kernel<LAT, DITHER, KV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

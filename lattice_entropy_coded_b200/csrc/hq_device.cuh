@@ -31,19 +31,50 @@ __device__ __forceinline__ uint32_t sign_bit(uint64_t seed, uint64_t j) {
     return (uint32_t)(splitmix64(seed ^ kSignSalt, j) >> 63);
 }
 
+// ------------------------------------------------------------------ packed fp32
+// sm_100 executes two IEEE round-to-nearest fp32 operations per instruction on
+// a register pair (add/sub/mul .rn.f32x2); each lane is rounded exactly like the
+// scalar operation, so results are bit-identical to scalar code.
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<unsigned long long *>(&a)),
+        "l"(*reinterpret_cast<unsigned long long *>(&b)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b) {
+    unsigned long long r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<unsigned long long *>(&a)),
+        "l"(*reinterpret_cast<unsigned long long *>(&b)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<unsigned long long *>(&a)),
+        "l"(*reinterpret_cast<unsigned long long *>(&b)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+
 // ------------------------------------------------------------------ FWHT-128
 // Unnormalised Walsh-Hadamard transform in Sylvester order, radix-2 stages
-// h = 1, 2, ..., 64, pair (i, i + h) -> (a + b, a - b).  The 1/sqrt(128) of the
-// orthonormal H_128 is folded into the scale factors.
-__device__ __forceinline__ void fwht128(float (&v)[kTile]) {
+// h = 1, 2, ..., 64, pair (i, i + h) -> (a + b, a - b).  The tile is held as
+// 64 float2 (elements 2j, 2j+1): stage 1 works inside each pair; for h >= 2
+// the butterflies of elements 2j and 2j+1 are independent and share a packed
+// add and a packed subtract.  The 1/sqrt(128) of the orthonormal H_128 is
+// folded into the scale factors.
+__device__ __forceinline__ void fwht128(float2 (&v)[kTile / 2]) {
 #pragma unroll
-    for (int h = 1; h < kTile; h <<= 1) {
+    for (int j = 0; j < kTile / 2; j++) {
+        float a = v[j].x, b = v[j].y;
+        v[j] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
 #pragma unroll
-        for (int i = 0; i < kTile; i++) {
-            if ((i & h) == 0) {
-                float a = v[i], b = v[i + h];
-                v[i] = __fadd_rn(a, b);
-                v[i + h] = __fsub_rn(a, b);
+    for (int hp = 1; hp < kTile / 2; hp <<= 1) {
+#pragma unroll
+        for (int j = 0; j < kTile / 2; j++) {
+            if ((j & hp) == 0) {
+                float2 a = v[j], b = v[j + hp];
+                v[j] = f2_add(a, b);
+                v[j + hp] = f2_sub(a, b);
             }
         }
     }

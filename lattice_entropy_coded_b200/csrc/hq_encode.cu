@@ -3,21 +3,20 @@
 // subtractive dither, nearest lattice point, bit-stripping, zigzag, Rice planes.
 //
 // Work decomposition (B200, sm_100a):
-//  * one warp encodes one chunk (32 tiles), one lane owns one tile: the whole
-//    transform runs in registers, no cross-lane traffic until the Rice scan;
+//  * one warp encodes one chunk (32 tiles), one lane owns one tile: load, sign
+//    flip, FWHT and scale run on 64 float2 registers with packed fp32 adds;
+//  * the transformed tile goes to a lane-private shared-memory row, and pass A
+//    walks it in a rolled loop over groups of 8 coordinates (one copy of the
+//    lattice decoder in the instruction stream), leaving the zigzag symbols in
+//    the row in place;
 //  * a persistent grid; warps take chunk tickets from a global counter, so a
-//    chunk's predecessors are always already running (look-back never waits on
-//    a warp that was not scheduled);
-//  * pass A (per lane, per group of 8 symbols): lattice decode, zigzag, the k
-//    remainder bits go straight into the lane's fixed region of a per-warp
-//    shared-memory stage, unary quotients are kept as packed bytes;
-//  * warp scan of unary lengths, single-pass decoupled look-back over 64-bit
-//    (flag, value) words for the chunk's word offset (every wait bounded:
+//    chunk's predecessors are always already running;
+//  * warp scan of the unary lengths and a single-pass decoupled look-back over
+//    64-bit (flag, value) words give the chunk's word offset (bounded waits:
 //    HQ_ST_TIMEOUT);
-//  * pass B: unary terminators placed into the stage, then the chunk is written
-//    with coalesced stores.  A chunk too large for the stage, or with a
-//    quotient above 255, is re-encoded by a slow path that writes global memory
-//    directly (same bits, bounded by the capacity).
+//  * pass B builds the remainder and unary planes in a per-warp shared stage
+//    and writes the chunk with coalesced stores; a chunk larger than the stage,
+//    or with quotients above 255, is written in place in global memory.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -39,8 +38,8 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
 
 // Exclusive prefix (in words) of chunk c over chunks [0, c) of this call.
 // Whole warp calls it; lane 0 publishes.  Bounded: gives up after spin_limit polls.
-__device__ unsigned long long lookback(unsigned long long *lb, unsigned long long c, unsigned long long agg,
-                                       uint32_t spin_limit, bool &timed_out) {
+__device__ __noinline__ unsigned long long lookback(unsigned long long *lb, unsigned long long c,
+                                                    unsigned long long agg, uint32_t spin_limit, bool &timed_out) {
     const int lane = threadIdx.x & 31;
     if (c == 0) {
         if (lane == 0) st_relaxed_u64(lb, kFlagInc | agg);
@@ -63,7 +62,7 @@ __device__ unsigned long long lookback(unsigned long long *lb, unsigned long lon
                 timed_out = true;
                 break;
             }
-            __nanosleep(64);
+            __nanosleep(32);
             continue;
         }
         excl += warp_sum_u64(lane <= first_inc ? (v & kValMask) : 0ull);
@@ -102,64 +101,65 @@ __device__ __forceinline__ bool tile_of(const TileMap &m, const uint16_t *x, uns
     return true;
 }
 
-// x (bf16, 128 elements) -> D x widened to fp32 -> H_128 -> * c.
-__device__ __forceinline__ void load_transform(const uint16_t *src, bool valid, const uint32_t *sg, float c_scale,
-                                               float (&v)[kTile]) {
+// x (bf16, 128 elements) -> D x widened to fp32 -> H_128 -> * c, stored to the
+// lane's row (16-byte stores).
+__device__ __forceinline__ void transform_to_row(const uint16_t *src, bool valid, const uint32_t *sg, float c_scale,
+                                                 float *row) {
+    float2 v[kTile / 2];
 #pragma unroll
     for (int j = 0; j < kTile / 8; j++) {
         uint4 w = valid ? ldg_nc_v4(src + 8 * j) : make_uint4(0, 0, 0, 0);
         uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
         uint32_t ww[4] = {w.x ^ s.x, w.y ^ s.y, w.z ^ s.z, w.w ^ s.w};
 #pragma unroll
-        for (int t = 0; t < 4; t++) {
-            v[8 * j + 2 * t] = __uint_as_float(ww[t] << 16);
-            v[8 * j + 2 * t + 1] = __uint_as_float(ww[t] & 0xFFFF0000u);
-        }
+        for (int t = 0; t < 4; t++)
+            v[4 * j + t] = make_float2(__uint_as_float(ww[t] << 16), __uint_as_float(ww[t] & 0xFFFF0000u));
     }
     fwht128(v);
+    const float2 c2 = make_float2(c_scale, c_scale);
 #pragma unroll
-    for (int i = 0; i < kTile; i++) v[i] = __fmul_rn(v[i], c_scale);
+    for (int j = 0; j < kTile / 4; j++) {
+        float2 a = f2_mul(v[2 * j], c2), b = f2_mul(v[2 * j + 1], c2);
+        *reinterpret_cast<float4 *>(row + 4 * j) = make_float4(a.x, a.y, b.x, b.y);
+    }
 }
 
-// Symbols z[0..7] of group g (8 consecutive coordinates) of the transformed tile;
-// ORs the E8 coset bits of the group's blocks into `coset`.
+// Symbols of group g (8 coordinates u[0..7]); returns the E8 coset bits of the
+// group's blocks (bit bb for block bb of the group).
 template <int LAT, bool DITHER>
-__device__ __forceinline__ void group_symbols(const float (&v)[kTile], int g, unsigned long long e0, uint64_t seed,
-                                              uint32_t (&z)[8], uint32_t &coset) {
+__device__ __forceinline__ uint32_t group_symbols(const float (&u)[8], int g, unsigned long long e0, uint64_t seed,
+                                                  uint32_t (&z)[8]) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
+    uint32_t cb = 0;
 #pragma unroll
     for (int bb = 0; bb < 8 / N; bb++) {
-        const int b = g * (8 / N) + bb;
         float blk[N];
 #pragma unroll
-        for (int i = 0; i < N; i++) blk[i] = v[b * N + i];
+        for (int i = 0; i < N; i++) blk[i] = u[bb * N + i];
         if (DITHER) {
             float d[N];
-            dither_block<LAT>(seed, e0 + (unsigned long long)(b * N), d);
+            dither_block<LAT>(seed, e0 + (unsigned long long)(8 * g + bb * N), d);
 #pragma unroll
             for (int i = 0; i < N; i++) blk[i] = __fadd_rn(blk[i], d[i]);
         }
         int32_t q[N], m[N];
         L::nearest(blk, q);
-        coset |= L::strip(q, m) << b;
+        cb |= L::strip(q, m) << bb;
 #pragma unroll
         for (int i = 0; i < N; i++) z[bb * N + i] = zigzag(m[i]);
     }
+    return cb;
 }
 
-// Pass-A writer of the remainder plane: k low bits per symbol, LSB first, into
-// the lane's own region `dst` (4k words).  k is warp-uniform, so every branch
-// here is uniform.
+// Remainder plane writer: k low bits per symbol, LSB first, into the lane's own
+// region `dst` (4k words).  k is warp-uniform, so the flushes are uniform.
 struct RemWriter {
     uint32_t *dst;
     int k;
-    uint32_t mask;
+    uint32_t mask, nb, w;
     bool store;
-    uint32_t acc;       // pending bits of the current word (k <= 4 path)
-    uint32_t nb;        // bits pending in acc
-    uint32_t w;         // next word index
-    unsigned long long acc64;
+    unsigned long long acc;
 
     __device__ __forceinline__ void init(uint32_t *d, int kk, bool st) {
         dst = d;
@@ -169,7 +169,6 @@ struct RemWriter {
         acc = 0;
         nb = 0;
         w = 0;
-        acc64 = 0;
     }
     __device__ __forceinline__ void put_group(const uint32_t (&z)[8]) {
         if (k == 0) return;
@@ -177,69 +176,68 @@ struct RemWriter {
             uint32_t gv = 0;   // 8k <= 32 bits, symbol 0 in the low bits
 #pragma unroll
             for (int i = 7; i >= 0; i--) gv = (gv << k) | (z[i] & mask);
-            const uint32_t len = 8u * (uint32_t)k;
-            acc |= gv << nb;
-            if (nb + len >= 32u) {
-                if (store) dst[w] = acc;
-                w++;
-                acc = nb ? (gv >> (32u - nb)) : 0u;
-                nb = nb + len - 32u;
-            } else {
-                nb += len;
-            }
+            acc |= (unsigned long long)gv << nb;
+            nb += 8u * (uint32_t)k;
         } else {
 #pragma unroll
             for (int i = 0; i < 8; i++) {
-                acc64 |= (unsigned long long)(z[i] & mask) << nb;
+                acc |= (unsigned long long)(z[i] & mask) << nb;
                 nb += (uint32_t)k;
                 if (nb >= 32u) {
-                    if (store) dst[w] = (uint32_t)acc64;
+                    if (store) dst[w] = (uint32_t)acc;
                     w++;
-                    acc64 >>= 32;
+                    acc >>= 32;
                     nb -= 32u;
                 }
             }
         }
+        if (nb >= 32u) {
+            if (store) dst[w] = (uint32_t)acc;
+            w++;
+            acc >>= 32;
+            nb -= 32u;
+        }
     }
 };
 
-// Slow path for one lane: re-encode the tile and write its remainder bits and
-// unary terminators straight into the chunk in global memory (already zeroed),
-// every access bounded by `room` words.
-template <int LAT, bool DITHER>
-__device__ __noinline__ void encode_tile_direct(const uint16_t *src, const uint32_t *sg, float c_scale, uint64_t seed,
-                                                unsigned long long e0, int k, uint32_t *g,
-                                                unsigned long long rem_bit0, unsigned long long un_bit0,
-                                                unsigned long long room) {
-    float v[kTile];
-    load_transform(src, true, sg, c_scale, v);
-    const uint32_t mask = k ? (1u << k) - 1u : 0u;
-    unsigned long long rb = rem_bit0, ub = un_bit0;
-    uint32_t coset = 0;
-#pragma unroll 1
-    for (int gi = 0; gi < kTile / 8; gi++) {
-        uint32_t z[8];
+// Unary terminators of 8 symbols with quotients q[0..7], starting at bit pos of
+// `un` (zeroed words).  A group whose codes fit in 32 bits is built in a
+// register (last symbol first) and ORed in with two shared atomics.
+__device__ __forceinline__ uint32_t unary_group_shared(uint32_t *un, uint32_t pos, const uint32_t (&q)[8]) {
+    uint32_t ug = 8;
 #pragma unroll
-        for (int gg = 0; gg < kTile / 8; gg++)
-            if (gg == gi) group_symbols<LAT, DITHER>(v, gg, e0, seed, z, coset);
+    for (int i = 0; i < 8; i++) ug += q[i];
+    if (ug <= 32u) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; i--) acc = ((acc << 1) | 1u) << q[i];
+        const uint32_t w0 = pos >> 5, sh = pos & 31u;
+        atomicOr(un + w0, acc << sh);
+        if (sh) {
+            const uint32_t hi = acc >> (32u - sh);
+            if (hi) atomicOr(un + w0 + 1, hi);
+        }
+    } else {
+        uint32_t p = pos;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            uint32_t r = z[i] & mask;
-            for (int b = 0; b < k; b++, rb++)
-                if (((r >> b) & 1u) && (rb >> 5) < room) atomicOr(g + (rb >> 5), 1u << (uint32_t)(rb & 31));
-            ub += z[i] >> k;
-            if ((ub >> 5) < room) atomicOr(g + (ub >> 5), 1u << (uint32_t)(ub & 31));
-            ub++;
+            p += q[i];
+            atomicOr(un + (p >> 5), 1u << (p & 31u));
+            p += 1;
         }
     }
+    return ug;
 }
 
 template <int LAT, bool DITHER>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const EncodeArgs a) {
-    extern __shared__ uint32_t smem[];
-    uint32_t *sign_tab = smem;                                   // tcols * kSignStride words
-    uint32_t *stage_all = smem + a.tcols * kSignStride;          // kWarpsPerCta * kStageWords
+__global__ void __launch_bounds__(kWarpsPerCta * 32, 1) encode_kernel(const EncodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *sign_tab = smem;                                                  // tcols * kSignStride
+    uint32_t *rows_all = smem + a.tcols * kSignStride;                          // warps * 32 * kRowStride
+    uint32_t *stage_all = rows_all + kWarpsPerCta * 32 * kRowStride;            // warps * kStageWords
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float *row = reinterpret_cast<float *>(rows_all + (warp * 32 + lane) * kRowStride);
+    uint32_t *zrow = rows_all + (warp * 32 + lane) * kRowStride;
     uint32_t *stage = stage_all + warp * kStageWords;
 
     // Sign masks per bf16x2 pair: bit 15 flips the even column, bit 31 the odd one.
@@ -266,36 +264,26 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         unsigned long long e0 = 0;
         const bool valid = tile_of(a.map, a.x, c, lane, src, tcol, e0, ntiles);
         const uint32_t *sg = sign_tab + tcol * kSignStride;
-        const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
-        const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
+        transform_to_row(src, valid, sg, a.c_scale, row);
 
-        // ---- transform
-        float v[kTile];
-        load_transform(src, valid, sg, a.c_scale, v);
-
-        // ---- pass A: symbols, remainder plane into the stage, packed unary quotients
-        uint32_t qpk[kTile / 4];
+        // ---- pass A: symbols in place of the transformed coordinates
         uint32_t coset = 0, usum = 0, zor = 0;
-        RemWriter rw;
-        rw.init(stage + nc + 4u * (uint32_t)k * (uint32_t)lane, k, valid);
-#pragma unroll
+#pragma unroll 1
         for (int g = 0; g < kTile / 8; g++) {
+            const float4 u0 = *reinterpret_cast<const float4 *>(row + 8 * g);
+            const float4 u1 = *reinterpret_cast<const float4 *>(row + 8 * g + 4);
+            const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
             uint32_t z[8];
-            group_symbols<LAT, DITHER>(v, g, e0, a.seed, z, coset);
-            if (!valid) {
-#pragma unroll
-                for (int i = 0; i < 8; i++) z[i] = 0;
-            }
-            rw.put_group(z);
-            uint32_t qq[8];
+            const uint32_t cb = group_symbols<LAT, DITHER>(u, g, e0, a.seed, z);
+            coset |= cb << (g * (8 / Lattice<LAT>::N));
 #pragma unroll
             for (int i = 0; i < 8; i++) {
+                if (!valid) z[i] = 0;
                 zor |= z[i];
-                qq[i] = z[i] >> k;
-                usum += qq[i];
+                usum += z[i] >> k;
             }
-            qpk[2 * g] = (qq[0] & 0xFFu) | ((qq[1] & 0xFFu) << 8) | ((qq[2] & 0xFFu) << 16) | (qq[3] << 24);
-            qpk[2 * g + 1] = (qq[4] & 0xFFu) | ((qq[5] & 0xFFu) << 8) | ((qq[6] & 0xFFu) << 16) | (qq[7] << 24);
+            *reinterpret_cast<uint4 *>(zrow + 8 * g) = make_uint4(z[0], z[1], z[2], z[3]);
+            *reinterpret_cast<uint4 *>(zrow + 8 * g + 4) = make_uint4(z[4], z[5], z[6], z[7]);
         }
         if (!valid) coset = 0;
         zor_all |= zor;
@@ -313,6 +301,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         const uint32_t wzor = __reduce_or_sync(0xffffffffu, zor);
         const bool range_bad = (wzor >> 22) != 0u || utotal >= kMaxUnaryBits;
         if (range_bad) status |= HQ_ST_RANGE;
+        const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
+        const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
         const unsigned long long nu = (utotal + 31) / 32;
         const unsigned long long total = nc + nr + nu;
         payload += utotal + (unsigned long long)nr * 32 + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
@@ -337,43 +327,25 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         const uint32_t cos_hi = __shfl_down_sync(0xffffffffu, coset, 1);
 
         if (fast) {
-            // ---- pass B: coset plane and unary terminators into the stage, then copy out
+            // ---- pass B: planes into the stage, then one coalesced copy
             for (uint32_t i = nc + nr + lane; i < (uint32_t)total; i += 32) stage[i] = 0u;
             if (LAT == HQ_E8 && (lane & 1) == 0 && (uint32_t)(lane >> 1) < nc) stage[lane >> 1] = coset | (cos_hi << 16);
             __syncwarp();
-            if (valid) {
-                uint32_t *un = stage + nc + nr;
-                uint32_t pos = (uint32_t)ustart;
+            RemWriter rw;
+            rw.init(stage + nc + 4u * (uint32_t)k * (uint32_t)lane, k, valid);
+            uint32_t *un = stage + nc + nr;
+            uint32_t pos = (uint32_t)ustart;
+#pragma unroll 1
+            for (int g = 0; g < kTile / 8; g++) {
+                const uint4 z0 = *reinterpret_cast<const uint4 *>(zrow + 8 * g);
+                const uint4 z1 = *reinterpret_cast<const uint4 *>(zrow + 8 * g + 4);
+                const uint32_t z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+                rw.put_group(z);
+                if (valid) {
+                    uint32_t q[8];
 #pragma unroll
-                for (int g = 0; g < kTile / 8; g++) {
-                    uint32_t qq[8];
-#pragma unroll
-                    for (int i = 0; i < 4; i++) {
-                        qq[i] = (qpk[2 * g] >> (8 * i)) & 0xFFu;
-                        qq[4 + i] = (qpk[2 * g + 1] >> (8 * i)) & 0xFFu;
-                    }
-                    uint32_t ug = 8;
-#pragma unroll
-                    for (int i = 0; i < 8; i++) ug += qq[i];
-                    if (ug <= 32u) {
-                        uint32_t acc = 0;
-#pragma unroll
-                        for (int i = 7; i >= 0; i--) acc = ((acc << 1) | 1u) << qq[i];
-                        const uint32_t w0 = pos >> 5, sh = pos & 31u;
-                        atomicOr(un + w0, acc << sh);
-                        if (sh) {
-                            const uint32_t hi = acc >> (32u - sh);
-                            if (hi) atomicOr(un + w0 + 1, hi);
-                        }
-                        pos += ug;
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 8; i++) {
-                            pos += qq[i];
-                            atomicOr(un + (pos >> 5), 1u << (pos & 31u));
-                            pos += 1;
-                        }
-                    }
+                    for (int i = 0; i < 8; i++) q[i] = z[i] >> k;
+                    pos += unary_group_shared(un, pos, q);
                 }
             }
             __syncwarp();
@@ -381,7 +353,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
                 if (start + i < a.cap_words) a.stream[start + i] = stage[i];
             __syncwarp();
         } else if (!range_bad) {
-            // ---- slow path: zero the chunk in place, then every lane re-encodes its tile into it
+            // ---- large chunk: zero it in place, then set every bit with a global atomic
             uint32_t *g = a.stream + start;
             const unsigned long long room = (start < a.cap_words) ? a.cap_words - start : 0ull;
             for (unsigned long long i = lane; i < total; i += 32)
@@ -390,10 +362,21 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             __threadfence_block();
             if (LAT == HQ_E8 && (lane & 1) == 0 && (uint32_t)(lane >> 1) < nc && (unsigned long long)(lane >> 1) < room)
                 atomicOr(g + (lane >> 1), coset | (cos_hi << 16));
-            if (valid)
-                encode_tile_direct<LAT, DITHER>(src, sg, a.c_scale, a.seed, e0, k, g,
-                                                32ull * (nc + 4ull * (unsigned long long)k * lane),
-                                                32ull * (nc + nr) + ustart, room);
+            if (valid) {
+                const uint32_t mask = k ? (1u << k) - 1u : 0u;
+                unsigned long long rb = 32ull * (nc + 4ull * (unsigned long long)k * lane);
+                unsigned long long ub = 32ull * (nc + nr) + ustart;
+#pragma unroll 1
+                for (int i = 0; i < kTile; i++) {
+                    const uint32_t zi = zrow[i];
+                    const uint32_t r = zi & mask;
+                    for (int b = 0; b < k; b++, rb++)
+                        if (((r >> b) & 1u) && (rb >> 5) < room) atomicOr(g + (rb >> 5), 1u << (uint32_t)(rb & 31));
+                    ub += zi >> k;
+                    if ((ub >> 5) < room) atomicOr(g + (ub >> 5), 1u << (uint32_t)(ub & 31));
+                    ub++;
+                }
+            }
             __syncwarp();
         }
     }
@@ -411,7 +394,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
 
 template <int LAT, bool DITHER>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
-    const size_t smem = (size_t)(a.tcols * kSignStride + kWarpsPerCta * kStageWords) * sizeof(uint32_t);
+    const size_t smem =
+        (size_t)(a.tcols * kSignStride + kWarpsPerCta * 32 * kRowStride + kWarpsPerCta * kStageWords) *
+        sizeof(uint32_t);
     auto kern = encode_kernel<LAT, DITHER>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -12,9 +12,11 @@ namespace hq {
 constexpr int kTile = 128;          // elements per RHT tile
 constexpr int kChunkTiles = 32;     // tiles per chunk = lanes per warp (one tile per lane)
 constexpr int kSignStride = 68;     // words per tile column in the shared sign table (64 used, padded)
-constexpr int kWarpsPerCta = 4;     // warps per CTA in both kernels
-constexpr int kStageWords = 2048;   // per-warp shared staging for one chunk's words (encode and decode);
-                                    // holds the coset and remainder planes for every k (16 + 128*15 words)
+constexpr int kWarpsPerCta = 8;     // warps per CTA in both kernels (one CTA per SM: shared memory bound)
+constexpr int kStageWords = 1024;   // per-warp shared staging for one chunk's words (encode and decode);
+                                    // larger chunks are written or read in place in global memory
+constexpr int kRowStride = 132;     // words per lane-private row of the transformed tile (128 + 4 pad:
+                                    // 16-byte accesses of 8 consecutive lanes hit distinct banks)
 constexpr uint32_t kSpinLimit = 1u << 22;   // look-back polls before giving up (HQ_ST_TIMEOUT)
 constexpr uint32_t kMaxUnaryBits = 1u << 31; // chunks with more unary bits are outside the supported range
 

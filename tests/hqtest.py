@@ -11,6 +11,7 @@ import torch
 
 import oracle as O
 
+POISON = 0xDEADBEEF          # fill of stream buffers: words nobody wrote keep it
 GOLD = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 THREADS = max(1, min(32, os.cpu_count() or 1))
 _POOL = ThreadPoolExecutor(THREADS)
@@ -65,13 +66,14 @@ def oracle_chunk(x: torch.Tensor, c: int, lat, alpha, k, seed, dither=0):
 
 
 # ---------------------------------------------------------------- CUDA path
-def gpu_quantize(x: torch.Tensor, params, cap_words: int | None = None, guard: int = 0, ld: int | None = None):
+def gpu_quantize(x: torch.Tensor, params, cap_words: int | None = None, guard: int = 0, ld: int | None = None,
+                 max_abs_symbol: int = 0):
     """x on the GPU (bf16).  -> dict(words np [total], offsets np, stats, words_t, offsets_t, cap)."""
     import lattice_entropy_coded_b200 as hq
     rows, cols = x.shape
-    bound, nch = hq.hq_stream_bound(rows, cols, params, 0)
+    bound, nch = hq.hq_stream_bound(rows, cols, params, max_abs_symbol)
     cap = bound if cap_words is None else cap_words
-    words = torch.full((cap + guard + 1,), -0x2152411, dtype=torch.int32, device=x.device)   # poison 0xDEADBEEF
+    words = torch.full((cap + guard + 1,), POISON - (1 << 32), dtype=torch.int32, device=x.device)
     offsets = torch.full((nch + 1,), -1, dtype=torch.int64, device=x.device)
     stats = hq.stats_tensor(x.device)
     ws = torch.empty(hq.hq_workspace_bytes(nch), dtype=torch.uint8, device=x.device)

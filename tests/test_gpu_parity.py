@@ -12,7 +12,7 @@ import torch
 
 import oracle as O
 import synth
-from hqtest import (assert_recon_equal, assert_same_words, gpu_dequantize, gpu_quantize, oracle_chunk,
+from hqtest import (POISON, assert_recon_equal, assert_same_words, gpu_dequantize, gpu_quantize, oracle_chunk,
                     oracle_dequantize, oracle_quantize, rate_points, u16)
 
 pytestmark = pytest.mark.gpu
@@ -26,7 +26,7 @@ def _hq():
     return hq
 
 
-def _roundtrip(x_cpu, lat, alpha, k, seed, dither=0, check_bf16=True, ld=None):
+def _roundtrip(x_cpu, lat, alpha, k, seed, dither=0, check_bf16=True, ld=None, max_abs_symbol=0):
     hq = _hq()
     p = hq.make_params(lat, alpha, k, seed, dither)
     if ld is None:
@@ -35,7 +35,7 @@ def _roundtrip(x_cpu, lat, alpha, k, seed, dither=0, check_bf16=True, ld=None):
         wide = torch.zeros(x_cpu.shape[0], ld, dtype=torch.bfloat16)
         wide[:, :x_cpu.shape[1]] = x_cpu
         xg = wide.cuda()[:, :x_cpu.shape[1]]
-    g = gpu_quantize(xg, p, ld=ld)
+    g = gpu_quantize(xg, p, ld=ld, max_abs_symbol=max_abs_symbol)
     ref_w, ref_off, ref_pay = oracle_quantize(x_cpu, lat, alpha, k, seed, dither)
     assert g["stats"]["status"] == 0, g["stats"]
     assert_same_words(g["words"], g["offsets"], ref_w, ref_off)
@@ -100,9 +100,10 @@ def test_ties_and_structured_inputs():
 def test_large_symbols_take_the_slow_path_with_the_same_bits():
     """alpha so large that chunks exceed the shared stage and quotients exceed 255."""
     x = synth.weight(64, 512, seed=12)
-    g, _ = _roundtrip(x, O.E8, 40000.0, 2, seed=2)
+    g, _ = _roundtrip(x, O.E8, 40000.0, 2, seed=2, max_abs_symbol=1 << 14)
     assert g["total"] / len(g["offsets"]) > 2048       # > stage size per chunk
-    g, _ = _roundtrip(x, O.Z, 3000.0, 0, seed=2)        # q > 255, chunks still small enough
+    assert g["stats"]["max_symbol"] >> 10                # quotients above 255
+    g, _ = _roundtrip(x, O.Z, 3000.0, 0, seed=2, max_abs_symbol=1 << 14)
 
 
 def test_config1_weight_tile_full():
@@ -150,7 +151,7 @@ def _kv_case(H, Ts, lat, alpha, k, seed, dither, source):
     hq = _hq()
     params = hq.make_params(lat, 1.0, k, seed, dither)
     total_t = sum(Ts)
-    cache = hq.KVCache(H, total_t, params, words_per_token_head=4.0, max_appends=len(Ts) + 1,
+    cache = hq.KVCache(H, total_t, params, words_per_token_head=16.0, max_appends=len(Ts) + 1,
                        max_append_tokens=max(Ts))
     appends, t0 = [], 0
     for T in Ts:
@@ -276,7 +277,7 @@ def test_capacity_overflow_is_flagged_and_bounded():
     assert g["stats"]["stream_words"] == need
     assert np.array_equal(g["offsets"], full["offsets"])
     assert np.array_equal(g["all_words"][:cap], full["words"][:cap])
-    assert np.all(g["all_words"][cap:] == np.uint32(0xDEADBEEF))   # nothing written past the cap
+    assert np.all(g["all_words"][cap:] == np.uint32(POISON))   # nothing written past the cap
 
 
 def test_corrupt_streams_are_flagged():
@@ -318,7 +319,7 @@ def test_lookback_spin_limit_never_hangs():
     finally:
         hq.hq_debug_set_spin_limit(0)
     assert g["stats"]["status"] & ~hq.HQ_ST_TIMEOUT == 0 or g["stats"]["status"] & hq.HQ_ST_CAPACITY
-    assert np.all(g["all_words"][g["cap"]:] == np.uint32(0xDEADBEEF))
+    assert np.all(g["all_words"][g["cap"]:] == np.uint32(POISON))
     if not g["stats"]["status"] & hq.HQ_ST_TIMEOUT:
         assert np.array_equal(g["words"], ref["words"])
     again = gpu_quantize(x, params)
