@@ -181,6 +181,35 @@ HQ_API int hq_dequantize(const uint32_t *d_stream, uint64_t stream_words, const 
                   int64_t cols, const hq_params *p, void *out, int out_dtype, int64_t ld, hq_stats *d_stats,
                   void *cuda_stream);
 
+/* No counterpart in the paper: an addition for callers that cannot allocate.
+ *
+ * hq_quantize without a workspace, for callers that hold only their input and
+ * output buffers and may not allocate device memory: for example a plug-in
+ * running inside a host application that owns every device allocation, or
+ * code on a path where cudaMalloc (which can synchronise the device) is not
+ * allowed.  Arguments, results and status are those of hq_quantize; the
+ * caller still passes x, d_stream, d_offsets and (optionally) d_stats.
+ *
+ * The encoder's scratch (8 bytes of chunk look-back state per chunk plus a
+ * ticket word) lives in a fixed array of HQ_STATIC_SCRATCH_BYTES inside
+ * libhq.so's device image; every GPU that loads the library holds it until the
+ * process exits.  Limit: at most HQ_STATIC_MAX_CHUNKS chunks (4096 elements
+ * each, about 537 million elements); a larger matrix returns HQ_EUNSUPPORTED
+ * and enqueues nothing.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and each clears the part it uses
+ * with a cudaMemsetAsync on its own stream, so calls that overlap on the GPU
+ * (other streams, or other host threads, without ordering between them) race
+ * and corrupt each other's streams: serialise them.  The call allocates
+ * nothing: no cudaMalloc, cudaFree or allocating library routine. */
+#define HQ_STATIC_SCRATCH_BYTES (1u << 20)
+#define HQ_STATIC_MAX_CHUNKS 131071u
+HQ_API int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p,
+                              uint32_t *d_stream, uint64_t cap_words, uint64_t *d_offsets, hq_stats *d_stats,
+                              void *cuda_stream);
+
 /* ----------------------------------------------------------------- KV path */
 
 /* Fill a hq_kv_cache with the caller's buffers and zero its two tail words

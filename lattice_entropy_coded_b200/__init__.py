@@ -70,6 +70,8 @@ EXPORTS = {
     "hq_status_string": (C.c_char_p, [C.c_int]),
     "hq_device_check": (C.c_int, []),
     "hq_debug_set_spin_limit": (None, [C.c_uint32]),
+    "hq_quantize_static": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.POINTER(hq_params), C.c_void_p,
+                                     C.c_uint64, C.c_void_p, C.c_void_p, C.c_void_p]),
 }
 
 
@@ -152,6 +154,16 @@ def hq_quantize(x: torch.Tensor, params: hq_params, stream: torch.Tensor, offset
     return _check(_lib.hq_quantize(_ptr(x), rows, cols, ld, C.byref(params), _ptr(stream), stream.numel(),
                                    _ptr(offsets), _ptr(stats), _ptr(workspace), workspace.numel(),
                                    _stream(cuda_stream)), "hq_quantize")
+
+
+def hq_quantize_static(x: torch.Tensor, params: hq_params, stream: torch.Tensor, offsets: torch.Tensor,
+                       stats: torch.Tensor | None, cuda_stream=None, ld: int | None = None) -> int:
+    """hq_quantize for callers that cannot allocate: its scratch is a fixed array inside
+    libhq.so (limit HQ_STATIC_MAX_CHUNKS chunks; overlapping calls on the GPU race)."""
+    rows, cols = x.shape
+    ld = x.stride(0) if ld is None else ld
+    return _check(_lib.hq_quantize_static(_ptr(x), rows, cols, ld, C.byref(params), _ptr(stream), stream.numel(),
+                                          _ptr(offsets), _ptr(stats), _stream(cuda_stream)), "hq_quantize_static")
 
 
 def hq_dequantize(stream: torch.Tensor, stream_words: int, offsets: torch.Tensor, rows: int, cols: int,
