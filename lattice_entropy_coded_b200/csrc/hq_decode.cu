@@ -27,10 +27,31 @@ __device__ __forceinline__ uint32_t fetch32(const uint32_t *p, uint32_t n, uint3
     return __funnelshift_r(a0, a1, b & 31u);
 }
 
+// Slow path of the unary reader: 8 quotients read one terminator at a time
+// (quotients may exceed the 32-bit window).  Kept out of line so the common
+// path stays compact.  Returns the new bit position; `ok` turns false if the
+// plane ends early.
+__device__ __noinline__ uint32_t unary_slow(const uint32_t *un, uint32_t nu, uint32_t bp, bool *ok, uint32_t *q) {
+    const uint32_t nbits = nu * 32u;
+    for (int i = 0; i < 8; i++) {
+        uint32_t t = 0;
+        uint32_t x = __brev(fetch32(un, nu, bp));
+        while (x == 0u && *ok) {
+            t += 32u;
+            bp += 32u;
+            if (bp >= nbits) *ok = false;
+            x = __brev(fetch32(un, nu, bp));
+        }
+        const uint32_t c = __clz(x);
+        q[i] = t + c;
+        bp += c + 1u;
+    }
+    return bp;
+}
+
 // Sequential reader of one lane's unary quotients: a bit-reversed 32-bit
-// window, so a quotient is one count-leading-zeros and one shift.  Groups of 8
-// whose codes fit in the window take the fast path; longer ones go bit-word by
-// bit-word.  `ok` turns false if the plane ends early.
+// window, so a quotient is one count-leading-zeros and one shift.  A group of 8
+// whose codes fit in the window takes the fast path.
 struct UnaryReader {
     const uint32_t *un;
     uint32_t nu, nbits, bp;
@@ -49,55 +70,39 @@ struct UnaryReader {
             uint32_t used = 8;
 #pragma unroll
             for (int i = 0; i < 8; i++) {
-                uint32_t t = __clz(w);
+                const uint32_t t = __clz(w);
                 q[i] = t;
                 used += t;
                 w = (w << t) << 1;
             }
             bp += used;
         } else {
+            uint32_t tmp[8];
+            bp = unary_slow(un, nu, bp, &ok, tmp);
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                uint32_t t = 0;
-                uint32_t x = __brev(fetch32(un, nu, bp));
-                while (x == 0u && ok) {
-                    t += 32u;
-                    bp += 32u;
-                    if (bp >= nbits) ok = false;
-                    x = __brev(fetch32(un, nu, bp));
-                }
-                uint32_t c = __clz(x);
-                t += c;
-                bp += c + 1u;
-                q[i] = t;
-            }
+            for (int i = 0; i < 8; i++) q[i] = tmp[i];
         }
         if (bp > nbits) ok = false;
     }
 };
 
-// k-bit remainders of one group of 8 symbols from the lane's region `rw` (4k words).
+// k-bit remainders of group g (8 symbols) from the lane's region `rw` (k words
+// per 32 symbols).  KSMALL (k <= 4): one 32-bit window per group.
+template <bool KSMALL>
 __device__ __forceinline__ void rem_group(const uint32_t *rw, int k, int g, uint32_t (&r)[8]) {
     if (k == 0) {
 #pragma unroll
         for (int i = 0; i < 8; i++) r[i] = 0;
         return;
     }
-    const uint32_t n = 4u * (uint32_t)k;
+    const uint32_t n = (uint32_t)k;   // words in the lane's region per round
     const uint32_t mask = (1u << k) - 1u;
     const uint32_t b = (uint32_t)(8 * g) * (uint32_t)k;
-    if (k <= 4) {
+    if (KSMALL) {
         uint32_t x = fetch32(rw, n, b);
 #pragma unroll
         for (int i = 0; i < 8; i++) {
             r[i] = x & mask;
-            x >>= k;
-        }
-    } else if (k <= 8) {
-        unsigned long long x = ((unsigned long long)fetch32(rw, n, b + 32u) << 32) | fetch32(rw, n, b);
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            r[i] = (uint32_t)x & mask;
             x >>= k;
         }
     } else {
@@ -106,84 +111,98 @@ __device__ __forceinline__ void rem_group(const uint32_t *rw, int k, int g, uint
     }
 }
 
-struct TileOut {
-    bool valid;
-    char *dst;          // first element of the tile in `out`
-    int tcol;
-    unsigned long long e0;
+// Where the tiles of one chunk go (computed once per chunk).
+template <bool KV>
+struct ChunkOut {
+    int ntiles;
     float e_scale;
+    long long row0, h, tok_base, tok0;
+    int tc0, tpr;
+
+    __device__ __forceinline__ void init(const DecodeArgs &a, unsigned long long c) {
+        if (KV) {
+            // the append that holds global chunk c (binary search on first_chunk)
+            unsigned long long lo = 0, hi = a.n_appends - 1;
+            while (lo < hi) {
+                const unsigned long long mid = (lo + hi + 1) >> 1;
+                if (a.table[mid].first_chunk <= c) lo = mid; else hi = mid - 1;
+            }
+            const hq_kv_append_row row = a.table[lo];
+            const long long T = row.tokens, cph = (T + 31) / 32;
+            const long long lc = (long long)(c - row.first_chunk);
+            h = lc / cph;
+            tok_base = (lc % cph) * 32;
+            tok0 = row.token0;
+            const long long left = T - tok_base;
+            ntiles = (int)(left < 32 ? left : 32);
+            e_scale = row.scale_inv;
+        } else {
+            tpr = (int)(a.map.cols / kTile);
+            const long long t0 = (long long)c * 32, all = a.map.rows * (long long)tpr;
+            ntiles = (int)((all - t0) < 32 ? (all - t0) : 32);
+            row0 = t0 / tpr;
+            tc0 = (int)(t0 - row0 * tpr);
+            e_scale = a.e_scale;
+        }
+    }
+    // Tile ti of the chunk: destination of its element 0 (null if not stored), sign
+    // column, dither counter of element 0.
+    __device__ __forceinline__ bool tile(const DecodeArgs &a, int ti, char *&dst, int &tcol,
+                                         unsigned long long &e0) const {
+        dst = nullptr;
+        if (ti >= ntiles) return false;
+        const size_t esz = a.out_fp32 ? 4 : 2;
+        if (KV) {
+            const long long gt = tok0 + tok_base + ti;
+            tcol = 0;
+            e0 = (unsigned long long)((gt * a.map.heads + h) * kTile);
+            if (gt < a.len) dst = (char *)a.out + (size_t)(h * a.out_ld_head + gt * a.out_ld) * esz;
+            return true;
+        }
+        int tc = tc0 + ti;
+        long long r = row0;
+        if (tc >= tpr) {
+            const int d = tc / tpr;
+            r += d;
+            tc -= d * tpr;
+        }
+        tcol = tc;
+        e0 = (unsigned long long)(r * a.map.cols + (long long)tc * kTile);
+        dst = (char *)a.out + (size_t)(r * a.out_ld + (long long)tc * kTile) * esz;
+        return true;
+    }
 };
 
-template <bool KV>
-__device__ __forceinline__ void tile_out(const DecodeArgs &a, unsigned long long c, int lane, TileOut &t,
-                                         int &ntiles) {
-    const size_t esz = a.out_fp32 ? 4 : 2;
-    if (KV) {
-        // the append that holds global chunk c (binary search on first_chunk)
-        unsigned long long lo = 0, hi = a.n_appends - 1;
-        while (lo < hi) {
-            unsigned long long mid = (lo + hi + 1) >> 1;
-            if (a.table[mid].first_chunk <= c) lo = mid; else hi = mid - 1;
-        }
-        const hq_kv_append_row row = a.table[lo];
-        long long T = row.tokens;
-        long long cph = (T + 31) / 32;
-        long long lc = (long long)(c - row.first_chunk);
-        long long h = lc / cph, tc = lc % cph;
-        long long tok = tc * 32 + lane;
-        long long ntok = T - tc * 32;
-        ntiles = (int)(ntok < 32 ? ntok : 32);
-        long long gt = row.token0 + tok;
-        t.valid = tok < T;
-        t.e_scale = row.scale_inv;
-        t.tcol = 0;
-        t.e0 = (unsigned long long)((gt * a.map.heads + h) * kTile);
-        t.dst = (t.valid && gt < a.len) ? (char *)a.out + (size_t)(h * a.out_ld_head + gt * a.out_ld) * esz : nullptr;
-        return;
-    }
-    long long tpr = a.map.cols / kTile;
-    long long ntile_all = a.map.rows * tpr;
-    long long t0 = (long long)c * 32;
-    long long ti = t0 + lane;
-    ntiles = (int)((ntile_all - t0) < 32 ? (ntile_all - t0) : 32);
-    t.valid = ti < ntile_all;
-    long long r = ti / tpr, tc = ti % tpr;
-    t.tcol = (int)tc;
-    t.e0 = (unsigned long long)(r * a.map.cols + tc * kTile);
-    t.e_scale = a.e_scale;
-    t.dst = t.valid ? (char *)a.out + (size_t)(r * a.out_ld + tc * kTile) * esz : nullptr;
-}
-
-template <int LAT, bool DITHER, bool KV>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, 1) decode_kernel(const DecodeArgs a) {
+template <int LAT, bool DITHER, bool KV, bool KSMALL>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const DecodeArgs a) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *sign_tab = smem;
-    uint32_t *rows_all = smem + a.tcols * kSignStride;
-    uint32_t *stage_all = rows_all + kWarpsPerCta * 32 * kRowStride;
+    uint32_t *stage_all = smem + a.tcols * kSignStride;
     uint32_t *start_all = stage_all + kWarpsPerCta * kStageWords;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float *row = reinterpret_cast<float *>(rows_all + (warp * 32 + lane) * kRowStride);
     uint32_t *stage = stage_all + warp * kStageWords;
-    uint32_t *startbit = start_all + warp * 32;
+    uint32_t *startbit = start_all + warp * 128;   // first unary bit of every 32-symbol segment
 
     for (int i = threadIdx.x; i < a.tcols * 64; i += blockDim.x) {
-        int tc = i >> 6, p = i & 63;
-        unsigned long long col = (unsigned long long)tc * kTile + 2 * p;
-        sign_tab[tc * kSignStride + p] = (sign_bit(a.seed, col) << 15) | (sign_bit(a.seed, col + 1) << 31);
+        const int tc = i >> 6, p = i & 63;
+        const unsigned long long col = (unsigned long long)tc * kTile + 2 * p;
+        sign_tab[tc * kSignStride + (p >> 4) * kSignQuarter + (p & 15)] =
+            (sign_bit(a.seed, col) << 15) | (sign_bit(a.seed, col + 1) << 31);
     }
     __syncthreads();
 
     const int k = a.k;
+    const int q = lane & 3;
     uint32_t status = 0;
     const unsigned long long nwarps = (unsigned long long)gridDim.x * kWarpsPerCta;
     for (unsigned long long c = (unsigned long long)blockIdx.x * kWarpsPerCta + warp; c < a.n_chunks; c += nwarps) {
-        TileOut t;
-        int ntiles = 0;
-        tile_out<KV>(a, c, lane, t, ntiles);
+        ChunkOut<KV> geo;
+        geo.init(a, c);
+        const int ntiles = geo.ntiles;
         const unsigned long long w0 = a.offsets[c], w1 = a.offsets[c + 1];
-        const uint32_t nsym = (uint32_t)ntiles * kTile;
+        const uint32_t nsym = (uint32_t)ntiles * kTile, nseg = 4u * (uint32_t)ntiles;
         const unsigned long long nc = (LAT == HQ_E8) ? (unsigned long long)(16 * ntiles + 31) / 32 : 0ull;
         const unsigned long long nr = 4ull * (unsigned long long)k * (unsigned long long)ntiles;
         bool ok = w0 <= w1 && w1 <= a.stream_words && (w1 - w0) >= nc + nr &&
@@ -198,7 +217,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 1) decode_kernel(const Deco
         const uint32_t nu = ok ? (uint32_t)(nw - nc - nr) : 0u;
         const uint32_t *un = src + nc + nr;
 
-        // ---- where does each tile's first codeword start?  (popc + scan over 32 segments)
+        // ---- first unary bit of every 32-symbol segment: popc + scan over 32 word ranges
         const uint32_t seg = (nu + 31u) / 32u;
         const uint32_t s0 = min(nu, (uint32_t)lane * seg), s1 = min(nu, s0 + seg);
         uint32_t cnt = 0;
@@ -206,19 +225,19 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 1) decode_kernel(const Deco
         uint32_t incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
         const uint32_t ones = __shfl_sync(0xffffffffu, incl, 31);
         ok = ok && ones == nsym;
         if (ok) {
             const uint32_t before = incl - cnt;
-            // terminator index j = 128 t - 1 of tile t = 1..ntiles-1 inside [before, incl)
-            uint32_t tt = (before + 1u + 127u) / 128u;
-            if (tt == 0) tt = 1;
+            // terminator j = 32 s - 1 closes segment s - 1; find those inside [before, incl)
+            uint32_t ss = (before + 1u + 31u) / 32u;
+            if (ss == 0) ss = 1;
             uint32_t i = s0, seen = before;
-            for (; tt < (uint32_t)ntiles && 128u * tt - 1u < incl; tt++) {
-                const uint32_t j = 128u * tt - 1u;
+            for (; ss < nseg && 32u * ss - 1u < incl; ss++) {
+                const uint32_t j = 32u * ss - 1u;
                 uint32_t w = un[i], pc = __popc(w);
                 while (seen + pc <= j) {
                     seen += pc;
@@ -227,93 +246,105 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 1) decode_kernel(const Deco
                     pc = __popc(w);
                 }
                 for (uint32_t r = j - seen; r; r--) w &= w - 1u;   // drop the lower set bits
-                startbit[tt] = i * 32u + (uint32_t)(__ffs(w) - 1) + 1u;
+                startbit[ss] = i * 32u + (uint32_t)(__ffs(w) - 1) + 1u;
             }
             if (lane == 0) startbit[0] = 0;
         }
         __syncwarp();
 
-        // ---- symbols -> lattice points -> scaled coordinates, group by group into the row
-        bool lane_ok = ok;
-        if (ok && t.valid) {
-            UnaryReader ur;
-            ur.init(un, nu, startbit[lane]);
-            const uint32_t *rw = src + nc + 4ull * k * lane;
-            const uint32_t coset = (LAT == HQ_E8) ? (src[lane >> 1] >> (16 * (lane & 1))) & 0xFFFFu : 0u;
+        // ---- 4 rounds of 8 tiles: lane decodes segment 32 r + lane = quarter q of tile 8 r + lane / 4
+        bool bad = false;
+        const int nrounds = (ntiles + kTilesPerRound - 1) / kTilesPerRound;
 #pragma unroll 1
-            for (int g = 0; g < kTile / 8; g++) {
-                uint32_t qv[8], rv[8];
-                ur.group(qv);
-                rem_group(rw, k, g, rv);
-                float u[8];
+        for (int r = 0; r < nrounds; r++) {
+            char *dst = nullptr;
+            int tcol = 0;
+            unsigned long long e0 = 0;
+            const bool valid = geo.tile(a, r * kTilesPerRound + (lane >> 2), dst, tcol, e0);
+            const uint32_t segi = 32u * r + lane;
+            float2 v[16];
+            bool lane_ok = ok;
+            if (ok && valid) {
+                UnaryReader ur;
+                ur.init(un, nu, startbit[segi]);
+                const uint32_t *rw = src + nc + (unsigned long long)segi * k;
+                const uint32_t cw = (LAT == HQ_E8) ? src[4 * r + (lane >> 3)] : 0u;
+                const uint32_t coset = (cw >> (4 * (lane & 7))) & 0xFu;
+                const unsigned long long eq = e0 + 32ull * q;
 #pragma unroll
-                for (int bb = 0; bb < 8 / N; bb++) {
-                    const int b = g * (8 / N) + bb;
-                    int32_t m[N], q[N];
-                    float p[N];
+                for (int g = 0; g < 4; g++) {
+                    uint32_t qv[8], rv[8];
+                    ur.group(qv);
+                    rem_group<KSMALL>(rw, k, g, rv);
+                    float u[8];
 #pragma unroll
-                    for (int i = 0; i < N; i++) m[i] = unzigzag((qv[bb * N + i] << k) | rv[bb * N + i]);
-                    L::reinsert(m, (coset >> b) & 1u, q);
-                    L::point(q, p);
-                    if (DITHER) {
-                        float d[N];
-                        dither_block<LAT>(a.seed, t.e0 + (unsigned long long)(8 * g + bb * N), d);
+                    for (int bb = 0; bb < 8 / N; bb++) {
+                        const int b = g * (8 / N) + bb;
+                        int32_t m[N], qq[N];
+                        float p[N];
 #pragma unroll
-                        for (int i = 0; i < N; i++) p[i] = __fsub_rn(p[i], d[i]);
+                        for (int i = 0; i < N; i++) m[i] = unzigzag((qv[bb * N + i] << k) | rv[bb * N + i]);
+                        L::reinsert(m, (coset >> b) & 1u, qq);
+                        L::point(qq, p);
+                        if (DITHER) {
+                            float d[N];
+                            dither_block<LAT>(a.seed, eq + (unsigned long long)(8 * g + bb * N), d);
+#pragma unroll
+                            for (int i = 0; i < N; i++) p[i] = __fsub_rn(p[i], d[i]);
+                        }
+#pragma unroll
+                        for (int i = 0; i < N; i++) u[bb * N + i] = p[i];
                     }
+                    const float2 e2 = make_float2(geo.e_scale, geo.e_scale);
 #pragma unroll
-                    for (int i = 0; i < N; i++) u[bb * N + i] = p[i];
+                    for (int j = 0; j < 4; j++) v[4 * g + j] = f2_mul(make_float2(u[2 * j], u[2 * j + 1]), e2);
                 }
-                const float2 e2 = make_float2(t.e_scale, t.e_scale);
-                float2 s0v = f2_mul(make_float2(u[0], u[1]), e2), s1v = f2_mul(make_float2(u[2], u[3]), e2);
-                float2 s2v = f2_mul(make_float2(u[4], u[5]), e2), s3v = f2_mul(make_float2(u[6], u[7]), e2);
-                *reinterpret_cast<float4 *>(row + 8 * g) = make_float4(s0v.x, s0v.y, s1v.x, s1v.y);
-                *reinterpret_cast<float4 *>(row + 8 * g + 4) = make_float4(s2v.x, s2v.y, s3v.x, s3v.y);
-            }
-            lane_ok = ur.ok;
-        }
-        if (__any_sync(0xffffffffu, t.valid && !(ok && lane_ok))) status |= HQ_ST_CORRUPT;
-
-        // ---- FWHT, sign, round, store
-        if (t.dst) {
-            const bool good = ok && lane_ok;
-            float2 v[kTile / 2];
-#pragma unroll
-            for (int j = 0; j < kTile / 4; j++) {
-                float4 f = good ? *reinterpret_cast<const float4 *>(row + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[2 * j] = make_float2(f.x, f.y);
-                v[2 * j + 1] = make_float2(f.z, f.w);
-            }
-            fwht128(v);
-            const uint32_t *sg = sign_tab + t.tcol * kSignStride;
-            if (a.out_fp32) {
-                uint4 *o = reinterpret_cast<uint4 *>(t.dst);
-#pragma unroll
-                for (int j = 0; j < kTile / 4; j++) {
-                    const uint32_t s0w = sg[2 * j], s1w = sg[2 * j + 1];
-                    uint4 w;
-                    w.x = __float_as_uint(v[2 * j].x) ^ (s0w << 16);
-                    w.y = __float_as_uint(v[2 * j].y) ^ (s0w & 0x80000000u);
-                    w.z = __float_as_uint(v[2 * j + 1].x) ^ (s1w << 16);
-                    w.w = __float_as_uint(v[2 * j + 1].y) ^ (s1w & 0x80000000u);
-                    o[j] = w;
-                }
+                lane_ok = ur.ok;
             } else {
-                uint4 *o = reinterpret_cast<uint4 *>(t.dst);
 #pragma unroll
-                for (int j = 0; j < kTile / 8; j++) {
-                    const uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
-                    const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
-                    uint32_t pk[4];
+                for (int j = 0; j < 16; j++) v[j] = make_float2(0.0f, 0.0f);
+            }
+            if (valid && !lane_ok) {
+                bad = true;
 #pragma unroll
-                    for (int u2 = 0; u2 < 4; u2++) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(v[4 * j + u2].x, v[4 * j + u2].y);
-                        pk[u2] = *reinterpret_cast<uint32_t *>(&h) ^ sw[u2];
+                for (int j = 0; j < 16; j++) v[j] = make_float2(0.0f, 0.0f);
+            }
+            fwht128_quarter(v, lane);
+            // a tile is good only if all four of its lanes are
+            const unsigned bad_lanes = __ballot_sync(0xffffffffu, valid && !lane_ok);
+            const bool tile_bad = (bad_lanes >> (lane & ~3)) & 0xFu;
+            if (dst) {
+                const uint32_t *sg = sign_tab + tcol * kSignStride + q * kSignQuarter;
+                if (a.out_fp32) {
+                    uint4 *o = reinterpret_cast<uint4 *>(dst) + 8 * q;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        const uint32_t s0w = sg[2 * j], s1w = sg[2 * j + 1];
+                        uint4 w;
+                        w.x = tile_bad ? 0u : __float_as_uint(v[2 * j].x) ^ (s0w << 16);
+                        w.y = tile_bad ? 0u : __float_as_uint(v[2 * j].y) ^ (s0w & 0x80000000u);
+                        w.z = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].x) ^ (s1w << 16);
+                        w.w = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].y) ^ (s1w & 0x80000000u);
+                        o[j] = w;
                     }
-                    o[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                } else {
+                    uint4 *o = reinterpret_cast<uint4 *>(dst) + 4 * q;
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
+                        const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int u2 = 0; u2 < 4; u2++) {
+                            __nv_bfloat162 hb = __floats2bfloat162_rn(v[4 * j + u2].x, v[4 * j + u2].y);
+                            pk[u2] = tile_bad ? 0u : (*reinterpret_cast<uint32_t *>(&hb) ^ sw[u2]);
+                        }
+                        o[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
                 }
             }
         }
+        if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) status |= HQ_ST_CORRUPT;
         __syncwarp();
     }
     if (a.stats) {
@@ -324,10 +355,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 1) decode_kernel(const Deco
 
 template <int LAT, bool DITHER, bool KV>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
-    const size_t smem = (size_t)(a.tcols * kSignStride + kWarpsPerCta * 32 * kRowStride + kWarpsPerCta * kStageWords +
-                                 kWarpsPerCta * 32) *
-                        sizeof(uint32_t);
-    auto kern = decode_kernel<LAT, DITHER, KV>;
+    const size_t smem =
+        (size_t)(a.tcols * kSignStride + kWarpsPerCta * kStageWords + kWarpsPerCta * 128) * sizeof(uint32_t);
+    auto kern = a.k <= 4 ? decode_kernel<LAT, DITHER, KV, true> : decode_kernel<LAT, DITHER, KV, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;

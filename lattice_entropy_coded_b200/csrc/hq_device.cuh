@@ -54,23 +54,33 @@ __device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
     return *reinterpret_cast<float2 *>(&r);
 }
 
-// ------------------------------------------------------------------ FWHT-128
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(*reinterpret_cast<unsigned long long *>(&a)),
+        "l"(*reinterpret_cast<unsigned long long *>(&b)), "l"(*reinterpret_cast<unsigned long long *>(&c)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+
+// ------------------------------------------------------------------ FWHT-128 on 4 lanes
 // Unnormalised Walsh-Hadamard transform in Sylvester order, radix-2 stages
-// h = 1, 2, ..., 64, pair (i, i + h) -> (a + b, a - b).  The tile is held as
-// 64 float2 (elements 2j, 2j+1): stage 1 works inside each pair; for h >= 2
-// the butterflies of elements 2j and 2j+1 are independent and share a packed
-// add and a packed subtract.  The 1/sqrt(128) of the orthonormal H_128 is
-// folded into the scale factors.
-__device__ __forceinline__ void fwht128(float2 (&v)[kTile / 2]) {
+// h = 1, 2, ..., 64, pair (i, i + h) -> (a + b, a - b).  Four consecutive lanes
+// hold one tile, lane quarter q = lane & 3 holding elements [32q, 32q + 32) as
+// 16 float2.  Stages 1..16 are inside a lane (stage 1 inside each float2, the
+// others with packed adds); stage 32 pairs quarters q and q ^ 1, stage 64 q and
+// q ^ 2: the partner's values arrive by shuffle and the lower quarter keeps
+// a + b = fma(+1, x, y), the upper a - b = fma(-1, x, y) (exact product, one
+// rounding: identical to the subtraction).  The 1/sqrt(128) of the orthonormal
+// H_128 is folded into the scale factors.
+__device__ __forceinline__ void fwht128_quarter(float2 (&v)[16], int lane) {
 #pragma unroll
-    for (int j = 0; j < kTile / 2; j++) {
+    for (int j = 0; j < 16; j++) {
         float a = v[j].x, b = v[j].y;
         v[j] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
     }
 #pragma unroll
-    for (int hp = 1; hp < kTile / 2; hp <<= 1) {
+    for (int hp = 1; hp < 16; hp <<= 1) {
 #pragma unroll
-        for (int j = 0; j < kTile / 2; j++) {
+        for (int j = 0; j < 16; j++) {
             if ((j & hp) == 0) {
                 float2 a = v[j], b = v[j + hp];
                 v[j] = f2_add(a, b);
@@ -78,37 +88,53 @@ __device__ __forceinline__ void fwht128(float2 (&v)[kTile / 2]) {
             }
         }
     }
+#pragma unroll
+    for (int m = 1; m <= 2; m <<= 1) {
+        const float sg = (lane & m) ? -1.0f : 1.0f;
+        const float2 s2 = make_float2(sg, sg);
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+            float2 y;
+            y.x = __shfl_xor_sync(0xffffffffu, v[j].x, m);
+            y.y = __shfl_xor_sync(0xffffffffu, v[j].y, m);
+            v[j] = f2_fma(s2, v[j], y);
+        }
+    }
 }
 
 // ------------------------------------------------------------------ lattices
-// D_n nearest point (Conway & Sloane): round every coordinate to nearest-even;
-// if the integer sum is odd, move the coordinate farthest from its integer
-// (first index on ties) one step toward its input.
+// Rounding without the conversion pipe: for |x| < 2^22, x + 1.5*2^23 lands in
+// [2^23, 2^24) where the fp32 spacing is 1, so the add rounds x to the nearest
+// integer with ties to even (1.5*2^23 is even), exactly like rint; subtracting
+// the constant gives rint(x) as a float, and the integer is the bit pattern minus
+// that of the constant.  Larger |x| are outside the supported range: they give
+// large codes, which the range check (symbols >= 2^22) flags.
+constexpr float kRoundMagic = 12582912.0f;
+constexpr int32_t kRoundMagicBits = 0x4B400000;
+
+__device__ __forceinline__ int32_t rint_int(float x) {
+    return __float_as_int(__fadd_rn(x, kRoundMagic)) - kRoundMagicBits;
+}
+
+// D_n nearest point (Conway & Sloane) on one candidate: round every coordinate
+// to nearest-even; if the integer sum is odd, move the coordinate farthest from
+// its integer (first index on ties) one step toward its input.  Branch-free:
+// the argmax is a compare/select chain and the step is a predicated add.
+// In: t[i] = y[i] + kRoundMagic (rounded), f[i] = t[i] - kRoundMagic, r[i] = y[i] - f[i].
+// Out: f[] with the fix applied.
 template <int N>
-__device__ __forceinline__ void dn_nearest(const float (&y)[N], int32_t (&f)[N]) {
-    float r[N];
-    int32_t par = 0;
-#pragma unroll
-    for (int i = 0; i < N; i++) {
-        float fi = rintf(y[i]);
-        f[i] = __float2int_rn(fi);
-        r[i] = __fsub_rn(y[i], fi);
-        par ^= f[i];
-    }
-    float best = fabsf(r[0]);
+__device__ __forceinline__ void dn_fix(const float (&r)[N], uint32_t par, float (&f)[N]) {
+    float rb = r[0];
     int j = 0;
 #pragma unroll
     for (int i = 1; i < N; i++) {
-        float a = fabsf(r[i]);
-        bool gt = a > best;
-        best = gt ? a : best;
+        const bool gt = fabsf(r[i]) > fabsf(rb);
+        rb = gt ? r[i] : rb;
         j = gt ? i : j;
     }
-    if (par & 1) {
+    const float d = (par & 1u) ? ((rb >= 0.0f) ? 1.0f : -1.0f) : 0.0f;
 #pragma unroll
-        for (int i = 0; i < N; i++)
-            if (i == j) f[i] += (r[i] >= 0.0f) ? 1 : -1;
-    }
+    for (int i = 0; i < N; i++) f[i] = __fadd_rn(f[i], (i == j) ? d : 0.0f);
 }
 
 // sqrt(3)-related constants of the A2 embedding, rounded to fp32.
@@ -116,39 +142,54 @@ __device__ __forceinline__ void dn_nearest(const float (&y)[N], int32_t (&f)[N])
 #define HQ_SQRT3_2 0.86602540378443864676f
 #define HQ_SQRT3 1.73205080756887729353f
 
+__device__ __forceinline__ uint32_t zigzag(int32_t m);
+
 template <int LAT> struct Lattice;
 
 // Z: plain rounding; symbol = code.
 template <> struct Lattice<HQ_Z> {
     static constexpr int N = 1;
-    __device__ static __forceinline__ void nearest(const float (&v)[1], int32_t (&q)[1]) {
-        q[0] = __float2int_rn(v[0]);
+    __device__ static __forceinline__ void nearest(const float (&v)[1], int32_t (&q)[1]) { q[0] = rint_int(v[0]); }
+    __device__ static __forceinline__ uint32_t symbols(const float (&v)[1], uint32_t (&z)[1]) {
+        z[0] = zigzag(rint_int(v[0]));
+        return 0;
     }
     __device__ static __forceinline__ void point(const int32_t (&q)[1], float (&p)[1]) { p[0] = (float)q[0]; }
     __device__ static __forceinline__ float box(int) { return 1.0f; }
-    __device__ static __forceinline__ uint32_t strip(const int32_t (&q)[1], int32_t (&m)[1]) {
-        m[0] = q[0];
-        return 0;
-    }
     __device__ static __forceinline__ void reinsert(const int32_t (&m)[1], uint32_t, int32_t (&q)[1]) { q[0] = m[0]; }
 };
 
 // D4 = {q in Z^4 : sum even}; q3's parity is implied by q0 + q1 + q2.
 template <> struct Lattice<HQ_D4> {
     static constexpr int N = 4;
-    __device__ static __forceinline__ void nearest(const float (&v)[4], int32_t (&q)[4]) { dn_nearest<4>(v, q); }
+    __device__ static __forceinline__ void nearest(const float (&v)[4], int32_t (&q)[4]) {
+        float f[4], r[4];
+        uint32_t par = 0;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float t = __fadd_rn(v[i], kRoundMagic);
+            f[i] = __fsub_rn(t, kRoundMagic);
+            r[i] = __fsub_rn(v[i], f[i]);
+            par ^= __float_as_uint(t);
+        }
+        dn_fix<4>(r, par, f);
+#pragma unroll
+        for (int i = 0; i < 4; i++) q[i] = rint_int(f[i]);
+    }
+    __device__ static __forceinline__ uint32_t symbols(const float (&v)[4], uint32_t (&z)[4]) {
+        int32_t q[4];
+        nearest(v, q);
+        z[0] = zigzag(q[0]);
+        z[1] = zigzag(q[1]);
+        z[2] = zigzag(q[2]);
+        z[3] = zigzag((q[3] - ((q[0] + q[1] + q[2]) & 1)) >> 1);
+        return 0;
+    }
     __device__ static __forceinline__ void point(const int32_t (&q)[4], float (&p)[4]) {
 #pragma unroll
         for (int i = 0; i < 4; i++) p[i] = (float)q[i];
     }
     __device__ static __forceinline__ float box(int) { return 2.0f; }
-    __device__ static __forceinline__ uint32_t strip(const int32_t (&q)[4], int32_t (&m)[4]) {
-        m[0] = q[0];
-        m[1] = q[1];
-        m[2] = q[2];
-        m[3] = (q[3] - ((q[0] + q[1] + q[2]) & 1)) >> 1;
-        return 0;
-    }
     __device__ static __forceinline__ void reinsert(const int32_t (&m)[4], uint32_t, int32_t (&q)[4]) {
         q[0] = m[0];
         q[1] = m[1];
@@ -167,27 +208,26 @@ template <> struct Lattice<HQ_A2> {
         p[1] = __fmul_rn((float)q[1], HQ_SQRT3_2);
     }
     __device__ static __forceinline__ void nearest(const float (&u)[2], int32_t (&q)[2]) {
-        float t1 = __fmul_rn(u[1], HQ_INV_SQRT3);
-        int32_t c0[2] = {2 * __float2int_rn(u[0]), 2 * __float2int_rn(t1)};
-        int32_t c1[2] = {2 * __float2int_rn(__fsub_rn(u[0], 0.5f)) + 1, 2 * __float2int_rn(__fsub_rn(t1, 0.5f)) + 1};
-        float p0[2], p1[2];
-        point(c0, p0);
-        point(c1, p1);
+        const float t1 = __fmul_rn(u[1], HQ_INV_SQRT3);
+        const int32_t c0a = 2 * rint_int(u[0]), c0b = 2 * rint_int(t1);
+        const int32_t c1a = 2 * rint_int(__fsub_rn(u[0], 0.5f)) + 1, c1b = 2 * rint_int(__fsub_rn(t1, 0.5f)) + 1;
         float r, d0 = 0.0f, d1 = 0.0f;
-        r = __fsub_rn(u[0], p0[0]); d0 = __fmaf_rn(r, r, d0);
-        r = __fsub_rn(u[1], p0[1]); d0 = __fmaf_rn(r, r, d0);
-        r = __fsub_rn(u[0], p1[0]); d1 = __fmaf_rn(r, r, d1);
-        r = __fsub_rn(u[1], p1[1]); d1 = __fmaf_rn(r, r, d1);
-        bool odd = d1 < d0;
-        q[0] = odd ? c1[0] : c0[0];
-        q[1] = odd ? c1[1] : c0[1];
+        r = __fsub_rn(u[0], __fmul_rn((float)c0a, 0.5f)); d0 = __fmaf_rn(r, r, d0);
+        r = __fsub_rn(u[1], __fmul_rn((float)c0b, HQ_SQRT3_2)); d0 = __fmaf_rn(r, r, d0);
+        r = __fsub_rn(u[0], __fmul_rn((float)c1a, 0.5f)); d1 = __fmaf_rn(r, r, d1);
+        r = __fsub_rn(u[1], __fmul_rn((float)c1b, HQ_SQRT3_2)); d1 = __fmaf_rn(r, r, d1);
+        const bool odd = d1 < d0;
+        q[0] = odd ? c1a : c0a;
+        q[1] = odd ? c1b : c0b;
     }
-    __device__ static __forceinline__ float box(int i) { return (i & 1) ? HQ_SQRT3 : 1.0f; }
-    __device__ static __forceinline__ uint32_t strip(const int32_t (&q)[2], int32_t (&m)[2]) {
-        m[0] = q[0];
-        m[1] = (q[1] - (q[0] & 1)) >> 1;
+    __device__ static __forceinline__ uint32_t symbols(const float (&u)[2], uint32_t (&z)[2]) {
+        int32_t q[2];
+        nearest(u, q);
+        z[0] = zigzag(q[0]);
+        z[1] = zigzag((q[1] - (q[0] & 1)) >> 1);
         return 0;
     }
+    __device__ static __forceinline__ float box(int i) { return (i & 1) ? HQ_SQRT3 : 1.0f; }
     __device__ static __forceinline__ void reinsert(const int32_t (&m)[2], uint32_t, int32_t (&q)[2]) {
         q[0] = m[0];
         q[1] = 2 * m[1] + (m[0] & 1);
@@ -196,48 +236,64 @@ template <> struct Lattice<HQ_A2> {
 
 // E8 as 2E8 = 2D8 u (2D8 + 1) in Z^8: candidate A = 2 D8(v/2), candidate
 // B = 2 D8((v - 1)/2) + 1, keep B only if strictly nearer (sequential fma
-// distance).  Stripping: coset bit c raw; m_i = (q_i - c) / 2; m_7's parity is
-// implied by m_0..m_6, so m_7' = (m_7 - p) / 2 is coded.
+// distance, index order).  The two candidates run side by side in the two
+// halves of packed fp32 operations.  The symbols come straight from the D8
+// integers of the winner: coset bit c (0 for A, 1 for B), m_i = (q_i - c)/2 is
+// the D8 coordinate, and m_7's parity (implied by m_0..m_6) is stripped.
 template <> struct Lattice<HQ_E8> {
     static constexpr int N = 8;
     __device__ static __forceinline__ void point(const int32_t (&q)[8], float (&p)[8]) {
 #pragma unroll
         for (int i = 0; i < 8; i++) p[i] = (float)q[i];
     }
+    // D8 coordinates of both candidates after their parity fixes, and which wins.
+    __device__ static __forceinline__ bool decide(const float (&v)[8], float (&fa)[8], float (&fb)[8]) {
+        const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
+        float ra[8], rb[8];
+        uint32_t pa = 0, pb = 0;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float2 y = f2_mul(make_float2(v[i], __fsub_rn(v[i], 1.0f)), make_float2(0.5f, 0.5f));
+            const float2 t = f2_add(y, M2);
+            const float2 f = f2_sub(t, M2);
+            const float2 r = f2_sub(y, f);
+            fa[i] = f.x;
+            fb[i] = f.y;
+            ra[i] = r.x;
+            rb[i] = r.y;
+            pa ^= __float_as_uint(t.x);
+            pb ^= __float_as_uint(t.y);
+        }
+        dn_fix<8>(ra, pa, fa);
+        dn_fix<8>(rb, pb, fb);
+        float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float2 pt = f2_fma(make_float2(fa[i], fb[i]), make_float2(2.0f, 2.0f), make_float2(0.0f, 1.0f));
+            const float2 rho = f2_sub(make_float2(v[i], v[i]), pt);
+            acc = f2_fma(rho, rho, acc);
+        }
+        return acc.y < acc.x;
+    }
     __device__ static __forceinline__ void nearest(const float (&v)[8], int32_t (&q)[8]) {
-        float y[8];
-        int32_t fa[8], fb[8];
+        float fa[8], fb[8];
+        const bool odd = decide(v, fa, fb);
 #pragma unroll
-        for (int i = 0; i < 8; i++) y[i] = __fmul_rn(v[i], 0.5f);
-        dn_nearest<8>(y, fa);
+        for (int i = 0; i < 8; i++) q[i] = 2 * rint_int(odd ? fb[i] : fa[i]) + (odd ? 1 : 0);
+    }
+    __device__ static __forceinline__ uint32_t symbols(const float (&v)[8], uint32_t (&z)[8]) {
+        float fa[8], fb[8];
+        const bool odd = decide(v, fa, fb);
+        int32_t m[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) y[i] = __fmul_rn(__fsub_rn(v[i], 1.0f), 0.5f);
-        dn_nearest<8>(y, fb);
-        float dA = 0.0f, dB = 0.0f;
+        for (int i = 0; i < 8; i++) m[i] = rint_int(odd ? fb[i] : fa[i]);
+        const int32_t s = m[0] + m[1] + m[2] + m[3] + m[4] + m[5] + m[6];
+        m[7] = (m[7] - (s & 1)) >> 1;
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            float r = __fsub_rn(v[i], (float)(2 * fa[i]));
-            dA = __fmaf_rn(r, r, dA);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            float r = __fsub_rn(v[i], (float)(2 * fb[i] + 1));
-            dB = __fmaf_rn(r, r, dB);
-        }
-        bool odd = dB < dA;
-#pragma unroll
-        for (int i = 0; i < 8; i++) q[i] = odd ? 2 * fb[i] + 1 : 2 * fa[i];
+        for (int i = 0; i < 8; i++) z[i] = zigzag(m[i]);
+        return odd ? 1u : 0u;
     }
     __device__ static __forceinline__ float box(int) { return 4.0f; }
-    __device__ static __forceinline__ uint32_t strip(const int32_t (&q)[8], int32_t (&m)[8]) {
-        int32_t c = q[0] & 1, s = 0;
-#pragma unroll
-        for (int i = 0; i < 8; i++) m[i] = (q[i] - c) >> 1;
-#pragma unroll
-        for (int i = 0; i < 7; i++) s += m[i];
-        m[7] = (m[7] - (s & 1)) >> 1;
-        return (uint32_t)c;
-    }
     __device__ static __forceinline__ void reinsert(const int32_t (&m)[8], uint32_t c, int32_t (&q)[8]) {
         int32_t s = 0;
 #pragma unroll
@@ -286,7 +342,7 @@ __device__ __forceinline__ void dither_block<HQ_Z>(uint64_t seed, uint64_t e, fl
     uint64_t h = splitmix64(seed ^ kDitherSalt, e >> 1);
     uint32_t r24 = (e & 1ull) ? ((uint32_t)h >> 8) : (uint32_t)(h >> 40);
     float w = __fmul_rn((float)r24, 0x1p-24f);
-    d[0] = __fsub_rn(w, (float)__float2int_rn(w));
+    d[0] = __fsub_rn(w, (float)rint_int(w));
 }
 
 // ------------------------------------------------------------------ memory helpers
@@ -299,12 +355,6 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned l
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
 
 }  // namespace hq

@@ -3,20 +3,20 @@
 // subtractive dither, nearest lattice point, bit-stripping, zigzag, Rice planes.
 //
 // Work decomposition (B200, sm_100a):
-//  * one warp encodes one chunk (32 tiles), one lane owns one tile: load, sign
-//    flip, FWHT and scale run on 64 float2 registers with packed fp32 adds;
-//  * the transformed tile goes to a lane-private shared-memory row, and pass A
-//    walks it in a rolled loop over groups of 8 coordinates (one copy of the
-//    lattice decoder in the instruction stream), leaving the zigzag symbols in
-//    the row in place;
-//  * a persistent grid; warps take chunk tickets from a global counter, so a
-//    chunk's predecessors are always already running;
-//  * warp scan of the unary lengths and a single-pass decoupled look-back over
-//    64-bit (flag, value) words give the chunk's word offset (bounded waits:
-//    HQ_ST_TIMEOUT);
-//  * pass B builds the remainder and unary planes in a per-warp shared stage
-//    and writes the chunk with coalesced stores; a chunk larger than the stage,
-//    or with quotients above 255, is written in place in global memory.
+//  * one warp encodes one chunk (32 tiles) in 4 rounds of 8 tiles; four lanes
+//    share a tile, 32 elements each, loaded as 64 contiguous bytes per lane;
+//  * the transform runs in registers (16 float2 per lane, packed fp32 adds;
+//    the last two butterfly stages cross lanes by shuffle), then each lane
+//    decodes its 32/N lattice blocks and keeps 32 zigzag symbols;
+//  * per round a warp scan of unary lengths places every lane's codewords;
+//    remainder bits, E8 coset bits and unary terminators go into a per-warp
+//    shared-memory stage that holds the whole chunk;
+//  * a persistent grid takes chunk tickets from a global counter, so a chunk's
+//    predecessors are always already running; a single-pass decoupled
+//    look-back over 64-bit (flag, value) words gives the chunk's word offset
+//    (bounded waits: HQ_ST_TIMEOUT), and the stage is written out coalesced;
+//  * a chunk larger than the stage is re-encoded by a separate path that sets
+//    its bits in place in global memory (same stream; only for extreme codes).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -73,115 +73,136 @@ __device__ __noinline__ unsigned long long lookback(unsigned long long *lb, unsi
     return excl;
 }
 
-// Tile of lane `lane` in chunk c: source pointer, sign-table column, dither counter.
-__device__ __forceinline__ bool tile_of(const TileMap &m, const uint16_t *x, unsigned long long c, int lane,
-                                        const uint16_t *&src, int &tcol, unsigned long long &e0, int &ntiles) {
-    if (m.kv) {
-        long long cph = (m.tokens + 31) / 32;
-        long long h = (long long)c / cph, tc = (long long)c % cph;
-        long long tok = tc * 32 + lane;
-        long long left = m.tokens - tc * 32;
-        ntiles = (int)(left < 32 ? left : 32);
-        if (tok >= m.tokens) return false;
-        src = x + h * m.ld_head + tok * m.ld_tok;
-        tcol = 0;
-        e0 = (unsigned long long)(((m.tok0 + tok) * m.heads + h) * kTile);
+// Where the tiles of one chunk are (computed once per chunk).
+struct ChunkGeo {
+    int ntiles;
+    // weights: tile ti of the chunk is row row0 + (tc0 + ti) / tpr, tile column (tc0 + ti) % tpr
+    long long row0;
+    int tc0, tpr;
+    // kv: head h, tokens tok_base + ti
+    long long h, tok_base;
+
+    __device__ __forceinline__ void init(const TileMap &m, unsigned long long c) {
+        if (m.kv) {
+            long long cph = (m.tokens + 31) / 32;
+            h = (long long)c / cph;
+            tok_base = ((long long)c % cph) * 32;
+            long long left = m.tokens - tok_base;
+            ntiles = (int)(left < 32 ? left : 32);
+        } else {
+            tpr = (int)(m.cols / kTile);
+            long long t0 = (long long)c * 32;
+            long long all = m.rows * (long long)tpr;
+            ntiles = (int)((all - t0) < 32 ? (all - t0) : 32);
+            row0 = t0 / tpr;
+            tc0 = (int)(t0 - row0 * tpr);
+        }
+    }
+    // Tile ti (< 32) of the chunk: first element, sign-table column, dither counter of its element 0.
+    __device__ __forceinline__ bool tile(const TileMap &m, const uint16_t *x, int ti, const uint16_t *&src,
+                                         int &tcol, unsigned long long &e0) const {
+        if (ti >= ntiles) return false;
+        if (m.kv) {
+            long long tok = tok_base + ti;
+            src = x + h * m.ld_head + tok * m.ld_tok;
+            tcol = 0;
+            e0 = (unsigned long long)(((m.tok0 + tok) * m.heads + h) * kTile);
+            return true;
+        }
+        int tc = tc0 + ti;
+        long long r = row0;
+        if (tc >= tpr) {
+            int d = tc / tpr;
+            r += d;
+            tc -= d * tpr;
+        }
+        src = x + r * m.ld + (long long)tc * kTile;
+        tcol = tc;
+        e0 = (unsigned long long)(r * m.cols + (long long)tc * kTile);
         return true;
     }
-    long long tpr = m.cols / kTile;
-    long long all = m.rows * tpr;
-    long long t0 = (long long)c * 32;
-    ntiles = (int)((all - t0) < 32 ? (all - t0) : 32);
-    long long t = t0 + lane;
-    if (t >= all) return false;
-    long long r = t / tpr, tc = t % tpr;
-    src = x + r * m.ld + tc * kTile;
-    tcol = (int)tc;
-    e0 = (unsigned long long)(r * m.cols + tc * kTile);
-    return true;
-}
+};
 
-// x (bf16, 128 elements) -> D x widened to fp32 -> H_128 -> * c, stored to the
-// lane's row (16-byte stores).
-__device__ __forceinline__ void transform_to_row(const uint16_t *src, bool valid, const uint32_t *sg, float c_scale,
-                                                 float *row) {
-    float2 v[kTile / 2];
+// One round for one lane: its quarter (32 elements) of tile 8r + lane/4 ->
+// D x -> H_128 (with the three partner lanes) -> * c -> [+ d] -> lattice
+// blocks -> 32 zigzag symbols and the E8 coset bits of its blocks.
+// Whole warp must call it (shuffles).
+template <int LAT, bool DITHER>
+__device__ __forceinline__ bool round_symbols(const EncodeArgs &a, const ChunkGeo &geo, int r, int lane,
+                                              const uint32_t *sign_tab, uint32_t (&z)[32], uint32_t &cbits) {
+    using L = Lattice<LAT>;
+    constexpr int N = L::N;
+    const int q = lane & 3;
+    const uint16_t *src = nullptr;
+    int tcol = 0;
+    unsigned long long e0 = 0;
+    const bool valid = geo.tile(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, tcol, e0);
+    const uint32_t *sg = sign_tab + tcol * kSignStride + q * kSignQuarter;
+    float2 v[16];
 #pragma unroll
-    for (int j = 0; j < kTile / 8; j++) {
-        uint4 w = valid ? ldg_nc_v4(src + 8 * j) : make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < 4; j++) {
+        uint4 w = valid ? ldg_nc_v4(src + 32 * q + 8 * j) : make_uint4(0, 0, 0, 0);
         uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
         uint32_t ww[4] = {w.x ^ s.x, w.y ^ s.y, w.z ^ s.z, w.w ^ s.w};
 #pragma unroll
         for (int t = 0; t < 4; t++)
             v[4 * j + t] = make_float2(__uint_as_float(ww[t] << 16), __uint_as_float(ww[t] & 0xFFFF0000u));
     }
-    fwht128(v);
-    const float2 c2 = make_float2(c_scale, c_scale);
+    fwht128_quarter(v, lane);
+    const float2 c2 = make_float2(a.c_scale, a.c_scale);
 #pragma unroll
-    for (int j = 0; j < kTile / 4; j++) {
-        float2 a = f2_mul(v[2 * j], c2), b = f2_mul(v[2 * j + 1], c2);
-        *reinterpret_cast<float4 *>(row + 4 * j) = make_float4(a.x, a.y, b.x, b.y);
-    }
-}
+    for (int j = 0; j < 16; j++) v[j] = f2_mul(v[j], c2);
 
-// Symbols of group g (8 coordinates u[0..7]); returns the E8 coset bits of the
-// group's blocks (bit bb for block bb of the group).
-template <int LAT, bool DITHER>
-__device__ __forceinline__ uint32_t group_symbols(const float (&u)[8], int g, unsigned long long e0, uint64_t seed,
-                                                  uint32_t (&z)[8]) {
-    using L = Lattice<LAT>;
-    constexpr int N = L::N;
-    uint32_t cb = 0;
+    cbits = 0;
+    const unsigned long long eq = e0 + 32ull * q;
 #pragma unroll
-    for (int bb = 0; bb < 8 / N; bb++) {
+    for (int b = 0; b < 32 / N; b++) {
         float blk[N];
 #pragma unroll
-        for (int i = 0; i < N; i++) blk[i] = u[bb * N + i];
+        for (int i = 0; i < N; i++) {
+            const int e = b * N + i;
+            blk[i] = (e & 1) ? v[e >> 1].y : v[e >> 1].x;
+        }
         if (DITHER) {
             float d[N];
-            dither_block<LAT>(seed, e0 + (unsigned long long)(8 * g + bb * N), d);
+            dither_block<LAT>(a.seed, eq + (unsigned long long)(b * N), d);
 #pragma unroll
             for (int i = 0; i < N; i++) blk[i] = __fadd_rn(blk[i], d[i]);
         }
-        int32_t q[N], m[N];
-        L::nearest(blk, q);
-        cb |= L::strip(q, m) << bb;
+        uint32_t zz[N];
+        cbits |= L::symbols(blk, zz) << b;
 #pragma unroll
-        for (int i = 0; i < N; i++) z[bb * N + i] = zigzag(m[i]);
+        for (int i = 0; i < N; i++) z[b * N + i] = zz[i];
     }
-    return cb;
+    if (!valid) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) z[i] = 0;
+        cbits = 0;
+    }
+    return valid;
 }
 
-// Remainder plane writer: k low bits per symbol, LSB first, into the lane's own
-// region `dst` (4k words).  k is warp-uniform, so the flushes are uniform.
-struct RemWriter {
-    uint32_t *dst;
-    int k;
-    uint32_t mask, nb, w;
-    bool store;
-    unsigned long long acc;
-
-    __device__ __forceinline__ void init(uint32_t *d, int kk, bool st) {
-        dst = d;
-        k = kk;
-        mask = kk ? (1u << kk) - 1u : 0u;
-        store = st;
-        acc = 0;
-        nb = 0;
-        w = 0;
-    }
-    __device__ __forceinline__ void put_group(const uint32_t (&z)[8]) {
-        if (k == 0) return;
-        if (k <= 4) {
-            uint32_t gv = 0;   // 8k <= 32 bits, symbol 0 in the low bits
+// Remainder bits of 32 symbols (warp-uniform k) into the lane's k words.
+// KSMALL (k <= 4): a group of 8 remainders is built in one register, last
+// symbol first, two operations per symbol; otherwise a 64-bit accumulator.
+template <bool KSMALL>
+__device__ __forceinline__ void put_rem(uint32_t *dst, const uint32_t (&z)[32], int k, bool store) {
+    if (k == 0) return;
+    const uint32_t mask = (1u << k) - 1u;
+    unsigned long long acc = 0;
+    uint32_t nb = 0, w = 0;
 #pragma unroll
-            for (int i = 7; i >= 0; i--) gv = (gv << k) | (z[i] & mask);
+    for (int g = 0; g < 4; g++) {
+        if (KSMALL) {
+            uint32_t gv = 0;
+#pragma unroll
+            for (int i = 7; i >= 0; i--) gv = (gv << k) | (z[8 * g + i] & mask);
             acc |= (unsigned long long)gv << nb;
             nb += 8u * (uint32_t)k;
         } else {
 #pragma unroll
             for (int i = 0; i < 8; i++) {
-                acc |= (unsigned long long)(z[i] & mask) << nb;
+                acc |= (unsigned long long)(z[8 * g + i] & mask) << nb;
                 nb += (uint32_t)k;
                 if (nb >= 32u) {
                     if (store) dst[w] = (uint32_t)acc;
@@ -198,11 +219,11 @@ struct RemWriter {
             nb -= 32u;
         }
     }
-};
+}
 
 // Unary terminators of 8 symbols with quotients q[0..7], starting at bit pos of
-// `un` (zeroed words).  A group whose codes fit in 32 bits is built in a
-// register (last symbol first) and ORed in with two shared atomics.
+// `un` (zeroed shared words).  A group whose codes fit in 32 bits is built in a
+// register (last symbol first) and ORed in with at most two shared atomics.
 __device__ __forceinline__ uint32_t unary_group_shared(uint32_t *un, uint32_t pos, const uint32_t (&q)[8]) {
     uint32_t ug = 8;
 #pragma unroll
@@ -229,22 +250,63 @@ __device__ __forceinline__ uint32_t unary_group_shared(uint32_t *un, uint32_t po
     return ug;
 }
 
+// Slow path for a chunk that does not fit the stage: recompute every round and
+// set each bit of the chunk (already zeroed in global memory) with an atomic;
+// every access is bounded by `room` words.  Whole warp calls it.
 template <int LAT, bool DITHER>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, 1) encode_kernel(const EncodeArgs a) {
+__device__ __noinline__ void encode_chunk_global(const EncodeArgs &a, const ChunkGeo &geo, const uint32_t *sign_tab,
+                                                 uint32_t *g, unsigned long long room, uint32_t nc, uint32_t nr) {
+    const int lane = threadIdx.x & 31;
+    const int k = a.k;
+    const uint32_t mask = k ? (1u << k) - 1u : 0u;
+    const int nrounds = (geo.ntiles + kTilesPerRound - 1) / kTilesPerRound;
+    unsigned long long urun = 0;
+    for (int r = 0; r < nrounds; r++) {
+        uint32_t z[32], cbits;
+        const bool valid = round_symbols<LAT, DITHER>(a, geo, r, lane, sign_tab, z, cbits);
+        unsigned long long ub = 0;
+#pragma unroll
+        for (int i = 0; i < 32; i++) ub += z[i] >> k;
+        ub = valid ? ub + 32 : 0;
+        unsigned long long incl = ub;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const unsigned long long rtot = __shfl_sync(0xffffffffu, incl, 31);
+        if (valid) {
+            const unsigned long long cw = 4ull * r + (lane >> 3);
+            if (LAT == HQ_E8 && cbits && cw < room) atomicOr(g + cw, cbits << (4 * (lane & 7)));
+            unsigned long long rb = 32ull * (nc + (unsigned long long)(32 * r + lane) * k);
+            unsigned long long pos = 32ull * (nc + nr) + urun + incl - ub;
+            for (int i = 0; i < 32; i++) {
+                const uint32_t rr = z[i] & mask;
+                for (int b = 0; b < k; b++, rb++)
+                    if (((rr >> b) & 1u) && (rb >> 5) < room) atomicOr(g + (rb >> 5), 1u << (uint32_t)(rb & 31));
+                pos += z[i] >> k;
+                if ((pos >> 5) < room) atomicOr(g + (pos >> 5), 1u << (uint32_t)(pos & 31));
+                pos++;
+            }
+        }
+        urun += rtot;
+    }
+}
+
+template <int LAT, bool DITHER, bool KSMALL>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t *sign_tab = smem;                                                  // tcols * kSignStride
-    uint32_t *rows_all = smem + a.tcols * kSignStride;                          // warps * 32 * kRowStride
-    uint32_t *stage_all = rows_all + kWarpsPerCta * 32 * kRowStride;            // warps * kStageWords
+    uint32_t *sign_tab = smem;                                        // tcols * kSignStride
+    uint32_t *stage_all = smem + a.tcols * kSignStride;               // warps * kStageWords
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float *row = reinterpret_cast<float *>(rows_all + (warp * 32 + lane) * kRowStride);
-    uint32_t *zrow = rows_all + (warp * 32 + lane) * kRowStride;
     uint32_t *stage = stage_all + warp * kStageWords;
 
     // Sign masks per bf16x2 pair: bit 15 flips the even column, bit 31 the odd one.
     for (int i = threadIdx.x; i < a.tcols * 64; i += blockDim.x) {
-        int tc = i >> 6, p = i & 63;
-        unsigned long long col = (unsigned long long)tc * kTile + 2 * p;
-        sign_tab[tc * kSignStride + p] = (sign_bit(a.seed, col) << 15) | (sign_bit(a.seed, col + 1) << 31);
+        const int tc = i >> 6, p = i & 63;
+        const unsigned long long col = (unsigned long long)tc * kTile + 2 * p;
+        sign_tab[tc * kSignStride + (p >> 4) * kSignQuarter + (p & 15)] =
+            (sign_bit(a.seed, col) << 15) | (sign_bit(a.seed, col + 1) << 31);
     }
     __syncthreads();
 
@@ -259,54 +321,65 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 1) encode_kernel(const Enco
         c = __shfl_sync(0xffffffffu, c, 0);
         if (c >= a.n_chunks) break;
 
-        const uint16_t *src = nullptr;
-        int tcol = 0, ntiles = 0;
-        unsigned long long e0 = 0;
-        const bool valid = tile_of(a.map, a.x, c, lane, src, tcol, e0, ntiles);
-        const uint32_t *sg = sign_tab + tcol * kSignStride;
-        transform_to_row(src, valid, sg, a.c_scale, row);
-
-        // ---- pass A: symbols in place of the transformed coordinates
-        uint32_t coset = 0, usum = 0, zor = 0;
-#pragma unroll 1
-        for (int g = 0; g < kTile / 8; g++) {
-            const float4 u0 = *reinterpret_cast<const float4 *>(row + 8 * g);
-            const float4 u1 = *reinterpret_cast<const float4 *>(row + 8 * g + 4);
-            const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-            uint32_t z[8];
-            const uint32_t cb = group_symbols<LAT, DITHER>(u, g, e0, a.seed, z);
-            coset |= cb << (g * (8 / Lattice<LAT>::N));
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                if (!valid) z[i] = 0;
-                zor |= z[i];
-                usum += z[i] >> k;
-            }
-            *reinterpret_cast<uint4 *>(zrow + 8 * g) = make_uint4(z[0], z[1], z[2], z[3]);
-            *reinterpret_cast<uint4 *>(zrow + 8 * g + 4) = make_uint4(z[4], z[5], z[6], z[7]);
-        }
-        if (!valid) coset = 0;
-        zor_all |= zor;
-
-        // ---- unary lengths: warp scan
-        const unsigned long long ubits = valid ? (unsigned long long)usum + kTile : 0ull;
-        unsigned long long incl = ubits;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const unsigned long long utotal = __shfl_sync(0xffffffffu, incl, 31);
-        const unsigned long long ustart = incl - ubits;
-        const uint32_t wzor = __reduce_or_sync(0xffffffffu, zor);
-        const bool range_bad = (wzor >> 22) != 0u || utotal >= kMaxUnaryBits;
-        if (range_bad) status |= HQ_ST_RANGE;
+        ChunkGeo geo;
+        geo.init(a.map, c);
+        const int ntiles = geo.ntiles;
+        const int nrounds = (ntiles + kTilesPerRound - 1) / kTilesPerRound;
         const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
         const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
-        const unsigned long long nu = (utotal + 31) / 32;
+        {
+            uint4 *s4 = reinterpret_cast<uint4 *>(stage);
+            for (int i = lane; i < kStageWords / 4; i += 32) s4[i] = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+
+        uint32_t urun = 0, zor = 0;
+        bool overflow = (nc + nr) > (uint32_t)kStageWords, range_bad = false;
+#pragma unroll 1
+        for (int r = 0; r < nrounds; r++) {
+            uint32_t z[32], cbits;
+            const bool valid = round_symbols<LAT, DITHER>(a, geo, r, lane, sign_tab, z, cbits);
+            uint32_t usum = 0, lor = 0;
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                usum += z[i] >> k;
+                lor |= z[i];
+            }
+            zor |= lor;
+            const uint32_t ub = valid ? usum + 32u : 0u;
+            uint32_t incl = ub;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const uint32_t rtot = __shfl_sync(0xffffffffu, incl, 31);
+            const uint32_t rzor = __reduce_or_sync(0xffffffffu, lor);
+            if ((rzor >> 22) != 0u || (unsigned long long)urun + rtot >= kMaxUnaryBits) range_bad = true;
+            if (!overflow && nc + nr + (uint32_t)(((unsigned long long)urun + rtot + 31) >> 5) > (uint32_t)kStageWords)
+                overflow = true;
+            if (!overflow && !range_bad) {
+                put_rem<KSMALL>(stage + nc + (uint32_t)(32 * r + lane) * (uint32_t)k, z, k, valid);
+                if (valid) {
+                    if (LAT == HQ_E8 && cbits) atomicOr(stage + 4 * r + (lane >> 3), cbits << (4 * (lane & 7)));
+                    uint32_t *un = stage + nc + nr;
+                    uint32_t pos = urun + incl - ub;
+#pragma unroll
+                    for (int g = 0; g < 4; g++) {
+                        uint32_t qg[8];
+#pragma unroll
+                        for (int i = 0; i < 8; i++) qg[i] = z[8 * g + i] >> k;
+                        pos += unary_group_shared(un, pos, qg);
+                    }
+                }
+            }
+            urun += rtot;
+        }
+        zor_all |= zor;
+        if (range_bad) status |= HQ_ST_RANGE;
+        const unsigned long long nu = ((unsigned long long)urun + 31) / 32;
         const unsigned long long total = nc + nr + nu;
-        payload += utotal + (unsigned long long)nr * 32 + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
-        const bool fast = !range_bad && total <= (unsigned long long)kStageWords && (wzor >> (k + 8)) == 0u;
+        payload += urun + (unsigned long long)nr * 32 + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
 
         // ---- chunk offset
         bool to = false;
@@ -316,7 +389,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 1) encode_kernel(const Enco
         if (lane == 0) {
             a.offsets[a.chunk_base + c] = start;
             if (c + 1 == a.n_chunks) {
-                unsigned long long end = start + total;
+                const unsigned long long end = start + total;
                 a.offsets[a.chunk_base + a.n_chunks] = end;
                 if (a.tail_out) *a.tail_out = end;
                 if (a.stats) a.stats->stream_words = end;
@@ -324,61 +397,20 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 1) encode_kernel(const Enco
             }
             if (c == 0 && a.row) *a.row = a.row_val;
         }
-        const uint32_t cos_hi = __shfl_down_sync(0xffffffffu, coset, 1);
-
-        if (fast) {
-            // ---- pass B: planes into the stage, then one coalesced copy
-            for (uint32_t i = nc + nr + lane; i < (uint32_t)total; i += 32) stage[i] = 0u;
-            if (LAT == HQ_E8 && (lane & 1) == 0 && (uint32_t)(lane >> 1) < nc) stage[lane >> 1] = coset | (cos_hi << 16);
-            __syncwarp();
-            RemWriter rw;
-            rw.init(stage + nc + 4u * (uint32_t)k * (uint32_t)lane, k, valid);
-            uint32_t *un = stage + nc + nr;
-            uint32_t pos = (uint32_t)ustart;
-#pragma unroll 1
-            for (int g = 0; g < kTile / 8; g++) {
-                const uint4 z0 = *reinterpret_cast<const uint4 *>(zrow + 8 * g);
-                const uint4 z1 = *reinterpret_cast<const uint4 *>(zrow + 8 * g + 4);
-                const uint32_t z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-                rw.put_group(z);
-                if (valid) {
-                    uint32_t q[8];
-#pragma unroll
-                    for (int i = 0; i < 8; i++) q[i] = z[i] >> k;
-                    pos += unary_group_shared(un, pos, q);
-                }
-            }
-            __syncwarp();
+        __syncwarp();
+        if (!range_bad && !overflow) {
             for (uint32_t i = lane; i < (uint32_t)total; i += 32)
                 if (start + i < a.cap_words) a.stream[start + i] = stage[i];
-            __syncwarp();
         } else if (!range_bad) {
-            // ---- large chunk: zero it in place, then set every bit with a global atomic
             uint32_t *g = a.stream + start;
             const unsigned long long room = (start < a.cap_words) ? a.cap_words - start : 0ull;
             for (unsigned long long i = lane; i < total; i += 32)
                 if (i < room) g[i] = 0u;
             __syncwarp();
             __threadfence_block();
-            if (LAT == HQ_E8 && (lane & 1) == 0 && (uint32_t)(lane >> 1) < nc && (unsigned long long)(lane >> 1) < room)
-                atomicOr(g + (lane >> 1), coset | (cos_hi << 16));
-            if (valid) {
-                const uint32_t mask = k ? (1u << k) - 1u : 0u;
-                unsigned long long rb = 32ull * (nc + 4ull * (unsigned long long)k * lane);
-                unsigned long long ub = 32ull * (nc + nr) + ustart;
-#pragma unroll 1
-                for (int i = 0; i < kTile; i++) {
-                    const uint32_t zi = zrow[i];
-                    const uint32_t r = zi & mask;
-                    for (int b = 0; b < k; b++, rb++)
-                        if (((r >> b) & 1u) && (rb >> 5) < room) atomicOr(g + (rb >> 5), 1u << (uint32_t)(rb & 31));
-                    ub += zi >> k;
-                    if ((ub >> 5) < room) atomicOr(g + (ub >> 5), 1u << (uint32_t)(ub & 31));
-                    ub++;
-                }
-            }
-            __syncwarp();
+            encode_chunk_global<LAT, DITHER>(a, geo, sign_tab, g, room, nc, nr);
         }
+        __syncwarp();
     }
 
     if (a.stats) {
@@ -394,10 +426,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 1) encode_kernel(const Enco
 
 template <int LAT, bool DITHER>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
-    const size_t smem =
-        (size_t)(a.tcols * kSignStride + kWarpsPerCta * 32 * kRowStride + kWarpsPerCta * kStageWords) *
-        sizeof(uint32_t);
-    auto kern = encode_kernel<LAT, DITHER>;
+    const size_t smem = (size_t)(a.tcols * kSignStride + kWarpsPerCta * kStageWords) * sizeof(uint32_t);
+    auto kern = a.k <= 4 ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;

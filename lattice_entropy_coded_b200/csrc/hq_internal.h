@@ -11,12 +11,14 @@ namespace hq {
 
 constexpr int kTile = 128;          // elements per RHT tile
 constexpr int kChunkTiles = 32;     // tiles per chunk = lanes per warp (one tile per lane)
-constexpr int kSignStride = 68;     // words per tile column in the shared sign table (64 used, padded)
-constexpr int kWarpsPerCta = 8;     // warps per CTA in both kernels (one CTA per SM: shared memory bound)
+constexpr int kSignQuarter = 20;    // words per tile quarter in the shared sign table (16 used, padded so
+                                    // the 8 lanes of a 16-byte access phase hit distinct banks)
+constexpr int kSignStride = 4 * kSignQuarter;  // words per tile column in the sign table
+constexpr int kWarpsPerCta = 8;     // warps per CTA in both kernels
 constexpr int kStageWords = 1024;   // per-warp shared staging for one chunk's words (encode and decode);
                                     // larger chunks are written or read in place in global memory
-constexpr int kRowStride = 132;     // words per lane-private row of the transformed tile (128 + 4 pad:
-                                    // 16-byte accesses of 8 consecutive lanes hit distinct banks)
+constexpr int kLanesPerTile = 4;    // lanes sharing one tile (32 elements each)
+constexpr int kTilesPerRound = 32 / kLanesPerTile;  // tiles a warp transforms at once; 4 rounds per chunk
 constexpr uint32_t kSpinLimit = 1u << 22;   // look-back polls before giving up (HQ_ST_TIMEOUT)
 constexpr uint32_t kMaxUnaryBits = 1u << 31; // chunks with more unary bits are outside the supported range
 
