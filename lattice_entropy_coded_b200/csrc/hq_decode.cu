@@ -2,14 +2,21 @@
 // 1-4 inverted): Rice planes -> symbols -> re-inserted membership bits ->
 // lattice point [- dither] -> scale -> FWHT-128 -> sign -> bf16 (or fp32).
 //
-// Work decomposition (B200, sm_100a): one warp decodes one chunk, one lane owns
-// one tile.  The chunk's words are staged in shared memory with coalesced
-// loads; the lanes split the unary plane into 32 segments, count terminators
-// (popc) and scan, so every lane learns where its tile's first codeword starts;
-// then each lane decodes its 128 quotients sequentially from a bit-reversed
-// 32-bit window (one count-leading-zeros and one shift per symbol), pulls the k
-// remainder bits from its own fixed region, and runs the inverse transform in
-// registers.  Chunks are independent (offsets are given), so no look-back.
+// Work decomposition (B200, sm_100a):
+//  * one warp decodes one chunk (32 tiles) in 4 rounds of 8 tiles; four lanes
+//    share a tile, 32 symbols / elements each;
+//  * the chunk's words are brought into a per-warp shared-memory stage with
+//    cp.async while the warp is still decoding the previous chunk (two stages
+//    per warp); chunks too large for a stage are read from global memory;
+//  * the lanes split the unary plane into 32 word ranges, count terminators
+//    (popc) and scan, so every 32-symbol segment learns where its first
+//    codeword starts; each lane then reads its 32 quotients from bit-reversed
+//    32-bit windows, four symbols per window (one count-leading-zeros and one
+//    shift per symbol), its k remainder bits from its own fixed region, and
+//    rebuilds and scales the lattice points;
+//  * the inverse FWHT runs in registers (two stages across the four lanes by
+//    shuffle), followed by the sign flip and 16-byte stores.
+// Chunks are independent (their offsets are given), so there is no look-back.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -19,28 +26,53 @@ namespace hq {
 
 namespace {
 
-// 32 bits of a plane of `n` words starting at bit `b` (bits past the plane are 0).
-__device__ __forceinline__ uint32_t fetch32(const uint32_t *p, uint32_t n, uint32_t b) {
-    uint32_t w = b >> 5;
-    uint32_t a0 = (w < n) ? p[w] : 0u;
-    uint32_t a1 = (w + 1 < n) ? p[w + 1] : 0u;
+constexpr int kStagePad = 4;   // zero words after a staged chunk: unchecked 2-word reads stay inside
+
+// 32 bits of a plane of `n` words starting at bit `b`; words at or past n read as 0.
+__device__ __forceinline__ uint32_t fetch32_checked(const uint32_t *p, uint32_t n, uint32_t b) {
+    const uint32_t w = b >> 5;
+    const uint32_t a0 = (w < n) ? p[w] : 0u;
+    const uint32_t a1 = (w + 1 < n) ? p[w + 1] : 0u;
     return __funnelshift_r(a0, a1, b & 31u);
 }
 
-// Slow path of the unary reader: 8 quotients read one terminator at a time
-// (quotients may exceed the 32-bit window).  Kept out of line so the common
-// path stays compact.  Returns the new bit position; `ok` turns false if the
-// plane ends early.
+// The same from a staged chunk: the stage is zero-padded after the chunk and
+// the word index is clamped to the plane's end, so both reads stay inside.
+__device__ __forceinline__ uint32_t fetch32_staged(const uint32_t *p, uint32_t n, uint32_t b) {
+    const uint32_t w = min(b >> 5, n);
+    return __funnelshift_r(p[w], p[w + 1], b & 31u);
+}
+
+template <bool STAGED>
+__device__ __forceinline__ uint32_t fetch32(const uint32_t *p, uint32_t n, uint32_t b) {
+    return STAGED ? fetch32_staged(p, n, b) : fetch32_checked(p, n, b);
+}
+
+// Bit index of the n-th (0-based) set bit of w (n < popc(w)): binary search on
+// popcounts of the low halves, branch-free.
+__device__ __forceinline__ uint32_t select_bit(uint32_t w, uint32_t n) {
+    uint32_t pos = 0, c;
+    c = __popc(w & 0xFFFFu); if (n >= c) { n -= c; pos += 16; w >>= 16; }
+    c = __popc(w & 0xFFu);   if (n >= c) { n -= c; pos += 8;  w >>= 8; }
+    c = __popc(w & 0xFu);    if (n >= c) { n -= c; pos += 4;  w >>= 4; }
+    c = __popc(w & 0x3u);    if (n >= c) { n -= c; pos += 2;  w >>= 2; }
+    c = w & 1u;              if (n >= c) { pos += 1; }
+    return pos;
+}
+
+// Slow path of the unary reader: 4 quotients read one terminator at a time
+// (quotients may exceed the 32-bit window).  Out of line: rare.  Returns the
+// new bit position; *ok turns false if the plane ends early.
 __device__ __noinline__ uint32_t unary_slow(const uint32_t *un, uint32_t nu, uint32_t bp, bool *ok, uint32_t *q) {
     const uint32_t nbits = nu * 32u;
-    for (int i = 0; i < 8; i++) {
+    for (int i = 0; i < 4; i++) {
         uint32_t t = 0;
-        uint32_t x = __brev(fetch32(un, nu, bp));
+        uint32_t x = __brev(fetch32_checked(un, nu, bp));
         while (x == 0u && *ok) {
             t += 32u;
             bp += 32u;
             if (bp >= nbits) *ok = false;
-            x = __brev(fetch32(un, nu, bp));
+            x = __brev(fetch32_checked(un, nu, bp));
         }
         const uint32_t c = __clz(x);
         q[i] = t + c;
@@ -49,57 +81,44 @@ __device__ __noinline__ uint32_t unary_slow(const uint32_t *un, uint32_t nu, uin
     return bp;
 }
 
-// Sequential reader of one lane's unary quotients: a bit-reversed 32-bit
-// window, so a quotient is one count-leading-zeros and one shift.  A group of 8
-// whose codes fit in the window takes the fast path.
-struct UnaryReader {
-    const uint32_t *un;
-    uint32_t nu, nbits, bp;
-    bool ok;
-
-    __device__ __forceinline__ void init(const uint32_t *p, uint32_t n, uint32_t start) {
-        un = p;
-        nu = n;
-        nbits = n * 32u;
-        bp = start;
-        ok = true;
-    }
-    __device__ __forceinline__ void group(uint32_t (&q)[8]) {
-        uint32_t w = __brev(fetch32(un, nu, bp));   // next 32 stream bits, first at the MSB
-        if (__popc(w) >= 8) {
-            uint32_t used = 8;
+// Quotients of 4 symbols from bit bp of the unary plane: the next 32 stream
+// bits bit-reversed (first bit at the MSB); if they hold 4 terminators each
+// quotient is a count-leading-zeros, else the slow path.
+template <bool STAGED>
+__device__ __forceinline__ void unary4(const uint32_t *un, uint32_t nu, uint32_t &bp, bool &ok, uint32_t *q) {
+    uint32_t w = __brev(fetch32<STAGED>(un, nu, bp));
+    if (__popc(w) >= 4) {
+        uint32_t used = 4;
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const uint32_t t = __clz(w);
-                q[i] = t;
-                used += t;
-                w = (w << t) << 1;
-            }
-            bp += used;
-        } else {
-            uint32_t tmp[8];
-            bp = unary_slow(un, nu, bp, &ok, tmp);
-#pragma unroll
-            for (int i = 0; i < 8; i++) q[i] = tmp[i];
+        for (int i = 0; i < 4; i++) {
+            const uint32_t t = __clz(w);
+            q[i] = t;
+            used += t;
+            w = (w << t) << 1;
         }
-        if (bp > nbits) ok = false;
+        bp += used;
+    } else {
+        uint32_t tmp[4];
+        bp = unary_slow(un, nu, bp, &ok, tmp);
+#pragma unroll
+        for (int i = 0; i < 4; i++) q[i] = tmp[i];
     }
-};
+}
 
-// k-bit remainders of group g (8 symbols) from the lane's region `rw` (k words
-// per 32 symbols).  KSMALL (k <= 4): one 32-bit window per group.
-template <bool KSMALL>
+// k-bit remainders of group g (8 symbols) from the lane's region `rw`
+// (k words per 32 symbols).  KSMALL (k <= 4): one 32-bit window per group.
+template <bool KSMALL, bool STAGED>
 __device__ __forceinline__ void rem_group(const uint32_t *rw, int k, int g, uint32_t (&r)[8]) {
     if (k == 0) {
 #pragma unroll
         for (int i = 0; i < 8; i++) r[i] = 0;
         return;
     }
-    const uint32_t n = (uint32_t)k;   // words in the lane's region per round
+    const uint32_t n = (uint32_t)k;
     const uint32_t mask = (1u << k) - 1u;
     const uint32_t b = (uint32_t)(8 * g) * (uint32_t)k;
     if (KSMALL) {
-        uint32_t x = fetch32(rw, n, b);
+        uint32_t x = fetch32<STAGED>(rw, n, b);
 #pragma unroll
         for (int i = 0; i < 8; i++) {
             r[i] = x & mask;
@@ -107,7 +126,7 @@ __device__ __forceinline__ void rem_group(const uint32_t *rw, int k, int g, uint
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < 8; i++) r[i] = fetch32(rw, n, b + (uint32_t)(i * k)) & mask;
+        for (int i = 0; i < 8; i++) r[i] = fetch32_checked(rw, n, b + (uint32_t)(i * k)) & mask;
     }
 }
 
@@ -173,16 +192,145 @@ struct ChunkOut {
     }
 };
 
-template <int LAT, bool DITHER, bool KV, bool KSMALL>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const DecodeArgs a) {
+// Valid word range of chunk c, or nw = 0 if the offsets are not consistent.
+struct ChunkWords {
+    unsigned long long w0, nw;
+    bool ok;
+};
+
+__device__ __forceinline__ ChunkWords chunk_words(const DecodeArgs &a, unsigned long long c) {
+    ChunkWords r;
+    r.w0 = a.offsets[c];
+    const unsigned long long w1 = a.offsets[c + 1];
+    r.ok = r.w0 <= w1 && w1 <= a.stream_words;
+    r.nw = r.ok ? w1 - r.w0 : 0ull;
+    return r;
+}
+
+// Start the copy of a chunk's words into a stage (cp.async, 4 bytes per lane and
+// step) and zero the pad after them; one commit group per call.
+__device__ __forceinline__ void stage_chunk(const DecodeArgs &a, const ChunkWords &cw, uint32_t *stage, int lane) {
+    if (cw.nw <= (unsigned long long)kStageWords) {
+        const uint32_t n = (uint32_t)cw.nw;
+        const uint32_t *src = a.stream + cw.w0;
+        for (uint32_t i = lane; i < n; i += 32) {
+            const unsigned sa = (unsigned)__cvta_generic_to_shared(stage + i);
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(src + i) : "memory");
+        }
+        if (lane < kStagePad) stage[n + lane] = 0u;
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// The 4 rounds of one chunk, reading its planes from `src` (a stage when STAGED).
+template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED>
+__device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOut<KV> &geo, const uint32_t *src,
+                                              bool ok, uint32_t nc, uint32_t nr, uint32_t nu,
+                                              const uint32_t *startbit, const uint32_t *sign_tab, int lane) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
+    const int k = a.k;
+    const int q = lane & 3;
+    const uint32_t *un = src + nc + nr;
+    const float2 e2 = make_float2(geo.e_scale, geo.e_scale);
+    bool bad = false;
+    const int nrounds = (geo.ntiles + kTilesPerRound - 1) / kTilesPerRound;
+#pragma unroll 1
+    for (int r = 0; r < nrounds; r++) {
+        char *dst = nullptr;
+        int tcol = 0;
+        unsigned long long e0 = 0;
+        const bool valid = geo.tile(a, r * kTilesPerRound + (lane >> 2), dst, tcol, e0);
+        const uint32_t segi = 32u * r + lane;
+        float2 v[16];
+        bool lane_ok = ok;
+        if (ok && valid) {
+            uint32_t bp = startbit[segi];
+            const uint32_t *rw = src + nc + segi * (uint32_t)k;
+            const uint32_t cw = (LAT == HQ_E8) ? src[4 * r + (lane >> 3)] : 0u;
+            const uint32_t coset = (cw >> (4 * (lane & 7))) & 0xFu;
+            const unsigned long long eq = e0 + 32ull * q;
+#pragma unroll
+            for (int g = 0; g < 4; g++) {
+                uint32_t qv[8], rv[8];
+                unary4<STAGED>(un, nu, bp, lane_ok, qv);
+                unary4<STAGED>(un, nu, bp, lane_ok, qv + 4);
+                rem_group<KSMALL, STAGED>(rw, k, g, rv);
+                float u[8];
+#pragma unroll
+                for (int bb = 0; bb < 8 / N; bb++) {
+                    const int b = g * (8 / N) + bb;
+                    int32_t m[N], qq[N];
+                    float p[N];
+#pragma unroll
+                    for (int i = 0; i < N; i++) m[i] = unzigzag((qv[bb * N + i] << k) | rv[bb * N + i]);
+                    L::reinsert(m, (coset >> b) & 1u, qq);
+                    L::point(qq, p);
+                    if (DITHER) {
+                        float d[N];
+                        dither_block<LAT>(a.seed, eq + (unsigned long long)(8 * g + bb * N), d);
+#pragma unroll
+                        for (int i = 0; i < N; i++) p[i] = __fsub_rn(p[i], d[i]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < N; i++) u[bb * N + i] = p[i];
+                }
+#pragma unroll
+                for (int j = 0; j < 4; j++) v[4 * g + j] = f2_mul(make_float2(u[2 * j], u[2 * j + 1]), e2);
+            }
+            if (bp > nu * 32u) lane_ok = false;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; j++) v[j] = make_float2(0.0f, 0.0f);
+        }
+        if (valid && !lane_ok) bad = true;
+        fwht128_quarter(v, lane);
+        // a tile is written as zeros unless all four of its lanes decoded
+        const unsigned bad_lanes = __ballot_sync(0xffffffffu, valid && !lane_ok);
+        const bool tile_bad = (bad_lanes >> (lane & ~3)) & 0xFu;
+        if (dst) {
+            const uint32_t *sg = sign_tab + tcol * kSignStride + q * kSignQuarter;
+            if (a.out_fp32) {
+                uint4 *o = reinterpret_cast<uint4 *>(dst) + 8 * q;
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const uint32_t s0w = sg[2 * j], s1w = sg[2 * j + 1];
+                    uint4 w;
+                    w.x = tile_bad ? 0u : __float_as_uint(v[2 * j].x) ^ (s0w << 16);
+                    w.y = tile_bad ? 0u : __float_as_uint(v[2 * j].y) ^ (s0w & 0x80000000u);
+                    w.z = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].x) ^ (s1w << 16);
+                    w.w = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].y) ^ (s1w & 0x80000000u);
+                    o[j] = w;
+                }
+            } else {
+                uint4 *o = reinterpret_cast<uint4 *>(dst) + 4 * q;
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
+                    const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int u2 = 0; u2 < 4; u2++) {
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(v[4 * j + u2].x, v[4 * j + u2].y);
+                        pk[u2] = tile_bad ? 0u : (*reinterpret_cast<uint32_t *>(&hb) ^ sw[u2]);
+                    }
+                    o[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+        }
+    }
+    return bad;
+}
+
+template <int LAT, bool DITHER, bool KV, bool KSMALL>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
+    constexpr int kStageSlot = kStageWords + kStagePad;
     uint32_t *sign_tab = smem;
     uint32_t *stage_all = smem + a.tcols * kSignStride;
-    uint32_t *start_all = stage_all + kWarpsPerCta * kStageWords;
+    uint32_t *start_all = stage_all + kWarpsPerCta * 2 * kStageSlot;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t *stage = stage_all + warp * kStageWords;
+    uint32_t *stages = stage_all + warp * 2 * kStageSlot;
     uint32_t *startbit = start_all + warp * 128;   // first unary bit of every 32-symbol segment
 
     for (int i = threadIdx.x; i < a.tcols * 64; i += blockDim.x) {
@@ -194,27 +342,39 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
     __syncthreads();
 
     const int k = a.k;
-    const int q = lane & 3;
     uint32_t status = 0;
     const unsigned long long nwarps = (unsigned long long)gridDim.x * kWarpsPerCta;
-    for (unsigned long long c = (unsigned long long)blockIdx.x * kWarpsPerCta + warp; c < a.n_chunks; c += nwarps) {
+    unsigned long long c = (unsigned long long)blockIdx.x * kWarpsPerCta + warp;
+    int buf = 0;
+    ChunkWords cw = {0, 0, false};
+    if (c < a.n_chunks) {
+        cw = chunk_words(a, c);
+        stage_chunk(a, cw, stages, lane);
+    }
+    for (; c < a.n_chunks; c += nwarps, buf ^= 1) {
+        // start bringing in the next chunk while this one is decoded
+        const unsigned long long cn = c + nwarps;
+        ChunkWords cwn = {0, 0, false};
+        if (cn < a.n_chunks) {
+            cwn = chunk_words(a, cn);
+            stage_chunk(a, cwn, stages + (buf ^ 1) * kStageSlot, lane);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncwarp();
+
         ChunkOut<KV> geo;
         geo.init(a, c);
         const int ntiles = geo.ntiles;
-        const unsigned long long w0 = a.offsets[c], w1 = a.offsets[c + 1];
         const uint32_t nsym = (uint32_t)ntiles * kTile, nseg = 4u * (uint32_t)ntiles;
-        const unsigned long long nc = (LAT == HQ_E8) ? (unsigned long long)(16 * ntiles + 31) / 32 : 0ull;
-        const unsigned long long nr = 4ull * (unsigned long long)k * (unsigned long long)ntiles;
-        bool ok = w0 <= w1 && w1 <= a.stream_words && (w1 - w0) >= nc + nr &&
-                  (w1 - w0 - nc - nr) < (unsigned long long)(kMaxUnaryBits / 32u);
-        const unsigned long long nw = ok ? w1 - w0 : 0ull;
-        const bool staged = nw <= (unsigned long long)kStageWords;
-        const uint32_t *src = staged ? stage : a.stream + w0;
-        if (staged) {
-            for (unsigned long long i = lane; i < nw; i += 32) stage[i] = __ldg(a.stream + w0 + i);
-        }
-        __syncwarp();
-        const uint32_t nu = ok ? (uint32_t)(nw - nc - nr) : 0u;
+        const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
+        const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
+        bool ok = cw.ok && cw.nw >= (unsigned long long)(nc + nr) &&
+                  (cw.nw - nc - nr) < (unsigned long long)(kMaxUnaryBits / 32u);
+        const bool staged = cw.nw <= (unsigned long long)kStageWords;
+        const uint32_t *src = staged ? stages + buf * kStageSlot : a.stream + cw.w0;
+        const uint32_t nu = ok ? (uint32_t)(cw.nw - nc - nr) : 0u;
         const uint32_t *un = src + nc + nr;
 
         // ---- first unary bit of every 32-symbol segment: popc + scan over 32 word ranges
@@ -245,108 +405,21 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
                     w = un[i];
                     pc = __popc(w);
                 }
-                for (uint32_t r = j - seen; r; r--) w &= w - 1u;   // drop the lower set bits
-                startbit[ss] = i * 32u + (uint32_t)(__ffs(w) - 1) + 1u;
+                startbit[ss] = i * 32u + select_bit(w, j - seen) + 1u;
             }
             if (lane == 0) startbit[0] = 0;
         }
         __syncwarp();
 
-        // ---- 4 rounds of 8 tiles: lane decodes segment 32 r + lane = quarter q of tile 8 r + lane / 4
-        bool bad = false;
-        const int nrounds = (ntiles + kTilesPerRound - 1) / kTilesPerRound;
-#pragma unroll 1
-        for (int r = 0; r < nrounds; r++) {
-            char *dst = nullptr;
-            int tcol = 0;
-            unsigned long long e0 = 0;
-            const bool valid = geo.tile(a, r * kTilesPerRound + (lane >> 2), dst, tcol, e0);
-            const uint32_t segi = 32u * r + lane;
-            float2 v[16];
-            bool lane_ok = ok;
-            if (ok && valid) {
-                UnaryReader ur;
-                ur.init(un, nu, startbit[segi]);
-                const uint32_t *rw = src + nc + (unsigned long long)segi * k;
-                const uint32_t cw = (LAT == HQ_E8) ? src[4 * r + (lane >> 3)] : 0u;
-                const uint32_t coset = (cw >> (4 * (lane & 7))) & 0xFu;
-                const unsigned long long eq = e0 + 32ull * q;
-#pragma unroll
-                for (int g = 0; g < 4; g++) {
-                    uint32_t qv[8], rv[8];
-                    ur.group(qv);
-                    rem_group<KSMALL>(rw, k, g, rv);
-                    float u[8];
-#pragma unroll
-                    for (int bb = 0; bb < 8 / N; bb++) {
-                        const int b = g * (8 / N) + bb;
-                        int32_t m[N], qq[N];
-                        float p[N];
-#pragma unroll
-                        for (int i = 0; i < N; i++) m[i] = unzigzag((qv[bb * N + i] << k) | rv[bb * N + i]);
-                        L::reinsert(m, (coset >> b) & 1u, qq);
-                        L::point(qq, p);
-                        if (DITHER) {
-                            float d[N];
-                            dither_block<LAT>(a.seed, eq + (unsigned long long)(8 * g + bb * N), d);
-#pragma unroll
-                            for (int i = 0; i < N; i++) p[i] = __fsub_rn(p[i], d[i]);
-                        }
-#pragma unroll
-                        for (int i = 0; i < N; i++) u[bb * N + i] = p[i];
-                    }
-                    const float2 e2 = make_float2(geo.e_scale, geo.e_scale);
-#pragma unroll
-                    for (int j = 0; j < 4; j++) v[4 * g + j] = f2_mul(make_float2(u[2 * j], u[2 * j + 1]), e2);
-                }
-                lane_ok = ur.ok;
-            } else {
-#pragma unroll
-                for (int j = 0; j < 16; j++) v[j] = make_float2(0.0f, 0.0f);
-            }
-            if (valid && !lane_ok) {
-                bad = true;
-#pragma unroll
-                for (int j = 0; j < 16; j++) v[j] = make_float2(0.0f, 0.0f);
-            }
-            fwht128_quarter(v, lane);
-            // a tile is good only if all four of its lanes are
-            const unsigned bad_lanes = __ballot_sync(0xffffffffu, valid && !lane_ok);
-            const bool tile_bad = (bad_lanes >> (lane & ~3)) & 0xFu;
-            if (dst) {
-                const uint32_t *sg = sign_tab + tcol * kSignStride + q * kSignQuarter;
-                if (a.out_fp32) {
-                    uint4 *o = reinterpret_cast<uint4 *>(dst) + 8 * q;
-#pragma unroll
-                    for (int j = 0; j < 8; j++) {
-                        const uint32_t s0w = sg[2 * j], s1w = sg[2 * j + 1];
-                        uint4 w;
-                        w.x = tile_bad ? 0u : __float_as_uint(v[2 * j].x) ^ (s0w << 16);
-                        w.y = tile_bad ? 0u : __float_as_uint(v[2 * j].y) ^ (s0w & 0x80000000u);
-                        w.z = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].x) ^ (s1w << 16);
-                        w.w = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].y) ^ (s1w & 0x80000000u);
-                        o[j] = w;
-                    }
-                } else {
-                    uint4 *o = reinterpret_cast<uint4 *>(dst) + 4 * q;
-#pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        const uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
-                        const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int u2 = 0; u2 < 4; u2++) {
-                            __nv_bfloat162 hb = __floats2bfloat162_rn(v[4 * j + u2].x, v[4 * j + u2].y);
-                            pk[u2] = tile_bad ? 0u : (*reinterpret_cast<uint32_t *>(&hb) ^ sw[u2]);
-                        }
-                        o[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    }
-                }
-            }
-        }
+        const bool bad = staged ? decode_rounds<LAT, DITHER, KV, KSMALL, true>(a, geo, src, ok, nc, nr, nu, startbit,
+                                                                                sign_tab, lane)
+                                : decode_rounds<LAT, DITHER, KV, KSMALL, false>(a, geo, src, ok, nc, nr, nu, startbit,
+                                                                                 sign_tab, lane);
         if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) status |= HQ_ST_CORRUPT;
+        cw = cwn;
         __syncwarp();
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     if (a.stats) {
         status = __reduce_or_sync(0xffffffffu, status);
         if (lane == 0 && status) atomicOr(&a.stats->status, status);
@@ -355,8 +428,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
 
 template <int LAT, bool DITHER, bool KV>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
-    const size_t smem =
-        (size_t)(a.tcols * kSignStride + kWarpsPerCta * kStageWords + kWarpsPerCta * 128) * sizeof(uint32_t);
+    const size_t smem = (size_t)(a.tcols * kSignStride + kWarpsPerCta * 2 * (kStageWords + kStagePad) +
+                                 kWarpsPerCta * 128) *
+                        sizeof(uint32_t);
     auto kern = a.k <= 4 ? decode_kernel<LAT, DITHER, KV, true> : decode_kernel<LAT, DITHER, KV, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

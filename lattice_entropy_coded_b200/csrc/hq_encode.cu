@@ -11,10 +11,15 @@
 //  * per round a warp scan of unary lengths places every lane's codewords;
 //    remainder bits, E8 coset bits and unary terminators go into a per-warp
 //    shared-memory stage that holds the whole chunk;
+//  * the next round's input is copied into shared memory (cp.async) while the
+//    current round is computed;
 //  * a persistent grid takes chunk tickets from a global counter, so a chunk's
 //    predecessors are always already running; a single-pass decoupled
 //    look-back over 64-bit (flag, value) words gives the chunk's word offset
-//    (bounded waits: HQ_ST_TIMEOUT), and the stage is written out coalesced;
+//    (bounded waits: HQ_ST_TIMEOUT).  A chunk publishes its size as soon as it
+//    is encoded and resolves its offset after the warp has encoded its next
+//    chunk into a second stage, so predecessors have normally published by
+//    then; the stage is then written out coalesced;
 //  * a chunk larger than the stage is re-encoded by a separate path that sets
 //    its bits in place in global memory (same stream; only for extreme codes).
 #include <cuda_runtime.h>
@@ -36,27 +41,36 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
     return v;
 }
 
-// Exclusive prefix (in words) of chunk c over chunks [0, c) of this call.
-// Whole warp calls it; lane 0 publishes.  Bounded: gives up after spin_limit polls.
-__device__ __noinline__ unsigned long long lookback(unsigned long long *lb, unsigned long long c,
-                                                    unsigned long long agg, uint32_t spin_limit, bool &timed_out) {
+// Decoupled look-back over 64-bit words (flag in the top two bits, value
+// below): 0 = nothing yet, AGG = the chunk's own word count, INC = the chunk's
+// inclusive prefix.  A chunk publishes its count as soon as it is encoded and
+// resolves its offset later, so waits are short.
+
+// Publish chunk c's word count (chunk 0 publishes its inclusive prefix).
+__device__ __forceinline__ void lookback_publish(unsigned long long *lb, unsigned long long c,
+                                                 unsigned long long agg) {
+    if ((threadIdx.x & 31) == 0) st_relaxed_u64(lb + c, (c == 0 ? kFlagInc : kFlagAgg) | agg);
+}
+
+// Exclusive prefix (in words) of chunk c: walk back over predecessors 32 at a
+// time until one with an inclusive prefix, summing counts; then publish c's
+// inclusive prefix.  Whole warp calls it.  Bounded: gives up after spin_limit polls.
+__device__ __noinline__ unsigned long long lookback_resolve(unsigned long long *lb, unsigned long long c,
+                                                            unsigned long long agg, uint32_t spin_limit,
+                                                            bool &timed_out) {
     const int lane = threadIdx.x & 31;
-    if (c == 0) {
-        if (lane == 0) st_relaxed_u64(lb, kFlagInc | agg);
-        return 0;
-    }
-    if (lane == 0) st_relaxed_u64(lb + c, kFlagAgg | agg);
+    if (c == 0) return 0;
     unsigned long long excl = 0;
     long long pos = (long long)c - 1;
     uint32_t spins = 0;
     while (true) {
-        long long idx = pos - lane;
-        unsigned long long v = (idx >= 0) ? ld_relaxed_u64(lb + idx) : kFlagInc;
-        unsigned flag = (unsigned)(v >> 62);
-        unsigned inc = __ballot_sync(0xffffffffu, flag == 2u);
-        unsigned zero = __ballot_sync(0xffffffffu, flag == 0u);
-        int first_inc = inc ? __ffs(inc) - 1 : 32;
-        unsigned relevant = (first_inc >= 31) ? 0xffffffffu : ((2u << first_inc) - 1u);
+        const long long idx = pos - lane;
+        const unsigned long long v = (idx >= 0) ? ld_relaxed_u64(lb + idx) : kFlagInc;
+        const unsigned flag = (unsigned)(v >> 62);
+        const unsigned inc = __ballot_sync(0xffffffffu, flag == 2u);
+        const unsigned zero = __ballot_sync(0xffffffffu, flag == 0u);
+        const int first_inc = inc ? __ffs(inc) - 1 : 32;
+        const unsigned relevant = (first_inc >= 31) ? 0xffffffffu : ((2u << first_inc) - 1u);
         if (zero & relevant) {
             if (++spins > spin_limit) {
                 timed_out = true;
@@ -123,27 +137,60 @@ struct ChunkGeo {
     }
 };
 
-// One round for one lane: its quarter (32 elements) of tile 8r + lane/4 ->
-// D x -> H_128 (with the three partner lanes) -> * c -> [+ d] -> lattice
-// blocks -> 32 zigzag symbols and the E8 coset bits of its blocks.
-// Whole warp must call it (shuffles).
+// Input of one round for one lane: its quarter (32 bf16 = 64 bytes) of tile
+// 8r + lane/4.  The bytes are copied ahead of use with cp.async into the
+// lane's own 80-byte slot of a per-warp shared buffer (80: 8 consecutive lanes'
+// 16-byte accesses hit distinct banks); each lane reads back only what it
+// copied, so no warp barrier is needed.
+struct RoundInput {
+    bool valid;
+    int tcol;
+    unsigned long long e0;
+};
+
+constexpr int kInSlotWords = 20;
+
+__device__ __forceinline__ void prefetch_round(const EncodeArgs &a, const ChunkGeo &geo, int r, int lane,
+                                               uint32_t *slot) {
+    const uint16_t *src = nullptr;
+    int tcol;
+    unsigned long long e0;
+    if (geo.tile(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, tcol, e0)) {
+        const uint16_t *g = src + 32 * (lane & 3);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const unsigned sa = (unsigned)__cvta_generic_to_shared(slot + 4 * j);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(g + 8 * j) : "memory");
+        }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void round_input(const EncodeArgs &a, const ChunkGeo &geo, int r, int lane,
+                                            RoundInput &in) {
+    const uint16_t *src = nullptr;
+    in.tcol = 0;
+    in.e0 = 0;
+    in.valid = geo.tile(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, in.tcol, in.e0);
+}
+
+// One round for one lane: D x -> H_128 (with the three partner lanes) -> * c ->
+// [+ d] -> lattice blocks -> 32 zigzag symbols and the E8 coset bits of its
+// blocks.  Whole warp must call it (shuffles).
 template <int LAT, bool DITHER>
-__device__ __forceinline__ bool round_symbols(const EncodeArgs &a, const ChunkGeo &geo, int r, int lane,
-                                              const uint32_t *sign_tab, uint32_t (&z)[32], uint32_t &cbits) {
+__device__ __forceinline__ void round_symbols(const EncodeArgs &a, const RoundInput &in, const uint4 (&raw)[4],
+                                              int lane, const uint32_t *sign_tab, uint32_t (&z)[32],
+                                              uint32_t &cbits) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
     const int q = lane & 3;
-    const uint16_t *src = nullptr;
-    int tcol = 0;
-    unsigned long long e0 = 0;
-    const bool valid = geo.tile(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, tcol, e0);
-    const uint32_t *sg = sign_tab + tcol * kSignStride + q * kSignQuarter;
+    const uint32_t *sg = sign_tab + in.tcol * kSignStride + q * kSignQuarter;
     float2 v[16];
 #pragma unroll
     for (int j = 0; j < 4; j++) {
-        uint4 w = valid ? ldg_nc_v4(src + 32 * q + 8 * j) : make_uint4(0, 0, 0, 0);
-        uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
-        uint32_t ww[4] = {w.x ^ s.x, w.y ^ s.y, w.z ^ s.z, w.w ^ s.w};
+        const uint4 w = in.valid ? raw[j] : make_uint4(0, 0, 0, 0);
+        const uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
+        const uint32_t ww[4] = {w.x ^ s.x, w.y ^ s.y, w.z ^ s.z, w.w ^ s.w};
 #pragma unroll
         for (int t = 0; t < 4; t++)
             v[4 * j + t] = make_float2(__uint_as_float(ww[t] << 16), __uint_as_float(ww[t] & 0xFFFF0000u));
@@ -154,7 +201,7 @@ __device__ __forceinline__ bool round_symbols(const EncodeArgs &a, const ChunkGe
     for (int j = 0; j < 16; j++) v[j] = f2_mul(v[j], c2);
 
     cbits = 0;
-    const unsigned long long eq = e0 + 32ull * q;
+    const unsigned long long eq = in.e0 + 32ull * q;
 #pragma unroll
     for (int b = 0; b < 32 / N; b++) {
         float blk[N];
@@ -172,14 +219,9 @@ __device__ __forceinline__ bool round_symbols(const EncodeArgs &a, const ChunkGe
         uint32_t zz[N];
         cbits |= L::symbols(blk, zz) << b;
 #pragma unroll
-        for (int i = 0; i < N; i++) z[b * N + i] = zz[i];
+        for (int i = 0; i < N; i++) z[b * N + i] = in.valid ? zz[i] : 0u;
     }
-    if (!valid) {
-#pragma unroll
-        for (int i = 0; i < 32; i++) z[i] = 0;
-        cbits = 0;
-    }
-    return valid;
+    if (!in.valid) cbits = 0;
 }
 
 // Remainder bits of 32 symbols (warp-uniform k) into the lane's k words.
@@ -263,7 +305,20 @@ __device__ __noinline__ void encode_chunk_global(const EncodeArgs &a, const Chun
     unsigned long long urun = 0;
     for (int r = 0; r < nrounds; r++) {
         uint32_t z[32], cbits;
-        const bool valid = round_symbols<LAT, DITHER>(a, geo, r, lane, sign_tab, z, cbits);
+        RoundInput in;
+        round_input(a, geo, r, lane, in);
+        uint4 raw[4];
+        {
+            const uint16_t *src = nullptr;
+            int tc;
+            unsigned long long e;
+            geo.tile(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, tc, e);
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                raw[j] = in.valid ? ldg_nc_v4(src + 32 * (lane & 3) + 8 * j) : make_uint4(0, 0, 0, 0);
+        }
+        round_symbols<LAT, DITHER>(a, in, raw, lane, sign_tab, z, cbits);
+        const bool valid = in.valid;
         unsigned long long ub = 0;
 #pragma unroll
         for (int i = 0; i < 32; i++) ub += z[i] >> k;
@@ -293,13 +348,65 @@ __device__ __noinline__ void encode_chunk_global(const EncodeArgs &a, const Chun
     }
 }
 
+// A chunk that has been encoded into a stage and waits for its offset.
+struct Pending {
+    unsigned long long c, total;
+    bool overflow, range_bad;
+};
+
+template <int LAT, bool DITHER>
+__device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending &p, uint32_t *stage,
+                                             const uint32_t *sign_tab, unsigned long long base, uint32_t &status) {
+    const int lane = threadIdx.x & 31;
+    bool to = false;
+    const unsigned long long excl = lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to);
+    if (to) status |= HQ_ST_TIMEOUT;
+    const unsigned long long start = base + excl;
+    if (lane == 0) {
+        a.offsets[a.chunk_base + p.c] = start;
+        if (p.c + 1 == a.n_chunks) {
+            const unsigned long long end = start + p.total;
+            a.offsets[a.chunk_base + a.n_chunks] = end;
+            if (a.tail_out) *a.tail_out = end;
+            if (a.stats) a.stats->stream_words = end;
+            if (end > a.cap_words) status |= HQ_ST_CAPACITY;
+        }
+        if (p.c == 0 && a.row) *a.row = a.row_val;
+    }
+    if (!p.range_bad && !p.overflow) {
+        for (uint32_t i = lane; i < (uint32_t)p.total; i += 32)
+            if (start + i < a.cap_words) a.stream[start + i] = stage[i];
+    } else if (!p.range_bad) {
+        uint32_t *g = a.stream + start;
+        const unsigned long long room = (start < a.cap_words) ? a.cap_words - start : 0ull;
+        for (unsigned long long i = lane; i < p.total; i += 32)
+            if (i < room) g[i] = 0u;
+        __syncwarp();
+        __threadfence_block();
+        ChunkGeo geo;
+        geo.init(a.map, p.c);
+        const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * geo.ntiles + 31) / 32u : 0u;
+        const uint32_t nr = 4u * (uint32_t)a.k * (uint32_t)geo.ntiles;
+        encode_chunk_global<LAT, DITHER>(a, geo, sign_tab, g, room, nc, nr);
+    }
+    __syncwarp();
+}
+
+__device__ __forceinline__ unsigned long long take_ticket(const EncodeArgs &a) {
+    unsigned long long c = 0;
+    if ((threadIdx.x & 31) == 0) c = atomicAdd(a.ticket, 1u);
+    return __shfl_sync(0xffffffffu, c, 0);
+}
+
 template <int LAT, bool DITHER, bool KSMALL>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *sign_tab = smem;                                        // tcols * kSignStride
-    uint32_t *stage_all = smem + a.tcols * kSignStride;               // warps * kStageWords
+    uint32_t *stage_all = smem + a.tcols * kSignStride;               // warps * 2 * kStageWords
+    uint32_t *in_all = stage_all + kWarpsPerCta * 2 * kStageWords;    // warps * 32 * kInSlotWords
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t *stage = stage_all + warp * kStageWords;
+    uint32_t *stages = stage_all + warp * 2 * kStageWords;
+    uint32_t *slot = in_all + (warp * 32 + lane) * kInSlotWords;
 
     // Sign masks per bf16x2 pair: bit 15 flips the even column, bit 31 the odd one.
     for (int i = threadIdx.x; i < a.tcols * 64; i += blockDim.x) {
@@ -315,14 +422,21 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     uint32_t status = 0, zor_all = 0;
     unsigned long long payload = 0;
 
-    while (true) {
-        unsigned long long c = 0;
-        if (lane == 0) c = atomicAdd(a.ticket, 1u);
-        c = __shfl_sync(0xffffffffu, c, 0);
-        if (c >= a.n_chunks) break;
-
+    unsigned long long c = take_ticket(a);
+    if (c < a.n_chunks) {
+        ChunkGeo g0;
+        g0.init(a.map, c);
+        prefetch_round(a, g0, 0, lane, slot);
+    }
+    Pending pend;
+    bool have_pend = false;
+    int buf = 0;
+    while (c < a.n_chunks) {
+        const unsigned long long cn = take_ticket(a);
         ChunkGeo geo;
         geo.init(a.map, c);
+        uint32_t *stage = stages + buf * kStageWords;
+
         const int ntiles = geo.ntiles;
         const int nrounds = (ntiles + kTilesPerRound - 1) / kTilesPerRound;
         const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
@@ -337,8 +451,25 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         bool overflow = (nc + nr) > (uint32_t)kStageWords, range_bad = false;
 #pragma unroll 1
         for (int r = 0; r < nrounds; r++) {
+            // this round's bytes are arriving in the lane's slot; take them, then
+            // start the copy of the next round's
+            RoundInput cur;
+            round_input(a, geo, r, lane, cur);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            uint4 raw[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++) raw[j] = *reinterpret_cast<const uint4 *>(slot + 4 * j);
+            if (r + 1 < nrounds) {
+                prefetch_round(a, geo, r + 1, lane, slot);
+            } else if (cn < a.n_chunks) {
+                ChunkGeo gn;
+                gn.init(a.map, cn);
+                prefetch_round(a, gn, 0, lane, slot);
+            }
+
             uint32_t z[32], cbits;
-            const bool valid = round_symbols<LAT, DITHER>(a, geo, r, lane, sign_tab, z, cbits);
+            round_symbols<LAT, DITHER>(a, cur, raw, lane, sign_tab, z, cbits);
+            const bool valid = cur.valid;
             uint32_t usum = 0, lor = 0;
 #pragma unroll
             for (int i = 0; i < 32; i++) {
@@ -377,41 +508,22 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         }
         zor_all |= zor;
         if (range_bad) status |= HQ_ST_RANGE;
-        const unsigned long long nu = ((unsigned long long)urun + 31) / 32;
-        const unsigned long long total = nc + nr + nu;
+        const unsigned long long total = nc + nr + ((unsigned long long)urun + 31) / 32;
         payload += urun + (unsigned long long)nr * 32 + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
+        lookback_publish(a.lookback, c, total);
 
-        // ---- chunk offset
-        bool to = false;
-        const unsigned long long excl = lookback(a.lookback, c, total, a.spin_limit, to);
-        if (to) status |= HQ_ST_TIMEOUT;
-        const unsigned long long start = base + excl;
-        if (lane == 0) {
-            a.offsets[a.chunk_base + c] = start;
-            if (c + 1 == a.n_chunks) {
-                const unsigned long long end = start + total;
-                a.offsets[a.chunk_base + a.n_chunks] = end;
-                if (a.tail_out) *a.tail_out = end;
-                if (a.stats) a.stats->stream_words = end;
-                if (end > a.cap_words) status |= HQ_ST_CAPACITY;
-            }
-            if (c == 0 && a.row) *a.row = a.row_val;
-        }
-        __syncwarp();
-        if (!range_bad && !overflow) {
-            for (uint32_t i = lane; i < (uint32_t)total; i += 32)
-                if (start + i < a.cap_words) a.stream[start + i] = stage[i];
-        } else if (!range_bad) {
-            uint32_t *g = a.stream + start;
-            const unsigned long long room = (start < a.cap_words) ? a.cap_words - start : 0ull;
-            for (unsigned long long i = lane; i < total; i += 32)
-                if (i < room) g[i] = 0u;
-            __syncwarp();
-            __threadfence_block();
-            encode_chunk_global<LAT, DITHER>(a, geo, sign_tab, g, room, nc, nr);
-        }
-        __syncwarp();
+        // the previous chunk's predecessors have had a whole chunk's time to publish
+        if (have_pend) finish_chunk<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
+        pend.c = c;
+        pend.total = total;
+        pend.overflow = overflow;
+        pend.range_bad = range_bad;
+        have_pend = true;
+        c = cn;
+        buf ^= 1;
     }
+    if (have_pend) finish_chunk<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 
     if (a.stats) {
         zor_all = __reduce_or_sync(0xffffffffu, zor_all);
@@ -426,7 +538,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
 
 template <int LAT, bool DITHER>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
-    const size_t smem = (size_t)(a.tcols * kSignStride + kWarpsPerCta * kStageWords) * sizeof(uint32_t);
+    const size_t smem =
+        (size_t)(a.tcols * kSignStride + kWarpsPerCta * 2 * kStageWords + kWarpsPerCta * 32 * kInSlotWords) *
+        sizeof(uint32_t);
     auto kern = a.k <= 4 ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
