@@ -45,7 +45,8 @@ import synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "weight_4096x4096_rate_sweep"
 L2_FLUSH_BYTES = 256 << 20
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "encode_kernel_weight_4096x4096.md")
+PROFILE_ENCODE = os.path.join(ROOT, "profiles", "encode_kernel_e8_4bps.md")
+SM_COUNT, SMSP_PER_SM = 148, 4
 
 
 def rate_points():
@@ -70,19 +71,34 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """(bytes per launch of the encode kernel at the E8 4 bps point, from an ncu
-    capture) if the capture was taken with the current kernel source, else None."""
-    if not os.path.exists(PROFILE_TRAFFIC):
-        return None
-    src_hash, traffic = None, None
-    with open(PROFILE_TRAFFIC) as f:
+def profiled_encode():
+    """(DRAM bytes per launch, warp instructions per element) of the E8 4 bps encode
+    launch from the committed ncu capture, or (None, None) if the kernel source has
+    changed since it was taken."""
+    if not os.path.exists(PROFILE_ENCODE):
+        return None, None
+    vals = {}
+    with open(PROFILE_ENCODE) as f:
         for line in f:
-            if line.startswith("kernel_source_hash:"):
-                src_hash = line.split(":", 1)[1].strip()
-            if line.startswith("traffic_bytes_per_launch:"):
-                traffic = float(line.split(":", 1)[1].strip())
-    return traffic if src_hash == kernel_source_hash() else None
+            for key in ("kernel_source_hash", "traffic_bytes_per_launch", "warp_inst_per_element"):
+                if line.startswith(key + ":"):
+                    vals[key] = line.split(":", 1)[1].strip()
+    if vals.get("kernel_source_hash") != kernel_source_hash():
+        return None, None
+    return float(vals["traffic_bytes_per_launch"]), float(vals["warp_inst_per_element"])
+
+
+def reduce_max(values, device):
+    """Element-wise max over ranks (identity without a process group)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def weak_scaling_value(bytes_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job GB/s: every rank processes bytes_per_rank; the job takes the slowest rank's time."""
+    return world * bytes_per_rank / (max_ms * 1e6)
 
 
 # ------------------------------------------------------------------ clocks
@@ -228,37 +244,40 @@ def run_ours(args, rank: int, world: int, device: torch.device):
                               stream_words=words))
 
     # max over ranks of the summed kernel time
-    tot = torch.tensor([float(step_ms.sum()), float(enc_ms.sum()), float(dec_ms.sum()), wall_ms], device=device,
-                       dtype=torch.float64)
-    if world > 1:
-        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.MAX)
-    step_sum, enc_sum, dec_sum, wall_max = [float(v) for v in tot.cpu()]
+    step_sum, enc_sum, dec_sum, wall_max = reduce_max(
+        [float(step_ms.sum()), float(enc_ms.sum()), float(dec_ms.sum()), wall_ms], device)
     in_bytes = 2.0 * n * len(pts)               # bf16 input bytes per step, per rank
-    value = world * in_bytes * args.steps / (step_sum * 1e6)
-    enc_gbs = world * in_bytes * args.steps / (enc_sum * 1e6)
-    dec_gbs = world * in_bytes * args.steps / (dec_sum * 1e6)
+    value = weak_scaling_value(in_bytes * args.steps, world, step_sum)
+    enc_gbs = weak_scaling_value(in_bytes * args.steps, world, enc_sum)
+    dec_gbs = weak_scaling_value(in_bytes * args.steps, world, dec_sum)
 
-    # roofline of the dominant kernel (the encoder): algorithmic bytes per launch = bf16 in + stream + offsets
+    # roofline of the dominant kernel: the encoder at the E8 4 bps point (the slowest launch of a step)
     peak, peak_kind = measured_peaks()
+    clk = clk.summary()
     alg = [2.0 * n + 4.0 * pp["stream_words"] + 8.0 * (c.n_chunks + 1) for pp, c in zip(per_point, codecs)]
     enc_launch_ms = ms[:, :, 0].mean(0)
     dec_launch_ms = ms[:, :, 1].mean(0)
-    achieved = float(np.sum(alg) / (np.sum(enc_launch_ms) * 1e6))
-    achieved_dec = float(np.sum(alg) / (np.sum(dec_launch_ms) * 1e6))
-    dominant = "encode" if enc_sum >= dec_sum else "decode"
     e4 = [i for i, p in enumerate(per_point) if p["lattice"] == "E8" and p["bps_target"] == 4.0][0]
-    tr = profiled_traffic()
-    roofline = {"kernel": "hq::encode_kernel (all 12 points, averaged)" if dominant == "encode"
-                else "hq::decode_kernel (all 12 points, averaged)",
-                "bound": "hbm", "achieved": round(achieved if dominant == "encode" else achieved_dec, 1),
-                "peak": peak, "unit": "GB/s",
-                "frac": round((achieved if dominant == "encode" else achieved_dec) / peak, 4),
-                "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, burst copy)" if peak_kind == "measured"
-                else "fallback",
-                "traffic": tr, "traffic_launch": "E8 4 bps point" if tr else None,
-                "algorithmic_bytes_e8_4bps": alg[e4],
-                "decode_achieved": round(achieved_dec, 1), "decode_frac": round(achieved_dec / peak, 4),
-                "encode_achieved": round(achieved, 1), "encode_frac": round(achieved / peak, 4)}
+    hbm_achieved = alg[e4] / (enc_launch_ms[e4] * 1e6)
+    traffic, inst_per_elem = profiled_encode()
+    sm_mhz = clk["sm_mhz"] or 1965.0
+    issue_peak = SM_COUNT * SMSP_PER_SM * sm_mhz * 1e6 / 1e9          # G warp-instructions / s
+    roofline = {"kernel": "hq::encode_kernel<E8> at 4 bps (one launch, 4096x4096)",
+                "bound": "alu", "unit": "Ginst/s",
+                "achieved": None if inst_per_elem is None else round(inst_per_elem * n / (enc_launch_ms[e4] * 1e6), 1),
+                "peak": round(issue_peak, 1),
+                "frac": None if inst_per_elem is None else round(inst_per_elem * n / (enc_launch_ms[e4] * 1e6) / issue_peak, 4),
+                "peak_kind": f"issue slots: {SM_COUNT} SMs x {SMSP_PER_SM} schedulers x 1 warp-instruction/cycle at the "
+                             f"sampled {sm_mhz:.0f} MHz",
+                "traffic": traffic,
+                "hbm": {"achieved": round(hbm_achieved, 1), "peak": peak, "unit": "GB/s",
+                        "frac": round(hbm_achieved / peak, 4),
+                        "peak_kind": ("measured, MEASURED_PEAKS.json hbm_gbs (burst copy; kernels are timed alone)"
+                                      if peak_kind == "measured" else "fallback 6.65 TB/s"),
+                        "algorithmic_bytes": alg[e4]},
+                "all_points": {"encode_hbm_achieved": round(float(np.sum(alg) / (np.sum(enc_launch_ms) * 1e6)), 1),
+                               "decode_hbm_achieved": round(float(np.sum(alg) / (np.sum(dec_launch_ms) * 1e6)), 1),
+                               "unit": "GB/s"}}
 
     # end to end through the C ABI with host buffers: H2D of the input, quantize+decode per point,
     # D2H of every reconstruction and stats block
@@ -266,7 +285,7 @@ def run_ours(args, rank: int, world: int, device: torch.device):
 
     return dict(value=value, enc_gbs=enc_gbs, dec_gbs=dec_gbs, ms_per_step=step_sum / args.steps,
                 wall_ms_per_step=wall_max / args.steps, per_point=per_point, roofline=roofline,
-                clocks=clk.summary(), e2e=e2e, launches=2 * len(pts) * args.steps, n=n, in_bytes=in_bytes)
+                clocks=clk, e2e=e2e, launches=2 * len(pts) * args.steps, n=n, in_bytes=in_bytes)
 
 
 def run_e2e(args, hq, codecs, pts, rows, cols, device, stream, world):
@@ -297,14 +316,11 @@ def run_e2e(args, hq, codecs, pts, rows, cols, device, stream, world):
         step()
     t1.record(stream)
     torch.cuda.synchronize(device)
-    ms = torch.tensor([t0.elapsed_time(t1)], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
-    ms = float(ms.item())
+    ms = reduce_max([t0.elapsed_time(t1)], device)[0]
     for i in range(len(pts)):
         assert hq.read_stats(host_stats[i])["status"] == 0
     in_bytes = 2.0 * n * len(pts)
-    return {"value": round(world * in_bytes * steps / (ms * 1e6), 3), "unit": "GB/s",
+    return {"value": round(weak_scaling_value(in_bytes * steps, world, ms), 3), "unit": "GB/s",
             "h2d_bytes_per_step": 2 * n, "d2h_bytes_per_step": len(pts) * (2 * n + 32),
             "steps": steps, "ms_per_step": round(ms / steps, 3)}
 

@@ -222,6 +222,47 @@ __device__ __forceinline__ void stage_chunk(const DecodeArgs &a, const ChunkWord
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
+// First unary bit of every 32-symbol segment of a chunk (startbit[s]): the
+// lanes split the unary plane into 32 word ranges, count terminators (popc),
+// scan, and each lane locates the segment boundaries that fall in its range.
+// Returns false (chunk corrupt) unless the plane holds exactly nsym terminators.
+__device__ __forceinline__ bool find_segment_starts(const uint32_t *un, uint32_t nu, uint32_t nsym, uint32_t nseg,
+                                                    bool ok, uint32_t *startbit, int lane) {
+    const uint32_t seg = (nu + 31u) / 32u;
+    const uint32_t s0 = min(nu, (uint32_t)lane * seg), s1 = min(nu, s0 + seg);
+    uint32_t cnt = 0;
+    for (uint32_t i = s0; i < s1; i++) cnt += __popc(un[i]);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    const uint32_t ones = __shfl_sync(0xffffffffu, incl, 31);
+    ok = ok && ones == nsym;
+    if (ok) {
+        const uint32_t before = incl - cnt;
+        // terminator j = 32 s - 1 closes segment s - 1; find those inside [before, incl)
+        uint32_t ss = (before + 1u + 31u) / 32u;
+        if (ss == 0) ss = 1;
+        uint32_t i = s0, seen = before;
+        for (; ss < nseg && 32u * ss - 1u < incl; ss++) {
+            const uint32_t j = 32u * ss - 1u;
+            uint32_t w = un[i], pc = __popc(w);
+            while (seen + pc <= j) {
+                seen += pc;
+                i++;
+                w = un[i];
+                pc = __popc(w);
+            }
+            startbit[ss] = i * 32u + select_bit(w, j - seen) + 1u;
+        }
+        if (lane == 0) startbit[0] = 0;
+    }
+    __syncwarp();
+    return ok;
+}
+
 // The 4 rounds of one chunk, reading its planes from `src` (a stage when STAGED).
 template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED>
 __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOut<KV> &geo, const uint32_t *src,
@@ -373,48 +414,19 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
         bool ok = cw.ok && cw.nw >= (unsigned long long)(nc + nr) &&
                   (cw.nw - nc - nr) < (unsigned long long)(kMaxUnaryBits / 32u);
         const bool staged = cw.nw <= (unsigned long long)kStageWords;
-        const uint32_t *src = staged ? stages + buf * kStageSlot : a.stream + cw.w0;
         const uint32_t nu = ok ? (uint32_t)(cw.nw - nc - nr) : 0u;
-        const uint32_t *un = src + nc + nr;
-
-        // ---- first unary bit of every 32-symbol segment: popc + scan over 32 word ranges
-        const uint32_t seg = (nu + 31u) / 32u;
-        const uint32_t s0 = min(nu, (uint32_t)lane * seg), s1 = min(nu, s0 + seg);
-        uint32_t cnt = 0;
-        for (uint32_t i = s0; i < s1; i++) cnt += __popc(un[i]);
-        uint32_t incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
+        // the staged and in-place paths get distinct pointer expressions so the
+        // staged one keeps its shared-memory address space after inlining
+        bool bad;
+        if (staged) {
+            const uint32_t *src = stages + buf * kStageSlot;
+            ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, true>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab, lane);
+        } else {
+            const uint32_t *src = a.stream + cw.w0;
+            ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, false>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab, lane);
         }
-        const uint32_t ones = __shfl_sync(0xffffffffu, incl, 31);
-        ok = ok && ones == nsym;
-        if (ok) {
-            const uint32_t before = incl - cnt;
-            // terminator j = 32 s - 1 closes segment s - 1; find those inside [before, incl)
-            uint32_t ss = (before + 1u + 31u) / 32u;
-            if (ss == 0) ss = 1;
-            uint32_t i = s0, seen = before;
-            for (; ss < nseg && 32u * ss - 1u < incl; ss++) {
-                const uint32_t j = 32u * ss - 1u;
-                uint32_t w = un[i], pc = __popc(w);
-                while (seen + pc <= j) {
-                    seen += pc;
-                    i++;
-                    w = un[i];
-                    pc = __popc(w);
-                }
-                startbit[ss] = i * 32u + select_bit(w, j - seen) + 1u;
-            }
-            if (lane == 0) startbit[0] = 0;
-        }
-        __syncwarp();
-
-        const bool bad = staged ? decode_rounds<LAT, DITHER, KV, KSMALL, true>(a, geo, src, ok, nc, nr, nu, startbit,
-                                                                                sign_tab, lane)
-                                : decode_rounds<LAT, DITHER, KV, KSMALL, false>(a, geo, src, ok, nc, nr, nu, startbit,
-                                                                                 sign_tab, lane);
         if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) status |= HQ_ST_CORRUPT;
         cw = cwn;
         __syncwarp();
