@@ -391,6 +391,111 @@ def run_reference(args):
             "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------ the other workloads
+def _events():
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def run_bulk(args):
+    """Time one of the other workloads end to end on the device (inputs resident in HBM,
+    larger than L2, launches back to back on one stream); prints one JSON line."""
+    import lattice_entropy_coded_b200 as hq
+    device = torch.device("cuda", 0)
+    wl = args.workload
+    w = synth.WORKLOADS[wl]
+    pts = rate_points()[wl]["points"]
+    out = {"workload": wl, "steps": args.steps, "warmup": args.warmup}
+    peak, _ = measured_peaks()
+    if w["kind"] == "kv":
+        H, T, A = w["heads"], w["tokens"], w["append"]
+        K, V = synth.kv(H, T, w["seed"], device=device)
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+        res = []
+        for p in pts:
+            src = K if p["tensor"] == "K" else V
+            params = hq.make_params("E8", 1.0, p["k"], w["seed"], 1)
+            cache = hq.KVCache(H, T, params, bits_per_scalar=p["bps"] + 4.0, max_appends=T // A + 1,
+                               max_append_tokens=A, device=device)
+            slices = [src[:, t:t + A] for t in range(0, T, A)]
+            outb = torch.empty(H, T, 128, dtype=torch.bfloat16, device=device)
+            app_ms, read_ms = [], []
+            for it in range(args.warmup + args.steps):
+                flush.fill_(it)   # the K (or V) tensor fits in L2: evict it before each step
+                hq.hq_kv_init(cache.cache, H, 128, params, cache.words, cache.offsets, cache.table, cache.tail,
+                              cache.stats)
+                a0, a1 = _events()
+                a0.record()
+                for sl in slices:
+                    cache.append(sl, p["alpha"])
+                a1.record()
+                r0, r1 = _events()
+                r0.record()
+                cache.read(outb)
+                r1.record()
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    app_ms.append(a0.elapsed_time(a1))
+                    read_ms.append(r0.elapsed_time(r1))
+            st = hq.read_stats(cache.stats)
+            n = src.numel()
+            words = int(cache.tail[(len(slices)) & 1].item())
+            mse = float(((outb.double() - src.double()) ** 2).mean())
+            am, rm = float(np.median(app_ms)), float(np.median(read_ms))
+            alg = 2.0 * n + 4.0 * words + 8.0 * (cache.cache.chunks + 1)
+            res.append(dict(tensor=p["tensor"], bps_target=p["bps"], k=p["k"], alpha=p["alpha"], status=st["status"],
+                            bps_payload=st["payload_bits"] / n, bps_stream=words * 32.0 / n, mse=mse,
+                            d_over_sigma2=mse / float(src.double().var()), appends=len(slices),
+                            append_ms=am, read_ms=rm, append_gbs=2.0 * n / (am * 1e6), read_gbs=2.0 * n / (rm * 1e6),
+                            append_hbm_frac=alg / (am * 1e6) / peak, read_hbm_frac=alg / (rm * 1e6) / peak))
+        out["points"] = res
+    else:
+        if w["kind"] == "weight":
+            mats = [synth.weight(w["rows"], w["cols"], w["seed"], device=device)]
+        elif w["kind"] == "weight_set":
+            mats = [m for _, m in synth.weight_set(w["seed"], device=device, layers=w["layers"])]
+        else:
+            mats = list(synth.student_t(w["n"], w["rows"], w["cols"], w["seed"], device=device))
+        n = sum(m.numel() for m in mats)
+        res = []
+        for p in pts:
+            params = hq.make_params(p["lattice"], p["alpha"], p["k"], w["seed"], 0)
+            codecs = [hq.Codec(m.shape[0], m.shape[1], params, device=device,
+                               cap_words=int(m.numel() * (p["bps"] + 3.0) / 32) + 8192) for m in mats]
+            outs = [torch.empty_like(m) for m in mats]
+            enc_ms, dec_ms = [], []
+            for it in range(args.warmup + args.steps):
+                e0, e1 = _events()
+                e0.record()
+                comps = [c.quantize(m) for c, m in zip(codecs, mats)]
+                e1.record()
+                d0, d1 = _events()
+                d0.record()
+                for c, cp, o in zip(codecs, comps, outs):
+                    c.dequantize(cp, o)
+                d1.record()
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    enc_ms.append(e0.elapsed_time(e1))
+                    dec_ms.append(d0.elapsed_time(d1))
+            stats = [hq.read_stats(c.stats) for c in codecs]
+            words = sum(int(c.offsets[-1].item()) for c in codecs)
+            nch = sum(c.n_chunks + 1 for c in codecs)
+            se = sum(float(((o.double() - m.double()) ** 2).sum()) for o, m in zip(outs, mats))
+            var = sum(float(m.double().var()) * m.numel() for m in mats) / n
+            em, dm = float(np.median(enc_ms)), float(np.median(dec_ms))
+            alg = 2.0 * n + 4.0 * words + 8.0 * nch
+            res.append(dict(lattice=p["lattice"], bps_target=p["bps"], k=p["k"], alpha=p["alpha"],
+                            status=max(st["status"] for st in stats),
+                            bps_payload=sum(st["payload_bits"] for st in stats) / n, bps_stream=words * 32.0 / n,
+                            mse=se / n, d_over_sigma2=se / n / var, matrices=len(mats), elements=n,
+                            encode_ms=em, decode_ms=dm, encode_gbs=2.0 * n / (em * 1e6), decode_gbs=2.0 * n / (dm * 1e6),
+                            encode_hbm_frac=alg / (em * 1e6) / peak, decode_hbm_frac=alg / (dm * 1e6) / peak))
+            del codecs, outs, comps
+            torch.cuda.empty_cache()
+        out["points"] = res
+    print(json.dumps(out), flush=True)
+
+
 # ------------------------------------------------------------------ single-matrix case (profiling)
 def run_case(args):
     """Quantize + decode one R x C synthetic weight matrix (seed 1) at one operating point of
@@ -446,6 +551,9 @@ def main():
     args.warmup = max(3, args.warmup)
     if args.case:
         run_case(args)
+        return
+    if args.workload != DEFAULT_WORKLOAD and args.impl == "ours":
+        run_bulk(args)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -250,10 +250,10 @@ class Codec:
 class KVCache:
     """A compressed K or V cache (one layer) with torch-allocated device buffers."""
 
-    def __init__(self, heads: int, max_tokens: int, params: hq_params, words_per_token_head: float = 2.0,
+    def __init__(self, heads: int, max_tokens: int, params: hq_params, bits_per_scalar: float = 4.0,
                  max_appends: int = 4096, max_append_tokens: int = 4096, device="cuda"):
         max_chunks = heads * ((max_tokens + 31) // 32 + max_appends)
-        cap = int(heads * max_tokens * 128 * words_per_token_head / 32) + max_chunks * 64 + 1024
+        cap = int(heads * max_tokens * 128 * bits_per_scalar / 32) + max_chunks * 64 + 1024
         self.words = torch.empty(cap, dtype=torch.int32, device=device)
         self.offsets = torch.empty(max_chunks + 1, dtype=torch.int64, device=device)
         self.table = torch.zeros(max_appends * 32, dtype=torch.uint8, device=device)

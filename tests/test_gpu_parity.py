@@ -151,7 +151,7 @@ def _kv_case(H, Ts, lat, alpha, k, seed, dither, source):
     hq = _hq()
     params = hq.make_params(lat, 1.0, k, seed, dither)
     total_t = sum(Ts)
-    cache = hq.KVCache(H, total_t, params, words_per_token_head=16.0, max_appends=len(Ts) + 1,
+    cache = hq.KVCache(H, total_t, params, bits_per_scalar=16.0, max_appends=len(Ts) + 1,
                        max_append_tokens=max(Ts))
     appends, t0 = [], 0
     for T in Ts:
