@@ -330,30 +330,28 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
         const unsigned bad_lanes = __ballot_sync(0xffffffffu, valid && !lane_ok);
         const bool tile_bad = (bad_lanes >> (lane & ~3)) & 0xFu;
         if (dst) {
-            const uint32_t *sg = sign_tab + tcol * kSignStride + q * kSignQuarter;
+            const uint32_t es = sign_tab[tcol * kSignWords + q];
             if (a.out_fp32) {
                 uint4 *o = reinterpret_cast<uint4 *>(dst) + 8 * q;
 #pragma unroll
                 for (int j = 0; j < 8; j++) {
-                    const uint32_t s0w = sg[2 * j], s1w = sg[2 * j + 1];
+                    const uint32_t m0 = sign_pair_mask(es, 2 * j), m1 = sign_pair_mask(es, 2 * j + 1);
                     uint4 w;
-                    w.x = tile_bad ? 0u : __float_as_uint(v[2 * j].x) ^ (s0w << 16);
-                    w.y = tile_bad ? 0u : __float_as_uint(v[2 * j].y) ^ (s0w & 0x80000000u);
-                    w.z = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].x) ^ (s1w << 16);
-                    w.w = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].y) ^ (s1w & 0x80000000u);
+                    w.x = tile_bad ? 0u : __float_as_uint(v[2 * j].x) ^ (m0 << 16);
+                    w.y = tile_bad ? 0u : __float_as_uint(v[2 * j].y) ^ (m0 & 0x80000000u);
+                    w.z = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].x) ^ (m1 << 16);
+                    w.w = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].y) ^ (m1 & 0x80000000u);
                     o[j] = w;
                 }
             } else {
                 uint4 *o = reinterpret_cast<uint4 *>(dst) + 4 * q;
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
-                    const uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
-                    const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
                     uint32_t pk[4];
 #pragma unroll
                     for (int u2 = 0; u2 < 4; u2++) {
                         __nv_bfloat162 hb = __floats2bfloat162_rn(v[4 * j + u2].x, v[4 * j + u2].y);
-                        pk[u2] = tile_bad ? 0u : (*reinterpret_cast<uint32_t *>(&hb) ^ sw[u2]);
+                        pk[u2] = tile_bad ? 0u : (*reinterpret_cast<uint32_t *>(&hb) ^ sign_pair_mask(es, 4 * j + u2));
                     }
                     o[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
@@ -368,18 +366,13 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int kStageSlot = kStageWords + kStagePad;
     uint32_t *sign_tab = smem;
-    uint32_t *stage_all = smem + a.tcols * kSignStride;
+    uint32_t *stage_all = smem + a.tcols * kSignWords;
     uint32_t *start_all = stage_all + kWarpsPerCta * 2 * kStageSlot;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t *stages = stage_all + warp * 2 * kStageSlot;
     uint32_t *startbit = start_all + warp * 128;   // first unary bit of every 32-symbol segment
 
-    for (int i = threadIdx.x; i < a.tcols * 64; i += blockDim.x) {
-        const int tc = i >> 6, p = i & 63;
-        const unsigned long long col = (unsigned long long)tc * kTile + 2 * p;
-        sign_tab[tc * kSignStride + (p >> 4) * kSignQuarter + (p & 15)] =
-            (sign_bit(a.seed, col) << 15) | (sign_bit(a.seed, col + 1) << 31);
-    }
+    build_sign_table(sign_tab, a.tcols, a.seed);
     __syncthreads();
 
     const int k = a.k;
@@ -440,23 +433,17 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const Deco
 
 template <int LAT, bool DITHER, bool KV>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
-    const size_t smem = (size_t)(a.tcols * kSignStride + kWarpsPerCta * 2 * (kStageWords + kStagePad) +
+    const size_t smem = (size_t)(a.tcols * kSignWords + kWarpsPerCta * 2 * (kStageWords + kStagePad) +
                                  kWarpsPerCta * 128) *
                         sizeof(uint32_t);
-    auto kern = a.k <= 4 ? decode_kernel<LAT, DITHER, KV, true> : decode_kernel<LAT, DITHER, KV, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool small = a.k <= 4;
+    auto kern = small ? decode_kernel<LAT, DITHER, KV, true> : decode_kernel<LAT, DITHER, KV, false>;
+    static LaunchPlan plans[2];
+    unsigned grid = 0;
+    cudaError_t e = plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta,
+                                               grid);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarpsPerCta * 32, smem)) != cudaSuccess)
-        return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    unsigned long long want = (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta;
-    unsigned long long grid = (unsigned long long)sms * (unsigned long long)per_sm;
-    if (want < grid) grid = want;
-    if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, kWarpsPerCta * 32, smem, s>>>(a);
+    kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     return cudaGetLastError();
 }
 

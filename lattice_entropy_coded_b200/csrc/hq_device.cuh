@@ -31,6 +31,22 @@ __device__ __forceinline__ uint32_t sign_bit(uint64_t seed, uint64_t j) {
     return (uint32_t)(splitmix64(seed ^ kSignSalt, j) >> 63);
 }
 
+// Shared sign table: word 4 tc + q covers columns 128 tc + 32 q + [0, 32): bit t
+// (t < 16) is the sign bit of column 2t of the quarter and bit 16 + t that of
+// column 2t + 1.  So the XOR mask for the bf16 pair (2t, 2t + 1) held in one
+// word (even column in the low half) is sign_pair_mask(E, t): bits 15 and 31.
+// Each warp fills words with one generator call per lane and a ballot, lanes
+// 0-15 taking the even columns and 16-31 the odd ones.
+__device__ __forceinline__ void build_sign_table(uint32_t *tab, int tcols, uint64_t seed) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int off = (lane < 16) ? 2 * lane : 2 * (lane - 16) + 1;
+    for (int w = warp; w < tcols * kSignWords; w += nw) {
+        const uint32_t e = __ballot_sync(0xffffffffu, sign_bit(seed, (unsigned long long)w * 32ull + off) != 0u);
+        if (lane == 0) tab[w] = e;
+    }
+}
+__device__ __forceinline__ uint32_t sign_pair_mask(uint32_t e, int t) { return (e << (15 - t)) & 0x80008000u; }
+
 // ------------------------------------------------------------------ packed fp32
 // sm_100 executes two IEEE round-to-nearest fp32 operations per instruction on
 // a register pair (add/sub/mul .rn.f32x2); each lane is rounded exactly like the
@@ -235,21 +251,67 @@ template <> struct Lattice<HQ_A2> {
 };
 
 // E8 as 2E8 = 2D8 u (2D8 + 1) in Z^8: candidate A = 2 D8(v/2), candidate
-// B = 2 D8((v - 1)/2) + 1, keep B only if strictly nearer (sequential fma
-// distance, index order).  The two candidates run side by side in the two
-// halves of packed fp32 operations.  The symbols come straight from the D8
-// integers of the winner: coset bit c (0 for A, 1 for B), m_i = (q_i - c)/2 is
-// the D8 coordinate, and m_7's parity (implied by m_0..m_6) is stripped.
+// B = 2 D8((v - 1)/2) + 1, keep B only if strictly nearer by the sequential
+// fma distance in index order (the reading of the decoder).  The symbols come
+// straight from the D8 integers m of the winner: coset bit c (0 for A, 1 for B),
+// m_i = (q_i - c)/2, and m_7's parity (implied by m_0..m_6) is stripped.
+//
+// Exact decision, fast.  Both candidates' D8 points are found exactly as the
+// reading defines them (two candidates side by side in packed fp32 operations).
+// Only the distance comparison is estimated: with r = y - rint(y), a parity fix
+// moves the coordinate of largest |r| to residual 1 - |r|, so candidate X's
+// squared distance / 4 is S_X + p_X (1 - 2 max|r|) with S_X = sum r^2, in real
+// arithmetic (for B up to the rounding of v - 1).  Over both candidates the
+// estimates differ from the reading's fp32 sequential-fma distances / 4 by at most
+// 19.01u (E_A + E_B) + u sum|v| + 10u (u = 2^-24; terms: the reading's rounded
+// residuals and 8-step fma chain, 10.01u E each; this estimate's fma chain and two
+// roundings, 9u E + u each; the rounding of v - 1 in candidate B, u (sum|v| + 8)).
+// The margin below, 2^-18 (E_A + E_B + 4) + 2^-21 sum|v| = 64u (E_A + E_B) + 256u
+// + 8u sum|v|, is at least 3.3 times that bound.  Outside the margin the estimate
+// decides; inside it (near-ties, exact ties, huge inputs) the reading's own
+// distances are rebuilt from the same rounded values (exact_dist).
 template <> struct Lattice<HQ_E8> {
     static constexpr int N = 8;
     __device__ static __forceinline__ void point(const int32_t (&q)[8], float (&p)[8]) {
 #pragma unroll
         for (int i = 0; i < 8; i++) p[i] = (float)q[i];
     }
-    // D8 coordinates of both candidates after their parity fixes, and which wins.
-    __device__ static __forceinline__ bool decide(const float (&v)[8], float (&fa)[8], float (&fb)[8]) {
+    // Index of the largest |r_i| (first on ties) and r at that index.
+    __device__ static __forceinline__ int argmax_abs(const float (&r)[8], float &rb) {
+        rb = r[0];
+        int j = 0;
+#pragma unroll
+        for (int i = 1; i < 8; i++) {
+            const bool gt = fabsf(r[i]) > fabsf(rb);
+            rb = gt ? r[i] : rb;
+            j = gt ? i : j;
+        }
+        return j;
+    }
+    // The reading's sequential fma distance of one candidate, rebuilt from its rounded
+    // values (t = y + 1.5 * 2^23), residuals r and parity: the fixed D8 point f, the
+    // embedded point 2 f + c, then acc = fma(rho, rho, acc) in index order.
+    __device__ static __forceinline__ float exact_dist(const float (&v)[8], const uint32_t (&t)[8],
+                                                       const float (&r)[8], uint32_t par, float c) {
+        float rb;
+        const int j = argmax_abs(r, rb);
+        const float d = (par & 1u) ? ((rb >= 0.0f) ? 1.0f : -1.0f) : 0.0f;
+        float acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float f = __fadd_rn(__fsub_rn(__uint_as_float(t[i]), kRoundMagic), (i == j) ? d : 0.0f);
+            const float rho = __fsub_rn(v[i], __fmaf_rn(f, 2.0f, c));
+            acc = __fmaf_rn(rho, rho, acc);
+        }
+        return acc;
+    }
+    // D8 coordinates m of the nearest point (after the winner's parity fix); returns the coset bit.
+    __device__ static __forceinline__ uint32_t nearest_d8(const float (&v)[8], int32_t (&m)[8]) {
         const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
+        uint32_t ta[8], tb[8];
         float ra[8], rb[8];
+        float2 S = make_float2(0.0f, 0.0f);
+        float ma = 0.0f, mb = 0.0f, sv = 0.0f;
         uint32_t pa = 0, pb = 0;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
@@ -257,41 +319,52 @@ template <> struct Lattice<HQ_E8> {
             const float2 t = f2_add(y, M2);
             const float2 f = f2_sub(t, M2);
             const float2 r = f2_sub(y, f);
-            fa[i] = f.x;
-            fb[i] = f.y;
+            ta[i] = __float_as_uint(t.x);
+            tb[i] = __float_as_uint(t.y);
             ra[i] = r.x;
             rb[i] = r.y;
-            pa ^= __float_as_uint(t.x);
-            pb ^= __float_as_uint(t.y);
+            pa ^= ta[i];
+            pb ^= tb[i];
+            S = f2_fma(r, r, S);
+            ma = fmaxf(ma, fabsf(r.x));
+            mb = fmaxf(mb, fabsf(r.y));
+            sv = __fadd_rn(sv, fabsf(v[i]));
         }
-        dn_fix<8>(ra, pa, fa);
-        dn_fix<8>(rb, pb, fb);
-        float2 acc = make_float2(0.0f, 0.0f);
+        const float adja = (pa & 1u) ? __fmaf_rn(-2.0f, ma, 1.0f) : 0.0f;
+        const float adjb = (pb & 1u) ? __fmaf_rn(-2.0f, mb, 1.0f) : 0.0f;
+        const float2 E = f2_add(S, make_float2(adja, adjb));
+        const float diff = __fsub_rn(E.x, E.y);
+        const float margin =
+            __fmaf_rn(0x1p-21f, sv, __fmul_rn(0x1p-18f, __fadd_rn(__fadd_rn(E.x, E.y), 4.0f)));
+        bool odd = diff > 0.0f;
+        if (fabsf(diff) <= margin) odd = exact_dist(v, tb, rb, pb, 1.0f) < exact_dist(v, ta, ra, pa, 0.0f);
+        // the winner's parity fix: coordinate of largest |r| (first on ties) one step toward y
+        float rsel[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const float2 pt = f2_fma(make_float2(fa[i], fb[i]), make_float2(2.0f, 2.0f), make_float2(0.0f, 1.0f));
-            const float2 rho = f2_sub(make_float2(v[i], v[i]), pt);
-            acc = f2_fma(rho, rho, acc);
-        }
-        return acc.y < acc.x;
+        for (int i = 0; i < 8; i++) rsel[i] = odd ? rb[i] : ra[i];
+        float rw;
+        const int j = argmax_abs(rsel, rw);
+        const uint32_t pw = odd ? pb : pa;
+        const int32_t d = (pw & 1u) ? ((rw >= 0.0f) ? 1 : -1) : 0;
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+            m[i] = (int32_t)((odd ? tb[i] : ta[i]) - (uint32_t)kRoundMagicBits) + ((i == j) ? d : 0);
+        return odd ? 1u : 0u;
     }
     __device__ static __forceinline__ void nearest(const float (&v)[8], int32_t (&q)[8]) {
-        float fa[8], fb[8];
-        const bool odd = decide(v, fa, fb);
+        int32_t m[8];
+        const int32_t c = (int32_t)nearest_d8(v, m);
 #pragma unroll
-        for (int i = 0; i < 8; i++) q[i] = 2 * rint_int(odd ? fb[i] : fa[i]) + (odd ? 1 : 0);
+        for (int i = 0; i < 8; i++) q[i] = 2 * m[i] + c;
     }
     __device__ static __forceinline__ uint32_t symbols(const float (&v)[8], uint32_t (&z)[8]) {
-        float fa[8], fb[8];
-        const bool odd = decide(v, fa, fb);
         int32_t m[8];
-#pragma unroll
-        for (int i = 0; i < 8; i++) m[i] = rint_int(odd ? fb[i] : fa[i]);
+        const uint32_t c = nearest_d8(v, m);
         const int32_t s = m[0] + m[1] + m[2] + m[3] + m[4] + m[5] + m[6];
         m[7] = (m[7] - (s & 1)) >> 1;
 #pragma unroll
         for (int i = 0; i < 8; i++) z[i] = zigzag(m[i]);
-        return odd ? 1u : 0u;
+        return c;
     }
     __device__ static __forceinline__ float box(int) { return 4.0f; }
     __device__ static __forceinline__ void reinsert(const int32_t (&m)[8], uint32_t c, int32_t (&q)[8]) {

@@ -184,16 +184,17 @@ __device__ __forceinline__ void round_symbols(const EncodeArgs &a, const RoundIn
     using L = Lattice<LAT>;
     constexpr int N = L::N;
     const int q = lane & 3;
-    const uint32_t *sg = sign_tab + in.tcol * kSignStride + q * kSignQuarter;
+    const uint32_t es = sign_tab[in.tcol * kSignWords + q];
     float2 v[16];
 #pragma unroll
     for (int j = 0; j < 4; j++) {
         const uint4 w = in.valid ? raw[j] : make_uint4(0, 0, 0, 0);
-        const uint4 s = *reinterpret_cast<const uint4 *>(sg + 4 * j);
-        const uint32_t ww[4] = {w.x ^ s.x, w.y ^ s.y, w.z ^ s.z, w.w ^ s.w};
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int t = 0; t < 4; t++)
-            v[4 * j + t] = make_float2(__uint_as_float(ww[t] << 16), __uint_as_float(ww[t] & 0xFFFF0000u));
+        for (int t = 0; t < 4; t++) {
+            const uint32_t ww = wv[t] ^ sign_pair_mask(es, 4 * j + t);
+            v[4 * j + t] = make_float2(__uint_as_float(ww << 16), __uint_as_float(ww & 0xFFFF0000u));
+        }
     }
     fwht128_quarter(v, lane);
     const float2 c2 = make_float2(a.c_scale, a.c_scale);
@@ -401,20 +402,14 @@ __device__ __forceinline__ unsigned long long take_ticket(const EncodeArgs &a) {
 template <int LAT, bool DITHER, bool KSMALL>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t *sign_tab = smem;                                        // tcols * kSignStride
-    uint32_t *stage_all = smem + a.tcols * kSignStride;               // warps * 2 * kStageWords
+    uint32_t *sign_tab = smem;                                        // tcols * kSignWords
+    uint32_t *stage_all = smem + a.tcols * kSignWords;                // warps * 2 * kStageWords
     uint32_t *in_all = stage_all + kWarpsPerCta * 2 * kStageWords;    // warps * 32 * kInSlotWords
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t *stages = stage_all + warp * 2 * kStageWords;
     uint32_t *slot = in_all + (warp * 32 + lane) * kInSlotWords;
 
-    // Sign masks per bf16x2 pair: bit 15 flips the even column, bit 31 the odd one.
-    for (int i = threadIdx.x; i < a.tcols * 64; i += blockDim.x) {
-        const int tc = i >> 6, p = i & 63;
-        const unsigned long long col = (unsigned long long)tc * kTile + 2 * p;
-        sign_tab[tc * kSignStride + (p >> 4) * kSignQuarter + (p & 15)] =
-            (sign_bit(a.seed, col) << 15) | (sign_bit(a.seed, col + 1) << 31);
-    }
+    build_sign_table(sign_tab, a.tcols, a.seed);
     __syncthreads();
 
     const int k = a.k;
@@ -539,22 +534,16 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
 template <int LAT, bool DITHER>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     const size_t smem =
-        (size_t)(a.tcols * kSignStride + kWarpsPerCta * 2 * kStageWords + kWarpsPerCta * 32 * kInSlotWords) *
+        (size_t)(a.tcols * kSignWords + kWarpsPerCta * 2 * kStageWords + kWarpsPerCta * 32 * kInSlotWords) *
         sizeof(uint32_t);
-    auto kern = a.k <= 4 ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool small = a.k <= 4;
+    auto kern = small ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
+    static LaunchPlan plans[2];
+    unsigned grid = 0;
+    cudaError_t e = plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta,
+                                               grid);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarpsPerCta * 32, smem)) != cudaSuccess)
-        return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    unsigned long long want = (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta;
-    unsigned long long grid = (unsigned long long)sms * (unsigned long long)per_sm;
-    if (want < grid) grid = want;
-    if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, kWarpsPerCta * 32, smem, s>>>(a);
+    kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     return cudaGetLastError();
 }
 

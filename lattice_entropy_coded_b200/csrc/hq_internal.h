@@ -5,15 +5,15 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "hq.h"
 
 namespace hq {
 
 constexpr int kTile = 128;          // elements per RHT tile
 constexpr int kChunkTiles = 32;     // tiles per chunk = lanes per warp (one tile per lane)
-constexpr int kSignQuarter = 20;    // words per tile quarter in the shared sign table (16 used, padded so
-                                    // the 8 lanes of a 16-byte access phase hit distinct banks)
-constexpr int kSignStride = 4 * kSignQuarter;  // words per tile column in the sign table
+constexpr int kSignWords = 4;       // shared sign-table words per tile column (one per 32-column quarter)
 constexpr int kWarpsPerCta = 8;     // warps per CTA in both kernels
 constexpr int kStageWords = 1024;   // per-warp shared staging for one chunk's words (encode and decode);
                                     // larger chunks are written or read in place in global memory
@@ -75,6 +75,46 @@ struct DecodeArgs {
     uint64_t n_appends;
     hq_stats *stats;
     int tcols;
+};
+
+// Persistent-grid size of one kernel on the current device: SM count x resident CTAs per SM at
+// `smem` dynamic shared bytes, capped at `want` CTAs.  The shared-memory attribute and the
+// occupancy query run once per device and shared-memory size; later calls of the same kernel
+// (every KV append, every small matrix) reuse the cached answer.
+struct LaunchPlan {
+    static constexpr int kMaxDevices = 64;
+    std::mutex mu;
+    int sms[kMaxDevices] = {};
+    size_t configured[kMaxDevices] = {};   // dynamic shared bytes the attribute allows
+    size_t smem_key[kMaxDevices] = {};
+    int per_sm[kMaxDevices] = {};
+
+    template <typename K>
+    cudaError_t grid(K kern, int threads, size_t smem, unsigned long long want, unsigned &out) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        std::lock_guard<std::mutex> lk(mu);
+        if (!sms[dev] && (e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return e;
+        if (smem > configured[dev]) {
+            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+                return e;
+            configured[dev] = smem;
+        }
+        if (smem_key[dev] != smem || per_sm[dev] == 0) {
+            int n = 0;
+            if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem)) != cudaSuccess) return e;
+            if (n < 1) return cudaErrorInvalidConfiguration;
+            smem_key[dev] = smem;
+            per_sm[dev] = n;
+        }
+        unsigned long long g = (unsigned long long)sms[dev] * (unsigned long long)per_sm[dev];
+        if (want < g) g = want;
+        out = (unsigned)(g < 1 ? 1 : g);
+        return cudaSuccess;
+    }
 };
 
 // Launchers (defined in hq_encode.cu / hq_decode.cu).  Return cudaSuccess or the launch error.
