@@ -251,6 +251,25 @@ HQ_API int hq_device_check(void);
  * stays inside [0, cap_words). */
 HQ_API void hq_debug_set_spin_limit(uint32_t polls);
 
+/* Testing aid: which form of the quantize kernel runs.  0 (default) chooses by
+ * size: launches of at most 592 chunks (one wave of four-warp chunk groups on a
+ * B200) use the grouped form, where four warps share a chunk (lower latency);
+ * larger ones the per-warp form, where a warp encodes whole chunks (higher
+ * throughput).  1 forces per-warp, 2 forces grouped.  Both give identical
+ * streams, offsets and stats.  Process-wide; HQ_EINVAL outside 0..2. */
+HQ_API int hq_debug_set_encode_path(int path);
+
+/* Testing aid: the nearest point of the lattice in its integer embedding
+ * (the decoder the quantize kernels run; HyperQuant explainer pages,
+ * "Methodology" 2) for n_blocks vectors.
+ *   d_v : device, n_blocks x dim fp32 values (dim = 1, 2, 4, 8 for Z, A2, D4,
+ *         E8), 4-byte aligned, read only.
+ *   d_q : device, n_blocks x dim int32 codes out (E8: 2E8 = 2D8 u (2D8 + 1);
+ *         D4: sum even; A2: (a, b) with a = b mod 2; Z: the rounded value).
+ * Asynchronous on cuda_stream.  HQ_EINVAL for a bad lattice, a negative count
+ * or a null / misaligned pointer; HQ_ECUDA if the launch fails. */
+HQ_API int hq_debug_nearest(int lattice, const float *d_v, int64_t n_blocks, int32_t *d_q, void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -60,6 +60,8 @@ EXPORTS = {
                               C.c_uint64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "hq_dequantize": (C.c_int, [C.c_void_p, C.c_uint64, C.c_void_p, C.c_int64, C.c_int64, C.POINTER(hq_params),
                                 C.c_void_p, C.c_int, C.c_int64, C.c_void_p, C.c_void_p]),
+    "hq_debug_set_encode_path": (C.c_int, [C.c_int]),
+    "hq_debug_nearest": (C.c_int, [C.c_int, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p]),
     "hq_kv_init": (C.c_int, [C.POINTER(hq_kv_cache), C.c_int32, C.c_int32, C.POINTER(hq_params), C.c_void_p,
                              C.c_uint64, C.c_void_p, C.c_uint64, C.c_void_p, C.c_uint64, C.c_void_p, C.c_void_p,
                              C.c_void_p]),
@@ -130,6 +132,19 @@ def hq_device_check() -> int:
 
 def hq_debug_set_spin_limit(polls: int) -> None:
     _lib.hq_debug_set_spin_limit(int(polls))
+
+
+def hq_debug_set_encode_path(path: int) -> int:
+    """0 = by size, 1 = per-warp encoder, 2 = grouped encoder (testing aid)."""
+    return _check(_lib.hq_debug_set_encode_path(int(path)), "hq_debug_set_encode_path")
+
+
+def hq_debug_nearest(lattice, v: torch.Tensor, q: torch.Tensor, cuda_stream=None) -> int:
+    """v: fp32 [n, dim] on the device; q: int32 [n, dim] (codes out)."""
+    lat = LATTICES[lattice] if isinstance(lattice, str) else int(lattice)
+    assert v.dtype == torch.float32 and q.dtype == torch.int32 and v.is_contiguous() and q.is_contiguous()
+    assert v.shape == q.shape and v.dim() == 2
+    return _check(_lib.hq_debug_nearest(lat, _ptr(v), v.shape[0], _ptr(q), _stream(cuda_stream)), "hq_debug_nearest")
 
 
 def hq_stream_bound(rows: int, cols: int, params: hq_params, max_abs_symbol: int = 0):

@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libhq.so")
-SOURCES = ["hq_api.cu", "hq_encode.cu", "hq_decode.cu", "hq_static.cu"]
+SOURCES = ["hq_api.cu", "hq_encode.cu", "hq_decode.cu", "hq_static.cu", "hq_debug.cu"]
 HEADERS = ["hq_internal.h", "hq_device.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -10,6 +10,10 @@
 
 using namespace hq;
 
+namespace hq {
+int g_encode_path = 0;
+}
+
 namespace {
 
 constexpr int64_t kMaxCols = 65536;  // the shared sign table holds cols / 128 columns
@@ -305,5 +309,11 @@ int hq_device_check(void) {
 }
 
 void hq_debug_set_spin_limit(uint32_t polls) { g_spin_limit = polls ? polls : kSpinLimit; }
+
+int hq_debug_set_encode_path(int path) {
+    if (path < 0 || path > 2) return HQ_EINVAL;
+    hq::g_encode_path = path;
+    return HQ_OK;
+}
 
 }  // extern "C"

@@ -52,20 +52,30 @@ __device__ __forceinline__ void lookback_publish(unsigned long long *lb, unsigne
     if ((threadIdx.x & 31) == 0) st_relaxed_u64(lb + c, (c == 0 ? kFlagInc : kFlagAgg) | agg);
 }
 
+// The look-back word of predecessor c - 1 - lane (INC with value 0 before chunk 0):
+// the first window of a resolve, loaded early so its latency overlaps other work.
+__device__ __forceinline__ unsigned long long lookback_peek(const unsigned long long *lb, unsigned long long c) {
+    const long long idx = (long long)c - 1 - (threadIdx.x & 31);
+    return (idx >= 0) ? ld_relaxed_u64(lb + idx) : kFlagInc;
+}
+
 // Exclusive prefix (in words) of chunk c: walk back over predecessors 32 at a
 // time until one with an inclusive prefix, summing counts; then publish c's
-// inclusive prefix.  Whole warp calls it.  Bounded: gives up after spin_limit polls.
+// inclusive prefix.  `first` is lookback_peek(lb, c), taken earlier.  Whole warp
+// calls it.  Bounded: gives up after spin_limit polls.
 __device__ __noinline__ unsigned long long lookback_resolve(unsigned long long *lb, unsigned long long c,
                                                             unsigned long long agg, uint32_t spin_limit,
-                                                            bool &timed_out) {
+                                                            bool &timed_out, unsigned long long first) {
     const int lane = threadIdx.x & 31;
     if (c == 0) return 0;
     unsigned long long excl = 0;
     long long pos = (long long)c - 1;
     uint32_t spins = 0;
+    bool use_first = true;
     while (true) {
         const long long idx = pos - lane;
-        const unsigned long long v = (idx >= 0) ? ld_relaxed_u64(lb + idx) : kFlagInc;
+        const unsigned long long v = use_first ? first : (idx >= 0) ? ld_relaxed_u64(lb + idx) : kFlagInc;
+        use_first = false;
         const unsigned flag = (unsigned)(v >> 62);
         const unsigned inc = __ballot_sync(0xffffffffu, flag == 2u);
         const unsigned zero = __ballot_sync(0xffffffffu, flag == 0u);
@@ -148,7 +158,8 @@ struct RoundInput {
     unsigned long long e0;
 };
 
-constexpr int kInSlotWords = 20;
+constexpr int kInSlotWords = 20;     // per-lane input slot of the per-warp kernel (80 B)
+constexpr int kGroupSlotWords = 36;  // grouped kernel: the slot also parks the 32 symbols (144 B)
 
 __device__ __forceinline__ void prefetch_round(const EncodeArgs &a, const ChunkGeo &geo, int r, int lane,
                                                uint32_t *slot) {
@@ -220,7 +231,7 @@ __device__ __forceinline__ void round_symbols(const EncodeArgs &a, const RoundIn
         uint32_t zz[N];
         cbits |= L::symbols(blk, zz) << b;
 #pragma unroll
-        for (int i = 0; i < N; i++) z[b * N + i] = in.valid ? zz[i] : 0u;
+        for (int i = 0; i < N; i++) z[b * N + i] = (!DITHER || in.valid) ? zz[i] : 0u;
     }
     if (!in.valid) cbits = 0;
 }
@@ -356,11 +367,12 @@ struct Pending {
 };
 
 template <int LAT, bool DITHER>
-__device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending &p, uint32_t *stage,
-                                             const uint32_t *sign_tab, unsigned long long base, uint32_t &status) {
+__device__ __forceinline__ void finish_chunk_warp(const EncodeArgs &a, const Pending &p, uint32_t *stage,
+                                                  const uint32_t *sign_tab, unsigned long long base, uint32_t &status) {
     const int lane = threadIdx.x & 31;
     bool to = false;
-    const unsigned long long excl = lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to);
+    const unsigned long long excl =
+        lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to, lookback_peek(a.lookback, p.c));
     if (to) status |= HQ_ST_TIMEOUT;
     const unsigned long long start = base + excl;
     if (lane == 0) {
@@ -399,6 +411,8 @@ __device__ __forceinline__ unsigned long long take_ticket(const EncodeArgs &a) {
     return __shfl_sync(0xffffffffu, c, 0);
 }
 
+// Throughput form: persistent CTAs of kWarpsPerCta warps, each warp encoding whole
+// chunks (4 rounds of 8 tiles) taken by ticket, with a two-chunk stage pipeline.
 template <int LAT, bool DITHER, bool KSMALL>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
@@ -508,7 +522,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         lookback_publish(a.lookback, c, total);
 
         // the previous chunk's predecessors have had a whole chunk's time to publish
-        if (have_pend) finish_chunk<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
+        if (have_pend) finish_chunk_warp<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
         pend.c = c;
         pend.total = total;
         pend.overflow = overflow;
@@ -517,7 +531,241 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         c = cn;
         buf ^= 1;
     }
-    if (have_pend) finish_chunk<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
+    if (have_pend) finish_chunk_warp<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+    if (a.stats) {
+        zor_all = __reduce_or_sync(0xffffffffu, zor_all);
+        status = __reduce_or_sync(0xffffffffu, status);
+        if (lane == 0) {
+            if (status) atomicOr(&a.stats->status, status);
+            if (zor_all) atomicOr(&a.stats->max_symbol, zor_all);
+            if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
+        }
+    }
+}
+
+// Four warps share a chunk: warp w of a group encodes round w (tiles 8w..8w+7).
+constexpr int kGroupWarps = kChunkTiles / kTilesPerRound;
+constexpr int kGroups = kWarpsPerCta / kGroupWarps;
+static_assert(kGroups * kGroupWarps == kWarpsPerCta, "whole groups per CTA");
+
+// Per-group control words in shared memory, double-buffered by iteration parity.
+struct GroupCtl {
+    uint32_t tot[2][kGroupWarps];   // unary bits of each warp's round
+    uint32_t bad[2][kGroupWarps];   // nonzero: that round is outside the supported range
+    unsigned int tk[2];             // ticket taken during the iteration (the chunk after next)
+    unsigned int first[2];          // the group's first two tickets
+};
+static_assert(sizeof(GroupCtl) % 16 == 0, "keeps the input slots 16-byte aligned");
+
+__device__ __forceinline__ void group_sync(int g) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(kGroupWarps * 32) : "memory");
+}
+
+// Resolve a pending chunk's offset and write it out (one warp).  The stage words
+// are zeroed as they are copied, so the stage is clean for its next chunk.
+template <int LAT, bool DITHER>
+__device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending &p, uint32_t *stage,
+                                             const uint32_t *sign_tab, unsigned long long base, uint32_t &status,
+                                             unsigned long long first) {
+    const int lane = threadIdx.x & 31;
+    bool to = false;
+    const unsigned long long excl = lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to, first);
+    if (to) status |= HQ_ST_TIMEOUT;
+    const unsigned long long start = base + excl;
+    if (lane == 0) {
+        a.offsets[a.chunk_base + p.c] = start;
+        if (p.c + 1 == a.n_chunks) {
+            const unsigned long long end = start + p.total;
+            a.offsets[a.chunk_base + a.n_chunks] = end;
+            if (a.tail_out) *a.tail_out = end;
+            if (a.stats) a.stats->stream_words = end;
+            if (end > a.cap_words) status |= HQ_ST_CAPACITY;
+        }
+        if (p.c == 0 && a.row) *a.row = a.row_val;
+    }
+    if (!p.range_bad && !p.overflow) {
+        for (uint32_t i = lane; i < (uint32_t)p.total; i += 32) {
+            const uint32_t v = stage[i];
+            stage[i] = 0u;
+            if (start + i < a.cap_words) a.stream[start + i] = v;
+        }
+    } else if (!p.range_bad) {
+        uint32_t *g = a.stream + start;
+        const unsigned long long room = (start < a.cap_words) ? a.cap_words - start : 0ull;
+        for (unsigned long long i = lane; i < p.total; i += 32)
+            if (i < room) g[i] = 0u;
+        __syncwarp();
+        __threadfence_block();
+        ChunkGeo geo;
+        geo.init(a.map, p.c);
+        const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * geo.ntiles + 31) / 32u : 0u;
+        const uint32_t nr = 4u * (uint32_t)a.k * (uint32_t)geo.ntiles;
+        encode_chunk_global<LAT, DITHER>(a, geo, sign_tab, g, room, nc, nr);
+    }
+    __syncwarp();
+}
+
+// Latency form, for launches that fit in one wave of groups (a KV append, a small
+// matrix): persistent CTAs of kGroups groups.  A group takes chunk tickets in increasing
+// order (so a chunk's predecessors are always already running) and per chunk:
+// each warp encodes its round; the four round totals meet in shared memory
+// (group barrier); each warp places its codewords in the group's stage; warp 0
+// publishes the chunk's word count; and one warp, in turn, resolves the previous
+// chunk's offset and copies that chunk's stage out.
+template <int LAT, bool DITHER, bool KSMALL>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel_grouped(const EncodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gi = warp / kGroupWarps, w = warp % kGroupWarps;
+    uint32_t *sign_tab = smem;                                              // tcols * kSignWords
+    uint32_t *stage_all = sign_tab + a.tcols * kSignWords;                  // groups * 2 * kStageWords
+    GroupCtl *ctl_all = reinterpret_cast<GroupCtl *>(stage_all + kGroups * 2 * kStageWords);
+    uint32_t *in_all = reinterpret_cast<uint32_t *>(ctl_all + kGroups);    // warps * 32 * kGroupSlotWords
+    uint32_t *stages = stage_all + gi * 2 * kStageWords;
+    GroupCtl &ctl = ctl_all[gi];
+    uint32_t *slot = in_all + (warp * 32 + lane) * kGroupSlotWords;
+
+    build_sign_table(sign_tab, a.tcols, a.seed);
+    for (int i = threadIdx.x; i < kGroups * 2 * kStageWords / 4; i += blockDim.x)
+        reinterpret_cast<uint4 *>(stage_all)[i] = make_uint4(0, 0, 0, 0);
+    if (w == 0 && lane == 0) {
+        ctl.first[0] = atomicAdd(a.ticket, 1u);
+        ctl.first[1] = atomicAdd(a.ticket, 1u);
+    }
+    __syncthreads();
+
+    const unsigned long long n = a.n_chunks;
+    const int k = a.k;
+    const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
+    uint32_t status = 0, zor_all = 0;
+    unsigned long long payload = 0;
+    unsigned long long c = ctl.first[0], cn = ctl.first[1];
+    if (c < n) {
+        ChunkGeo g0;
+        g0.init(a.map, c);
+        prefetch_round(a, g0, w, lane, slot);
+    }
+    Pending pend = {0, 0, false, false};
+    bool have_pend = false;
+    int buf = 0;
+    unsigned it = 0;
+    while (true) {
+        const bool live = c < n;
+        const bool duty = w == (int)(it & (kGroupWarps - 1));   // this warp finishes the previous chunk
+        unsigned long long first = 0;
+        if (!live && have_pend && duty) first = lookback_peek(a.lookback, pend.c);
+        uint32_t *stage = stages + buf * kStageWords;
+        ChunkGeo geo;
+        uint32_t z[32], cbits = 0, ub = 0, incl = 0;
+        bool valid = false;
+        if (live) {
+            geo.init(a.map, c);
+            RoundInput cur;
+            round_input(a, geo, w, lane, cur);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            uint4 raw[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++) raw[j] = *reinterpret_cast<const uint4 *>(slot + 4 * j);
+            if (w == 0 && lane == 0) ctl.tk[buf] = atomicAdd(a.ticket, 1u);
+            if (have_pend && duty) first = lookback_peek(a.lookback, pend.c);
+            round_symbols<LAT, DITHER>(a, cur, raw, lane, sign_tab, z, cbits);
+            valid = cur.valid;
+            // the symbols wait in the lane's slot while the group meets
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                reinterpret_cast<uint4 *>(slot)[j] = make_uint4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
+            uint32_t usum = 0, lor = 0;
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                usum += z[i] >> k;
+                lor |= z[i];
+            }
+            zor_all |= lor;
+            ub = valid ? usum + 32u : 0u;
+            incl = ub;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            // symbols below 2^22 keep ub below 2^28; the coarse sum says whether the
+            // round's total could reach 2^31 bits (and the 32-bit scan wrap)
+            const uint32_t coarse = __reduce_add_sync(0xffffffffu, ub >> 8);
+            const uint32_t rzor = __reduce_or_sync(0xffffffffu, lor);
+            if (lane == 31) {
+                ctl.tot[buf][w] = incl;
+                ctl.bad[buf][w] = ((rzor >> 22) != 0u || coarse >= (1u << 23)) ? 1u : 0u;
+            }
+        }
+        group_sync(gi);
+        unsigned long long total = 0;
+        bool overflow = false, range_bad = false;
+        if (live) {
+            unsigned long long before = 0, U = 0;
+            uint32_t badw = 0;
+#pragma unroll
+            for (int j = 0; j < kGroupWarps; j++) {
+                const uint32_t t = ctl.tot[buf][j];
+                before += (j < w) ? t : 0u;
+                U += t;
+                badw |= ctl.bad[buf][j];
+            }
+            const int ntiles = geo.ntiles;
+            const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
+            const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
+            range_bad = badw != 0u || U >= kMaxUnaryBits;
+            total = nc + nr + (U + 31) / 32;
+            overflow = total > (unsigned long long)kStageWords;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const uint4 t = reinterpret_cast<const uint4 *>(slot)[j];
+                z[4 * j] = t.x;
+                z[4 * j + 1] = t.y;
+                z[4 * j + 2] = t.z;
+                z[4 * j + 3] = t.w;
+            }
+            if (cn < n) {
+                ChunkGeo gn;
+                gn.init(a.map, cn);
+                prefetch_round(a, gn, w, lane, slot);
+            }
+            if (!overflow && !range_bad) {
+                put_rem<KSMALL>(stage + nc + (uint32_t)(32 * w + lane) * (uint32_t)k, z, k, valid);
+                if (valid) {
+                    if (LAT == HQ_E8 && cbits) atomicOr(stage + 4 * w + (lane >> 3), cbits << (4 * (lane & 7)));
+                    uint32_t *un = stage + nc + nr;
+                    uint32_t pos = (uint32_t)before + incl - ub;
+#pragma unroll
+                    for (int gq = 0; gq < 4; gq++) {
+                        uint32_t qg[8];
+#pragma unroll
+                        for (int i = 0; i < 8; i++) qg[i] = z[8 * gq + i] >> k;
+                        pos += unary_group_shared(un, pos, qg);
+                    }
+                }
+            }
+            if (w == 0) {
+                lookback_publish(a.lookback, c, total);
+                if (range_bad) status |= HQ_ST_RANGE;
+                if (lane == 0) payload += U + (unsigned long long)nr * 32 + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
+            }
+        }
+        // the previous chunk: its predecessors have had a whole chunk's time to publish
+        if (have_pend && duty)
+            finish_chunk<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status, first);
+        if (!live) break;
+        pend.c = c;
+        pend.total = total;
+        pend.overflow = overflow;
+        pend.range_bad = range_bad;
+        have_pend = true;
+        c = cn;
+        cn = ctl.tk[buf];
+        buf ^= 1;
+        it++;
+    }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 
     if (a.stats) {
@@ -533,17 +781,34 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
 
 template <int LAT, bool DITHER>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
-    const size_t smem =
-        (size_t)(a.tcols * kSignWords + kWarpsPerCta * 2 * kStageWords + kWarpsPerCta * 32 * kInSlotWords) *
-        sizeof(uint32_t);
     const bool small = a.k <= 4;
-    auto kern = small ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
-    static LaunchPlan plans[2];
+    cudaError_t e;
     unsigned grid = 0;
-    cudaError_t e = plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta,
-                                               grid);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
+    // the grouped kernel when every chunk gets a group of its own in one wave
+    // (148 SMs x 2 CTAs x kGroups on a B200), else the per-warp kernel
+    int mode = g_encode_path;
+    if (mode == 0) mode = (a.n_chunks <= 592ull) ? 2 : 1;
+    if (mode == 2) {
+        const size_t smem = (size_t)(a.tcols * kSignWords + kGroups * 2 * kStageWords +
+                                     kWarpsPerCta * 32 * kGroupSlotWords) * sizeof(uint32_t) +
+                            kGroups * sizeof(GroupCtl);
+        auto kern = small ? encode_kernel_grouped<LAT, DITHER, true> : encode_kernel_grouped<LAT, DITHER, false>;
+        static LaunchPlan plans[2];
+        if ((e = plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kGroups - 1) / kGroups, grid)) !=
+            cudaSuccess)
+            return e;
+        kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
+    } else {
+        const size_t smem =
+            (size_t)(a.tcols * kSignWords + kWarpsPerCta * 2 * kStageWords + kWarpsPerCta * 32 * kInSlotWords) *
+            sizeof(uint32_t);
+        auto kern = small ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
+        static LaunchPlan plans[2];
+        if ((e = plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta,
+                                           grid)) != cudaSuccess)
+            return e;
+        kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
+    }
     return cudaGetLastError();
 }
 

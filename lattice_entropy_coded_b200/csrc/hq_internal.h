@@ -117,6 +117,11 @@ struct LaunchPlan {
     }
 };
 
+// Encoder form: 0 = by size (grouped for launches of at most one wave of chunk
+// groups, per-warp otherwise), 1 = per-warp, 2 = grouped.  Set by
+// hq_debug_set_encode_path (hq_api.cu); both forms give identical streams.
+extern int g_encode_path;
+
 // Launchers (defined in hq_encode.cu / hq_decode.cu).  Return cudaSuccess or the launch error.
 cudaError_t launch_encode(int lattice, int dither, const EncodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode(int lattice, int dither, const DecodeArgs &a, cudaStream_t s);

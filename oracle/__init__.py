@@ -95,6 +95,7 @@ def _bind(L):
         "hqref_scale_inv": (_f32, [_f32]),
         "hqref_lattice_dim": (_i32, [_i32]),
         "hqref_decode": (None, [_i32, _p, _p]),
+        "hqref_decode_many": (None, [_i32, _p, C.c_int64, _p]),
         "hqref_point": (None, [_i32, _p, _p]),
         "hqref_is_member": (_i32, [_i32, _p]),
         "hqref_dither_uniform": (_f32, [_u64, _u64]),
@@ -178,6 +179,15 @@ def decode(lat: int, v) -> np.ndarray:
     assert a.shape == (DIM[lat],)
     q = np.zeros(DIM[lat], dtype=np.int32)
     lib().hqref_decode(lat, _ptr(a), _ptr(q))
+    return q
+
+
+def decode_many(lat: int, v) -> np.ndarray:
+    """hqref_decode on every row of v [n, dim]."""
+    a = np.ascontiguousarray(v, dtype=np.float32)
+    assert a.ndim == 2 and a.shape[1] == DIM[lat]
+    q = np.zeros(a.shape, dtype=np.int32)
+    lib().hqref_decode_many(lat, _ptr(a), a.shape[0], _ptr(q))
     return q
 
 

@@ -219,6 +219,14 @@ void hqref_decode(int lat, const float *v, int32_t *q)
     }
 }
 
+/* hqref_decode on n consecutive blocks (a plain loop; used by tests that decode
+ * many vectors at once). */
+void hqref_decode_many(int lat, const float *v, int64_t n, int32_t *q)
+{
+    const int d = hqref_lattice_dim(lat);
+    for (int64_t b = 0; b < n; b++) hqref_decode(lat, v + b * d, q + b * d);
+}
+
 /* Membership predicate of the integer embeddings (used by tests). */
 int hqref_is_member(int lat, const int32_t *q)
 {

@@ -25,6 +25,7 @@ void hqref_decode_d4(const float *v, int32_t *q);
 void hqref_decode_z(const float *v, int32_t *q);
 void hqref_decode_a2(const float *u, int32_t *q);
 void hqref_decode(int lat, const float *v, int32_t *q);
+void hqref_decode_many(int lat, const float *v, int64_t n, int32_t *q);
 void hqref_point(int lat, const int32_t *q, float *p);
 int hqref_is_member(int lat, const int32_t *q);
 

@@ -101,6 +101,14 @@ def test_entry_points_validate_before_touching_the_device():
     assert lib.hq_kv_append(C.byref(cache), None, 16, 128, 2048, C.c_float(1.0), None, 0, None) == hq.HQ_EINVAL
     assert lib.hq_kv_read(C.byref(cache), None, 0, 1, 128, 2048, None) == hq.HQ_EINVAL
     assert hq.hq_status_string(hq.HQ_ST_TIMEOUT) == "look-back timed out"
+    # testing aids: encoder form switch and the nearest-point entry point
+    assert lib.hq_debug_set_encode_path(3) == hq.HQ_EINVAL
+    assert lib.hq_debug_set_encode_path(-1) == hq.HQ_EINVAL
+    assert lib.hq_debug_set_encode_path(0) == hq.HQ_OK
+    assert lib.hq_debug_nearest(4, None, 1, None, None) == hq.HQ_EINVAL
+    assert lib.hq_debug_nearest(3, None, -1, None, None) == hq.HQ_EINVAL
+    assert lib.hq_debug_nearest(3, None, 0, None, None) == hq.HQ_OK
+    assert lib.hq_debug_nearest(3, None, 5, None, None) == hq.HQ_EINVAL
 
 
 def test_binding_fails_loudly_without_the_library(tmp_path):

@@ -1,0 +1,75 @@
+"""Both forms of the quantize kernel against the oracle.
+
+The encoder has a per-warp form (a warp encodes whole chunks; used for large
+launches) and a grouped form (four warps share a chunk; used for launches of at
+most one wave of groups, such as a KV append).  By default the size decides;
+here each form is forced in turn on the cases that exercise its control flow:
+ragged last chunks, every Rice parameter, strided rows, exact ties, chunks too
+large for the shared stage, capacity overflow, bounded look-back waits, KV
+appends, and a 4096 x 4096 matrix (many chunks per group or warp).
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+import synth
+import test_gpu_parity as P
+from hqtest import assert_same_words, gpu_quantize, oracle_quantize, rate_points
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(params=[1, 2], ids=["per_warp", "grouped"])
+def path(request):
+    import lattice_entropy_coded_b200 as hq
+    hq.hq_debug_set_encode_path(request.param)
+    yield request.param
+    hq.hq_debug_set_encode_path(0)
+
+
+@pytest.mark.parametrize("lat", ["E8", "D4", "A2", "Z"])
+@pytest.mark.parametrize("dither", [0, 1])
+def test_small_matrices(path, lat, dither):
+    P.test_weights_bit_exact_small(lat, dither, (37, 384))
+    P.test_weights_bit_exact_small(lat, dither, (64, 4096))
+
+
+@pytest.mark.parametrize("k", [0, 3, 8, 15])
+def test_rice_parameters(path, k):
+    P.test_every_rice_parameter(k)
+
+
+def test_strided_ties_zero(path):
+    P.test_strided_rows()
+    P.test_all_zero_and_tiny_alpha()
+    P.test_ties_and_structured_inputs()
+
+
+def test_stage_overflow_slow_path(path):
+    P.test_large_symbols_take_the_slow_path_with_the_same_bits()
+
+
+def test_capacity_and_timeouts(path):
+    P.test_capacity_overflow_is_flagged_and_bounded()
+    P.test_lookback_spin_limit_never_hangs()
+    P.test_empty_matrix()
+
+
+@pytest.mark.parametrize("lat", ["E8", "Z"])
+def test_kv_appends(path, lat):
+    P.test_kv_appends_bit_exact(lat)
+
+
+def test_many_chunks_per_worker(path):
+    """4096 x 4096 (4096 chunks): every group or warp encodes several chunks in turn."""
+    import lattice_entropy_coded_b200 as hq
+    x = synth.weight(4096, 4096, seed=1)
+    p = [q for q in rate_points()["weight_4096x4096_rate_sweep"]["points"]
+         if q["lattice"] == "E8" and q["bps"] == 4.0][0]
+    params = hq.make_params(O.E8, p["alpha"], p["k"], 1, 0)
+    g = gpu_quantize(x.cuda(), params)
+    ref_w, ref_off, ref_pay = oracle_quantize(x, O.E8, p["alpha"], p["k"], 1)
+    assert g["stats"]["status"] == 0
+    assert_same_words(g["words"], g["offsets"], ref_w, ref_off)
+    assert g["stats"]["payload_bits"] == ref_pay
+    assert np.uint64(g["stats"]["stream_words"]) == ref_off[-1]
