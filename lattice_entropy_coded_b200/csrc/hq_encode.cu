@@ -236,6 +236,101 @@ __device__ __forceinline__ void round_symbols(const EncodeArgs &a, const RoundIn
     if (!in.valid) cbits = 0;
 }
 
+// N consecutive floats of a lane's shared row (16-byte aligned rows; offsets are
+// multiples of N words).
+template <int N>
+__device__ __forceinline__ void row_load(const uint32_t *r, float (&x)[N]) {
+    if (N == 8) {
+        const float4 a = reinterpret_cast<const float4 *>(r)[0], b = reinterpret_cast<const float4 *>(r)[1];
+        const float t[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < N; i++) x[i] = t[i];
+    } else if (N == 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(r);
+        const float t[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int i = 0; i < N; i++) x[i] = t[i];
+    } else if (N == 2) {
+        const float2 a = *reinterpret_cast<const float2 *>(r);
+        x[0] = a.x;
+        x[N - 1] = a.y;
+    } else {
+        x[0] = __uint_as_float(r[0]);
+    }
+}
+template <int N>
+__device__ __forceinline__ void row_store(uint32_t *r, const uint32_t (&z)[N]) {
+    if (N == 8) {
+        reinterpret_cast<uint4 *>(r)[0] = make_uint4(z[0], z[1 % N], z[2 % N], z[3 % N]);
+        reinterpret_cast<uint4 *>(r)[1] = make_uint4(z[4 % N], z[5 % N], z[6 % N], z[7 % N]);
+    } else if (N == 4) {
+        *reinterpret_cast<uint4 *>(r) = make_uint4(z[0], z[1 % N], z[2 % N], z[3 % N]);
+    } else if (N == 2) {
+        *reinterpret_cast<uint2 *>(r) = make_uint2(z[0], z[N - 1]);
+    } else {
+        r[0] = z[0];
+    }
+}
+
+// The same round with the lattice-block loop rolled over a lane-private shared row
+// (the 32 transformed values, then their symbols in place): one copy of the block
+// code instead of 32/N.  For the latency form, where each warp runs a round once
+// and fetching the unrolled code from a cold instruction cache, not issue, bounds
+// it.  Leaves the 32 symbols in row[0, 32) and their quotient sum and OR.
+template <int LAT, bool DITHER>
+__device__ __forceinline__ void round_symbols_rolled(const EncodeArgs &a, const RoundInput &in, const uint4 (&raw)[4],
+                                                     int lane, const uint32_t *sign_tab, uint32_t *row,
+                                                     uint32_t &cbits, uint32_t &usum, uint32_t &lor) {
+    using L = Lattice<LAT>;
+    constexpr int N = L::N;
+    const int q = lane & 3;
+    const uint32_t es = sign_tab[in.tcol * kSignWords + q];
+    float2 v[16];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const uint4 w = in.valid ? raw[j] : make_uint4(0, 0, 0, 0);
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int t = 0; t < 4; t++) {
+            const uint32_t ww = wv[t] ^ sign_pair_mask(es, 4 * j + t);
+            v[4 * j + t] = make_float2(__uint_as_float(ww << 16), __uint_as_float(ww & 0xFFFF0000u));
+        }
+    }
+    fwht128_quarter(v, lane);
+    const float2 c2 = make_float2(a.c_scale, a.c_scale);
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const float2 lo = f2_mul(v[2 * j], c2), hi = f2_mul(v[2 * j + 1], c2);
+        reinterpret_cast<float4 *>(row)[j] = make_float4(lo.x, lo.y, hi.x, hi.y);
+    }
+    cbits = 0;
+    usum = 0;
+    lor = 0;
+    const int k = a.k;
+    const unsigned long long eq = in.e0 + 32ull * q;
+#pragma unroll 1
+    for (int b = 0; b < 32 / N; b++) {
+        float blk[N];
+        row_load<N>(row + b * N, blk);
+        if (DITHER) {
+            float d[N];
+            dither_block<LAT>(a.seed, eq + (unsigned long long)(b * N), d);
+#pragma unroll
+            for (int i = 0; i < N; i++) blk[i] = __fadd_rn(blk[i], d[i]);
+        }
+        uint32_t zz[N];
+        cbits |= L::symbols(blk, zz) << b;
+#pragma unroll
+        for (int i = 0; i < N; i++) {
+            zz[i] = (!DITHER || in.valid) ? zz[i] : 0u;
+            usum += zz[i] >> k;
+            lor |= zz[i];
+        }
+        row_store<N>(row + b * N, zz);
+    }
+    if (!in.valid) cbits = 0;
+}
+
 // Remainder bits of 32 symbols (warp-uniform k) into the lane's k words.
 // KSMALL (k <= 4): a group of 8 remainders is built in one register, last
 // symbol first, two operations per symbol; otherwise a 64-bit accumulator.
@@ -670,18 +765,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel_grouped(co
             for (int j = 0; j < 4; j++) raw[j] = *reinterpret_cast<const uint4 *>(slot + 4 * j);
             if (w == 0 && lane == 0) ctl.tk[buf] = atomicAdd(a.ticket, 1u);
             if (have_pend && duty) first = lookback_peek(a.lookback, pend.c);
-            round_symbols<LAT, DITHER>(a, cur, raw, lane, sign_tab, z, cbits);
+            // the symbols are left in the lane's slot, where they wait while the group meets
+            uint32_t usum, lor;
+            round_symbols_rolled<LAT, DITHER>(a, cur, raw, lane, sign_tab, slot, cbits, usum, lor);
             valid = cur.valid;
-            // the symbols wait in the lane's slot while the group meets
-#pragma unroll
-            for (int j = 0; j < 8; j++)
-                reinterpret_cast<uint4 *>(slot)[j] = make_uint4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
-            uint32_t usum = 0, lor = 0;
-#pragma unroll
-            for (int i = 0; i < 32; i++) {
-                usum += z[i] >> k;
-                lor |= z[i];
-            }
             zor_all |= lor;
             ub = valid ? usum + 32u : 0u;
             incl = ub;
