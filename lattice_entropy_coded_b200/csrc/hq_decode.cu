@@ -274,6 +274,7 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
     const int q = lane & 3;
     const uint32_t *un = src + nc + nr;
     const float2 e2 = make_float2(geo.e_scale, geo.e_scale);
+    const uint32_t pk = 1u << k;   // quotient weight 2^k
     bool bad = false;
     const int nrounds = (geo.ntiles + kTilesPerRound - 1) / kTilesPerRound;
 #pragma unroll 1
@@ -301,11 +302,19 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
 #pragma unroll
                 for (int bb = 0; bb < 8 / N; bb++) {
                     const int b = g * (8 / N) + bb;
-                    int32_t m[N], qq[N];
+                    int32_t qq[N];
                     float p[N];
+                    if constexpr (LAT == HQ_E8) {
+                        uint32_t zb[8];
 #pragma unroll
-                    for (int i = 0; i < N; i++) m[i] = unzigzag((qv[bb * N + i] << k) | rv[bb * N + i]);
-                    L::reinsert(m, (coset >> b) & 1u, qq);
+                        for (int i = 0; i < 8; i++) zb[i] = imad(qv[bb * N + i], pk, rv[bb * N + i]);
+                        e8_codes_from_symbols(zb, (coset >> b) & 1u, qq);
+                    } else {
+                        int32_t m[N];
+#pragma unroll
+                        for (int i = 0; i < N; i++) m[i] = unzigzag(imad(qv[bb * N + i], pk, rv[bb * N + i]));
+                        L::reinsert(m, (coset >> b) & 1u, qq);
+                    }
                     L::point(qq, p);
                     if (DITHER) {
                         float d[N];
@@ -361,8 +370,10 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
     return bad;
 }
 
+// Three CTAs (24 warps) per SM without dither, where the decoder fits 80 registers with
+// almost no spills; two with dither, whose second lattice search needs more.
 template <int LAT, bool DITHER, bool KV, bool KSMALL>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kWarpsPerCta * 32, DITHER ? 2 : 3) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int kStageSlot = kStageWords + kStagePad;
     uint32_t *sign_tab = smem;

@@ -380,6 +380,30 @@ template <> struct Lattice<HQ_E8> {
 __device__ __forceinline__ uint32_t zigzag(int32_t m) { return ((uint32_t)m << 1) ^ (uint32_t)(m >> 31); }
 __device__ __forceinline__ int32_t unzigzag(uint32_t z) { return (int32_t)(z >> 1) ^ -(int32_t)(z & 1u); }
 
+// a * b + c in one integer multiply-add (b a runtime power of two: a Rice quotient
+// shifted up by k without a shift instruction).
+__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
+// E8 codes of a block straight from its 8 symbols and coset bit c: twice the zigzag
+// inverse is 2m = z ^ -(z & 1) (bit 0 clear), so q_i = 2 m_i + c = (z_i ^ s_i) | c;
+// the stripped parity of m_7 is bit 1 of q_0 ^ ... ^ q_6 (= the parity of sum m_i),
+// and q_7 = 2 (2 m_7' + p) + c.  Equal to Lattice<E8>::reinsert of the unzigzagged m.
+__device__ __forceinline__ void e8_codes_from_symbols(const uint32_t (&z)[8], uint32_t c, int32_t (&q)[8]) {
+    uint32_t x = 0;
+#pragma unroll
+    for (int i = 0; i < 7; i++) {
+        const uint32_t t = (z[i] ^ (0u - (z[i] & 1u))) | c;
+        q[i] = (int32_t)t;
+        x ^= t;
+    }
+    const uint32_t t7 = z[7] ^ (0u - (z[7] & 1u));
+    q[7] = (int32_t)((t7 << 1) | (x & 2u) | c);
+}
+
 // ------------------------------------------------------------------ dither
 // Section 4 subtractive dither: uniform r in [0,1) from 24 bits of the
 // generator output for pair e >> 1 (bits 40..63 for even e, 8..31 for odd e);

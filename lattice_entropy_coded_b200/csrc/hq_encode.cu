@@ -333,7 +333,7 @@ __device__ __forceinline__ void round_symbols_rolled(const EncodeArgs &a, const 
 
 // Remainder bits of 32 symbols (warp-uniform k) into the lane's k words.
 // KSMALL (k <= 4): a group of 8 remainders is built in one register, last
-// symbol first, two operations per symbol; otherwise a 64-bit accumulator.
+// symbol first (an and and a multiply-add per symbol); otherwise a 64-bit accumulator.
 template <bool KSMALL>
 __device__ __forceinline__ void put_rem(uint32_t *dst, const uint32_t (&z)[32], int k, bool store) {
     if (k == 0) return;
@@ -343,9 +343,10 @@ __device__ __forceinline__ void put_rem(uint32_t *dst, const uint32_t (&z)[32], 
 #pragma unroll
     for (int g = 0; g < 4; g++) {
         if (KSMALL) {
+            const uint32_t pk = 1u << k;
             uint32_t gv = 0;
 #pragma unroll
-            for (int i = 7; i >= 0; i--) gv = (gv << k) | (z[8 * g + i] & mask);
+            for (int i = 7; i >= 0; i--) gv = imad(gv, pk, z[8 * g + i] & mask);
             acc |= (unsigned long long)gv << nb;
             nb += 8u * (uint32_t)k;
         } else {
