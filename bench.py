@@ -518,7 +518,38 @@ def run_bulk(args):
             del codecs, outs, comps
             torch.cuda.empty_cache()
         out["points"] = res
+        if w["kind"] == "student_t":
+            out["calibration"] = calibrate_set(hq, mats, pts, w["seed"])
     print(json.dumps(out), flush=True)
+
+
+def calibrate_set(hq, mats, pts, seed):
+    """alpha and k for every rate point of a matrix set, chosen on the device over the
+    whole set (one contiguous tensor), with the time it takes and one rate pass's time."""
+    big = torch.cat(mats, dim=0)
+    st = hq.stats_tensor(big.device)
+    res = []
+    for p in pts:
+        params = hq.make_params(p["lattice"], p["alpha"], p["k"], seed, 0)
+        e0, e1 = _events()
+        e0.record()
+        hq.hq_rate(big, params, st)
+        e1.record()
+        torch.cuda.synchronize()
+        pass_ms = e0.elapsed_time(e1)
+        r = hq.read_stats(st)
+        t0 = time.perf_counter()
+        c = hq.hq_calibrate(big, hq.make_params(p["lattice"], 1.0, 0, seed, 0), hq.calib_spec(p["bps"], k_lo=0, k_hi=6),
+                            st)
+        wall = time.perf_counter() - t0
+        res.append(dict(lattice=p["lattice"], bps_target=p["bps"], elements=big.numel(),
+                        rate_pass_ms=pass_ms, rate_pass_gbs=2.0 * big.numel() / (pass_ms * 1e6),
+                        bps_at_sample_alpha=r["payload_bits"] / big.numel(),
+                        sample_alpha=p["alpha"], sample_k=p["k"], calibrated_alpha=c["alpha"], calibrated_k=c["k"],
+                        calibrated_bps=c["bps"], evaluations=c["evaluations"], calibrate_wall_s=wall))
+    del big
+    torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------------ single-matrix case (profiling)
@@ -544,8 +575,19 @@ def run_case(args):
         c.record()
         if i >= args.warmup:
             ev.append((a, b, c))
+    rst = hq.stats_tensor(device)
+    rev = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        hq.hq_rate(x, params, rst)
+        b.record()
+        if i >= args.warmup:
+            rev.append((a, b))
     torch.cuda.synchronize()
     st = hq.read_stats(codec.stats)
+    rate_ms = float(np.median([a.elapsed_time(b) for a, b in rev]))
+    assert hq.read_stats(rst)["payload_bits"] == st["payload_bits"]
     enc = float(np.median([a.elapsed_time(b) for a, b, _ in ev]))
     dec = float(np.median([b.elapsed_time(c) for _, b, c in ev]))
     n = x.numel()
@@ -556,7 +598,7 @@ def run_case(args):
                       "status": st["status"], "bps_payload": st["payload_bits"] / n,
                       "enc_ms": enc, "dec_ms": dec, "enc_gbs_in": 2.0 * n / enc / 1e6, "dec_gbs_in": 2.0 * n / dec / 1e6,
                       "enc_frac": alg / enc / 1e6 / peak, "dec_frac": alg / dec / 1e6 / peak,
-                      "alg_bytes": alg}), flush=True)
+                      "alg_bytes": alg, "rate_ms": rate_ms, "rate_gbs_in": 2.0 * n / rate_ms / 1e6}), flush=True)
 
 
 # ------------------------------------------------------------------ main

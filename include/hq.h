@@ -210,6 +210,74 @@ HQ_API int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t
                               uint32_t *d_stream, uint64_t cap_words, uint64_t *d_offsets, hq_stats *d_stats,
                               void *cuda_stream);
 
+/* ----------------------------------------------------------------- rate targeting */
+
+/* The rate of a quantize call, without its stream.  The pages state that alpha
+ * is calibrated and that the realized rate lands within about 0.01 bit per
+ * scalar of any target (HyperQuant explainer pages, "Methodology" 2 and 3).
+ * This runs the quantize path up to the Rice code lengths and adds into *d_stats
+ * (zeroed first, on cuda_stream) exactly what hq_quantize with the same
+ * arguments reports:
+ *   payload_bits  Rice codeword bits plus E8 coset bits (HQ_ST_RANGE clear);
+ *   stream_words  the words hq_quantize would write (coset, remainder and unary
+ *                 planes of every chunk), an exact capacity for it;
+ *   max_symbol    the OR of all symbols; status  HQ_ST_RANGE as in hq_quantize.
+ * x, rows, cols, ld, p and errors are those of hq_quantize; nothing else is
+ * written and no workspace is needed.  Asynchronous on cuda_stream. */
+HQ_API int hq_rate(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p, hq_stats *d_stats,
+                   void *cuda_stream);
+
+/* hq_rate for a block of KV tokens: kv is bf16 [heads, T, 128] with token stride
+ * ld_token and head stride ld_head (elements), the tokens being positions
+ * tok0 .. tok0 + T - 1 of the cache (their dither counters).  The rate equals
+ * that of hq_kv_append of the same tokens at that position, in any split into
+ * appends.  HQ_EINVAL for heads <= 0, T < 0, tok0 < 0 or a bad pointer/stride. */
+HQ_API int hq_rate_kv(const void *kv, int32_t heads, int64_t T, int64_t ld_token, int64_t ld_head, int64_t tok0,
+                      const hq_params *p, hq_stats *d_stats, void *cuda_stream);
+
+/* What to calibrate: payload bits per scalar to reach, its tolerance, the alpha
+ * bracket and the Rice parameters to try. */
+typedef struct hq_calib_spec {
+    double target_bps;           /* > 0 */
+    double tol;                  /* >= 0; stop when |rate - target| <= tol (e.g. 0.002) */
+    double alpha_lo, alpha_hi;   /* 0 < lo < hi; the bracket (e.g. 1e-3, 1e4) */
+    int32_t k_lo, k_hi;          /* 0 <= k_lo <= k_hi <= 15 */
+    int32_t max_iter;            /* bisection steps per k, 0..200 (e.g. 60) */
+    int32_t reserved;            /* 0 */
+} hq_calib_spec;                 /* 48 bytes */
+
+typedef struct hq_calib_result {
+    float alpha;                 /* the calibrated alpha (fp32, as hq_params holds it) */
+    int32_t k;                   /* the chosen Rice parameter, -1 if none */
+    double bps;                  /* payload bits per scalar at (alpha, k) */
+    int32_t evaluations;         /* rate passes run */
+    uint32_t status;             /* OR of the HQ_ST_* bits the passes saw */
+} hq_calib_result;               /* 24 bytes */
+
+/* Choose alpha (and k) on the device so that the payload rate of quantizing x
+ * meets a target.  For each k in [k_lo, k_hi], if rate(alpha_lo) <= target <=
+ * rate(alpha_hi), alpha is bisected at the geometric mid point sqrt(lo * hi)
+ * (evaluated at its fp32 rounding) until |rate - target| <= tol, at most
+ * max_iter steps; without convergence the result is the mid point of the final
+ * bracket.  The k with the largest alpha (the finest lattice at that rate)
+ * wins, the first on ties.  rate = hq_rate's payload_bits / (rows * cols); a
+ * pass that flags HQ_ST_RANGE counts as +infinity.
+ *
+ * p gives the lattice, seed and dither (its alpha and rice_k are ignored);
+ * d_stats is device scratch.  Unlike every other entry point this one
+ * SYNCHRONISES: each pass is copied back and waited for on cuda_stream, and the
+ * result is in *out when the call returns.  Returns HQ_OK; HQ_EUNSUPPORTED if
+ * no k brackets the target (out->k = -1); HQ_EINVAL for a bad spec, pointer or
+ * empty matrix; HQ_ECUDA on a CUDA error. */
+HQ_API int hq_calibrate(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p,
+                        const hq_calib_spec *spec, hq_stats *d_stats, void *cuda_stream, hq_calib_result *out);
+
+/* hq_calibrate for KV tokens (layout as hq_rate_kv); rate = payload bits /
+ * (heads * T * 128). */
+HQ_API int hq_calibrate_kv(const void *kv, int32_t heads, int64_t T, int64_t ld_token, int64_t ld_head,
+                           int64_t tok0, const hq_params *p, const hq_calib_spec *spec, hq_stats *d_stats,
+                           void *cuda_stream, hq_calib_result *out);
+
 /* ----------------------------------------------------------------- KV path */
 
 /* Fill a hq_kv_cache with the caller's buffers and zero its two tail words

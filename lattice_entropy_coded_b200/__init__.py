@@ -48,6 +48,17 @@ class hq_kv_cache(C.Structure):
                 ("params", hq_params), ("tokens", C.c_int64), ("chunks", C.c_uint64), ("appends", C.c_uint64)]
 
 
+class hq_calib_spec(C.Structure):
+    _fields_ = [("target_bps", C.c_double), ("tol", C.c_double), ("alpha_lo", C.c_double), ("alpha_hi", C.c_double),
+                ("k_lo", C.c_int32), ("k_hi", C.c_int32), ("max_iter", C.c_int32), ("reserved", C.c_int32)]
+
+
+class hq_calib_result(C.Structure):
+    _fields_ = [("alpha", C.c_float), ("k", C.c_int32), ("bps", C.c_double), ("evaluations", C.c_int32),
+                ("status", C.c_uint32)]
+
+
+assert C.sizeof(hq_calib_spec) == 48 and C.sizeof(hq_calib_result) == 24
 assert C.sizeof(hq_params) == 32 and C.sizeof(hq_stats) == 32 and C.sizeof(hq_kv_append_row) == 32
 assert C.sizeof(hq_kv_cache) == 128
 
@@ -60,6 +71,14 @@ EXPORTS = {
                               C.c_uint64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "hq_dequantize": (C.c_int, [C.c_void_p, C.c_uint64, C.c_void_p, C.c_int64, C.c_int64, C.POINTER(hq_params),
                                 C.c_void_p, C.c_int, C.c_int64, C.c_void_p, C.c_void_p]),
+    "hq_rate": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.POINTER(hq_params), C.c_void_p, C.c_void_p]),
+    "hq_rate_kv": (C.c_int, [C.c_void_p, C.c_int32, C.c_int64, C.c_int64, C.c_int64, C.c_int64, C.POINTER(hq_params),
+                             C.c_void_p, C.c_void_p]),
+    "hq_calibrate": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.POINTER(hq_params),
+                               C.POINTER(hq_calib_spec), C.c_void_p, C.c_void_p, C.POINTER(hq_calib_result)]),
+    "hq_calibrate_kv": (C.c_int, [C.c_void_p, C.c_int32, C.c_int64, C.c_int64, C.c_int64, C.c_int64,
+                                  C.POINTER(hq_params), C.POINTER(hq_calib_spec), C.c_void_p, C.c_void_p,
+                                  C.POINTER(hq_calib_result)]),
     "hq_debug_set_encode_path": (C.c_int, [C.c_int]),
     "hq_debug_nearest": (C.c_int, [C.c_int, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p]),
     "hq_kv_init": (C.c_int, [C.POINTER(hq_kv_cache), C.c_int32, C.c_int32, C.POINTER(hq_params), C.c_void_p,
@@ -132,6 +151,53 @@ def hq_device_check() -> int:
 
 def hq_debug_set_spin_limit(polls: int) -> None:
     _lib.hq_debug_set_spin_limit(int(polls))
+
+
+def hq_rate(x: torch.Tensor, params: hq_params, stats: torch.Tensor, cuda_stream=None, ld: int | None = None) -> int:
+    """Rate of hq_quantize(x, params) without its stream, into stats (payload_bits, stream_words, ...)."""
+    rows, cols = x.shape
+    ld = x.stride(0) if ld is None else ld
+    return _check(_lib.hq_rate(_ptr(x), rows, cols, ld, C.byref(params), _ptr(stats), _stream(cuda_stream)), "hq_rate")
+
+
+def hq_rate_kv(kv: torch.Tensor, params: hq_params, stats: torch.Tensor, tok0: int = 0, cuda_stream=None) -> int:
+    """kv: bf16 [heads, T, 128], unit stride in the last dimension; tokens at positions tok0..tok0+T-1."""
+    H, T, D = kv.shape
+    assert D == 128 and kv.stride(2) == 1
+    return _check(_lib.hq_rate_kv(_ptr(kv), H, T, kv.stride(1), kv.stride(0), tok0, C.byref(params), _ptr(stats),
+                                  _stream(cuda_stream)), "hq_rate_kv")
+
+
+def calib_spec(target_bps: float, tol: float = 0.002, k_lo: int = 0, k_hi: int = 6, alpha_lo: float = 1e-3,
+               alpha_hi: float = 1e4, max_iter: int = 60) -> hq_calib_spec:
+    return hq_calib_spec(float(target_bps), float(tol), float(alpha_lo), float(alpha_hi), int(k_lo), int(k_hi),
+                         int(max_iter), 0)
+
+
+def _calib_result(r: hq_calib_result) -> dict:
+    return {"alpha": float(r.alpha), "k": int(r.k), "bps": float(r.bps), "evaluations": int(r.evaluations),
+            "status": int(r.status)}
+
+
+def hq_calibrate(x: torch.Tensor, params: hq_params, spec: hq_calib_spec, stats: torch.Tensor, cuda_stream=None,
+                 ld: int | None = None) -> dict:
+    """Synchronous: alpha (and k) for spec.target_bps on the device; see hq.h."""
+    rows, cols = x.shape
+    ld = x.stride(0) if ld is None else ld
+    out = hq_calib_result()
+    _check(_lib.hq_calibrate(_ptr(x), rows, cols, ld, C.byref(params), C.byref(spec), _ptr(stats),
+                             _stream(cuda_stream), C.byref(out)), "hq_calibrate")
+    return _calib_result(out)
+
+
+def hq_calibrate_kv(kv: torch.Tensor, params: hq_params, spec: hq_calib_spec, stats: torch.Tensor, tok0: int = 0,
+                    cuda_stream=None) -> dict:
+    H, T, D = kv.shape
+    assert D == 128 and kv.stride(2) == 1
+    out = hq_calib_result()
+    _check(_lib.hq_calibrate_kv(_ptr(kv), H, T, kv.stride(1), kv.stride(0), tok0, C.byref(params), C.byref(spec),
+                                _ptr(stats), _stream(cuda_stream), C.byref(out)), "hq_calibrate_kv")
+    return _calib_result(out)
 
 
 def hq_debug_set_encode_path(path: int) -> int:

@@ -283,6 +283,168 @@ int hq_kv_read(const hq_kv_cache *cache, void *out, int out_dtype, int64_t len, 
     return cuda_rc(launch_decode(cache->params.lattice, cache->params.dither, a, (cudaStream_t)cuda_stream));
 }
 
+// ------------------------------------------------------------------ rate and calibration
+}  // extern "C"
+
+namespace {
+
+// Rate-only launch over the tile map in `a` (weights or KV), stats zeroed first.
+int rate_launch(const hq_params *p, EncodeArgs &a, hq_stats *d_stats, cudaStream_t s) {
+    if (cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
+    if (a.n_chunks == 0) return HQ_OK;
+    a.c_scale = scale_fwd(p->alpha);
+    a.k = p->rice_k;
+    a.seed = p->seed;
+    a.stats = d_stats;
+    return cuda_rc(launch_rate(p->lattice, p->dither, a, s));
+}
+
+int weights_rate_args(const void *x, int64_t rows, int64_t cols, int64_t ld, EncodeArgs &a) {
+    int rc = check_matrix(rows, cols);
+    if (rc) return rc;
+    memset(&a, 0, sizeof(a));
+    a.n_chunks = chunks_of(rows, cols);
+    if (a.n_chunks && (!x || !aligned(x, 16) || ld < cols || ld % 8)) return HQ_EINVAL;
+    a.x = (const uint16_t *)x;
+    a.map.kv = 0;
+    a.map.rows = rows;
+    a.map.cols = cols;
+    a.map.ld = ld;
+    a.tcols = (int)(cols / kTile);
+    return HQ_OK;
+}
+
+int kv_rate_args(const void *kv, int32_t heads, int64_t T, int64_t ld_token, int64_t ld_head, int64_t tok0,
+                 EncodeArgs &a) {
+    if (heads <= 0 || T < 0 || tok0 < 0) return HQ_EINVAL;
+    memset(&a, 0, sizeof(a));
+    a.n_chunks = (uint64_t)heads * (uint64_t)((T + 31) / 32);
+    if (a.n_chunks && (!kv || !aligned(kv, 16) || ld_token < kTile || ld_token % 8 || ld_head % 8 || ld_head < 0))
+        return HQ_EINVAL;
+    a.x = (const uint16_t *)kv;
+    a.map.kv = 1;
+    a.map.heads = heads;
+    a.map.tokens = T;
+    a.map.ld_tok = ld_token;
+    a.map.ld_head = ld_head;
+    a.map.tok0 = tok0;
+    a.tcols = 1;
+    return HQ_OK;
+}
+
+int check_spec(const hq_calib_spec *sp) {
+    if (!sp) return HQ_EINVAL;
+    if (!(sp->target_bps > 0.0) || !(sp->tol >= 0.0) || !(sp->alpha_lo > 0.0) || !(sp->alpha_hi > sp->alpha_lo) ||
+        !isfinite(sp->alpha_hi) || !isfinite(sp->target_bps))
+        return HQ_EINVAL;
+    if (sp->k_lo < 0 || sp->k_hi > 15 || sp->k_lo > sp->k_hi || sp->max_iter < 0 || sp->max_iter > 200)
+        return HQ_EINVAL;
+    return HQ_OK;
+}
+
+// Payload bits per scalar at (alpha, k): one rate launch, copied back and waited for.
+// A launch that flags HQ_ST_RANGE counts as +infinity (the rate only grows with alpha).
+int rate_at(const hq_params &base, float alpha, int k, EncodeArgs a, double n, hq_stats *d_stats, cudaStream_t s,
+            double &bps, uint32_t &seen) {
+    hq_params p = base;
+    p.alpha = alpha;
+    p.rice_k = k;
+    int rc = rate_launch(&p, a, d_stats, s);
+    if (rc) return rc;
+    hq_stats h;
+    if (cudaMemcpyAsync(&h, d_stats, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return HQ_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return HQ_ECUDA;
+    seen |= h.status;
+    bps = (h.status & HQ_ST_RANGE) ? INFINITY : (double)h.payload_bits / n;
+    return HQ_OK;
+}
+
+// For each k in [k_lo, k_hi]: if rate(lo) <= target <= rate(hi), bisect alpha at the
+// geometric mid point until |rate - target| <= tol (at most max_iter steps; then the
+// mid point of the last bracket).  The k with the largest alpha wins (the first on ties).
+int calibrate(const hq_params *p, const hq_calib_spec *sp, const EncodeArgs &a, double n, hq_stats *d_stats,
+              cudaStream_t s, hq_calib_result *out) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if ((rc = check_spec(sp))) return rc;
+    if (!out || !d_stats || !aligned(d_stats, 8)) return HQ_EINVAL;
+    memset(out, 0, sizeof(*out));
+    out->k = -1;
+    if (a.n_chunks == 0) return HQ_EINVAL;
+    bool found = false;
+    double best = 0.0;
+    for (int k = sp->k_lo; k <= sp->k_hi; k++) {
+        double lo = sp->alpha_lo, hi = sp->alpha_hi, rlo, rhi, r, mid;
+        if ((rc = rate_at(*p, (float)lo, k, a, n, d_stats, s, rlo, out->status))) return rc;
+        if ((rc = rate_at(*p, (float)hi, k, a, n, d_stats, s, rhi, out->status))) return rc;
+        out->evaluations += 2;
+        if (!(rlo <= sp->target_bps && sp->target_bps <= rhi)) continue;
+        bool done = false;
+        for (int it = 0; it < sp->max_iter && !done; it++) {
+            mid = sqrt(lo * hi);
+            if ((rc = rate_at(*p, (float)mid, k, a, n, d_stats, s, r, out->status))) return rc;
+            out->evaluations++;
+            if (fabs(r - sp->target_bps) <= sp->tol) done = true;
+            else if (r < sp->target_bps) lo = mid;
+            else hi = mid;
+        }
+        if (!done) {
+            mid = sqrt(lo * hi);
+            if ((rc = rate_at(*p, (float)mid, k, a, n, d_stats, s, r, out->status))) return rc;
+            out->evaluations++;
+        }
+        if (!found || mid > best) {
+            found = true;
+            best = mid;
+            out->alpha = (float)mid;
+            out->k = k;
+            out->bps = r;
+        }
+    }
+    return found ? HQ_OK : HQ_EUNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hq_rate(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p, hq_stats *d_stats,
+            void *cuda_stream) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (!d_stats || !aligned(d_stats, 8)) return HQ_EINVAL;
+    EncodeArgs a;
+    if ((rc = weights_rate_args(x, rows, cols, ld, a))) return rc;
+    return rate_launch(p, a, d_stats, (cudaStream_t)cuda_stream);
+}
+
+int hq_rate_kv(const void *kv, int32_t heads, int64_t T, int64_t ld_token, int64_t ld_head, int64_t tok0,
+               const hq_params *p, hq_stats *d_stats, void *cuda_stream) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (!d_stats || !aligned(d_stats, 8)) return HQ_EINVAL;
+    EncodeArgs a;
+    if ((rc = kv_rate_args(kv, heads, T, ld_token, ld_head, tok0, a))) return rc;
+    return rate_launch(p, a, d_stats, (cudaStream_t)cuda_stream);
+}
+
+int hq_calibrate(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p, const hq_calib_spec *spec,
+                 hq_stats *d_stats, void *cuda_stream, hq_calib_result *out) {
+    EncodeArgs a;
+    int rc = weights_rate_args(x, rows, cols, ld, a);
+    if (rc) return rc;
+    return calibrate(p, spec, a, (double)rows * (double)cols, d_stats, (cudaStream_t)cuda_stream, out);
+}
+
+int hq_calibrate_kv(const void *kv, int32_t heads, int64_t T, int64_t ld_token, int64_t ld_head, int64_t tok0,
+                    const hq_params *p, const hq_calib_spec *spec, hq_stats *d_stats, void *cuda_stream,
+                    hq_calib_result *out) {
+    EncodeArgs a;
+    int rc = kv_rate_args(kv, heads, T, ld_token, ld_head, tok0, a);
+    if (rc) return rc;
+    return calibrate(p, spec, a, (double)heads * (double)T * kTile, d_stats, (cudaStream_t)cuda_stream, out);
+}
+
 const char *hq_status_string(int code) {
     switch (code) {
     case HQ_OK: return "ok";

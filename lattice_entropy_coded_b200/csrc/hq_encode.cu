@@ -900,6 +900,82 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ rate only
+// The quantize path up to the Rice code lengths, without a stream: per chunk the
+// unary bits U, so payload = U + remainder bits + coset bits and the chunk's words
+// = coset + remainder + ceil(U / 32), exactly as the encoder counts them.  Chunks
+// are independent here (no offsets), so warps take them by a static stride.
+template <int LAT, bool DITHER>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, 2) rate_kernel(const EncodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *sign_tab = smem;
+    build_sign_table(sign_tab, a.tcols, a.seed);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int k = a.k;
+    const unsigned long long nwarps = (unsigned long long)gridDim.x * kWarpsPerCta;
+    unsigned long long payload = 0, words = 0;
+    uint32_t status = 0, zor_all = 0;
+    for (unsigned long long c = (unsigned long long)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); c < a.n_chunks;
+         c += nwarps) {
+        ChunkGeo geo;
+        geo.init(a.map, c);
+        const int nrounds = (geo.ntiles + kTilesPerRound - 1) / kTilesPerRound;
+        unsigned long long U = 0;
+        uint32_t lor = 0;
+#pragma unroll 1
+        for (int r = 0; r < nrounds; r++) {
+            RoundInput in;
+            const uint16_t *src = nullptr;
+            in.tcol = 0;
+            in.e0 = 0;
+            in.valid = geo.tile(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, in.tcol, in.e0);
+            uint4 raw[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                raw[j] = in.valid ? ldg_nc_v4(src + 32 * (lane & 3) + 8 * j) : make_uint4(0, 0, 0, 0);
+            uint32_t z[32], cbits;
+            round_symbols<LAT, DITHER>(a, in, raw, lane, sign_tab, z, cbits);
+            uint32_t usum = 0;
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                usum += z[i] >> k;
+                lor |= z[i];
+            }
+            // symbols below 2^22 keep ub below 2^28: two 32-bit sums of its halves are exact
+            const uint32_t ub = in.valid ? usum + 32u : 0u;
+            const uint32_t lo = __reduce_add_sync(0xffffffffu, ub & 0xFFFFu);
+            const uint32_t hi = __reduce_add_sync(0xffffffffu, ub >> 16);
+            U += (unsigned long long)lo + ((unsigned long long)hi << 16);
+        }
+        lor = __reduce_or_sync(0xffffffffu, lor);
+        zor_all |= lor;
+        const unsigned long long nc = (LAT == HQ_E8) ? (16ull * geo.ntiles + 31) / 32 : 0ull;
+        const unsigned long long nr = 4ull * (unsigned long long)k * (unsigned long long)geo.ntiles;
+        payload += U + nr * 32 + ((LAT == HQ_E8) ? 16ull * geo.ntiles : 0ull);
+        words += nc + nr + (U + 31) / 32;
+        if ((lor >> 22) != 0u || U >= kMaxUnaryBits) status |= HQ_ST_RANGE;
+    }
+    if (lane == 0) {
+        if (status) atomicOr(&a.stats->status, status);
+        if (zor_all) atomicOr(&a.stats->max_symbol, zor_all);
+        if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
+        if (words) atomicAdd((unsigned long long *)&a.stats->stream_words, words);
+    }
+}
+
+template <int LAT, bool DITHER>
+cudaError_t launch_rate_t(const EncodeArgs &a, cudaStream_t s) {
+    const size_t smem = (size_t)a.tcols * kSignWords * sizeof(uint32_t);
+    auto kern = rate_kernel<LAT, DITHER>;
+    static LaunchPlan plan;
+    unsigned grid = 0;
+    cudaError_t e = plan.grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_encode(int lattice, int dither, const EncodeArgs &a, cudaStream_t s) {
@@ -912,6 +988,20 @@ cudaError_t launch_encode(int lattice, int dither, const EncodeArgs &a, cudaStre
     case HQ_D4 * 2 + 1: return launch_t<HQ_D4, true>(a, s);
     case HQ_E8 * 2: return launch_t<HQ_E8, false>(a, s);
     case HQ_E8 * 2 + 1: return launch_t<HQ_E8, true>(a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_rate(int lattice, int dither, const EncodeArgs &a, cudaStream_t s) {
+    switch (lattice * 2 + (dither ? 1 : 0)) {
+    case HQ_Z * 2: return launch_rate_t<HQ_Z, false>(a, s);
+    case HQ_Z * 2 + 1: return launch_rate_t<HQ_Z, true>(a, s);
+    case HQ_A2 * 2: return launch_rate_t<HQ_A2, false>(a, s);
+    case HQ_A2 * 2 + 1: return launch_rate_t<HQ_A2, true>(a, s);
+    case HQ_D4 * 2: return launch_rate_t<HQ_D4, false>(a, s);
+    case HQ_D4 * 2 + 1: return launch_rate_t<HQ_D4, true>(a, s);
+    case HQ_E8 * 2: return launch_rate_t<HQ_E8, false>(a, s);
+    case HQ_E8 * 2 + 1: return launch_rate_t<HQ_E8, true>(a, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -125,5 +125,8 @@ extern int g_encode_path;
 // Launchers (defined in hq_encode.cu / hq_decode.cu).  Return cudaSuccess or the launch error.
 cudaError_t launch_encode(int lattice, int dither, const EncodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode(int lattice, int dither, const DecodeArgs &a, cudaStream_t s);
+// Rate only: adds payload_bits, stream_words, max_symbol and HQ_ST_RANGE of the call into a.stats
+// (zeroed by the caller); reads a.x, a.map, a.n_chunks, a.c_scale, a.k, a.seed, a.tcols.
+cudaError_t launch_rate(int lattice, int dither, const EncodeArgs &a, cudaStream_t s);
 
 }  // namespace hq

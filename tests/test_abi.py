@@ -39,6 +39,8 @@ def test_struct_layouts_match_header():
     assert C.sizeof(hq.hq_stats) == 32 and hq.hq_stats.payload_bits.offset == 8
     assert C.sizeof(hq.hq_kv_append_row) == 32
     assert C.sizeof(hq.hq_kv_cache) == 128 and hq.hq_kv_cache.params.offset == 72
+    assert C.sizeof(hq.hq_calib_spec) == 48 and hq.hq_calib_spec.k_lo.offset == 32
+    assert C.sizeof(hq.hq_calib_result) == 24 and hq.hq_calib_result.bps.offset == 8
 
 
 def test_stream_bound_and_workspace():
@@ -101,6 +103,22 @@ def test_entry_points_validate_before_touching_the_device():
     assert lib.hq_kv_append(C.byref(cache), None, 16, 128, 2048, C.c_float(1.0), None, 0, None) == hq.HQ_EINVAL
     assert lib.hq_kv_read(C.byref(cache), None, 0, 1, 128, 2048, None) == hq.HQ_EINVAL
     assert hq.hq_status_string(hq.HQ_ST_TIMEOUT) == "look-back timed out"
+    # rate and calibration: argument errors before any device work
+    st = C.c_void_p(64)
+    assert lib.hq_rate(None, 32, 128, 128, C.byref(p), st, None) == hq.HQ_EINVAL          # null x
+    assert lib.hq_rate(None, 32, 100, 128, C.byref(p), st, None) == hq.HQ_EINVAL          # cols % 128
+    assert lib.hq_rate(None, 32, 128, 128, C.byref(p), None, None) == hq.HQ_EINVAL        # null stats
+    assert lib.hq_rate_kv(None, 0, 16, 128, 2048, 0, C.byref(p), st, None) == hq.HQ_EINVAL  # heads 0
+    assert lib.hq_rate_kv(None, 8, 16, 128, 2048, -1, C.byref(p), st, None) == hq.HQ_EINVAL  # tok0 < 0
+    res = hq.hq_calib_result()
+    good = hq.calib_spec(4.0)
+    assert lib.hq_calibrate(None, 32, 128, 128, C.byref(p), C.byref(good), st, None, C.byref(res)) == hq.HQ_EINVAL
+    for bad in (hq.calib_spec(0.0), hq.calib_spec(4.0, alpha_lo=2.0, alpha_hi=1.0), hq.calib_spec(4.0, k_lo=3, k_hi=2),
+                hq.calib_spec(4.0, k_hi=16), hq.calib_spec(4.0, tol=-1.0), hq.calib_spec(4.0, max_iter=201)):
+        assert lib.hq_calibrate(C.c_void_p(256), 32, 128, 128, C.byref(p), C.byref(bad), st, None,
+                                C.byref(res)) == hq.HQ_EINVAL
+    assert lib.hq_calibrate(C.c_void_p(256), 0, 128, 128, C.byref(p), C.byref(good), st, None,
+                            C.byref(res)) == hq.HQ_EINVAL                                   # empty
     # testing aids: encoder form switch and the nearest-point entry point
     assert lib.hq_debug_set_encode_path(3) == hq.HQ_EINVAL
     assert lib.hq_debug_set_encode_path(-1) == hq.HQ_EINVAL
