@@ -181,6 +181,28 @@ HQ_API int hq_dequantize(const uint32_t *d_stream, uint64_t stream_words, const 
                   int64_t cols, const hq_params *p, void *out, int out_dtype, int64_t ld, hq_stats *d_stats,
                   void *cuda_stream);
 
+/* Decode fused into its consumer: y = W x for a compressed matrix W, without
+ * writing W to memory.  The pages name the cost of the variable-length format at
+ * inference ("Results": decode adds latency on an H100); here each decoded
+ * 128-element tile goes straight into a dot product, so W is read at its
+ * compressed size (about R/8 bytes per element) instead of 2 bytes of bf16.
+ *   W      : the stream of hq_quantize (d_stream, stream_words, d_offsets, rows,
+ *            cols, p as for hq_dequantize); its elements are taken exactly as
+ *            hq_dequantize stores them in bf16.
+ *   d_x    : device, bf16 [cols], 16-byte aligned.
+ *   d_y    : device, fp32 [rows]: y[r] = sum_j W[r, j] * x[j], bf16 products
+ *            (exact in fp32) accumulated in fp32: per tile a sequential fma over
+ *            each lane's 32 elements and a fixed 4-lane tree, then the row's
+ *            tiles in column order (results do not depend on scheduling).
+ *   workspace, ws_bytes : device, >= hq_gemv_workspace_bytes (one float per
+ *            tile), 16-byte aligned.
+ * d_stats as hq_dequantize (HQ_ST_CORRUPT; a corrupt chunk's tiles count as 0).
+ * Asynchronous on cuda_stream; errors as hq_dequantize. */
+HQ_API int hq_gemv_workspace_bytes(int64_t rows, int64_t cols, size_t *bytes);
+HQ_API int hq_gemv(const uint32_t *d_stream, uint64_t stream_words, const uint64_t *d_offsets, int64_t rows,
+                   int64_t cols, const hq_params *p, const void *d_x, float *d_y, void *workspace, size_t ws_bytes,
+                   hq_stats *d_stats, void *cuda_stream);
+
 /* No counterpart in the paper: an addition for callers that cannot allocate.
  *
  * hq_quantize without a workspace, for callers that hold only their input and
@@ -302,6 +324,19 @@ HQ_API int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t l
  * hq_dequantize.  len <= cache->tokens. */
 HQ_API int hq_kv_read(const hq_kv_cache *cache, void *out, int out_dtype, int64_t len, int64_t out_ld_token,
                int64_t out_ld_head, void *cuda_stream);
+
+/* Attention scores over a compressed K cache, without writing K to memory:
+ * scores[(h * group + g) * scores_ld + t] = sum_d K[h, t, d] * q[h * group + g, d]
+ * for every KV head h, query head g of its group and token t < len; K[h, t, :]
+ * is exactly the bf16 row hq_kv_read stores (after un-dithering), products are
+ * exact in fp32 and accumulated as in hq_gemv.
+ *   d_q       : device, bf16 [heads * group, 128], 16-byte aligned.
+ *   group     : query heads per KV head (grouped-query attention), >= 1.
+ *   d_scores  : device, fp32 [heads * group, scores_ld], scores_ld >= len;
+ *               columns >= len are not written.
+ * Status bits go to the cache's d_stats as for hq_kv_read.  Asynchronous. */
+HQ_API int hq_kv_scores(const hq_kv_cache *cache, const void *d_q, int32_t group, float *d_scores, int64_t len,
+                        int64_t scores_ld, void *cuda_stream);
 
 /* ---------------------------------------------------------------- misc */
 

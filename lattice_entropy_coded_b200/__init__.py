@@ -79,6 +79,11 @@ EXPORTS = {
     "hq_calibrate_kv": (C.c_int, [C.c_void_p, C.c_int32, C.c_int64, C.c_int64, C.c_int64, C.c_int64,
                                   C.POINTER(hq_params), C.POINTER(hq_calib_spec), C.c_void_p, C.c_void_p,
                                   C.POINTER(hq_calib_result)]),
+    "hq_gemv_workspace_bytes": (C.c_int, [C.c_int64, C.c_int64, C.POINTER(C.c_size_t)]),
+    "hq_gemv": (C.c_int, [C.c_void_p, C.c_uint64, C.c_void_p, C.c_int64, C.c_int64, C.POINTER(hq_params),
+                          C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p]),
+    "hq_kv_scores": (C.c_int, [C.POINTER(hq_kv_cache), C.c_void_p, C.c_int32, C.c_void_p, C.c_int64, C.c_int64,
+                               C.c_void_p]),
     "hq_debug_set_encode_path": (C.c_int, [C.c_int]),
     "hq_debug_nearest": (C.c_int, [C.c_int, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p]),
     "hq_kv_init": (C.c_int, [C.POINTER(hq_kv_cache), C.c_int32, C.c_int32, C.POINTER(hq_params), C.c_void_p,
@@ -151,6 +156,30 @@ def hq_device_check() -> int:
 
 def hq_debug_set_spin_limit(polls: int) -> None:
     _lib.hq_debug_set_spin_limit(int(polls))
+
+
+def hq_gemv_workspace_bytes(rows: int, cols: int) -> int:
+    b = C.c_size_t()
+    _check(_lib.hq_gemv_workspace_bytes(rows, cols, C.byref(b)), "hq_gemv_workspace_bytes")
+    return int(b.value)
+
+
+def hq_gemv(stream: torch.Tensor, stream_words: int, offsets: torch.Tensor, rows: int, cols: int, params: hq_params,
+            x: torch.Tensor, y: torch.Tensor, workspace: torch.Tensor, stats: torch.Tensor | None = None,
+            cuda_stream=None) -> int:
+    """y (fp32 [rows]) = W x for the compressed W; x bf16 [cols]."""
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and y.dtype == torch.float32
+    return _check(_lib.hq_gemv(_ptr(stream), stream_words, _ptr(offsets), rows, cols, C.byref(params), _ptr(x),
+                               _ptr(y), _ptr(workspace), workspace.numel(), _ptr(stats), _stream(cuda_stream)),
+                  "hq_gemv")
+
+
+def hq_kv_scores(cache: hq_kv_cache, q: torch.Tensor, group: int, scores: torch.Tensor, length: int,
+                 cuda_stream=None) -> int:
+    """q bf16 [heads * group, 128]; scores fp32 [heads * group, >= length]."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous() and scores.dtype == torch.float32
+    return _check(_lib.hq_kv_scores(C.byref(cache), _ptr(q), group, _ptr(scores), length, scores.stride(0),
+                                    _stream(cuda_stream)), "hq_kv_scores")
 
 
 def hq_rate(x: torch.Tensor, params: hq_params, stats: torch.Tensor, cuda_stream=None, ld: int | None = None) -> int:
@@ -327,6 +356,15 @@ class Codec:
         hq_dequantize(c.words, self.cap_words, c.offsets, c.rows, c.cols, c.params, out, stats, cuda_stream)
         return out
 
+    def gemv(self, c: Compressed, x: torch.Tensor, y: torch.Tensor, stats: torch.Tensor | None = None,
+             cuda_stream=None) -> torch.Tensor:
+        """y = W x straight from the compressed W (no bf16 copy of W is made)."""
+        if getattr(self, "_gemv_ws", None) is None:
+            self._gemv_ws = torch.empty(hq_gemv_workspace_bytes(self.rows, self.cols), dtype=torch.uint8,
+                                        device=self.words.device)
+        hq_gemv(c.words, self.cap_words, c.offsets, c.rows, c.cols, c.params, x, y, self._gemv_ws, stats, cuda_stream)
+        return y
+
 
 class KVCache:
     """A compressed K or V cache (one layer) with torch-allocated device buffers."""
@@ -355,4 +393,10 @@ class KVCache:
 
     def read(self, out: torch.Tensor, length: int | None = None, cuda_stream=None) -> torch.Tensor:
         hq_kv_read(self.cache, out, self.tokens if length is None else length, cuda_stream)
+        return out
+
+    def scores(self, q: torch.Tensor, group: int, out: torch.Tensor, length: int | None = None,
+               cuda_stream=None) -> torch.Tensor:
+        """out[h * group + g, t] = K[h, t] . q[h * group + g] straight from the compressed cache."""
+        hq_kv_scores(self.cache, q, group, out, self.tokens if length is None else length, cuda_stream)
         return out

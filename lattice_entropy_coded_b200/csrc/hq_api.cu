@@ -165,6 +165,53 @@ int hq_dequantize(const uint32_t *d_stream, uint64_t stream_words, const uint64_
     return cuda_rc(launch_decode(p->lattice, p->dither, a, s));
 }
 
+int hq_gemv_workspace_bytes(int64_t rows, int64_t cols, size_t *bytes) {
+    if (!bytes) return HQ_EINVAL;
+    int rc = check_matrix(rows, cols);
+    if (rc) return rc;
+    const size_t b = (size_t)rows * (size_t)(cols / kTile) * sizeof(float);
+    *bytes = (b + 255) & ~(size_t)255;
+    return HQ_OK;
+}
+
+int hq_gemv(const uint32_t *d_stream, uint64_t stream_words, const uint64_t *d_offsets, int64_t rows, int64_t cols,
+            const hq_params *p, const void *d_x, float *d_y, void *workspace, size_t ws_bytes, hq_stats *d_stats,
+            void *cuda_stream) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if ((rc = check_matrix(rows, cols))) return rc;
+    if (d_stats && !aligned(d_stats, 8)) return HQ_EINVAL;
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    if (d_stats && cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
+    if (rows == 0) return HQ_OK;
+    if (!d_y || !aligned(d_y, 4)) return HQ_EINVAL;
+    if (cols == 0) return cuda_rc(cudaMemsetAsync(d_y, 0, (size_t)rows * sizeof(float), s));
+    if (!d_stream || !aligned(d_stream, 4) || !d_offsets || !aligned(d_offsets, 8)) return HQ_EINVAL;
+    if (!d_x || !aligned(d_x, 16)) return HQ_EINVAL;
+    size_t need = 0;
+    hq_gemv_workspace_bytes(rows, cols, &need);
+    if (!workspace || !aligned(workspace, 16) || ws_bytes < need) return HQ_EINVAL;
+
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.stream = d_stream;
+    a.stream_words = stream_words;
+    a.offsets = d_offsets;
+    a.map.kv = 0;
+    a.map.rows = rows;
+    a.map.cols = cols;
+    a.n_chunks = chunks_of(rows, cols);
+    a.e_scale = scale_inv(p->alpha);
+    a.k = p->rice_k;
+    a.seed = p->seed;
+    a.out = nullptr;
+    a.stats = d_stats;
+    a.tcols = (int)(cols / kTile);
+    a.vec = (const uint16_t *)d_x;
+    a.res = (float *)workspace;
+    return cuda_rc(launch_gemv(p->lattice, p->dither, a, d_y, s));
+}
+
 int hq_kv_init(hq_kv_cache *cache, int32_t heads, int32_t head_dim, const hq_params *p, uint32_t *d_words,
                uint64_t cap_words, uint64_t *d_offsets, uint64_t offsets_cap, hq_kv_append_row *d_table,
                uint64_t table_cap, uint64_t *d_tail, hq_stats *d_stats, void *cuda_stream) {
@@ -443,6 +490,35 @@ int hq_calibrate_kv(const void *kv, int32_t heads, int64_t T, int64_t ld_token, 
     int rc = kv_rate_args(kv, heads, T, ld_token, ld_head, tok0, a);
     if (rc) return rc;
     return calibrate(p, spec, a, (double)heads * (double)T * kTile, d_stats, (cudaStream_t)cuda_stream, out);
+}
+
+int hq_kv_scores(const hq_kv_cache *cache, const void *d_q, int32_t group, float *d_scores, int64_t len,
+                 int64_t scores_ld, void *cuda_stream) {
+    if (!cache || !cache->d_words) return HQ_EINVAL;
+    if (group < 1 || len < 0 || len > cache->tokens) return HQ_EINVAL;
+    if (len == 0 || cache->chunks == 0) return HQ_OK;
+    if (!d_q || !aligned(d_q, 16) || !d_scores || !aligned(d_scores, 4) || scores_ld < len) return HQ_EINVAL;
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.stream = cache->d_words;
+    a.stream_words = cache->cap_words;
+    a.offsets = cache->d_offsets;
+    a.map.kv = 1;
+    a.map.heads = cache->heads;
+    a.n_chunks = cache->chunks;
+    a.k = cache->params.rice_k;
+    a.seed = cache->params.seed;
+    a.out = nullptr;
+    a.out_ld = scores_ld;
+    a.len = len;
+    a.table = cache->d_table;
+    a.n_appends = cache->appends;
+    a.stats = cache->d_stats;
+    a.tcols = 1;
+    a.vec = (const uint16_t *)d_q;
+    a.res = d_scores;
+    a.group = group;
+    return cuda_rc(launch_kv_scores(cache->params.lattice, cache->params.dither, a, (cudaStream_t)cuda_stream));
 }
 
 const char *hq_status_string(int code) {

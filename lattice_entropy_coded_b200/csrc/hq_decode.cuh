@@ -1,0 +1,529 @@
+// hq_decode.cuh -- the decode + dequantize kernel (HyperQuant "Methodology"
+// sections 1-4 inverted): Rice planes -> symbols -> re-inserted membership bits
+// -> lattice point [- dither] -> scale -> FWHT-128 -> sign, and then one of three
+// outputs: the bf16 or fp32 tile (hq_dequantize, hq_kv_read), the tile's dot
+// product with a bf16 vector (hq_gemv: one partial per tile), or a KV tile's dot
+// products with the query heads of its group (hq_kv_scores).  Included by
+// hq_decode.cu (stored tiles) and hq_consume.cu (dot products), each of which
+// instantiates the modes it launches.
+//
+// Work decomposition (B200, sm_100a):
+//  * one warp decodes one chunk (32 tiles) in 4 rounds of 8 tiles; four lanes
+//    share a tile, 32 symbols / elements each;
+//  * the chunk's words are brought into a per-warp shared-memory stage with
+//    cp.async while the warp is still decoding the previous chunk (two stages
+//    per warp); chunks too large for a stage are read from global memory;
+//  * the lanes split the unary plane into 32 word ranges, count terminators
+//    (popc) and scan, so every 32-symbol segment learns where its first
+//    codeword starts; each lane then reads its 32 quotients from bit-reversed
+//    32-bit windows, four symbols per window (one count-leading-zeros and one
+//    shift per symbol), its k remainder bits from its own fixed region, and
+//    rebuilds and scales the lattice points;
+//  * the inverse FWHT runs in registers (two stages across the four lanes by
+//    shuffle), followed by the sign flip and 16-byte stores.
+// Chunks are independent (their offsets are given), so there is no look-back.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hq_device.cuh"
+
+namespace hq {
+
+namespace {
+
+constexpr int kStagePad = 4;   // zero words after a staged chunk: unchecked 2-word reads stay inside
+
+// 32 bits of a plane of `n` words starting at bit `b`; words at or past n read as 0.
+__device__ __forceinline__ uint32_t fetch32_checked(const uint32_t *p, uint32_t n, uint32_t b) {
+    const uint32_t w = b >> 5;
+    const uint32_t a0 = (w < n) ? p[w] : 0u;
+    const uint32_t a1 = (w + 1 < n) ? p[w + 1] : 0u;
+    return __funnelshift_r(a0, a1, b & 31u);
+}
+
+// The same from a staged chunk: the stage is zero-padded after the chunk and
+// the word index is clamped to the plane's end, so both reads stay inside.
+__device__ __forceinline__ uint32_t fetch32_staged(const uint32_t *p, uint32_t n, uint32_t b) {
+    const uint32_t w = min(b >> 5, n);
+    return __funnelshift_r(p[w], p[w + 1], b & 31u);
+}
+
+template <bool STAGED>
+__device__ __forceinline__ uint32_t fetch32(const uint32_t *p, uint32_t n, uint32_t b) {
+    return STAGED ? fetch32_staged(p, n, b) : fetch32_checked(p, n, b);
+}
+
+// Bit index of the n-th (0-based) set bit of w (n < popc(w)): binary search on
+// popcounts of the low halves, branch-free.
+__device__ __forceinline__ uint32_t select_bit(uint32_t w, uint32_t n) {
+    uint32_t pos = 0, c;
+    c = __popc(w & 0xFFFFu); if (n >= c) { n -= c; pos += 16; w >>= 16; }
+    c = __popc(w & 0xFFu);   if (n >= c) { n -= c; pos += 8;  w >>= 8; }
+    c = __popc(w & 0xFu);    if (n >= c) { n -= c; pos += 4;  w >>= 4; }
+    c = __popc(w & 0x3u);    if (n >= c) { n -= c; pos += 2;  w >>= 2; }
+    c = w & 1u;              if (n >= c) { pos += 1; }
+    return pos;
+}
+
+// Slow path of the unary reader: 4 quotients read one terminator at a time
+// (quotients may exceed the 32-bit window).  Out of line: rare.  Returns the
+// new bit position; *ok turns false if the plane ends early.
+__device__ __noinline__ uint32_t unary_slow(const uint32_t *un, uint32_t nu, uint32_t bp, bool *ok, uint32_t *q) {
+    const uint32_t nbits = nu * 32u;
+    for (int i = 0; i < 4; i++) {
+        uint32_t t = 0;
+        uint32_t x = __brev(fetch32_checked(un, nu, bp));
+        while (x == 0u && *ok) {
+            t += 32u;
+            bp += 32u;
+            if (bp >= nbits) *ok = false;
+            x = __brev(fetch32_checked(un, nu, bp));
+        }
+        const uint32_t c = __clz(x);
+        q[i] = t + c;
+        bp += c + 1u;
+    }
+    return bp;
+}
+
+// Quotients of 4 symbols from bit bp of the unary plane: the next 32 stream
+// bits bit-reversed (first bit at the MSB); if they hold 4 terminators each
+// quotient is a count-leading-zeros, else the slow path.
+template <bool STAGED>
+__device__ __forceinline__ void unary4(const uint32_t *un, uint32_t nu, uint32_t &bp, bool &ok, uint32_t *q) {
+    uint32_t w = __brev(fetch32<STAGED>(un, nu, bp));
+    if (__popc(w) >= 4) {
+        uint32_t used = 4;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const uint32_t t = __clz(w);
+            q[i] = t;
+            used += t;
+            w = (w << t) << 1;
+        }
+        bp += used;
+    } else {
+        uint32_t tmp[4];
+        bp = unary_slow(un, nu, bp, &ok, tmp);
+#pragma unroll
+        for (int i = 0; i < 4; i++) q[i] = tmp[i];
+    }
+}
+
+// k-bit remainders of group g (8 symbols) from the lane's region `rw` (k words per
+// 32 symbols), for k > 4: one bounded read per symbol.
+__device__ __forceinline__ void rem_group(const uint32_t *rw, int k, int g, uint32_t (&r)[8]) {
+    const uint32_t n = (uint32_t)k;
+    const uint32_t mask = (1u << k) - 1u;
+    const uint32_t b = (uint32_t)(8 * g) * (uint32_t)k;
+#pragma unroll
+    for (int i = 0; i < 8; i++) r[i] = fetch32_checked(rw, n, b + (uint32_t)(i * k)) & mask;
+}
+
+// The four 32-bit remainder windows of a lane (k <= 4: group g's 8k bits start at
+// bit 8gk of the lane's k words), read once: k loads instead of eight, and no
+// bank conflicts between lanes whose regions are k words apart.
+__device__ __forceinline__ void rem_windows(const uint32_t *rw, int k, uint32_t (&x)[4]) {
+    switch (k) {
+    case 1: {
+        const uint32_t w0 = rw[0];
+        x[0] = w0; x[1] = w0 >> 8; x[2] = w0 >> 16; x[3] = w0 >> 24;
+        break;
+    }
+    case 2: {
+        const uint32_t w0 = rw[0], w1 = rw[1];
+        x[0] = w0; x[1] = __funnelshift_r(w0, w1, 16); x[2] = w1; x[3] = w1 >> 16;
+        break;
+    }
+    case 3: {
+        const uint32_t w0 = rw[0], w1 = rw[1], w2 = rw[2];
+        x[0] = w0; x[1] = __funnelshift_r(w0, w1, 24); x[2] = __funnelshift_r(w1, w2, 16); x[3] = w2 >> 8;
+        break;
+    }
+    default: {
+        x[0] = rw[0]; x[1] = rw[1]; x[2] = rw[2]; x[3] = rw[3];
+        break;
+    }
+    }
+}
+
+// Where the tiles of one chunk go (computed once per chunk).
+template <bool KV>
+struct ChunkOut {
+    int ntiles;
+    float e_scale;
+    long long row0, h, tok_base, tok0;
+    int tc0, tpr;
+
+    __device__ __forceinline__ void init(const DecodeArgs &a, unsigned long long c) {
+        if (KV) {
+            // the append that holds global chunk c (binary search on first_chunk)
+            unsigned long long lo = 0, hi = a.n_appends - 1;
+            while (lo < hi) {
+                const unsigned long long mid = (lo + hi + 1) >> 1;
+                if (a.table[mid].first_chunk <= c) lo = mid; else hi = mid - 1;
+            }
+            const hq_kv_append_row row = a.table[lo];
+            const long long T = row.tokens, cph = (T + 31) / 32;
+            const long long lc = (long long)(c - row.first_chunk);
+            h = lc / cph;
+            tok_base = (lc % cph) * 32;
+            tok0 = row.token0;
+            const long long left = T - tok_base;
+            ntiles = (int)(left < 32 ? left : 32);
+            e_scale = row.scale_inv;
+        } else {
+            tpr = (int)(a.map.cols / kTile);
+            const long long t0 = (long long)c * 32, all = a.map.rows * (long long)tpr;
+            ntiles = (int)((all - t0) < 32 ? (all - t0) : 32);
+            row0 = t0 / tpr;
+            tc0 = (int)(t0 - row0 * tpr);
+            e_scale = a.e_scale;
+        }
+    }
+    // Tile ti of the chunk: destination of its element 0 (null if not stored), sign
+    // column, dither counter of element 0, and its position for dot-product outputs
+    // (weights: row * tiles per row + tile column; KV: the token, or -1 past len).
+    __device__ __forceinline__ bool tile(const DecodeArgs &a, int ti, char *&dst, int &tcol,
+                                         unsigned long long &e0, long long &pos) const {
+        dst = nullptr;
+        pos = -1;
+        if (ti >= ntiles) return false;
+        const size_t esz = a.out_fp32 ? 4 : 2;
+        if (KV) {
+            const long long gt = tok0 + tok_base + ti;
+            tcol = 0;
+            e0 = (unsigned long long)((gt * a.map.heads + h) * kTile);
+            if (gt < a.len) {
+                pos = gt;
+                if (a.out) dst = (char *)a.out + (size_t)(h * a.out_ld_head + gt * a.out_ld) * esz;
+            }
+            return true;
+        }
+        int tc = tc0 + ti;
+        long long r = row0;
+        if (tc >= tpr) {
+            const int d = tc / tpr;
+            r += d;
+            tc -= d * tpr;
+        }
+        tcol = tc;
+        e0 = (unsigned long long)(r * a.map.cols + (long long)tc * kTile);
+        pos = r * tpr + tc;
+        if (a.out) dst = (char *)a.out + (size_t)(r * a.out_ld + (long long)tc * kTile) * esz;
+        return true;
+    }
+};
+
+// Valid word range of chunk c, or nw = 0 if the offsets are not consistent.
+struct ChunkWords {
+    unsigned long long w0, nw;
+    bool ok;
+};
+
+__device__ __forceinline__ ChunkWords chunk_words(const DecodeArgs &a, unsigned long long c) {
+    ChunkWords r;
+    r.w0 = a.offsets[c];
+    const unsigned long long w1 = a.offsets[c + 1];
+    r.ok = r.w0 <= w1 && w1 <= a.stream_words;
+    r.nw = r.ok ? w1 - r.w0 : 0ull;
+    return r;
+}
+
+// Start the copy of a chunk's words into a stage (cp.async, 4 bytes per lane and
+// step) and zero the pad after them; one commit group per call.
+__device__ __forceinline__ void stage_chunk(const DecodeArgs &a, const ChunkWords &cw, uint32_t *stage, int lane) {
+    if (cw.nw <= (unsigned long long)kStageWords) {
+        const uint32_t n = (uint32_t)cw.nw;
+        const uint32_t *src = a.stream + cw.w0;
+        for (uint32_t i = lane; i < n; i += 32) {
+            const unsigned sa = (unsigned)__cvta_generic_to_shared(stage + i);
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(src + i) : "memory");
+        }
+        if (lane < kStagePad) stage[n + lane] = 0u;
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// First unary bit of every 32-symbol segment of a chunk (startbit[s]): the
+// lanes split the unary plane into 32 word ranges, count terminators (popc),
+// scan, and each lane locates the segment boundaries that fall in its range.
+// Returns false (chunk corrupt) unless the plane holds exactly nsym terminators.
+__device__ __forceinline__ bool find_segment_starts(const uint32_t *un, uint32_t nu, uint32_t nsym, uint32_t nseg,
+                                                    bool ok, uint32_t *startbit, int lane) {
+    const uint32_t seg = (nu + 31u) / 32u;
+    const uint32_t s0 = min(nu, (uint32_t)lane * seg), s1 = min(nu, s0 + seg);
+    uint32_t cnt = 0;
+    for (uint32_t i = s0; i < s1; i++) cnt += __popc(un[i]);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    const uint32_t ones = __shfl_sync(0xffffffffu, incl, 31);
+    ok = ok && ones == nsym;
+    if (ok) {
+        const uint32_t before = incl - cnt;
+        // terminator j = 32 s - 1 closes segment s - 1; find those inside [before, incl)
+        uint32_t ss = (before + 1u + 31u) / 32u;
+        if (ss == 0) ss = 1;
+        uint32_t i = s0, seen = before;
+        for (; ss < nseg && 32u * ss - 1u < incl; ss++) {
+            const uint32_t j = 32u * ss - 1u;
+            uint32_t w = un[i], pc = __popc(w);
+            while (seen + pc <= j) {
+                seen += pc;
+                i++;
+                w = un[i];
+                pc = __popc(w);
+            }
+            startbit[ss] = i * 32u + select_bit(w, j - seen) + 1u;
+        }
+        if (lane == 0) startbit[0] = 0;
+    }
+    __syncwarp();
+    return ok;
+}
+
+// The 4 rounds of one chunk, reading its planes from `src` (a stage when STAGED).
+// Dot product of a lane's 32 decoded values (bf16-rounded, signs applied: exactly the
+// stored bf16 tile) with 32 bf16 values of v: sequential fma in element order (the
+// products of two bf16 values are exact in fp32).
+__device__ __forceinline__ float lane_dot(const uint32_t (&w)[16], const uint16_t *v) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const uint4 x = ldg_nc_v4(v + 8 * j);
+        const uint32_t xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int t = 0; t < 4; t++) {
+            const uint32_t ww = w[4 * j + t];
+            acc = __fmaf_rn(__uint_as_float(ww << 16), __uint_as_float(xv[t] << 16), acc);
+            acc = __fmaf_rn(__uint_as_float(ww & 0xFFFF0000u), __uint_as_float(xv[t] & 0xFFFF0000u), acc);
+        }
+    }
+    return acc;
+}
+
+// Sum over the four lanes of a tile, the same in all four: (a0 + a1) + (a2 + a3).
+__device__ __forceinline__ float tile_sum(float acc) {
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 1));
+    return __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
+}
+
+template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED, int MODE>
+__device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOut<KV> &geo, const uint32_t *src,
+                                              bool ok, uint32_t nc, uint32_t nr, uint32_t nu,
+                                              const uint32_t *startbit, const uint32_t *sign_tab, int lane) {
+    using L = Lattice<LAT>;
+    constexpr int N = L::N;
+    const int k = a.k;
+    const int q = lane & 3;
+    const uint32_t *un = src + nc + nr;
+    const float2 e2 = make_float2(geo.e_scale, geo.e_scale);
+    const uint32_t pk = 1u << k;   // quotient weight 2^k
+    bool bad = false;
+    const int nrounds = (geo.ntiles + kTilesPerRound - 1) / kTilesPerRound;
+#pragma unroll 1
+    for (int r = 0; r < nrounds; r++) {
+        char *dst = nullptr;
+        int tcol = 0;
+        unsigned long long e0 = 0;
+        long long pos = -1;
+        const bool valid = geo.tile(a, r * kTilesPerRound + (lane >> 2), dst, tcol, e0, pos);
+        const uint32_t segi = 32u * r + lane;
+        float2 v[16];
+        bool lane_ok = ok;
+        if (ok && valid) {
+            uint32_t bp = startbit[segi];
+            const uint32_t *rw = src + nc + segi * (uint32_t)k;
+            uint32_t rx[4] = {0u, 0u, 0u, 0u};
+            if (KSMALL && k > 0) rem_windows(rw, k, rx);
+            const uint32_t cw = (LAT == HQ_E8) ? src[4 * r + (lane >> 3)] : 0u;
+            const uint32_t coset = (cw >> (4 * (lane & 7))) & 0xFu;
+            const unsigned long long eq = e0 + 32ull * q;
+#pragma unroll
+            for (int g = 0; g < 4; g++) {
+                uint32_t qv[8], rv[8];
+                unary4<STAGED>(un, nu, bp, lane_ok, qv);
+                unary4<STAGED>(un, nu, bp, lane_ok, qv + 4);
+                if (KSMALL) {
+                    const uint32_t mask = (1u << k) - 1u;
+                    uint32_t xw = rx[g];
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        rv[i] = xw & mask;
+                        xw >>= k;
+                    }
+                } else {
+                    rem_group(rw, k, g, rv);
+                }
+                float u[8];
+#pragma unroll
+                for (int bb = 0; bb < 8 / N; bb++) {
+                    const int b = g * (8 / N) + bb;
+                    int32_t qq[N];
+                    float p[N];
+                    if constexpr (LAT == HQ_E8) {
+                        uint32_t zb[8];
+#pragma unroll
+                        for (int i = 0; i < 8; i++) zb[i] = imad(qv[bb * N + i], pk, rv[bb * N + i]);
+                        e8_codes_from_symbols(zb, (coset >> b) & 1u, qq);
+                    } else {
+                        int32_t m[N];
+#pragma unroll
+                        for (int i = 0; i < N; i++) m[i] = unzigzag(imad(qv[bb * N + i], pk, rv[bb * N + i]));
+                        L::reinsert(m, (coset >> b) & 1u, qq);
+                    }
+                    L::point(qq, p);
+                    if (DITHER) {
+                        float d[N];
+                        dither_block<LAT>(a.seed, eq + (unsigned long long)(8 * g + bb * N), d);
+#pragma unroll
+                        for (int i = 0; i < N; i++) p[i] = __fsub_rn(p[i], d[i]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < N; i++) u[bb * N + i] = p[i];
+                }
+#pragma unroll
+                for (int j = 0; j < 4; j++) v[4 * g + j] = f2_mul(make_float2(u[2 * j], u[2 * j + 1]), e2);
+            }
+            if (bp > nu * 32u) lane_ok = false;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; j++) v[j] = make_float2(0.0f, 0.0f);
+        }
+        if (valid && !lane_ok) bad = true;
+        fwht128_quarter(v, lane);
+        // a tile is written as zeros unless all four of its lanes decoded
+        const unsigned bad_lanes = __ballot_sync(0xffffffffu, valid && !lane_ok);
+        const bool tile_bad = (bad_lanes >> (lane & ~3)) & 0xFu;
+        if constexpr (MODE != kStoreTiles) {
+            // the tile as hq_dequantize stores it in bf16, then dot products with the vector(s)
+            const uint32_t es = sign_tab[tcol * kSignWords + q];
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+                __nv_bfloat162 hb = __floats2bfloat162_rn(v[j].x, v[j].y);
+                w[j] = tile_bad ? 0u : (*reinterpret_cast<uint32_t *>(&hb) ^ sign_pair_mask(es, j));
+            }
+            if constexpr (MODE == kGemvPartials) {
+                const float acc = tile_sum(valid ? lane_dot(w, a.vec + (long long)tcol * kTile + 32 * q) : 0.0f);
+                if (valid && q == 0) a.res[pos] = acc;
+            } else {
+                // every query head of the KV head's group; a tile past len (pos < 0) only joins the shuffles
+                for (int gq = 0; gq < a.group; gq++) {
+                    const long long qh = geo.h * a.group + gq;
+                    const float acc = tile_sum(pos >= 0 ? lane_dot(w, a.vec + qh * kTile + 32 * q) : 0.0f);
+                    if (pos >= 0 && q == 0) a.res[qh * a.out_ld + pos] = acc;
+                }
+            }
+        } else if (dst) {
+            const uint32_t es = sign_tab[tcol * kSignWords + q];
+            if (a.out_fp32) {
+                uint4 *o = reinterpret_cast<uint4 *>(dst) + 8 * q;
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const uint32_t m0 = sign_pair_mask(es, 2 * j), m1 = sign_pair_mask(es, 2 * j + 1);
+                    uint4 w;
+                    w.x = tile_bad ? 0u : __float_as_uint(v[2 * j].x) ^ (m0 << 16);
+                    w.y = tile_bad ? 0u : __float_as_uint(v[2 * j].y) ^ (m0 & 0x80000000u);
+                    w.z = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].x) ^ (m1 << 16);
+                    w.w = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].y) ^ (m1 & 0x80000000u);
+                    o[j] = w;
+                }
+            } else {
+                uint4 *o = reinterpret_cast<uint4 *>(dst) + 4 * q;
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int u2 = 0; u2 < 4; u2++) {
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(v[4 * j + u2].x, v[4 * j + u2].y);
+                        pk[u2] = tile_bad ? 0u : (*reinterpret_cast<uint32_t *>(&hb) ^ sign_pair_mask(es, 4 * j + u2));
+                    }
+                    o[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+        }
+    }
+    return bad;
+}
+
+// Three CTAs (24 warps) per SM without dither, where the decoder fits 80 registers with
+// almost no spills; two with dither, whose second lattice search needs more.
+template <int LAT, bool DITHER, bool KV, bool KSMALL, int MODE>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, DITHER ? 2 : 3) decode_kernel(const DecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    constexpr int kStageSlot = kStageWords + kStagePad;
+    uint32_t *sign_tab = smem;
+    uint32_t *stage_all = smem + a.tcols * kSignWords;
+    uint32_t *start_all = stage_all + kWarpsPerCta * 2 * kStageSlot;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t *stages = stage_all + warp * 2 * kStageSlot;
+    uint32_t *startbit = start_all + warp * 128;   // first unary bit of every 32-symbol segment
+
+    build_sign_table(sign_tab, a.tcols, a.seed);
+    __syncthreads();
+
+    const int k = a.k;
+    uint32_t status = 0;
+    const unsigned long long nwarps = (unsigned long long)gridDim.x * kWarpsPerCta;
+    unsigned long long c = (unsigned long long)blockIdx.x * kWarpsPerCta + warp;
+    int buf = 0;
+    ChunkWords cw = {0, 0, false};
+    if (c < a.n_chunks) {
+        cw = chunk_words(a, c);
+        stage_chunk(a, cw, stages, lane);
+    }
+    for (; c < a.n_chunks; c += nwarps, buf ^= 1) {
+        // start bringing in the next chunk while this one is decoded
+        const unsigned long long cn = c + nwarps;
+        ChunkWords cwn = {0, 0, false};
+        if (cn < a.n_chunks) {
+            cwn = chunk_words(a, cn);
+            stage_chunk(a, cwn, stages + (buf ^ 1) * kStageSlot, lane);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncwarp();
+
+        ChunkOut<KV> geo;
+        geo.init(a, c);
+        const int ntiles = geo.ntiles;
+        const uint32_t nsym = (uint32_t)ntiles * kTile, nseg = 4u * (uint32_t)ntiles;
+        const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
+        const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
+        bool ok = cw.ok && cw.nw >= (unsigned long long)(nc + nr) &&
+                  (cw.nw - nc - nr) < (unsigned long long)(kMaxUnaryBits / 32u);
+        const bool staged = cw.nw <= (unsigned long long)kStageWords;
+        const uint32_t nu = ok ? (uint32_t)(cw.nw - nc - nr) : 0u;
+        // the staged and in-place paths get distinct pointer expressions so the
+        // staged one keeps its shared-memory address space after inlining
+        bool bad;
+        if (staged) {
+            const uint32_t *src = stages + buf * kStageSlot;
+            ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, true, MODE>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab, lane);
+        } else {
+            const uint32_t *src = a.stream + cw.w0;
+            ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, false, MODE>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab, lane);
+        }
+        if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) status |= HQ_ST_CORRUPT;
+        cw = cwn;
+        __syncwarp();
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (a.stats) {
+        status = __reduce_or_sync(0xffffffffu, status);
+        if (lane == 0 && status) atomicOr(&a.stats->status, status);
+    }
+}
+
+}  // namespace
+}  // namespace hq

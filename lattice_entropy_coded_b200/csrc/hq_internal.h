@@ -75,7 +75,14 @@ struct DecodeArgs {
     uint64_t n_appends;
     hq_stats *stats;
     int tcols;
+    // dot-product outputs (hq_gemv, hq_kv_scores) instead of stored tiles
+    const uint16_t *vec;      // bf16 x [cols] (gemv) or queries [heads * group, 128] (scores)
+    float *res;               // gemv: one partial per tile [rows * tcols]; scores: [heads * group, out_ld]
+    int group;                // scores: query heads per KV head
 };
+
+// Decoder outputs: the tile itself, its dot product with x, or its dot products with queries.
+enum DecodeMode { kStoreTiles = 0, kGemvPartials = 1, kKvScores = 2 };
 
 // Persistent-grid size of one kernel on the current device: SM count x resident CTAs per SM at
 // `smem` dynamic shared bytes, capped at `want` CTAs.  The shared-memory attribute and the
@@ -125,6 +132,10 @@ extern int g_encode_path;
 // Launchers (defined in hq_encode.cu / hq_decode.cu).  Return cudaSuccess or the launch error.
 cudaError_t launch_encode(int lattice, int dither, const EncodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode(int lattice, int dither, const DecodeArgs &a, cudaStream_t s);
+// hq_gemv: per-tile partials into a.res, then y[r] = sum of row r's partials in column order.
+cudaError_t launch_gemv(int lattice, int dither, const DecodeArgs &a, float *y, cudaStream_t s);
+// hq_kv_scores: a.res[(h * group + g) * out_ld + t] for every cached token t < len.
+cudaError_t launch_kv_scores(int lattice, int dither, const DecodeArgs &a, cudaStream_t s);
 // Rate only: adds payload_bits, stream_words, max_symbol and HQ_ST_RANGE of the call into a.stats
 // (zeroed by the caller); reads a.x, a.map, a.n_chunks, a.c_scale, a.k, a.seed, a.tcols.
 cudaError_t launch_rate(int lattice, int dither, const EncodeArgs &a, cudaStream_t s);
