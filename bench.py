@@ -439,6 +439,28 @@ def run_bulk(args):
             st = hq.read_stats(cache.stats)
             n = src.numel()
             words = int(cache.tail[(len(slices)) & 1].item())
+            # attention scores of 4 query heads per KV head straight from the compressed cache,
+            # against reading the cache to bf16 and multiplying
+            G = 4
+            qh = (torch.randn(H * G, 128, device=device) * 0.1).to(torch.bfloat16)
+            sc = torch.empty(H * G, T, device=device)
+            sc_ms, rd_ms = [], []
+            for it in range(args.warmup + args.steps):
+                flush.fill_(it)
+                s0, s1 = _events()
+                s0.record()
+                cache.scores(qh, G, sc)
+                s1.record()
+                flush.fill_(it + 0.5)
+                r0, r1 = _events()
+                r0.record()
+                cache.read(outb)
+                torch.matmul(outb.float(), qh.view(H, G, 128).float().transpose(1, 2))
+                r1.record()
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    sc_ms.append(s0.elapsed_time(s1))
+                    rd_ms.append(r0.elapsed_time(r1))
             # the same appends captured once in a CUDA graph and replayed: device time
             # without the per-call host work (Python, argument checks, launch calls)
             graph = torch.cuda.CUDAGraph()
@@ -471,6 +493,8 @@ def run_bulk(args):
                             graph_append_ms=float(np.median(graph_ms)),
                             graph_append_gbs=2.0 * n / (float(np.median(graph_ms)) * 1e6),
                             graph_stream_words_match=graph_words == words,
+                            scores_ms=float(np.median(sc_ms)), read_then_matmul_ms=float(np.median(rd_ms)),
+                            scores_query_heads=H * G,
                             append_hbm_frac=alg / (am * 1e6) / peak, read_hbm_frac=alg / (rm * 1e6) / peak))
         out["points"] = res
     else:
@@ -575,6 +599,27 @@ def run_case(args):
         c.record()
         if i >= args.warmup:
             ev.append((a, b, c))
+    # decode fused into a GEMV vs decode then GEMV vs a plain bf16 GEMV on the uncompressed matrix
+    comp = codec.quantize(x)
+    xv = (torch.randn(cols, device=device) * 0.5).to(torch.bfloat16)
+    y = torch.empty(rows, device=device)
+    gev = {"fused": [], "decode_then_gemv": [], "bf16_gemv": []}
+    for i in range(args.warmup + args.steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        evs[0].record()
+        codec.gemv(comp, xv, y)
+        evs[1].record()
+        evs[2].record()
+        codec.dequantize(comp, out)
+        torch.mv(out, xv)
+        evs[3].record()
+        evs[4].record()
+        torch.mv(x, xv)
+        evs[5].record()
+        if i >= args.warmup:
+            gev["fused"].append((evs[0], evs[1]))
+            gev["decode_then_gemv"].append((evs[2], evs[3]))
+            gev["bf16_gemv"].append((evs[4], evs[5]))
     rst = hq.stats_tensor(device)
     rev = []
     for i in range(args.warmup + args.steps):
@@ -587,6 +632,7 @@ def run_case(args):
     torch.cuda.synchronize()
     st = hq.read_stats(codec.stats)
     rate_ms = float(np.median([a.elapsed_time(b) for a, b in rev]))
+    gemv_ms = {k: float(np.median([a.elapsed_time(b) for a, b in v])) for k, v in gev.items()}
     assert hq.read_stats(rst)["payload_bits"] == st["payload_bits"]
     enc = float(np.median([a.elapsed_time(b) for a, b, _ in ev]))
     dec = float(np.median([b.elapsed_time(c) for _, b, c in ev]))
@@ -598,7 +644,10 @@ def run_case(args):
                       "status": st["status"], "bps_payload": st["payload_bits"] / n,
                       "enc_ms": enc, "dec_ms": dec, "enc_gbs_in": 2.0 * n / enc / 1e6, "dec_gbs_in": 2.0 * n / dec / 1e6,
                       "enc_frac": alg / enc / 1e6 / peak, "dec_frac": alg / dec / 1e6 / peak,
-                      "alg_bytes": alg, "rate_ms": rate_ms, "rate_gbs_in": 2.0 * n / rate_ms / 1e6}), flush=True)
+                      "alg_bytes": alg, "rate_ms": rate_ms, "rate_gbs_in": 2.0 * n / rate_ms / 1e6,
+                      "gemv_ms": gemv_ms,
+                      "gemv_read_bytes": {"fused": 4.0 * words + 8.0 * (codec.n_chunks + 1) + 2.0 * cols,
+                                          "bf16_gemv": 2.0 * n + 2.0 * cols}}), flush=True)
 
 
 # ------------------------------------------------------------------ main
