@@ -32,6 +32,7 @@ def path(request):
 def test_small_matrices(path, lat, dither):
     P.test_weights_bit_exact_small(lat, dither, (37, 384))
     P.test_weights_bit_exact_small(lat, dither, (64, 4096))
+    P.test_weights_bit_exact_small(lat, dither, (3, 65536))    # the widest rows (512 tile columns)
 
 
 @pytest.mark.parametrize("k", [0, 3, 8, 15])
