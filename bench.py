@@ -294,15 +294,23 @@ def run_e2e(args, hq, codecs, pts, rows, cols, device, stream, world):
     host_out = [torch.empty(rows, cols, dtype=torch.bfloat16).pin_memory() for _ in pts]
     host_stats = [torch.empty(32, dtype=torch.uint8).pin_memory() for _ in pts]
     dev_x = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
-    dev_out = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
+    dev_out = [torch.empty(rows, cols, dtype=torch.bfloat16, device=device) for _ in pts]
+    # device-to-host copies on their own stream, so point i's copy overlaps point i+1's codec work
+    copy_stream = torch.cuda.Stream(device)
+    done = [torch.cuda.Event() for _ in pts]
 
     def step():
         dev_x.copy_(host_x, non_blocking=True)
         for i, c in enumerate(codecs):
             comp = c.quantize(dev_x)
-            c.dequantize(comp, dev_out)
-            host_out[i].copy_(dev_out, non_blocking=True)
-            host_stats[i].copy_(c.stats, non_blocking=True)
+            c.dequantize(comp, dev_out[i])
+            done[i].record(stream)
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(done[i])
+                host_out[i].copy_(dev_out[i], non_blocking=True)
+                host_stats[i].copy_(c.stats, non_blocking=True)
+        # the step ends when its copies have landed (and the next step may reuse the buffers)
+        stream.wait_stream(copy_stream)
 
     for _ in range(max(1, args.warmup)):
         step()
