@@ -355,11 +355,12 @@ HQ_API int hq_device_check(void);
 HQ_API void hq_debug_set_spin_limit(uint32_t polls);
 
 /* Testing aid: which form of the quantize kernel runs.  0 (default) chooses by
- * size: launches of at most 592 chunks (one wave of four-warp chunk groups on a
- * B200) use the grouped form, where four warps share a chunk (lower latency);
- * larger ones the per-warp form, where a warp encodes whole chunks (higher
- * throughput).  1 forces per-warp, 2 forces grouped.  Both give identical
- * streams, offsets and stats.  Process-wide; HQ_EINVAL outside 0..2. */
+ * size: launches of at most 296 chunks use the wide form (16 warps share a
+ * chunk, 16 lanes per tile: the lowest latency), of at most 592 the grouped form
+ * (4 warps share a chunk), larger ones the per-warp form (a warp encodes whole
+ * chunks: the highest throughput); the limits are one wave of chunk groups on a
+ * B200.  1 forces per-warp, 2 grouped, 3 wide.  All give identical streams,
+ * offsets and stats.  Process-wide; HQ_EINVAL outside 0..3. */
 HQ_API int hq_debug_set_encode_path(int path);
 
 /* Testing aid: the nearest point of the lattice in its integer embedding

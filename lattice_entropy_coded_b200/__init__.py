@@ -230,7 +230,7 @@ def hq_calibrate_kv(kv: torch.Tensor, params: hq_params, spec: hq_calib_spec, st
 
 
 def hq_debug_set_encode_path(path: int) -> int:
-    """0 = by size, 1 = per-warp encoder, 2 = grouped encoder (testing aid)."""
+    """0 = by size, 1 = per-warp, 2 = grouped, 3 = wide encoder (testing aid)."""
     return _check(_lib.hq_debug_set_encode_path(int(path)), "hq_debug_set_encode_path")
 
 

@@ -549,7 +549,7 @@ int hq_device_check(void) {
 void hq_debug_set_spin_limit(uint32_t polls) { g_spin_limit = polls ? polls : kSpinLimit; }
 
 int hq_debug_set_encode_path(int path) {
-    if (path < 0 || path > 2) return HQ_EINVAL;
+    if (path < 0 || path > 3) return HQ_EINVAL;
     hq::g_encode_path = path;
     return HQ_OK;
 }

@@ -167,9 +167,10 @@ struct ChunkOut {
             }
             const hq_kv_append_row row = a.table[lo];
             const long long T = row.tokens, cph = (T + 31) / 32;
-            const long long lc = (long long)(c - row.first_chunk);
-            h = lc / cph;
-            tok_base = (lc % cph) * 32;
+            unsigned long long hq_, rq;
+            divmod_u64(c - row.first_chunk, (unsigned long long)cph, hq_, rq);
+            h = (long long)hq_;
+            tok_base = (long long)rq * 32;
             tok0 = row.token0;
             const long long left = T - tok_base;
             ntiles = (int)(left < 32 ? left : 32);
@@ -178,8 +179,10 @@ struct ChunkOut {
             tpr = (int)(a.map.cols / kTile);
             const long long t0 = (long long)c * 32, all = a.map.rows * (long long)tpr;
             ntiles = (int)((all - t0) < 32 ? (all - t0) : 32);
-            row0 = t0 / tpr;
-            tc0 = (int)(t0 - row0 * tpr);
+            unsigned long long rq, cq;
+            divmod_u64((unsigned long long)t0, (unsigned long long)tpr, rq, cq);
+            row0 = (long long)rq;
+            tc0 = (int)cq;
             e_scale = a.e_scale;
         }
     }

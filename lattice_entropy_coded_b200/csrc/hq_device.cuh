@@ -118,6 +118,42 @@ __device__ __forceinline__ void fwht128_quarter(float2 (&v)[16], int lane) {
     }
 }
 
+// The same transform with sixteen lanes per tile (two tiles per warp): lane l of
+// its half-warp holds elements [8l, 8l + 8) as 4 float2.  Stages 1, 2, 4 are inside
+// the lane (stage 1 inside each float2, 2 and 4 packed); stages 8, 16, 32, 64 pair
+// lane l with l ^ 1, 2, 4, 8 by shuffle, with the same exact fma(+-1, x, y).  The
+// butterflies and their order are those of fwht128_quarter, element for element.
+__device__ __forceinline__ void fwht128_sixteenth(float2 (&v)[4], int lane) {
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const float a = v[j].x, b = v[j].y;
+        v[j] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+#pragma unroll
+    for (int hp = 1; hp < 4; hp <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            if ((j & hp) == 0) {
+                const float2 a = v[j], b = v[j + hp];
+                v[j] = f2_add(a, b);
+                v[j + hp] = f2_sub(a, b);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 1; m <= 8; m <<= 1) {
+        const float sg = (lane & m) ? -1.0f : 1.0f;
+        const float2 s2 = make_float2(sg, sg);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            float2 y;
+            y.x = __shfl_xor_sync(0xffffffffu, v[j].x, m);
+            y.y = __shfl_xor_sync(0xffffffffu, v[j].y, m);
+            v[j] = f2_fma(s2, v[j], y);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ lattices
 // Rounding without the conversion pipe: for |x| < 2^22, x + 1.5*2^23 lands in
 // [2^23, 2^24) where the fp32 spacing is 1, so the add rounds x to the nearest
@@ -440,6 +476,21 @@ __device__ __forceinline__ void dither_block<HQ_Z>(uint64_t seed, uint64_t e, fl
     uint32_t r24 = (e & 1ull) ? ((uint32_t)h >> 8) : (uint32_t)(h >> 40);
     float w = __fmul_rn((float)r24, 0x1p-24f);
     d[0] = __fsub_rn(w, (float)rint_int(w));
+}
+
+// ------------------------------------------------------------------ integer helpers
+// q = a / b, r = a % b (b > 0) with one 32-bit division when both fit, which is the
+// usual case for chunk and tile counts; the 64-bit division otherwise.
+__device__ __forceinline__ void divmod_u64(unsigned long long a, unsigned long long b, unsigned long long &q,
+                                           unsigned long long &r) {
+    if (((a | b) >> 32) == 0) {
+        const uint32_t qq = (uint32_t)a / (uint32_t)b;
+        q = qq;
+        r = (uint32_t)a - qq * (uint32_t)b;
+    } else {
+        q = a / b;
+        r = a - q * b;
+    }
 }
 
 // ------------------------------------------------------------------ memory helpers

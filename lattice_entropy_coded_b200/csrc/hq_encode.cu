@@ -108,9 +108,11 @@ struct ChunkGeo {
 
     __device__ __forceinline__ void init(const TileMap &m, unsigned long long c) {
         if (m.kv) {
-            long long cph = (m.tokens + 31) / 32;
-            h = (long long)c / cph;
-            tok_base = ((long long)c % cph) * 32;
+            const long long cph = (m.tokens + 31) / 32;
+            unsigned long long hq_, rq;
+            divmod_u64(c, (unsigned long long)cph, hq_, rq);
+            h = (long long)hq_;
+            tok_base = (long long)rq * 32;
             long long left = m.tokens - tok_base;
             ntiles = (int)(left < 32 ? left : 32);
         } else {
@@ -118,8 +120,10 @@ struct ChunkGeo {
             long long t0 = (long long)c * 32;
             long long all = m.rows * (long long)tpr;
             ntiles = (int)((all - t0) < 32 ? (all - t0) : 32);
-            row0 = t0 / tpr;
-            tc0 = (int)(t0 - row0 * tpr);
+            unsigned long long rq, cq;
+            divmod_u64((unsigned long long)t0, (unsigned long long)tpr, rq, cq);
+            row0 = (long long)rq;
+            tc0 = (int)cq;
         }
     }
     // Tile ti (< 32) of the chunk: first element, sign-table column, dither counter of its element 0.
@@ -867,16 +871,265 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel_grouped(co
     }
 }
 
+
+// ------------------------------------------------------------------ wide form
+// Latency form for the smallest launches (a KV append of a few tokens or heads, a
+// small matrix): sixteen lanes per tile, one 8-element E8 block (or 2 D4, 4 A2, 8 Z
+// blocks) per lane, so a chunk's 32 tiles are spread over 16 warps, each holding
+// two tiles.  A lane's serial work is a quarter of the grouped form's.
+constexpr int kWideWarps = kChunkTiles / 2;   // warps per chunk, two tiles each
+static_assert(kWideWarps == 16, "two tiles per warp");
+
+struct WideCtl {
+    uint32_t tot[2][kWideWarps];
+    uint32_t bad[2][kWideWarps];
+    unsigned int tk[2];
+    unsigned int first[2];
+};
+static_assert(sizeof(WideCtl) % 16 == 0, "16-byte multiple");
+
+__device__ __forceinline__ void wide_sync() {
+    asm volatile("bar.sync 1, %0;" ::"r"(kWideWarps * 32) : "memory");
+}
+
+// A lane's 8 elements of its tile: signs, FWHT-128 with its 15 partner lanes,
+// scale, [+ dither], lattice blocks -> 8 zigzag symbols and (E8) the coset bit.
+template <int LAT, bool DITHER>
+__device__ __forceinline__ void wide_symbols(const EncodeArgs &a, bool valid, int tcol, unsigned long long e0,
+                                             uint4 raw, int lane, const uint32_t *sign_tab, uint32_t (&z)[8],
+                                             uint32_t &cbit) {
+    using L = Lattice<LAT>;
+    constexpr int N = L::N;
+    const int l16 = lane & 15;
+    const uint32_t es = sign_tab[tcol * kSignWords + (l16 >> 2)];
+    const uint4 w = valid ? raw : make_uint4(0, 0, 0, 0);
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+    float2 v[4];
+#pragma unroll
+    for (int t = 0; t < 4; t++) {
+        const uint32_t ww = wv[t] ^ sign_pair_mask(es, 4 * (l16 & 3) + t);
+        v[t] = make_float2(__uint_as_float(ww << 16), __uint_as_float(ww & 0xFFFF0000u));
+    }
+    fwht128_sixteenth(v, lane);
+    const float2 c2 = make_float2(a.c_scale, a.c_scale);
+#pragma unroll
+    for (int t = 0; t < 4; t++) v[t] = f2_mul(v[t], c2);
+    const float x[8] = {v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y};
+    cbit = 0;
+    const unsigned long long eq = e0 + 8ull * l16;
+#pragma unroll
+    for (int b = 0; b < 8 / N; b++) {
+        float blk[N];
+#pragma unroll
+        for (int i = 0; i < N; i++) blk[i] = x[b * N + i];
+        if (DITHER) {
+            float d[N];
+            dither_block<LAT>(a.seed, eq + (unsigned long long)(b * N), d);
+#pragma unroll
+            for (int i = 0; i < N; i++) blk[i] = __fadd_rn(blk[i], d[i]);
+        }
+        uint32_t zz[N];
+        cbit |= L::symbols(blk, zz);
+#pragma unroll
+        for (int i = 0; i < N; i++) z[b * N + i] = (!DITHER || valid) ? zz[i] : 0u;
+    }
+    if (!valid) cbit = 0;
+}
+
+// k remainder bits of 8 symbols into the remainder plane at bit `off` (any
+// alignment: ORed into the stage, at most two words per value group).
+__device__ __forceinline__ void wide_put_rem(uint32_t *rem, uint32_t off, const uint32_t (&z)[8], int k) {
+    if (k == 0) return;
+    const uint32_t mask = (1u << k) - 1u;
+    if (k <= 4) {
+        const uint32_t pk = 1u << k;
+        uint32_t gv = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; i--) gv = imad(gv, pk, z[i] & mask);
+        const uint32_t w0 = off >> 5, sh = off & 31u;
+        atomicOr(rem + w0, gv << sh);
+        if (sh + 8u * (uint32_t)k > 32u) atomicOr(rem + w0 + 1, gv >> (32u - sh));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const uint32_t b = off + (uint32_t)(i * k), w0 = b >> 5, sh = b & 31u, val = z[i] & mask;
+            atomicOr(rem + w0, val << sh);
+            if (sh + (uint32_t)k > 32u) atomicOr(rem + w0 + 1, val >> (32u - sh));
+        }
+    }
+}
+
+// One group of 16 warps per CTA.  Per chunk: every warp encodes its two tiles; the
+// 16 warp totals meet in shared memory (barrier 1); each warp places its codewords
+// in the stage (the coset word of its 32 blocks by one ballot, remainder bits and
+// unary terminators by shared atomics); warp 0 publishes the chunk's count; one
+// warp, in turn, resolves the previous chunk's offset and copies its stage out.
+template <int LAT, bool DITHER>
+__global__ void __launch_bounds__(kWideWarps * 32, 1) encode_kernel_wide(const EncodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint32_t *sign_tab = smem;                                         // tcols * kSignWords
+    uint32_t *stages = sign_tab + a.tcols * kSignWords;                // 2 * kStageWords
+    WideCtl &ctl = *reinterpret_cast<WideCtl *>(stages + 2 * kStageWords);
+
+    build_sign_table(sign_tab, a.tcols, a.seed);
+    for (int i = threadIdx.x; i < 2 * kStageWords / 4; i += blockDim.x)
+        reinterpret_cast<uint4 *>(stages)[i] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) {
+        ctl.first[0] = atomicAdd(a.ticket, 1u);
+        ctl.first[1] = atomicAdd(a.ticket, 1u);
+    }
+    __syncthreads();
+
+    const unsigned long long n = a.n_chunks;
+    const int k = a.k;
+    const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
+    const int ti = 2 * w + (lane >> 4);          // the lane's tile in the chunk
+    uint32_t status = 0, zor_all = 0;
+    unsigned long long payload = 0;
+    unsigned long long c = ctl.first[0], cn = ctl.first[1];
+    // the next chunk's 16 bytes are loaded one iteration ahead
+    uint4 raw_next = make_uint4(0, 0, 0, 0);
+    if (c < n) {
+        ChunkGeo g0;
+        g0.init(a.map, c);
+        const uint16_t *src;
+        int tc;
+        unsigned long long e0;
+        if (g0.tile(a.map, a.x, ti, src, tc, e0)) raw_next = ldg_nc_v4(src + 8 * (lane & 15));
+    }
+    Pending pend = {0, 0, false, false};
+    bool have_pend = false;
+    int buf = 0;
+    unsigned it = 0;
+    while (true) {
+        const bool live = c < n;
+        const bool duty = w == (int)(it % kWideWarps);
+        unsigned long long first = 0;
+        if (have_pend && duty) first = lookback_peek(a.lookback, pend.c);
+        uint32_t *stage = stages + buf * kStageWords;
+        ChunkGeo geo;
+        uint32_t z[8], cbit = 0, ub = 0, incl = 0;
+        bool valid = false;
+        if (live) {
+            geo.init(a.map, c);
+            const uint16_t *src = nullptr;
+            int tcol = 0;
+            unsigned long long e0 = 0;
+            valid = geo.tile(a.map, a.x, ti, src, tcol, e0);
+            const uint4 raw = raw_next;
+            if (cn < n) {
+                ChunkGeo gn;
+                gn.init(a.map, cn);
+                const uint16_t *s2;
+                int tc2;
+                unsigned long long e2;
+                raw_next = gn.tile(a.map, a.x, ti, s2, tc2, e2) ? ldg_nc_v4(s2 + 8 * (lane & 15))
+                                                                : make_uint4(0, 0, 0, 0);
+            }
+            if (threadIdx.x == 0) ctl.tk[buf] = atomicAdd(a.ticket, 1u);
+            wide_symbols<LAT, DITHER>(a, valid, tcol, e0, raw, lane, sign_tab, z, cbit);
+            uint32_t usum = 0, lor = 0;
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                usum += z[i] >> k;
+                lor |= z[i];
+            }
+            zor_all |= lor;
+            ub = valid ? usum + 8u : 0u;   // symbols below 2^22: a warp's total stays below 2^30
+            incl = ub;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const uint32_t rzor = __reduce_or_sync(0xffffffffu, lor);
+            if (lane == 31) {
+                ctl.tot[buf][w] = incl;
+                ctl.bad[buf][w] = (rzor >> 22) != 0u ? 1u : 0u;
+            }
+        }
+        wide_sync();
+        unsigned long long total = 0;
+        bool overflow = false, range_bad = false;
+        if (live) {
+            unsigned long long before = 0, U = 0;
+            uint32_t badw = 0;
+#pragma unroll
+            for (int j = 0; j < kWideWarps; j++) {
+                const uint32_t t = ctl.tot[buf][j];
+                before += (j < w) ? t : 0u;
+                U += t;
+                badw |= ctl.bad[buf][j];
+            }
+            const int ntiles = geo.ntiles;
+            const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
+            const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
+            range_bad = badw != 0u || U >= kMaxUnaryBits;
+            total = nc + nr + (U + 31) / 32;
+            overflow = total > (unsigned long long)kStageWords;
+            if (!overflow && !range_bad) {
+                if (LAT == HQ_E8) {
+                    const uint32_t cw = __ballot_sync(0xffffffffu, cbit != 0u);
+                    if (lane == 0 && cw) stage[w] = cw;
+                }
+                if (valid) {
+                    wide_put_rem(stage + nc, (uint32_t)(32 * w + lane) * 8u * (uint32_t)k, z, k);
+                    uint32_t qg[8];
+#pragma unroll
+                    for (int i = 0; i < 8; i++) qg[i] = z[i] >> k;
+                    unary_group_shared(stage + nc + nr, (uint32_t)before + incl - ub, qg);
+                }
+            }
+            if (w == 0) {
+                lookback_publish(a.lookback, c, total);
+                if (range_bad) status |= HQ_ST_RANGE;
+                if (lane == 0) payload += U + (unsigned long long)nr * 32 + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
+            }
+        }
+        if (have_pend && duty)
+            finish_chunk<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status, first);
+        if (!live) break;
+        pend.c = c;
+        pend.total = total;
+        pend.overflow = overflow;
+        pend.range_bad = range_bad;
+        have_pend = true;
+        c = cn;
+        cn = ctl.tk[buf];
+        buf ^= 1;
+        it++;
+    }
+
+    if (a.stats) {
+        zor_all = __reduce_or_sync(0xffffffffu, zor_all);
+        status = __reduce_or_sync(0xffffffffu, status);
+        if (lane == 0) {
+            if (status) atomicOr(&a.stats->status, status);
+            if (zor_all) atomicOr(&a.stats->max_symbol, zor_all);
+            if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
+        }
+    }
+}
+
 template <int LAT, bool DITHER>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     const bool small = a.k <= 4;
     cudaError_t e;
     unsigned grid = 0;
-    // the grouped kernel when every chunk gets a group of its own in one wave
-    // (148 SMs x 2 CTAs x kGroups on a B200), else the per-warp kernel
+    // by size: the wide form while every chunk gets a 16-warp group of its own in one
+    // wave (148 SMs x 2 CTAs on a B200), the grouped form while it gets a 4-warp group
+    // (148 x 2 x kGroups), else the per-warp form
     int mode = g_encode_path;
-    if (mode == 0) mode = (a.n_chunks <= 592ull) ? 2 : 1;
-    if (mode == 2) {
+    if (mode == 0) mode = (a.n_chunks <= 296ull) ? 3 : (a.n_chunks <= 592ull) ? 2 : 1;
+    if (mode == 3) {
+        const size_t smem =
+            (size_t)(a.tcols * kSignWords + 2 * kStageWords) * sizeof(uint32_t) + sizeof(WideCtl);
+        auto kern = encode_kernel_wide<LAT, DITHER>;
+        static LaunchPlan plan;
+        if ((e = plan.grid(kern, kWideWarps * 32, smem, a.n_chunks, grid)) != cudaSuccess) return e;
+        kern<<<grid, kWideWarps * 32, smem, s>>>(a);
+    } else if (mode == 2) {
         const size_t smem = (size_t)(a.tcols * kSignWords + kGroups * 2 * kStageWords +
                                      kWarpsPerCta * 32 * kGroupSlotWords) * sizeof(uint32_t) +
                             kGroups * sizeof(GroupCtl);

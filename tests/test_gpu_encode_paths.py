@@ -19,7 +19,7 @@ from hqtest import assert_same_words, gpu_quantize, oracle_quantize, rate_points
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=[1, 2], ids=["per_warp", "grouped"])
+@pytest.fixture(params=[1, 2, 3], ids=["per_warp", "grouped", "wide"])
 def path(request):
     import lattice_entropy_coded_b200 as hq
     hq.hq_debug_set_encode_path(request.param)
