@@ -67,6 +67,24 @@ def test_gemv_matches_the_oracle_reconstruction(lat, dither, shape):
     assert np.array_equal(y.cpu().numpy(), y1)
 
 
+@pytest.mark.parametrize("k", [0, 8])
+def test_gemv_every_remainder_path(k):
+    """k = 0 (no remainder plane) and k = 8 (remainders read one by one, not in windows)."""
+    hq = _hq()
+    rows, cols = 21, 1024
+    W = synth.weight(rows, cols, seed=77)
+    alpha = 300.0 * 2 ** (k - 2) if k else 40.0
+    p = hq.make_params("E8", alpha, k, 3, 0)
+    g = gpu_quantize(W.cuda(), p, max_abs_symbol=1 << 14)
+    ref_w, ref_off, _ = oracle_quantize(W, O.E8, alpha, k, 3)
+    w_bits = oracle_dequantize(ref_w, ref_off, rows, cols, O.E8, alpha, k, 3, fp32=False)
+    x = (torch.randn(cols, generator=torch.Generator().manual_seed(k)) * 2).to(torch.bfloat16)
+    ws = torch.empty(hq.hq_gemv_workspace_bytes(rows, cols), dtype=torch.uint8, device="cuda")
+    y = torch.empty(rows, device="cuda")
+    hq.hq_gemv(g["words_t"], g["cap"], g["offsets_t"], rows, cols, p, x.cuda(), y, ws)
+    _check_dot(y.cpu().numpy(), w_bits, u16(x), cols // 128)
+
+
 def test_gemv_full_size_point_and_codec_method():
     """4096 x 4096 at the E8 4 bps point, through Codec.gemv, against dequantize + fp64 GEMV."""
     hq = _hq()
