@@ -15,9 +15,10 @@
  * ---------------------------------------
  *  - Every pointer named d_* or documented as "device" is device memory of the
  *    current CUDA device; host pointers are named h_* or documented as host.
- *  - The caller owns all memory.  The library allocates nothing and never
- *    synchronises; every call is asynchronous on the CUDA stream it is given
- *    (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *  - The caller owns all memory.  The library allocates nothing, and every call
+ *    is asynchronous on the CUDA stream it is given (a cudaStream_t passed as
+ *    void*; NULL = legacy default stream), except hq_calibrate and
+ *    hq_calibrate_kv, which wait for each of their rate passes.
  *  - A negative return value is a synchronous argument or launch error
  *    (HQ_EINVAL, HQ_EUNSUPPORTED, HQ_ECUDA); nothing was enqueued.  Errors that
  *    depend on the data are reported on the device in hq_stats.status, which

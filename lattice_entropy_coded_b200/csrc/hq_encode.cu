@@ -1,27 +1,28 @@
-// hq_encode.cu -- quantize + encode kernel (HyperQuant "Methodology" sections
+// hq_encode.cu -- quantize + encode kernels (HyperQuant "Methodology" sections
 // 1-4): per 128-element tile, seeded sign flip, FWHT-128, scale, optional
-// subtractive dither, nearest lattice point, bit-stripping, zigzag, Rice planes.
+// subtractive dither, nearest lattice point, bit-stripping, zigzag, Rice planes;
+// and the rate-only pass that counts the same codes without writing them.
 //
-// Work decomposition (B200, sm_100a):
-//  * one warp encodes one chunk (32 tiles) in 4 rounds of 8 tiles; four lanes
-//    share a tile, 32 elements each, loaded as 64 contiguous bytes per lane;
-//  * the transform runs in registers (16 float2 per lane, packed fp32 adds;
-//    the last two butterfly stages cross lanes by shuffle), then each lane
-//    decodes its 32/N lattice blocks and keeps 32 zigzag symbols;
-//  * per round a warp scan of unary lengths places every lane's codewords;
-//    remainder bits, E8 coset bits and unary terminators go into a per-warp
-//    shared-memory stage that holds the whole chunk;
-//  * the next round's input is copied into shared memory (cp.async) while the
-//    current round is computed;
-//  * a persistent grid takes chunk tickets from a global counter, so a chunk's
-//    predecessors are always already running; a single-pass decoupled
-//    look-back over 64-bit (flag, value) words gives the chunk's word offset
-//    (bounded waits: HQ_ST_TIMEOUT).  A chunk publishes its size as soon as it
-//    is encoded and resolves its offset after the warp has encoded its next
-//    chunk into a second stage, so predecessors have normally published by
-//    then; the stage is then written out coalesced;
-//  * a chunk larger than the stage is re-encoded by a separate path that sets
-//    its bits in place in global memory (same stream; only for extreme codes).
+// Three forms with identical output, chosen by launch size (hq_api.cu):
+//  * per-warp (throughput; more than 592 chunks): one warp encodes one chunk
+//    (32 tiles) in 4 rounds of 8 tiles; four lanes share a tile, 32 elements
+//    each, loaded as 64 contiguous bytes per lane with cp.async one round ahead;
+//    the transform runs in registers (16 float2 per lane, packed fp32 adds, the
+//    last two butterfly stages across lanes by shuffle); each lane decodes its
+//    32/N lattice blocks into 32 zigzag symbols; a warp scan of unary lengths
+//    places every codeword in a per-warp shared stage holding the chunk;
+//  * grouped (latency; up to 592 chunks): four warps share a chunk, one round
+//    each, meeting at a named barrier per chunk;
+//  * wide (lowest latency; up to 296 chunks): sixteen warps share a chunk,
+//    sixteen lanes per tile, one 8-element block per lane.
+// In every form a persistent grid takes chunk tickets from a global counter, so
+// a chunk's predecessors are always already running, and a single-pass
+// decoupled look-back over 64-bit (flag, value) words gives each chunk's word
+// offset (bounded waits: HQ_ST_TIMEOUT).  A chunk publishes its size as soon as
+// it is encoded and resolves its offset one chunk later, when its predecessors
+// have normally published; its stage is then copied out coalesced.  A chunk
+// larger than the stage is re-encoded by a path that sets its bits in place in
+// global memory (the same bits; only for extreme codes).
 #include <cuda_runtime.h>
 #include <stdint.h>
 

@@ -12,12 +12,12 @@
 namespace hq {
 
 constexpr int kTile = 128;          // elements per RHT tile
-constexpr int kChunkTiles = 32;     // tiles per chunk = lanes per warp (one tile per lane)
+constexpr int kChunkTiles = 32;     // tiles per chunk (the stream's unit: one offset per chunk)
 constexpr int kSignWords = 4;       // shared sign-table words per tile column (one per 32-column quarter)
-constexpr int kWarpsPerCta = 8;     // warps per CTA in both kernels
-constexpr int kStageWords = 1024;   // per-warp shared staging for one chunk's words (encode and decode);
+constexpr int kWarpsPerCta = 8;     // warps per CTA of the per-warp and grouped encoders and the decoder
+constexpr int kStageWords = 1024;   // shared staging for one chunk's words (encode and decode);
                                     // larger chunks are written or read in place in global memory
-constexpr int kLanesPerTile = 4;    // lanes sharing one tile (32 elements each)
+constexpr int kLanesPerTile = 4;    // lanes sharing one tile (32 elements each), except the wide encoder
 constexpr int kTilesPerRound = 32 / kLanesPerTile;  // tiles a warp transforms at once; 4 rounds per chunk
 constexpr uint32_t kSpinLimit = 1u << 22;   // look-back polls before giving up (HQ_ST_TIMEOUT)
 constexpr uint32_t kMaxUnaryBits = 1u << 31; // chunks with more unary bits are outside the supported range
