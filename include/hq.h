@@ -150,7 +150,8 @@ HQ_API int hq_stream_bound(int64_t rows, int64_t cols, const hq_params *p, uint3
                     uint64_t *max_words, uint64_t *n_chunks);
 
 /* Bytes of device workspace hq_quantize / hq_kv_append need for n_chunks
- * chunks (chunk look-back state and a chunk ticket).  Host only. */
+ * chunks (8 bytes of chunk look-back state per chunk, a chunk ticket, a CTA
+ * counter and the call's stats accumulator), rounded up to 256.  Host only. */
 HQ_API int hq_workspace_bytes(uint64_t n_chunks, size_t *bytes);
 
 /* ------------------------------------------------------------ weights path */
@@ -160,7 +161,8 @@ HQ_API int hq_workspace_bytes(uint64_t n_chunks, size_t *bytes);
  *   x         device, bf16, element (r, c) at x[r * ld + c]; ld >= cols, ld % 8 == 0.
  *   d_stream  device, cap_words uint32 words, written [0, stream_words).
  *   d_offsets device, n_chunks + 1 uint64 entries, all written.
- *   d_stats   device hq_stats or NULL; zeroed then filled.
+ *   d_stats   device hq_stats or NULL; replaced by this call's stats, written by
+ *             the kernel when it finishes.
  *   workspace device, >= hq_workspace_bytes(n_chunks); overwritten (contents
  *             need no initialisation; the call clears what it uses).
  * Sign index of element (r, c) is c; dither counter (if any) is r * cols + c.
@@ -213,8 +215,8 @@ HQ_API int hq_gemv(const uint32_t *d_stream, uint64_t stream_words, const uint64
  * allowed.  Arguments, results and status are those of hq_quantize; the
  * caller still passes x, d_stream, d_offsets and (optionally) d_stats.
  *
- * The encoder's scratch (8 bytes of chunk look-back state per chunk plus a
- * ticket word) lives in a fixed array of HQ_STATIC_SCRATCH_BYTES inside
+ * The encoder's scratch (8 bytes of chunk look-back state per chunk, a ticket
+ * and a counter word, and a stats accumulator) lives in a fixed array of HQ_STATIC_SCRATCH_BYTES inside
  * libhq.so's device image; every GPU that loads the library holds it until the
  * process exits.  Limit: at most HQ_STATIC_MAX_CHUNKS chunks (4096 elements
  * each, about 537 million elements); a larger matrix returns HQ_EUNSUPPORTED
@@ -228,7 +230,7 @@ HQ_API int hq_gemv(const uint32_t *d_stream, uint64_t stream_words, const uint64
  * and corrupt each other's streams: serialise them.  The call allocates
  * nothing: no cudaMalloc, cudaFree or allocating library routine. */
 #define HQ_STATIC_SCRATCH_BYTES (1u << 20)
-#define HQ_STATIC_MAX_CHUNKS 131071u
+#define HQ_STATIC_MAX_CHUNKS 131067u
 HQ_API int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p,
                               uint32_t *d_stream, uint64_t cap_words, uint64_t *d_offsets, hq_stats *d_stats,
                               void *cuda_stream);

@@ -47,8 +47,17 @@ float scale_fwd(float alpha) { return (float)((double)alpha / sqrt(128.0)); }
 float scale_inv(float alpha) { return (float)(1.0 / ((double)alpha * sqrt(128.0))); }
 
 size_t ws_bytes_for(uint64_t n_chunks) {
-    size_t b = (size_t)n_chunks * 8 + 8;
+    const size_t b = encode_scratch_bytes(n_chunks);
     return (b + 255) & ~(size_t)255;
+}
+
+// The encoder's workspace pointers (layout in hq_internal.h).
+void set_scratch(EncodeArgs &a, void *ws, uint64_t nch) {
+    char *b = (char *)ws;
+    a.lookback = (unsigned long long *)b;
+    a.ticket = (unsigned int *)(b + nch * 8);
+    a.done = (unsigned int *)(b + nch * 8 + 4);
+    a.acc = (hq_stats *)(b + nch * 8 + 8);
 }
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ECUDA; }
@@ -100,12 +109,16 @@ int hq_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_
     if (!d_offsets || !aligned(d_offsets, 8)) return HQ_EINVAL;
     if (d_stats && !aligned(d_stats, 8)) return HQ_EINVAL;
     cudaStream_t s = (cudaStream_t)cuda_stream;
-    if (d_stats && cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
-    if (nch == 0) return cuda_rc(cudaMemsetAsync(d_offsets, 0, sizeof(uint64_t), s));
+    if (nch == 0) {
+        if (d_stats && cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
+        return cuda_rc(cudaMemsetAsync(d_offsets, 0, sizeof(uint64_t), s));
+    }
     if (!x || !aligned(x, 16) || ld < cols || ld % 8) return HQ_EINVAL;
     if (!d_stream || !aligned(d_stream, 4)) return HQ_EINVAL;
     if (!workspace || !aligned(workspace, 8) || ws_bytes < ws_bytes_for(nch)) return HQ_EINVAL;
-    if (cudaMemsetAsync(workspace, 0, (size_t)nch * 8 + 8, s) != cudaSuccess) return HQ_ECUDA;
+    // one memset clears the look-back words, the ticket, the done counter and the stats
+    // accumulator; the kernel's last CTA writes *d_stats
+    if (cudaMemsetAsync(workspace, 0, encode_scratch_bytes(nch), s) != cudaSuccess) return HQ_ECUDA;
 
     EncodeArgs a;
     memset(&a, 0, sizeof(a));
@@ -123,8 +136,8 @@ int hq_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_
     a.cap_words = cap_words;
     a.offsets = d_offsets;
     a.stats = d_stats;
-    a.lookback = (unsigned long long *)workspace;
-    a.ticket = (unsigned int *)((char *)workspace + nch * 8);
+    a.stats_add = 0;
+    set_scratch(a, workspace, nch);
     a.tcols = (int)(cols / kTile);
     a.spin_limit = g_spin_limit;
     return cuda_rc(launch_encode(p->lattice, p->dither, a, s));
@@ -258,7 +271,7 @@ int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t ld_token
     if (cache->chunks + nch + 1 > cache->offsets_cap || cache->appends + 1 > cache->table_cap) return HQ_EINVAL;
     if (!workspace || !aligned(workspace, 8) || ws_bytes < ws_bytes_for(nch)) return HQ_EINVAL;
     cudaStream_t s = (cudaStream_t)cuda_stream;
-    if (cudaMemsetAsync(workspace, 0, (size_t)nch * 8 + 8, s) != cudaSuccess) return HQ_ECUDA;
+    if (cudaMemsetAsync(workspace, 0, encode_scratch_bytes(nch), s) != cudaSuccess) return HQ_ECUDA;
 
     EncodeArgs a;
     memset(&a, 0, sizeof(a));
@@ -287,8 +300,8 @@ int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t ld_token
     a.row_val.scale_fwd = a.c_scale;
     a.row_val.scale_inv = scale_inv(alpha);
     a.stats = cache->d_stats;
-    a.lookback = (unsigned long long *)workspace;
-    a.ticket = (unsigned int *)((char *)workspace + nch * 8);
+    a.stats_add = 1;
+    set_scratch(a, workspace, nch);
     a.tcols = 1;
     a.spin_limit = g_spin_limit;
     rc = cuda_rc(launch_encode(p.lattice, p.dither, a, s));

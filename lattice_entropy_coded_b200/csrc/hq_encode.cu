@@ -98,6 +98,44 @@ __device__ __noinline__ unsigned long long lookback_resolve(unsigned long long *
     return excl;
 }
 
+// Stats of an encode call.  Every warp adds its part to the workspace accumulator
+// (the warp's payload is lane 0's; the accumulator is cleared with the look-back
+// words, so the caller's stats need no separate clearing); the last CTA to finish moves the totals to the caller's stats,
+// replacing them (hq_quantize) or adding to them (a KV cache's running stats).
+__device__ __forceinline__ void stats_add_warp(const EncodeArgs &a, uint32_t status, uint32_t zor_all,
+                                               unsigned long long payload) {
+    status = __reduce_or_sync(0xffffffffu, status);
+    zor_all = __reduce_or_sync(0xffffffffu, zor_all);
+    if ((threadIdx.x & 31) == 0) {
+        if (status) atomicOr(&a.acc->status, status);
+        if (zor_all) atomicOr(&a.acc->max_symbol, zor_all);
+        if (payload) atomicAdd((unsigned long long *)&a.acc->payload_bits, payload);
+    }
+}
+
+// Whole CTA calls it once, at its end.
+__device__ __forceinline__ void stats_finish_cta(const EncodeArgs &a) {
+    __syncthreads();
+    if (threadIdx.x != 0) return;
+    __threadfence();
+    if (atomicAdd(a.done, 1u) != gridDim.x - 1) return;
+    __threadfence();
+    if (!a.stats) return;
+    const uint32_t st = ld_relaxed_u32(&a.acc->status), mx = ld_relaxed_u32(&a.acc->max_symbol);
+    const unsigned long long pb = ld_relaxed_u64((const unsigned long long *)&a.acc->payload_bits);
+    const unsigned long long sw = ld_relaxed_u64((const unsigned long long *)&a.acc->stream_words);
+    if (a.stats_add) {
+        if (st) atomicOr(&a.stats->status, st);
+        if (mx) atomicOr(&a.stats->max_symbol, mx);
+        if (pb) atomicAdd((unsigned long long *)&a.stats->payload_bits, pb);
+    } else {
+        a.stats->status = st;
+        a.stats->max_symbol = mx;
+        a.stats->payload_bits = pb;
+    }
+    a.stats->stream_words = sw;
+}
+
 // Where the tiles of one chunk are (computed once per chunk).
 struct ChunkGeo {
     int ntiles;
@@ -482,7 +520,7 @@ __device__ __forceinline__ void finish_chunk_warp(const EncodeArgs &a, const Pen
             const unsigned long long end = start + p.total;
             a.offsets[a.chunk_base + a.n_chunks] = end;
             if (a.tail_out) *a.tail_out = end;
-            if (a.stats) a.stats->stream_words = end;
+            a.acc->stream_words = end;
             if (end > a.cap_words) status |= HQ_ST_CAPACITY;
         }
         if (p.c == 0 && a.row) *a.row = a.row_val;
@@ -635,15 +673,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     if (have_pend) finish_chunk_warp<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 
-    if (a.stats) {
-        zor_all = __reduce_or_sync(0xffffffffu, zor_all);
-        status = __reduce_or_sync(0xffffffffu, status);
-        if (lane == 0) {
-            if (status) atomicOr(&a.stats->status, status);
-            if (zor_all) atomicOr(&a.stats->max_symbol, zor_all);
-            if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
-        }
-    }
+    stats_add_warp(a, status, zor_all, payload);
+    stats_finish_cta(a);
 }
 
 // Four warps share a chunk: warp w of a group encodes round w (tiles 8w..8w+7).
@@ -681,7 +712,7 @@ __device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending 
             const unsigned long long end = start + p.total;
             a.offsets[a.chunk_base + a.n_chunks] = end;
             if (a.tail_out) *a.tail_out = end;
-            if (a.stats) a.stats->stream_words = end;
+            a.acc->stream_words = end;
             if (end > a.cap_words) status |= HQ_ST_CAPACITY;
         }
         if (p.c == 0 && a.row) *a.row = a.row_val;
@@ -861,15 +892,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel_grouped(co
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 
-    if (a.stats) {
-        zor_all = __reduce_or_sync(0xffffffffu, zor_all);
-        status = __reduce_or_sync(0xffffffffu, status);
-        if (lane == 0) {
-            if (status) atomicOr(&a.stats->status, status);
-            if (zor_all) atomicOr(&a.stats->max_symbol, zor_all);
-            if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
-        }
-    }
+    stats_add_warp(a, status, zor_all, payload);
+    stats_finish_cta(a);
 }
 
 
@@ -1102,15 +1126,8 @@ __global__ void __launch_bounds__(kWideWarps * 32, 1) encode_kernel_wide(const E
         it++;
     }
 
-    if (a.stats) {
-        zor_all = __reduce_or_sync(0xffffffffu, zor_all);
-        status = __reduce_or_sync(0xffffffffu, status);
-        if (lane == 0) {
-            if (status) atomicOr(&a.stats->status, status);
-            if (zor_all) atomicOr(&a.stats->max_symbol, zor_all);
-            if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
-        }
-    }
+    stats_add_warp(a, status, zor_all, payload);
+    stats_finish_cta(a);
 }
 
 template <int LAT, bool DITHER>

@@ -22,6 +22,10 @@ constexpr int kTilesPerRound = 32 / kLanesPerTile;  // tiles a warp transforms a
 constexpr uint32_t kSpinLimit = 1u << 22;   // look-back polls before giving up (HQ_ST_TIMEOUT)
 constexpr uint32_t kMaxUnaryBits = 1u << 31; // chunks with more unary bits are outside the supported range
 
+// Encoder workspace of n chunks: look-back words [0, 8n), ticket at 8n, done counter at
+// 8n + 4, stats accumulator at 8n + 8; all cleared by one memset of encode_scratch_bytes(n).
+inline size_t encode_scratch_bytes(uint64_t n_chunks) { return (size_t)n_chunks * 8 + 8 + sizeof(hq_stats); }
+
 // Salts xor-ed into the seed: "SIGN" for the sign diagonal, "DITH" for the dither.
 constexpr uint64_t kSignSalt = 0x5349474Eull;
 constexpr uint64_t kDitherSalt = 0x44495448ull;
@@ -50,9 +54,12 @@ struct EncodeArgs {
     uint64_t *tail_out;       // device word updated with the end of this call's stream, or null
     hq_kv_append_row *row;    // KV: table row written by the warp of chunk 0, or null
     hq_kv_append_row row_val;
-    hq_stats *stats;          // may be null
+    hq_stats *stats;          // the caller's stats, or null
+    int stats_add;            // 1: add this call's stats to *stats (a KV cache's running stats); 0: replace
     unsigned long long *lookback;  // n_chunks words, zeroed
     unsigned int *ticket;          // one word, zeroed
+    unsigned int *done;            // one word, zeroed: CTAs finished
+    hq_stats *acc;                 // zeroed: this call's stats, moved to *stats by the last CTA
     int tcols;                // tile columns in the sign table (cols / 128, or 1 for KV)
     uint32_t spin_limit;
 };

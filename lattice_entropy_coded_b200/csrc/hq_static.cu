@@ -21,7 +21,7 @@ namespace {
 constexpr size_t kStaticScratchBytes = HQ_STATIC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
 
-// Look-back words (8 bytes per chunk) followed by the ticket word.
+// Look-back words (8 bytes per chunk), the ticket and done words, the stats accumulator.
 static __device__ __align__(256) unsigned char g_hq_scratch[kStaticScratchBytes];
 
 std::mutex g_mu;
@@ -65,12 +65,15 @@ int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, co
     int rc = scratch_address(&scratch);
     if (rc) return rc;
     cudaStream_t s = (cudaStream_t)cuda_stream;
-    if (d_stats && cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
-    if (nch == 0) return cudaMemsetAsync(d_offsets, 0, sizeof(uint64_t), s) == cudaSuccess ? HQ_OK : HQ_ECUDA;
+    if (nch == 0) {
+        if (d_stats && cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
+        return cudaMemsetAsync(d_offsets, 0, sizeof(uint64_t), s) == cudaSuccess ? HQ_OK : HQ_ECUDA;
+    }
     if (!x || !aligned(x, 16) || ld < cols || ld % 8) return HQ_EINVAL;
     if (!d_stream || !aligned(d_stream, 4)) return HQ_EINVAL;
-    // the previous call's look-back words and ticket are still there: clear what this call uses
-    if (cudaMemsetAsync(scratch, 0, (size_t)nch * 8 + 8, s) != cudaSuccess) return HQ_ECUDA;
+    // the previous call's look-back words, ticket, counter and stats are still there:
+    // clear what this call uses
+    if (cudaMemsetAsync(scratch, 0, encode_scratch_bytes(nch), s) != cudaSuccess) return HQ_ECUDA;
 
     EncodeArgs a;
     memset(&a, 0, sizeof(a));
@@ -88,8 +91,11 @@ int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, co
     a.cap_words = cap_words;
     a.offsets = d_offsets;
     a.stats = d_stats;
+    a.stats_add = 0;
     a.lookback = (unsigned long long *)scratch;
     a.ticket = (unsigned int *)((char *)scratch + nch * 8);
+    a.done = (unsigned int *)((char *)scratch + nch * 8 + 4);
+    a.acc = (hq_stats *)((char *)scratch + nch * 8 + 8);
     a.tcols = (int)(cols / kTile);
     a.spin_limit = kSpinLimit;
     return launch_encode(p->lattice, p->dither, a, s) == cudaSuccess ? HQ_OK : HQ_ECUDA;
@@ -97,4 +103,5 @@ int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, co
 
 }  // extern "C"
 
-static_assert(kStaticScratchBytes >= (size_t)HQ_STATIC_MAX_CHUNKS * 8 + 8, "scratch too small for the limit");
+static_assert(kStaticScratchBytes >= (size_t)HQ_STATIC_MAX_CHUNKS * 8 + 8 + sizeof(hq_stats),
+              "scratch too small for the limit");

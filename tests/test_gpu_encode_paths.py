@@ -74,3 +74,22 @@ def test_many_chunks_per_worker(path):
     assert_same_words(g["words"], g["offsets"], ref_w, ref_off)
     assert g["stats"]["payload_bits"] == ref_pay
     assert np.uint64(g["stats"]["stream_words"]) == ref_off[-1]
+
+
+def test_stats_are_replaced_not_accumulated(path):
+    """hq_quantize's stats block is written by the kernel's last CTA: whatever it held
+    before (here all bytes 0xFF) is replaced by exactly this call's stats."""
+    import torch
+    import lattice_entropy_coded_b200 as hq
+    x = synth.weight(64, 4096, seed=13).cuda()
+    params = hq.make_params("E8", 300.0, 2, 1, 0)
+    ref = gpu_quantize(x, params)
+    bound, nch = hq.hq_stream_bound(64, 4096, params)
+    words = torch.empty(bound, dtype=torch.int32, device="cuda")
+    offs = torch.empty(nch + 1, dtype=torch.int64, device="cuda")
+    ws = torch.empty(hq.hq_workspace_bytes(nch), dtype=torch.uint8, device="cuda")
+    st = torch.full((32,), 0xFF, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        hq.hq_quantize(x, params, words, offs, st, ws)
+        got = hq.read_stats(st)
+        assert got == ref["stats"], (got, ref["stats"])

@@ -66,7 +66,7 @@ def test_static_scratch_matches_workspace_entry_point(lattice, alpha, k, dither,
 def test_static_scratch_rejects_sizes_beyond_its_limit():
     import lattice_entropy_coded_b200 as hq
     params = hq.make_params("E8", 300.0, 2, 0, 0)
-    too_many_rows = (131071 * 32 + 32) // 32 + 1          # cols = 4096: one chunk per row
+    too_many_rows = (131067 * 32 + 32) // 32 + 1          # cols = 4096: one chunk per row
     x = torch.empty(1, 4096, dtype=torch.bfloat16, device="cuda")
     rc = hq._lib.hq_quantize_static(x.data_ptr(), too_many_rows, 4096, 4096, C.byref(params), x.data_ptr(), 0,
                                     x.data_ptr(), None, None)
