@@ -364,6 +364,77 @@ def oracle_sample_rate(workload: str, rows_sample: int, threads: int, repeat: in
     return 2.0 * elems / dt / 1e9, dt, elems
 
 
+def oracle_workload(workload: str, threads: int, budget_s: float = 60.0):
+    """The CPU oracle's quantize+encode and decode over a workload's tensors, generated on the
+    host, on `threads` threads (chunk ranges, or KV appends, in parallel), until `budget_s` of
+    wall time per operating point is spent.  -> one dict per point; where the budget ran out
+    first, the rate is over the tensors done and `extrapolated` is true."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle as O
+    w = synth.WORKLOADS[workload]
+    pts = rate_points()[workload]["points"]
+    O.lib()
+
+    def u16(t):
+        return np.ascontiguousarray(t.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+    def tensors():
+        if w["kind"] == "weight":
+            yield synth.weight(w["rows"], w["cols"], w["seed"])
+        elif w["kind"] == "weight_set":
+            for _, m in synth.weight_set(w["seed"], layers=w["layers"]):
+                yield m
+        elif w["kind"] == "student_t":
+            yield from synth.student_t(w["n"], w["rows"], w["cols"], w["seed"])
+        else:
+            K, V = synth.kv(w["heads"], w["tokens"], w["seed"])
+            yield {"K": K, "V": V}
+
+    total = {"weight": w.get("rows", 0) * w.get("cols", 0), "weight_set": synth.weight_set_elems(w.get("layers", 8)),
+             "student_t": w.get("n", 0) * w.get("rows", 0) * w.get("cols", 0),
+             "kv": w.get("heads", 0) * w.get("tokens", 0) * 128}[w["kind"]]
+    out = []
+    with ThreadPoolExecutor(threads) as ex:
+        for p in pts:
+            lat = O.LATTICES[p["lattice"]]
+            busy, elems, t_start = 0.0, 0, time.perf_counter()
+            for t in tensors():
+                if w["kind"] == "kv":
+                    xu = u16(t[p["tensor"]])
+                    H, T, _ = xu.shape
+                    A = w["append"]
+                    dec = np.zeros((H, T, 128), np.uint16)     # appends write disjoint token ranges
+
+                    def job(t0, xu=xu, H=H, T=T, A=A, dec=dec):
+                        blk = np.ascontiguousarray(xu[:, t0:t0 + A])
+                        s_, off, _ = O.kv_append(blk, t0, lat, p["alpha"], p["k"], w["seed"], 1)
+                        O.kv_read_append(s_, off, H, blk.shape[1], t0, lat, p["alpha"], p["k"], w["seed"], 1, dec, T)
+                    jobs = list(range(0, T, A))
+                    n_el = xu.size
+                else:
+                    xu = u16(t)
+                    R, Cc = xu.shape
+                    nch = O.n_chunks(R, Cc)
+                    step = max(1, -(-nch // threads))
+                    jobs = [(a, min(nch, a + step)) for a in range(0, nch, step)]
+
+                    def job(r, xu=xu, R=R, Cc=Cc):
+                        s_, off, _ = O.quantize(xu, lat, p["alpha"], p["k"], w["seed"], 0, r[0], r[1])
+                        O.dequantize(s_, off, R, Cc, lat, p["alpha"], p["k"], w["seed"], 0, False, r[0], r[1])
+                    n_el = xu.size
+                t0 = time.perf_counter()
+                list(ex.map(job, jobs))
+                busy += time.perf_counter() - t0
+                elems += n_el
+                if time.perf_counter() - t_start > budget_s:
+                    break
+            out.append({"lattice": p["lattice"], "bps_target": p["bps"], "tensor": p.get("tensor"),
+                        "gbs": round(2.0 * elems / busy / 1e9, 4), "seconds": round(busy, 2), "elements": elems,
+                        "of_elements": total, "extrapolated": elems < total, "threads": threads})
+    return out
+
+
 def host_threads() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -552,6 +623,11 @@ def run_bulk(args):
         out["points"] = res
         if w["kind"] == "student_t":
             out["calibration"] = calibrate_set(hq, mats, pts, w["seed"])
+    if args.oracle:
+        threads = host_threads()
+        out["oracle"] = {"threads": threads, "points": oracle_workload(wl, threads)}
+        if w["kind"] == "weight":
+            out["oracle"]["single_thread"] = oracle_workload(wl, 1)
     print(json.dumps(out), flush=True)
 
 
@@ -667,6 +743,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle", action="store_true",
+                    help="with --workload: also time the CPU oracle on the workload (about a minute per point)")
     ap.add_argument("--case", default=None, help="RxC: time one matrix (profiling case)")
     ap.add_argument("--lattice", default="E8")
     ap.add_argument("--bps", type=float, default=4.0)
