@@ -116,9 +116,15 @@ def _bind(L):
         "hqref_dequantize": (_i32, [_p, _p, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _i64, _i64, _i32, _p,
                                     _i64]),
         "hqref_kv_append": (_i64, [_p, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _p, _u64,
-                                   _u64, _p, _p]),
+                                   _u64, _p, _p, _p]),
         "hqref_kv_read_append": (_i32, [_p, _p, _i64, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _i32, _p,
-                                        _i64, _i64, _i64]),
+                                        _i64, _i64, _i64, _p]),
+        "hqref_rotate_fwd": (None, [_p, _p, _p]),
+        "hqref_rotate_inv": (None, [_p, _p, _p]),
+        "hqref_scale_inv_rot": (_f32, [_f32]),
+        "hqref_quantize_tile_rot": (None, [_p, _i32, _f32, _p, _u64, _i32, _u64, _p]),
+        "hqref_dequantize_tile_rot": (None, [_p, _i32, _f32, _p, _u64, _i32, _u64, _p]),
+        "hqref_rot_gaussian": (C.c_double, [_u64, _u64]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -286,6 +292,46 @@ def dequantize_tile(q, lat, alpha, seed, sign_col0=0, dither=0, e0=0) -> np.ndar
     return out
 
 
+def rotate_fwd(Q, x) -> np.ndarray:
+    q = np.ascontiguousarray(Q, dtype=np.float32)
+    a = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.zeros(128, dtype=np.float32)
+    lib().hqref_rotate_fwd(_ptr(q), _ptr(a), _ptr(out))
+    return out
+
+
+def rotate_inv(Q, z) -> np.ndarray:
+    q = np.ascontiguousarray(Q, dtype=np.float32)
+    a = np.ascontiguousarray(z, dtype=np.float32)
+    out = np.zeros(128, dtype=np.float32)
+    lib().hqref_rotate_inv(_ptr(q), _ptr(a), _ptr(out))
+    return out
+
+
+def scale_inv_rot(alpha: float) -> float:
+    return float(lib().hqref_scale_inv_rot(alpha))
+
+
+def quantize_tile_rot(x_u16, lat, alpha, Q, seed, dither=0, e0=0) -> np.ndarray:
+    x = np.ascontiguousarray(x_u16, dtype=np.uint16)
+    r_keep, rp = _rot_ptr(Q)
+    q = np.zeros(128, dtype=np.int32)
+    lib().hqref_quantize_tile_rot(_ptr(x), lat, alpha, rp, seed, dither, e0, _ptr(q))
+    return q
+
+
+def dequantize_tile_rot(q, lat, alpha, Q, seed, dither=0, e0=0) -> np.ndarray:
+    a = np.ascontiguousarray(q, dtype=np.int32)
+    r_keep, rp = _rot_ptr(Q)
+    out = np.zeros(128, dtype=np.float32)
+    lib().hqref_dequantize_tile_rot(_ptr(a), lat, alpha, rp, seed, dither, e0, _ptr(out))
+    return out
+
+
+def rot_gaussian(seed: int, e: int) -> float:
+    return float(lib().hqref_rot_gaussian(seed & (2**64 - 1), e & (2**64 - 1)))
+
+
 # ---------------------------------------------------------------- whole tensors
 def n_chunks(rows: int, cols: int) -> int:
     return int(lib().hqref_n_chunks(rows, cols))
@@ -331,8 +377,20 @@ def dequantize(stream, offsets, rows: int, cols: int, lat: int, alpha: float, k:
     return out
 
 
-def kv_append(kv, tok0: int, lat: int, alpha: float, k: int, seed: int, dither: int = 1, base_word: int = 0):
-    """One KV append: bf16 [H, T, 128] -> (stream words, absolute offsets (n+1), payload bits)."""
+def _rot_ptr(rot):
+    """A dense rotation as a C pointer (None: the sign diagonal and H_128)."""
+    if rot is None:
+        return None, None
+    r = np.ascontiguousarray(rot, dtype=np.float32)
+    assert r.shape == (128, 128)
+    return r, _ptr(r)
+
+
+def kv_append(kv, tok0: int, lat: int, alpha: float, k: int, seed: int, dither: int = 1, base_word: int = 0,
+              rot=None):
+    """One KV append: bf16 [H, T, 128] -> (stream words, absolute offsets (n+1), payload bits).
+    rot: a 128 x 128 orthogonal fp32 matrix in place of H_128 D / sqrt(128), or None."""
+    r_keep, rp = _rot_ptr(rot)
     x = _as_u16(kv)
     H, T, D = x.shape
     assert D == 128
@@ -341,21 +399,24 @@ def kv_append(kv, tok0: int, lat: int, alpha: float, k: int, seed: int, dither: 
     off = np.zeros(nch + 1, dtype=np.uint64)
     pb = np.zeros(1, dtype=np.uint64)
     end = abs(int(L.hqref_kv_append(_ptr(x), H, T, 128, T * 128, tok0, lat, alpha, k, seed, dither, None,
-                                    base_word, 0, _ptr(off), _ptr(pb))))
+                                    base_word, 0, _ptr(off), _ptr(pb), rp)))
     total = end - base_word
     stream = np.zeros(max(end, 1), dtype=np.uint32)
     L.hqref_kv_append(_ptr(x), H, T, 128, T * 128, tok0, lat, alpha, k, seed, dither, _ptr(stream), base_word,
-                      stream.size, _ptr(off), _ptr(pb))
+                      stream.size, _ptr(off), _ptr(pb), rp)
+    del r_keep
     return stream[base_word:end].copy(), off, int(pb[0])
 
 
 def kv_read_append(stream_abs, offsets_abs, H: int, T: int, tok0: int, lat: int, alpha: float, k: int, seed: int,
-                   dither: int, out: np.ndarray, length: int):
+                   dither: int, out: np.ndarray, length: int, rot=None):
     """Decode one append into out [H, len, 128] (float32 or uint16 bf16 bits)."""
+    r_keep, rp = _rot_ptr(rot)
     s = np.ascontiguousarray(stream_abs, dtype=np.uint32)
     o = np.ascontiguousarray(offsets_abs, dtype=np.uint64)
     assert out.flags["C_CONTIGUOUS"] and out.shape[2] == 128
     rc = lib().hqref_kv_read_append(_ptr(s), _ptr(o), H, T, tok0, lat, alpha, k, seed, dither,
-                                    int(out.dtype == np.float32), _ptr(out), 128, out.shape[1] * 128, length)
+                                    int(out.dtype == np.float32), _ptr(out), 128, out.shape[1] * 128, length, rp)
+    del r_keep
     if rc != 0:
         raise ValueError("corrupt stream")

@@ -10,7 +10,7 @@
  * 2606.23406, sections "Methodology": 1 per-tile RHT, 2 lattice quantization,
  * 3 bit-stripping and Rice coding, 4 KV bias correction) and the arXiv abstract
  * (items (i)-(iv)).  The pages give no constants, no bitstream and no code; the
- * readings taken where they are silent are marked [R1]..[R16] and listed in the
+ * readings taken where they are silent are marked [R1]..[R18] and listed in the
  * design notes of the repository.
  *
  * Build: gcc -std=c99 -O2 -ffp-contract=off -fno-fast-math -shared -fPIC.
@@ -471,21 +471,11 @@ int hqref_decode_chunk(int lat, int k, const uint32_t *w, uint64_t nwords, int n
 }
 
 /* ------------------------------------------------------------------------ */
-/* One tile, forward [R1]-[R6], [R13]: x (128 bf16) -> codes.  sign_col0 is the
- * sign index of element 0 (element i uses sign index sign_col0 + i); e0 is the
- * dither counter of element 0 (counters are consecutive along the tile). */
-void hqref_quantize_tile(const uint16_t *x, int lat, float alpha, uint64_t seed, uint64_t sign_col0, int dither,
-                         uint64_t e0, int32_t *q)
+/* The lattice stage of a transformed, scaled tile v (128 fp32): per block of
+ * n coordinates [+ d, R13], nearest point [R6]-[R8]. */
+static void quantize_blocks(const float *v, int lat, uint64_t seed, int dither, uint64_t e0, int32_t *q)
 {
-    float v[128];
     int n = hqref_lattice_dim(lat);
-    for (int i = 0; i < 128; i++) {
-        float xi = hqref_bf16_to_f32(x[i]);
-        v[i] = (hqref_sign(seed, sign_col0 + (uint64_t)i) < 0) ? -xi : xi;
-    }
-    hqref_fwht128(v);
-    float c = hqref_scale_fwd(alpha);
-    for (int i = 0; i < 128; i++) v[i] = v[i] * c;
     for (int b = 0; b < 128; b += n) {
         float blk[8];
         for (int i = 0; i < n; i++) blk[i] = v[b + i];
@@ -498,11 +488,9 @@ void hqref_quantize_tile(const uint16_t *x, int lat, float alpha, uint64_t seed,
     }
 }
 
-/* One tile, inverse [R14]: codes -> fp32 reconstruction (before bf16 rounding). */
-void hqref_dequantize_tile(const int32_t *q, int lat, float alpha, uint64_t seed, uint64_t sign_col0, int dither,
-                           uint64_t e0, float *out)
+/* Its inverse up to the scale: v = lattice point [- d] per block [R14]. */
+static void dequantize_blocks(const int32_t *q, int lat, uint64_t seed, int dither, uint64_t e0, float *v)
 {
-    float v[128];
     int n = hqref_lattice_dim(lat);
     for (int b = 0; b < 128; b += n) {
         float p[8];
@@ -514,11 +502,99 @@ void hqref_dequantize_tile(const int32_t *q, int lat, float alpha, uint64_t seed
         }
         for (int i = 0; i < n; i++) v[b + i] = p[i];
     }
+}
+
+/* One tile, forward [R1]-[R6], [R13]: x (128 bf16) -> codes.  sign_col0 is the
+ * sign index of element 0 (element i uses sign index sign_col0 + i); e0 is the
+ * dither counter of element 0 (counters are consecutive along the tile). */
+void hqref_quantize_tile(const uint16_t *x, int lat, float alpha, uint64_t seed, uint64_t sign_col0, int dither,
+                         uint64_t e0, int32_t *q)
+{
+    float v[128];
+    for (int i = 0; i < 128; i++) {
+        float xi = hqref_bf16_to_f32(x[i]);
+        v[i] = (hqref_sign(seed, sign_col0 + (uint64_t)i) < 0) ? -xi : xi;
+    }
+    hqref_fwht128(v);
+    float c = hqref_scale_fwd(alpha);
+    for (int i = 0; i < 128; i++) v[i] = v[i] * c;
+    quantize_blocks(v, lat, seed, dither, e0, q);
+}
+
+/* One tile, inverse [R14]: codes -> fp32 reconstruction (before bf16 rounding). */
+void hqref_dequantize_tile(const int32_t *q, int lat, float alpha, uint64_t seed, uint64_t sign_col0, int dither,
+                           uint64_t e0, float *out)
+{
+    float v[128];
+    dequantize_blocks(q, lat, seed, dither, e0, v);
     float e = hqref_scale_inv(alpha);
     for (int i = 0; i < 128; i++) v[i] = v[i] * e;
     hqref_fwht128(v);
     for (int i = 0; i < 128; i++)
         out[i] = (hqref_sign(seed, sign_col0 + (uint64_t)i) < 0) ? -v[i] : v[i];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dense rotation of the KV path [R17] (explainer pages, "Methodology" 4: each
+ * layer's keys and values are rotated either by a full Haar-uniform matrix or
+ * by the cheap sign diagonal).  Q is a 128 x 128 orthogonal fp32 matrix,
+ * row-major, and takes the place of H_128 D / sqrt(128):
+ *   forward  y_i = sum_j Q[i][j] x_j,  u = y * alpha;
+ *   inverse  z = (point [- d]) * fp32(1 / alpha),  x_j = sum_i Q[i][j] z_i.
+ * Each sum is one fmaf per term, in increasing index, from +0.  Pinned by the
+ * basis-vector cases (a single nonzero term is exact: a column or a row of Q)
+ * and by the round trip Q^T (Q x) = x within fp32 rounding. */
+void hqref_rotate_fwd(const float *Q, const float *x, float *y)
+{
+    for (int i = 0; i < 128; i++) {
+        float acc = 0.0f;
+        for (int j = 0; j < 128; j++) acc = fmaf(Q[i * 128 + j], x[j], acc);
+        y[i] = acc;
+    }
+}
+
+void hqref_rotate_inv(const float *Q, const float *z, float *x)
+{
+    for (int j = 0; j < 128; j++) {
+        float acc = 0.0f;
+        for (int i = 0; i < 128; i++) acc = fmaf(Q[i * 128 + j], z[i], acc);
+        x[j] = acc;
+    }
+}
+
+float hqref_scale_inv_rot(float alpha) { return (float)(1.0 / (double)alpha); }
+
+void hqref_quantize_tile_rot(const uint16_t *x, int lat, float alpha, const float *Q, uint64_t seed, int dither,
+                             uint64_t e0, int32_t *q)
+{
+    float xf[128], v[128];
+    for (int i = 0; i < 128; i++) xf[i] = hqref_bf16_to_f32(x[i]);
+    hqref_rotate_fwd(Q, xf, v);
+    for (int i = 0; i < 128; i++) v[i] = v[i] * alpha;
+    quantize_blocks(v, lat, seed, dither, e0, q);
+}
+
+void hqref_dequantize_tile_rot(const int32_t *q, int lat, float alpha, const float *Q, uint64_t seed, int dither,
+                               uint64_t e0, float *out)
+{
+    float v[128];
+    dequantize_blocks(q, lat, seed, dither, e0, v);
+    float e = hqref_scale_inv_rot(alpha);
+    for (int i = 0; i < 128; i++) v[i] = v[i] * e;
+    hqref_rotate_inv(Q, v, out);
+}
+
+/* Gaussian draw e of the rotation generator [R18]: h = splitmix64(seed ^ "ROTN",
+ * e), u1 = (hi32(h) + 1/2) 2^-32 in (0, 1), u2 = lo32(h) 2^-32 in [0, 1),
+ * g = sqrt(-2 ln u1) cos(2 pi u2) (the Box-Muller transform, cosine branch), in
+ * double.  Pinned by a Kolmogorov-Smirnov test against the normal CDF. */
+double hqref_rot_gaussian(uint64_t seed, uint64_t e)
+{
+    const double two_pi = 6.283185307179586476925;
+    uint64_t h = hqref_splitmix64(seed ^ 0x524F544EULL, e);
+    double u1 = ((double)(h >> 32) + 0.5) * 0x1p-32;
+    double u2 = (double)(h & 0xFFFFFFFFULL) * 0x1p-32;
+    return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -533,6 +609,7 @@ typedef struct {
     const uint16_t *x;
     int64_t rows, cols, ld;              /* weights */
     int64_t H, T, ld_tok, ld_head, tok0; /* kv */
+    const float *rot;                    /* kv: dense rotation [R17], or NULL for H_128 D */
 } tiles_t;
 
 static int64_t n_chunks_of(const tiles_t *t)
@@ -585,7 +662,10 @@ static int64_t encode_all(const tiles_t *t, int lat, float alpha, int k, uint64_
             uint64_t scol, e0;
             int64_t a, b;
             if (!tile_of(t, c, i, &p, &scol, &e0, &a, &b)) break;
-            hqref_quantize_tile(p, lat, alpha, seed, scol, dither, e0, q + i * 128);
+            if (t->rot)
+                hqref_quantize_tile_rot(p, lat, alpha, t->rot, seed, dither, e0, q + i * 128);
+            else
+                hqref_quantize_tile(p, lat, alpha, seed, scol, dither, e0, q + i * 128);
             nt++;
         }
         uint64_t pb = 0;
@@ -623,7 +703,10 @@ static int decode_all(const tiles_t *t, int lat, float alpha, int k, uint64_t se
         }
         for (int i = 0; i < nt; i++) {
             float f[128];
-            hqref_dequantize_tile(q + i * 128, lat, alpha, seed, sc[i], dither, ee[i], f);
+            if (t->rot)
+                hqref_dequantize_tile_rot(q + i * 128, lat, alpha, t->rot, seed, dither, ee[i], f);
+            else
+                hqref_dequantize_tile(q + i * 128, lat, alpha, seed, sc[i], dither, ee[i], f);
             int64_t off;
             if (t->kv) {
                 int64_t tok = t->tok0 + rt[i];
@@ -680,10 +763,12 @@ int hqref_dequantize(const uint32_t *stream, const uint64_t *offsets, int64_t ro
 }
 
 /* KV append [R15]: the chunks of one append are written from base_word on;
- * offsets gets n_chunks + 1 entries (absolute word indices). */
+ * offsets gets n_chunks + 1 entries (absolute word indices).  rot: the dense
+ * rotation [R17], or NULL for H_128 D. */
 int64_t hqref_kv_append(const uint16_t *kv, int64_t H, int64_t T, int64_t ld_tok, int64_t ld_head, int64_t tok0,
                         int lat, float alpha, int k, uint64_t seed, int dither, uint32_t *stream,
-                        uint64_t base_word, uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits)
+                        uint64_t base_word, uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits,
+                        const float *rot)
 {
     tiles_t t = {0};
     t.kv = 1;
@@ -693,6 +778,7 @@ int64_t hqref_kv_append(const uint16_t *kv, int64_t H, int64_t T, int64_t ld_tok
     t.ld_tok = ld_tok;
     t.ld_head = ld_head;
     t.tok0 = tok0;
+    t.rot = rot;
     return encode_all(&t, lat, alpha, k, seed, dither, 0, n_chunks_of(&t), stream, base_word, cap_words, offsets,
                       payload_bits);
 }
@@ -701,13 +787,14 @@ int64_t hqref_kv_append(const uint16_t *kv, int64_t H, int64_t T, int64_t ld_tok
  * tokens at or beyond len skipped. */
 int hqref_kv_read_append(const uint32_t *stream, const uint64_t *offsets, int64_t H, int64_t T, int64_t tok0,
                          int lat, float alpha, int k, uint64_t seed, int dither, int out_fp32, void *out,
-                         int64_t out_ld_tok, int64_t out_ld_head, int64_t len)
+                         int64_t out_ld_tok, int64_t out_ld_head, int64_t len, const float *rot)
 {
     tiles_t t = {0};
     t.kv = 1;
     t.H = H;
     t.T = T;
     t.tok0 = tok0;
+    t.rot = rot;
     return decode_all(&t, lat, alpha, k, seed, dither, 0, n_chunks_of(&t), stream, offsets, out_fp32, out,
                       out_ld_tok, out_ld_head, len);
 }

@@ -48,6 +48,15 @@ void hqref_quantize_tile(const uint16_t *x, int lat, float alpha, uint64_t seed,
 void hqref_dequantize_tile(const int32_t *q, int lat, float alpha, uint64_t seed, uint64_t sign_col0, int dither,
                            uint64_t e0, float *out);
 
+void hqref_rotate_fwd(const float *Q, const float *x, float *y);
+void hqref_rotate_inv(const float *Q, const float *z, float *x);
+float hqref_scale_inv_rot(float alpha);
+void hqref_quantize_tile_rot(const uint16_t *x, int lat, float alpha, const float *Q, uint64_t seed, int dither,
+                             uint64_t e0, int32_t *q);
+void hqref_dequantize_tile_rot(const int32_t *q, int lat, float alpha, const float *Q, uint64_t seed, int dither,
+                               uint64_t e0, float *out);
+double hqref_rot_gaussian(uint64_t seed, uint64_t e);
+
 int64_t hqref_n_chunks(int64_t rows, int64_t cols);
 int64_t hqref_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int lat, float alpha, int k,
                        uint64_t seed, int dither, int64_t chunk_lo, int64_t chunk_hi, uint32_t *stream,
@@ -57,9 +66,10 @@ int hqref_dequantize(const uint32_t *stream, const uint64_t *offsets, int64_t ro
                      int out_fp32, void *out, int64_t ld);
 int64_t hqref_kv_append(const uint16_t *kv, int64_t H, int64_t T, int64_t ld_tok, int64_t ld_head, int64_t tok0,
                         int lat, float alpha, int k, uint64_t seed, int dither, uint32_t *stream,
-                        uint64_t base_word, uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits);
+                        uint64_t base_word, uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits,
+                        const float *rot);
 int hqref_kv_read_append(const uint32_t *stream, const uint64_t *offsets, int64_t H, int64_t T, int64_t tok0,
                          int lat, float alpha, int k, uint64_t seed, int dither, int out_fp32, void *out,
-                         int64_t out_ld_tok, int64_t out_ld_head, int64_t len);
+                         int64_t out_ld_tok, int64_t out_ld_head, int64_t len, const float *rot);
 
 #endif

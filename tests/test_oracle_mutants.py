@@ -8,6 +8,7 @@ import pytest
 
 import oracle as O
 import test_oracle_pins as P
+import test_oracle_rotation as PR
 
 # (what the mistake is, text to find, replacement, pins expected to catch it)
 MUTANTS = [
@@ -43,6 +44,19 @@ MUTANTS = [
     ("Rice unary drops a bit of the quotient", "pos += z[i] >> k;\n            put_bit(un, pos++, 1);",
      "pos += z[i] >> (k + 1);\n            put_bit(un, pos++, 1);",
      [lambda: P.test_chunk_planes_roundtrip_and_same_bits_as_concatenated(O.E8, 2)]),
+    ("forward rotation uses Q transposed", "acc = fmaf(Q[i * 128 + j], x[j], acc);",
+     "acc = fmaf(Q[j * 128 + i], x[j], acc);", [PR.test_rotation_of_basis_vectors_is_exact]),
+    ("inverse rotation not transposed", "acc = fmaf(Q[i * 128 + j], z[i], acc);",
+     "acc = fmaf(Q[j * 128 + i], z[i], acc);",
+     [PR.test_rotation_of_basis_vectors_is_exact, lambda: PR.test_rotated_roundtrip_error_within_covering_bound(O.E8)]),
+    ("rotated inverse scale keeps the Hadamard 1/sqrt(128)",
+     "float hqref_scale_inv_rot(float alpha) { return (float)(1.0 / (double)alpha); }",
+     "float hqref_scale_inv_rot(float alpha) { return (float)(1.0 / ((double)alpha * sqrt(128.0))); }",
+     [PR.test_rotated_dithered_reconstruction_is_unbiased_regression]),
+    ("Box-Muller radius loses its factor 2", "return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);",
+     "return sqrt(-log(u1)) * cos(two_pi * u2);", [PR.test_gaussian_draws_are_standard_normal]),
+    ("Gaussian radius from one bit too few", "double u1 = ((double)(h >> 32) + 0.5) * 0x1p-32;",
+     "double u1 = ((double)(h >> 33) + 0.5) * 0x1p-32;", [PR.test_gaussian_draws_are_standard_normal]),
 ]
 
 
