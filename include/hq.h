@@ -9,7 +9,10 @@
  * (Walsh-Hadamard) -> scale by alpha / sqrt(128) -> [+ dither d] -> nearest
  * point of the lattice (Z, A2, D4 or E8 in an integer embedding) -> strip the
  * membership-implied bits -> zigzag -> Rice code with parameter k into a
- * chunked bitstream.  The inverse undoes every step.
+ * chunked bitstream.  The inverse undoes every step.  A KV cache may instead
+ * rotate each token's head vector by a full Haar-uniform 128 x 128 orthogonal
+ * matrix ("Methodology" 4: a per-layer rotation, full Haar-uniform or the cheap
+ * sign diagonal); see hq_params.rotation and hq_haar_rotation.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -88,11 +91,20 @@ enum hq_lattice { HQ_Z = 0, HQ_A2 = 1, HQ_D4 = 2, HQ_E8 = 3 };
 typedef struct hq_params {
     int32_t tile;        /* elements per RHT tile; must be 128 */
     int32_t lattice;     /* enum hq_lattice */
-    float alpha;         /* scale: u = H_128 D x * alpha / sqrt(128); finite, > 0 */
+    float alpha;         /* scale: u = H_128 D x * alpha / sqrt(128) (or (Q x) * alpha); finite, > 0 */
     int32_t rice_k;      /* Rice parameter, 0..15 */
     uint64_t seed;       /* seeds the sign diagonal D and the dither */
     int32_t dither;      /* 0: none; 1: subtractive dither (page section 4; the KV path) */
     int32_t chunk_tiles; /* tiles per chunk; must be 32 */
+    const float *rotation; /* KV caches only (hq_kv_init, hq_rate_kv, hq_calibrate_kv); NULL elsewhere.
+                            * NULL: the sign diagonal D and H_128 (the default).  Otherwise device
+                            * memory, 16-byte aligned: a 128 x 128 orthogonal fp32 matrix Q,
+                            * row-major, used in place of H_128 D / sqrt(128):
+                            *   u_i = (sum_j Q[i][j] x_j) * alpha,
+                            *   x_hat_j = sum_i Q[i][j] ((point - d)_i * fp32(1 / alpha)),
+                            * each sum one fp32 fma per term in increasing index from +0.  Must
+                            * stay valid and unchanged while the cache is in use.  The weights
+                            * entry points return HQ_EUNSUPPORTED when it is set.  40 bytes. */
 } hq_params;
 
 /* Device-resident statistics written by the kernels (zeroed by each call
@@ -112,8 +124,8 @@ typedef struct hq_kv_append_row {
     int64_t token0;       /* first token of the append */
     int32_t tokens;       /* T */
     float alpha;          /* alpha used for this append */
-    float scale_fwd;      /* fp32(alpha / sqrt(128)) */
-    float scale_inv;      /* fp32(1 / (alpha * sqrt(128))) */
+    float scale_fwd;      /* fp32(alpha / sqrt(128)); alpha with a dense rotation */
+    float scale_inv;      /* fp32(1 / (alpha * sqrt(128))); fp32(1 / alpha) with a dense rotation */
 } hq_kv_append_row;
 
 /* A compressed KV cache for one of K or V of one layer (page section 4: KV
@@ -307,7 +319,9 @@ HQ_API int hq_calibrate_kv(const void *kv, int32_t heads, int64_t T, int64_t ld_
 
 /* Fill a hq_kv_cache with the caller's buffers and zero its two tail words
  * and its stats (two small cudaMemsetAsync on cuda_stream).  p->dither is
- * normally 1; p->alpha is unused (each append gives its own). */
+ * normally 1; p->alpha is unused (each append gives its own).  p->rotation, if
+ * set, rotates every append, read and score of this cache (the table rows then
+ * hold scale_fwd = alpha and scale_inv = fp32(1 / alpha)). */
 HQ_API int hq_kv_init(hq_kv_cache *cache, int32_t heads, int32_t head_dim, const hq_params *p, uint32_t *d_words,
                uint64_t cap_words, uint64_t *d_offsets, uint64_t offsets_cap, hq_kv_append_row *d_table,
                uint64_t table_cap, uint64_t *d_tail, hq_stats *d_stats, void *cuda_stream);
@@ -340,6 +354,18 @@ HQ_API int hq_kv_read(const hq_kv_cache *cache, void *out, int out_dtype, int64_
  * Status bits go to the cache's d_stats as for hq_kv_read.  Asynchronous. */
 HQ_API int hq_kv_scores(const hq_kv_cache *cache, const void *d_q, int32_t group, float *d_scores, int64_t len,
                         int64_t scores_ld, void *cuda_stream);
+
+/* Draw a Haar-uniform rotation for hq_params.rotation: d_q (device, 16-byte
+ * aligned, 128 x 128 fp32 row-major) = the orthogonal factor Q of G = Q R with R
+ * upper triangular and positive on its diagonal, where G[i][j] is the standard
+ * normal draw e = 128 i + j: h = splitmix64(seed ^ 0x524F544E, e), u1 = (h >> 32
+ * + 1/2) 2^-32, u2 = (h & 0xFFFFFFFF) 2^-32, g = sqrt(-2 ln u1) cos(2 pi u2).  That
+ * factor is Haar-distributed on O(128) (Mezzadri 2007).  Computed in double on one
+ * CTA (modified Gram-Schmidt) and rounded once to fp32; another QR method gives the
+ * same fp32 matrix to within one unit in the last place.  One call per cache
+ * (per layer and K/V, each with its own seed); asynchronous on cuda_stream.
+ * HQ_EINVAL for a null or misaligned d_q. */
+HQ_API int hq_haar_rotation(uint64_t seed, float *d_q, void *cuda_stream);
 
 /* ---------------------------------------------------------------- misc */
 

@@ -28,7 +28,7 @@ HQ_ST_CAPACITY, HQ_ST_CORRUPT, HQ_ST_TIMEOUT, HQ_ST_RANGE = 1, 2, 4, 8
 
 class hq_params(C.Structure):
     _fields_ = [("tile", C.c_int32), ("lattice", C.c_int32), ("alpha", C.c_float), ("rice_k", C.c_int32),
-                ("seed", C.c_uint64), ("dither", C.c_int32), ("chunk_tiles", C.c_int32)]
+                ("seed", C.c_uint64), ("dither", C.c_int32), ("chunk_tiles", C.c_int32), ("rotation", C.c_void_p)]
 
 
 class hq_stats(C.Structure):
@@ -59,8 +59,8 @@ class hq_calib_result(C.Structure):
 
 
 assert C.sizeof(hq_calib_spec) == 48 and C.sizeof(hq_calib_result) == 24
-assert C.sizeof(hq_params) == 32 and C.sizeof(hq_stats) == 32 and C.sizeof(hq_kv_append_row) == 32
-assert C.sizeof(hq_kv_cache) == 128
+assert C.sizeof(hq_params) == 40 and C.sizeof(hq_stats) == 32 and C.sizeof(hq_kv_append_row) == 32
+assert C.sizeof(hq_kv_cache) == 136
 
 # C entry points: name -> (restype, argtypes)
 EXPORTS = {
@@ -98,6 +98,7 @@ EXPORTS = {
     "hq_debug_set_spin_limit": (None, [C.c_uint32]),
     "hq_quantize_static": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.POINTER(hq_params), C.c_void_p,
                                      C.c_uint64, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "hq_haar_rotation": (C.c_int, [C.c_uint64, C.c_void_p, C.c_void_p]),
 }
 
 
@@ -140,9 +141,16 @@ def _stream(s) -> int | None:
     return int(s)
 
 
-def make_params(lattice="E8", alpha=1.0, rice_k=2, seed=0, dither=0) -> hq_params:
+def make_params(lattice="E8", alpha=1.0, rice_k=2, seed=0, dither=0, rotation: torch.Tensor | None = None) -> hq_params:
+    """rotation: a KV cache's dense rotation (fp32 [128, 128] on the device, e.g. from
+    hq_haar_rotation), or None for the sign diagonal and H_128.  The params hold only its
+    address: the caller keeps the tensor alive and unchanged."""
     lat = LATTICES[lattice] if isinstance(lattice, str) else int(lattice)
-    return hq_params(128, lat, float(alpha), int(rice_k), int(seed) & (2**64 - 1), int(dither), 32)
+    rot = None
+    if rotation is not None:
+        assert rotation.dtype == torch.float32 and rotation.is_contiguous() and tuple(rotation.shape) == (128, 128)
+        rot = rotation.data_ptr()
+    return hq_params(128, lat, float(alpha), int(rice_k), int(seed) & (2**64 - 1), int(dither), 32, rot)
 
 
 # ------------------------------------------------------------------ C entry points
@@ -227,6 +235,15 @@ def hq_calibrate_kv(kv: torch.Tensor, params: hq_params, spec: hq_calib_spec, st
     _check(_lib.hq_calibrate_kv(_ptr(kv), H, T, kv.stride(1), kv.stride(0), tok0, C.byref(params), C.byref(spec),
                                 _ptr(stats), _stream(cuda_stream), C.byref(out)), "hq_calibrate_kv")
     return _calib_result(out)
+
+
+def hq_haar_rotation(seed: int, out: torch.Tensor | None = None, cuda_stream=None) -> torch.Tensor:
+    """A Haar-uniform 128 x 128 orthogonal fp32 matrix drawn on the device for this seed."""
+    if out is None:
+        out = torch.empty(128, 128, dtype=torch.float32, device="cuda")
+    assert out.dtype == torch.float32 and out.is_contiguous() and tuple(out.shape) == (128, 128)
+    _check(_lib.hq_haar_rotation(int(seed) & (2**64 - 1), _ptr(out), _stream(cuda_stream)), "hq_haar_rotation")
+    return out
 
 
 def hq_debug_set_encode_path(path: int) -> int:
@@ -367,10 +384,18 @@ class Codec:
 
 
 class KVCache:
-    """A compressed K or V cache (one layer) with torch-allocated device buffers."""
+    """A compressed K or V cache (one layer) with torch-allocated device buffers.
+    rotation: a dense rotation for this cache (fp32 [128, 128], e.g. hq_haar_rotation(seed)),
+    used in place of the sign diagonal and H_128; the cache keeps a reference to it."""
 
     def __init__(self, heads: int, max_tokens: int, params: hq_params, bits_per_scalar: float = 4.0,
-                 max_appends: int = 4096, max_append_tokens: int = 4096, device="cuda"):
+                 max_appends: int = 4096, max_append_tokens: int = 4096, device="cuda",
+                 rotation: torch.Tensor | None = None):
+        if rotation is not None:
+            assert rotation.dtype == torch.float32 and rotation.is_contiguous() and tuple(rotation.shape) == (128, 128)
+            params = hq_params.from_buffer_copy(bytes(params))
+            params.rotation = rotation.data_ptr()
+        self.rotation = rotation
         max_chunks = heads * ((max_tokens + 31) // 32 + max_appends)
         cap = int(heads * max_tokens * 128 * bits_per_scalar / 32) + max_chunks * 64 + 1024
         self.words = torch.empty(cap, dtype=torch.int32, device=device)

@@ -28,7 +28,15 @@ int check_params(const hq_params *p) {
     if (p->rice_k < 0 || p->rice_k > 15) return HQ_EINVAL;
     if (p->dither != 0 && p->dither != 1) return HQ_EINVAL;
     if (p->tile != kTile || p->chunk_tiles != kChunkTiles) return HQ_EUNSUPPORTED;
+    if (p->rotation && !aligned(p->rotation, 16)) return HQ_EINVAL;
     return HQ_OK;
+}
+
+// The weights entry points take no dense rotation (a KV-cache option).
+int check_weight_params(const hq_params *p) {
+    const int rc = check_params(p);
+    if (rc) return rc;
+    return p->rotation ? HQ_EUNSUPPORTED : HQ_OK;
 }
 
 int check_matrix(int64_t rows, int64_t cols) {
@@ -45,6 +53,12 @@ uint64_t chunks_of(int64_t rows, int64_t cols) {
 
 float scale_fwd(float alpha) { return (float)((double)alpha / sqrt(128.0)); }
 float scale_inv(float alpha) { return (float)(1.0 / ((double)alpha * sqrt(128.0))); }
+// With the dense rotation Q (orthonormal: no 1/sqrt(128) to fold in): u = (Q x) alpha,
+// and the inverse scales by fp32(1 / alpha).
+float scale_fwd_of(const hq_params &p, float alpha) { return p.rotation ? alpha : scale_fwd(alpha); }
+float scale_inv_of(const hq_params &p, float alpha) {
+    return p.rotation ? (float)(1.0 / (double)alpha) : scale_inv(alpha);
+}
 
 size_t ws_bytes_for(uint64_t n_chunks) {
     const size_t b = encode_scratch_bytes(n_chunks);
@@ -102,7 +116,7 @@ int hq_workspace_bytes(uint64_t n_chunks, size_t *bytes) {
 int hq_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p, uint32_t *d_stream,
                 uint64_t cap_words, uint64_t *d_offsets, hq_stats *d_stats, void *workspace, size_t ws_bytes,
                 void *cuda_stream) {
-    int rc = check_params(p);
+    int rc = check_weight_params(p);
     if (rc) return rc;
     if ((rc = check_matrix(rows, cols))) return rc;
     const uint64_t nch = chunks_of(rows, cols);
@@ -146,7 +160,7 @@ int hq_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_
 int hq_dequantize(const uint32_t *d_stream, uint64_t stream_words, const uint64_t *d_offsets, int64_t rows,
                   int64_t cols, const hq_params *p, void *out, int out_dtype, int64_t ld, hq_stats *d_stats,
                   void *cuda_stream) {
-    int rc = check_params(p);
+    int rc = check_weight_params(p);
     if (rc) return rc;
     if ((rc = check_matrix(rows, cols))) return rc;
     if (out_dtype != 0 && out_dtype != 1) return HQ_EINVAL;
@@ -190,7 +204,7 @@ int hq_gemv_workspace_bytes(int64_t rows, int64_t cols, size_t *bytes) {
 int hq_gemv(const uint32_t *d_stream, uint64_t stream_words, const uint64_t *d_offsets, int64_t rows, int64_t cols,
             const hq_params *p, const void *d_x, float *d_y, void *workspace, size_t ws_bytes, hq_stats *d_stats,
             void *cuda_stream) {
-    int rc = check_params(p);
+    int rc = check_weight_params(p);
     if (rc) return rc;
     if ((rc = check_matrix(rows, cols))) return rc;
     if (d_stats && !aligned(d_stats, 8)) return HQ_EINVAL;
@@ -232,6 +246,7 @@ int hq_kv_init(hq_kv_cache *cache, int32_t heads, int32_t head_dim, const hq_par
     if (p->lattice < HQ_Z || p->lattice > HQ_E8 || p->rice_k < 0 || p->rice_k > 15) return HQ_EINVAL;
     if (p->dither != 0 && p->dither != 1) return HQ_EINVAL;
     if (p->tile != kTile || p->chunk_tiles != kChunkTiles) return HQ_EUNSUPPORTED;
+    if (p->rotation && !aligned(p->rotation, 16)) return HQ_EINVAL;
     if (head_dim != kTile) return HQ_EUNSUPPORTED;
     if (heads <= 0) return HQ_EINVAL;
     if (!d_words || !aligned(d_words, 4) || !d_offsets || !aligned(d_offsets, 8) || offsets_cap < 1) return HQ_EINVAL;
@@ -284,9 +299,10 @@ int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t ld_token
     a.map.tok0 = cache->tokens;
     a.n_chunks = nch;
     a.chunk_base = cache->chunks;
-    a.c_scale = scale_fwd(alpha);
+    a.c_scale = scale_fwd_of(p, alpha);
     a.k = p.rice_k;
     a.seed = p.seed;
+    a.rot = p.rotation;
     a.stream = cache->d_words;
     a.cap_words = cache->cap_words;
     a.offsets = cache->d_offsets;
@@ -298,7 +314,7 @@ int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t ld_token
     a.row_val.tokens = (int32_t)T;
     a.row_val.alpha = alpha;
     a.row_val.scale_fwd = a.c_scale;
-    a.row_val.scale_inv = scale_inv(alpha);
+    a.row_val.scale_inv = scale_inv_of(p, alpha);
     a.stats = cache->d_stats;
     a.stats_add = 1;
     set_scratch(a, workspace, nch);
@@ -340,6 +356,7 @@ int hq_kv_read(const hq_kv_cache *cache, void *out, int out_dtype, int64_t len, 
     a.n_appends = cache->appends;
     a.stats = cache->d_stats;
     a.tcols = 1;
+    a.rot = cache->params.rotation;
     return cuda_rc(launch_decode(cache->params.lattice, cache->params.dither, a, (cudaStream_t)cuda_stream));
 }
 
@@ -352,9 +369,10 @@ namespace {
 int rate_launch(const hq_params *p, EncodeArgs &a, hq_stats *d_stats, cudaStream_t s) {
     if (cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
     if (a.n_chunks == 0) return HQ_OK;
-    a.c_scale = scale_fwd(p->alpha);
+    a.c_scale = scale_fwd_of(*p, p->alpha);
     a.k = p->rice_k;
     a.seed = p->seed;
+    a.rot = p->rotation;
     a.stats = d_stats;
     return cuda_rc(launch_rate(p->lattice, p->dither, a, s));
 }
@@ -470,7 +488,7 @@ extern "C" {
 
 int hq_rate(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p, hq_stats *d_stats,
             void *cuda_stream) {
-    int rc = check_params(p);
+    int rc = check_weight_params(p);
     if (rc) return rc;
     if (!d_stats || !aligned(d_stats, 8)) return HQ_EINVAL;
     EncodeArgs a;
@@ -493,6 +511,7 @@ int hq_calibrate(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq
     EncodeArgs a;
     int rc = weights_rate_args(x, rows, cols, ld, a);
     if (rc) return rc;
+    if (p && p->rotation) return HQ_EUNSUPPORTED;
     return calibrate(p, spec, a, (double)rows * (double)cols, d_stats, (cudaStream_t)cuda_stream, out);
 }
 
@@ -531,6 +550,7 @@ int hq_kv_scores(const hq_kv_cache *cache, const void *d_q, int32_t group, float
     a.vec = (const uint16_t *)d_q;
     a.res = d_scores;
     a.group = group;
+    a.rot = cache->params.rotation;
     return cuda_rc(launch_kv_scores(cache->params.lattice, cache->params.dither, a, (cudaStream_t)cuda_stream));
 }
 
@@ -557,6 +577,11 @@ int hq_device_check(void) {
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return HQ_ECUDA;
     if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return HQ_ECUDA;
     return (major == 10 && minor == 0) ? HQ_OK : HQ_EUNSUPPORTED;
+}
+
+int hq_haar_rotation(uint64_t seed, float *d_q, void *cuda_stream) {
+    if (!d_q || !aligned(d_q, 16)) return HQ_EINVAL;
+    return cuda_rc(launch_haar(seed, d_q, (cudaStream_t)cuda_stream));
 }
 
 void hq_debug_set_spin_limit(uint32_t polls) { g_spin_limit = polls ? polls : kSpinLimit; }

@@ -71,6 +71,7 @@ cudaError_t launch_gemv(int lattice, int dither, const DecodeArgs &a, float *y, 
 }
 
 cudaError_t launch_kv_scores(int lattice, int dither, const DecodeArgs &a, cudaStream_t s) {
+    if (a.rot) return launch_kv_scores_rot(lattice, dither, a, s);
     return dispatch<true, kKvScores>(lattice, dither, a, s);
 }
 

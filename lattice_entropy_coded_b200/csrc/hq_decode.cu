@@ -46,6 +46,7 @@ cudaError_t dispatch(int lattice, int dither, const DecodeArgs &a, cudaStream_t 
 }  // namespace
 
 cudaError_t launch_decode(int lattice, int dither, const DecodeArgs &a, cudaStream_t s) {
+    if (a.rot) return launch_decode_rot(lattice, dither, a, s);
     return a.map.kv ? dispatch<true>(lattice, dither, a, s) : dispatch<false>(lattice, dither, a, s);
 }
 

@@ -20,7 +20,8 @@
 //    shift per symbol), its k remainder bits from its own fixed region, and
 //    rebuilds and scales the lattice points;
 //  * the inverse FWHT runs in registers (two stages across the four lanes by
-//    shuffle), followed by the sign flip and 16-byte stores.
+//    shuffle), followed by the sign flip and 16-byte stores; or, for a KV cache
+//    with the dense rotation, x = Q^T z with Q^T in shared memory (rotate_quarter).
 // Chunks are independent (their offsets are given), so there is no look-back.
 #pragma once
 
@@ -317,10 +318,13 @@ __device__ __forceinline__ float tile_sum(float acc) {
     return __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
 }
 
-template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED, int MODE>
+// ROT: the dense KV rotation's inverse (rot_s: its shared form) in place of H_128
+// and the sign diagonal.
+template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED, int MODE, bool ROT>
 __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOut<KV> &geo, const uint32_t *src,
                                               bool ok, uint32_t nc, uint32_t nr, uint32_t nu,
-                                              const uint32_t *startbit, const uint32_t *sign_tab, int lane) {
+                                              const uint32_t *startbit, const uint32_t *sign_tab,
+                                              const float *rot_s, int lane) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
     const int k = a.k;
@@ -400,13 +404,23 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
             for (int j = 0; j < 16; j++) v[j] = make_float2(0.0f, 0.0f);
         }
         if (valid && !lane_ok) bad = true;
-        fwht128_quarter(v, lane);
+        if constexpr (ROT) {
+            uint32_t in[32];
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+                in[2 * j] = __float_as_uint(v[j].x);
+                in[2 * j + 1] = __float_as_uint(v[j].y);
+            }
+            rotate_quarter<false, 32>(in, v, rot_s, lane);
+        } else {
+            fwht128_quarter(v, lane);
+        }
         // a tile is written as zeros unless all four of its lanes decoded
         const unsigned bad_lanes = __ballot_sync(0xffffffffu, valid && !lane_ok);
         const bool tile_bad = (bad_lanes >> (lane & ~3)) & 0xFu;
         if constexpr (MODE != kStoreTiles) {
             // the tile as hq_dequantize stores it in bf16, then dot products with the vector(s)
-            const uint32_t es = sign_tab[tcol * kSignWords + q];
+            const uint32_t es = ROT ? 0u : sign_tab[tcol * kSignWords + q];
             uint32_t w[16];
 #pragma unroll
             for (int j = 0; j < 16; j++) {
@@ -425,7 +439,7 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
                 }
             }
         } else if (dst) {
-            const uint32_t es = sign_tab[tcol * kSignWords + q];
+            const uint32_t es = ROT ? 0u : sign_tab[tcol * kSignWords + q];
             if (a.out_fp32) {
                 uint4 *o = reinterpret_cast<uint4 *>(dst) + 8 * q;
 #pragma unroll
@@ -457,19 +471,24 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
 }
 
 // Three CTAs (24 warps) per SM without dither, where the decoder fits 80 registers with
-// almost no spills; two with dither, whose second lattice search needs more.
-template <int LAT, bool DITHER, bool KV, bool KSMALL, int MODE>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, DITHER ? 2 : 3) decode_kernel(const DecodeArgs a) {
+// almost no spills; two with dither, whose second lattice search needs more; one with
+// the dense rotation, whose shared form (kRotSmemBytes) comes first.
+template <int LAT, bool DITHER, bool KV, bool KSMALL, int MODE, bool ROT = false>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : (DITHER ? 2 : 3)) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int kStageSlot = kStageWords + kStagePad;
-    uint32_t *sign_tab = smem;
-    uint32_t *stage_all = smem + a.tcols * kSignWords;
+    const float *rot_s = ROT ? reinterpret_cast<const float *>(smem) : nullptr;
+    uint32_t *sign_tab = smem + (ROT ? kRotSmemBytes / sizeof(uint32_t) : 0);
+    uint32_t *stage_all = sign_tab + a.tcols * kSignWords;
     uint32_t *start_all = stage_all + kWarpsPerCta * 2 * kStageSlot;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t *stages = stage_all + warp * 2 * kStageSlot;
     uint32_t *startbit = start_all + warp * 128;   // first unary bit of every 32-symbol segment
 
-    build_sign_table(sign_tab, a.tcols, a.seed);
+    if (ROT)
+        load_rotation<false>(reinterpret_cast<float *>(smem), a.rot);
+    else
+        build_sign_table(sign_tab, a.tcols, a.seed);
     __syncthreads();
 
     const int k = a.k;
@@ -511,11 +530,13 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, DITHER ? 2 : 3) decode_kern
         if (staged) {
             const uint32_t *src = stages + buf * kStageSlot;
             ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
-            bad = decode_rounds<LAT, DITHER, KV, KSMALL, true, MODE>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab, lane);
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, true, MODE, ROT>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab,
+                                                                          rot_s, lane);
         } else {
             const uint32_t *src = a.stream + cw.w0;
             ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
-            bad = decode_rounds<LAT, DITHER, KV, KSMALL, false, MODE>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab, lane);
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, false, MODE, ROT>(a, geo, src, ok, nc, nr, nu, startbit,
+                                                                           sign_tab, rot_s, lane);
         }
         if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) status |= HQ_ST_CORRUPT;
         cw = cwn;

@@ -154,6 +154,73 @@ __device__ __forceinline__ void fwht128_sixteenth(float2 (&v)[4], int lane) {
     }
 }
 
+// ------------------------------------------------------------------ dense rotation (KV)
+// The KV path may rotate each token's head vector by a full 128 x 128 orthogonal
+// matrix Q (a Haar-uniform draw) instead of the sign diagonal and H_128 (explainer
+// pages, "Methodology" 4).  Forward y = Q x, inverse x = Q^T z; each output is one
+// fp32 fma per term in increasing input index from +0.
+//
+// rotate_quarter applies a matrix M to a tile held in the FWHT's quarter layout:
+// lane q = lane & 3 of the tile holds inputs and outputs [32q, 32q + 32).  Input k
+// lives in lane 4 (lane / 4) + k / 32 and reaches the tile's four lanes by shuffle.
+// M sits in shared memory with row k (pitch kRotPitch floats) holding M[o][k] of
+// the 128 outputs o at rot_pos(o) = 16 m + 4 q + r for o = 32 q + 4 m + r: for one
+// (k, m) the four quarters' float4 are adjacent, one 64-byte wavefront broadcast
+// to the warp's eight tiles.  The pitch keeps rows 16-byte aligned and limits the
+// transposing writes of load_rotation to 4-way bank conflicts.
+constexpr int kRotPitch = 132;
+constexpr size_t kRotSmemBytes = (size_t)128 * kRotPitch * sizeof(float);
+
+__device__ __forceinline__ int rot_pos(int o) { return ((o & 31) >> 2) * 16 + (o >> 5) * 4 + (o & 3); }
+
+// Shared form of M from the row-major fp32 Q in global memory (coalesced reads, by
+// the whole CTA): M = Q when FORWARD, else M = Q^T.  The caller synchronises.
+template <bool FORWARD>
+__device__ __forceinline__ void load_rotation(float *S, const float *Q) {
+    for (int idx = threadIdx.x; idx < 128 * 128; idx += blockDim.x) {
+        const int a = idx >> 7, b = idx & 127;
+        const float v = __ldg(Q + idx);
+        if (FORWARD)
+            S[b * kRotPitch + rot_pos(a)] = v;   // M[a][b] = Q[a][b]: output a, input b
+        else
+            S[a * kRotPitch + rot_pos(b)] = v;   // M[b][a] = Q[a][b]: output b, input a
+    }
+}
+
+// out (16 float2: out[j] = outputs 2j, 2j + 1 of the lane's quarter, as the FWHT
+// leaves them) = M in.  BF16: in[w] holds inputs 2w (low half) and 2w + 1 (high
+// half) of the quarter as bf16; otherwise in[w] is input w as fp32 bits.  The
+// packed fma rounds each half exactly like fmaf.  Whole warp.
+template <bool BF16, int NW>
+__device__ __forceinline__ void rotate_quarter(const uint32_t (&in)[NW], float2 (&out)[16], const float *S, int lane) {
+    static_assert(NW == (BF16 ? 16 : 32), "one quarter of a tile");
+    constexpr int P = BF16 ? 2 : 1;   // inputs per word
+    const int src0 = lane & ~3;
+    const float *Sq = S + 4 * (lane & 3);
+#pragma unroll
+    for (int j = 0; j < 16; j++) out[j] = make_float2(0.0f, 0.0f);
+#pragma unroll 1
+    for (int src = 0; src < 4; src++) {
+        const float *Sk = Sq + 32 * src * kRotPitch;
+#pragma unroll
+        for (int w = 0; w < NW; w++) {
+            const uint32_t word = __shfl_sync(0xffffffffu, in[w], src0 + src);
+#pragma unroll
+            for (int h = 0; h < P; h++) {
+                const float xk = BF16 ? __uint_as_float(h ? (word & 0xFFFF0000u) : (word << 16)) : __uint_as_float(word);
+                const float2 x2 = make_float2(xk, xk);
+                const float *row = Sk + (P * w + h) * kRotPitch;
+#pragma unroll
+                for (int m = 0; m < 8; m++) {
+                    const float4 s = *reinterpret_cast<const float4 *>(row + 16 * m);
+                    out[2 * m] = f2_fma(make_float2(s.x, s.y), x2, out[2 * m]);
+                    out[2 * m + 1] = f2_fma(make_float2(s.z, s.w), x2, out[2 * m + 1]);
+                }
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ lattices
 // Rounding without the conversion pipe: for |x| < 2^22, x + 1.5*2^23 lands in
 // [2^23, 2^24) where the fp32 spacing is 1, so the add rounds x to the nearest

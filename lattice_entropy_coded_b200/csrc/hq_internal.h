@@ -62,6 +62,7 @@ struct EncodeArgs {
     hq_stats *acc;                 // zeroed: this call's stats, moved to *stats by the last CTA
     int tcols;                // tile columns in the sign table (cols / 128, or 1 for KV)
     uint32_t spin_limit;
+    const float *rot;         // KV: the dense rotation Q (128 x 128 fp32, row-major) or null (sign diagonal, H_128)
 };
 
 struct DecodeArgs {
@@ -86,6 +87,7 @@ struct DecodeArgs {
     const uint16_t *vec;      // bf16 x [cols] (gemv) or queries [heads * group, 128] (scores)
     float *res;               // gemv: one partial per tile [rows * tcols]; scores: [heads * group, out_ld]
     int group;                // scores: query heads per KV head
+    const float *rot;         // KV: the dense rotation Q, or null
 };
 
 // Decoder outputs: the tile itself, its dot product with x, or its dot products with queries.
@@ -147,5 +149,13 @@ cudaError_t launch_kv_scores(int lattice, int dither, const DecodeArgs &a, cudaS
 // Rate only: adds payload_bits, stream_words, max_symbol and HQ_ST_RANGE of the call into a.stats
 // (zeroed by the caller); reads a.x, a.map, a.n_chunks, a.c_scale, a.k, a.seed, a.tcols.
 cudaError_t launch_rate(int lattice, int dither, const EncodeArgs &a, cudaStream_t s);
+// The same with the dense KV rotation a.rot (hq_rot_encode.cu, hq_rot_decode.cu); the launchers
+// above forward to these when a.rot is set.
+cudaError_t launch_encode_rot(int lattice, int dither, const EncodeArgs &a, cudaStream_t s);
+cudaError_t launch_rate_rot(int lattice, int dither, const EncodeArgs &a, cudaStream_t s);
+cudaError_t launch_decode_rot(int lattice, int dither, const DecodeArgs &a, cudaStream_t s);
+cudaError_t launch_kv_scores_rot(int lattice, int dither, const DecodeArgs &a, cudaStream_t s);
+// Haar-uniform rotation for the seed (hq_haar.cu): one CTA, q = 128 x 128 fp32 row-major.
+cudaError_t launch_haar(uint64_t seed, float *q, cudaStream_t s);
 
 }  // namespace hq

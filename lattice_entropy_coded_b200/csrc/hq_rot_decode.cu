@@ -1,0 +1,61 @@
+// hq_rot_decode.cu -- the decoder of a KV cache with the dense rotation (a 128 x 128
+// orthogonal matrix in place of the sign diagonal and H_128; explainer pages,
+// "Methodology" 4): hq_kv_read's stored tiles and hq_kv_scores' dot products.  The
+// kernel is hq_decode.cuh's with ROT = true, instantiated here so that it compiles in
+// parallel with the rest.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hq_decode.cuh"
+
+namespace hq {
+
+namespace {
+
+// One CTA of 8 warps per SM: the rotation's shared form (kRotSmemBytes) comes on
+// top of the two stages per warp.
+template <int LAT, bool DITHER, int MODE>
+cudaError_t launch_rot_t(const DecodeArgs &a, cudaStream_t s) {
+    const size_t smem = kRotSmemBytes + (size_t)(a.tcols * kSignWords + kWarpsPerCta * 2 * (kStageWords + kStagePad) +
+                                                 kWarpsPerCta * 128) *
+                                            sizeof(uint32_t);
+    const bool small = a.k <= 4;
+    auto kern = small ? decode_kernel<LAT, DITHER, true, true, MODE, true>
+                      : decode_kernel<LAT, DITHER, true, false, MODE, true>;
+    static LaunchPlan plans[2];
+    unsigned grid = 0;
+    cudaError_t e = plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem,
+                                               (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t dispatch(int lattice, int dither, const DecodeArgs &a, cudaStream_t s) {
+    switch (lattice * 2 + (dither ? 1 : 0)) {
+    case HQ_Z * 2: return launch_rot_t<HQ_Z, false, MODE>(a, s);
+    case HQ_Z * 2 + 1: return launch_rot_t<HQ_Z, true, MODE>(a, s);
+    case HQ_A2 * 2: return launch_rot_t<HQ_A2, false, MODE>(a, s);
+    case HQ_A2 * 2 + 1: return launch_rot_t<HQ_A2, true, MODE>(a, s);
+    case HQ_D4 * 2: return launch_rot_t<HQ_D4, false, MODE>(a, s);
+    case HQ_D4 * 2 + 1: return launch_rot_t<HQ_D4, true, MODE>(a, s);
+    case HQ_E8 * 2: return launch_rot_t<HQ_E8, false, MODE>(a, s);
+    case HQ_E8 * 2 + 1: return launch_rot_t<HQ_E8, true, MODE>(a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_rot(int lattice, int dither, const DecodeArgs &a, cudaStream_t s) {
+    if (!a.map.kv) return cudaErrorInvalidValue;
+    return dispatch<kStoreTiles>(lattice, dither, a, s);
+}
+
+cudaError_t launch_kv_scores_rot(int lattice, int dither, const DecodeArgs &a, cudaStream_t s) {
+    if (!a.map.kv) return cudaErrorInvalidValue;
+    return dispatch<kKvScores>(lattice, dither, a, s);
+}
+
+}  // namespace hq

@@ -1,0 +1,74 @@
+// hq_rot_encode.cu -- launchers of the quantize + encode kernel and of the rate pass
+// with the dense KV rotation (a 128 x 128 orthogonal matrix per cache in place of
+// the sign diagonal and H_128; explainer pages, "Methodology" 4).  The kernels are
+// the grouped form and the rate kernel of hq_encode.cuh with ROT = true; they are
+// instantiated in this file of their own so that they compile in parallel with
+// the rest.
+#include "hq_encode.cuh"
+
+namespace hq {
+
+namespace {
+
+// Every launch size takes the grouped form: four warps per chunk, one CTA of two
+// groups per SM (the rotation's 66 KB shared form).
+template <int LAT, bool DITHER>
+cudaError_t launch_rot_t(const EncodeArgs &a, cudaStream_t s) {
+    const bool small = a.k <= 4;
+    const size_t smem = kRotSmemBytes +
+                        (size_t)(a.tcols * kSignWords + kGroups * 2 * kStageWords + kWarpsPerCta * 32 * kGroupSlotWords) *
+                            sizeof(uint32_t) +
+                        kGroups * sizeof(GroupCtl);
+    auto kern = small ? encode_kernel_grouped<LAT, DITHER, true, true> : encode_kernel_grouped<LAT, DITHER, false, true>;
+    static LaunchPlan plans[2];
+    unsigned grid = 0;
+    cudaError_t e =
+        plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kGroups - 1) / kGroups, grid);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int LAT, bool DITHER>
+cudaError_t launch_rate_rot_t(const EncodeArgs &a, cudaStream_t s) {
+    const size_t smem = kRotSmemBytes + (size_t)a.tcols * kSignWords * sizeof(uint32_t);
+    auto kern = rate_kernel<LAT, DITHER, true>;
+    static LaunchPlan plan;
+    unsigned grid = 0;
+    cudaError_t e = plan.grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_encode_rot(int lattice, int dither, const EncodeArgs &a, cudaStream_t s) {
+    switch (lattice * 2 + (dither ? 1 : 0)) {
+    case HQ_Z * 2: return launch_rot_t<HQ_Z, false>(a, s);
+    case HQ_Z * 2 + 1: return launch_rot_t<HQ_Z, true>(a, s);
+    case HQ_A2 * 2: return launch_rot_t<HQ_A2, false>(a, s);
+    case HQ_A2 * 2 + 1: return launch_rot_t<HQ_A2, true>(a, s);
+    case HQ_D4 * 2: return launch_rot_t<HQ_D4, false>(a, s);
+    case HQ_D4 * 2 + 1: return launch_rot_t<HQ_D4, true>(a, s);
+    case HQ_E8 * 2: return launch_rot_t<HQ_E8, false>(a, s);
+    case HQ_E8 * 2 + 1: return launch_rot_t<HQ_E8, true>(a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_rate_rot(int lattice, int dither, const EncodeArgs &a, cudaStream_t s) {
+    switch (lattice * 2 + (dither ? 1 : 0)) {
+    case HQ_Z * 2: return launch_rate_rot_t<HQ_Z, false>(a, s);
+    case HQ_Z * 2 + 1: return launch_rate_rot_t<HQ_Z, true>(a, s);
+    case HQ_A2 * 2: return launch_rate_rot_t<HQ_A2, false>(a, s);
+    case HQ_A2 * 2 + 1: return launch_rate_rot_t<HQ_A2, true>(a, s);
+    case HQ_D4 * 2: return launch_rate_rot_t<HQ_D4, false>(a, s);
+    case HQ_D4 * 2 + 1: return launch_rate_rot_t<HQ_D4, true>(a, s);
+    case HQ_E8 * 2: return launch_rate_rot_t<HQ_E8, false>(a, s);
+    case HQ_E8 * 2 + 1: return launch_rate_rot_t<HQ_E8, true>(a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace hq

@@ -55,6 +55,7 @@ int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, co
     if (!(p->alpha > 0.0f) || !(p->alpha < __builtin_inff())) return HQ_EINVAL;
     if (p->rice_k < 0 || p->rice_k > 15 || (p->dither != 0 && p->dither != 1)) return HQ_EINVAL;
     if (p->tile != kTile || p->chunk_tiles != kChunkTiles) return HQ_EUNSUPPORTED;
+    if (p->rotation) return HQ_EUNSUPPORTED;   // the dense rotation is a KV-cache option
     if (rows < 0 || cols < 0 || cols % kTile) return HQ_EINVAL;
     if (cols > 65536) return HQ_EUNSUPPORTED;
     const uint64_t tiles = (uint64_t)rows * (uint64_t)(cols / kTile);

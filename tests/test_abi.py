@@ -34,11 +34,13 @@ def test_library_exports_every_declared_symbol():
 
 def test_struct_layouts_match_header():
     import lattice_entropy_coded_b200 as hq
-    assert C.sizeof(hq.hq_params) == 32
+    assert C.sizeof(hq.hq_params) == 40
     assert hq.hq_params.seed.offset == 16 and hq.hq_params.chunk_tiles.offset == 28
+    assert hq.hq_params.rotation.offset == 32
     assert C.sizeof(hq.hq_stats) == 32 and hq.hq_stats.payload_bits.offset == 8
     assert C.sizeof(hq.hq_kv_append_row) == 32
-    assert C.sizeof(hq.hq_kv_cache) == 128 and hq.hq_kv_cache.params.offset == 72
+    assert C.sizeof(hq.hq_kv_cache) == 136 and hq.hq_kv_cache.params.offset == 72
+    assert hq.hq_kv_cache.tokens.offset == 112
     assert C.sizeof(hq.hq_calib_spec) == 48 and hq.hq_calib_spec.k_lo.offset == 32
     assert C.sizeof(hq.hq_calib_result) == 24 and hq.hq_calib_result.bps.offset == 8
 
@@ -65,7 +67,7 @@ def test_invalid_params_rejected(bad):
     import lattice_entropy_coded_b200 as hq
     kw = dict(lattice=3, alpha=1.0, rice_k=2, seed=0, dither=0)
     kw.update(bad)
-    p = hq.hq_params(128, kw["lattice"], kw["alpha"], kw["rice_k"], 0, kw["dither"], 32)
+    p = hq.hq_params(128, kw["lattice"], kw["alpha"], kw["rice_k"], 0, kw["dither"], 32, None)
     with pytest.raises(hq.HQError, match="invalid"):
         hq.hq_stream_bound(32, 128, p)
 
@@ -127,6 +129,36 @@ def test_entry_points_validate_before_touching_the_device():
     assert lib.hq_debug_nearest(3, None, -1, None, None) == hq.HQ_EINVAL
     assert lib.hq_debug_nearest(3, None, 0, None, None) == hq.HQ_OK
     assert lib.hq_debug_nearest(3, None, 5, None, None) == hq.HQ_EINVAL
+
+
+def test_dense_rotation_is_a_kv_option():
+    """The weights entry points refuse a dense rotation (HQ_EUNSUPPORTED) and every entry
+    point refuses a misaligned one (HQ_EINVAL), before any device work."""
+    import lattice_entropy_coded_b200 as hq
+    lib = hq._lib
+    p = hq.make_params()
+    p.rotation = 4096
+    st = C.c_void_p(64)
+    res = hq.hq_calib_result()
+    good = hq.calib_spec(4.0)
+    assert lib.hq_quantize(C.c_void_p(256), 32, 128, 128, C.byref(p), C.c_void_p(256), 64, C.c_void_p(256), None,
+                           C.c_void_p(256), 1 << 20, None) == hq.HQ_EUNSUPPORTED
+    assert lib.hq_quantize_static(C.c_void_p(256), 32, 128, 128, C.byref(p), C.c_void_p(256), 64, C.c_void_p(256),
+                                  None, None) == hq.HQ_EUNSUPPORTED
+    assert lib.hq_dequantize(C.c_void_p(256), 64, C.c_void_p(256), 32, 128, C.byref(p), C.c_void_p(256), 0, 128,
+                             None, None) == hq.HQ_EUNSUPPORTED
+    assert lib.hq_rate(C.c_void_p(256), 32, 128, 128, C.byref(p), st, None) == hq.HQ_EUNSUPPORTED
+    assert lib.hq_calibrate(C.c_void_p(256), 32, 128, 128, C.byref(p), C.byref(good), st, None,
+                            C.byref(res)) == hq.HQ_EUNSUPPORTED
+    assert lib.hq_gemv(C.c_void_p(256), 64, C.c_void_p(256), 32, 128, C.byref(p), C.c_void_p(256),
+                       C.c_void_p(256), C.c_void_p(256), 1 << 20, None, None) == hq.HQ_EUNSUPPORTED
+    p.rotation = 4100                    # not 16-byte aligned
+    cache = hq.hq_kv_cache()
+    assert lib.hq_kv_init(C.byref(cache), 8, 128, C.byref(p), C.c_void_p(256), 64, C.c_void_p(256), 8,
+                          C.c_void_p(256), 8, C.c_void_p(256), C.c_void_p(256), None) == hq.HQ_EINVAL
+    assert lib.hq_rate_kv(C.c_void_p(256), 8, 16, 128, 2048, 0, C.byref(p), st, None) == hq.HQ_EINVAL
+    assert lib.hq_haar_rotation(1, None, None) == hq.HQ_EINVAL
+    assert lib.hq_haar_rotation(1, C.c_void_p(4100), None) == hq.HQ_EINVAL
 
 
 def test_binding_fails_loudly_without_the_library(tmp_path):
