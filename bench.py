@@ -47,6 +47,7 @@ DEFAULT_WORKLOAD = "weight_4096x4096_rate_sweep"
 L2_FLUSH_BYTES = 256 << 20
 PROFILE_ENCODE = os.path.join(ROOT, "profiles", "encode_kernel_e8_4bps.md")
 SM_COUNT, SMSP_PER_SM = 148, 4
+FP32_FMA_PEAK = SM_COUNT * 128 * 1.965e9      # fp32 fma per second at the maximum SM clock
 
 
 def rate_points():
@@ -364,16 +365,23 @@ def oracle_sample_rate(workload: str, rows_sample: int, threads: int, repeat: in
     return 2.0 * elems / dt / 1e9, dt, elems
 
 
-def oracle_workload(workload: str, threads: int, budget_s: float = 60.0):
+def kv_rotation_seed(workload_seed: int, tensor: str) -> int:
+    """Seed of the dense rotation of the K or V cache of a rotated KV workload."""
+    return 1000 * workload_seed + (0 if tensor == "K" else 1)
+
+
+def oracle_workload(workload: str, threads: int, budget_s: float = 60.0, pts=None):
     """The CPU oracle's quantize+encode and decode over a workload's tensors, generated on the
     host, on `threads` threads (chunk ranges, or KV appends, in parallel), until `budget_s` of
     wall time per operating point is spent.  -> one dict per point; where the budget ran out
-    first, the rate is over the tensors done and `extrapolated` is true."""
+    first, the rate is over the tensors done and `extrapolated` is true.  pts: the operating
+    points (default: the stored ones)."""
     from concurrent.futures import ThreadPoolExecutor
 
     import oracle as O
+    from oracle import rotation as ORot
     w = synth.WORKLOADS[workload]
-    pts = rate_points()[workload]["points"]
+    pts = rate_points()[workload]["points"] if pts is None else pts
     O.lib()
 
     def u16(t):
@@ -405,11 +413,14 @@ def oracle_workload(workload: str, threads: int, budget_s: float = 60.0):
                     H, T, _ = xu.shape
                     A = w["append"]
                     dec = np.zeros((H, T, 128), np.uint16)     # appends write disjoint token ranges
+                    rot = (ORot.haar_rotation(kv_rotation_seed(w["seed"], p["tensor"])) if w.get("rotation")
+                           else None)
 
-                    def job(t0, xu=xu, H=H, T=T, A=A, dec=dec):
+                    def job(t0, xu=xu, H=H, T=T, A=A, dec=dec, rot=rot):
                         blk = np.ascontiguousarray(xu[:, t0:t0 + A])
-                        s_, off, _ = O.kv_append(blk, t0, lat, p["alpha"], p["k"], w["seed"], 1)
-                        O.kv_read_append(s_, off, H, blk.shape[1], t0, lat, p["alpha"], p["k"], w["seed"], 1, dec, T)
+                        s_, off, _ = O.kv_append(blk, t0, lat, p["alpha"], p["k"], w["seed"], 1, rot=rot)
+                        O.kv_read_append(s_, off, H, blk.shape[1], t0, lat, p["alpha"], p["k"], w["seed"], 1, dec, T,
+                                         rot=rot)
                     jobs = list(range(0, T, A))
                     n_el = xu.size
                 else:
@@ -482,19 +493,35 @@ def run_bulk(args):
     device = torch.device("cuda", 0)
     wl = args.workload
     w = synth.WORKLOADS[wl]
-    pts = rate_points()[wl]["points"]
     out = {"workload": wl, "steps": args.steps, "warmup": args.warmup}
     peak, _ = measured_peaks()
     if w["kind"] == "kv":
         H, T, A = w["heads"], w["tokens"], w["append"]
         K, V = synth.kv(H, T, w["seed"], device=device)
         flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+        rots = {}
+        if w.get("rotation"):
+            # a dense Haar rotation per tensor, drawn on the device; alpha and k for each rate
+            # calibrated on the device over the whole tensor (untimed setup)
+            pts = []
+            for name, src in (("K", K), ("V", V)):
+                rots[name] = hq.hq_haar_rotation(kv_rotation_seed(w["seed"], name))
+                for bps in (2.0, 1.7):
+                    pr = hq.make_params("E8", 1.0, 0, w["seed"], 1, rotation=rots[name])
+                    cal = hq.hq_calibrate_kv(src, pr, hq.calib_spec(bps, tol=0.002, k_lo=0, k_hi=4),
+                                             hq.stats_tensor(device))
+                    pts.append({"tensor": name, "lattice": "E8", "bps": bps, "alpha": cal["alpha"], "k": cal["k"]})
+        else:
+            pts = rate_points()[wl]["points"]
         res = []
         for p in pts:
             src = K if p["tensor"] == "K" else V
+            rot = rots.get(p["tensor"])
             params = hq.make_params("E8", 1.0, p["k"], w["seed"], 1)
+            if rot is not None:
+                params.rotation = rot.data_ptr()
             cache = hq.KVCache(H, T, params, bits_per_scalar=p["bps"] + 4.0, max_appends=T // A + 1,
-                               max_append_tokens=A, device=device)
+                               max_append_tokens=A, device=device, rotation=rot)
             slices = [src[:, t:t + A] for t in range(0, T, A)]
             outb = torch.empty(H, T, 128, dtype=torch.bfloat16, device=device)
             app_ms, read_ms = [], []
@@ -562,6 +589,22 @@ def run_bulk(args):
                     graph_ms.append(g0.elapsed_time(g1))
             graph_words = int(cache.tail[(len(slices)) & 1].item())
             del graph
+            # one append of all T tokens at once (a prefill: H * T / 32 chunks in one launch)
+            pre = hq.KVCache(H, T, params, bits_per_scalar=p["bps"] + 4.0, max_appends=2, max_append_tokens=T,
+                             device=device, rotation=rot)
+            pre_ms = []
+            for it in range(args.warmup + args.steps):
+                flush.fill_(it)
+                hq.hq_kv_init(pre.cache, H, 128, params, pre.words, pre.offsets, pre.table, pre.tail, pre.stats)
+                p0, p1 = _events()
+                p0.record()
+                pre.append(src, p["alpha"])
+                p1.record()
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    pre_ms.append(p0.elapsed_time(p1))
+            pre_words = int(pre.tail[1].item())
+            del pre
             mse = float(((outb.double() - src.double()) ** 2).mean())
             am, rm = float(np.median(app_ms)), float(np.median(read_ms))
             alg = 2.0 * n + 4.0 * words + 8.0 * (cache.cache.chunks + 1)
@@ -572,11 +615,24 @@ def run_bulk(args):
                             graph_append_ms=float(np.median(graph_ms)),
                             graph_append_gbs=2.0 * n / (float(np.median(graph_ms)) * 1e6),
                             graph_stream_words_match=graph_words == words,
+                            prefill_append_ms=float(np.median(pre_ms)),
+                            prefill_append_gbs=2.0 * n / (float(np.median(pre_ms)) * 1e6),
+                            prefill_stream_words=pre_words,
+                            # with a dense rotation: the rotation's 128 fp32 fma per element (forward
+                            # in the append, inverse in the read) against the fp32 fma peak of
+                            # 148 SMs x 128 lanes at the 1965 MHz maximum clock
+                            **({"prefill_rotation_fma_frac": 128.0 * n / (float(np.median(pre_ms)) * 1e-3) /
+                                FP32_FMA_PEAK,
+                                "read_rotation_fma_frac": 128.0 * n / (rm * 1e-3) / FP32_FMA_PEAK} if rot is not None
+                               else {}),
                             scores_ms=float(np.median(sc_ms)), read_then_matmul_ms=float(np.median(rd_ms)),
                             scores_query_heads=H * G,
                             append_hbm_frac=alg / (am * 1e6) / peak, read_hbm_frac=alg / (rm * 1e6) / peak))
         out["points"] = res
+        if rots:
+            out["rotation"] = "Haar-uniform 128x128 per tensor (hq_haar_rotation), alpha/k calibrated on the device"
     else:
+        pts = rate_points()[wl]["points"]
         if w["kind"] == "weight":
             mats = [synth.weight(w["rows"], w["cols"], w["seed"], device=device)]
         elif w["kind"] == "weight_set":
@@ -625,7 +681,8 @@ def run_bulk(args):
             out["calibration"] = calibrate_set(hq, mats, pts, w["seed"])
     if args.oracle:
         threads = host_threads()
-        out["oracle"] = {"threads": threads, "points": oracle_workload(wl, threads)}
+        out["oracle"] = {"threads": threads,
+                         "points": oracle_workload(wl, threads, pts=pts if w["kind"] == "kv" else None)}
         if w["kind"] == "weight":
             out["oracle"]["single_thread"] = oracle_workload(wl, 1)
     print(json.dumps(out), flush=True)

@@ -21,7 +21,7 @@
 //    rebuilds and scales the lattice points;
 //  * the inverse FWHT runs in registers (two stages across the four lanes by
 //    shuffle), followed by the sign flip and 16-byte stores; or, for a KV cache
-//    with the dense rotation, x = Q^T z with Q^T in shared memory (rotate_quarter).
+//    with the dense rotation, x = Q^T z with Q^T in shared memory (rotate_round).
 // Chunks are independent (their offsets are given), so there is no look-back.
 #pragma once
 
@@ -405,13 +405,7 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
         }
         if (valid && !lane_ok) bad = true;
         if constexpr (ROT) {
-            uint32_t in[32];
-#pragma unroll
-            for (int j = 0; j < 16; j++) {
-                in[2 * j] = __float_as_uint(v[j].x);
-                in[2 * j + 1] = __float_as_uint(v[j].y);
-            }
-            rotate_quarter<false, 32>(in, v, rot_s, lane);
+            rotate_round(v, rot_s, lane);
         } else {
             fwht128_quarter(v, lane);
         }

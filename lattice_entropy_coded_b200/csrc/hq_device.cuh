@@ -160,65 +160,85 @@ __device__ __forceinline__ void fwht128_sixteenth(float2 (&v)[4], int lane) {
 // pages, "Methodology" 4).  Forward y = Q x, inverse x = Q^T z; each output is one
 // fp32 fma per term in increasing input index from +0.
 //
-// rotate_quarter applies a matrix M to a tile held in the FWHT's quarter layout:
-// lane q = lane & 3 of the tile holds inputs and outputs [32q, 32q + 32).  Input k
-// lives in lane 4 (lane / 4) + k / 32 and reaches the tile's four lanes by shuffle.
-// M sits in shared memory with row k (pitch kRotPitch floats) holding M[o][k] of
-// the 128 outputs o at rot_pos(o) = 16 m + 4 q + r for o = 32 q + 4 m + r: for one
-// (k, m) the four quarters' float4 are adjacent, one 64-byte wavefront broadcast
-// to the warp's eight tiles.  The pitch keeps rows 16-byte aligned and limits the
-// transposing writes of load_rotation to 4-way bank conflicts.
-constexpr int kRotPitch = 132;
-constexpr size_t kRotSmemBytes = (size_t)128 * kRotPitch * sizeof(float);
+// rotate_round applies a matrix M to the eight tiles a warp holds in the FWHT's
+// quarter layout (lane 4 t + q holds elements [32q, 32q + 32) of tile t), as a
+// register-blocked product: each lane computes 4 tiles x 8 outputs (tile group
+// g = lane >> 4; outputs 4j .. 4j + 3 and 64 + 4j .. 64 + 4j + 3 for j = lane & 15),
+// so that per input k a lane issues three 16-byte shared loads (4 inputs, 8 matrix
+// entries) for 32 fma.  The inputs reach that layout, and the results return to the
+// quarter layout, through a per-warp shared buffer.  Shared memory of a CTA of
+// kWarpsPerCta warps, 16-byte aligned, kRotSmemBytes: M as S[k][o] = M[o][k] (row k
+// over the 128 outputs, pitch kRotPitch), then one buffer of kRotBufFloats per warp.
+constexpr int kRotPitch = 132;          // 16-byte rows; transposing writes at most 4-way bank conflicts
+constexpr int kRotBufFloats = 8 * 132;  // inputs k-major 8 k + t + 8 (k >> 5), or results 132 t + o
+constexpr size_t kRotSmemBytes = ((size_t)128 * kRotPitch + (size_t)kWarpsPerCta * kRotBufFloats) * sizeof(float);
 
-__device__ __forceinline__ int rot_pos(int o) { return ((o & 31) >> 2) * 16 + (o >> 5) * 4 + (o & 3); }
-
-// Shared form of M from the row-major fp32 Q in global memory (coalesced reads, by
-// the whole CTA): M = Q when FORWARD, else M = Q^T.  The caller synchronises.
+// Shared form of M from the row-major fp32 Q in global memory (coalesced reads, by the
+// whole CTA): M = Q when FORWARD, else M = Q^T.  The caller synchronises.
 template <bool FORWARD>
 __device__ __forceinline__ void load_rotation(float *S, const float *Q) {
     for (int idx = threadIdx.x; idx < 128 * 128; idx += blockDim.x) {
         const int a = idx >> 7, b = idx & 127;
         const float v = __ldg(Q + idx);
         if (FORWARD)
-            S[b * kRotPitch + rot_pos(a)] = v;   // M[a][b] = Q[a][b]: output a, input b
+            S[b * kRotPitch + a] = v;   // M[a][b] = Q[a][b]: output a, input b
         else
-            S[a * kRotPitch + rot_pos(b)] = v;   // M[b][a] = Q[a][b]: output b, input a
+            S[a * kRotPitch + b] = v;   // M[b][a] = Q[a][b]: output b, input a
     }
 }
 
-// out (16 float2: out[j] = outputs 2j, 2j + 1 of the lane's quarter, as the FWHT
-// leaves them) = M in.  BF16: in[w] holds inputs 2w (low half) and 2w + 1 (high
-// half) of the quarter as bf16; otherwise in[w] is input w as fp32 bits.  The
-// packed fma rounds each half exactly like fmaf.  Whole warp.
-template <bool BF16, int NW>
-__device__ __forceinline__ void rotate_quarter(const uint32_t (&in)[NW], float2 (&out)[16], const float *S, int lane) {
-    static_assert(NW == (BF16 ? 16 : 32), "one quarter of a tile");
-    constexpr int P = BF16 ? 2 : 1;   // inputs per word
-    const int src0 = lane & ~3;
-    const float *Sq = S + 4 * (lane & 3);
+// v (16 float2 per lane: v[i] = elements 2i, 2i + 1 of the lane's quarter) <- M v for
+// each of the warp's eight tiles.  Whole warp; S as load_rotation leaves it.
+__device__ __forceinline__ void rotate_round(float2 (&v)[16], const float *S, int lane) {
+    float *buf = const_cast<float *>(S) + 128 * kRotPitch + (threadIdx.x >> 5) * kRotBufFloats;
+    const int t = lane >> 2, q = lane & 3;
+    // inputs, k-major: the 32 lanes of one store hit 32 distinct banks
 #pragma unroll
-    for (int j = 0; j < 16; j++) out[j] = make_float2(0.0f, 0.0f);
-#pragma unroll 1
-    for (int src = 0; src < 4; src++) {
-        const float *Sk = Sq + 32 * src * kRotPitch;
+    for (int i = 0; i < 16; i++) {
+        const int k = 32 * q + 2 * i;
+        buf[8 * k + t + 8 * q] = v[i].x;
+        buf[8 * (k + 1) + t + 8 * q] = v[i].y;
+    }
+    __syncwarp();
+    const int g = lane >> 4, j = lane & 15;
+    float2 acc[4][4];   // [tile 4g + tt][outputs (4j, 4j+1), (4j+2, 4j+3), (64+4j, ..), (66+4j, ..)]
 #pragma unroll
-        for (int w = 0; w < NW; w++) {
-            const uint32_t word = __shfl_sync(0xffffffffu, in[w], src0 + src);
+    for (int tt = 0; tt < 4; tt++)
 #pragma unroll
-            for (int h = 0; h < P; h++) {
-                const float xk = BF16 ? __uint_as_float(h ? (word & 0xFFFF0000u) : (word << 16)) : __uint_as_float(word);
-                const float2 x2 = make_float2(xk, xk);
-                const float *row = Sk + (P * w + h) * kRotPitch;
+        for (int c = 0; c < 4; c++) acc[tt][c] = make_float2(0.0f, 0.0f);
+#pragma unroll 8
+    for (int k = 0; k < 128; k++) {
+        const float4 z = *reinterpret_cast<const float4 *>(buf + 8 * k + 8 * (k >> 5) + 4 * g);
+        const float4 m0 = *reinterpret_cast<const float4 *>(S + k * kRotPitch + 4 * j);
+        const float4 m1 = *reinterpret_cast<const float4 *>(S + k * kRotPitch + 64 + 4 * j);
+        const float zz[4] = {z.x, z.y, z.z, z.w};
 #pragma unroll
-                for (int m = 0; m < 8; m++) {
-                    const float4 s = *reinterpret_cast<const float4 *>(row + 16 * m);
-                    out[2 * m] = f2_fma(make_float2(s.x, s.y), x2, out[2 * m]);
-                    out[2 * m + 1] = f2_fma(make_float2(s.z, s.w), x2, out[2 * m + 1]);
-                }
-            }
+        for (int tt = 0; tt < 4; tt++) {
+            const float2 x2 = make_float2(zz[tt], zz[tt]);
+            acc[tt][0] = f2_fma(make_float2(m0.x, m0.y), x2, acc[tt][0]);
+            acc[tt][1] = f2_fma(make_float2(m0.z, m0.w), x2, acc[tt][1]);
+            acc[tt][2] = f2_fma(make_float2(m1.x, m1.y), x2, acc[tt][2]);
+            acc[tt][3] = f2_fma(make_float2(m1.z, m1.w), x2, acc[tt][3]);
         }
     }
+    __syncwarp();
+    // results, tile-major
+#pragma unroll
+    for (int tt = 0; tt < 4; tt++) {
+        float *row = buf + kRotPitch * (4 * g + tt);
+        *reinterpret_cast<float4 *>(row + 4 * j) = make_float4(acc[tt][0].x, acc[tt][0].y, acc[tt][1].x, acc[tt][1].y);
+        *reinterpret_cast<float4 *>(row + 64 + 4 * j) =
+            make_float4(acc[tt][2].x, acc[tt][2].y, acc[tt][3].x, acc[tt][3].y);
+    }
+    __syncwarp();
+    const float *row = buf + kRotPitch * t + 32 * q;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const float4 r = *reinterpret_cast<const float4 *>(row + 4 * i);
+        v[2 * i] = make_float2(r.x, r.y);
+        v[2 * i + 1] = make_float2(r.z, r.w);
+    }
+    __syncwarp();
 }
 
 // ------------------------------------------------------------------ lattices

@@ -237,16 +237,15 @@ template <bool ROT>
 __device__ __forceinline__ void round_transform(const RoundInput &in, const uint4 (&raw)[4], int lane,
                                                 const uint32_t *sign_tab, const float *rot_s, float2 (&v)[16]) {
     if constexpr (ROT) {
-        uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             const uint4 r = in.valid ? raw[j] : make_uint4(0, 0, 0, 0);
-            w[4 * j] = r.x;
-            w[4 * j + 1] = r.y;
-            w[4 * j + 2] = r.z;
-            w[4 * j + 3] = r.w;
+            const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int t = 0; t < 4; t++)
+                v[4 * j + t] = make_float2(__uint_as_float(wv[t] << 16), __uint_as_float(wv[t] & 0xFFFF0000u));
         }
-        rotate_quarter<true, 16>(w, v, rot_s, lane);
+        rotate_round(v, rot_s, lane);
     } else {
         const uint32_t es = sign_tab[in.tcol * kSignWords + (lane & 3)];
 #pragma unroll

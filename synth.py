@@ -110,6 +110,8 @@ WORKLOADS = {
     "weight_1024x1024_e8_4bps": dict(kind="weight", rows=1024, cols=1024, seed=0),
     "weight_4096x4096_rate_sweep": dict(kind="weight", rows=4096, cols=4096, seed=1),
     "kv_8h_32768tok_e8_dither": dict(kind="kv", heads=8, tokens=32768, seed=2, append=256),
+    # the same cache with a dense Haar-uniform rotation per tensor instead of the sign diagonal and H_128
+    "kv_8h_32768tok_e8_dither_haar": dict(kind="kv", heads=8, tokens=32768, seed=2, append=256, rotation=True),
     "weights_8b_8layers_e8_4bps": dict(kind="weight_set", layers=8, seed=3),
     "student_t_64x8192x8192_e8": dict(kind="student_t", n=64, rows=8192, cols=8192, seed=4),
 }
