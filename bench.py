@@ -66,7 +66,7 @@ def measured_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("hq_encode.cu", "hq_device.cuh", "hq_internal.h"):
+    for f in ("hq_encode.cuh", "hq_encode.cu", "hq_device.cuh", "hq_internal.h"):
         with open(os.path.join(ROOT, "lattice_entropy_coded_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
