@@ -20,3 +20,4 @@ def test_readme_python_example_runs():
     assert hq.read_stats(env["codec"].stats)["status"] == 0
     assert abs(env["cal"]["bps"] - 4.0) <= 0.002
     assert env["s"].shape == (32, 256) and bool(torch.isfinite(env["s"]).all())
+    assert hq.read_stats(env["rcache"].stats)["status"] == 0 and env["rcache"].tokens == 256
