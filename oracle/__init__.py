@@ -106,19 +106,21 @@ def _bind(L):
         "hqref_unzigzag": (C.c_int32, [_u32]),
         "hqref_rice_concat": (_u64, [_p, _i64, _i32, _p, _u64]),
         "hqref_rice_concat_decode": (_i32, [_p, _u64, _i64, _i32, _p]),
-        "hqref_encode_chunk": (_u64, [_i32, _i32, _p, _i32, _p, _u64, _p]),
-        "hqref_decode_chunk": (_i32, [_i32, _i32, _p, _u64, _i32, _p]),
+        "hqref_encode_chunk": (_u64, [_i32, _i32, _p, _i32, _p, _u64, _p, _i32]),
+        "hqref_decode_chunk": (_i32, [_i32, _i32, _p, _u64, _i32, _p, _i32]),
+        "hqref_symbol_k": (_i32, [_i32, _i32, _i32, _i32]),
+        "hqref_rice_concat_k": (_u64, [_p, _i64, _p, _p, _u64]),
         "hqref_quantize_tile": (None, [_p, _i32, _f32, _u64, _u64, _i32, _u64, _p]),
         "hqref_dequantize_tile": (None, [_p, _i32, _f32, _u64, _u64, _i32, _u64, _p]),
         "hqref_n_chunks": (_i64, [_i64, _i64]),
         "hqref_quantize": (_i64, [_p, _i64, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _i64, _i64, _p, _u64,
-                                  _p, _p]),
+                                  _p, _p, _i32]),
         "hqref_dequantize": (_i32, [_p, _p, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _i64, _i64, _i32, _p,
-                                    _i64]),
+                                    _i64, _i32]),
         "hqref_kv_append": (_i64, [_p, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _p, _u64,
-                                   _u64, _p, _p, _p]),
+                                   _u64, _p, _p, _p, _i32]),
         "hqref_kv_read_append": (_i32, [_p, _p, _i64, _i64, _i64, _i32, _f32, _i32, _u64, _i32, _i32, _p,
-                                        _i64, _i64, _i64, _p]),
+                                        _i64, _i64, _i64, _p, _i32]),
         "hqref_rotate_fwd": (None, [_p, _p, _p]),
         "hqref_rotate_inv": (None, [_p, _p, _p]),
         "hqref_scale_inv_rot": (_f32, [_f32]),
@@ -259,21 +261,35 @@ def rice_concat_decode(words, nbits: int, n: int, k: int) -> np.ndarray:
     return z
 
 
-def encode_chunk(lat: int, k: int, codes):
+def symbol_k(lat: int, k: int, dk_last: int, i: int) -> int:
+    return int(lib().hqref_symbol_k(lat, k, dk_last, i))
+
+
+def rice_concat_k(z, ks):
+    zz = np.ascontiguousarray(z, dtype=np.uint32)
+    kk = np.ascontiguousarray(ks, dtype=np.int32)
+    assert kk.size == zz.size
+    nbits = int(lib().hqref_rice_concat_k(_ptr(zz), zz.size, _ptr(kk), None, 0))
+    out = np.zeros((nbits + 31) // 32, dtype=np.uint32)
+    lib().hqref_rice_concat_k(_ptr(zz), zz.size, _ptr(kk), _ptr(out), out.size)
+    return out, nbits
+
+
+def encode_chunk(lat: int, k: int, codes, dk_last: int = 0):
     q = np.ascontiguousarray(codes, dtype=np.int32)
     assert q.size % 128 == 0
     nt = q.size // 128
     pb = np.zeros(1, dtype=np.uint64)
-    n = int(lib().hqref_encode_chunk(lat, k, _ptr(q), nt, None, 0, _ptr(pb)))
+    n = int(lib().hqref_encode_chunk(lat, k, _ptr(q), nt, None, 0, _ptr(pb), dk_last))
     out = np.zeros(n, dtype=np.uint32)
-    lib().hqref_encode_chunk(lat, k, _ptr(q), nt, _ptr(out), n, _ptr(pb))
+    lib().hqref_encode_chunk(lat, k, _ptr(q), nt, _ptr(out), n, _ptr(pb), dk_last)
     return out, int(pb[0])
 
 
-def decode_chunk(lat: int, k: int, words, ntiles: int) -> np.ndarray:
+def decode_chunk(lat: int, k: int, words, ntiles: int, dk_last: int = 0) -> np.ndarray:
     w = np.ascontiguousarray(words, dtype=np.uint32)
     q = np.zeros(ntiles * 128, dtype=np.int32)
-    if lib().hqref_decode_chunk(lat, k, _ptr(w), w.size, ntiles, _ptr(q)) != 0:
+    if lib().hqref_decode_chunk(lat, k, _ptr(w), w.size, ntiles, _ptr(q), dk_last) != 0:
         raise ValueError("corrupt chunk")
     return q
 
@@ -338,7 +354,7 @@ def n_chunks(rows: int, cols: int) -> int:
 
 
 def quantize(x, lat: int, alpha: float, k: int, seed: int, dither: int = 0, chunk_lo: int = 0,
-             chunk_hi: int | None = None):
+             chunk_hi: int | None = None, dk_last: int = 0):
     """Weights path: bf16 [R, C] -> (stream words, offsets (n+1, relative), payload bits)."""
     xu = _as_u16(x)
     R, Cc = xu.shape
@@ -348,18 +364,18 @@ def quantize(x, lat: int, alpha: float, k: int, seed: int, dither: int = 0, chun
     off = np.zeros(chunk_hi - chunk_lo + 1, dtype=np.uint64)
     pb = np.zeros(1, dtype=np.uint64)
     total = int(L.hqref_quantize(_ptr(xu), R, Cc, Cc, lat, alpha, k, seed, dither, chunk_lo, chunk_hi, None, 0,
-                                 _ptr(off), _ptr(pb)))
+                                 _ptr(off), _ptr(pb), dk_last))
     total = abs(total)
     stream = np.zeros(max(total, 1), dtype=np.uint32)
     rc = int(L.hqref_quantize(_ptr(xu), R, Cc, Cc, lat, alpha, k, seed, dither, chunk_lo, chunk_hi,
-                              _ptr(stream), stream.size, _ptr(off), _ptr(pb)))
+                              _ptr(stream), stream.size, _ptr(off), _ptr(pb), dk_last))
     assert rc == total
     return stream[:total], off, int(pb[0])
 
 
 def dequantize(stream, offsets, rows: int, cols: int, lat: int, alpha: float, k: int, seed: int, dither: int = 0,
                out_fp32: bool = False, chunk_lo: int = 0, chunk_hi: int | None = None,
-               out: np.ndarray | None = None) -> np.ndarray:
+               out: np.ndarray | None = None, dk_last: int = 0) -> np.ndarray:
     """Weights path inverse: float32 [R, C] (fp32 mode) or uint16 bf16 bits [R, C].
     offsets[0] belongs to chunk chunk_lo; only that range's tiles of `out` are written."""
     if chunk_hi is None:
@@ -371,7 +387,7 @@ def dequantize(stream, offsets, rows: int, cols: int, lat: int, alpha: float, k:
     assert out.shape == (rows, cols) and out.flags["C_CONTIGUOUS"]
     assert out.dtype == (np.float32 if out_fp32 else np.uint16)
     rc = lib().hqref_dequantize(_ptr(s), _ptr(o), rows, cols, lat, alpha, k, seed, dither, chunk_lo, chunk_hi,
-                                int(out_fp32), _ptr(out), cols)
+                                int(out_fp32), _ptr(out), cols, dk_last)
     if rc != 0:
         raise ValueError("corrupt stream")
     return out
@@ -387,7 +403,7 @@ def _rot_ptr(rot):
 
 
 def kv_append(kv, tok0: int, lat: int, alpha: float, k: int, seed: int, dither: int = 1, base_word: int = 0,
-              rot=None):
+              rot=None, dk_last: int = 0):
     """One KV append: bf16 [H, T, 128] -> (stream words, absolute offsets (n+1), payload bits).
     rot: a 128 x 128 orthogonal fp32 matrix in place of H_128 D / sqrt(128), or None."""
     r_keep, rp = _rot_ptr(rot)
@@ -399,24 +415,25 @@ def kv_append(kv, tok0: int, lat: int, alpha: float, k: int, seed: int, dither: 
     off = np.zeros(nch + 1, dtype=np.uint64)
     pb = np.zeros(1, dtype=np.uint64)
     end = abs(int(L.hqref_kv_append(_ptr(x), H, T, 128, T * 128, tok0, lat, alpha, k, seed, dither, None,
-                                    base_word, 0, _ptr(off), _ptr(pb), rp)))
+                                    base_word, 0, _ptr(off), _ptr(pb), rp, dk_last)))
     total = end - base_word
     stream = np.zeros(max(end, 1), dtype=np.uint32)
     L.hqref_kv_append(_ptr(x), H, T, 128, T * 128, tok0, lat, alpha, k, seed, dither, _ptr(stream), base_word,
-                      stream.size, _ptr(off), _ptr(pb), rp)
+                      stream.size, _ptr(off), _ptr(pb), rp, dk_last)
     del r_keep
     return stream[base_word:end].copy(), off, int(pb[0])
 
 
 def kv_read_append(stream_abs, offsets_abs, H: int, T: int, tok0: int, lat: int, alpha: float, k: int, seed: int,
-                   dither: int, out: np.ndarray, length: int, rot=None):
+                   dither: int, out: np.ndarray, length: int, rot=None, dk_last: int = 0):
     """Decode one append into out [H, len, 128] (float32 or uint16 bf16 bits)."""
     r_keep, rp = _rot_ptr(rot)
     s = np.ascontiguousarray(stream_abs, dtype=np.uint32)
     o = np.ascontiguousarray(offsets_abs, dtype=np.uint64)
     assert out.flags["C_CONTIGUOUS"] and out.shape[2] == 128
     rc = lib().hqref_kv_read_append(_ptr(s), _ptr(o), H, T, tok0, lat, alpha, k, seed, dither,
-                                    int(out.dtype == np.float32), _ptr(out), 128, out.shape[1] * 128, length, rp)
+                                    int(out.dtype == np.float32), _ptr(out), 128, out.shape[1] * 128, length, rp,
+                                    dk_last)
     del r_keep
     if rc != 0:
         raise ValueError("corrupt stream")

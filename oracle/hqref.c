@@ -10,7 +10,7 @@
  * 2606.23406, sections "Methodology": 1 per-tile RHT, 2 lattice quantization,
  * 3 bit-stripping and Rice coding, 4 KV bias correction) and the arXiv abstract
  * (items (i)-(iv)).  The pages give no constants, no bitstream and no code; the
- * readings taken where they are silent are marked [R1]..[R18] and listed in the
+ * readings taken where they are silent are marked [R1]..[R19] and listed in the
  * design notes of the repository.
  *
  * Build: gcc -std=c99 -O2 -ffp-contract=off -fno-fast-math -shared -fPIC.
@@ -390,14 +390,47 @@ int hqref_rice_concat_decode(const uint32_t *in, uint64_t nbits, int64_t n, int 
     return 0;
 }
 
+/* Rice parameter of the symbol at position i of its lattice block [R19]: the
+ * last symbol of an A2, D4 or E8 block (b', q3', m7': the one whose implied
+ * bit R9 strips) takes max(k - dk_last, 0); every other symbol takes k.  With
+ * dk_last = 0 every symbol takes k. */
+int hqref_symbol_k(int lat, int k, int dk_last, int i)
+{
+    int n = hqref_lattice_dim(lat);
+    if (n > 1 && i == n - 1) return (k > dk_last) ? k - dk_last : 0;
+    return k;
+}
+
+/* Concatenated Rice codes with a parameter per symbol (ks[i]); the same as
+ * hqref_rice_concat when every ks[i] is k. */
+uint64_t hqref_rice_concat_k(const uint32_t *z, int64_t n, const int32_t *ks, uint32_t *out, uint64_t cap_words)
+{
+    uint64_t pos = 0;
+    for (int64_t i = 0; i < n; i++) {
+        int k = ks[i];
+        uint64_t q = z[i] >> k;
+        uint64_t need = pos + q + 1 + (uint64_t)k;
+        if (out && need <= 32ull * cap_words) {
+            pos += q;
+            put_bit(out, pos++, 1);
+            for (int b = 0; b < k; b++) put_bit(out, pos++, (z[i] >> b) & 1u);
+        } else {
+            pos = need;
+        }
+    }
+    return pos;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Chunk planes [R12].  A chunk holds the symbols of ntiles tiles in order
  * (symbol index = tile * 128 + coordinate).  Layout, each plane starting on a
- * word boundary: [coset plane: 1 bit per E8 block] [remainder plane: k bits
- * per symbol at bit i*k] [unary plane: per symbol, floor(z/2^k) zeros then a
- * one].  Returns the chunk's word count; writes only if it fits in cap. */
+ * word boundary: [coset plane: 1 bit per E8 block] [remainder plane: the k_i
+ * low bits of each symbol i, in symbol order, at the running sum of the k_i
+ * (i * k when every k_i = k)] [unary plane: per symbol, floor(z/2^k_i) zeros
+ * then a one], k_i = hqref_symbol_k(lat, k, dk_last, i mod n).  Returns the
+ * chunk's word count; writes only if it fits in cap. */
 uint64_t hqref_encode_chunk(int lat, int k, const int32_t *q, int ntiles, uint32_t *out, uint64_t cap_words,
-                            uint64_t *payload_bits)
+                            uint64_t *payload_bits, int dk_last)
 {
     int n = hqref_lattice_dim(lat);
     int64_t nsym = (int64_t)ntiles * 128;
@@ -410,24 +443,30 @@ uint64_t hqref_encode_chunk(int lat, int k, const int32_t *q, int ntiles, uint32
         for (int i = 0; i < n; i++) z[b * n + i] = hqref_zigzag(m[i]);
     }
     uint64_t wc = (lat == HQREF_E8) ? (uint64_t)(nblk + 31) / 32 : 0;
-    uint64_t wr = ((uint64_t)nsym * (uint64_t)k + 31) / 32;
-    uint64_t ubits = 0;
-    for (int64_t i = 0; i < nsym; i++) ubits += (uint64_t)(z[i] >> k) + 1;
+    uint64_t rbits = 0, ubits = 0;
+    for (int64_t i = 0; i < nsym; i++) {
+        int ki = hqref_symbol_k(lat, k, dk_last, (int)(i % n));
+        rbits += (uint64_t)ki;
+        ubits += (uint64_t)(z[i] >> ki) + 1;
+    }
+    uint64_t wr = (rbits + 31) / 32;
     uint64_t wu = (ubits + 31) / 32;
     uint64_t total = wc + wr + wu;
-    if (payload_bits)
-        *payload_bits = ubits + (uint64_t)nsym * (uint64_t)k + ((lat == HQREF_E8) ? (uint64_t)nblk : 0);
+    if (payload_bits) *payload_bits = ubits + rbits + ((lat == HQREF_E8) ? (uint64_t)nblk : 0);
     if (out && total <= cap_words) {
         memset(out, 0, sizeof(uint32_t) * (size_t)total);
         if (lat == HQREF_E8)
             for (int64_t b = 0; b < nblk; b++) put_bit(out, (uint64_t)b, cb[b]);
         uint32_t *rem = out + wc;
-        for (int64_t i = 0; i < nsym; i++)
-            for (int b = 0; b < k; b++) put_bit(rem, (uint64_t)i * (uint64_t)k + (uint64_t)b, (z[i] >> b) & 1u);
+        uint64_t rpos = 0;
+        for (int64_t i = 0; i < nsym; i++) {
+            int ki = hqref_symbol_k(lat, k, dk_last, (int)(i % n));
+            for (int b = 0; b < ki; b++) put_bit(rem, rpos++, (z[i] >> b) & 1u);
+        }
         uint32_t *un = out + wc + wr;
         uint64_t pos = 0;
         for (int64_t i = 0; i < nsym; i++) {
-            pos += z[i] >> k;
+            pos += z[i] >> hqref_symbol_k(lat, k, dk_last, (int)(i % n));
             put_bit(un, pos++, 1);
         }
     }
@@ -438,28 +477,31 @@ uint64_t hqref_encode_chunk(int lat, int k, const int32_t *q, int ntiles, uint32
 
 /* Inverse of hqref_encode_chunk.  Returns 0, or -1 if the words do not hold
  * exactly nsym unary terminators inside the chunk. */
-int hqref_decode_chunk(int lat, int k, const uint32_t *w, uint64_t nwords, int ntiles, int32_t *q)
+int hqref_decode_chunk(int lat, int k, const uint32_t *w, uint64_t nwords, int ntiles, int32_t *q, int dk_last)
 {
     int n = hqref_lattice_dim(lat);
     int64_t nsym = (int64_t)ntiles * 128;
     int64_t nblk = nsym / n;
     uint64_t wc = (lat == HQREF_E8) ? (uint64_t)(nblk + 31) / 32 : 0;
-    uint64_t wr = ((uint64_t)nsym * (uint64_t)k + 31) / 32;
+    uint64_t rbits = 0;
+    for (int i = 0; i < n; i++) rbits += (uint64_t)hqref_symbol_k(lat, k, dk_last, i);
+    rbits *= (uint64_t)nblk;
+    uint64_t wr = (rbits + 31) / 32;
     if (nwords < wc + wr) return -1;
     const uint32_t *rem = w + wc, *un = w + wc + wr;
     uint64_t ubits = 32 * (nwords - wc - wr);
-    uint64_t pos = 0;
+    uint64_t pos = 0, rpos = 0;
     for (int64_t b = 0; b < nblk; b++) {
         int32_t m[8];
         for (int i = 0; i < n; i++) {
-            int64_t s = b * n + i;
+            int ki = hqref_symbol_k(lat, k, dk_last, i);
             uint64_t qq = 0;
             while (pos < ubits && !get_bit(un, pos)) { qq++; pos++; }
             if (pos >= ubits) return -1;
             pos++;
             uint32_t r = 0;
-            for (int t = 0; t < k; t++) r |= get_bit(rem, (uint64_t)s * (uint64_t)k + (uint64_t)t) << t;
-            m[i] = hqref_unzigzag((uint32_t)(qq << k) | r);
+            for (int t = 0; t < ki; t++) r |= get_bit(rem, rpos++) << t;
+            m[i] = hqref_unzigzag((uint32_t)(qq << ki) | r);
         }
         uint32_t c = (lat == HQREF_E8) ? get_bit(w, (uint64_t)b) : 0;
         hqref_reinsert(lat, m, c, q + b * n);
@@ -650,7 +692,7 @@ static int tile_of(const tiles_t *t, int64_t c, int i, const uint16_t **p, uint6
 
 static int64_t encode_all(const tiles_t *t, int lat, float alpha, int k, uint64_t seed, int dither,
                           int64_t chunk_lo, int64_t chunk_hi, uint32_t *stream, uint64_t base_word,
-                          uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits)
+                          uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits, int dk_last)
 {
     int32_t *q = (int32_t *)malloc(sizeof(int32_t) * 32 * 128);
     uint64_t pos = base_word, pay = 0;
@@ -670,7 +712,7 @@ static int64_t encode_all(const tiles_t *t, int lat, float alpha, int k, uint64_
         }
         uint64_t pb = 0;
         uint64_t room = (pos < cap_words) ? cap_words - pos : 0;
-        uint64_t nw = hqref_encode_chunk(lat, k, q, nt, stream ? stream + pos : NULL, stream ? room : 0, &pb);
+        uint64_t nw = hqref_encode_chunk(lat, k, q, nt, stream ? stream + pos : NULL, stream ? room : 0, &pb, dk_last);
         if (nw > room) over = 1;
         if (offsets) offsets[c - chunk_lo] = pos;
         pos += nw;
@@ -684,7 +726,7 @@ static int64_t encode_all(const tiles_t *t, int lat, float alpha, int k, uint64_
 
 static int decode_all(const tiles_t *t, int lat, float alpha, int k, uint64_t seed, int dither, int64_t chunk_lo,
                       int64_t chunk_hi, const uint32_t *stream, const uint64_t *offsets, int out_fp32, void *out,
-                      int64_t out_ld, int64_t out_ld_head, int64_t len)
+                      int64_t out_ld, int64_t out_ld_head, int64_t len, int dk_last)
 {
     int32_t *q = (int32_t *)malloc(sizeof(int32_t) * 32 * 128);
     int bad = 0;
@@ -697,7 +739,7 @@ static int decode_all(const tiles_t *t, int lat, float alpha, int k, uint64_t se
             nt++;
         }
         uint64_t w0 = offsets[c - chunk_lo], w1 = offsets[c - chunk_lo + 1];
-        if (w1 < w0 || hqref_decode_chunk(lat, k, stream + w0, w1 - w0, nt, q) != 0) {
+        if (w1 < w0 || hqref_decode_chunk(lat, k, stream + w0, w1 - w0, nt, q, dk_last) != 0) {
             bad = 1;
             continue;
         }
@@ -740,7 +782,7 @@ int64_t hqref_n_chunks(int64_t rows, int64_t cols)
 
 int64_t hqref_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int lat, float alpha, int k,
                        uint64_t seed, int dither, int64_t chunk_lo, int64_t chunk_hi, uint32_t *stream,
-                       uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits)
+                       uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits, int dk_last)
 {
     tiles_t t = {0};
     t.x = x;
@@ -748,18 +790,18 @@ int64_t hqref_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld
     t.cols = cols;
     t.ld = ld;
     return encode_all(&t, lat, alpha, k, seed, dither, chunk_lo, chunk_hi, stream, 0, cap_words, offsets,
-                      payload_bits);
+                      payload_bits, dk_last);
 }
 
 int hqref_dequantize(const uint32_t *stream, const uint64_t *offsets, int64_t rows, int64_t cols, int lat,
                      float alpha, int k, uint64_t seed, int dither, int64_t chunk_lo, int64_t chunk_hi,
-                     int out_fp32, void *out, int64_t ld)
+                     int out_fp32, void *out, int64_t ld, int dk_last)
 {
     tiles_t t = {0};
     t.rows = rows;
     t.cols = cols;
     return decode_all(&t, lat, alpha, k, seed, dither, chunk_lo, chunk_hi, stream, offsets, out_fp32, out, ld, 0,
-                      0);
+                      0, dk_last);
 }
 
 /* KV append [R15]: the chunks of one append are written from base_word on;
@@ -768,7 +810,7 @@ int hqref_dequantize(const uint32_t *stream, const uint64_t *offsets, int64_t ro
 int64_t hqref_kv_append(const uint16_t *kv, int64_t H, int64_t T, int64_t ld_tok, int64_t ld_head, int64_t tok0,
                         int lat, float alpha, int k, uint64_t seed, int dither, uint32_t *stream,
                         uint64_t base_word, uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits,
-                        const float *rot)
+                        const float *rot, int dk_last)
 {
     tiles_t t = {0};
     t.kv = 1;
@@ -780,14 +822,14 @@ int64_t hqref_kv_append(const uint16_t *kv, int64_t H, int64_t T, int64_t ld_tok
     t.tok0 = tok0;
     t.rot = rot;
     return encode_all(&t, lat, alpha, k, seed, dither, 0, n_chunks_of(&t), stream, base_word, cap_words, offsets,
-                      payload_bits);
+                      payload_bits, dk_last);
 }
 
 /* Decode the chunks of one append into out[h * out_ld_head + tok * out_ld_tok + dim],
  * tokens at or beyond len skipped. */
 int hqref_kv_read_append(const uint32_t *stream, const uint64_t *offsets, int64_t H, int64_t T, int64_t tok0,
                          int lat, float alpha, int k, uint64_t seed, int dither, int out_fp32, void *out,
-                         int64_t out_ld_tok, int64_t out_ld_head, int64_t len, const float *rot)
+                         int64_t out_ld_tok, int64_t out_ld_head, int64_t len, const float *rot, int dk_last)
 {
     tiles_t t = {0};
     t.kv = 1;
@@ -796,5 +838,5 @@ int hqref_kv_read_append(const uint32_t *stream, const uint64_t *offsets, int64_
     t.tok0 = tok0;
     t.rot = rot;
     return decode_all(&t, lat, alpha, k, seed, dither, 0, n_chunks_of(&t), stream, offsets, out_fp32, out,
-                      out_ld_tok, out_ld_head, len);
+                      out_ld_tok, out_ld_head, len, dk_last);
 }

@@ -39,9 +39,11 @@ int32_t hqref_unzigzag(uint32_t z);
 
 uint64_t hqref_rice_concat(const uint32_t *z, int64_t n, int k, uint32_t *out, uint64_t cap_words);
 int hqref_rice_concat_decode(const uint32_t *in, uint64_t nbits, int64_t n, int k, uint32_t *z);
+int hqref_symbol_k(int lat, int k, int dk_last, int i);
+uint64_t hqref_rice_concat_k(const uint32_t *z, int64_t n, const int32_t *ks, uint32_t *out, uint64_t cap_words);
 uint64_t hqref_encode_chunk(int lat, int k, const int32_t *q, int ntiles, uint32_t *out, uint64_t cap_words,
-                            uint64_t *payload_bits);
-int hqref_decode_chunk(int lat, int k, const uint32_t *w, uint64_t nwords, int ntiles, int32_t *q);
+                            uint64_t *payload_bits, int dk_last);
+int hqref_decode_chunk(int lat, int k, const uint32_t *w, uint64_t nwords, int ntiles, int32_t *q, int dk_last);
 
 void hqref_quantize_tile(const uint16_t *x, int lat, float alpha, uint64_t seed, uint64_t sign_col0, int dither,
                          uint64_t e0, int32_t *q);
@@ -60,16 +62,16 @@ double hqref_rot_gaussian(uint64_t seed, uint64_t e);
 int64_t hqref_n_chunks(int64_t rows, int64_t cols);
 int64_t hqref_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int lat, float alpha, int k,
                        uint64_t seed, int dither, int64_t chunk_lo, int64_t chunk_hi, uint32_t *stream,
-                       uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits);
+                       uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits, int dk_last);
 int hqref_dequantize(const uint32_t *stream, const uint64_t *offsets, int64_t rows, int64_t cols, int lat,
                      float alpha, int k, uint64_t seed, int dither, int64_t chunk_lo, int64_t chunk_hi,
-                     int out_fp32, void *out, int64_t ld);
+                     int out_fp32, void *out, int64_t ld, int dk_last);
 int64_t hqref_kv_append(const uint16_t *kv, int64_t H, int64_t T, int64_t ld_tok, int64_t ld_head, int64_t tok0,
                         int lat, float alpha, int k, uint64_t seed, int dither, uint32_t *stream,
                         uint64_t base_word, uint64_t cap_words, uint64_t *offsets, uint64_t *payload_bits,
-                        const float *rot);
+                        const float *rot, int dk_last);
 int hqref_kv_read_append(const uint32_t *stream, const uint64_t *offsets, int64_t H, int64_t T, int64_t tok0,
                          int lat, float alpha, int k, uint64_t seed, int dither, int out_fp32, void *out,
-                         int64_t out_ld_tok, int64_t out_ld_head, int64_t len, const float *rot);
+                         int64_t out_ld_tok, int64_t out_ld_head, int64_t len, const float *rot, int dk_last);
 
 #endif

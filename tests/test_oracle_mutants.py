@@ -8,6 +8,7 @@ import pytest
 
 import oracle as O
 import test_oracle_pins as P
+import test_oracle_rice_k as PK
 import test_oracle_rotation as PR
 
 # (what the mistake is, text to find, replacement, pins expected to catch it)
@@ -41,8 +42,9 @@ MUTANTS = [
      [lambda: P.test_subtractive_dither_error_is_uniform_on_voronoi_cell(O.E8, "E8", "2E8")]),
     ("generator increment starts at i", "(i + 1u) * 0x9E3779B97F4A7C15ull", "i * 0x9E3779B97F4A7C15ull",
      [P.test_splitmix64_published_vectors]),
-    ("Rice unary drops a bit of the quotient", "pos += z[i] >> k;\n            put_bit(un, pos++, 1);",
-     "pos += z[i] >> (k + 1);\n            put_bit(un, pos++, 1);",
+    ("Rice unary drops a bit of the quotient",
+     "pos += z[i] >> hqref_symbol_k(lat, k, dk_last, (int)(i % n));\n            put_bit(un, pos++, 1);",
+     "pos += z[i] >> (hqref_symbol_k(lat, k, dk_last, (int)(i % n)) + 1);\n            put_bit(un, pos++, 1);",
      [lambda: P.test_chunk_planes_roundtrip_and_same_bits_as_concatenated(O.E8, 2)]),
     ("forward rotation uses Q transposed", "acc = fmaf(Q[i * 128 + j], x[j], acc);",
      "acc = fmaf(Q[j * 128 + i], x[j], acc);", [PR.test_rotation_of_basis_vectors_is_exact]),
@@ -55,6 +57,15 @@ MUTANTS = [
      [PR.test_rotated_dithered_reconstruction_is_unbiased_regression]),
     ("Box-Muller radius loses its factor 2", "return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);",
      "return sqrt(-log(u1)) * cos(two_pi * u2);", [PR.test_gaussian_draws_are_standard_normal]),
+    ("last symbol keeps the full Rice parameter", "if (n > 1 && i == n - 1) return (k > dk_last) ? k - dk_last : 0;",
+     "if (n > 1 && i == n - 1) return k;",
+     [PK.test_symbol_k_follows_the_definition, lambda: PK.test_two_k_planes_hold_the_textbook_codewords(O.E8, 2, 1)]),
+    ("first symbol of the block takes the reduced parameter", "if (n > 1 && i == n - 1) return",
+     "if (n > 1 && i == 0) return", [lambda: PK.test_two_k_planes_hold_the_textbook_codewords(O.D4, 2, 1)]),
+    ("remainders at i * k_i instead of the running sum",
+     "for (int b = 0; b < ki; b++) put_bit(rem, rpos++, (z[i] >> b) & 1u);",
+     "for (int b = 0; b < ki; b++) put_bit(rem, (uint64_t)i * (uint64_t)ki + (uint64_t)b, (z[i] >> b) & 1u);",
+     [lambda: PK.test_two_k_planes_hold_the_textbook_codewords(O.A2, 2, 1)]),
     ("Gaussian radius from one bit too few", "double u1 = ((double)(h >> 32) + 0.5) * 0x1p-32;",
      "double u1 = ((double)(h >> 33) + 0.5) * 0x1p-32;", [PR.test_gaussian_draws_are_standard_normal]),
 ]
