@@ -37,8 +37,9 @@
  * Bitstream (all planes LSB-first in little-endian uint32 words, each plane
  * starting on a word boundary), per chunk of n tiles (N = 128 n symbols):
  *   [coset plane, E8 only: one bit per 8-element block, ceil(16 n / 32) words]
- *   [remainder plane: k bits per symbol at bit i*k, 4 k n words]
- *   [unary plane: per symbol floor(z / 2^k) zeros then a one, zero padded]
+ *   [remainder plane: k bits per symbol at bit i*k, 4 k n words; with
+ *    rice_dk_last > 0, symbol i's k_i bits at the running sum of the k_i]
+ *   [unary plane: per symbol floor(z / 2^k_i) zeros then a one, zero padded]
  * offsets[c] is the index of chunk c's first word; offsets[n_chunks] is the
  * total.  The codewords are exactly the concatenated Rice codewords of the
  * symbols; the plane split lets a decoder work on all tiles of a chunk at once.
@@ -104,8 +105,14 @@ typedef struct hq_params {
                             *   x_hat_j = sum_i Q[i][j] ((point - d)_i * fp32(1 / alpha)),
                             * each sum one fp32 fma per term in increasing index from +0.  Must
                             * stay valid and unchanged while the cache is in use.  The weights
-                            * entry points return HQ_EUNSUPPORTED when it is set.  40 bytes. */
-} hq_params;
+                            * entry points return HQ_EUNSUPPORTED when it is set. */
+    int32_t rice_dk_last;  /* 0..15.  Bit-stripping halves the last symbol of each A2, D4 or E8 block
+                            * (b', q3', m7'), so its best Rice parameter is smaller: it is coded with
+                            * max(rice_k - rice_dk_last, 0), every other symbol with rice_k (Z: all
+                            * with rice_k).  0: one parameter for all symbols.  The remainder plane
+                            * then holds each symbol's k_i low bits at the running sum of the k_i. */
+    int32_t reserved;      /* 0 */
+} hq_params;               /* 48 bytes */
 
 /* Device-resident statistics written by the kernels (zeroed by each call
  * that takes it).  32 bytes, 8-byte aligned. */

@@ -28,7 +28,8 @@ HQ_ST_CAPACITY, HQ_ST_CORRUPT, HQ_ST_TIMEOUT, HQ_ST_RANGE = 1, 2, 4, 8
 
 class hq_params(C.Structure):
     _fields_ = [("tile", C.c_int32), ("lattice", C.c_int32), ("alpha", C.c_float), ("rice_k", C.c_int32),
-                ("seed", C.c_uint64), ("dither", C.c_int32), ("chunk_tiles", C.c_int32), ("rotation", C.c_void_p)]
+                ("seed", C.c_uint64), ("dither", C.c_int32), ("chunk_tiles", C.c_int32), ("rotation", C.c_void_p),
+                ("rice_dk_last", C.c_int32), ("reserved", C.c_int32)]
 
 
 class hq_stats(C.Structure):
@@ -59,8 +60,8 @@ class hq_calib_result(C.Structure):
 
 
 assert C.sizeof(hq_calib_spec) == 48 and C.sizeof(hq_calib_result) == 24
-assert C.sizeof(hq_params) == 40 and C.sizeof(hq_stats) == 32 and C.sizeof(hq_kv_append_row) == 32
-assert C.sizeof(hq_kv_cache) == 136
+assert C.sizeof(hq_params) == 48 and C.sizeof(hq_stats) == 32 and C.sizeof(hq_kv_append_row) == 32
+assert C.sizeof(hq_kv_cache) == 144
 
 # C entry points: name -> (restype, argtypes)
 EXPORTS = {
@@ -141,16 +142,19 @@ def _stream(s) -> int | None:
     return int(s)
 
 
-def make_params(lattice="E8", alpha=1.0, rice_k=2, seed=0, dither=0, rotation: torch.Tensor | None = None) -> hq_params:
+def make_params(lattice="E8", alpha=1.0, rice_k=2, seed=0, dither=0, rotation: torch.Tensor | None = None,
+                dk_last: int = 0) -> hq_params:
     """rotation: a KV cache's dense rotation (fp32 [128, 128] on the device, e.g. from
     hq_haar_rotation), or None for the sign diagonal and H_128.  The params hold only its
-    address: the caller keeps the tensor alive and unchanged."""
+    address: the caller keeps the tensor alive and unchanged.  dk_last: the last symbol of
+    each A2 / D4 / E8 block is Rice coded with max(rice_k - dk_last, 0) (0: one parameter)."""
     lat = LATTICES[lattice] if isinstance(lattice, str) else int(lattice)
     rot = None
     if rotation is not None:
         assert rotation.dtype == torch.float32 and rotation.is_contiguous() and tuple(rotation.shape) == (128, 128)
         rot = rotation.data_ptr()
-    return hq_params(128, lat, float(alpha), int(rice_k), int(seed) & (2**64 - 1), int(dither), 32, rot)
+    return hq_params(128, lat, float(alpha), int(rice_k), int(seed) & (2**64 - 1), int(dither), 32, rot,
+                     int(dk_last), 0)
 
 
 # ------------------------------------------------------------------ C entry points

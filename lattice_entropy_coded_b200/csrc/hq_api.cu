@@ -29,7 +29,14 @@ int check_params(const hq_params *p) {
     if (p->dither != 0 && p->dither != 1) return HQ_EINVAL;
     if (p->tile != kTile || p->chunk_tiles != kChunkTiles) return HQ_EUNSUPPORTED;
     if (p->rotation && !aligned(p->rotation, 16)) return HQ_EINVAL;
+    if (p->rice_dk_last < 0 || p->rice_dk_last > 15) return HQ_EINVAL;
     return HQ_OK;
+}
+
+// Rice parameter of the last symbol of each A2 / D4 / E8 block (Z has none).
+int k_last_of(const hq_params &p) {
+    if (p.lattice == HQ_Z) return p.rice_k;
+    return p.rice_k > p.rice_dk_last ? p.rice_k - p.rice_dk_last : 0;
 }
 
 // The weights entry points take no dense rotation (a KV-cache option).
@@ -76,13 +83,15 @@ void set_scratch(EncodeArgs &a, void *ws, uint64_t nch) {
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ECUDA; }
 
-// Per-chunk word bound for ntiles tiles with symbols <= zmax.
-uint64_t chunk_bound(int lattice, int k, uint64_t ntiles, uint64_t zmax) {
-    uint64_t nsym = ntiles * kTile;
-    uint64_t nc = (lattice == HQ_E8) ? (16 * ntiles + 31) / 32 : 0;
-    uint64_t nr = 4 * (uint64_t)k * ntiles;
-    uint64_t ubits = nsym * (1 + (zmax >> k));
-    return nc + nr + (ubits + 31) / 32;
+// Per-chunk word bound for ntiles tiles with symbols <= zmax; the last symbol of each
+// block (1 in n of them) takes Rice parameter kl.
+uint64_t chunk_bound(int lattice, int k, int kl, uint64_t ntiles, uint64_t zmax) {
+    const uint64_t n = lattice == HQ_E8 ? 8 : lattice == HQ_D4 ? 4 : lattice == HQ_A2 ? 2 : 1;
+    const uint64_t nsym = ntiles * kTile, nlast = n > 1 ? nsym / n : 0;
+    const uint64_t nc = (lattice == HQ_E8) ? (16 * ntiles + 31) / 32 : 0;
+    const uint64_t rbits = (nsym - nlast) * (uint64_t)k + nlast * (uint64_t)kl;
+    const uint64_t ubits = (nsym - nlast) * (1 + (zmax >> k)) + nlast * (1 + (zmax >> kl));
+    return nc + (rbits + 31) / 32 + (ubits + 31) / 32;
 }
 
 }  // namespace
@@ -100,8 +109,8 @@ int hq_stream_bound(int64_t rows, int64_t cols, const hq_params *p, uint32_t max
     uint64_t tiles = (uint64_t)rows * (uint64_t)(cols / kTile);
     uint64_t nch = chunks_of(rows, cols);
     uint64_t full = tiles / kChunkTiles, rest = tiles % kChunkTiles;
-    uint64_t words = full * chunk_bound(p->lattice, p->rice_k, kChunkTiles, zmax);
-    if (rest) words += chunk_bound(p->lattice, p->rice_k, rest, zmax);
+    uint64_t words = full * chunk_bound(p->lattice, p->rice_k, k_last_of(*p), kChunkTiles, zmax);
+    if (rest) words += chunk_bound(p->lattice, p->rice_k, k_last_of(*p), rest, zmax);
     *max_words = words;
     *n_chunks = nch;
     return HQ_OK;
@@ -145,6 +154,7 @@ int hq_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_
     a.chunk_base = 0;
     a.c_scale = scale_fwd(p->alpha);
     a.k = p->rice_k;
+    a.k_last = k_last_of(*p);
     a.seed = p->seed;
     a.stream = d_stream;
     a.cap_words = cap_words;
@@ -183,6 +193,7 @@ int hq_dequantize(const uint32_t *d_stream, uint64_t stream_words, const uint64_
     a.n_chunks = nch;
     a.e_scale = scale_inv(p->alpha);
     a.k = p->rice_k;
+    a.k_last = k_last_of(*p);
     a.seed = p->seed;
     a.out = out;
     a.out_fp32 = out_dtype;
@@ -230,6 +241,7 @@ int hq_gemv(const uint32_t *d_stream, uint64_t stream_words, const uint64_t *d_o
     a.n_chunks = chunks_of(rows, cols);
     a.e_scale = scale_inv(p->alpha);
     a.k = p->rice_k;
+    a.k_last = k_last_of(*p);
     a.seed = p->seed;
     a.out = nullptr;
     a.stats = d_stats;
@@ -247,6 +259,7 @@ int hq_kv_init(hq_kv_cache *cache, int32_t heads, int32_t head_dim, const hq_par
     if (p->dither != 0 && p->dither != 1) return HQ_EINVAL;
     if (p->tile != kTile || p->chunk_tiles != kChunkTiles) return HQ_EUNSUPPORTED;
     if (p->rotation && !aligned(p->rotation, 16)) return HQ_EINVAL;
+    if (p->rice_dk_last < 0 || p->rice_dk_last > 15) return HQ_EINVAL;
     if (head_dim != kTile) return HQ_EUNSUPPORTED;
     if (heads <= 0) return HQ_EINVAL;
     if (!d_words || !aligned(d_words, 4) || !d_offsets || !aligned(d_offsets, 8) || offsets_cap < 1) return HQ_EINVAL;
@@ -301,6 +314,7 @@ int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t ld_token
     a.chunk_base = cache->chunks;
     a.c_scale = scale_fwd_of(p, alpha);
     a.k = p.rice_k;
+    a.k_last = k_last_of(p);
     a.seed = p.seed;
     a.rot = p.rotation;
     a.stream = cache->d_words;
@@ -346,6 +360,7 @@ int hq_kv_read(const hq_kv_cache *cache, void *out, int out_dtype, int64_t len, 
     a.map.heads = cache->heads;
     a.n_chunks = cache->chunks;
     a.k = cache->params.rice_k;
+    a.k_last = k_last_of(cache->params);
     a.seed = cache->params.seed;
     a.out = out;
     a.out_fp32 = out_dtype;
@@ -371,6 +386,7 @@ int rate_launch(const hq_params *p, EncodeArgs &a, hq_stats *d_stats, cudaStream
     if (a.n_chunks == 0) return HQ_OK;
     a.c_scale = scale_fwd_of(*p, p->alpha);
     a.k = p->rice_k;
+    a.k_last = k_last_of(*p);
     a.seed = p->seed;
     a.rot = p->rotation;
     a.stats = d_stats;
@@ -539,6 +555,7 @@ int hq_kv_scores(const hq_kv_cache *cache, const void *d_q, int32_t group, float
     a.map.heads = cache->heads;
     a.n_chunks = cache->chunks;
     a.k = cache->params.rice_k;
+    a.k_last = k_last_of(cache->params);
     a.seed = cache->params.seed;
     a.out = nullptr;
     a.out_ld = scores_ld;

@@ -32,12 +32,13 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
     const size_t smem = (size_t)(a.tcols * kSignWords + kWarpsPerCta * 2 * (kStageWords + kStagePad) +
                                  kWarpsPerCta * 128) *
                         sizeof(uint32_t);
-    const bool small = a.k <= 4;
-    auto kern = small ? decode_kernel<LAT, DITHER, KV, true, MODE> : decode_kernel<LAT, DITHER, KV, false, MODE>;
-    static LaunchPlan plans[2];
+    const bool small = a.k <= 4, mixed = a.k_last != a.k;
+    auto kern = mixed ? decode_kernel<LAT, DITHER, KV, false, MODE, false, true>
+                : small ? decode_kernel<LAT, DITHER, KV, true, MODE> : decode_kernel<LAT, DITHER, KV, false, MODE>;
+    static LaunchPlan plans[3];
     unsigned grid = 0;
-    cudaError_t e = plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta,
-                                               grid);
+    cudaError_t e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem,
+                                                           (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid);
     if (e != cudaSuccess) return e;
     kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     return cudaGetLastError();

@@ -150,6 +150,31 @@ __device__ __forceinline__ void rem_windows(const uint32_t *rw, int k, uint32_t 
     }
 }
 
+// Remainders of group g (8 symbols) of a lane whose 32 remainders start at bit `lb`
+// of the remainder plane `rem` (nr words), with the last symbol of each lattice block
+// taking kl bits and the others k (sym_k).  A group of at most 32 bits is one window.
+template <int N, bool STAGED>
+__device__ __forceinline__ void rem_group_mixed(const uint32_t *rem, uint32_t nr, uint32_t lb, int g, int k, int kl,
+                                                uint32_t gbits, uint32_t (&r)[8]) {
+    uint32_t b = lb + (uint32_t)g * gbits;
+    if (gbits <= 32u) {
+        uint32_t x = gbits ? fetch32<STAGED>(rem, nr, b) : 0u;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const int ki = sym_k<N>(i, k, kl);
+            r[i] = x & ((1u << ki) - 1u);
+            x >>= ki;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const int ki = sym_k<N>(i, k, kl);
+            r[i] = fetch32<STAGED>(rem, nr, b) & ((1u << ki) - 1u);
+            b += (uint32_t)ki;
+        }
+    }
+}
+
 // Where the tiles of one chunk go (computed once per chunk).
 template <bool KV>
 struct ChunkOut {
@@ -320,18 +345,19 @@ __device__ __forceinline__ float tile_sum(float acc) {
 
 // ROT: the dense KV rotation's inverse (rot_s: its shared form) in place of H_128
 // and the sign diagonal.
-template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED, int MODE, bool ROT>
+template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED, int MODE, bool ROT, bool MIXED>
 __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOut<KV> &geo, const uint32_t *src,
                                               bool ok, uint32_t nc, uint32_t nr, uint32_t nu,
                                               const uint32_t *startbit, const uint32_t *sign_tab,
                                               const float *rot_s, int lane) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
-    const int k = a.k;
+    const int k = a.k, kl = a.k_last;
     const int q = lane & 3;
     const uint32_t *un = src + nc + nr;
     const float2 e2 = make_float2(geo.e_scale, geo.e_scale);
-    const uint32_t pk = 1u << k;   // quotient weight 2^k
+    const uint32_t pk = 1u << k, pkl = 1u << kl;   // quotient weights 2^k, and 2^kl of a block's last symbol
+    const uint32_t gbits = group_rem_bits<N>(k, kl), lane_bits = 4u * gbits;
     bool bad = false;
     const int nrounds = (geo.ntiles + kTilesPerRound - 1) / kTilesPerRound;
 #pragma unroll 1
@@ -366,7 +392,10 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
                         xw >>= k;
                     }
                 } else {
-                    rem_group(rw, k, g, rv);
+                    if (MIXED)
+                        rem_group_mixed<N, STAGED>(src + nc, nr, segi * lane_bits, g, k, kl, gbits, rv);
+                    else
+                        rem_group(rw, k, g, rv);
                 }
                 float u[8];
 #pragma unroll
@@ -377,12 +406,13 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
                     if constexpr (LAT == HQ_E8) {
                         uint32_t zb[8];
 #pragma unroll
-                        for (int i = 0; i < 8; i++) zb[i] = imad(qv[bb * N + i], pk, rv[bb * N + i]);
+                        for (int i = 0; i < 8; i++) zb[i] = imad(qv[bb * N + i], i == N - 1 ? pkl : pk, rv[bb * N + i]);
                         e8_codes_from_symbols(zb, (coset >> b) & 1u, qq);
                     } else {
                         int32_t m[N];
 #pragma unroll
-                        for (int i = 0; i < N; i++) m[i] = unzigzag(imad(qv[bb * N + i], pk, rv[bb * N + i]));
+                        for (int i = 0; i < N; i++)
+                            m[i] = unzigzag(imad(qv[bb * N + i], (N > 1 && i == N - 1) ? pkl : pk, rv[bb * N + i]));
                         L::reinsert(m, (coset >> b) & 1u, qq);
                     }
                     L::point(qq, p);
@@ -467,7 +497,8 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
 // Three CTAs (24 warps) per SM without dither, where the decoder fits 80 registers with
 // almost no spills; two with dither, whose second lattice search needs more; one with
 // the dense rotation, whose shared form (kRotSmemBytes) comes first.
-template <int LAT, bool DITHER, bool KV, bool KSMALL, int MODE, bool ROT = false>
+// MIXED: the last symbol of each block has its own Rice parameter (a.k_last != a.k).
+template <int LAT, bool DITHER, bool KV, bool KSMALL, int MODE, bool ROT = false, bool MIXED = false>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : (DITHER ? 2 : 3)) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int kStageSlot = kStageWords + kStagePad;
@@ -513,7 +544,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : (DITHER ? 2 : 3))
         const int ntiles = geo.ntiles;
         const uint32_t nsym = (uint32_t)ntiles * kTile, nseg = 4u * (uint32_t)ntiles;
         const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
-        const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
+        const uint32_t nr = ((uint32_t)ntiles * tile_rem_bits<Lattice<LAT>::N>(k, a.k_last) + 31u) >> 5;
         bool ok = cw.ok && cw.nw >= (unsigned long long)(nc + nr) &&
                   (cw.nw - nc - nr) < (unsigned long long)(kMaxUnaryBits / 32u);
         const bool staged = cw.nw <= (unsigned long long)kStageWords;
@@ -524,12 +555,12 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : (DITHER ? 2 : 3))
         if (staged) {
             const uint32_t *src = stages + buf * kStageSlot;
             ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
-            bad = decode_rounds<LAT, DITHER, KV, KSMALL, true, MODE, ROT>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab,
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, true, MODE, ROT, MIXED>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab,
                                                                           rot_s, lane);
         } else {
             const uint32_t *src = a.stream + cw.w0;
             ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
-            bad = decode_rounds<LAT, DITHER, KV, KSMALL, false, MODE, ROT>(a, geo, src, ok, nc, nr, nu, startbit,
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, false, MODE, ROT, MIXED>(a, geo, src, ok, nc, nr, nu, startbit,
                                                                            sign_tab, rot_s, lane);
         }
         if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) status |= HQ_ST_CORRUPT;

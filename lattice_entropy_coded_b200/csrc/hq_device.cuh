@@ -565,6 +565,24 @@ __device__ __forceinline__ void dither_block<HQ_Z>(uint64_t seed, uint64_t e, fl
     d[0] = __fsub_rn(w, (float)rint_int(w));
 }
 
+// ------------------------------------------------------------------ Rice parameters
+// The Rice parameter of symbol i of a lane's run (its position i mod N in the lattice
+// block): bit-stripping halves the last symbol of an A2, D4 or E8 block, which may take
+// its own parameter kl (kl = k gives the single-parameter code).  Z has no such symbol.
+template <int N>
+__device__ __forceinline__ int sym_k(int i, int k, int kl) {
+    return (N > 1 && (i % N) == N - 1) ? kl : k;
+}
+// Remainder bits of one 128-element tile, and of a group of 8 symbols.
+template <int N>
+__device__ __forceinline__ uint32_t tile_rem_bits(int k, int kl) {
+    return N > 1 ? (uint32_t)(128 / N) * (uint32_t)((N - 1) * k + kl) : 128u * (uint32_t)k;
+}
+template <int N>
+__device__ __forceinline__ uint32_t group_rem_bits(int k, int kl) {
+    return N > 1 ? (uint32_t)(8 / N) * (uint32_t)((N - 1) * k + kl) : 8u * (uint32_t)k;
+}
+
 // ------------------------------------------------------------------ integer helpers
 // q = a / b, r = a % b (b > 0) with one 32-bit division when both fit, which is the
 // usual case for chunk and tile counts; the 64-bit division otherwise.

@@ -10,6 +10,7 @@ namespace {
 template <int LAT, bool DITHER>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     const bool small = a.k <= 4;
+    const bool mixed = a.k_last != a.k;   // a second Rice parameter: per-warp or grouped forms only
     cudaError_t e;
     unsigned grid = 0;
     // by size: the wide form while every chunk gets a 16-warp group of its own in one
@@ -17,6 +18,7 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     // (148 x 2 x kGroups), else the per-warp form
     int mode = g_encode_path;
     if (mode == 0) mode = (a.n_chunks <= 296ull) ? 3 : (a.n_chunks <= 592ull) ? 2 : 1;
+    if (mixed && mode == 3) mode = 2;
     if (mode == 3) {
         const size_t smem =
             (size_t)(a.tcols * kSignWords + 2 * kStageWords) * sizeof(uint32_t) + sizeof(WideCtl);
@@ -28,20 +30,23 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
         const size_t smem = (size_t)(a.tcols * kSignWords + kGroups * 2 * kStageWords +
                                      kWarpsPerCta * 32 * kGroupSlotWords) * sizeof(uint32_t) +
                             kGroups * sizeof(GroupCtl);
-        auto kern = small ? encode_kernel_grouped<LAT, DITHER, true, false> : encode_kernel_grouped<LAT, DITHER, false, false>;
-        static LaunchPlan plans[2];
-        if ((e = plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kGroups - 1) / kGroups, grid)) !=
-            cudaSuccess)
+        auto kern = mixed ? encode_kernel_grouped<LAT, DITHER, false, false, true>
+                    : small ? encode_kernel_grouped<LAT, DITHER, true, false> : encode_kernel_grouped<LAT, DITHER, false, false>;
+        static LaunchPlan plans[3];
+        if ((e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kGroups - 1) / kGroups,
+                                                        grid)) != cudaSuccess)
             return e;
         kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     } else {
         const size_t smem =
             (size_t)(a.tcols * kSignWords + kWarpsPerCta * 2 * kStageWords + kWarpsPerCta * 32 * kInSlotWords) *
             sizeof(uint32_t);
-        auto kern = small ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
-        static LaunchPlan plans[2];
-        if ((e = plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta,
-                                           grid)) != cudaSuccess)
+        auto kern = mixed ? encode_kernel<LAT, DITHER, false, true>
+                    : small ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
+        static LaunchPlan plans[3];
+        if ((e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem,
+                                                        (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid)) !=
+            cudaSuccess)
             return e;
         kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     }

@@ -361,7 +361,7 @@ __device__ __forceinline__ void round_symbols_rolled(const EncodeArgs &a, const 
     cbits = 0;
     usum = 0;
     lor = 0;
-    const int k = a.k;
+    const int k = a.k, kl = a.k_last;
     const unsigned long long eq = in.e0 + 32ull * q;
 #pragma unroll 1
     for (int b = 0; b < 32 / N; b++) {
@@ -378,7 +378,7 @@ __device__ __forceinline__ void round_symbols_rolled(const EncodeArgs &a, const 
 #pragma unroll
         for (int i = 0; i < N; i++) {
             zz[i] = (!DITHER || in.valid) ? zz[i] : 0u;
-            usum += zz[i] >> k;
+            usum += zz[i] >> sym_k<N>(i, k, kl);
             lor |= zz[i];
         }
         row_store<N>(row + b * N, zz);
@@ -426,6 +426,44 @@ __device__ __forceinline__ void put_rem(uint32_t *dst, const uint32_t (&z)[32], 
     }
 }
 
+// Remainder bits of a lane's 32 symbols with a second Rice parameter kl for the last
+// symbol of each lattice block (sym_k): the lane's run starts at bit `lb` of the
+// remainder plane, so it shares its first and last words with its neighbours; every
+// word is ORed in (the plane is zeroed).  A group of 8 remainders that fits in 32 bits
+// is built in one register, last symbol first.
+template <int N>
+__device__ __forceinline__ void put_rem_mixed(uint32_t *rem, uint32_t lb, const uint32_t (&z)[32], int k, int kl) {
+    const uint32_t gbits = group_rem_bits<N>(k, kl);
+    if (gbits == 0u) return;
+#pragma unroll
+    for (int g = 0; g < 4; g++) {
+        const uint32_t b0 = lb + (uint32_t)g * gbits;
+        if (gbits <= 32u) {
+            uint32_t gv = 0;
+#pragma unroll
+            for (int i = 7; i >= 0; i--) {
+                const int ki = sym_k<N>(i, k, kl);
+                gv = imad(gv, 1u << ki, z[8 * g + i] & ((1u << ki) - 1u));
+            }
+            const uint32_t w0 = b0 >> 5, sh = b0 & 31u;
+            atomicOr(rem + w0, gv << sh);
+            if (sh + gbits > 32u) atomicOr(rem + w0 + 1, gv >> (32u - sh));
+        } else {
+            uint32_t b = b0;
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const int ki = sym_k<N>(i, k, kl);
+                const uint32_t w0 = b >> 5, sh = b & 31u, val = z[8 * g + i] & ((1u << ki) - 1u);
+                if (ki) {
+                    atomicOr(rem + w0, val << sh);
+                    if (sh + (uint32_t)ki > 32u) atomicOr(rem + w0 + 1, val >> (32u - sh));
+                }
+                b += (uint32_t)ki;
+            }
+        }
+    }
+}
+
 // Unary terminators of 8 symbols with quotients q[0..7], starting at bit pos of
 // `un` (zeroed shared words).  A group whose codes fit in 32 bits is built in a
 // register (last symbol first) and ORed in with at most two shared atomics.
@@ -463,8 +501,9 @@ __device__ __noinline__ void encode_chunk_global(const EncodeArgs &a, const Chun
                                                  const float *rot_s, uint32_t *g, unsigned long long room,
                                                  uint32_t nc, uint32_t nr) {
     const int lane = threadIdx.x & 31;
-    const int k = a.k;
-    const uint32_t mask = k ? (1u << k) - 1u : 0u;
+    constexpr int N = Lattice<LAT>::N;
+    const int k = a.k, kl = a.k_last;
+    const unsigned long long lane_bits = 4ull * group_rem_bits<N>(k, kl);   // remainder bits of 32 symbols
     const int nrounds = (geo.ntiles + kTilesPerRound - 1) / kTilesPerRound;
     unsigned long long urun = 0;
     for (int r = 0; r < nrounds; r++) {
@@ -485,7 +524,7 @@ __device__ __noinline__ void encode_chunk_global(const EncodeArgs &a, const Chun
         const bool valid = in.valid;
         unsigned long long ub = 0;
 #pragma unroll
-        for (int i = 0; i < 32; i++) ub += z[i] >> k;
+        for (int i = 0; i < 32; i++) ub += z[i] >> sym_k<N>(i, k, kl);
         ub = valid ? ub + 32 : 0;
         unsigned long long incl = ub;
 #pragma unroll
@@ -497,13 +536,14 @@ __device__ __noinline__ void encode_chunk_global(const EncodeArgs &a, const Chun
         if (valid) {
             const unsigned long long cw = 4ull * r + (lane >> 3);
             if (LAT == HQ_E8 && cbits && cw < room) atomicOr(g + cw, cbits << (4 * (lane & 7)));
-            unsigned long long rb = 32ull * (nc + (unsigned long long)(32 * r + lane) * k);
+            unsigned long long rb = 32ull * nc + (unsigned long long)(32 * r + lane) * lane_bits;
             unsigned long long pos = 32ull * (nc + nr) + urun + incl - ub;
             for (int i = 0; i < 32; i++) {
-                const uint32_t rr = z[i] & mask;
-                for (int b = 0; b < k; b++, rb++)
+                const int ki = sym_k<N>(i, k, kl);
+                const uint32_t rr = z[i] & ((1u << ki) - 1u);
+                for (int b = 0; b < ki; b++, rb++)
                     if (((rr >> b) & 1u) && (rb >> 5) < room) atomicOr(g + (rb >> 5), 1u << (uint32_t)(rb & 31));
-                pos += z[i] >> k;
+                pos += z[i] >> ki;
                 if ((pos >> 5) < room) atomicOr(g + (pos >> 5), 1u << (uint32_t)(pos & 31));
                 pos++;
             }
@@ -551,7 +591,7 @@ __device__ __forceinline__ void finish_chunk_warp(const EncodeArgs &a, const Pen
         ChunkGeo geo;
         geo.init(a.map, p.c);
         const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * geo.ntiles + 31) / 32u : 0u;
-        const uint32_t nr = 4u * (uint32_t)a.k * (uint32_t)geo.ntiles;
+        const uint32_t nr = ((uint32_t)geo.ntiles * tile_rem_bits<Lattice<LAT>::N>(a.k, a.k_last) + 31u) >> 5;
         encode_chunk_global<LAT, DITHER, false>(a, geo, sign_tab, nullptr, g, room, nc, nr);
     }
     __syncwarp();
@@ -565,7 +605,9 @@ __device__ __forceinline__ unsigned long long take_ticket(const EncodeArgs &a) {
 
 // Throughput form: persistent CTAs of kWarpsPerCta warps, each warp encoding whole
 // chunks (4 rounds of 8 tiles) taken by ticket, with a two-chunk stage pipeline.
-template <int LAT, bool DITHER, bool KSMALL>
+// MIXED: the last symbol of each block has its own Rice parameter (a.k_last != a.k),
+// so lanes' remainder runs are not word-aligned (put_rem_mixed).
+template <int LAT, bool DITHER, bool KSMALL, bool MIXED = false>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *sign_tab = smem;                                        // tcols * kSignWords
@@ -578,7 +620,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     build_sign_table(sign_tab, a.tcols, a.seed);
     __syncthreads();
 
-    const int k = a.k;
+    constexpr int N = Lattice<LAT>::N;
+    const int k = a.k, kl = a.k_last;
+    const uint32_t lane_bits = 4u * group_rem_bits<N>(k, kl);   // remainder bits of a lane's 32 symbols
     const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
     uint32_t status = 0, zor_all = 0;
     unsigned long long payload = 0;
@@ -601,7 +645,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         const int ntiles = geo.ntiles;
         const int nrounds = (ntiles + kTilesPerRound - 1) / kTilesPerRound;
         const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
-        const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
+        const uint32_t rbits = (uint32_t)ntiles * tile_rem_bits<N>(k, kl);
+        const uint32_t nr = (rbits + 31u) >> 5;
         {
             uint4 *s4 = reinterpret_cast<uint4 *>(stage);
             for (int i = lane; i < kStageWords / 4; i += 32) s4[i] = make_uint4(0, 0, 0, 0);
@@ -634,7 +679,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             uint32_t usum = 0, lor = 0;
 #pragma unroll
             for (int i = 0; i < 32; i++) {
-                usum += z[i] >> k;
+                usum += z[i] >> sym_k<N>(i, k, kl);
                 lor |= z[i];
             }
             zor |= lor;
@@ -651,7 +696,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             if (!overflow && nc + nr + (uint32_t)(((unsigned long long)urun + rtot + 31) >> 5) > (uint32_t)kStageWords)
                 overflow = true;
             if (!overflow && !range_bad) {
-                put_rem<KSMALL>(stage + nc + (uint32_t)(32 * r + lane) * (uint32_t)k, z, k, valid);
+                if (MIXED) {
+                    if (valid) put_rem_mixed<N>(stage + nc, (uint32_t)(32 * r + lane) * lane_bits, z, k, kl);
+                } else {
+                    put_rem<KSMALL>(stage + nc + (uint32_t)(32 * r + lane) * (uint32_t)k, z, k, valid);
+                }
                 if (valid) {
                     if (LAT == HQ_E8 && cbits) atomicOr(stage + 4 * r + (lane >> 3), cbits << (4 * (lane & 7)));
                     uint32_t *un = stage + nc + nr;
@@ -660,7 +709,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
                     for (int g = 0; g < 4; g++) {
                         uint32_t qg[8];
 #pragma unroll
-                        for (int i = 0; i < 8; i++) qg[i] = z[8 * g + i] >> k;
+                        for (int i = 0; i < 8; i++) qg[i] = z[8 * g + i] >> sym_k<N>(i, k, kl);
                         pos += unary_group_shared(un, pos, qg);
                     }
                 }
@@ -670,7 +719,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         zor_all |= zor;
         if (range_bad) status |= HQ_ST_RANGE;
         const unsigned long long total = nc + nr + ((unsigned long long)urun + 31) / 32;
-        payload += urun + (unsigned long long)nr * 32 + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
+        payload += urun + (unsigned long long)rbits + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
         lookback_publish(a.lookback, c, total);
 
         // the previous chunk's predecessors have had a whole chunk's time to publish
@@ -746,7 +795,7 @@ __device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending 
         ChunkGeo geo;
         geo.init(a.map, p.c);
         const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * geo.ntiles + 31) / 32u : 0u;
-        const uint32_t nr = 4u * (uint32_t)a.k * (uint32_t)geo.ntiles;
+        const uint32_t nr = ((uint32_t)geo.ntiles * tile_rem_bits<Lattice<LAT>::N>(a.k, a.k_last) + 31u) >> 5;
         encode_chunk_global<LAT, DITHER, ROT>(a, geo, sign_tab, rot_s, g, room, nc, nr);
     }
     __syncwarp();
@@ -762,7 +811,7 @@ __device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending 
 // ROT: the dense KV rotation instead of the sign diagonal and H_128, its shared form
 // (kRotSmemBytes) ahead of the rest; one CTA per SM (the shared memory).  The
 // rotation runs at the fp32 fma rate, so this form serves every launch size.
-template <int LAT, bool DITHER, bool KSMALL, bool ROT>
+template <int LAT, bool DITHER, bool KSMALL, bool ROT, bool MIXED = false>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) encode_kernel_grouped(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -789,7 +838,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) encode_kernel_
     __syncthreads();
 
     const unsigned long long n = a.n_chunks;
-    const int k = a.k;
+    constexpr int N = Lattice<LAT>::N;
+    const int k = a.k, kl = a.k_last;
+    const uint32_t lane_bits = 4u * group_rem_bits<N>(k, kl);
     const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
     uint32_t status = 0, zor_all = 0;
     unsigned long long payload = 0;
@@ -858,7 +909,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) encode_kernel_
             }
             const int ntiles = geo.ntiles;
             const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
-            const uint32_t nr = 4u * (uint32_t)k * (uint32_t)ntiles;
+            const uint32_t rbits = (uint32_t)ntiles * tile_rem_bits<N>(k, kl);
+            const uint32_t nr = (rbits + 31u) >> 5;
             range_bad = badw != 0u || U >= kMaxUnaryBits;
             total = nc + nr + (U + 31) / 32;
             overflow = total > (unsigned long long)kStageWords;
@@ -876,7 +928,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) encode_kernel_
                 prefetch_round(a, gn, w, lane, slot);
             }
             if (!overflow && !range_bad) {
-                put_rem<KSMALL>(stage + nc + (uint32_t)(32 * w + lane) * (uint32_t)k, z, k, valid);
+                if (MIXED) {
+                    if (valid) put_rem_mixed<N>(stage + nc, (uint32_t)(32 * w + lane) * lane_bits, z, k, kl);
+                } else {
+                    put_rem<KSMALL>(stage + nc + (uint32_t)(32 * w + lane) * (uint32_t)k, z, k, valid);
+                }
                 if (valid) {
                     if (LAT == HQ_E8 && cbits) atomicOr(stage + 4 * w + (lane >> 3), cbits << (4 * (lane & 7)));
                     uint32_t *un = stage + nc + nr;
@@ -885,7 +941,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) encode_kernel_
                     for (int gq = 0; gq < 4; gq++) {
                         uint32_t qg[8];
 #pragma unroll
-                        for (int i = 0; i < 8; i++) qg[i] = z[8 * gq + i] >> k;
+                        for (int i = 0; i < 8; i++) qg[i] = z[8 * gq + i] >> sym_k<N>(i, k, kl);
                         pos += unary_group_shared(un, pos, qg);
                     }
                 }
@@ -893,7 +949,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) encode_kernel_
             if (w == 0) {
                 lookback_publish(a.lookback, c, total);
                 if (range_bad) status |= HQ_ST_RANGE;
-                if (lane == 0) payload += U + (unsigned long long)nr * 32 + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
+                if (lane == 0) payload += U + (unsigned long long)rbits + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
             }
         }
         // the previous chunk: its predecessors have had a whole chunk's time to publish
@@ -1168,7 +1224,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) rate_kernel(co
         build_sign_table(sign_tab, a.tcols, a.seed);
     __syncthreads();
     const int lane = threadIdx.x & 31;
-    const int k = a.k;
+    constexpr int N = Lattice<LAT>::N;
+    const int k = a.k, kl = a.k_last;
     const unsigned long long nwarps = (unsigned long long)gridDim.x * kWarpsPerCta;
     unsigned long long payload = 0, words = 0;
     uint32_t status = 0, zor_all = 0;
@@ -1195,7 +1252,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) rate_kernel(co
             uint32_t usum = 0;
 #pragma unroll
             for (int i = 0; i < 32; i++) {
-                usum += z[i] >> k;
+                usum += z[i] >> sym_k<N>(i, k, kl);
                 lor |= z[i];
             }
             // symbols below 2^22 keep ub below 2^28: two 32-bit sums of its halves are exact
@@ -1207,8 +1264,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) rate_kernel(co
         lor = __reduce_or_sync(0xffffffffu, lor);
         zor_all |= lor;
         const unsigned long long nc = (LAT == HQ_E8) ? (16ull * geo.ntiles + 31) / 32 : 0ull;
-        const unsigned long long nr = 4ull * (unsigned long long)k * (unsigned long long)geo.ntiles;
-        payload += U + nr * 32 + ((LAT == HQ_E8) ? 16ull * geo.ntiles : 0ull);
+        const unsigned long long rbits = (unsigned long long)geo.ntiles * tile_rem_bits<N>(k, kl);
+        const unsigned long long nr = (rbits + 31) / 32;
+        payload += U + rbits + ((LAT == HQ_E8) ? 16ull * geo.ntiles : 0ull);
         words += nc + nr + (U + 31) / 32;
         if ((lor >> 22) != 0u || U >= kMaxUnaryBits) status |= HQ_ST_RANGE;
     }

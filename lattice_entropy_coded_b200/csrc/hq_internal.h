@@ -46,6 +46,7 @@ struct EncodeArgs {
     uint64_t chunk_base;      // global index of this call's first chunk (offset array position)
     float c_scale;            // alpha / sqrt(128), rounded to fp32 on the host
     int k;                    // Rice parameter
+    int k_last;               // Rice parameter of the last symbol of each A2 / D4 / E8 block (k: single code)
     uint64_t seed;
     uint32_t *stream;
     uint64_t cap_words;
@@ -73,6 +74,7 @@ struct DecodeArgs {
     uint64_t n_chunks;
     float e_scale;            // 1 / (alpha sqrt(128)), weights path
     int k;
+    int k_last;               // as EncodeArgs::k_last
     uint64_t seed;
     void *out;
     int out_fp32;

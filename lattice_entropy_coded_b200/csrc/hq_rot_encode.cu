@@ -14,16 +14,17 @@ namespace {
 // groups per SM (the rotation's 66 KB shared form).
 template <int LAT, bool DITHER>
 cudaError_t launch_rot_t(const EncodeArgs &a, cudaStream_t s) {
-    const bool small = a.k <= 4;
+    const bool small = a.k <= 4, mixed = a.k_last != a.k;
     const size_t smem = kRotSmemBytes +
                         (size_t)(a.tcols * kSignWords + kGroups * 2 * kStageWords + kWarpsPerCta * 32 * kGroupSlotWords) *
                             sizeof(uint32_t) +
                         kGroups * sizeof(GroupCtl);
-    auto kern = small ? encode_kernel_grouped<LAT, DITHER, true, true> : encode_kernel_grouped<LAT, DITHER, false, true>;
-    static LaunchPlan plans[2];
+    auto kern = mixed ? encode_kernel_grouped<LAT, DITHER, false, true, true>
+                : small ? encode_kernel_grouped<LAT, DITHER, true, true> : encode_kernel_grouped<LAT, DITHER, false, true>;
+    static LaunchPlan plans[3];
     unsigned grid = 0;
     cudaError_t e =
-        plans[small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kGroups - 1) / kGroups, grid);
+        plans[mixed ? 2 : small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kGroups - 1) / kGroups, grid);
     if (e != cudaSuccess) return e;
     kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     return cudaGetLastError();

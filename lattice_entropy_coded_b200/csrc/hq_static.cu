@@ -56,6 +56,7 @@ int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, co
     if (p->rice_k < 0 || p->rice_k > 15 || (p->dither != 0 && p->dither != 1)) return HQ_EINVAL;
     if (p->tile != kTile || p->chunk_tiles != kChunkTiles) return HQ_EUNSUPPORTED;
     if (p->rotation) return HQ_EUNSUPPORTED;   // the dense rotation is a KV-cache option
+    if (p->rice_dk_last < 0 || p->rice_dk_last > 15) return HQ_EINVAL;
     if (rows < 0 || cols < 0 || cols % kTile) return HQ_EINVAL;
     if (cols > 65536) return HQ_EUNSUPPORTED;
     const uint64_t tiles = (uint64_t)rows * (uint64_t)(cols / kTile);
@@ -87,6 +88,7 @@ int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, co
     a.chunk_base = 0;
     a.c_scale = (float)((double)p->alpha / __builtin_sqrt(128.0));
     a.k = p->rice_k;
+    a.k_last = (p->lattice == HQ_Z) ? p->rice_k : (p->rice_k > p->rice_dk_last ? p->rice_k - p->rice_dk_last : 0);
     a.seed = p->seed;
     a.stream = d_stream;
     a.cap_words = cap_words;

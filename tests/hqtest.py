@@ -27,7 +27,7 @@ def u16(t: torch.Tensor) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- oracle (threaded over chunk ranges)
-def oracle_quantize(x: torch.Tensor, lat: int, alpha: float, k: int, seed: int, dither: int = 0):
+def oracle_quantize(x: torch.Tensor, lat: int, alpha: float, k: int, seed: int, dither: int = 0, dk_last: int = 0):
     """-> (words uint32 [total], offsets uint64 [n+1] absolute, payload bits)."""
     xu = u16(x)
     R, Cc = xu.shape
@@ -36,7 +36,7 @@ def oracle_quantize(x: torch.Tensor, lat: int, alpha: float, k: int, seed: int, 
         return np.zeros(0, np.uint32), np.zeros(1, np.uint64), 0
     step = max(1, -(-nch // THREADS))
     ranges = [(a, min(nch, a + step)) for a in range(0, nch, step)]
-    parts = list(_POOL.map(lambda r: O.quantize(xu, lat, alpha, k, seed, dither, r[0], r[1]), ranges))
+    parts = list(_POOL.map(lambda r: O.quantize(xu, lat, alpha, k, seed, dither, r[0], r[1], dk_last=dk_last), ranges))
     words, offs, pay, base = [], [], 0, 0
     for (s, off, pb) in parts:
         words.append(s[:int(off[-1])])
@@ -47,7 +47,7 @@ def oracle_quantize(x: torch.Tensor, lat: int, alpha: float, k: int, seed: int, 
     return np.concatenate(words), np.concatenate(offs), pay
 
 
-def oracle_dequantize(words, offsets, rows, cols, lat, alpha, k, seed, dither=0, fp32=True):
+def oracle_dequantize(words, offsets, rows, cols, lat, alpha, k, seed, dither=0, fp32=True, dk_last=0):
     out = np.zeros((rows, cols), np.float32 if fp32 else np.uint16)
     nch = len(offsets) - 1
     if nch == 0:
@@ -55,7 +55,7 @@ def oracle_dequantize(words, offsets, rows, cols, lat, alpha, k, seed, dither=0,
     step = max(1, -(-nch // THREADS))
     ranges = [(a, min(nch, a + step)) for a in range(0, nch, step)]
     list(_POOL.map(lambda r: O.dequantize(words, offsets[r[0]:r[1] + 1], rows, cols, lat, alpha, k, seed, dither,
-                                          fp32, r[0], r[1], out=out), ranges))
+                                          fp32, r[0], r[1], out=out, dk_last=dk_last), ranges))
     return out
 
 

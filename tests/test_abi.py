@@ -34,13 +34,13 @@ def test_library_exports_every_declared_symbol():
 
 def test_struct_layouts_match_header():
     import lattice_entropy_coded_b200 as hq
-    assert C.sizeof(hq.hq_params) == 40
+    assert C.sizeof(hq.hq_params) == 48
     assert hq.hq_params.seed.offset == 16 and hq.hq_params.chunk_tiles.offset == 28
-    assert hq.hq_params.rotation.offset == 32
+    assert hq.hq_params.rotation.offset == 32 and hq.hq_params.rice_dk_last.offset == 40
     assert C.sizeof(hq.hq_stats) == 32 and hq.hq_stats.payload_bits.offset == 8
     assert C.sizeof(hq.hq_kv_append_row) == 32
-    assert C.sizeof(hq.hq_kv_cache) == 136 and hq.hq_kv_cache.params.offset == 72
-    assert hq.hq_kv_cache.tokens.offset == 112
+    assert C.sizeof(hq.hq_kv_cache) == 144 and hq.hq_kv_cache.params.offset == 72
+    assert hq.hq_kv_cache.tokens.offset == 120
     assert C.sizeof(hq.hq_calib_spec) == 48 and hq.hq_calib_spec.k_lo.offset == 32
     assert C.sizeof(hq.hq_calib_result) == 24 and hq.hq_calib_result.bps.offset == 8
 
@@ -56,18 +56,23 @@ def test_stream_bound_and_workspace():
     assert n2 == 1
     assert w2 == math.ceil(16 * 9 / 32) + 4 * 2 * 9 + math.ceil(9 * 128 * (1 + (15 >> 2)) / 32)
     assert hq.hq_stream_bound(0, 4096, p) == (0, 0)
+    # a second Rice parameter for the last symbol of each block: 1 in 8 E8 symbols at k - 1
+    p2 = hq.make_params("E8", 300.0, 2, dk_last=1)
+    w3, _ = hq.hq_stream_bound(3, 384, p2, 7)
+    assert w3 == (math.ceil(16 * 9 / 32) + math.ceil((1008 * 2 + 144 * 1) / 32)
+                  + math.ceil((1008 * (1 + (15 >> 2)) + 144 * (1 + (15 >> 1))) / 32))
     assert hq.hq_workspace_bytes(1000) >= 1000 * 8 + 8
     assert hq.hq_workspace_bytes(1000) % 256 == 0
 
 
 @pytest.mark.parametrize("bad", [
     dict(lattice=7), dict(alpha=0.0), dict(alpha=float("nan")), dict(alpha=-1.0), dict(rice_k=16),
-    dict(rice_k=-1), dict(dither=2)])
+    dict(rice_k=-1), dict(dither=2), dict(dk_last=-1), dict(dk_last=16)])
 def test_invalid_params_rejected(bad):
     import lattice_entropy_coded_b200 as hq
-    kw = dict(lattice=3, alpha=1.0, rice_k=2, seed=0, dither=0)
+    kw = dict(lattice=3, alpha=1.0, rice_k=2, seed=0, dither=0, dk_last=0)
     kw.update(bad)
-    p = hq.hq_params(128, kw["lattice"], kw["alpha"], kw["rice_k"], 0, kw["dither"], 32, None)
+    p = hq.hq_params(128, kw["lattice"], kw["alpha"], kw["rice_k"], 0, kw["dither"], 32, None, kw["dk_last"], 0)
     with pytest.raises(hq.HQError, match="invalid"):
         hq.hq_stream_bound(32, 128, p)
 
