@@ -381,7 +381,7 @@ def oracle_workload(workload: str, threads: int, budget_s: float = 60.0, pts=Non
     import oracle as O
     from oracle import rotation as ORot
     w = synth.WORKLOADS[workload]
-    pts = rate_points()[workload]["points"] if pts is None else pts
+    pts = rate_points()[workload if workload in rate_points() else w["points_of"]]["points"] if pts is None else pts
     O.lib()
 
     def u16(t):
@@ -431,8 +431,9 @@ def oracle_workload(workload: str, threads: int, budget_s: float = 60.0, pts=Non
                     jobs = [(a, min(nch, a + step)) for a in range(0, nch, step)]
 
                     def job(r, xu=xu, R=R, Cc=Cc):
-                        s_, off, _ = O.quantize(xu, lat, p["alpha"], p["k"], w["seed"], 0, r[0], r[1])
-                        O.dequantize(s_, off, R, Cc, lat, p["alpha"], p["k"], w["seed"], 0, False, r[0], r[1])
+                        dk = p.get("dk_last", 0)
+                        s_, off, _ = O.quantize(xu, lat, p["alpha"], p["k"], w["seed"], 0, r[0], r[1], dk_last=dk)
+                        O.dequantize(s_, off, R, Cc, lat, p["alpha"], p["k"], w["seed"], 0, False, r[0], r[1], dk_last=dk)
                     n_el = xu.size
                 t0 = time.perf_counter()
                 list(ex.map(job, jobs))
@@ -632,7 +633,7 @@ def run_bulk(args):
         if rots:
             out["rotation"] = "Haar-uniform 128x128 per tensor (hq_haar_rotation), alpha/k calibrated on the device"
     else:
-        pts = rate_points()[wl]["points"]
+        pts = rate_points()[wl if wl in rate_points() else w["points_of"]]["points"]
         if w["kind"] == "weight":
             mats = [synth.weight(w["rows"], w["cols"], w["seed"], device=device)]
         elif w["kind"] == "weight_set":
@@ -640,18 +641,40 @@ def run_bulk(args):
         else:
             mats = list(synth.student_t(w["n"], w["rows"], w["cols"], w["seed"], device=device))
         n = sum(m.numel() for m in mats)
+        if w.get("dk_last"):
+            # a second Rice parameter for the last symbol of each block: alpha and k for each
+            # target rate calibrated on the device in that mode (untimed); each is timed next to
+            # the single-parameter point of the same rate, the same way
+            big = torch.cat(mats, dim=0)
+            cal_pts = []
+            for p in pts:
+                dk = w["dk_last"][p["lattice"]]
+                cal_pts.append(dict(p, dk_last=0))
+                if dk:
+                    c = hq.hq_calibrate(big, hq.make_params(p["lattice"], 1.0, 0, w["seed"], 0, dk_last=dk),
+                                        hq.calib_spec(p["bps"], tol=0.002, k_lo=0, k_hi=6), hq.stats_tensor(device))
+                    cal_pts.append(dict(p, alpha=c["alpha"], k=c["k"], dk_last=dk))
+            pts = cal_pts
+            del big
+        # inputs that fit in L2 are evicted before each step (a buffer larger than L2 is written)
+        flush = (torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+                 if 2 * n < L2_FLUSH_BYTES else None)
         res = []
         for p in pts:
-            params = hq.make_params(p["lattice"], p["alpha"], p["k"], w["seed"], 0)
+            params = hq.make_params(p["lattice"], p["alpha"], p["k"], w["seed"], 0, dk_last=p.get("dk_last", 0))
             codecs = [hq.Codec(m.shape[0], m.shape[1], params, device=device,
                                cap_words=int(m.numel() * (p["bps"] + 3.0) / 32) + 8192) for m in mats]
             outs = [torch.empty_like(m) for m in mats]
             enc_ms, dec_ms = [], []
             for it in range(args.warmup + args.steps):
+                if flush is not None:
+                    flush.fill_(it)
                 e0, e1 = _events()
                 e0.record()
                 comps = [c.quantize(m) for c, m in zip(codecs, mats)]
                 e1.record()
+                if flush is not None:
+                    flush.fill_(it + 1)
                 d0, d1 = _events()
                 d0.record()
                 for c, cp, o in zip(codecs, comps, outs):
@@ -673,7 +696,8 @@ def run_bulk(args):
                             bps_payload=sum(st["payload_bits"] for st in stats) / n, bps_stream=words * 32.0 / n,
                             mse=se / n, d_over_sigma2=se / n / var, matrices=len(mats), elements=n,
                             encode_ms=em, decode_ms=dm, encode_gbs=2.0 * n / (em * 1e6), decode_gbs=2.0 * n / (dm * 1e6),
-                            encode_hbm_frac=alg / (em * 1e6) / peak, decode_hbm_frac=alg / (dm * 1e6) / peak))
+                            encode_hbm_frac=alg / (em * 1e6) / peak, decode_hbm_frac=alg / (dm * 1e6) / peak,
+                            **({"dk_last": p["dk_last"]} if "dk_last" in p else {})))
             del codecs, outs, comps
             torch.cuda.empty_cache()
         out["points"] = res
@@ -682,9 +706,10 @@ def run_bulk(args):
     if args.oracle:
         threads = host_threads()
         out["oracle"] = {"threads": threads,
-                         "points": oracle_workload(wl, threads, pts=pts if w["kind"] == "kv" else None)}
+                         "points": oracle_workload(wl, threads,
+                                                   pts=pts if (w["kind"] == "kv" or w.get("dk_last")) else None)}
         if w["kind"] == "weight":
-            out["oracle"]["single_thread"] = oracle_workload(wl, 1)
+            out["oracle"]["single_thread"] = oracle_workload(wl, 1, pts=pts if w.get("dk_last") else None)
     print(json.dumps(out), flush=True)
 
 

@@ -109,6 +109,10 @@ def student_t(n: int, rows: int, cols: int, seed: int, device="cpu", nu: int = 5
 WORKLOADS = {
     "weight_1024x1024_e8_4bps": dict(kind="weight", rows=1024, cols=1024, seed=0),
     "weight_4096x4096_rate_sweep": dict(kind="weight", rows=4096, cols=4096, seed=1),
+    # the same sweep with a second Rice parameter for the last symbol of each block
+    "weight_4096x4096_rate_sweep_dk": dict(kind="weight", rows=4096, cols=4096, seed=1,
+                                           points_of="weight_4096x4096_rate_sweep",
+                                           dk_last={"E8": 1, "D4": 1, "A2": 2, "Z": 0}),
     "kv_8h_32768tok_e8_dither": dict(kind="kv", heads=8, tokens=32768, seed=2, append=256),
     # the same cache with a dense Haar-uniform rotation per tensor instead of the sign diagonal and H_128
     "kv_8h_32768tok_e8_dither_haar": dict(kind="kv", heads=8, tokens=32768, seed=2, append=256, rotation=True),
