@@ -35,6 +35,7 @@ namespace hq {
 namespace {
 
 constexpr int kStagePad = 4;   // zero words after a staged chunk: unchecked 2-word reads stay inside
+constexpr int kRotDecodeWarps = 12;   // warps per CTA of the dense-rotation decoder (one CTA per SM)
 
 // 32 bits of a plane of `n` words starting at bit `b`; words at or past n read as 0.
 __device__ __forceinline__ uint32_t fetch32_checked(const uint32_t *p, uint32_t n, uint32_t b) {
@@ -495,17 +496,20 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
 }
 
 // Three CTAs (24 warps) per SM without dither, where the decoder fits 80 registers with
-// almost no spills; two with dither, whose second lattice search needs more; one with
-// the dense rotation, whose shared form (kRotSmemBytes) comes first.
+// almost no spills; two with dither, whose second lattice search needs more; with the
+// dense rotation one CTA of kRotDecodeWarps warps, whose shared form of Q^T and per-warp
+// rotation buffers (rot_smem_bytes) come first.
 // MIXED: the last symbol of each block has its own Rice parameter (a.k_last != a.k).
 template <int LAT, bool DITHER, bool KV, bool KSMALL, int MODE, bool ROT = false, bool MIXED = false>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : (DITHER ? 2 : 3)) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, ROT ? 1 : (DITHER ? 2 : 3))
+    decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int kStageSlot = kStageWords + kStagePad;
+    constexpr int W = ROT ? kRotDecodeWarps : kWarpsPerCta;
     const float *rot_s = ROT ? reinterpret_cast<const float *>(smem) : nullptr;
-    uint32_t *sign_tab = smem + (ROT ? kRotSmemBytes / sizeof(uint32_t) : 0);
+    uint32_t *sign_tab = smem + (ROT ? rot_smem_bytes(W) / sizeof(uint32_t) : 0);
     uint32_t *stage_all = sign_tab + a.tcols * kSignWords;
-    uint32_t *start_all = stage_all + kWarpsPerCta * 2 * kStageSlot;
+    uint32_t *start_all = stage_all + W * 2 * kStageSlot;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t *stages = stage_all + warp * 2 * kStageSlot;
     uint32_t *startbit = start_all + warp * 128;   // first unary bit of every 32-symbol segment
@@ -518,8 +522,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : (DITHER ? 2 : 3))
 
     const int k = a.k;
     uint32_t status = 0;
-    const unsigned long long nwarps = (unsigned long long)gridDim.x * kWarpsPerCta;
-    unsigned long long c = (unsigned long long)blockIdx.x * kWarpsPerCta + warp;
+    const unsigned long long nwarps = (unsigned long long)gridDim.x * W;
+    // the rotation decoder numbers chunks across CTAs first, so that a short read spreads
+    // over as many SMs as it has chunks
+    unsigned long long c = ROT ? (unsigned long long)warp * gridDim.x + blockIdx.x
+                               : (unsigned long long)blockIdx.x * W + warp;
     int buf = 0;
     ChunkWords cw = {0, 0, false};
     if (c < a.n_chunks) {

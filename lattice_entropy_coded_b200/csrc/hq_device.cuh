@@ -166,12 +166,15 @@ __device__ __forceinline__ void fwht128_sixteenth(float2 (&v)[4], int lane) {
 // g = lane >> 4; outputs 4j .. 4j + 3 and 64 + 4j .. 64 + 4j + 3 for j = lane & 15),
 // so that per input k a lane issues three 16-byte shared loads (4 inputs, 8 matrix
 // entries) for 32 fma.  The inputs reach that layout, and the results return to the
-// quarter layout, through a per-warp shared buffer.  Shared memory of a CTA of
-// kWarpsPerCta warps, 16-byte aligned, kRotSmemBytes: M as S[k][o] = M[o][k] (row k
-// over the 128 outputs, pitch kRotPitch), then one buffer of kRotBufFloats per warp.
+// quarter layout, through a per-warp shared buffer.  Shared memory of a CTA of W
+// warps, 16-byte aligned, rot_smem_bytes(W): M as S[k][o] = M[o][k] (row k over the
+// 128 outputs, pitch kRotPitch), then one buffer of kRotBufFloats per warp.
 constexpr int kRotPitch = 132;          // 16-byte rows; transposing writes at most 4-way bank conflicts
 constexpr int kRotBufFloats = 8 * 132;  // inputs k-major 8 k + t + 8 (k >> 5), or results 132 t + o
-constexpr size_t kRotSmemBytes = ((size_t)128 * kRotPitch + (size_t)kWarpsPerCta * kRotBufFloats) * sizeof(float);
+__host__ __device__ constexpr size_t rot_smem_bytes(int warps) {
+    return ((size_t)128 * kRotPitch + (size_t)warps * kRotBufFloats) * sizeof(float);
+}
+constexpr size_t kRotSmemBytes = rot_smem_bytes(kWarpsPerCta);
 
 // Shared form of M from the row-major fp32 Q in global memory (coalesced reads, by the
 // whole CTA): M = Q when FORWARD, else M = Q^T.  The caller synchronises.
@@ -206,7 +209,7 @@ __device__ __forceinline__ void rotate_round(float2 (&v)[16], const float *S, in
     for (int tt = 0; tt < 4; tt++)
 #pragma unroll
         for (int c = 0; c < 4; c++) acc[tt][c] = make_float2(0.0f, 0.0f);
-#pragma unroll 8
+#pragma unroll 4
     for (int k = 0; k < 128; k++) {
         const float4 z = *reinterpret_cast<const float4 *>(buf + 8 * k + 8 * (k >> 5) + 4 * g);
         const float4 m0 = *reinterpret_cast<const float4 *>(S + k * kRotPitch + 4 * j);

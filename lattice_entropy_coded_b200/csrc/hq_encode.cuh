@@ -809,18 +809,22 @@ __device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending 
 // publishes the chunk's word count; and one warp, in turn, resolves the previous
 // chunk's offset and copies that chunk's stage out.
 // ROT: the dense KV rotation instead of the sign diagonal and H_128, its shared form
-// (kRotSmemBytes) ahead of the rest; one CTA per SM (the shared memory).  The
-// rotation runs at the fp32 fma rate, so this form serves every launch size.
+// and per-warp rotation buffers (rot_smem_bytes) ahead of the rest; one CTA of
+// kRotGroups groups per SM (the shared memory).  The rotation runs at the fp32 fma
+// rate, so this form serves every launch size.
+constexpr int kRotGroups = 3;
 template <int LAT, bool DITHER, bool KSMALL, bool ROT, bool MIXED = false>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) encode_kernel_grouped(const EncodeArgs a) {
+__global__ void __launch_bounds__((ROT ? kRotGroups : kGroups) * kGroupWarps * 32, ROT ? 1 : 2)
+    encode_kernel_grouped(const EncodeArgs a) {
+    constexpr int G = ROT ? kRotGroups : kGroups;
     extern __shared__ __align__(16) uint32_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gi = warp / kGroupWarps, w = warp % kGroupWarps;
     float *rot_s = ROT ? reinterpret_cast<float *>(smem) : nullptr;
-    uint32_t *sign_tab = smem + (ROT ? kRotSmemBytes / sizeof(uint32_t) : 0);   // tcols * kSignWords
+    uint32_t *sign_tab = smem + (ROT ? rot_smem_bytes(G * kGroupWarps) / sizeof(uint32_t) : 0);   // tcols * kSignWords
     uint32_t *stage_all = sign_tab + a.tcols * kSignWords;                  // groups * 2 * kStageWords
-    GroupCtl *ctl_all = reinterpret_cast<GroupCtl *>(stage_all + kGroups * 2 * kStageWords);
-    uint32_t *in_all = reinterpret_cast<uint32_t *>(ctl_all + kGroups);    // warps * 32 * kGroupSlotWords
+    GroupCtl *ctl_all = reinterpret_cast<GroupCtl *>(stage_all + G * 2 * kStageWords);
+    uint32_t *in_all = reinterpret_cast<uint32_t *>(ctl_all + G);    // warps * 32 * kGroupSlotWords
     uint32_t *stages = stage_all + gi * 2 * kStageWords;
     GroupCtl &ctl = ctl_all[gi];
     uint32_t *slot = in_all + (warp * 32 + lane) * kGroupSlotWords;
@@ -829,7 +833,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) encode_kernel_
         load_rotation<true>(rot_s, a.rot);
     else
         build_sign_table(sign_tab, a.tcols, a.seed);
-    for (int i = threadIdx.x; i < kGroups * 2 * kStageWords / 4; i += blockDim.x)
+    for (int i = threadIdx.x; i < G * 2 * kStageWords / 4; i += blockDim.x)
         reinterpret_cast<uint4 *>(stage_all)[i] = make_uint4(0, 0, 0, 0);
     if (w == 0 && lane == 0) {
         ctl.first[0] = atomicAdd(a.ticket, 1u);

@@ -12,22 +12,22 @@ namespace hq {
 
 namespace {
 
-// One CTA of 8 warps per SM: the rotation's shared form (kRotSmemBytes) comes on
-// top of the two stages per warp.
+// One CTA of kRotDecodeWarps warps per SM: the rotation's shared form of Q^T and the
+// per-warp rotation buffers come on top of two stages per warp (223 KB at 12 warps).
 template <int LAT, bool DITHER, int MODE>
 cudaError_t launch_rot_t(const DecodeArgs &a, cudaStream_t s) {
-    const size_t smem = kRotSmemBytes + (size_t)(a.tcols * kSignWords + kWarpsPerCta * 2 * (kStageWords + kStagePad) +
-                                                 kWarpsPerCta * 128) *
-                                            sizeof(uint32_t);
+    constexpr int W = kRotDecodeWarps;
+    const size_t smem = rot_smem_bytes(W) + (size_t)(a.tcols * kSignWords + W * 2 * (kStageWords + kStagePad) + W * 128) *
+                                                sizeof(uint32_t);
     const bool small = a.k <= 4, mixed = a.k_last != a.k;
     auto kern = mixed ? decode_kernel<LAT, DITHER, true, false, MODE, true, true>
                 : small ? decode_kernel<LAT, DITHER, true, true, MODE, true> : decode_kernel<LAT, DITHER, true, false, MODE, true>;
     static LaunchPlan plans[3];
     unsigned grid = 0;
-    cudaError_t e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem,
-                                                           (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid);
+    // one CTA per chunk up to one per SM; the kernel numbers chunks across CTAs first
+    cudaError_t e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, W * 32, smem, a.n_chunks, grid);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
+    kern<<<grid, W * 32, smem, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -10,23 +10,25 @@ namespace hq {
 
 namespace {
 
-// Every launch size takes the grouped form: four warps per chunk, one CTA of two
-// groups per SM (the rotation's 66 KB shared form).
+// Every launch size takes the grouped form: four warps per chunk, one CTA of
+// kRotGroups groups per SM (the rotation's shared form and per-warp buffers, 194 KB).
 template <int LAT, bool DITHER>
 cudaError_t launch_rot_t(const EncodeArgs &a, cudaStream_t s) {
     const bool small = a.k <= 4, mixed = a.k_last != a.k;
-    const size_t smem = kRotSmemBytes +
-                        (size_t)(a.tcols * kSignWords + kGroups * 2 * kStageWords + kWarpsPerCta * 32 * kGroupSlotWords) *
+    constexpr int W = kRotGroups * kGroupWarps;
+    const size_t smem = rot_smem_bytes(W) +
+                        (size_t)(a.tcols * kSignWords + kRotGroups * 2 * kStageWords + W * 32 * kGroupSlotWords) *
                             sizeof(uint32_t) +
-                        kGroups * sizeof(GroupCtl);
+                        kRotGroups * sizeof(GroupCtl);
     auto kern = mixed ? encode_kernel_grouped<LAT, DITHER, false, true, true>
                 : small ? encode_kernel_grouped<LAT, DITHER, true, true> : encode_kernel_grouped<LAT, DITHER, false, true>;
     static LaunchPlan plans[3];
     unsigned grid = 0;
-    cudaError_t e =
-        plans[mixed ? 2 : small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kGroups - 1) / kGroups, grid);
+    // one CTA per chunk up to one per SM: a short append spreads over as many SMs as it
+    // has chunks (the rotation is bound by each SM's fma rate), idle groups exit at once
+    cudaError_t e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, W * 32, smem, a.n_chunks, grid);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
+    kern<<<grid, W * 32, smem, s>>>(a);
     return cudaGetLastError();
 }
 
