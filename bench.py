@@ -606,6 +606,28 @@ def run_bulk(args):
                     pre_ms.append(p0.elapsed_time(p1))
             pre_words = int(pre.tail[1].item())
             del pre
+            # decode steps: 128 appends of one token each (8 one-tile chunks per launch), captured
+            # once in a CUDA graph and replayed; the time per append is the per-token latency
+            one = hq.KVCache(H, 128, params, bits_per_scalar=p["bps"] + 8.0, max_appends=129, max_append_tokens=1,
+                             device=device, rotation=rot)
+            toks = [src[:, t:t + 1] for t in range(128)]
+            hq.hq_kv_init(one.cache, H, 128, params, one.words, one.offsets, one.table, one.tail, one.stats)
+            g1 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g1):
+                for tk in toks:
+                    one.append(tk, p["alpha"])
+            one_ms = []
+            for it in range(args.warmup + args.steps):
+                hq.hq_kv_init(one.cache, H, 128, params, one.words, one.offsets, one.table, one.tail, one.stats)
+                o0, o1 = _events()
+                o0.record()
+                g1.replay()
+                o1.record()
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    one_ms.append(o0.elapsed_time(o1))
+            one_status = hq.read_stats(one.stats)["status"]
+            del g1, one
             mse = float(((outb.double() - src.double()) ** 2).mean())
             am, rm = float(np.median(app_ms)), float(np.median(read_ms))
             alg = 2.0 * n + 4.0 * words + 8.0 * (cache.cache.chunks + 1)
@@ -619,6 +641,7 @@ def run_bulk(args):
                             prefill_append_ms=float(np.median(pre_ms)),
                             prefill_append_gbs=2.0 * n / (float(np.median(pre_ms)) * 1e6),
                             prefill_stream_words=pre_words,
+                            token_append_us=float(np.median(one_ms)) * 1e3 / 128, token_append_status=one_status,
                             # with a dense rotation: the rotation's 128 fp32 fma per element (forward
                             # in the append, inverse in the read) against the fp32 fma peak of
                             # 148 SMs x 128 lanes at the 1965 MHz maximum clock

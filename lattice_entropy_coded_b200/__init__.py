@@ -251,7 +251,7 @@ def hq_haar_rotation(seed: int, out: torch.Tensor | None = None, cuda_stream=Non
 
 
 def hq_debug_set_encode_path(path: int) -> int:
-    """0 = by size, 1 = per-warp, 2 = grouped, 3 = wide encoder (testing aid)."""
+    """0 = by size, 1 = per-warp, 2 = grouped, 3 = wide, 4 = single-CTA encoder (testing aid)."""
     return _check(_lib.hq_debug_set_encode_path(int(path)), "hq_debug_set_encode_path")
 
 

@@ -139,9 +139,8 @@ int hq_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_
     if (!x || !aligned(x, 16) || ld < cols || ld % 8) return HQ_EINVAL;
     if (!d_stream || !aligned(d_stream, 4)) return HQ_EINVAL;
     if (!workspace || !aligned(workspace, 8) || ws_bytes < ws_bytes_for(nch)) return HQ_EINVAL;
-    // one memset clears the look-back words, the ticket, the done counter and the stats
-    // accumulator; the kernel's last CTA writes *d_stats
-    if (cudaMemsetAsync(workspace, 0, encode_scratch_bytes(nch), s) != cudaSuccess) return HQ_ECUDA;
+    // the launcher clears the workspace (look-back words, ticket, done counter, stats
+    // accumulator) when the form it picks uses it; the kernel writes *d_stats
 
     EncodeArgs a;
     memset(&a, 0, sizeof(a));
@@ -299,8 +298,6 @@ int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t ld_token
     if (cache->chunks + nch + 1 > cache->offsets_cap || cache->appends + 1 > cache->table_cap) return HQ_EINVAL;
     if (!workspace || !aligned(workspace, 8) || ws_bytes < ws_bytes_for(nch)) return HQ_EINVAL;
     cudaStream_t s = (cudaStream_t)cuda_stream;
-    if (cudaMemsetAsync(workspace, 0, encode_scratch_bytes(nch), s) != cudaSuccess) return HQ_ECUDA;
-
     EncodeArgs a;
     memset(&a, 0, sizeof(a));
     a.x = (const uint16_t *)kv;
@@ -604,7 +601,7 @@ int hq_haar_rotation(uint64_t seed, float *d_q, void *cuda_stream) {
 void hq_debug_set_spin_limit(uint32_t polls) { g_spin_limit = polls ? polls : kSpinLimit; }
 
 int hq_debug_set_encode_path(int path) {
-    if (path < 0 || path > 3) return HQ_EINVAL;
+    if (path < 0 || path > 4) return HQ_EINVAL;
     hq::g_encode_path = path;
     return HQ_OK;
 }

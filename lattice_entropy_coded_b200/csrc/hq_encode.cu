@@ -8,17 +8,40 @@ namespace hq {
 namespace {
 
 template <int LAT, bool DITHER>
+cudaError_t launch_tiny_t(const EncodeArgs &a, cudaStream_t s, bool small, bool mixed) {
+    const size_t smem = (size_t)(a.tcols * kSignWords + kTinyMaxChunks * kStageWords) * sizeof(uint32_t) +
+                        kTinyMaxChunks * (sizeof(TinyChunk) + sizeof(unsigned long long));
+    auto kern = mixed ? encode_kernel_tiny<LAT, DITHER, false, false, true>
+                : small ? encode_kernel_tiny<LAT, DITHER, true, false, false>
+                        : encode_kernel_tiny<LAT, DITHER, false, false, false>;
+    static LaunchPlan plans[3];
+    unsigned grid = 0;
+    cudaError_t e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, kTinyWarps * 32, smem, 1, grid);
+    if (e != cudaSuccess) return e;
+    kern<<<1, kTinyWarps * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int LAT, bool DITHER>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     const bool small = a.k <= 4;
     const bool mixed = a.k_last != a.k;   // a second Rice parameter: per-warp or grouped forms only
     cudaError_t e;
     unsigned grid = 0;
-    // by size: the wide form while every chunk gets a 16-warp group of its own in one
-    // wave (148 SMs x 2 CTAs on a B200), the grouped form while it gets a 4-warp group
-    // (148 x 2 x kGroups), else the per-warp form
+    // by size: one CTA for the whole launch up to kTinyMaxChunks chunks; the wide form
+    // while every chunk gets a 16-warp group of its own in one wave (148 SMs x 2 CTAs on
+    // a B200), the grouped form while it gets a 4-warp group (148 x 2 x kGroups), else
+    // the per-warp form
     int mode = g_encode_path;
-    if (mode == 0) mode = (a.n_chunks <= 296ull) ? 3 : (a.n_chunks <= 592ull) ? 2 : 1;
+    if (mode == 0)
+        mode = (a.n_chunks <= (unsigned long long)kTinyMaxChunks) ? 4
+               : (a.n_chunks <= 296ull) ? 3 : (a.n_chunks <= 592ull) ? 2 : 1;
+    if (mode == 4 && a.n_chunks > (unsigned long long)kTinyMaxChunks) mode = 1;
     if (mixed && mode == 3) mode = 2;
+    if (mode == 4) return launch_tiny_t<LAT, DITHER>(a, s, small, mixed);
+    // the multi-CTA forms share the workspace: look-back words, ticket, done counter and
+    // stats accumulator, cleared by one memset
+    if ((e = cudaMemsetAsync(a.lookback, 0, encode_scratch_bytes(a.n_chunks), s)) != cudaSuccess) return e;
     if (mode == 3) {
         const size_t smem =
             (size_t)(a.tcols * kSignWords + 2 * kStageWords) * sizeof(uint32_t) + sizeof(WideCtl);

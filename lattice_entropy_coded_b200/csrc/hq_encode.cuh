@@ -1212,6 +1212,195 @@ __global__ void __launch_bounds__(kWideWarps * 32, 1) encode_kernel_wide(const E
     stats_finish_cta(a);
 }
 
+// ------------------------------------------------------------------ single-CTA form
+// For launches of a few chunks (a KV append of a few tokens: one chunk per head), the
+// multi-CTA machinery costs more than the work: the ticket, the look-back across CTAs,
+// the done counter and the workspace clearing before the launch.  Here one CTA of
+// kTinyWarps warps does it all: warp w encodes chunks w, w + kTinyWarps, ... each into
+// its own stage (the per-warp form's rounds, inputs read straight from global memory);
+// one warp scans the chunk sizes into offsets; the warps copy their stages out (or
+// set an oversize chunk's bits in place).  No workspace is read or written.
+constexpr int kTinyWarps = 8;
+constexpr int kTinyMaxChunks = 32;      // stages in shared memory: 128 KB
+constexpr int kTinyMaxChunksRot = 16;   // with the dense rotation's 99 KB: 64 KB of stages
+
+struct TinyChunk {
+    uint32_t total;      // words of the chunk
+    uint32_t status;     // HQ_ST_RANGE
+    uint32_t overflow;   // larger than its stage: set in place after the scan
+    uint32_t zor;
+    unsigned long long payload;
+};
+
+template <int LAT, bool DITHER, bool KSMALL, bool ROT, bool MIXED>
+__global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tiny(const EncodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    constexpr int N = Lattice<LAT>::N;
+    constexpr int kMax = ROT ? kTinyMaxChunksRot : kTinyMaxChunks;
+    float *rot_s = ROT ? reinterpret_cast<float *>(smem) : nullptr;
+    uint32_t *sign_tab = smem + (ROT ? kRotSmemBytes / sizeof(uint32_t) : 0);   // tcols * kSignWords
+    uint32_t *stage_all = sign_tab + a.tcols * kSignWords;                         // kMax * kStageWords
+    TinyChunk *info = reinterpret_cast<TinyChunk *>(stage_all + kMax * kStageWords);
+    unsigned long long *start = reinterpret_cast<unsigned long long *>(info + kMax);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = (int)a.n_chunks;   // <= kMax (host)
+
+    if (ROT)
+        load_rotation<true>(rot_s, a.rot);
+    else
+        build_sign_table(sign_tab, a.tcols, a.seed);
+    for (int i = threadIdx.x; i < n * kStageWords / 4; i += blockDim.x)
+        reinterpret_cast<uint4 *>(stage_all)[i] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+
+    const int k = a.k, kl = a.k_last;
+    const uint32_t lane_bits = 4u * group_rem_bits<N>(k, kl);
+    for (int c = warp; c < n; c += kTinyWarps) {
+        ChunkGeo geo;
+        geo.init(a.map, (unsigned long long)c);
+        uint32_t *stage = stage_all + c * kStageWords;
+        const int ntiles = geo.ntiles;
+        const int nrounds = (ntiles + kTilesPerRound - 1) / kTilesPerRound;
+        const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
+        const uint32_t rbits = (uint32_t)ntiles * tile_rem_bits<N>(k, kl);
+        const uint32_t nr = (rbits + 31u) >> 5;
+        uint32_t urun = 0, zor = 0;
+        bool overflow = (nc + nr) > (uint32_t)kStageWords, range_bad = false;
+#pragma unroll 1
+        for (int r = 0; r < nrounds; r++) {
+            RoundInput in;
+            round_input(a, geo, r, lane, in);
+            uint4 raw[4];
+            {
+                const uint16_t *src = nullptr;
+                int tc;
+                unsigned long long e;
+                geo.tile(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, tc, e);
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    raw[j] = in.valid ? ldg_nc_v4(src + 32 * (lane & 3) + 8 * j) : make_uint4(0, 0, 0, 0);
+            }
+            uint32_t z[32], cbits;
+            round_symbols<LAT, DITHER, ROT>(a, in, raw, lane, sign_tab, z, cbits, rot_s);
+            const bool valid = in.valid;
+            uint32_t usum = 0, lor = 0;
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                usum += z[i] >> sym_k<N>(i, k, kl);
+                lor |= z[i];
+            }
+            zor |= lor;
+            const uint32_t ub = valid ? usum + 32u : 0u;
+            uint32_t incl = ub;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const uint32_t rtot = __shfl_sync(0xffffffffu, incl, 31);
+            const uint32_t rzor = __reduce_or_sync(0xffffffffu, lor);
+            if ((rzor >> 22) != 0u || (unsigned long long)urun + rtot >= kMaxUnaryBits) range_bad = true;
+            if (!overflow && nc + nr + (uint32_t)(((unsigned long long)urun + rtot + 31) >> 5) > (uint32_t)kStageWords)
+                overflow = true;
+            if (!overflow && !range_bad) {
+                if (MIXED) {
+                    if (valid) put_rem_mixed<N>(stage + nc, (uint32_t)(32 * r + lane) * lane_bits, z, k, kl);
+                } else {
+                    put_rem<KSMALL>(stage + nc + (uint32_t)(32 * r + lane) * (uint32_t)k, z, k, valid);
+                }
+                if (valid) {
+                    if (LAT == HQ_E8 && cbits) atomicOr(stage + 4 * r + (lane >> 3), cbits << (4 * (lane & 7)));
+                    uint32_t *un = stage + nc + nr;
+                    uint32_t pos = urun + incl - ub;
+#pragma unroll
+                    for (int g = 0; g < 4; g++) {
+                        uint32_t qg[8];
+#pragma unroll
+                        for (int i = 0; i < 8; i++) qg[i] = z[8 * g + i] >> sym_k<N>(i, k, kl);
+                        pos += unary_group_shared(un, pos, qg);
+                    }
+                }
+            }
+            urun += rtot;
+        }
+        zor = __reduce_or_sync(0xffffffffu, zor);
+        if (lane == 0) {
+            TinyChunk t;
+            t.total = nc + nr + (uint32_t)(((unsigned long long)urun + 31) / 32);
+            t.status = range_bad ? HQ_ST_RANGE : 0u;
+            t.overflow = overflow ? 1u : 0u;
+            t.zor = zor;
+            t.payload = urun + (unsigned long long)rbits + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
+            info[c] = t;
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+
+    // offsets: one warp scans the chunk sizes (at most 32); the same warp writes the
+    // offsets, the tail, the append row and the stats
+    if (warp == 0) {
+        const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
+        const TinyChunk t = lane < n ? info[lane] : TinyChunk{0u, 0u, 0u, 0u, 0ull};
+        unsigned long long incl = t.total;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        const unsigned long long st = base + incl - t.total;
+        if (lane < n) {
+            start[lane] = st;
+            a.offsets[a.chunk_base + lane] = st;
+        }
+        const unsigned long long end = base + __shfl_sync(0xffffffffu, incl, 31);
+        const uint32_t status = __reduce_or_sync(0xffffffffu, t.status) | (end > a.cap_words ? HQ_ST_CAPACITY : 0u);
+        const uint32_t zor = __reduce_or_sync(0xffffffffu, t.zor);
+        const unsigned long long payload = warp_sum_u64(t.payload);
+        if (lane == 0) {
+            a.offsets[a.chunk_base + n] = end;
+            if (a.tail_out) *a.tail_out = end;
+            if (a.row) *a.row = a.row_val;
+            if (a.stats) {
+                if (a.stats_add) {
+                    if (status) atomicOr(&a.stats->status, status);
+                    if (zor) atomicOr(&a.stats->max_symbol, zor);
+                    if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
+                } else {
+                    a.stats->status = status;
+                    a.stats->max_symbol = zor;
+                    a.stats->payload_bits = payload;
+                }
+                a.stats->stream_words = end;
+            }
+        }
+    }
+    __syncthreads();
+
+    for (int c = warp; c < n; c += kTinyWarps) {
+        const TinyChunk t = info[c];
+        const unsigned long long st = start[c];
+        if (t.status) continue;   // outside the supported range: nothing written
+        if (!t.overflow) {
+            const uint32_t *stage = stage_all + c * kStageWords;
+            for (uint32_t i = lane; i < t.total; i += 32)
+                if (st + i < a.cap_words) a.stream[st + i] = stage[i];
+        } else {
+            uint32_t *g = a.stream + st;
+            const unsigned long long room = (st < a.cap_words) ? a.cap_words - st : 0ull;
+            for (unsigned long long i = lane; i < t.total; i += 32)
+                if (i < room) g[i] = 0u;
+            __syncwarp();
+            __threadfence_block();
+            ChunkGeo geo;
+            geo.init(a.map, (unsigned long long)c);
+            const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * geo.ntiles + 31) / 32u : 0u;
+            const uint32_t nr = ((uint32_t)geo.ntiles * tile_rem_bits<N>(a.k, a.k_last) + 31u) >> 5;
+            encode_chunk_global<LAT, DITHER, ROT>(a, geo, sign_tab, rot_s, g, room, nc, nr);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ rate only
 // The quantize path up to the Rice code lengths, without a stream: per chunk the
 // unary bits U, so payload = U + remainder bits + coset bits and the chunk's words

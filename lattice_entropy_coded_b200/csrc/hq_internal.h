@@ -135,10 +135,11 @@ struct LaunchPlan {
     }
 };
 
-// Encoder form: 0 = by size (wide, then grouped, for launches of at most one wave
-// of their chunk groups, per-warp otherwise), 1 = per-warp, 2 = grouped (4 warps
-// per chunk), 3 = wide (16 warps per chunk, 16 lanes per tile).  Set by
-// hq_debug_set_encode_path (hq_api.cu); all forms give identical streams.
+// Encoder form: 0 = by size (one CTA for a few chunks, then wide, then grouped, for
+// launches of at most one wave of their chunk groups, per-warp otherwise), 1 =
+// per-warp, 2 = grouped (4 warps per chunk), 3 = wide (16 warps per chunk, 16 lanes
+// per tile), 4 = one CTA.  Set by hq_debug_set_encode_path (hq_api.cu); all forms
+// give identical streams.
 extern int g_encode_path;
 
 // Launchers (defined in hq_encode.cu / hq_decode.cu).  Return cudaSuccess or the launch error.

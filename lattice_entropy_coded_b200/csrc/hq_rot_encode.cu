@@ -10,11 +10,28 @@ namespace hq {
 
 namespace {
 
-// Every launch size takes the grouped form: four warps per chunk, one CTA of
-// kRotGroups groups per SM (the rotation's shared form and per-warp buffers, 194 KB).
+// Up to kTinyMaxChunksRot chunks: one CTA for the whole launch.  Beyond: the grouped
+// form, four warps per chunk, one CTA of kRotGroups groups per SM (the rotation's shared
+// form and per-warp buffers, 194 KB).
 template <int LAT, bool DITHER>
 cudaError_t launch_rot_t(const EncodeArgs &a, cudaStream_t s) {
     const bool small = a.k <= 4, mixed = a.k_last != a.k;
+    if (a.n_chunks <= (unsigned long long)kTinyMaxChunksRot && (g_encode_path == 0 || g_encode_path == 4)) {
+        const size_t smem = kRotSmemBytes + (size_t)(a.tcols * kSignWords + kTinyMaxChunksRot * kStageWords) *
+                                                sizeof(uint32_t) +
+                            kTinyMaxChunksRot * (sizeof(TinyChunk) + sizeof(unsigned long long));
+        auto kern = mixed ? encode_kernel_tiny<LAT, DITHER, false, true, true>
+                    : small ? encode_kernel_tiny<LAT, DITHER, true, true, false>
+                            : encode_kernel_tiny<LAT, DITHER, false, true, false>;
+        static LaunchPlan tplans[3];
+        unsigned tgrid = 0;
+        cudaError_t e = tplans[mixed ? 2 : small ? 1 : 0].grid(kern, kTinyWarps * 32, smem, 1, tgrid);
+        if (e != cudaSuccess) return e;
+        kern<<<1, kTinyWarps * 32, smem, s>>>(a);
+        return cudaGetLastError();
+    }
+    cudaError_t me = cudaMemsetAsync(a.lookback, 0, encode_scratch_bytes(a.n_chunks), s);
+    if (me != cudaSuccess) return me;
     constexpr int W = kRotGroups * kGroupWarps;
     const size_t smem = rot_smem_bytes(W) +
                         (size_t)(a.tcols * kSignWords + kRotGroups * 2 * kStageWords + W * 32 * kGroupSlotWords) *

@@ -75,7 +75,6 @@ int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, co
     if (!d_stream || !aligned(d_stream, 4)) return HQ_EINVAL;
     // the previous call's look-back words, ticket, counter and stats are still there:
     // clear what this call uses
-    if (cudaMemsetAsync(scratch, 0, encode_scratch_bytes(nch), s) != cudaSuccess) return HQ_ECUDA;
 
     EncodeArgs a;
     memset(&a, 0, sizeof(a));

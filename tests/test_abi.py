@@ -127,7 +127,8 @@ def test_entry_points_validate_before_touching_the_device():
     assert lib.hq_calibrate(C.c_void_p(256), 0, 128, 128, C.byref(p), C.byref(good), st, None,
                             C.byref(res)) == hq.HQ_EINVAL                                   # empty
     # testing aids: encoder form switch and the nearest-point entry point
-    assert lib.hq_debug_set_encode_path(4) == hq.HQ_EINVAL
+    assert lib.hq_debug_set_encode_path(5) == hq.HQ_EINVAL
+    assert lib.hq_debug_set_encode_path(4) == hq.HQ_OK
     assert lib.hq_debug_set_encode_path(-1) == hq.HQ_EINVAL
     assert lib.hq_debug_set_encode_path(0) == hq.HQ_OK
     assert lib.hq_debug_nearest(4, None, 1, None, None) == hq.HQ_EINVAL

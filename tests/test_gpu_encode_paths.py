@@ -1,8 +1,10 @@
-"""Both forms of the quantize kernel against the oracle.
+"""Every form of the quantize kernel against the oracle.
 
 The encoder has a per-warp form (a warp encodes whole chunks; used for large
-launches) and a grouped form (four warps share a chunk; used for launches of at
-most one wave of groups, such as a KV append).  By default the size decides;
+launches), a grouped form (four warps share a chunk), a wide form (sixteen warps
+share a chunk) and a single-CTA form (one CTA for a launch of at most 32 chunks,
+such as a KV append of a few tokens; forced on a larger launch, the per-warp form
+runs).  By default the size decides;
 here each form is forced in turn on the cases that exercise its control flow:
 ragged last chunks, every Rice parameter, strided rows, exact ties, chunks too
 large for the shared stage, capacity overflow, bounded look-back waits, KV
@@ -19,7 +21,7 @@ from hqtest import assert_same_words, gpu_quantize, oracle_quantize, rate_points
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=[1, 2, 3], ids=["per_warp", "grouped", "wide"])
+@pytest.fixture(params=[1, 2, 3, 4], ids=["per_warp", "grouped", "wide", "single_cta"])
 def path(request):
     import lattice_entropy_coded_b200 as hq
     hq.hq_debug_set_encode_path(request.param)
