@@ -75,7 +75,7 @@ enum hq_lattice { HQ_Z = 0, HQ_A2 = 1, HQ_D4 = 2, HQ_E8 = 3 };
 /* Synchronous return codes. */
 #define HQ_OK 0
 #define HQ_EINVAL (-1)       /* bad argument: null pointer, size, stride, alignment, parameter */
-#define HQ_EUNSUPPORTED (-2) /* valid request outside what this build supports (tile != 128, ...) */
+#define HQ_EUNSUPPORTED (-2) /* valid request outside what this library supports (tile != 128, ...) */
 #define HQ_ECUDA (-3)        /* a CUDA launch or runtime call failed */
 
 /* Device-side status bits (hq_stats.status). */
@@ -88,7 +88,7 @@ enum hq_lattice { HQ_Z = 0, HQ_A2 = 1, HQ_D4 = 2, HQ_E8 = 3 };
                                codes of that call are outside the supported range and unspecified */
 
 /* Parameters of one call (page sections 1-4).  tile and chunk_tiles are
- * fixed by this build; the others select the operating point. */
+ * fixed in this library; the others select the operating point. */
 typedef struct hq_params {
     int32_t tile;        /* elements per RHT tile; must be 128 */
     int32_t lattice;     /* enum hq_lattice */

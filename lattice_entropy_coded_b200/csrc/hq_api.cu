@@ -572,7 +572,7 @@ const char *hq_status_string(int code) {
     switch (code) {
     case HQ_OK: return "ok";
     case HQ_EINVAL: return "invalid argument";
-    case HQ_EUNSUPPORTED: return "unsupported by this build";
+    case HQ_EUNSUPPORTED: return "unsupported by this library";
     case HQ_ECUDA: return "CUDA error";
     }
     if (code > 0) {
