@@ -501,7 +501,7 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
 // rotation buffers (rot_smem_bytes) come first.
 // MIXED: the last symbol of each block has its own Rice parameter (a.k_last != a.k).
 template <int LAT, bool DITHER, bool KV, bool KSMALL, int MODE, bool ROT = false, bool MIXED = false>
-__global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, ROT ? 1 : (DITHER ? 2 : 3))
+__global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, ROT ? 1 : ((DITHER || MIXED) ? 2 : 3))
     decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int kStageSlot = kStageWords + kStagePad;
