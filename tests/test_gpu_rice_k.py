@@ -93,9 +93,12 @@ def test_two_k_large_symbols_slow_path():
 
 
 @pytest.mark.parametrize("rot", [False, True])
-def test_two_k_kv_cache(rot):
+@pytest.mark.parametrize("H", [3, 8])
+def test_two_k_kv_cache(rot, H):
+    """3 heads: every append fits the single-CTA form; 8 heads: the 100- and 155-token
+    appends (32 and 40 chunks) take the multi-CTA forms."""
     hq = _hq()
-    H, Ts = 3, [100, 1, 155]
+    Ts = [100, 1, 155]
     total = sum(Ts)
     K, _ = synth.kv(H, total, seed=23)
     Q = R.haar_rotation(41) if rot else None

@@ -102,11 +102,13 @@ def test_rotated_kv_appends_and_reads_bit_exact(lat, dither):
 
 
 @pytest.mark.parametrize("k", [0, 3, 6])
-def test_rotated_kv_rice_parameters(k):
+@pytest.mark.parametrize("Ts", [[300], [40, 1]])
+def test_rotated_kv_rice_parameters(k, Ts):
+    """k <= 4 and k > 4, in the grouped form (20 chunks) and the single-CTA form (4 and 2)."""
     Q = R.haar_rotation(32)
     _, V = synth.kv(2, 300, seed=5)
     alpha = {0: 0.3, 3: 2.5, 6: 20.0}[k]
-    _rot_cache_case(2, [300], O.E8, alpha, k, 8, 1, V, Q)
+    _rot_cache_case(2, Ts, O.E8, alpha, k, 8, 1, V, Q)
 
 
 def test_rotated_kv_same_stream_whatever_the_encoder_switch():
