@@ -3,7 +3,7 @@
 // subtractive dither, nearest lattice point, bit-stripping, zigzag, Rice planes;
 // and the rate-only pass that counts the same codes without writing them.
 //
-// Three forms with identical output, chosen by launch size (hq_encode.cu):
+// Four forms with identical output, chosen by launch size (hq_encode.cu):
 //  * per-warp (throughput; more than 592 chunks): one warp encodes one chunk
 //    (32 tiles) in 4 rounds of 8 tiles; four lanes share a tile, 32 elements
 //    each, loaded as 64 contiguous bytes per lane with cp.async one round ahead;
@@ -14,15 +14,21 @@
 //  * grouped (latency; up to 592 chunks): four warps share a chunk, one round
 //    each, meeting at a named barrier per chunk;
 //  * wide (lowest latency; up to 296 chunks): sixteen warps share a chunk,
-//    sixteen lanes per tile, one 8-element block per lane.
-// In every form a persistent grid takes chunk tickets from a global counter, so
-// a chunk's predecessors are always already running, and a single-pass
-// decoupled look-back over 64-bit (flag, value) words gives each chunk's word
-// offset (bounded waits: HQ_ST_TIMEOUT).  A chunk publishes its size as soon as
-// it is encoded and resolves its offset one chunk later, when its predecessors
-// have normally published; its stage is then copied out coalesced.  A chunk
-// larger than the stage is re-encoded by a path that sets its bits in place in
-// global memory (the same bits; only for extreme codes).
+//    sixteen lanes per tile, one 8-element block per lane;
+//  * single CTA (up to 32 chunks, such as a KV append of a few tokens): the
+//    CTA's warps encode the chunks into their own stages and one warp scans
+//    the sizes into offsets, with no workspace, ticket or look-back.
+// In the first three a persistent grid takes chunk tickets from a global
+// counter, so a chunk's predecessors are always already running, and a
+// single-pass decoupled look-back over 64-bit (flag, value) words gives each
+// chunk's word offset (bounded waits: HQ_ST_TIMEOUT).  A chunk publishes its
+// size as soon as it is encoded and resolves its offset one chunk later, when
+// its predecessors have normally published; its stage is then copied out
+// coalesced.  A chunk larger than the stage is re-encoded by a path that sets
+// its bits in place in global memory (the same bits; only for extreme codes).
+// Options: the dense KV rotation in place of the sign diagonal and H_128 (ROT;
+// grouped and single-CTA forms), a second Rice parameter for the last symbol of
+// each lattice block (MIXED; all forms but the wide one).
 #pragma once
 
 #include <cuda_runtime.h>
