@@ -162,3 +162,22 @@ def test_two_k_calibration():
     assert res["k"] >= 1 and abs(res["bps"] - 4.0) <= 0.002
     _, _, pay = oracle_quantize(x, O.E8, res["alpha"], res["k"], 9, dk_last=1)
     assert pay / x.numel() == res["bps"]
+
+
+def test_two_k_static_entry_point():
+    """hq_quantize_static (no workspace) gives hq_quantize's stream in this mode too, in the
+    single-CTA form (16 chunks) and in the multi-CTA forms (64 chunks)."""
+    hq = _hq()
+    for rows in (64, 256):
+        x = synth.weight(rows, 1024, seed=26).cuda()
+        p = hq.make_params("A2", ALPHA["A2"], 3, 4, 0, dk_last=2)
+        ref = gpu_quantize(x, p)
+        bound, nch = hq.hq_stream_bound(rows, 1024, p)
+        words = torch.empty(bound, dtype=torch.int32, device="cuda")
+        offs = torch.empty(nch + 1, dtype=torch.int64, device="cuda")
+        st = hq.stats_tensor()
+        hq.hq_quantize_static(x, p, words, offs, st)
+        torch.cuda.synchronize()
+        assert hq.read_stats(st) == ref["stats"]
+        assert np.array_equal(offs.cpu().numpy().view(np.uint64), ref["offsets"])
+        assert np.array_equal(words[:ref["total"]].cpu().numpy().view(np.uint32), ref["words"])
