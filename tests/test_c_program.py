@@ -1,6 +1,8 @@
-"""libhq.so from a C program: tests/c/hq_roundtrip.c includes include/hq.h and the
-CUDA runtime only.  It compiles and links here (no GPU needed); on a GPU its
-stream, offsets, bf16 reconstruction and fused GEMV are compared with the oracle."""
+"""libhq.so from C programs that include include/hq.h and the CUDA runtime only:
+tests/c/hq_roundtrip.c (a weight matrix: quantize, rate, dequantize, fused GEMV) and
+tests/c/hq_kv_roundtrip.c (a KV cache with a dense rotation, dither and a second Rice
+parameter, and the library's Haar draw).  They compile and link here (no GPU needed);
+on a GPU their outputs are compared with the oracle."""
 import json
 import os
 import subprocess
@@ -11,25 +13,27 @@ import torch
 
 import oracle as O
 import synth
-from hqtest import oracle_dequantize, oracle_quantize, u16
+from hqtest import assert_recon_equal, oracle_dequantize, oracle_quantize, u16
+from oracle import rotation as R
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PKG = os.path.join(ROOT, "lattice_entropy_coded_b200")
 CUDA = "/usr/local/cuda"
 
 
-def _compile(out_dir) -> str:
-    exe = os.path.join(str(out_dir), "hq_roundtrip")
+def _compile(out_dir, name="hq_roundtrip") -> str:
+    exe = os.path.join(str(out_dir), name)
     cmd = ["gcc", "-std=c99", "-O2", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
-           "-I", os.path.join(CUDA, "include"), os.path.join(ROOT, "tests", "c", "hq_roundtrip.c"),
+           "-I", os.path.join(CUDA, "include"), os.path.join(ROOT, "tests", "c", name + ".c"),
            "-L", PKG, "-lhq", "-L", os.path.join(CUDA, "lib64"), "-lcudart", f"-Wl,-rpath,{PKG}", "-o", exe]
     r = subprocess.run(cmd, capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     return exe
 
 
-def test_c_program_compiles_and_links(tmp_path):
-    exe = _compile(tmp_path)
+@pytest.mark.parametrize("name", ["hq_roundtrip", "hq_kv_roundtrip"])
+def test_c_program_compiles_and_links(tmp_path, name):
+    exe = _compile(tmp_path, name)
     r = subprocess.run([exe], capture_output=True, text=True)
     assert r.returncode == 1 and "usage" in r.stderr      # runs (library resolved), prints usage
 
@@ -58,3 +62,37 @@ def test_c_program_matches_the_oracle(tmp_path):
     y = np.fromfile(prefix + "y.bin", np.float32).astype(np.float64)
     lim = (40 + cols // 128) * 2.0 ** -24 * (np.abs(w) @ np.abs(x)) + 1e-30
     assert np.all(np.abs(y - w @ x) <= lim)
+
+
+@pytest.mark.gpu
+def test_c_kv_program_matches_the_oracle(tmp_path):
+    exe = _compile(tmp_path, "hq_kv_roundtrip")
+    H, t1, t2, alpha, k, dk, seed = 3, 70, 45, 0.6, 1, 1, 29
+    K, _ = synth.kv(H, t1 + t2, seed=42)
+    Q = R.haar_rotation(seed)
+    (tmp_path / "in.bin").write_bytes(u16(K).tobytes())
+    (tmp_path / "q.bin").write_bytes(Q.tobytes())
+    prefix = str(tmp_path / "kv_")
+    r = subprocess.run([exe, str(tmp_path / "in.bin"), str(tmp_path / "q.bin"), str(H), str(t1), str(t2), repr(alpha),
+                        str(k), str(dk), str(seed), prefix], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    info = json.loads(r.stdout)
+    assert info["appends"] == 2
+    words, offs, base, pay = [], [], 0, 0
+    ref = np.zeros((H, t1 + t2, 128), np.float32)
+    for t0, T in ((0, t1), (t1, t2)):
+        a = K[:, t0:t0 + T].contiguous()
+        s_, off, pb = O.kv_append(a, t0, O.E8, alpha, k, seed, 1, base_word=base, rot=Q, dk_last=dk)
+        O.kv_read_append(s_, off - np.uint64(base), H, T, t0, O.E8, alpha, k, seed, 1, ref, t1 + t2, rot=Q, dk_last=dk)
+        words.append(s_)
+        offs.append(off[:-1])
+        base = int(off[-1])
+        pay += pb
+    offs.append(np.array([base], np.uint64))
+    assert info["payload_bits"] == pay and info["stream_words"] == base
+    assert np.array_equal(np.fromfile(prefix + "stream.bin", np.uint32), np.concatenate(words))
+    assert np.array_equal(np.fromfile(prefix + "offsets.bin", np.uint64), np.concatenate(offs))
+    assert_recon_equal(np.fromfile(prefix + "out.bin", np.float32).reshape(H, t1 + t2, 128), ref)
+    d = (np.fromfile(prefix + "qdraw.bin", np.float32).reshape(128, 128).view(np.int32).astype(np.int64)
+         - Q.view(np.int32).astype(np.int64))
+    assert np.abs(d).max() <= 1          # the library's Haar draw: the oracle's to one ulp
