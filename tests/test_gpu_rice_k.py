@@ -181,3 +181,26 @@ def test_two_k_static_entry_point():
         assert hq.read_stats(st) == ref["stats"]
         assert np.array_equal(offs.cpu().numpy().view(np.uint64), ref["offsets"])
         assert np.array_equal(words[:ref["total"]].cpu().numpy().view(np.uint32), ref["words"])
+
+
+def test_two_k_corrupt_streams_are_flagged():
+    """The decoder's MIXED variant on bad data: swapped offsets and a flipped unary bit
+    flag HQ_ST_CORRUPT and zero that chunk's tiles; the other chunks decode exactly."""
+    hq = _hq()
+    x = synth.weight(16, 1024, seed=27)
+    p = hq.make_params("D4", ALPHA["D4"], 2, 3, 0, dk_last=1)
+    g = gpu_quantize(x.cuda(), p)
+    good, st, _ = gpu_dequantize(g["words_t"], g["cap"], g["offsets_t"], 16, 1024, p)
+    assert st["status"] == 0
+    off = g["offsets_t"].clone()
+    off[2], off[3] = off[3], off[2]
+    y, st, _ = gpu_dequantize(g["words_t"], g["cap"], off, 16, 1024, p)
+    assert st["status"] & hq.HQ_ST_CORRUPT
+    assert np.all(y[8:12] == 0)
+    assert np.array_equal(y[:4], good[:4]) and np.array_equal(y[12:], good[12:])
+    w = g["words_t"].clone()
+    b = int(g["offsets"][2])
+    w[b - 3] ^= 0x10
+    y, st, _ = gpu_dequantize(w, g["cap"], g["offsets_t"], 16, 1024, p)
+    assert st["status"] & hq.HQ_ST_CORRUPT
+    assert np.array_equal(y[:4], good[:4]) and np.array_equal(y[8:], good[8:])

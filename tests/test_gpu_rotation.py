@@ -202,3 +202,23 @@ def test_rotated_kv_scores(group):
             exact = w[h] @ qh
             lim = 40 * U * (np.abs(w[h]) @ np.abs(qh)) + 1e-30
             assert np.all(np.abs(got[h * group + g] - exact) <= lim)
+
+
+def test_rotated_read_of_a_corrupt_chunk_is_flagged():
+    """The rotated decoder on bad data: a flipped unary bit in one chunk flags HQ_ST_CORRUPT
+    and zeroes that chunk's tokens; the rest of the cache reads exactly."""
+    hq = _hq()
+    Q = R.haar_rotation(37)
+    K, _ = synth.kv(2, 96, seed=12)
+    cache = hq.KVCache(2, 96, hq.make_params("E8", 1.0, 1, 5, 1), bits_per_scalar=16.0, max_appends=2,
+                       max_append_tokens=96, rotation=torch.from_numpy(Q).cuda())
+    cache.append(K.cuda(), 0.5)
+    good = cache.read(torch.empty(2, 96, 128, device="cuda")).cpu().numpy()
+    off = cache.offsets[:7].cpu().numpy().view(np.uint64)      # 2 heads x 3 chunks
+    cache.words[int(off[2]) - 2] ^= 0x100                      # the last words of chunk 1 (head 0, tokens 32..63)
+    bad = cache.read(torch.empty(2, 96, 128, device="cuda")).cpu().numpy()
+    torch.cuda.synchronize()
+    assert hq.read_stats(cache.stats)["status"] & hq.HQ_ST_CORRUPT
+    assert np.all(bad[0, 32:64] == 0)
+    assert np.array_equal(bad[0, :32], good[0, :32]) and np.array_equal(bad[0, 64:], good[0, 64:])
+    assert np.array_equal(bad[1], good[1])
