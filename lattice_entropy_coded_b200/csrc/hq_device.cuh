@@ -209,7 +209,7 @@ __device__ __forceinline__ void rotate_round(float2 (&v)[16], const float *S, in
     for (int tt = 0; tt < 4; tt++)
 #pragma unroll
         for (int c = 0; c < 4; c++) acc[tt][c] = make_float2(0.0f, 0.0f);
-#pragma unroll 4
+#pragma unroll 8
     for (int k = 0; k < 128; k++) {
         const float4 z = *reinterpret_cast<const float4 *>(buf + 8 * k + 8 * (k >> 5) + 4 * g);
         const float4 m0 = *reinterpret_cast<const float4 *>(S + k * kRotPitch + 4 * j);
