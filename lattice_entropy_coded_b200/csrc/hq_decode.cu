@@ -22,8 +22,9 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
                 : small ? decode_kernel<LAT, DITHER, KV, true, kStoreTiles> : decode_kernel<LAT, DITHER, KV, false, kStoreTiles>;
     static LaunchPlan plans[3];
     unsigned grid = 0;
+    // at most one CTA per round (the kernel deals rounds to CTAs first)
     cudaError_t e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem,
-                                                           (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid);
+                                                           (unsigned long long)kRoundsPerChunk * a.n_chunks, grid);
     if (e != cudaSuccess) return e;
     kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     return cudaGetLastError();

@@ -8,8 +8,11 @@
 // instantiates the modes it launches.
 //
 // Work decomposition (B200, sm_100a):
-//  * one warp decodes one chunk (32 tiles) in 4 rounds of 8 tiles; four lanes
-//    share a tile, 32 symbols / elements each;
+//  * a chunk (32 tiles) decodes in 4 rounds of 8 tiles, four lanes to a tile and
+//    32 symbols / elements to a lane; a warp decodes whole chunks, strided over
+//    the grid, unless the launch has at most half as many chunks as the grid has
+//    warps: then two or four warps share a chunk, two rounds or one each, so a
+//    short launch still reaches every SM;
 //  * the chunk's words are brought into a per-warp shared-memory stage with
 //    cp.async while the warp is still decoding the previous chunk (two stages
 //    per warp); chunks too large for a stage are read from global memory;
@@ -22,7 +25,8 @@
 //  * the inverse FWHT runs in registers (two stages across the four lanes by
 //    shuffle), followed by the sign flip and 16-byte stores; or, for a KV cache
 //    with the dense rotation, x = Q^T z with Q^T in shared memory (rotate_round).
-// Chunks are independent (their offsets are given), so there is no look-back.
+// Chunks are independent (their offsets are given), so there is no look-back; a
+// chunk shared by several warps is staged and scanned by each.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -36,6 +40,7 @@ namespace {
 
 constexpr int kStagePad = 4;   // zero words after a staged chunk: unchecked 2-word reads stay inside
 constexpr int kRotDecodeWarps = 12;   // warps per CTA of the dense-rotation decoder (one CTA per SM)
+constexpr int kRoundsPerChunk = 32 / kTilesPerRound;   // the decoder's unit of work is one round
 
 // 32 bits of a plane of `n` words starting at bit `b`; words at or past n read as 0.
 __device__ __forceinline__ uint32_t fetch32_checked(const uint32_t *p, uint32_t n, uint32_t b) {
@@ -318,7 +323,6 @@ __device__ __forceinline__ bool find_segment_starts(const uint32_t *un, uint32_t
     return ok;
 }
 
-// The 4 rounds of one chunk, reading its planes from `src` (a stage when STAGED).
 // Dot product of a lane's 32 decoded values (bf16-rounded, signs applied: exactly the
 // stored bf16 tile) with 32 bf16 values of v: sequential fma in element order (the
 // products of two bf16 values are exact in fp32).
@@ -344,13 +348,14 @@ __device__ __forceinline__ float tile_sum(float acc) {
     return __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
 }
 
+// Rounds [r0, r1) of one chunk, reading its planes from `src` (a stage when STAGED).
 // ROT: the dense KV rotation's inverse (rot_s: its shared form) in place of H_128
 // and the sign diagonal.
 template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED, int MODE, bool ROT, bool MIXED>
 __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOut<KV> &geo, const uint32_t *src,
                                               bool ok, uint32_t nc, uint32_t nr, uint32_t nu,
                                               const uint32_t *startbit, const uint32_t *sign_tab,
-                                              const float *rot_s, int lane) {
+                                              const float *rot_s, int r0, int r1, int lane) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
     const int k = a.k, kl = a.k_last;
@@ -360,9 +365,9 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
     const uint32_t pk = 1u << k, pkl = 1u << kl;   // quotient weights 2^k, and 2^kl of a block's last symbol
     const uint32_t gbits = group_rem_bits<N>(k, kl), lane_bits = 4u * gbits;
     bool bad = false;
-    const int nrounds = (geo.ntiles + kTilesPerRound - 1) / kTilesPerRound;
+    const int nrounds = min((geo.ntiles + kTilesPerRound - 1) / kTilesPerRound, r1);
 #pragma unroll 1
-    for (int r = 0; r < nrounds; r++) {
+    for (int r = r0; r < nrounds; r++) {
         char *dst = nullptr;
         int tcol = 0;
         unsigned long long e0 = 0;
@@ -522,20 +527,24 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
 
     const int k = a.k;
     uint32_t status = 0;
+    // Which rounds this warp decodes: m = 2^lg = 1, 2 or 4 warps share a chunk, 4 / m
+    // rounds each, with m as large as the launch's chunks leave warps for.  The warp's
+    // slices are v = gw, gw + nwarps, ... (one when m > 1): chunk v / m, rounds from
+    // (v mod m) * 4 / m.  Warps are numbered across CTAs first when m > 1 (always in the
+    // rotation decoder), so that a short launch spreads over every SM.
     const unsigned long long nwarps = (unsigned long long)gridDim.x * W;
-    // the rotation decoder numbers chunks across CTAs first, so that a short read spreads
-    // over as many SMs as it has chunks
-    unsigned long long c = ROT ? (unsigned long long)warp * gridDim.x + blockIdx.x
-                               : (unsigned long long)blockIdx.x * W + warp;
+    const int lg = 4 * a.n_chunks <= nwarps ? 2 : 2 * a.n_chunks <= nwarps ? 1 : 0;
+    unsigned long long v = (ROT || lg) ? (unsigned long long)warp * gridDim.x + blockIdx.x
+                                       : (unsigned long long)blockIdx.x * W + warp;
     int buf = 0;
     ChunkWords cw = {0, 0, false};
-    if (c < a.n_chunks) {
-        cw = chunk_words(a, c);
+    if ((v >> lg) < a.n_chunks) {
+        cw = chunk_words(a, v >> lg);
         stage_chunk(a, cw, stages, lane);
     }
-    for (; c < a.n_chunks; c += nwarps, buf ^= 1) {
+    for (; (v >> lg) < a.n_chunks; v += nwarps, buf ^= 1) {
         // start bringing in the next chunk while this one is decoded
-        const unsigned long long cn = c + nwarps;
+        const unsigned long long cn = (v + nwarps) >> lg;
         ChunkWords cwn = {0, 0, false};
         if (cn < a.n_chunks) {
             cwn = chunk_words(a, cn);
@@ -546,6 +555,8 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
         }
         __syncwarp();
 
+        const unsigned long long c = v >> lg;
+        const int r0 = (int)(v & ((1u << lg) - 1u)) << (2 - lg), r1 = r0 + (kRoundsPerChunk >> lg);
         ChunkOut<KV> geo;
         geo.init(a, c);
         const int ntiles = geo.ntiles;
@@ -563,12 +574,12 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
             const uint32_t *src = stages + buf * kStageSlot;
             ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
             bad = decode_rounds<LAT, DITHER, KV, KSMALL, true, MODE, ROT, MIXED>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab,
-                                                                          rot_s, lane);
+                                                                          rot_s, r0, r1, lane);
         } else {
             const uint32_t *src = a.stream + cw.w0;
             ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
             bad = decode_rounds<LAT, DITHER, KV, KSMALL, false, MODE, ROT, MIXED>(a, geo, src, ok, nc, nr, nu, startbit,
-                                                                           sign_tab, rot_s, lane);
+                                                                           sign_tab, rot_s, r0, r1, lane);
         }
         if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) status |= HQ_ST_CORRUPT;
         cw = cwn;

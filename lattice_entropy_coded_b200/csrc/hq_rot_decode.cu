@@ -24,8 +24,9 @@ cudaError_t launch_rot_t(const DecodeArgs &a, cudaStream_t s) {
                 : small ? decode_kernel<LAT, DITHER, true, true, MODE, true> : decode_kernel<LAT, DITHER, true, false, MODE, true>;
     static LaunchPlan plans[3];
     unsigned grid = 0;
-    // one CTA per chunk up to one per SM; the kernel numbers chunks across CTAs first
-    cudaError_t e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, W * 32, smem, a.n_chunks, grid);
+    // one CTA per round up to one per SM (the kernel deals rounds to CTAs first)
+    cudaError_t e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, W * 32, smem,
+                                                           (unsigned long long)kRoundsPerChunk * a.n_chunks, grid);
     if (e != cudaSuccess) return e;
     kern<<<grid, W * 32, smem, s>>>(a);
     return cudaGetLastError();
