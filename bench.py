@@ -893,7 +893,7 @@ def main():
                 "roofline": r["roofline"], "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": r["launches"],
                 "points": r["per_point"],
             }
-            if not args.no_cpu_baseline:
+            if not args.no_cpu_baseline and world == 1:   # the oracle is timed at N = 1 only
                 line["cpu_baseline"] = cpu_baseline(args.workload)
             print(json.dumps(line), flush=True)
     finally:
