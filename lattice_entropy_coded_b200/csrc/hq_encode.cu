@@ -29,13 +29,22 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     cudaError_t e;
     unsigned grid = 0;
     // by size: one CTA for the whole launch up to kTinyMaxChunks chunks; the wide form
-    // while every chunk gets a 16-warp group of its own in one wave (148 SMs x 2 CTAs on
-    // a B200), the grouped form while it gets a 4-warp group (148 x 2 x kGroups), else
-    // the per-warp form
+    // while every chunk gets a 16-warp group of its own in one wave (2 CTAs per SM); the
+    // grouped form up to three quarters of the per-warp form's resident warps (2 CTAs of
+    // kWarpsPerCta per SM), or all of them with dither, because a warp encoding a lone
+    // chunk is latency-bound and four warps per chunk finish it sooner (B200, E8 4 bps:
+    // 1200 chunks 45.5 -> 37.9 us, 69.5 -> 48.2 us with dither); else the per-warp form
     int mode = g_encode_path;
-    if (mode == 0)
+    if (mode == 0) {
+        int dev = 0, sms = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return e;
+        const unsigned long long per_warp = 2ull * kWarpsPerCta * (unsigned long long)sms;
         mode = (a.n_chunks <= (unsigned long long)kTinyMaxChunks) ? 4
-               : (a.n_chunks <= 296ull) ? 3 : (a.n_chunks <= 592ull) ? 2 : 1;
+               : (a.n_chunks <= 2ull * (unsigned long long)sms) ? 3
+               : (a.n_chunks <= (DITHER ? per_warp : per_warp * 3 / 4)) ? 2 : 1;
+    }
     if (mode == 4 && a.n_chunks > (unsigned long long)kTinyMaxChunks) mode = 1;
     if (mixed && mode == 3) mode = 2;
     if (mode == 4) return launch_tiny_t<LAT, DITHER>(a, s, small, mixed);

@@ -4,15 +4,16 @@
 // and the rate-only pass that counts the same codes without writing them.
 //
 // Four forms with identical output, chosen by launch size (hq_encode.cu):
-//  * per-warp (throughput; more than 592 chunks): one warp encodes one chunk
+//  * per-warp (throughput; more than 1776 chunks on a B200, 2368 with dither):
+//    one warp encodes one chunk
 //    (32 tiles) in 4 rounds of 8 tiles; four lanes share a tile, 32 elements
 //    each, loaded as 64 contiguous bytes per lane with cp.async one round ahead;
 //    the transform runs in registers (16 float2 per lane, packed fp32 adds, the
 //    last two butterfly stages across lanes by shuffle); each lane decodes its
 //    32/N lattice blocks into 32 zigzag symbols; a warp scan of unary lengths
 //    places every codeword in a per-warp shared stage holding the chunk;
-//  * grouped (latency; up to 592 chunks): four warps share a chunk, one round
-//    each, meeting at a named barrier per chunk;
+//  * grouped (latency; up to 1776 chunks, 2368 with dither): four warps share
+//    a chunk, one round each, meeting at a named barrier per chunk;
 //  * wide (lowest latency; up to 296 chunks): sixteen warps share a chunk,
 //    sixteen lanes per tile, one 8-element block per lane;
 //  * single CTA (up to 32 chunks, such as a KV append of a few tokens): the

@@ -136,7 +136,7 @@ struct LaunchPlan {
 };
 
 // Encoder form: 0 = by size (one CTA for a few chunks, then wide, then grouped, for
-// launches of at most one wave of their chunk groups, per-warp otherwise), 1 =
+// launches of fewer chunks than the per-warp form has resident warps, per-warp otherwise), 1 =
 // per-warp, 2 = grouped (4 warps per chunk), 3 = wide (16 warps per chunk, 16 lanes
 // per tile), 4 = one CTA.  Set by hq_debug_set_encode_path (hq_api.cu); all forms
 // give identical streams.
