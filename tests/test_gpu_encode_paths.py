@@ -95,3 +95,21 @@ def test_stats_are_replaced_not_accumulated(path):
         hq.hq_quantize(x, params, words, offs, st, ws)
         got = hq.read_stats(st)
         assert got == ref["stats"], (got, ref["stats"])
+
+
+@pytest.mark.parametrize("chunks,lat,dither,dk", [(296, "E8", 0, 0), (297, "E8", 0, 0), (1776, "E8", 0, 0),
+                                                  (1777, "E8", 0, 0), (2368, "D4", 1, 0), (2369, "D4", 1, 0),
+                                                  (1500, "A2", 0, 1)])
+def test_default_form_boundaries(chunks, lat, dither, dk):
+    """The size rule's boundaries on a B200 (wide up to 296 chunks; grouped up to 1776, or 2368
+    with dither; per-warp above), on R x 4096 matrices (one chunk per row), default form."""
+    import lattice_entropy_coded_b200 as hq
+    alpha = {q["lattice"]: q["alpha"] for q in rate_points()["weight_4096x4096_rate_sweep"]["points"]
+             if q["bps"] == 4.0}[lat]
+    x = synth.weight(chunks, 4096, seed=chunks)
+    params = hq.make_params(lat, alpha, 2, 3, dither, dk_last=dk)
+    g = gpu_quantize(x.cuda(), params)
+    ref_w, ref_off, ref_pay = oracle_quantize(x, O.LATTICES[lat], alpha, 2, 3, dither, dk_last=dk)
+    assert g["stats"]["status"] == 0
+    assert_same_words(g["words"], g["offsets"], ref_w, ref_off)
+    assert g["stats"]["payload_bits"] == ref_pay
