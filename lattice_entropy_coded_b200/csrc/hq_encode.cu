@@ -22,6 +22,20 @@ cudaError_t launch_tiny_t(const EncodeArgs &a, cudaStream_t s, bool small, bool 
     return cudaGetLastError();
 }
 
+// One-token KV appends: every chunk is one tile.
+template <int LAT, bool DITHER>
+cudaError_t launch_tok_t(const EncodeArgs &a, cudaStream_t s) {
+    const size_t smem = (size_t)(a.tcols * kSignWords + kTinyMaxChunks * kTokStageWords) * sizeof(uint32_t) +
+                        kTinyMaxChunks * (sizeof(TinyChunk) + sizeof(unsigned long long));
+    auto kern = encode_kernel_tok<LAT, DITHER>;
+    static LaunchPlan plan;
+    unsigned grid = 0;
+    cudaError_t e = plan.grid(kern, kTinyWarps * 32, smem, 1, grid);
+    if (e != cudaSuccess) return e;
+    kern<<<1, kTinyWarps * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <int LAT, bool DITHER>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     const bool small = a.k <= 4;
@@ -47,7 +61,11 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     }
     if (mode == 4 && a.n_chunks > (unsigned long long)kTinyMaxChunks) mode = 1;
     if (mixed && mode == 3) mode = 2;
-    if (mode == 4) return launch_tiny_t<LAT, DITHER>(a, s, small, mixed);
+    if (mode == 4) {
+        // a one-token KV append (one tile per chunk) with a single Rice parameter
+        if (a.map.kv && a.map.tokens == 1 && !mixed) return launch_tok_t<LAT, DITHER>(a, s);
+        return launch_tiny_t<LAT, DITHER>(a, s, small, mixed);
+    }
     // the multi-CTA forms share the workspace: look-back words, ticket, done counter and
     // stats accumulator, cleared by one memset
     if ((e = cudaMemsetAsync(a.lookback, 0, encode_scratch_bytes(a.n_chunks), s)) != cudaSuccess) return e;

@@ -18,7 +18,9 @@
 //    sixteen lanes per tile, one 8-element block per lane;
 //  * single CTA (up to 32 chunks, such as a KV append of a few tokens): the
 //    CTA's warps encode the chunks into their own stages and one warp scans
-//    the sizes into offsets, with no workspace, ticket or look-back.
+//    the sizes into offsets, with no workspace, ticket or look-back; for a
+//    one-token append (one-tile chunks) each half-warp takes a chunk in the
+//    wide form's layout.
 // In the first three a persistent grid takes chunk tickets from a global
 // counter, so a chunk's predecessors are always already running, and a
 // single-pass decoupled look-back over 64-bit (flag, value) words gives each
@@ -1239,6 +1241,78 @@ struct TinyChunk {
     unsigned long long payload;
 };
 
+// The single-CTA forms' last steps, after a barrier that publishes info[]: one warp
+// scans the chunk sizes (at most 32) into offsets and writes the offsets, the tail, the
+// append row and the stats; then the warps copy their stages (`stage_words` apart) out,
+// or set an oversize chunk's bits in place.  Whole CTA calls it.
+template <int LAT, bool DITHER, bool ROT>
+__device__ __forceinline__ void tiny_finish(const EncodeArgs &a, int n, const TinyChunk *info,
+                                            unsigned long long *start, const uint32_t *stage_all, int stage_words,
+                                            const uint32_t *sign_tab, const float *rot_s) {
+    constexpr int N = Lattice<LAT>::N;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
+        const TinyChunk t = lane < n ? info[lane] : TinyChunk{0u, 0u, 0u, 0u, 0ull};
+        unsigned long long incl = t.total;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        const unsigned long long st = base + incl - t.total;
+        if (lane < n) {
+            start[lane] = st;
+            a.offsets[a.chunk_base + lane] = st;
+        }
+        const unsigned long long end = base + __shfl_sync(0xffffffffu, incl, 31);
+        const uint32_t status = __reduce_or_sync(0xffffffffu, t.status) | (end > a.cap_words ? HQ_ST_CAPACITY : 0u);
+        const uint32_t zor = __reduce_or_sync(0xffffffffu, t.zor);
+        const unsigned long long payload = warp_sum_u64(t.payload);
+        if (lane == 0) {
+            a.offsets[a.chunk_base + n] = end;
+            if (a.tail_out) *a.tail_out = end;
+            if (a.row) *a.row = a.row_val;
+            if (a.stats) {
+                if (a.stats_add) {
+                    if (status) atomicOr(&a.stats->status, status);
+                    if (zor) atomicOr(&a.stats->max_symbol, zor);
+                    if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
+                } else {
+                    a.stats->status = status;
+                    a.stats->max_symbol = zor;
+                    a.stats->payload_bits = payload;
+                }
+                a.stats->stream_words = end;
+            }
+        }
+    }
+    __syncthreads();
+
+    for (int c = warp; c < n; c += kTinyWarps) {
+        const TinyChunk t = info[c];
+        const unsigned long long st = start[c];
+        if (t.status) continue;   // outside the supported range: nothing written
+        if (!t.overflow) {
+            const uint32_t *stage = stage_all + c * stage_words;
+            for (uint32_t i = lane; i < t.total; i += 32)
+                if (st + i < a.cap_words) a.stream[st + i] = stage[i];
+        } else {
+            uint32_t *g = a.stream + st;
+            const unsigned long long room = (st < a.cap_words) ? a.cap_words - st : 0ull;
+            for (unsigned long long i = lane; i < t.total; i += 32)
+                if (i < room) g[i] = 0u;
+            __syncwarp();
+            __threadfence_block();
+            ChunkGeo geo;
+            geo.init(a.map, (unsigned long long)c);
+            const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * geo.ntiles + 31) / 32u : 0u;
+            const uint32_t nr = ((uint32_t)geo.ntiles * tile_rem_bits<N>(a.k, a.k_last) + 31u) >> 5;
+            encode_chunk_global<LAT, DITHER, ROT>(a, geo, sign_tab, rot_s, g, room, nc, nr);
+        }
+    }
+}
+
 template <int LAT, bool DITHER, bool KSMALL, bool ROT, bool MIXED>
 __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tiny(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
@@ -1344,68 +1418,96 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tiny(const E
     }
     __syncthreads();
 
-    // offsets: one warp scans the chunk sizes (at most 32); the same warp writes the
-    // offsets, the tail, the append row and the stats
-    if (warp == 0) {
-        const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
-        const TinyChunk t = lane < n ? info[lane] : TinyChunk{0u, 0u, 0u, 0u, 0ull};
-        unsigned long long incl = t.total;
+    tiny_finish<LAT, DITHER, ROT>(a, n, info, start, stage_all, kStageWords, sign_tab, rot_s);
+}
+
+// One-token KV appends (every chunk one tile: one token of one head), up to kTinyMaxChunks
+// chunks: the single-CTA form, with each half-warp encoding one chunk in the wide form's
+// layout (16 lanes to the tile, one 8-element lattice block each).  A lane then carries
+// one lattice block and one dither block instead of four, which shortens the chain that
+// sets a decode step's append latency.  The chunk's unary bits are placed by a scan over
+// its 16 lanes; its stage is kTokStageWords long (larger chunks take the in-place path).
+// Without the dense rotation or a second Rice parameter.
+constexpr int kTokStageWords = 256;
+
+template <int LAT, bool DITHER>
+__global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tok(const EncodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *sign_tab = smem;                                       // tcols * kSignWords
+    uint32_t *stage_all = sign_tab + a.tcols * kSignWords;           // kTinyMaxChunks * kTokStageWords
+    TinyChunk *info = reinterpret_cast<TinyChunk *>(stage_all + kTinyMaxChunks * kTokStageWords);
+    unsigned long long *start = reinterpret_cast<unsigned long long *>(info + kTinyMaxChunks);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, l16 = lane & 15;
+    const int n = (int)a.n_chunks;   // <= kTinyMaxChunks, one tile each (host)
+
+    build_sign_table(sign_tab, a.tcols, a.seed);
+    for (int i = threadIdx.x; i < n * kTokStageWords / 4; i += blockDim.x)
+        reinterpret_cast<uint4 *>(stage_all)[i] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+
+    const int k = a.k;
+    const uint32_t nc = (LAT == HQ_E8) ? 1u : 0u;   // the coset word of the tile's 16 blocks
+    const uint32_t nr = 4u * (uint32_t)k;           // 128 remainders of k bits
+    for (int c0 = 2 * warp; c0 < n; c0 += 2 * kTinyWarps) {
+        const int c = c0 + (lane >> 4);
+        const bool live = c < n;
+        const uint16_t *src = nullptr;
+        int tcol = 0;
+        unsigned long long e0 = 0;
+        bool valid = false;
+        if (live) {
+            ChunkGeo geo;
+            geo.init(a.map, (unsigned long long)c);
+            valid = geo.tile(a.map, a.x, 0, src, tcol, e0);
+        }
+        const uint4 raw = valid ? ldg_nc_v4(src + 8 * l16) : make_uint4(0, 0, 0, 0);
+        uint32_t z[8], cbit;
+        wide_symbols<LAT, DITHER>(a, valid, tcol, e0, raw, lane, sign_tab, z, cbit);
+        uint32_t usum = 0, hz = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long u = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += u;
+        for (int i = 0; i < 8; i++) {
+            usum += z[i] >> k;
+            hz |= z[i];
         }
-        const unsigned long long st = base + incl - t.total;
-        if (lane < n) {
-            start[lane] = st;
-            a.offsets[a.chunk_base + lane] = st;
+        const uint32_t ub = valid ? usum + 8u : 0u;
+        uint32_t incl = ub;   // within the half-warp
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (l16 >= o) incl += t;
         }
-        const unsigned long long end = base + __shfl_sync(0xffffffffu, incl, 31);
-        const uint32_t status = __reduce_or_sync(0xffffffffu, t.status) | (end > a.cap_words ? HQ_ST_CAPACITY : 0u);
-        const uint32_t zor = __reduce_or_sync(0xffffffffu, t.zor);
-        const unsigned long long payload = warp_sum_u64(t.payload);
-        if (lane == 0) {
-            a.offsets[a.chunk_base + n] = end;
-            if (a.tail_out) *a.tail_out = end;
-            if (a.row) *a.row = a.row_val;
-            if (a.stats) {
-                if (a.stats_add) {
-                    if (status) atomicOr(&a.stats->status, status);
-                    if (zor) atomicOr(&a.stats->max_symbol, zor);
-                    if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
-                } else {
-                    a.stats->status = status;
-                    a.stats->max_symbol = zor;
-                    a.stats->payload_bits = payload;
-                }
-                a.stats->stream_words = end;
+        const uint32_t U = __shfl_sync(0xffffffffu, incl, lane | 15);
+#pragma unroll
+        for (int o = 8; o; o >>= 1) hz |= __shfl_xor_sync(0xffffffffu, hz, o);
+        const bool range_bad = (hz >> 22) != 0u || U >= kMaxUnaryBits;
+        const uint32_t total = nc + nr + (U + 31u) / 32u;
+        const bool overflow = total > (uint32_t)kTokStageWords;
+        const uint32_t cw = __ballot_sync(0xffffffffu, cbit != 0u);
+        if (valid && !overflow && !range_bad) {
+            uint32_t *stage = stage_all + c * kTokStageWords;
+            if (LAT == HQ_E8 && l16 == 0) {
+                const uint32_t bits = (lane & 16) ? (cw >> 16) : (cw & 0xFFFFu);
+                if (bits) stage[0] = bits;
             }
+            wide_put_rem(stage + nc, (uint32_t)l16 * 8u * (uint32_t)k, z, k);
+            uint32_t qg[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) qg[i] = z[i] >> k;
+            unary_group_shared(stage + nc + nr, incl - ub, qg);
+        }
+        if (live && l16 == 0) {
+            TinyChunk t;
+            t.total = total;
+            t.status = range_bad ? HQ_ST_RANGE : 0u;
+            t.overflow = overflow ? 1u : 0u;
+            t.zor = hz;
+            t.payload = U + 128ull * (unsigned long long)k + ((LAT == HQ_E8) ? 16ull : 0ull);
+            info[c] = t;
         }
     }
     __syncthreads();
 
-    for (int c = warp; c < n; c += kTinyWarps) {
-        const TinyChunk t = info[c];
-        const unsigned long long st = start[c];
-        if (t.status) continue;   // outside the supported range: nothing written
-        if (!t.overflow) {
-            const uint32_t *stage = stage_all + c * kStageWords;
-            for (uint32_t i = lane; i < t.total; i += 32)
-                if (st + i < a.cap_words) a.stream[st + i] = stage[i];
-        } else {
-            uint32_t *g = a.stream + st;
-            const unsigned long long room = (st < a.cap_words) ? a.cap_words - st : 0ull;
-            for (unsigned long long i = lane; i < t.total; i += 32)
-                if (i < room) g[i] = 0u;
-            __syncwarp();
-            __threadfence_block();
-            ChunkGeo geo;
-            geo.init(a.map, (unsigned long long)c);
-            const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * geo.ntiles + 31) / 32u : 0u;
-            const uint32_t nr = ((uint32_t)geo.ntiles * tile_rem_bits<N>(a.k, a.k_last) + 31u) >> 5;
-            encode_chunk_global<LAT, DITHER, ROT>(a, geo, sign_tab, rot_s, g, room, nc, nr);
-        }
-    }
+    tiny_finish<LAT, DITHER, false>(a, n, info, start, stage_all, kTokStageWords, sign_tab, nullptr);
 }
 
 // ------------------------------------------------------------------ rate only
