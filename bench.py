@@ -839,6 +839,50 @@ def run_case(args):
                                           "bf16_gemv": 2.0 * n + 2.0 * cols}}), flush=True)
 
 
+def run_token_case(args):
+    """One-token KV appends, as a decode step makes them: 8 heads, E8 with dither at the K 2.0 bps
+    point of the 8-head KV workload; 128 appends replayed from a CUDA graph, then the same appends
+    as plain calls.  Prints the device time per append.  The small case the ncu capture of the
+    one-token encoder runs on."""
+    import lattice_entropy_coded_b200 as hq
+    wl = "kv_8h_32768tok_e8_dither"
+    w = synth.WORKLOADS[wl]
+    H = w["heads"]
+    p = [q for q in rate_points()[wl]["points"] if q["tensor"] == "K" and q["bps"] == 2.0][0]
+    device = torch.device("cuda", 0)
+    K, _ = synth.kv(H, 128, seed=w["seed"], device=device)
+    params = hq.make_params("E8", 1.0, p["k"], w["seed"], 1)
+    one = hq.KVCache(H, 128, params, bits_per_scalar=p["bps"] + 8.0, max_appends=129, max_append_tokens=1,
+                     device=device)
+    toks = [K[:, t:t + 1].contiguous() for t in range(128)]
+    # plain calls first (these are the launches an ncu capture sees), then the graph
+    for _ in range(args.warmup):
+        hq.hq_kv_init(one.cache, H, 128, params, one.words, one.offsets, one.table, one.tail, one.stats)
+        for tk in toks:
+            one.append(tk, p["alpha"])
+    torch.cuda.synchronize()
+    hq.hq_kv_init(one.cache, H, 128, params, one.words, one.offsets, one.table, one.tail, one.stats)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for tk in toks:
+            one.append(tk, p["alpha"])
+    ms = []
+    for it in range(args.warmup + args.steps):
+        hq.hq_kv_init(one.cache, H, 128, params, one.words, one.offsets, one.table, one.tail, one.stats)
+        a, b = _events()
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            ms.append(a.elapsed_time(b))
+    st = hq.read_stats(one.stats)
+    del g
+    print(json.dumps({"case": "kv one-token appends", "heads": H, "appends": 128, "k": p["k"], "alpha": p["alpha"],
+                      "status": st["status"], "bps_payload": st["payload_bits"] / (H * 128 * 128),
+                      "token_append_us": float(np.median(ms)) * 1e3 / 128}), flush=True)
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -851,6 +895,7 @@ def main():
     ap.add_argument("--oracle", action="store_true",
                     help="with --workload: also time the CPU oracle on the workload (about a minute per point)")
     ap.add_argument("--case", default=None, help="RxC: time one matrix (profiling case)")
+    ap.add_argument("--token-case", action="store_true", help="time one-token KV appends (profiling case)")
     ap.add_argument("--lattice", default="E8")
     ap.add_argument("--bps", type=float, default=4.0)
     ap.add_argument("--dither", type=int, default=0)
@@ -858,6 +903,9 @@ def main():
     args.warmup = max(3, args.warmup)
     if args.case:
         run_case(args)
+        return
+    if args.token_case:
+        run_token_case(args)
         return
     if args.workload != DEFAULT_WORKLOAD and args.impl == "ours":
         run_bulk(args)
