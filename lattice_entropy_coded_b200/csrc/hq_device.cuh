@@ -244,6 +244,41 @@ __device__ __forceinline__ void rotate_round(float2 (&v)[16], const float *S, in
     __syncwarp();
 }
 
+// v (4 float2 per lane: elements 8 l, 8 l + 1, ..., 8 l + 7 of the half-warp's tile, l =
+// lane & 15, the wide layout) <- M v for each half-warp's tile.  Each lane computes its own
+// 8 outputs: per input k, two 16-byte loads of S[k][8 l ..] (the other half-warp reads the
+// same words) and a 16-byte broadcast of 4 inputs from xs, the half-warp's 128-float copy
+// of its tile (16-byte aligned, at xs + 128 * (lane >> 4)).  Whole warp.
+__device__ __forceinline__ void rotate_sixteenth(float2 (&v)[4], const float *S, float *xs, int lane) {
+    const int l16 = lane & 15;
+    float *x = xs + 128 * (lane >> 4);
+    reinterpret_cast<float4 *>(x)[2 * l16] = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+    reinterpret_cast<float4 *>(x)[2 * l16 + 1] = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
+    __syncwarp();
+    float2 acc[4];
+#pragma unroll
+    for (int c = 0; c < 4; c++) acc[c] = make_float2(0.0f, 0.0f);
+#pragma unroll 4
+    for (int k4 = 0; k4 < 32; k4++) {
+        const float4 x4 = reinterpret_cast<const float4 *>(x)[k4];
+        const float xk[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const float *row = S + (4 * k4 + u) * kRotPitch + 8 * l16;
+            const float4 m0 = *reinterpret_cast<const float4 *>(row);
+            const float4 m1 = *reinterpret_cast<const float4 *>(row + 4);
+            const float2 x2 = make_float2(xk[u], xk[u]);
+            acc[0] = f2_fma(make_float2(m0.x, m0.y), x2, acc[0]);
+            acc[1] = f2_fma(make_float2(m0.z, m0.w), x2, acc[1]);
+            acc[2] = f2_fma(make_float2(m1.x, m1.y), x2, acc[2]);
+            acc[3] = f2_fma(make_float2(m1.z, m1.w), x2, acc[3]);
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 4; c++) v[c] = acc[c];
+}
+
 // ------------------------------------------------------------------ lattices
 // Rounding without the conversion pipe: for |x| < 2^22, x + 1.5*2^23 lands in
 // [2^23, 2^24) where the fp32 spacing is 1, so the add rounds x to the nearest

@@ -27,7 +27,7 @@ template <int LAT, bool DITHER>
 cudaError_t launch_tok_t(const EncodeArgs &a, cudaStream_t s) {
     const size_t smem = (size_t)(a.tcols * kSignWords + kTinyMaxChunks * kTokStageWords) * sizeof(uint32_t) +
                         kTinyMaxChunks * (sizeof(TinyChunk) + sizeof(unsigned long long));
-    auto kern = encode_kernel_tok<LAT, DITHER>;
+    auto kern = encode_kernel_tok<LAT, DITHER, false>;
     static LaunchPlan plan;
     unsigned grid = 0;
     cudaError_t e = plan.grid(kern, kTinyWarps * 32, smem, 1, grid);

@@ -1007,25 +1007,33 @@ __device__ __forceinline__ void wide_sync() {
     asm volatile("bar.sync 1, %0;" ::"r"(kWideWarps * 32) : "memory");
 }
 
-// A lane's 8 elements of its tile: signs, FWHT-128 with its 15 partner lanes,
+// A lane's 8 elements of its tile: signs, FWHT-128 with its 15 partner lanes (or with
+// ROT the dense rotation, rot_s its shared form and xs the warp's 256-float buffer),
 // scale, [+ dither], lattice blocks -> 8 zigzag symbols and (E8) the coset bit.
-template <int LAT, bool DITHER>
+template <int LAT, bool DITHER, bool ROT = false>
 __device__ __forceinline__ void wide_symbols(const EncodeArgs &a, bool valid, int tcol, unsigned long long e0,
                                              uint4 raw, int lane, const uint32_t *sign_tab, uint32_t (&z)[8],
-                                             uint32_t &cbit) {
+                                             uint32_t &cbit, const float *rot_s = nullptr, float *xs = nullptr) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
     const int l16 = lane & 15;
-    const uint32_t es = sign_tab[tcol * kSignWords + (l16 >> 2)];
     const uint4 w = valid ? raw : make_uint4(0, 0, 0, 0);
     const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
     float2 v[4];
+    if constexpr (ROT) {
 #pragma unroll
-    for (int t = 0; t < 4; t++) {
-        const uint32_t ww = wv[t] ^ sign_pair_mask(es, 4 * (l16 & 3) + t);
-        v[t] = make_float2(__uint_as_float(ww << 16), __uint_as_float(ww & 0xFFFF0000u));
+        for (int t = 0; t < 4; t++)
+            v[t] = make_float2(__uint_as_float(wv[t] << 16), __uint_as_float(wv[t] & 0xFFFF0000u));
+        rotate_sixteenth(v, rot_s, xs, lane);
+    } else {
+        const uint32_t es = sign_tab[tcol * kSignWords + (l16 >> 2)];
+#pragma unroll
+        for (int t = 0; t < 4; t++) {
+            const uint32_t ww = wv[t] ^ sign_pair_mask(es, 4 * (l16 & 3) + t);
+            v[t] = make_float2(__uint_as_float(ww << 16), __uint_as_float(ww & 0xFFFF0000u));
+        }
+        fwht128_sixteenth(v, lane);
     }
-    fwht128_sixteenth(v, lane);
     const float2 c2 = make_float2(a.c_scale, a.c_scale);
 #pragma unroll
     for (int t = 0; t < 4; t++) v[t] = f2_mul(v[t], c2);
@@ -1427,20 +1435,27 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tiny(const E
 // one lattice block and one dither block instead of four, which shortens the chain that
 // sets a decode step's append latency.  The chunk's unary bits are placed by a scan over
 // its 16 lanes; its stage is kTokStageWords long (larger chunks take the in-place path).
-// Without the dense rotation or a second Rice parameter.
+// With ROT the dense rotation replaces the sign diagonal and H_128 (each lane computes
+// its 8 outputs in full, rotate_sixteenth).  Single Rice parameter only.
 constexpr int kTokStageWords = 256;
 
-template <int LAT, bool DITHER>
+template <int LAT, bool DITHER, bool ROT>
 __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tok(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t *sign_tab = smem;                                       // tcols * kSignWords
+    float *rot_s = ROT ? reinterpret_cast<float *>(smem) : nullptr;   // rot_smem_bytes(kTinyWarps)
+    uint32_t *sign_tab = smem + (ROT ? rot_smem_bytes(kTinyWarps) / sizeof(uint32_t) : 0);   // tcols * kSignWords
     uint32_t *stage_all = sign_tab + a.tcols * kSignWords;           // kTinyMaxChunks * kTokStageWords
     TinyChunk *info = reinterpret_cast<TinyChunk *>(stage_all + kTinyMaxChunks * kTokStageWords);
     unsigned long long *start = reinterpret_cast<unsigned long long *>(info + kTinyMaxChunks);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, l16 = lane & 15;
     const int n = (int)a.n_chunks;   // <= kTinyMaxChunks, one tile each (host)
 
-    build_sign_table(sign_tab, a.tcols, a.seed);
+    if (ROT)
+        load_rotation<true>(rot_s, a.rot);
+    else
+        build_sign_table(sign_tab, a.tcols, a.seed);
+    // with ROT: the first 256 floats of the warp's rotation buffer hold its two tiles
+    float *xs = ROT ? rot_s + 128 * kRotPitch + warp * kRotBufFloats : nullptr;
     for (int i = threadIdx.x; i < n * kTokStageWords / 4; i += blockDim.x)
         reinterpret_cast<uint4 *>(stage_all)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
@@ -1462,7 +1477,7 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tok(const En
         }
         const uint4 raw = valid ? ldg_nc_v4(src + 8 * l16) : make_uint4(0, 0, 0, 0);
         uint32_t z[8], cbit;
-        wide_symbols<LAT, DITHER>(a, valid, tcol, e0, raw, lane, sign_tab, z, cbit);
+        wide_symbols<LAT, DITHER, ROT>(a, valid, tcol, e0, raw, lane, sign_tab, z, cbit, rot_s, xs);
         uint32_t usum = 0, hz = 0;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
@@ -1507,7 +1522,7 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tok(const En
     }
     __syncthreads();
 
-    tiny_finish<LAT, DITHER, false>(a, n, info, start, stage_all, kTokStageWords, sign_tab, nullptr);
+    tiny_finish<LAT, DITHER, ROT>(a, n, info, start, stage_all, kTokStageWords, sign_tab, rot_s);
 }
 
 // ------------------------------------------------------------------ rate only

@@ -1,9 +1,9 @@
 // hq_rot_encode.cu -- launchers of the quantize + encode kernel and of the rate pass
 // with the dense KV rotation (a 128 x 128 orthogonal matrix per cache in place of
 // the sign diagonal and H_128; explainer pages, "Methodology" 4).  The kernels are
-// the grouped form and the rate kernel of hq_encode.cuh with ROT = true; they are
-// instantiated in this file of their own so that they compile in parallel with
-// the rest.
+// the grouped, single-CTA and one-token forms and the rate kernel of hq_encode.cuh
+// with ROT = true, instantiated in this file of their own so that they compile in
+// parallel with the rest.
 #include "hq_encode.cuh"
 
 namespace hq {
@@ -13,10 +13,25 @@ namespace {
 // Up to kTinyMaxChunksRot chunks: one CTA for the whole launch.  Beyond: the grouped
 // form, four warps per chunk, one CTA of kRotGroups groups per SM (the rotation's shared
 // form and per-warp buffers, 194 KB).
+// A one-token append (one tile per chunk) with a single Rice parameter: the one-token
+// form, a half-warp per chunk, up to kTinyMaxChunks chunks.
 template <int LAT, bool DITHER>
 cudaError_t launch_rot_t(const EncodeArgs &a, cudaStream_t s) {
     const bool small = a.k <= 4, mixed = a.k_last != a.k;
-    if (a.n_chunks <= (unsigned long long)kTinyMaxChunksRot && (g_encode_path == 0 || g_encode_path == 4)) {
+    const bool single_cta = g_encode_path == 0 || g_encode_path == 4;
+    if (single_cta && a.map.kv && a.map.tokens == 1 && !mixed && a.n_chunks <= (unsigned long long)kTinyMaxChunks) {
+        const size_t smem = rot_smem_bytes(kTinyWarps) +
+                            (size_t)(a.tcols * kSignWords + kTinyMaxChunks * kTokStageWords) * sizeof(uint32_t) +
+                            kTinyMaxChunks * (sizeof(TinyChunk) + sizeof(unsigned long long));
+        auto kern = encode_kernel_tok<LAT, DITHER, true>;
+        static LaunchPlan kplan;
+        unsigned kgrid = 0;
+        cudaError_t e = kplan.grid(kern, kTinyWarps * 32, smem, 1, kgrid);
+        if (e != cudaSuccess) return e;
+        kern<<<1, kTinyWarps * 32, smem, s>>>(a);
+        return cudaGetLastError();
+    }
+    if (a.n_chunks <= (unsigned long long)kTinyMaxChunksRot && single_cta) {
         const size_t smem = kRotSmemBytes + (size_t)(a.tcols * kSignWords + kTinyMaxChunksRot * kStageWords) *
                                                 sizeof(uint32_t) +
                             kTinyMaxChunksRot * (sizeof(TinyChunk) + sizeof(unsigned long long));
