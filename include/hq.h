@@ -391,12 +391,14 @@ HQ_API int hq_device_check(void);
 HQ_API void hq_debug_set_spin_limit(uint32_t polls);
 
 /* Testing aid: which form of the quantize kernel runs.  0 (default) chooses by
- * size: launches of at most 32 chunks (16 with a dense rotation) run in one CTA
- * (no workspace is touched: the fewest steps for a KV append of a few tokens), of
- * at most 296 chunks the wide form (16 warps share a chunk, 16 lanes per tile),
- * of at most 592 the grouped form (4 warps share a chunk), larger ones the
- * per-warp form (a warp encodes whole chunks: the highest throughput); the limits
- * are one wave of chunk groups on a B200.  1 forces per-warp, 2 grouped, 3 wide,
+ * size: launches of at most 32 chunks (16 with a dense rotation, except one-token
+ * appends) run in one CTA (no workspace is touched: the fewest steps for a KV
+ * append of a few tokens; a one-token append gives each chunk to a half-warp), of
+ * at most 2 chunks per SM the wide form (16 warps share a chunk, 16 lanes per
+ * tile), of at most three quarters of the per-warp form's resident warps (all of
+ * them with dither; 1776 and 2368 chunks on a B200) the grouped form (4 warps
+ * share a chunk), larger ones the per-warp form (a warp encodes whole chunks: the
+ * highest throughput).  1 forces per-warp, 2 grouped, 3 wide,
  * 4 the single CTA (per-warp beyond its limit).  A dense rotation uses the grouped
  * form unless the single CTA applies; a second Rice parameter replaces the wide
  * form by the grouped one.  All give identical streams, offsets and stats.
