@@ -1249,34 +1249,31 @@ struct TinyChunk {
     unsigned long long payload;
 };
 
-// The single-CTA forms' last steps, after a barrier that publishes info[]: one warp
-// scans the chunk sizes (at most 32) into offsets and writes the offsets, the tail, the
-// append row and the stats; then the warps copy their stages (`stage_words` apart) out,
-// or set an oversize chunk's bits in place.  Whole CTA calls it.
+// The single-CTA forms' last steps, after a barrier that publishes info[]: every warp
+// scans the chunk sizes (at most 32) into offsets from `base` (the stream's end before
+// this call, loaded at the kernel's start), so that it can copy its own stages out (or
+// set an oversize chunk's bits in place) without a second barrier; warp 0 also writes
+// the offsets, the tail, the append row and the stats.  Whole CTA calls it.
 template <int LAT, bool DITHER, bool ROT>
 __device__ __forceinline__ void tiny_finish(const EncodeArgs &a, int n, const TinyChunk *info,
-                                            unsigned long long *start, const uint32_t *stage_all, int stage_words,
+                                            unsigned long long base, const uint32_t *stage_all, int stage_words,
                                             const uint32_t *sign_tab, const float *rot_s) {
     constexpr int N = Lattice<LAT>::N;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (warp == 0) {
-        const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
-        const TinyChunk t = lane < n ? info[lane] : TinyChunk{0u, 0u, 0u, 0u, 0ull};
-        unsigned long long incl = t.total;
+    const TinyChunk mine = lane < n ? info[lane] : TinyChunk{0u, 0u, 0u, 0u, 0ull};
+    unsigned long long incl = mine.total;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long u = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += u;
-        }
-        const unsigned long long st = base + incl - t.total;
-        if (lane < n) {
-            start[lane] = st;
-            a.offsets[a.chunk_base + lane] = st;
-        }
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    const unsigned long long st_lane = base + incl - mine.total;   // chunk `lane`'s first word
+    if (warp == 0) {
+        if (lane < n) a.offsets[a.chunk_base + lane] = st_lane;
         const unsigned long long end = base + __shfl_sync(0xffffffffu, incl, 31);
-        const uint32_t status = __reduce_or_sync(0xffffffffu, t.status) | (end > a.cap_words ? HQ_ST_CAPACITY : 0u);
-        const uint32_t zor = __reduce_or_sync(0xffffffffu, t.zor);
-        const unsigned long long payload = warp_sum_u64(t.payload);
+        const uint32_t status = __reduce_or_sync(0xffffffffu, mine.status) | (end > a.cap_words ? HQ_ST_CAPACITY : 0u);
+        const uint32_t zor = __reduce_or_sync(0xffffffffu, mine.zor);
+        const unsigned long long payload = warp_sum_u64(mine.payload);
         if (lane == 0) {
             a.offsets[a.chunk_base + n] = end;
             if (a.tail_out) *a.tail_out = end;
@@ -1295,11 +1292,10 @@ __device__ __forceinline__ void tiny_finish(const EncodeArgs &a, int n, const Ti
             }
         }
     }
-    __syncthreads();
 
-    for (int c = warp; c < n; c += kTinyWarps) {
+    for (int c = warp; c < n; c += kTinyWarps) {   // warp-uniform
         const TinyChunk t = info[c];
-        const unsigned long long st = start[c];
+        const unsigned long long st = __shfl_sync(0xffffffffu, st_lane, c);
         if (t.status) continue;   // outside the supported range: nothing written
         if (!t.overflow) {
             const uint32_t *stage = stage_all + c * stage_words;
@@ -1330,9 +1326,11 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tiny(const E
     uint32_t *sign_tab = smem + (ROT ? kRotSmemBytes / sizeof(uint32_t) : 0);   // tcols * kSignWords
     uint32_t *stage_all = sign_tab + a.tcols * kSignWords;                         // kMax * kStageWords
     TinyChunk *info = reinterpret_cast<TinyChunk *>(stage_all + kMax * kStageWords);
-    unsigned long long *start = reinterpret_cast<unsigned long long *>(info + kMax);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int n = (int)a.n_chunks;   // <= kMax (host)
+    // the stream's end before this call (the previous append's tail), loaded now so that its
+    // latency passes under the encoding
+    const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
 
     if (ROT)
         load_rotation<true>(rot_s, a.rot);
@@ -1426,7 +1424,7 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tiny(const E
     }
     __syncthreads();
 
-    tiny_finish<LAT, DITHER, ROT>(a, n, info, start, stage_all, kStageWords, sign_tab, rot_s);
+    tiny_finish<LAT, DITHER, ROT>(a, n, info, base, stage_all, kStageWords, sign_tab, rot_s);
 }
 
 // One-token KV appends (every chunk one tile: one token of one head), up to kTinyMaxChunks
@@ -1446,9 +1444,9 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tok(const En
     uint32_t *sign_tab = smem + (ROT ? rot_smem_bytes(kTinyWarps) / sizeof(uint32_t) : 0);   // tcols * kSignWords
     uint32_t *stage_all = sign_tab + a.tcols * kSignWords;           // kTinyMaxChunks * kTokStageWords
     TinyChunk *info = reinterpret_cast<TinyChunk *>(stage_all + kTinyMaxChunks * kTokStageWords);
-    unsigned long long *start = reinterpret_cast<unsigned long long *>(info + kTinyMaxChunks);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, l16 = lane & 15;
     const int n = (int)a.n_chunks;   // <= kTinyMaxChunks, one tile each (host)
+    const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;   // early, as in the single-CTA form
 
     if (ROT)
         load_rotation<true>(rot_s, a.rot);
@@ -1522,7 +1520,7 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tok(const En
     }
     __syncthreads();
 
-    tiny_finish<LAT, DITHER, ROT>(a, n, info, start, stage_all, kTokStageWords, sign_tab, rot_s);
+    tiny_finish<LAT, DITHER, ROT>(a, n, info, base, stage_all, kTokStageWords, sign_tab, rot_s);
 }
 
 // ------------------------------------------------------------------ rate only
