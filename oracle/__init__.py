@@ -127,6 +127,9 @@ def _bind(L):
         "hqref_quantize_tile_rot": (None, [_p, _i32, _f32, _p, _u64, _i32, _u64, _p]),
         "hqref_dequantize_tile_rot": (None, [_p, _i32, _f32, _p, _u64, _i32, _u64, _p]),
         "hqref_rot_gaussian": (C.c_double, [_u64, _u64]),
+        "hqref_code_range": (None, [_p, _i64, _p, _p]),
+        "hqref_quantize_range": (None, [_p, _i64, _i64, _i64, _i32, _f32, _u64, _i32, _i64, _i64, _p, _p]),
+        "hqref_kv_range": (None, [_p, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _u64, _i32, _p, _p, _p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -371,6 +374,41 @@ def quantize(x, lat: int, alpha: float, k: int, seed: int, dither: int = 0, chun
                               _ptr(stream), stream.size, _ptr(off), _ptr(pb), dk_last))
     assert rc == total
     return stream[:total], off, int(pb[0])
+
+
+def code_range(q):
+    """[R11] (largest |q_i|, count of q_i outside [-128, 127]) over integer codes q."""
+    a = np.ascontiguousarray(q, dtype=np.int32).ravel()
+    mx = np.zeros(1, dtype=np.uint32)
+    ov = np.zeros(1, dtype=np.uint64)
+    lib().hqref_code_range(_ptr(a), a.size, _ptr(mx), _ptr(ov))
+    return int(mx[0]), int(ov[0])
+
+
+def quantize_range(x, lat: int, alpha: float, seed: int, dither: int = 0, chunk_lo: int = 0,
+                   chunk_hi: int | None = None):
+    """[R11] code range of the weights path's codes of chunks [chunk_lo, chunk_hi)."""
+    xu = _as_u16(x)
+    R, Cc = xu.shape
+    if chunk_hi is None:
+        chunk_hi = n_chunks(R, Cc)
+    mx = np.zeros(1, dtype=np.uint32)
+    ov = np.zeros(1, dtype=np.uint64)
+    lib().hqref_quantize_range(_ptr(xu), R, Cc, Cc, lat, alpha, seed, dither, chunk_lo, chunk_hi, _ptr(mx), _ptr(ov))
+    return int(mx[0]), int(ov[0])
+
+
+def kv_range(kv, tok0: int, lat: int, alpha: float, seed: int, dither: int = 1, rot=None):
+    """[R11] code range of one KV append's codes (bf16 [H, T, 128] at token tok0)."""
+    r_keep, rp = _rot_ptr(rot)
+    x = _as_u16(kv)
+    H, T, D = x.shape
+    assert D == 128
+    mx = np.zeros(1, dtype=np.uint32)
+    ov = np.zeros(1, dtype=np.uint64)
+    lib().hqref_kv_range(_ptr(x), H, T, 128, T * 128, tok0, lat, alpha, seed, dither, rp, _ptr(mx), _ptr(ov))
+    del r_keep
+    return int(mx[0]), int(ov[0])
 
 
 def dequantize(stream, offsets, rows: int, cols: int, lat: int, alpha: float, k: int, seed: int, dither: int = 0,

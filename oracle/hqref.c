@@ -770,6 +770,46 @@ static int decode_all(const tiles_t *t, int lat, float alpha, int k, uint64_t se
     return bad ? -1 : 0;
 }
 
+/* [R11] The codes against 8-bit storage.  The pages store the lattice points'
+ * integers in 8 bits and calibrate alpha so that they do not overflow
+ * (explainer pages, "Methodology" 2, the integer implementation); the Rice
+ * code is unbounded, so nothing is clamped and the range is only reported:
+ * over the n code coordinates q (the embedding's integers, before
+ * bit-stripping), the largest |q_i| is kept in *max_abs if it is larger, and
+ * the number of q_i outside [-128, 127] is added to *overflow. */
+void hqref_code_range(const int32_t *q, int64_t n, uint32_t *max_abs, uint64_t *overflow)
+{
+    for (int64_t i = 0; i < n; i++) {
+        int64_t v = q[i];
+        uint64_t a = (uint64_t)(v < 0 ? -v : v);
+        if (a > *max_abs) *max_abs = (uint32_t)a;
+        if (v < -128 || v > 127) *overflow += 1;
+    }
+}
+
+/* The code range of every tile of chunks [chunk_lo, chunk_hi), from the same
+ * per-tile quantization as encode_all. */
+static void range_all(const tiles_t *t, int lat, float alpha, uint64_t seed, int dither, int64_t chunk_lo,
+                      int64_t chunk_hi, uint32_t *max_abs, uint64_t *overflow)
+{
+    int32_t q[128];
+    *max_abs = 0;
+    *overflow = 0;
+    for (int64_t c = chunk_lo; c < chunk_hi; c++) {
+        for (int i = 0; i < 32; i++) {
+            const uint16_t *p;
+            uint64_t scol, e0;
+            int64_t a, b;
+            if (!tile_of(t, c, i, &p, &scol, &e0, &a, &b)) break;
+            if (t->rot)
+                hqref_quantize_tile_rot(p, lat, alpha, t->rot, seed, dither, e0, q);
+            else
+                hqref_quantize_tile(p, lat, alpha, seed, scol, dither, e0, q);
+            hqref_code_range(q, 128, max_abs, overflow);
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Whole-matrix API (weights). */
 int64_t hqref_n_chunks(int64_t rows, int64_t cols)
@@ -802,6 +842,36 @@ int hqref_dequantize(const uint32_t *stream, const uint64_t *offsets, int64_t ro
     t.cols = cols;
     return decode_all(&t, lat, alpha, k, seed, dither, chunk_lo, chunk_hi, stream, offsets, out_fp32, out, ld, 0,
                       0, dk_last);
+}
+
+/* [R11] code range of a weight matrix's chunks [chunk_lo, chunk_hi). */
+void hqref_quantize_range(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int lat, float alpha,
+                          uint64_t seed, int dither, int64_t chunk_lo, int64_t chunk_hi, uint32_t *max_abs,
+                          uint64_t *overflow)
+{
+    tiles_t t = {0};
+    t.x = x;
+    t.rows = rows;
+    t.cols = cols;
+    t.ld = ld;
+    range_all(&t, lat, alpha, seed, dither, chunk_lo, chunk_hi, max_abs, overflow);
+}
+
+/* [R11] code range of one KV append (the tokens of hqref_kv_append's arguments). */
+void hqref_kv_range(const uint16_t *kv, int64_t H, int64_t T, int64_t ld_tok, int64_t ld_head, int64_t tok0,
+                    int lat, float alpha, uint64_t seed, int dither, const float *rot, uint32_t *max_abs,
+                    uint64_t *overflow)
+{
+    tiles_t t = {0};
+    t.kv = 1;
+    t.x = kv;
+    t.H = H;
+    t.T = T;
+    t.ld_tok = ld_tok;
+    t.ld_head = ld_head;
+    t.tok0 = tok0;
+    t.rot = rot;
+    range_all(&t, lat, alpha, seed, dither, 0, n_chunks_of(&t), max_abs, overflow);
 }
 
 /* KV append [R15]: the chunks of one append are written from base_word on;

@@ -59,6 +59,13 @@ void hqref_dequantize_tile_rot(const int32_t *q, int lat, float alpha, const flo
                                uint64_t e0, float *out);
 double hqref_rot_gaussian(uint64_t seed, uint64_t e);
 
+void hqref_code_range(const int32_t *q, int64_t n, uint32_t *max_abs, uint64_t *overflow);
+void hqref_quantize_range(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int lat, float alpha,
+                          uint64_t seed, int dither, int64_t chunk_lo, int64_t chunk_hi, uint32_t *max_abs,
+                          uint64_t *overflow);
+void hqref_kv_range(const uint16_t *kv, int64_t H, int64_t T, int64_t ld_tok, int64_t ld_head, int64_t tok0,
+                    int lat, float alpha, uint64_t seed, int dither, const float *rot, uint32_t *max_abs,
+                    uint64_t *overflow);
 int64_t hqref_n_chunks(int64_t rows, int64_t cols);
 int64_t hqref_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int lat, float alpha, int k,
                        uint64_t seed, int dither, int64_t chunk_lo, int64_t chunk_hi, uint32_t *stream,

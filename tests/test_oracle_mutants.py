@@ -8,6 +8,7 @@ import pytest
 
 import oracle as O
 import test_oracle_pins as P
+import test_oracle_range as PG
 import test_oracle_rice_k as PK
 import test_oracle_rotation as PR
 
@@ -66,6 +67,18 @@ MUTANTS = [
      "for (int b = 0; b < ki; b++) put_bit(rem, rpos++, (z[i] >> b) & 1u);",
      "for (int b = 0; b < ki; b++) put_bit(rem, (uint64_t)i * (uint64_t)ki + (uint64_t)b, (z[i] >> b) & 1u);",
      [lambda: PK.test_two_k_planes_hold_the_textbook_codewords(O.A2, 2, 1)]),
+    ("int8 range counts 128 as fitting", "if (v < -128 || v > 127) *overflow += 1;",
+     "if (v < -128 || v > 128) *overflow += 1;",
+     [PG.test_code_range_definition, lambda: PG.test_range_of_constant_tiles_is_closed_form(O.E8)]),
+    ("int8 range counts -128 as overflow", "if (v < -128 || v > 127) *overflow += 1;",
+     "if (v <= -128 || v > 127) *overflow += 1;",
+     [PG.test_code_range_definition, lambda: PG.test_range_of_alternating_tiles_is_closed_form(O.Z, 2)]),
+    ("range taken over the stripped symbols", "            hqref_code_range(q, 128, max_abs, overflow);",
+     "            { int32_t m[128]; uint32_t cs; for (int b = 0; b < 128; b += hqref_lattice_dim(lat))"
+     " hqref_strip(lat, q + b, m + b, &cs); hqref_code_range(m, 128, max_abs, overflow); }",
+     [lambda: PG.test_range_of_constant_tiles_is_closed_form(O.E8)]),
+    ("weights dither counter ignores the row", "*e0 = (uint64_t)(r * t->cols + tc * 128);",
+     "*e0 = (uint64_t)(tc * 128);", [PG.test_weights_dither_counter_is_row_major_element_index]),
     ("Gaussian radius from one bit too few", "double u1 = ((double)(h >> 32) + 0.5) * 0x1p-32;",
      "double u1 = ((double)(h >> 33) + 0.5) * 0x1p-32;", [PR.test_gaussian_draws_are_standard_normal]),
 ]
