@@ -115,13 +115,28 @@ typedef struct hq_params {
 } hq_params;               /* 48 bytes */
 
 /* Device-resident statistics written by the kernels (zeroed by each call
- * that takes it).  32 bytes, 8-byte aligned. */
+ * that takes it).  40 bytes, 8-byte aligned.
+ *
+ * The integer range of the codes: the pages map lattice points to an integer
+ * embedding that is meant to fit 8-bit storage, with alpha calibrated so that
+ * the codes do not overflow it (HyperQuant explainer pages, "Methodology" 2,
+ * the integer implementation).  The Rice code itself is unbounded, so nothing
+ * is clamped; the encoder reports how the call's codes sit against int8:
+ *   max_abs_code        the largest |q_i| over every code coordinate q_i of the
+ *                       call (the embedding's integers before bit-stripping:
+ *                       Z q; A2 (a, b); D4 q; E8 the 2E8 coordinates 2 m + c);
+ *   int8_overflow_count the number of code coordinates outside [-128, 127].
+ * The encoders (hq_quantize, hq_quantize_static, hq_kv_append) and the rate
+ * passes (hq_rate, hq_rate_kv, hq_calibrate*) report both; a KV cache's running
+ * stats keep the maximum and the sum over its appends.  Decoding leaves them 0. */
 typedef struct hq_stats {
     uint32_t status;       /* HQ_ST_* bits */
     uint32_t max_symbol;   /* bitwise OR of all zigzag symbols coded: its bit length bounds them */
     uint64_t payload_bits; /* sum of Rice codeword lengths plus E8 coset bits */
     uint64_t stream_words; /* words the stream needs (= offsets[n_chunks] when it fit) */
-    uint64_t reserved;
+    uint32_t max_abs_code; /* max |code coordinate| (above) */
+    uint32_t reserved;     /* 0 */
+    uint64_t int8_overflow_count; /* code coordinates outside [-128, 127] (above) */
 } hq_stats;
 
 /* One row of a KV cache's append table (device memory; written by
@@ -241,15 +256,18 @@ HQ_API int hq_gemv(const uint32_t *d_stream, uint64_t stream_words, const uint64
  * each, about 537 million elements); a larger matrix returns HQ_EUNSUPPORTED
  * and enqueues nothing.
  *
- * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array and each clears the part it uses
- * with a cudaMemsetAsync on its own stream, so calls that overlap on the GPU
- * (other streams, or other host threads, without ordering between them) race
- * and corrupt each other's streams: serialise them.  The call allocates
- * nothing: no cudaMalloc, cudaFree or allocating library routine. */
+ * Every call looks up the array's device address in the current context
+ * (cudaGetSymbolAddress, with the caller's device current), so a call made
+ * after cudaDeviceReset, or from another context, finds the array where that
+ * context has it.  The first call in a context may load the library's device
+ * code (lazy module loading): make that first call before any stream capture.
+ * All calls share the one array and each clears the part it uses with a
+ * cudaMemsetAsync on its own stream, so calls that overlap on the GPU (other
+ * streams, or other host threads, without ordering between them) race and
+ * corrupt each other's streams: serialise them.  The call allocates nothing:
+ * no cudaMalloc, cudaFree or allocating library routine. */
 #define HQ_STATIC_SCRATCH_BYTES (1u << 20)
-#define HQ_STATIC_MAX_CHUNKS 131067u
+#define HQ_STATIC_MAX_CHUNKS 131066u
 HQ_API int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p,
                               uint32_t *d_stream, uint64_t cap_words, uint64_t *d_offsets, hq_stats *d_stats,
                               void *cuda_stream);
@@ -333,7 +351,12 @@ HQ_API int hq_kv_init(hq_kv_cache *cache, int32_t heads, int32_t head_dim, const
                uint64_t cap_words, uint64_t *d_offsets, uint64_t offsets_cap, hq_kv_append_row *d_table,
                uint64_t table_cap, uint64_t *d_tail, hq_stats *d_stats, void *cuda_stream);
 
-/* Append T tokens: kv is device bf16 [H, T, 128], element (h, t, d) at
+/* Append T tokens to a compressed KV cache: the KV-cache quantizer of the pages
+ * (HyperQuant explainer pages, "Methodology" 4, KV bias correction: a
+ * per-layer rotation, here the seeded sign diagonal with H_128 or the cache's
+ * dense rotation, then the lattice quantizer with subtractive dither; sections
+ * 1-3 for the RHT, the lattice and the Rice code; arXiv abstract, step (iv)).
+ * kv is device bf16 [H, T, 128], element (h, t, d) at
  * kv[h * ld_head + t * ld_token + d] (both strides % 8 == 0).  The chunks are
  * written from the cache's device-resident tail on, so appends queue without a
  * host sync.  Dither counter of (token, head, dim) is (token * H + head) * 128
@@ -343,7 +366,10 @@ HQ_API int hq_kv_init(hq_kv_cache *cache, int32_t heads, int32_t head_dim, const
 HQ_API int hq_kv_append(hq_kv_cache *cache, const void *kv, int64_t T, int64_t ld_token, int64_t ld_head, float alpha,
                  void *workspace, size_t ws_bytes, void *cuda_stream);
 
-/* Decode the first len tokens of every head: out [H, len, 128], element
+/* Read a compressed KV cache back: the exact inverse of every append (the same
+ * pages and sections as hq_kv_append: Rice decode, re-inserted membership bits,
+ * the dither subtracted, unscaled, the inverse rotation).  Decode the first len
+ * tokens of every head: out [H, len, 128], element
  * (h, t, d) at out[h * out_ld_head + t * out_ld_token + d]; out_dtype as in
  * hq_dequantize.  len <= cache->tokens. */
 HQ_API int hq_kv_read(const hq_kv_cache *cache, void *out, int out_dtype, int64_t len, int64_t out_ld_token,

@@ -24,6 +24,7 @@ HQ_Z, HQ_A2, HQ_D4, HQ_E8 = 0, 1, 2, 3
 LATTICES = {"Z": HQ_Z, "A2": HQ_A2, "D4": HQ_D4, "E8": HQ_E8}
 HQ_OK, HQ_EINVAL, HQ_EUNSUPPORTED, HQ_ECUDA = 0, -1, -2, -3
 HQ_ST_CAPACITY, HQ_ST_CORRUPT, HQ_ST_TIMEOUT, HQ_ST_RANGE = 1, 2, 4, 8
+HQ_STATIC_MAX_CHUNKS = 131066     # include/hq.h: chunks hq_quantize_static's fixed scratch holds
 
 
 class hq_params(C.Structure):
@@ -34,7 +35,8 @@ class hq_params(C.Structure):
 
 class hq_stats(C.Structure):
     _fields_ = [("status", C.c_uint32), ("max_symbol", C.c_uint32), ("payload_bits", C.c_uint64),
-                ("stream_words", C.c_uint64), ("reserved", C.c_uint64)]
+                ("stream_words", C.c_uint64), ("max_abs_code", C.c_uint32), ("reserved", C.c_uint32),
+                ("int8_overflow_count", C.c_uint64)]
 
 
 class hq_kv_append_row(C.Structure):
@@ -59,8 +61,9 @@ class hq_calib_result(C.Structure):
                 ("status", C.c_uint32)]
 
 
+STATS_BYTES = 40
 assert C.sizeof(hq_calib_spec) == 48 and C.sizeof(hq_calib_result) == 24
-assert C.sizeof(hq_params) == 48 and C.sizeof(hq_stats) == 32 and C.sizeof(hq_kv_append_row) == 32
+assert C.sizeof(hq_params) == 48 and C.sizeof(hq_stats) == STATS_BYTES and C.sizeof(hq_kv_append_row) == 32
 assert C.sizeof(hq_kv_cache) == 144
 
 # C entry points: name -> (restype, argtypes)
@@ -279,7 +282,7 @@ def hq_workspace_bytes(n_chunks: int) -> int:
 def hq_quantize(x: torch.Tensor, params: hq_params, stream: torch.Tensor, offsets: torch.Tensor,
                 stats: torch.Tensor | None, workspace: torch.Tensor, cuda_stream=None, ld: int | None = None) -> int:
     """x: bf16 [rows, cols] (row stride ld, default x.stride(0)); stream: int32/uint32 words;
-    offsets: int64 [n_chunks + 1]; stats: uint8 [32] or None; workspace: uint8."""
+    offsets: int64 [n_chunks + 1]; stats: uint8 [STATS_BYTES] or None; workspace: uint8."""
     rows, cols = x.shape
     ld = x.stride(0) if ld is None else ld
     return _check(_lib.hq_quantize(_ptr(x), rows, cols, ld, C.byref(params), _ptr(stream), stream.numel(),
@@ -333,14 +336,15 @@ def hq_kv_read(cache: hq_kv_cache, out: torch.Tensor, length: int, cuda_stream=N
 
 # ------------------------------------------------------------------ torch-allocated wrappers
 def stats_tensor(device="cuda") -> torch.Tensor:
-    return torch.zeros(32, dtype=torch.uint8, device=device)
+    return torch.zeros(STATS_BYTES, dtype=torch.uint8, device=device)
 
 
 def read_stats(t: torch.Tensor) -> dict:
     b = bytes(t.cpu().numpy().tobytes())
     s = hq_stats.from_buffer_copy(b)
     return {"status": s.status, "max_symbol": s.max_symbol, "payload_bits": s.payload_bits,
-            "stream_words": s.stream_words}
+            "stream_words": s.stream_words, "max_abs_code": s.max_abs_code,
+            "int8_overflow_count": s.int8_overflow_count}
 
 
 @dataclass
@@ -351,7 +355,7 @@ class Compressed:
     rows: int
     cols: int
     params: hq_params
-    stats: torch.Tensor      # uint8 [32] hq_stats
+    stats: torch.Tensor      # uint8 [STATS_BYTES] hq_stats
 
 
 class Codec:

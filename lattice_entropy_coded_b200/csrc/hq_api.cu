@@ -12,14 +12,14 @@ using namespace hq;
 
 namespace hq {
 int g_encode_path = 0;
-}
 
 namespace {
-
 constexpr int64_t kMaxCols = 65536;  // the shared sign table holds cols / 128 columns
 uint32_t g_spin_limit = kSpinLimit;
-
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+}  // namespace
+
+uint32_t spin_limit() { return g_spin_limit; }
 
 int check_params(const hq_params *p) {
     if (!p) return HQ_EINVAL;
@@ -80,6 +80,10 @@ void set_scratch(EncodeArgs &a, void *ws, uint64_t nch) {
     a.done = (unsigned int *)(b + nch * 8 + 4);
     a.acc = (hq_stats *)(b + nch * 8 + 8);
 }
+
+}  // namespace hq
+
+namespace {
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ECUDA; }
 

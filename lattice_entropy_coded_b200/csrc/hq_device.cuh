@@ -327,8 +327,9 @@ template <int LAT> struct Lattice;
 template <> struct Lattice<HQ_Z> {
     static constexpr int N = 1;
     __device__ static __forceinline__ void nearest(const float (&v)[1], int32_t (&q)[1]) { q[0] = rint_int(v[0]); }
-    __device__ static __forceinline__ uint32_t symbols(const float (&v)[1], uint32_t (&z)[1]) {
+    __device__ static __forceinline__ uint32_t symbols(const float (&v)[1], uint32_t (&z)[1], uint32_t &key) {
         z[0] = zigzag(rint_int(v[0]));
+        key = max(key, z[0]);
         return 0;
     }
     __device__ static __forceinline__ void point(const int32_t (&q)[1], float (&p)[1]) { p[0] = (float)q[0]; }
@@ -353,13 +354,14 @@ template <> struct Lattice<HQ_D4> {
 #pragma unroll
         for (int i = 0; i < 4; i++) q[i] = rint_int(f[i]);
     }
-    __device__ static __forceinline__ uint32_t symbols(const float (&v)[4], uint32_t (&z)[4]) {
+    __device__ static __forceinline__ uint32_t symbols(const float (&v)[4], uint32_t (&z)[4], uint32_t &key) {
         int32_t q[4];
         nearest(v, q);
         z[0] = zigzag(q[0]);
         z[1] = zigzag(q[1]);
         z[2] = zigzag(q[2]);
         z[3] = zigzag((q[3] - ((q[0] + q[1] + q[2]) & 1)) >> 1);
+        key = max(max(key, max(z[0], z[1])), max(z[2], zigzag(q[3])));
         return 0;
     }
     __device__ static __forceinline__ void point(const int32_t (&q)[4], float (&p)[4]) {
@@ -397,11 +399,12 @@ template <> struct Lattice<HQ_A2> {
         q[0] = odd ? c1a : c0a;
         q[1] = odd ? c1b : c0b;
     }
-    __device__ static __forceinline__ uint32_t symbols(const float (&u)[2], uint32_t (&z)[2]) {
+    __device__ static __forceinline__ uint32_t symbols(const float (&u)[2], uint32_t (&z)[2], uint32_t &key) {
         int32_t q[2];
         nearest(u, q);
         z[0] = zigzag(q[0]);
         z[1] = zigzag((q[1] - (q[0] & 1)) >> 1);
+        key = max(key, max(z[0], zigzag(q[1])));
         return 0;
     }
     __device__ static __forceinline__ float box(int i) { return (i & 1) ? HQ_SQRT3 : 1.0f; }
@@ -518,13 +521,18 @@ template <> struct Lattice<HQ_E8> {
 #pragma unroll
         for (int i = 0; i < 8; i++) q[i] = 2 * m[i] + c;
     }
-    __device__ static __forceinline__ uint32_t symbols(const float (&v)[8], uint32_t (&z)[8]) {
+    __device__ static __forceinline__ uint32_t symbols(const float (&v)[8], uint32_t (&z)[8], uint32_t &key) {
         int32_t m[8];
         const uint32_t c = nearest_d8(v, m);
         const int32_t s = m[0] + m[1] + m[2] + m[3] + m[4] + m[5] + m[6];
+        const uint32_t z7 = zigzag(m[7]);   // before the strip: the code q_7 = 2 m_7 + c
         m[7] = (m[7] - (s & 1)) >> 1;
 #pragma unroll
         for (int i = 0; i < 8; i++) z[i] = zigzag(m[i]);
+        // |2 m + c| is z + ((z ^ c) & 1) with z = zigzag(m): nondecreasing in z for a fixed c,
+        // so the block's largest |code| comes from its largest zigzag value
+        const uint32_t zm = max(max(max(z[0], z[1]), max(z[2], z[3])), max(max(z[4], z[5]), max(z[6], z7)));
+        key = max(key, zm + ((zm ^ c) & 1u));
         return c;
     }
     __device__ static __forceinline__ float box(int) { return 4.0f; }
@@ -563,6 +571,50 @@ __device__ __forceinline__ void e8_codes_from_symbols(const uint32_t (&z)[8], ui
     }
     const uint32_t t7 = z[7] ^ (0u - (z[7] & 1u));
     q[7] = (int32_t)((t7 << 1) | (x & 2u) | c);
+}
+
+// ------------------------------------------------------------------ integer range of the codes
+// The pages store the embedding's integers in 8 bits, with alpha chosen so that they fit
+// (explainer pages, "Methodology" 2, the integer implementation); the encoders report the
+// largest |code coordinate| and the number of coordinates outside [-128, 127].  symbols()
+// keeps a per-lattice key of the largest |code|: E8 the value itself; Z, A2, D4 the zigzag
+// value of the code coordinate, from which |q| = (key + 1) >> 1, and a coordinate lies
+// outside int8 exactly when its zigzag value is 256 or more.
+template <int LAT>
+__device__ __forceinline__ uint32_t code_abs_of_key(uint32_t key) {
+    return LAT == HQ_E8 ? key : (key >> 1) + (key & 1u);
+}
+// A key at or above this may hide a coordinate outside int8 (E8: |q| = 128 is fine for q = -128).
+template <int LAT>
+__device__ __forceinline__ uint32_t key_int8_limit() {
+    return LAT == HQ_E8 ? 128u : 256u;
+}
+
+// Code coordinates outside [-128, 127] among S symbols (S / N whole lattice blocks, E8 coset
+// bits in cbits, bit b for block b), rebuilt from the symbols.  The rare path: taken only when
+// a key reached key_int8_limit.
+template <int LAT, int S>
+__device__ __forceinline__ uint32_t int8_overflow(const uint32_t (&z)[S], uint32_t cbits) {
+    constexpr int N = Lattice<LAT>::N;
+    uint32_t n = 0;
+#pragma unroll
+    for (int b = 0; b < S / N; b++) {
+        int32_t q[N];
+        if constexpr (LAT == HQ_E8) {
+            uint32_t zb[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) zb[i] = z[8 * b + i];
+            e8_codes_from_symbols(zb, (cbits >> b) & 1u, q);
+        } else {
+            int32_t m[N];
+#pragma unroll
+            for (int i = 0; i < N; i++) m[i] = unzigzag(z[N * b + i]);
+            Lattice<LAT>::reinsert(m, 0u, q);
+        }
+#pragma unroll
+        for (int i = 0; i < N; i++) n += ((uint32_t)(q[i] + 128) > 255u) ? 1u : 0u;
+    }
+    return n;
 }
 
 // ------------------------------------------------------------------ dither

@@ -109,18 +109,35 @@ __device__ __noinline__ unsigned long long lookback_resolve(unsigned long long *
     return excl;
 }
 
+// A lane's integer range of the codes it has produced: the largest code key (see
+// code_abs_of_key) and the count of code coordinates outside int8, which is taken
+// from the symbols only when a round's key reaches key_int8_limit (rare).
+struct CodeRange {
+    uint32_t key = 0, ovf = 0;
+    template <int LAT, int S>
+    __device__ __forceinline__ void add(uint32_t rkey, const uint32_t (&z)[S], uint32_t cbits) {
+        key = max(key, rkey);
+        if (rkey >= key_int8_limit<LAT>()) ovf += int8_overflow<LAT, S>(z, cbits);
+    }
+};
+
 // Stats of an encode call.  Every warp adds its part to the workspace accumulator
 // (the warp's payload is lane 0's; the accumulator is cleared with the look-back
 // words, so the caller's stats need no separate clearing); the last CTA to finish moves the totals to the caller's stats,
 // replacing them (hq_quantize) or adding to them (a KV cache's running stats).
+template <int LAT>
 __device__ __forceinline__ void stats_add_warp(const EncodeArgs &a, uint32_t status, uint32_t zor_all,
-                                               unsigned long long payload) {
+                                               unsigned long long payload, const CodeRange &rng) {
     status = __reduce_or_sync(0xffffffffu, status);
     zor_all = __reduce_or_sync(0xffffffffu, zor_all);
+    const uint32_t key = __reduce_max_sync(0xffffffffu, rng.key);
+    const uint32_t ovf = __reduce_add_sync(0xffffffffu, rng.ovf);
     if ((threadIdx.x & 31) == 0) {
         if (status) atomicOr(&a.acc->status, status);
         if (zor_all) atomicOr(&a.acc->max_symbol, zor_all);
         if (payload) atomicAdd((unsigned long long *)&a.acc->payload_bits, payload);
+        if (key) atomicMax(&a.acc->max_abs_code, code_abs_of_key<LAT>(key));
+        if (ovf) atomicAdd((unsigned long long *)&a.acc->int8_overflow_count, (unsigned long long)ovf);
     }
 }
 
@@ -135,14 +152,21 @@ __device__ __forceinline__ void stats_finish_cta(const EncodeArgs &a) {
     const uint32_t st = ld_relaxed_u32(&a.acc->status), mx = ld_relaxed_u32(&a.acc->max_symbol);
     const unsigned long long pb = ld_relaxed_u64((const unsigned long long *)&a.acc->payload_bits);
     const unsigned long long sw = ld_relaxed_u64((const unsigned long long *)&a.acc->stream_words);
+    const uint32_t am = ld_relaxed_u32(&a.acc->max_abs_code);
+    const unsigned long long ov = ld_relaxed_u64((const unsigned long long *)&a.acc->int8_overflow_count);
     if (a.stats_add) {
         if (st) atomicOr(&a.stats->status, st);
         if (mx) atomicOr(&a.stats->max_symbol, mx);
         if (pb) atomicAdd((unsigned long long *)&a.stats->payload_bits, pb);
+        if (am) atomicMax(&a.stats->max_abs_code, am);
+        if (ov) atomicAdd((unsigned long long *)&a.stats->int8_overflow_count, ov);
     } else {
         a.stats->status = st;
         a.stats->max_symbol = mx;
         a.stats->payload_bits = pb;
+        a.stats->max_abs_code = am;
+        a.stats->reserved = 0u;
+        a.stats->int8_overflow_count = ov;
     }
     a.stats->stream_words = sw;
 }
@@ -272,11 +296,12 @@ __device__ __forceinline__ void round_transform(const RoundInput &in, const uint
 }
 
 // One round for one lane: the transform -> * c -> [+ d] -> lattice blocks -> 32
-// zigzag symbols and the E8 coset bits of its blocks.  Whole warp must call it.
+// zigzag symbols, the E8 coset bits of its blocks and the largest code key of the
+// round (0 for an invalid tile).  Whole warp must call it.
 template <int LAT, bool DITHER, bool ROT = false>
 __device__ __forceinline__ void round_symbols(const EncodeArgs &a, const RoundInput &in, const uint4 (&raw)[4],
                                               int lane, const uint32_t *sign_tab, uint32_t (&z)[32],
-                                              uint32_t &cbits, const float *rot_s = nullptr) {
+                                              uint32_t &cbits, uint32_t &rkey, const float *rot_s = nullptr) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
     const int q = lane & 3;
@@ -287,6 +312,7 @@ __device__ __forceinline__ void round_symbols(const EncodeArgs &a, const RoundIn
     for (int j = 0; j < 16; j++) v[j] = f2_mul(v[j], c2);
 
     cbits = 0;
+    rkey = 0;
     const unsigned long long eq = in.e0 + 32ull * q;
 #pragma unroll
     for (int b = 0; b < 32 / N; b++) {
@@ -303,11 +329,12 @@ __device__ __forceinline__ void round_symbols(const EncodeArgs &a, const RoundIn
             for (int i = 0; i < N; i++) blk[i] = __fadd_rn(blk[i], d[i]);
         }
         uint32_t zz[N];
-        cbits |= L::symbols(blk, zz) << b;
+        cbits |= L::symbols(blk, zz, rkey) << b;
 #pragma unroll
         for (int i = 0; i < N; i++) z[b * N + i] = (!DITHER || in.valid) ? zz[i] : 0u;
     }
     if (!in.valid) cbits = 0;
+    if (!in.valid) rkey = 0;
 }
 
 // N consecutive floats of a lane's shared row (16-byte aligned rows; offsets are
@@ -350,12 +377,13 @@ __device__ __forceinline__ void row_store(uint32_t *r, const uint32_t (&z)[N]) {
 // (the 32 transformed values, then their symbols in place): one copy of the block
 // code instead of 32/N.  For the latency form, where each warp runs a round once
 // and fetching the unrolled code from a cold instruction cache, not issue, bounds
-// it.  Leaves the 32 symbols in row[0, 32) and their quotient sum and OR.
+// it.  Leaves the 32 symbols in row[0, 32), their quotient sum and OR, and the largest
+// code key of the round (0 for an invalid tile).
 template <int LAT, bool DITHER, bool ROT>
 __device__ __forceinline__ void round_symbols_rolled(const EncodeArgs &a, const RoundInput &in, const uint4 (&raw)[4],
                                                      int lane, const uint32_t *sign_tab, uint32_t *row,
                                                      uint32_t &cbits, uint32_t &usum, uint32_t &lor,
-                                                     const float *rot_s) {
+                                                     uint32_t &rkey, const float *rot_s) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
     const int q = lane & 3;
@@ -370,6 +398,7 @@ __device__ __forceinline__ void round_symbols_rolled(const EncodeArgs &a, const 
     cbits = 0;
     usum = 0;
     lor = 0;
+    rkey = 0;
     const int k = a.k, kl = a.k_last;
     const unsigned long long eq = in.e0 + 32ull * q;
 #pragma unroll 1
@@ -383,7 +412,7 @@ __device__ __forceinline__ void round_symbols_rolled(const EncodeArgs &a, const 
             for (int i = 0; i < N; i++) blk[i] = __fadd_rn(blk[i], d[i]);
         }
         uint32_t zz[N];
-        cbits |= L::symbols(blk, zz) << b;
+        cbits |= L::symbols(blk, zz, rkey) << b;
 #pragma unroll
         for (int i = 0; i < N; i++) {
             zz[i] = (!DITHER || in.valid) ? zz[i] : 0u;
@@ -393,6 +422,7 @@ __device__ __forceinline__ void round_symbols_rolled(const EncodeArgs &a, const 
         row_store<N>(row + b * N, zz);
     }
     if (!in.valid) cbits = 0;
+    if (!in.valid) rkey = 0;
 }
 
 // Remainder bits of 32 symbols (warp-uniform k) into the lane's k words.
@@ -529,7 +559,8 @@ __device__ __noinline__ void encode_chunk_global(const EncodeArgs &a, const Chun
             for (int j = 0; j < 4; j++)
                 raw[j] = in.valid ? ldg_nc_v4(src + 32 * (lane & 3) + 8 * j) : make_uint4(0, 0, 0, 0);
         }
-        round_symbols<LAT, DITHER, ROT>(a, in, raw, lane, sign_tab, z, cbits, rot_s);
+        uint32_t rkey;   // counted when the chunk was first encoded
+        round_symbols<LAT, DITHER, ROT>(a, in, raw, lane, sign_tab, z, cbits, rkey, rot_s);
         const bool valid = in.valid;
         unsigned long long ub = 0;
 #pragma unroll
@@ -635,6 +666,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
     uint32_t status = 0, zor_all = 0;
     unsigned long long payload = 0;
+    CodeRange rng;
 
     unsigned long long c = take_ticket(a);
     if (c < a.n_chunks) {
@@ -682,8 +714,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
                 prefetch_round(a, gn, 0, lane, slot);
             }
 
-            uint32_t z[32], cbits;
-            round_symbols<LAT, DITHER>(a, cur, raw, lane, sign_tab, z, cbits);
+            uint32_t z[32], cbits, rkey;
+            round_symbols<LAT, DITHER>(a, cur, raw, lane, sign_tab, z, cbits, rkey);
+            rng.add<LAT>(rkey, z, cbits);
             const bool valid = cur.valid;
             uint32_t usum = 0, lor = 0;
 #pragma unroll
@@ -744,7 +777,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     if (have_pend) finish_chunk_warp<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 
-    stats_add_warp(a, status, zor_all, payload);
+    stats_add_warp<LAT>(a, status, zor_all, payload, rng);
     stats_finish_cta(a);
 }
 
@@ -857,6 +890,7 @@ __global__ void __launch_bounds__((ROT ? kRotGroups : kGroups) * kGroupWarps * 3
     const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
     uint32_t status = 0, zor_all = 0;
     unsigned long long payload = 0;
+    CodeRange rng;
     unsigned long long c = ctl.first[0], cn = ctl.first[1];
     if (c < n) {
         ChunkGeo g0;
@@ -874,7 +908,7 @@ __global__ void __launch_bounds__((ROT ? kRotGroups : kGroups) * kGroupWarps * 3
         if (!live && have_pend && duty) first = lookback_peek(a.lookback, pend.c);
         uint32_t *stage = stages + buf * kStageWords;
         ChunkGeo geo;
-        uint32_t z[32], cbits = 0, ub = 0, incl = 0;
+        uint32_t z[32], cbits = 0, ub = 0, incl = 0, rkey = 0;
         bool valid = false;
         if (live) {
             geo.init(a.map, c);
@@ -888,7 +922,8 @@ __global__ void __launch_bounds__((ROT ? kRotGroups : kGroups) * kGroupWarps * 3
             if (have_pend && duty) first = lookback_peek(a.lookback, pend.c);
             // the symbols are left in the lane's slot, where they wait while the group meets
             uint32_t usum, lor;
-            round_symbols_rolled<LAT, DITHER, ROT>(a, cur, raw, lane, sign_tab, slot, cbits, usum, lor, rot_s);
+            round_symbols_rolled<LAT, DITHER, ROT>(a, cur, raw, lane, sign_tab, slot, cbits, usum, lor, rkey,
+                                                   rot_s);
             valid = cur.valid;
             zor_all |= lor;
             ub = valid ? usum + 32u : 0u;
@@ -935,6 +970,7 @@ __global__ void __launch_bounds__((ROT ? kRotGroups : kGroups) * kGroupWarps * 3
                 z[4 * j + 2] = t.z;
                 z[4 * j + 3] = t.w;
             }
+            rng.add<LAT>(rkey, z, cbits);
             if (cn < n) {
                 ChunkGeo gn;
                 gn.init(a.map, cn);
@@ -982,7 +1018,7 @@ __global__ void __launch_bounds__((ROT ? kRotGroups : kGroups) * kGroupWarps * 3
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 
-    stats_add_warp(a, status, zor_all, payload);
+    stats_add_warp<LAT>(a, status, zor_all, payload, rng);
     stats_finish_cta(a);
 }
 
@@ -1009,11 +1045,13 @@ __device__ __forceinline__ void wide_sync() {
 
 // A lane's 8 elements of its tile: signs, FWHT-128 with its 15 partner lanes (or with
 // ROT the dense rotation, rot_s its shared form and xs the warp's 256-float buffer),
-// scale, [+ dither], lattice blocks -> 8 zigzag symbols and (E8) the coset bit.
+// scale, [+ dither], lattice blocks -> 8 zigzag symbols, (E8) the coset bit and the
+// largest code key (0 for an invalid tile).
 template <int LAT, bool DITHER, bool ROT = false>
 __device__ __forceinline__ void wide_symbols(const EncodeArgs &a, bool valid, int tcol, unsigned long long e0,
                                              uint4 raw, int lane, const uint32_t *sign_tab, uint32_t (&z)[8],
-                                             uint32_t &cbit, const float *rot_s = nullptr, float *xs = nullptr) {
+                                             uint32_t &cbit, uint32_t &rkey, const float *rot_s = nullptr,
+                                             float *xs = nullptr) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
     const int l16 = lane & 15;
@@ -1039,6 +1077,7 @@ __device__ __forceinline__ void wide_symbols(const EncodeArgs &a, bool valid, in
     for (int t = 0; t < 4; t++) v[t] = f2_mul(v[t], c2);
     const float x[8] = {v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y};
     cbit = 0;
+    rkey = 0;
     const unsigned long long eq = e0 + 8ull * l16;
 #pragma unroll
     for (int b = 0; b < 8 / N; b++) {
@@ -1052,11 +1091,12 @@ __device__ __forceinline__ void wide_symbols(const EncodeArgs &a, bool valid, in
             for (int i = 0; i < N; i++) blk[i] = __fadd_rn(blk[i], d[i]);
         }
         uint32_t zz[N];
-        cbit |= L::symbols(blk, zz);
+        cbit |= L::symbols(blk, zz, rkey) << b;
 #pragma unroll
         for (int i = 0; i < N; i++) z[b * N + i] = (!DITHER || valid) ? zz[i] : 0u;
     }
     if (!valid) cbit = 0;
+    if (!valid) rkey = 0;
 }
 
 // k remainder bits of 8 symbols into the remainder plane at bit `off` (any
@@ -1110,6 +1150,7 @@ __global__ void __launch_bounds__(kWideWarps * 32, 1) encode_kernel_wide(const E
     const int ti = 2 * w + (lane >> 4);          // the lane's tile in the chunk
     uint32_t status = 0, zor_all = 0;
     unsigned long long payload = 0;
+    CodeRange rng;
     unsigned long long c = ctl.first[0], cn = ctl.first[1];
     // the next chunk's 16 bytes are loaded one iteration ahead
     uint4 raw_next = make_uint4(0, 0, 0, 0);
@@ -1151,7 +1192,9 @@ __global__ void __launch_bounds__(kWideWarps * 32, 1) encode_kernel_wide(const E
                                                                 : make_uint4(0, 0, 0, 0);
             }
             if (threadIdx.x == 0) ctl.tk[buf] = atomicAdd(a.ticket, 1u);
-            wide_symbols<LAT, DITHER>(a, valid, tcol, e0, raw, lane, sign_tab, z, cbit);
+            uint32_t rkey;
+            wide_symbols<LAT, DITHER>(a, valid, tcol, e0, raw, lane, sign_tab, z, cbit, rkey);
+            rng.add<LAT>(rkey, z, cbit);
             uint32_t usum = 0, lor = 0;
 #pragma unroll
             for (int i = 0; i < 8; i++) {
@@ -1225,7 +1268,7 @@ __global__ void __launch_bounds__(kWideWarps * 32, 1) encode_kernel_wide(const E
         it++;
     }
 
-    stats_add_warp(a, status, zor_all, payload);
+    stats_add_warp<LAT>(a, status, zor_all, payload, rng);
     stats_finish_cta(a);
 }
 
@@ -1247,6 +1290,7 @@ struct TinyChunk {
     uint32_t overflow;   // larger than its stage: set in place after the scan
     uint32_t zor;
     unsigned long long payload;
+    uint32_t key, ovf;   // the chunk's integer range of the codes (CodeRange)
 };
 
 // The single-CTA forms' last steps, after a barrier that publishes info[]: every warp
@@ -1260,7 +1304,7 @@ __device__ __forceinline__ void tiny_finish(const EncodeArgs &a, int n, const Ti
                                             const uint32_t *sign_tab, const float *rot_s) {
     constexpr int N = Lattice<LAT>::N;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const TinyChunk mine = lane < n ? info[lane] : TinyChunk{0u, 0u, 0u, 0u, 0ull};
+    const TinyChunk mine = lane < n ? info[lane] : TinyChunk{0u, 0u, 0u, 0u, 0ull, 0u, 0u};
     unsigned long long incl = mine.total;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -1274,6 +1318,8 @@ __device__ __forceinline__ void tiny_finish(const EncodeArgs &a, int n, const Ti
         const uint32_t status = __reduce_or_sync(0xffffffffu, mine.status) | (end > a.cap_words ? HQ_ST_CAPACITY : 0u);
         const uint32_t zor = __reduce_or_sync(0xffffffffu, mine.zor);
         const unsigned long long payload = warp_sum_u64(mine.payload);
+        const uint32_t am = code_abs_of_key<LAT>(__reduce_max_sync(0xffffffffu, mine.key));
+        const unsigned long long ovf = warp_sum_u64(mine.ovf);
         if (lane == 0) {
             a.offsets[a.chunk_base + n] = end;
             if (a.tail_out) *a.tail_out = end;
@@ -1283,10 +1329,15 @@ __device__ __forceinline__ void tiny_finish(const EncodeArgs &a, int n, const Ti
                     if (status) atomicOr(&a.stats->status, status);
                     if (zor) atomicOr(&a.stats->max_symbol, zor);
                     if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
+                    if (am) atomicMax(&a.stats->max_abs_code, am);
+                    if (ovf) atomicAdd((unsigned long long *)&a.stats->int8_overflow_count, ovf);
                 } else {
                     a.stats->status = status;
                     a.stats->max_symbol = zor;
                     a.stats->payload_bits = payload;
+                    a.stats->max_abs_code = am;
+                    a.stats->reserved = 0u;
+                    a.stats->int8_overflow_count = ovf;
                 }
                 a.stats->stream_words = end;
             }
@@ -1352,6 +1403,7 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tiny(const E
         const uint32_t rbits = (uint32_t)ntiles * tile_rem_bits<N>(k, kl);
         const uint32_t nr = (rbits + 31u) >> 5;
         uint32_t urun = 0, zor = 0;
+        CodeRange rng;
         bool overflow = (nc + nr) > (uint32_t)kStageWords, range_bad = false;
 #pragma unroll 1
         for (int r = 0; r < nrounds; r++) {
@@ -1367,8 +1419,9 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tiny(const E
                 for (int j = 0; j < 4; j++)
                     raw[j] = in.valid ? ldg_nc_v4(src + 32 * (lane & 3) + 8 * j) : make_uint4(0, 0, 0, 0);
             }
-            uint32_t z[32], cbits;
-            round_symbols<LAT, DITHER, ROT>(a, in, raw, lane, sign_tab, z, cbits, rot_s);
+            uint32_t z[32], cbits, rkey;
+            round_symbols<LAT, DITHER, ROT>(a, in, raw, lane, sign_tab, z, cbits, rkey, rot_s);
+            rng.add<LAT>(rkey, z, cbits);
             const bool valid = in.valid;
             uint32_t usum = 0, lor = 0;
 #pragma unroll
@@ -1411,8 +1464,12 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tiny(const E
             urun += rtot;
         }
         zor = __reduce_or_sync(0xffffffffu, zor);
+        const uint32_t ckey = __reduce_max_sync(0xffffffffu, rng.key);
+        const uint32_t covf = __reduce_add_sync(0xffffffffu, rng.ovf);
         if (lane == 0) {
             TinyChunk t;
+            t.key = ckey;
+            t.ovf = covf;
             t.total = nc + nr + (uint32_t)(((unsigned long long)urun + 31) / 32);
             t.status = range_bad ? HQ_ST_RANGE : 0u;
             t.overflow = overflow ? 1u : 0u;
@@ -1474,8 +1531,10 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tok(const En
             valid = geo.tile(a.map, a.x, 0, src, tcol, e0);
         }
         const uint4 raw = valid ? ldg_nc_v4(src + 8 * l16) : make_uint4(0, 0, 0, 0);
-        uint32_t z[8], cbit;
-        wide_symbols<LAT, DITHER, ROT>(a, valid, tcol, e0, raw, lane, sign_tab, z, cbit, rot_s, xs);
+        uint32_t z[8], cbit, rkey;
+        wide_symbols<LAT, DITHER, ROT>(a, valid, tcol, e0, raw, lane, sign_tab, z, cbit, rkey, rot_s, xs);
+        CodeRange rng;
+        rng.add<LAT>(rkey, z, cbit);
         uint32_t usum = 0, hz = 0;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
@@ -1491,7 +1550,11 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tok(const En
         }
         const uint32_t U = __shfl_sync(0xffffffffu, incl, lane | 15);
 #pragma unroll
-        for (int o = 8; o; o >>= 1) hz |= __shfl_xor_sync(0xffffffffu, hz, o);
+        for (int o = 8; o; o >>= 1) {
+            hz |= __shfl_xor_sync(0xffffffffu, hz, o);
+            rng.key = max(rng.key, __shfl_xor_sync(0xffffffffu, rng.key, o));
+            rng.ovf += __shfl_xor_sync(0xffffffffu, rng.ovf, o);
+        }
         const bool range_bad = (hz >> 22) != 0u || U >= kMaxUnaryBits;
         const uint32_t total = nc + nr + (U + 31u) / 32u;
         const bool overflow = total > (uint32_t)kTokStageWords;
@@ -1515,6 +1578,8 @@ __global__ void __launch_bounds__(kTinyWarps * 32, 1) encode_kernel_tok(const En
             t.overflow = overflow ? 1u : 0u;
             t.zor = hz;
             t.payload = U + 128ull * (unsigned long long)k + ((LAT == HQ_E8) ? 16ull : 0ull);
+            t.key = rng.key;
+            t.ovf = rng.ovf;
             info[c] = t;
         }
     }
@@ -1544,6 +1609,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) rate_kernel(co
     const unsigned long long nwarps = (unsigned long long)gridDim.x * kWarpsPerCta;
     unsigned long long payload = 0, words = 0;
     uint32_t status = 0, zor_all = 0;
+    CodeRange rng;
     for (unsigned long long c = (unsigned long long)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); c < a.n_chunks;
          c += nwarps) {
         ChunkGeo geo;
@@ -1562,8 +1628,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) rate_kernel(co
 #pragma unroll
             for (int j = 0; j < 4; j++)
                 raw[j] = in.valid ? ldg_nc_v4(src + 32 * (lane & 3) + 8 * j) : make_uint4(0, 0, 0, 0);
-            uint32_t z[32], cbits;
-            round_symbols<LAT, DITHER, ROT>(a, in, raw, lane, sign_tab, z, cbits, rot_s);
+            uint32_t z[32], cbits, rkey;
+            round_symbols<LAT, DITHER, ROT>(a, in, raw, lane, sign_tab, z, cbits, rkey, rot_s);
+            rng.add<LAT>(rkey, z, cbits);
             uint32_t usum = 0;
 #pragma unroll
             for (int i = 0; i < 32; i++) {
@@ -1585,11 +1652,15 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, ROT ? 1 : 2) rate_kernel(co
         words += nc + nr + (U + 31) / 32;
         if ((lor >> 22) != 0u || U >= kMaxUnaryBits) status |= HQ_ST_RANGE;
     }
+    const uint32_t key = __reduce_max_sync(0xffffffffu, rng.key);
+    const uint32_t ovf = __reduce_add_sync(0xffffffffu, rng.ovf);
     if (lane == 0) {
         if (status) atomicOr(&a.stats->status, status);
         if (zor_all) atomicOr(&a.stats->max_symbol, zor_all);
         if (payload) atomicAdd((unsigned long long *)&a.stats->payload_bits, payload);
         if (words) atomicAdd((unsigned long long *)&a.stats->stream_words, words);
+        if (key) atomicMax(&a.stats->max_abs_code, code_abs_of_key<LAT>(key));
+        if (ovf) atomicAdd((unsigned long long *)&a.stats->int8_overflow_count, (unsigned long long)ovf);
     }
 }
 

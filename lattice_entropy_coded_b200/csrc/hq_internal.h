@@ -135,6 +135,17 @@ struct LaunchPlan {
     }
 };
 
+// Host-side argument checks and launch values shared by the entry points (hq_api.cu,
+// hq_static.cu), so that every entry point applies the same rules.
+int check_params(const hq_params *p);          // HQ_OK, HQ_EINVAL or HQ_EUNSUPPORTED
+int check_weight_params(const hq_params *p);   // check_params, and no dense rotation
+int check_matrix(int64_t rows, int64_t cols);  // cols % 128, cols <= 65536, rows * cols <= 2^40
+uint64_t chunks_of(int64_t rows, int64_t cols);
+int k_last_of(const hq_params &p);             // Rice parameter of the last symbol of a block
+float scale_fwd(float alpha);                  // fp32(alpha / sqrt(128))
+void set_scratch(EncodeArgs &a, void *ws, uint64_t nch);   // look-back, ticket, done, stats pointers
+uint32_t spin_limit();                         // look-back polls (hq_debug_set_spin_limit)
+
 // Encoder form: 0 = by size (one CTA for a few chunks, then wide, then grouped, for
 // launches of fewer chunks than the per-warp form has resident warps, per-warp otherwise), 1 =
 // per-warp, 2 = grouped (4 warps per chunk), 3 = wide (16 warps per chunk, 16 lanes

@@ -1,16 +1,17 @@
 // hq_static.cu -- hq_quantize_static: the weights-path quantize + encode for
 // callers that cannot allocate device memory.  The encoder's scratch (the
-// chunk look-back words and the chunk ticket) lives in a fixed array that is
-// part of this library's device image instead of in a caller workspace.
+// chunk look-back words, the chunk ticket and done counter, the stats
+// accumulator) lives in a fixed array that is part of this library's device
+// image instead of in a caller workspace.
 //
-// The array is a host-side stand-in in host code: its address on a device is
-// obtained once per device with cudaGetSymbolAddress (with that device
-// current) and cached; kernels receive that device address.
+// In host code the array's name is a host-side stand-in, not a device address:
+// every call asks the runtime for the array's address in the current context
+// (cudaGetSymbolAddress, with the caller's device current) and passes that to
+// the kernels.  Asking on every call, rather than caching per device, keeps the
+// address right after a cudaDeviceReset or in another context on the same device.
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
-
-#include <mutex>
 
 #include "hq_internal.h"
 
@@ -19,26 +20,15 @@ using namespace hq;
 namespace {
 
 constexpr size_t kStaticScratchBytes = HQ_STATIC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 // Look-back words (8 bytes per chunk), the ticket and done words, the stats accumulator.
 static __device__ __align__(256) unsigned char g_hq_scratch[kStaticScratchBytes];
 
-std::mutex g_mu;
-void *g_addr[kMaxDevices];   // device address of g_hq_scratch per device, null until set up
-
-// Device address of the scratch on the current device (set up on first use).
+// Device address of the scratch in the current context.
 int scratch_address(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ECUDA;
-    if (dev < 0 || dev >= kMaxDevices) return HQ_EUNSUPPORTED;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_hq_scratch) != cudaSuccess || !p) return HQ_ECUDA;
-        g_addr[dev] = p;
-    }
-    *out = g_addr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_hq_scratch) != cudaSuccess || !p) return HQ_ECUDA;
+    *out = p;
     return HQ_OK;
 }
 
@@ -50,22 +40,14 @@ extern "C" {
 
 int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, const hq_params *p, uint32_t *d_stream,
                        uint64_t cap_words, uint64_t *d_offsets, hq_stats *d_stats, void *cuda_stream) {
-    if (!p) return HQ_EINVAL;
-    if (p->lattice < HQ_Z || p->lattice > HQ_E8) return HQ_EINVAL;
-    if (!(p->alpha > 0.0f) || !(p->alpha < __builtin_inff())) return HQ_EINVAL;
-    if (p->rice_k < 0 || p->rice_k > 15 || (p->dither != 0 && p->dither != 1)) return HQ_EINVAL;
-    if (p->tile != kTile || p->chunk_tiles != kChunkTiles) return HQ_EUNSUPPORTED;
-    if (p->rotation) return HQ_EUNSUPPORTED;   // the dense rotation is a KV-cache option
-    if (p->rice_dk_last < 0 || p->rice_dk_last > 15) return HQ_EINVAL;
-    if (rows < 0 || cols < 0 || cols % kTile) return HQ_EINVAL;
-    if (cols > 65536) return HQ_EUNSUPPORTED;
-    const uint64_t tiles = (uint64_t)rows * (uint64_t)(cols / kTile);
-    const uint64_t nch = (tiles + kChunkTiles - 1) / kChunkTiles;
-    if (nch > HQ_STATIC_MAX_CHUNKS) return HQ_EUNSUPPORTED;   // beyond the fixed scratch
-    if (!d_offsets || !aligned(d_offsets, 8) || (d_stats && !aligned(d_stats, 8))) return HQ_EINVAL;
-    void *scratch = nullptr;
-    int rc = scratch_address(&scratch);
+    // the same argument rules as hq_quantize, then the scratch limit
+    int rc = check_weight_params(p);
     if (rc) return rc;
+    if ((rc = check_matrix(rows, cols))) return rc;
+    const uint64_t nch = chunks_of(rows, cols);
+    if (nch > HQ_STATIC_MAX_CHUNKS) return HQ_EUNSUPPORTED;   // beyond the fixed scratch
+    if (!d_offsets || !aligned(d_offsets, 8)) return HQ_EINVAL;
+    if (d_stats && !aligned(d_stats, 8)) return HQ_EINVAL;
     cudaStream_t s = (cudaStream_t)cuda_stream;
     if (nch == 0) {
         if (d_stats && cudaMemsetAsync(d_stats, 0, sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
@@ -73,8 +55,11 @@ int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, co
     }
     if (!x || !aligned(x, 16) || ld < cols || ld % 8) return HQ_EINVAL;
     if (!d_stream || !aligned(d_stream, 4)) return HQ_EINVAL;
-    // the previous call's look-back words, ticket, counter and stats are still there:
-    // clear what this call uses
+    void *scratch = nullptr;
+    if ((rc = scratch_address(&scratch))) return rc;
+    // the previous call's look-back words, ticket, counter and stats are still in the
+    // array: the launcher clears encode_scratch_bytes(nch) of it on this stream for the
+    // encoder forms that use a workspace (the single-CTA forms read none of it)
 
     EncodeArgs a;
     memset(&a, 0, sizeof(a));
@@ -85,21 +70,18 @@ int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t ld, co
     a.map.ld = ld;
     a.n_chunks = nch;
     a.chunk_base = 0;
-    a.c_scale = (float)((double)p->alpha / __builtin_sqrt(128.0));
+    a.c_scale = scale_fwd(p->alpha);
     a.k = p->rice_k;
-    a.k_last = (p->lattice == HQ_Z) ? p->rice_k : (p->rice_k > p->rice_dk_last ? p->rice_k - p->rice_dk_last : 0);
+    a.k_last = k_last_of(*p);
     a.seed = p->seed;
     a.stream = d_stream;
     a.cap_words = cap_words;
     a.offsets = d_offsets;
     a.stats = d_stats;
     a.stats_add = 0;
-    a.lookback = (unsigned long long *)scratch;
-    a.ticket = (unsigned int *)((char *)scratch + nch * 8);
-    a.done = (unsigned int *)((char *)scratch + nch * 8 + 4);
-    a.acc = (hq_stats *)((char *)scratch + nch * 8 + 8);
+    set_scratch(a, scratch, nch);
     a.tcols = (int)(cols / kTile);
-    a.spin_limit = kSpinLimit;
+    a.spin_limit = spin_limit();
     return launch_encode(p->lattice, p->dither, a, s) == cudaSuccess ? HQ_OK : HQ_ECUDA;
 }
 

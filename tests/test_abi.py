@@ -37,7 +37,8 @@ def test_struct_layouts_match_header():
     assert C.sizeof(hq.hq_params) == 48
     assert hq.hq_params.seed.offset == 16 and hq.hq_params.chunk_tiles.offset == 28
     assert hq.hq_params.rotation.offset == 32 and hq.hq_params.rice_dk_last.offset == 40
-    assert C.sizeof(hq.hq_stats) == 32 and hq.hq_stats.payload_bits.offset == 8
+    assert C.sizeof(hq.hq_stats) == 40 and hq.hq_stats.payload_bits.offset == 8
+    assert hq.hq_stats.max_abs_code.offset == 24 and hq.hq_stats.int8_overflow_count.offset == 32
     assert C.sizeof(hq.hq_kv_append_row) == 32
     assert C.sizeof(hq.hq_kv_cache) == 144 and hq.hq_kv_cache.params.offset == 72
     assert hq.hq_kv_cache.tokens.offset == 120
@@ -94,8 +95,19 @@ def test_unsupported_shapes_rejected():
         hq.hq_stream_bound(1, 128 * 1024, p)    # sign table too wide
 
 
+def _no_device_or_skip():
+    """Some checks below pass made-up device addresses and rely on the argument checks
+    returning before any launch.  Where a GPU is present, a regression in those checks
+    would launch a kernel on them, so these cases run only where no CUDA device is
+    visible (the tests' CPU tier)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("made-up device addresses: run only without a CUDA device")
+
+
 def test_entry_points_validate_before_touching_the_device():
     """Null or misaligned pointers come back as HQ_EINVAL with no CUDA call made."""
+    _no_device_or_skip()
     import lattice_entropy_coded_b200 as hq
     lib = hq._lib
     p = hq.make_params()
@@ -140,6 +152,7 @@ def test_entry_points_validate_before_touching_the_device():
 def test_dense_rotation_is_a_kv_option():
     """The weights entry points refuse a dense rotation (HQ_EUNSUPPORTED) and every entry
     point refuses a misaligned one (HQ_EINVAL), before any device work."""
+    _no_device_or_skip()
     import lattice_entropy_coded_b200 as hq
     lib = hq._lib
     p = hq.make_params()
@@ -165,6 +178,31 @@ def test_dense_rotation_is_a_kv_option():
     assert lib.hq_rate_kv(C.c_void_p(256), 8, 16, 128, 2048, 0, C.byref(p), st, None) == hq.HQ_EINVAL
     assert lib.hq_haar_rotation(1, None, None) == hq.HQ_EINVAL
     assert lib.hq_haar_rotation(1, C.c_void_p(4100), None) == hq.HQ_EINVAL
+
+
+def test_static_entry_point_applies_the_same_checks():
+    """hq_quantize_static rejects what hq_quantize rejects (the shared argument checks),
+    including a row count whose rows * (cols / 128) would wrap, and sizes beyond its
+    fixed scratch; null pointers only, so nothing can reach a device."""
+    import lattice_entropy_coded_b200 as hq
+    lib = hq._lib
+    p = hq.make_params("E8", 300.0, 2)
+    cases = [  # rows, cols, hq_quantize_static, hq_quantize (null pointers)
+        (1 << 55, 65536, hq.HQ_EUNSUPPORTED, hq.HQ_EUNSUPPORTED),
+        (32, 100, hq.HQ_EINVAL, hq.HQ_EINVAL),
+        (32, 131072, hq.HQ_EUNSUPPORTED, hq.HQ_EUNSUPPORTED),
+        (hq.HQ_STATIC_MAX_CHUNKS + 1, 4096, hq.HQ_EUNSUPPORTED, hq.HQ_EINVAL),
+        (hq.HQ_STATIC_MAX_CHUNKS, 4096, hq.HQ_EINVAL, hq.HQ_EINVAL),
+        (-1, 128, hq.HQ_EINVAL, hq.HQ_EINVAL),
+    ]
+    for rows, cols, want_static, want in cases:
+        assert lib.hq_quantize_static(None, rows, cols, cols, C.byref(p), None, 0, None, None, None) == want_static
+        assert lib.hq_quantize(None, rows, cols, cols, C.byref(p), None, 0, None, None, None, 0, None) == want
+    bad = hq.make_params("E8", 300.0, 2)
+    bad.rice_k = 16
+    assert lib.hq_quantize_static(None, 32, 128, 128, C.byref(bad), None, 0, None, None, None) == hq.HQ_EINVAL
+    p.rotation = 4096
+    assert lib.hq_quantize_static(None, 32, 128, 128, C.byref(p), None, 0, None, None, None) == hq.HQ_EUNSUPPORTED
 
 
 def test_binding_fails_loudly_without_the_library(tmp_path):
