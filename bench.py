@@ -2,25 +2,32 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
-Default workload: the 4096 x 4096 bf16 lattice / rate sweep (N(0, 0.02^2) with
-0.1 % x20 outliers, seed 1): 12 operating points {E8, D4, A2, Z} x {3, 4, 5}
-bits per scalar, alpha and Rice k per point from tests/golden/rate_points.json.
-One step = for every point, hq_quantize (quantize + encode) of the matrix and
-hq_dequantize of the stream back to bf16: the whole weights path.  The 32 MiB
-input fits in the 126 MB L2, so L2 is flushed (a 256 MiB write) before every
-timed kernel and each kernel is timed alone with CUDA events on the stream it
-runs on; the step time is the sum.
+Default workload: the large weight stream -- 64 bf16 matrices of 8192 x 8192
+(4.29 G elements, 8.6 GB) drawn Student-t (nu = 5) scaled to std 0.02, seed 4,
+E8 at 3 and 4 bits per scalar (alpha and Rice k from tests/golden/rate_points.json),
+all resident in HBM.  One step = for each of the two rates, hq_quantize
+(quantize + encode) of every matrix, then hq_dequantize of every stream back to
+bf16: the whole weights path over the whole set.  Inputs (8.6 GB per rate) are
+far larger than the 126 MB L2, so nothing is flushed; launches run back to back
+on one stream, each bracketed by CUDA events.
 
-metric: GB/s of bf16 input through quantize+encode and decode (the value is the
-round trip: input bytes / (encode time + decode time); each direction is also
-reported), with MSE and bits per scalar per point.
+metric: GB/s of bf16 input through quantize+encode and decode.  value = the
+round trip: input bytes of both rates / device time of the K steps (events
+around all of them); each direction is also reported, with MSE and bits per
+scalar per rate.  The roofline object is the dominant kernel's (the E8 encoder
+at 4 bps): algorithmic bytes per launch (2 B/element in + stream words and
+offsets out) / its mean event-timed launch duration, against the measured HBM
+copy bandwidth.
 
-Under torchrun (N > 1) every rank runs the same workload on its own GPU (the
-path shards into independent tensors; no collective in the data path): weak
-scaling, value = all ranks' bytes / the slowest rank's time.
+Under torchrun (N > 1) the 64 matrices are partitioned across ranks in
+contiguous blocks (lattice_entropy_coded_b200.shard): each rank codes only its
+share, with no collective on the data path; value = all ranks' bytes / the
+slowest rank's time (a fixed set: strong scaling).  After the timed region one
+all_gather of word counts places every rank's part in one global stream index.
 
---impl reference times the CPU oracle (plain C, tests' reference) on a bounded
-sample of the same workload on the host cores.
+--impl reference times the CPU oracle (plain C, the tests' reference) on a
+bounded sample of the same workload on the host cores.
+--workload NAME times one of the other workloads (one JSON line each).
 """
 from __future__ import annotations
 
@@ -43,11 +50,14 @@ import torch  # noqa: E402
 
 import synth  # noqa: E402
 
-DEFAULT_WORKLOAD = "weight_4096x4096_rate_sweep"
+DEFAULT_WORKLOAD = "student_t_64x8192x8192_e8"
+SWEEP_WORKLOAD = "weight_4096x4096_rate_sweep"
 L2_FLUSH_BYTES = 256 << 20
-PROFILE_ENCODE = os.path.join(ROOT, "profiles", "encode_kernel_e8_4bps.md")
+# ncu figures of the benched encoder (one 8192 x 8192 Student-t matrix, E8 4 bps), machine-readable
+PROFILE_ENCODE = os.path.join(ROOT, "profiles", "encode_kernel_e8_4bps_student_t_8192x8192.json")
 SM_COUNT, SMSP_PER_SM = 148, 4
 FP32_FMA_PEAK = SM_COUNT * 128 * 1.965e9      # fp32 fma per second at the maximum SM clock
+METRIC = "quantize+encode / decode GB/s of bf16 input vs B200 HBM peak; MSE at bps"
 
 
 def rate_points():
@@ -64,29 +74,26 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+ENCODER_SOURCES = ("hq_encode.cuh", "hq_encode.cu", "hq_device.cuh", "hq_internal.h")
+
+
 def kernel_source_hash() -> str:
+    """First 16 hex digits of sha256 over the encoder's sources (the profile's key)."""
     h = hashlib.sha256()
-    for f in ("hq_encode.cuh", "hq_encode.cu", "hq_device.cuh", "hq_internal.h"):
+    for f in ENCODER_SOURCES:
         with open(os.path.join(ROOT, "lattice_entropy_coded_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def profiled_encode():
-    """(DRAM bytes per launch, warp instructions per element) of the E8 4 bps encode
-    launch from the committed ncu capture, or (None, None) if the kernel source has
-    changed since it was taken."""
+    """The ncu capture of the benched encoder launch (profiles/*.json), or None when it is
+    missing or the encoder's sources have changed since it was taken."""
     if not os.path.exists(PROFILE_ENCODE):
-        return None, None
-    vals = {}
+        return None
     with open(PROFILE_ENCODE) as f:
-        for line in f:
-            for key in ("kernel_source_hash", "traffic_bytes_per_launch", "warp_inst_per_element"):
-                if line.startswith(key + ":"):
-                    vals[key] = line.split(":", 1)[1].strip()
-    if vals.get("kernel_source_hash") != kernel_source_hash():
-        return None, None
-    return float(vals["traffic_bytes_per_launch"]), float(vals["warp_inst_per_element"])
+        d = json.load(f)
+    return d if d.get("kernel_source_hash") == kernel_source_hash() else None
 
 
 def reduce_max(values, device):
@@ -97,9 +104,22 @@ def reduce_max(values, device):
     return [float(v) for v in t.cpu()]
 
 
+def reduce_sum(values, device):
+    """Element-wise sum over ranks (identity without a process group)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return [float(v) for v in t.cpu()]
+
+
+def job_gbs(total_bytes: float, max_ms: float) -> float:
+    """Whole-job GB/s: the bytes of all ranks over the slowest rank's time."""
+    return total_bytes / (max_ms * 1e6)
+
+
 def weak_scaling_value(bytes_per_rank: float, world: int, max_ms: float) -> float:
-    """Whole-job GB/s: every rank processes bytes_per_rank; the job takes the slowest rank's time."""
-    return world * bytes_per_rank / (max_ms * 1e6)
+    """Whole-job GB/s when every rank processes bytes_per_rank (the other workloads)."""
+    return job_gbs(world * bytes_per_rank, max_ms)
 
 
 # ------------------------------------------------------------------ clocks
@@ -159,202 +179,310 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
 
 
-# ------------------------------------------------------------------ workload
-def make_points(workload: str):
-    pts = rate_points()[workload]["points"]
-    return pts
+
+# ------------------------------------------------------------------ the headline workload
+def _events(n: int = 2):
+    return tuple(torch.cuda.Event(enable_timing=True) for _ in range(n))
 
 
 def run_ours(args, rank: int, world: int, device: torch.device):
+    """The large weight stream: this rank's share of the 64 Student-t matrices, E8 at 3 and
+    4 bps; quantize+encode every matrix, then decode every stream, for each rate."""
     import lattice_entropy_coded_b200 as hq
+    from lattice_entropy_coded_b200 import shard
     assert hq.hq_device_check() == hq.HQ_OK, "needs an sm_100 (B200) device"
     w = synth.WORKLOADS[args.workload]
-    assert w["kind"] == "weight", "the default bench workload is a single weight matrix"
+    assert w["kind"] == "student_t", "the default bench workload is the Student-t matrix set"
     rows, cols, seed = w["rows"], w["cols"], w["seed"]
-    x = synth.weight(rows, cols, seed=seed, device=device)
-    n = x.numel()
-    pts = make_points(args.workload)
+    lo, hi = shard.shard_range(w["n"], world, rank)
+    mats = list(synth.student_t(hi - lo, rows, cols, seed, device=device, first=lo))
+    n_mat, elems = len(mats), rows * cols
+    pts = rate_points()[args.workload]["points"]
     stream = torch.cuda.current_stream(device)
+    codecs = [[hq.Codec(rows, cols, hq.make_params(p["lattice"], p["alpha"], p["k"], seed, 0),
+                        cap_words=int(elems * (p["bps"] + 3.0) / 32) + 8192, device=device) for _ in mats]
+              for p in pts]
+    outs = [torch.empty(rows, cols, dtype=torch.bfloat16, device=device) for _ in mats]
+    per_step = 2 * len(pts) * n_mat          # launches of our kernels per step (one encode, one decode each)
 
-    codecs = []
-    for p in pts:
-        params = hq.make_params(p["lattice"], p["alpha"], p["k"], seed, 0)
-        cap = int(n * (p["bps"] + 3.0) / 32) + 8192
-        codecs.append(hq.Codec(rows, cols, params, cap_words=cap, device=device))
-    outs = [torch.empty(rows, cols, dtype=torch.bfloat16, device=device) for _ in pts]
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    def one_step(evs):
+        j = 0
+        for pi in range(len(pts)):
+            comps = []
+            for i, m in enumerate(mats):
+                evs[j][0].record(stream)
+                comps.append(codecs[pi][i].quantize(m))
+                evs[j][1].record(stream)
+                j += 1
+            for i in range(n_mat):
+                evs[j][0].record(stream)
+                codecs[pi][i].dequantize(comps[i], outs[i])
+                evs[j][1].record(stream)
+                j += 1
 
-    def one_step(record):
-        for i, c in enumerate(codecs):
-            flush.fill_(float(i))
-            e0, e1 = record()
-            e0.record(stream)
-            comp = c.quantize(x)
-            e1.record(stream)
-            flush.fill_(float(i) + 0.5)
-            d0, d1 = record()
-            d0.record(stream)
-            c.dequantize(comp, outs[i])
-            d1.record(stream)
-
-    events = []
-
-    def rec():
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        events.append((a, b))
-        return a, b
-
+    warm = [_events() for _ in range(per_step)]
     for _ in range(args.warmup):
-        one_step(rec)
+        one_step(warm)
+    timed = [[_events() for _ in range(per_step)] for _ in range(args.steps)]
     torch.cuda.synchronize(device)
-    events.clear()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
+    t0, t1 = _events()
     with ClockSampler(device.index if device.index is not None else 0) as clk:
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
-        for _ in range(args.steps):
-            one_step(rec)
+        for s in range(args.steps):
+            one_step(timed[s])
         t1.record(stream)
         torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
-    wall_ms = t0.elapsed_time(t1)
-    ms = np.array([a.elapsed_time(b) for a, b in events]).reshape(args.steps, len(pts), 2)
-    enc_ms = ms[:, :, 0].sum(1)      # per step
-    dec_ms = ms[:, :, 1].sum(1)
-    step_ms = enc_ms + dec_ms
+    step_ms_local = t0.elapsed_time(t1) / args.steps
+    # launch times [step, point, encode/decode, matrix]
+    ms = np.array([[a.elapsed_time(b) for a, b in evs] for evs in timed]).reshape(args.steps, len(pts), 2, n_mat)
 
-    # per-point results (outside the timed region): rate and MSE of the bf16 reconstruction
-    per_point = []
-    xf = x.double()
-    for i, (p, c) in enumerate(zip(pts, codecs)):
-        st = hq.read_stats(c.stats)
-        assert st["status"] == 0, (p, st)
-        mse = float(((outs[i].double() - xf) ** 2).mean())
-        words = int(c.offsets[-1].item())
-        per_point.append(dict(lattice=p["lattice"], bps_target=p["bps"], k=p["k"], alpha=p["alpha"],
-                              bps_payload=st["payload_bits"] / n, bps_stream=words * 32.0 / n,
-                              bps_total=(words * 32.0 + 64.0 * (c.n_chunks + 1)) / n, mse=mse,
-                              d_over_sigma2=mse / float(xf.var()),
-                              enc_us=float(np.median(ms[:, i, 0]) * 1e3), dec_us=float(np.median(ms[:, i, 1]) * 1e3),
-                              enc_gbs=2.0 * n / (np.median(ms[:, i, 0]) * 1e6),
-                              dec_gbs=2.0 * n / (np.median(ms[:, i, 1]) * 1e6),
-                              stream_words=words))
-
-    # max over ranks of the summed kernel time
-    step_sum, enc_sum, dec_sum, wall_max = reduce_max(
-        [float(step_ms.sum()), float(enc_ms.sum()), float(dec_ms.sum()), wall_ms], device)
-    in_bytes = 2.0 * n * len(pts)               # bf16 input bytes per step, per rank
-    value = weak_scaling_value(in_bytes * args.steps, world, step_sum)
-    enc_gbs = weak_scaling_value(in_bytes * args.steps, world, enc_sum)
-    dec_gbs = weak_scaling_value(in_bytes * args.steps, world, dec_sum)
-
-    # roofline of the dominant kernel: the encoder at the E8 4 bps point (the slowest launch of a step)
+    # per rate (outside the timed region): stats, stream size, MSE of the bf16 reconstruction
     peak, peak_kind = measured_peaks()
+    per_point, alg_launch = [], []
+    for pi, p in enumerate(pts):
+        stats = [hq.read_stats(c.stats) for c in codecs[pi]]
+        assert all(st["status"] == 0 for st in stats), (p, stats)
+        words = [int(c.offsets[-1].item()) for c in codecs[pi]]
+        se = 0.0
+        for i, m in enumerate(mats):
+            codecs[pi][i].dequantize(codecs[pi][i].quantize(m), outs[i])
+            se += float((outs[i].double() - m.double()).pow_(2).sum())
+        var = sum(float(m.double().var()) for m in mats) / n_mat
+        nch = codecs[pi][0].n_chunks
+        alg = [2.0 * elems + 4.0 * wd + 8.0 * (nch + 1) for wd in words]
+        alg_launch.append(alg)
+        enc = ms[:, pi, 0, :].mean(0)          # per matrix, mean over steps
+        dec = ms[:, pi, 1, :].mean(0)
+        tot = reduce_sum([float(sum(st["payload_bits"] for st in stats)), float(sum(words)), se,
+                          float(n_mat * (nch + 1)), float(n_mat)], device)
+        n_all = tot[4] * elems
+        per_point.append(dict(
+            lattice=p["lattice"], bps_target=p["bps"], k=p["k"], alpha=p["alpha"],
+            bps_payload=tot[0] / n_all, bps_stream=tot[1] * 32.0 / n_all,
+            bps_total=(tot[1] * 32.0 + 64.0 * tot[3]) / n_all, mse=tot[2] / n_all, d_over_sigma2=tot[2] / n_all / var,
+            max_abs_code=int(reduce_max([float(max(st["max_abs_code"] for st in stats))], device)[0]),
+            int8_overflow_count=int(reduce_sum([float(sum(st["int8_overflow_count"] for st in stats))], device)[0]),
+            encode_ms_per_matrix=float(enc.mean()), decode_ms_per_matrix=float(dec.mean()),
+            encode_gbs_per_gpu=2.0 * elems / (float(enc.mean()) * 1e6),
+            decode_gbs_per_gpu=2.0 * elems / (float(dec.mean()) * 1e6),
+            encode_hbm_frac=float(np.mean(alg)) / (float(enc.mean()) * 1e6) / peak,
+            decode_hbm_frac=float(np.mean(alg)) / (float(dec.mean()) * 1e6) / peak))
+
+    # the whole job: every rank's bytes over the slowest rank's time
+    step_ms, enc_ms, dec_ms = reduce_max([step_ms_local, float(ms[:, :, 0, :].sum() / args.steps),
+                                          float(ms[:, :, 1, :].sum() / args.steps)], device)
+    bytes_step = reduce_sum([2.0 * elems * n_mat * len(pts)], device)[0]
+    value = job_gbs(bytes_step, step_ms)
+
+    # roofline of the dominant kernel: the E8 encoder at 4 bps
+    e4 = [i for i, p in enumerate(pts) if p["bps"] == 4.0][0]
+    enc4 = ms[:, e4, 0, :]
+    launch_ms = float(enc4.mean())
+    alg4 = float(np.mean(alg_launch[e4]))
+    achieved = alg4 / (launch_ms * 1e6)
     clk = clk.summary()
-    alg = [2.0 * n + 4.0 * pp["stream_words"] + 8.0 * (c.n_chunks + 1) for pp, c in zip(per_point, codecs)]
-    enc_launch_ms = ms[:, :, 0].mean(0)
-    dec_launch_ms = ms[:, :, 1].mean(0)
-    e4 = [i for i, p in enumerate(per_point) if p["lattice"] == "E8" and p["bps_target"] == 4.0][0]
-    hbm_achieved = alg[e4] / (enc_launch_ms[e4] * 1e6)
-    traffic, inst_per_elem = profiled_encode()
+    prof = profiled_encode()
     sm_mhz = clk["sm_mhz"] or 1965.0
     issue_peak = SM_COUNT * SMSP_PER_SM * sm_mhz * 1e6 / 1e9          # G warp-instructions / s
-    roofline = {"kernel": "hq::encode_kernel<E8> at 4 bps (one launch, 4096x4096)",
-                "bound": "alu", "unit": "Ginst/s",
-                "achieved": None if inst_per_elem is None else round(inst_per_elem * n / (enc_launch_ms[e4] * 1e6), 1),
-                "peak": round(issue_peak, 1),
-                "frac": None if inst_per_elem is None else round(inst_per_elem * n / (enc_launch_ms[e4] * 1e6) / issue_peak, 4),
-                "peak_kind": f"issue slots: {SM_COUNT} SMs x {SMSP_PER_SM} schedulers x 1 warp-instruction/cycle at the "
-                             f"sampled {sm_mhz:.0f} MHz",
-                "traffic": traffic,
-                "hbm": {"achieved": round(hbm_achieved, 1), "peak": peak, "unit": "GB/s",
-                        "frac": round(hbm_achieved / peak, 4),
-                        "peak_kind": ("measured, MEASURED_PEAKS.json hbm_gbs (burst copy; kernels are timed alone)"
-                                      if peak_kind == "measured" else "fallback 6.65 TB/s"),
-                        "algorithmic_bytes": alg[e4]},
-                "all_points": {"encode_hbm_achieved": round(float(np.sum(alg) / (np.sum(enc_launch_ms) * 1e6)), 1),
-                               "decode_hbm_achieved": round(float(np.sum(alg) / (np.sum(dec_launch_ms) * 1e6)), 1),
-                               "unit": "GB/s"}}
+    roofline = {
+        "kernel": "hq::encode_kernel<E8> (per-warp form), one 8192 x 8192 matrix at 4 bps",
+        "bound": "hbm", "unit": "GB/s", "achieved": round(achieved, 1), "peak": peak,
+        "frac": round(achieved / peak, 4),
+        "peak_kind": ("of measured: MEASURED_PEAKS.json hbm_gbs (copy bandwidth)" if peak_kind == "measured"
+                      else "of fallback 6.65 TB/s"),
+        "algorithmic_bytes_per_launch": round(alg4, 1),
+        "launch_ms": round(launch_ms, 5), "launches_averaged": int(enc4.size),
+        "traffic": None if prof is None else prof["dram_bytes_per_launch"],
+        "traffic_source": None if prof is None else os.path.relpath(PROFILE_ENCODE, ROOT),
+        "issue": (None if prof is None else {
+            "warp_inst_per_element": prof["warp_inst_per_element"],
+            "achieved_ginst_s": round(prof["warp_inst_per_element"] * elems / (launch_ms * 1e6), 1),
+            "peak_ginst_s": round(issue_peak, 1),
+            "frac": round(prof["warp_inst_per_element"] * elems / (launch_ms * 1e6) / issue_peak, 4),
+            "peak_kind": f"{SM_COUNT} SMs x {SMSP_PER_SM} schedulers x 1 warp-instruction/cycle at the sampled "
+                         f"{sm_mhz:.0f} MHz"}),
+        "decoder": {"kernel": "hq::decode_kernel<E8> at 4 bps",
+                    "achieved": round(alg4 / (float(ms[:, e4, 1, :].mean()) * 1e6), 1),
+                    "frac": round(alg4 / (float(ms[:, e4, 1, :].mean()) * 1e6) / peak, 4)},
+    }
 
-    # end to end through the C ABI with host buffers: H2D of the input, quantize+decode per point,
-    # D2H of every reconstruction and stats block
-    e2e = run_e2e(args, hq, codecs, pts, rows, cols, device, stream, world)
+    # one global stream index over the ranks' parts (outside the timed region)
+    words4 = sum(int(c.offsets[-1].item()) for c in codecs[e4])
+    gbase, gtotal = shard.global_base(words4, device=device)
 
-    return dict(value=value, enc_gbs=enc_gbs, dec_gbs=dec_gbs, ms_per_step=step_sum / args.steps,
-                wall_ms_per_step=wall_max / args.steps, per_point=per_point, roofline=roofline,
-                clocks=clk, e2e=e2e, launches=2 * len(pts) * args.steps, n=n, in_bytes=in_bytes)
+    e2e = run_e2e(args, hq, codecs, pts, mats, outs, device, stream)
+    return dict(value=value, enc_gbs=job_gbs(bytes_step, enc_ms), dec_gbs=job_gbs(bytes_step, dec_ms),
+                ms_per_step=step_ms, per_point=per_point, roofline=roofline, clocks=clk, e2e=e2e,
+                launches=per_step * args.steps, matrices=(lo, hi), global_stream={"rank_base_words": gbase,
+                                                                                   "total_words_4bps": gtotal})
 
 
-def run_e2e(args, hq, codecs, pts, rows, cols, device, stream, world):
-    n = rows * cols
-    host_x = synth.weight(rows, cols, seed=synth.WORKLOADS[args.workload]["seed"]).pin_memory()
-    host_out = [torch.empty(rows, cols, dtype=torch.bfloat16).pin_memory() for _ in pts]
-    host_stats = [torch.empty(32, dtype=torch.uint8).pin_memory() for _ in pts]
-    dev_x = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
-    dev_out = [torch.empty(rows, cols, dtype=torch.bfloat16, device=device) for _ in pts]
-    # device-to-host copies on their own stream, so point i's copy overlaps point i+1's codec work
-    copy_stream = torch.cuda.Stream(device)
-    done = [torch.cuda.Event() for _ in pts]
+def run_e2e(args, hq, codecs, pts, mats, outs, device, stream):
+    """The same step through the C ABI from host memory: every step copies each matrix in
+    from pinned host memory, quantizes it at both rates and decodes the streams (the
+    reconstruction stays on the device, where its consumer runs), and copies every stream
+    (its exact words, read from the call's stats), offsets and stats block back to pinned
+    host memory.  Host-to-device copies run on their own stream, device-to-host copies on
+    another, so matrix i's copies overlap the coding of its neighbours."""
+    n_mat = len(mats)
+    rows, cols = mats[0].shape
+    host_x = []
+    for m in mats:
+        h = torch.empty(rows, cols, dtype=torch.bfloat16, pin_memory=True)
+        h.copy_(m)
+        host_x.append(h)
+    host_w = [[torch.empty(c.cap_words, dtype=torch.int32, pin_memory=True) for c in row] for row in codecs]
+    host_off = [[torch.empty(c.n_chunks + 1, dtype=torch.int64, pin_memory=True) for c in row] for row in codecs]
+    host_st = [[torch.empty(hq.STATS_BYTES, dtype=torch.uint8, pin_memory=True) for _ in row] for row in codecs]
+    dec_st = [hq.stats_tensor(device) for _ in mats]
+    host_dst = [torch.empty(hq.STATS_BYTES, dtype=torch.uint8, pin_memory=True) for _ in mats]
+    h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    landed = [torch.cuda.Event() for _ in mats]
+    coded = [[torch.cuda.Event() for _ in mats] for _ in pts]
+    small = [[torch.cuda.Event() for _ in mats] for _ in pts]
+    counts = {"h2d": 0, "d2h": 0}
 
     def step():
-        dev_x.copy_(host_x, non_blocking=True)
-        for i, c in enumerate(codecs):
-            comp = c.quantize(dev_x)
-            c.dequantize(comp, dev_out[i])
-            done[i].record(stream)
-            with torch.cuda.stream(copy_stream):
-                copy_stream.wait_event(done[i])
-                host_out[i].copy_(dev_out[i], non_blocking=True)
-                host_stats[i].copy_(c.stats, non_blocking=True)
-        # the step ends when its copies have landed (and the next step may reuse the buffers)
-        stream.wait_stream(copy_stream)
+        counts["h2d"] = counts["d2h"] = 0
+        h2d.wait_stream(stream)            # the previous step's coding has read the inputs
+        for i in range(n_mat):
+            with torch.cuda.stream(h2d):
+                mats[i].copy_(host_x[i], non_blocking=True)
+                landed[i].record(h2d)
+            counts["h2d"] += 2 * rows * cols
+        d2h.wait_stream(stream)
+        for i in range(n_mat):
+            stream.wait_event(landed[i])
+            for pi in range(len(pts)):
+                comp = codecs[pi][i].quantize(mats[i])
+                coded[pi][i].record(stream)
+                codecs[pi][i].dequantize(comp, outs[i], dec_st[i])
+                with torch.cuda.stream(d2h):
+                    d2h.wait_event(coded[pi][i])
+                    host_st[pi][i].copy_(codecs[pi][i].stats, non_blocking=True)
+                    host_off[pi][i].copy_(codecs[pi][i].offsets, non_blocking=True)
+                    small[pi][i].record(d2h)
+            with torch.cuda.stream(d2h):
+                d2h.wait_stream(stream)
+                host_dst[i].copy_(dec_st[i], non_blocking=True)
+        # the host reads each stream's size as soon as its stats land, then fetches exactly its words
+        for i in range(n_mat):
+            for pi in range(len(pts)):
+                small[pi][i].synchronize()
+                nw = hq.read_stats(host_st[pi][i])["stream_words"]
+                with torch.cuda.stream(d2h):
+                    host_w[pi][i][:nw].copy_(codecs[pi][i].words[:nw], non_blocking=True)
+                counts["d2h"] += 4 * nw + 8 * (codecs[pi][i].n_chunks + 1) + hq.STATS_BYTES
+            counts["d2h"] += hq.STATS_BYTES
+        stream.wait_stream(d2h)            # the step ends when its copies have landed
 
-    for _ in range(max(1, args.warmup)):
+    for _ in range(max(1, min(args.warmup, 2))):
         step()
     torch.cuda.synchronize(device)
-    steps = max(1, min(args.steps, 5))
+    steps = max(1, min(args.steps, 3))
+    world = torch.distributed.get_world_size() if torch.distributed.is_initialized() else 1
     if world > 1:
         torch.distributed.barrier()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0, t1 = _events()
     t0.record(stream)
     for _ in range(steps):
         step()
     t1.record(stream)
     torch.cuda.synchronize(device)
     ms = reduce_max([t0.elapsed_time(t1)], device)[0]
-    for i in range(len(pts)):
-        assert hq.read_stats(host_stats[i])["status"] == 0
-    in_bytes = 2.0 * n * len(pts)
-    return {"value": round(weak_scaling_value(in_bytes * steps, world, ms), 3), "unit": "GB/s",
-            "h2d_bytes_per_step": 2 * n, "d2h_bytes_per_step": len(pts) * (2 * n + 32),
-            "steps": steps, "ms_per_step": round(ms / steps, 3)}
+    for pi in range(len(pts)):
+        for i in range(n_mat):
+            assert hq.read_stats(host_st[pi][i])["status"] == 0
+    for i in range(n_mat):
+        assert hq.read_stats(host_dst[i])["status"] == 0
+    # the streams that came back are the device's
+    assert torch.equal(host_w[-1][0][:int(host_off[-1][0][-1])].to(device),
+                       codecs[-1][0].words[:int(host_off[-1][0][-1])])
+    bytes_step = reduce_sum([2.0 * rows * cols * n_mat * len(pts), float(counts["h2d"]), float(counts["d2h"])],
+                            device)
+    return {"value": round(job_gbs(bytes_step[0] * steps, ms), 3), "unit": "GB/s",
+            "h2d_bytes_per_step": int(bytes_step[1]), "d2h_bytes_per_step": int(bytes_step[2]),
+            "steps": steps, "ms_per_step": round(ms / steps, 3),
+            "step": "H2D of every matrix from pinned host memory, hq_quantize at both rates, hq_dequantize "
+                    "to bf16 on the device, D2H of every stream's words, offsets and stats"}
+
+
+def run_sweep(args, device: torch.device):
+    """The 4096 x 4096 lattice / rate sweep (12 points), reported next to the headline:
+    each quantize and decode launch timed alone with CUDA events, L2 flushed (a 256 MiB
+    write) before each, since the 32 MiB input fits in L2."""
+    import lattice_entropy_coded_b200 as hq
+    w = synth.WORKLOADS[SWEEP_WORKLOAD]
+    rows, cols, seed = w["rows"], w["cols"], w["seed"]
+    x = synth.weight(rows, cols, seed=seed, device=device)
+    n = x.numel()
+    pts = rate_points()[SWEEP_WORKLOAD]["points"]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    out = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
+    peak, _ = measured_peaks()
+    res = []
+    for p in pts:
+        c = hq.Codec(rows, cols, hq.make_params(p["lattice"], p["alpha"], p["k"], seed, 0),
+                     cap_words=int(n * (p["bps"] + 3.0) / 32) + 8192, device=device)
+        enc, dec = [], []
+        for it in range(args.warmup + min(args.steps, 5)):
+            flush.fill_(float(it))
+            e0, e1 = _events()
+            e0.record()
+            comp = c.quantize(x)
+            e1.record()
+            flush.fill_(float(it) + 0.5)
+            d0, d1 = _events()
+            d0.record()
+            c.dequantize(comp, out)
+            d1.record()
+            torch.cuda.synchronize(device)
+            if it >= args.warmup:
+                enc.append(e0.elapsed_time(e1))
+                dec.append(d0.elapsed_time(d1))
+        st = hq.read_stats(c.stats)
+        words = int(c.offsets[-1].item())
+        em, dm = float(np.median(enc)), float(np.median(dec))
+        alg = 2.0 * n + 4.0 * words + 8.0 * (c.n_chunks + 1)
+        res.append(dict(lattice=p["lattice"], bps_target=p["bps"], k=p["k"], alpha=p["alpha"],
+                        bps_payload=st["payload_bits"] / n, mse=float(((out.double() - x.double()) ** 2).mean()),
+                        max_abs_code=st["max_abs_code"], int8_overflow_count=st["int8_overflow_count"],
+                        enc_us=em * 1e3, dec_us=dm * 1e3, enc_gbs=2.0 * n / (em * 1e6), dec_gbs=2.0 * n / (dm * 1e6),
+                        enc_hbm_frac=alg / (em * 1e6) / peak, dec_hbm_frac=alg / (dm * 1e6) / peak))
+        del c
+    return {"workload": SWEEP_WORKLOAD, "l2": "flushed before every launch; launches timed alone", "points": res}
 
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
-def oracle_sample_rate(workload: str, rows_sample: int, threads: int, repeat: int = 1):
-    """Oracle quantize+decode of the first rows_sample rows at every point, chunk ranges on
-    `threads` host threads (ctypes releases the GIL).  -> (GB/s of bf16 input, seconds, elems)."""
+def host_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_rows_rate(x_u16: np.ndarray, pts, seed: int, threads: int, repeat: int = 1):
+    """The oracle's quantize+encode and decode of a bf16 matrix sample at every rate point,
+    over chunk ranges on `threads` host threads (ctypes releases the GIL).
+    -> (GB/s of bf16 input through the round trip, seconds, elements per direction)."""
     from concurrent.futures import ThreadPoolExecutor
 
     import oracle as O
-    w = synth.WORKLOADS[workload]
-    x = synth.weight(w["rows"], w["cols"], seed=w["seed"])[:rows_sample].contiguous()
-    xu = np.ascontiguousarray(x.view(torch.int16).numpy().view(np.uint16))
-    R, Cc = xu.shape
+    R, Cc = x_u16.shape
     nch = O.n_chunks(R, Cc)
     step = max(1, -(-nch // threads))
     ranges = [(a, min(nch, a + step)) for a in range(0, nch, step)]
-    pts = make_points(workload)
     O.lib()
 
     def job(r, p):
         lat = O.LATTICES[p["lattice"]]
-        s, off, _ = O.quantize(xu, lat, p["alpha"], p["k"], w["seed"], 0, r[0], r[1])
-        O.dequantize(s, off, R, Cc, lat, p["alpha"], p["k"], w["seed"], 0, False, r[0], r[1])
+        s, off, _ = O.quantize(x_u16, lat, p["alpha"], p["k"], seed, 0, r[0], r[1])
+        O.dequantize(s, off, R, Cc, lat, p["alpha"], p["k"], seed, 0, False, r[0], r[1])
 
     t = time.perf_counter()
     with ThreadPoolExecutor(threads) as ex:
@@ -363,6 +491,50 @@ def oracle_sample_rate(workload: str, rows_sample: int, threads: int, repeat: in
     dt = time.perf_counter() - t
     elems = R * Cc * len(pts) * repeat
     return 2.0 * elems / dt / 1e9, dt, elems
+
+
+def _student_t_sample(workload: str, rows: int) -> np.ndarray:
+    """The first `rows` rows of matrix 0 of the set, drawn with the CPU generator."""
+    w = synth.WORKLOADS[workload]
+    m = next(synth.student_t(1, w["rows"], w["cols"], w["seed"]))[:rows].contiguous()
+    return np.ascontiguousarray(m.view(torch.int16).numpy().view(np.uint16))
+
+
+def cpu_baseline(workload: str):
+    """The oracle on a bounded sample: the whole of matrix 0 (8192 x 8192) at both rates."""
+    threads = host_threads()
+    w = synth.WORKLOADS[workload]
+    xs = _student_t_sample(workload, w["rows"])
+    gbs, dt, elems = oracle_rows_rate(xs, rate_points()[workload]["points"], w["seed"], threads)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"matrix 0 of the set ({w['rows']}x{w['cols']}, CPU generator) at both rates (E8 3 and 4 bps), "
+                      f"quantize+encode and decode ({elems} elements per direction, {dt:.1f} s wall on "
+                      f"{threads} threads)"}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on a bounded sample of the workload per
+    step (the first rows of matrix 0 at both rates), on the host's threads."""
+    threads = host_threads()
+    w = synth.WORKLOADS[args.workload]
+    rows = max(64, min(2048, 64 * threads))
+    xs = _student_t_sample(args.workload, rows)
+    pts = rate_points()[args.workload]["points"]
+    for _ in range(args.warmup):
+        oracle_rows_rate(xs[:64], pts, w["seed"], threads)
+    gbs, dt, elems = oracle_rows_rate(xs, pts, w["seed"], threads, repeat=args.steps)
+    base = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"rows 0..{rows - 1} of matrix 0 ({w['rows']}x{w['cols']} Student-t, CPU generator) at both "
+                      f"rates per step, quantize+encode and decode, {args.steps} steps ({dt:.1f} s wall on "
+                      f"{threads} threads)"}
+    return {"metric": METRIC, "value": base["value"], "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "matrices": w["n"], "rows": w["rows"], "cols": w["cols"],
+                       "dtype_in": "bf16", "points": "E8 at 3 and 4 bps", "sample_rows": rows,
+                       "parallelism": "host threads"},
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def kv_rotation_seed(workload_seed: int, tensor: str) -> int:
@@ -447,46 +619,8 @@ def oracle_workload(workload: str, threads: int, budget_s: float = 60.0, pts=Non
     return out
 
 
-def host_threads() -> int:
-    try:
-        return len(os.sched_getaffinity(0))
-    except Exception:
-        return os.cpu_count() or 1
-
-
-def cpu_baseline(workload: str):
-    threads = host_threads()
-    rows = min(4096, max(256, 128 * threads))
-    gbs, dt, elems = oracle_sample_rate(workload, rows, threads)
-    return {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"rows 0..{rows - 1} of the 4096x4096 matrix at all 12 points, quantize+encode and "
-                      f"decode ({elems} elements per direction, {dt:.1f} s wall on {threads} threads)"}
-
-
-def run_reference(args):
-    threads = host_threads()
-    rows = max(32, min(1024, 32 * threads))
-    for _ in range(args.warmup):
-        oracle_sample_rate(args.workload, rows, threads)
-    gbs, dt, elems = oracle_sample_rate(args.workload, rows, threads, repeat=args.steps)
-    base = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"rows 0..{rows - 1} of the 4096x4096 matrix at all 12 points per step, quantize+encode and "
-                      f"decode, {args.steps} steps ({dt:.1f} s wall on {threads} threads)"}
-    return {"metric": "quantize+encode / decode GB/s of bf16 input vs B200 HBM peak; MSE at bps",
-            "value": base["value"], "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
-            "config": {"workload": args.workload, "rows": 4096, "cols": 4096, "points": 12,
-                       "sample_rows": rows, "parallelism": "host threads"},
-            "cpu_baseline": base,
-            "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-
 
 # ------------------------------------------------------------------ the other workloads
-def _events():
-    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-
 def run_bulk(args):
     """Time one of the other workloads end to end on the device (inputs resident in HBM,
     larger than L2, launches back to back on one stream); prints one JSON line."""
@@ -767,15 +901,22 @@ def calibrate_set(hq, mats, pts, seed):
 
 # ------------------------------------------------------------------ single-matrix case (profiling)
 def run_case(args):
-    """Quantize + decode one R x C synthetic weight matrix (seed 1) at one operating point of
-    the rate sweep, back to back, no L2 flush: the small case the ncu captures run on."""
+    """Quantize + decode one R x C matrix at one operating point, back to back, no L2 flush:
+    the small case the ncu captures run on.  --case-data weight: the sweep's Gaussian
+    weights (seed 1) at a point of the rate sweep; student_t: matrix 0 of the Student-t set
+    (its first R rows and C columns, seed 4) at a point of that set (E8 3 or 4 bps)."""
     import lattice_entropy_coded_b200 as hq
     rows, cols = (int(v) for v in args.case.lower().split("x"))
-    p = [q for q in rate_points()[DEFAULT_WORKLOAD]["points"]
-         if q["lattice"] == args.lattice and q["bps"] == args.bps][0]
+    wl = SWEEP_WORKLOAD if args.case_data == "weight" else DEFAULT_WORKLOAD
+    seed = synth.WORKLOADS[wl]["seed"]
+    p = [q for q in rate_points()[wl]["points"] if q["lattice"] == args.lattice and q["bps"] == args.bps][0]
     device = torch.device("cuda", 0)
-    x = synth.weight(rows, cols, seed=1, device=device)
-    params = hq.make_params(p["lattice"], p["alpha"], p["k"], 1, args.dither)
+    if args.case_data == "weight":
+        x = synth.weight(rows, cols, seed=seed, device=device)
+    else:
+        w = synth.WORKLOADS[wl]
+        x = next(synth.student_t(1, w["rows"], w["cols"], seed, device=device))[:rows, :cols].contiguous()
+    params = hq.make_params(p["lattice"], p["alpha"], p["k"], seed, args.dither)
     codec = hq.Codec(rows, cols, params, cap_words=int(x.numel() * (p["bps"] + 3.0) / 32) + 8192, device=device)
     out = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
     ev = []
@@ -892,9 +1033,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the 4096 x 4096 rate sweep reported beside the line")
     ap.add_argument("--oracle", action="store_true",
                     help="with --workload: also time the CPU oracle on the workload (about a minute per point)")
     ap.add_argument("--case", default=None, help="RxC: time one matrix (profiling case)")
+    ap.add_argument("--case-data", default="weight", choices=["weight", "student_t"],
+                    help="--case input: the sweep's Gaussian weights, or matrix 0 of the Student-t set")
     ap.add_argument("--token-case", action="store_true", help="time one-token KV appends (profiling case)")
     ap.add_argument("--lattice", default="E8")
     ap.add_argument("--bps", type=float, default=4.0)
@@ -907,17 +1051,19 @@ def main():
     if args.token_case:
         run_token_case(args)
         return
-    if args.workload != DEFAULT_WORKLOAD and args.impl == "ours":
-        run_bulk(args)
-        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
+        if args.workload != DEFAULT_WORKLOAD:
+            raise SystemExit("--impl reference times the default workload")
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.workload != DEFAULT_WORKLOAD:
+        run_bulk(args)
         return
 
     device = torch.device("cuda", local)
@@ -927,20 +1073,27 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     try:
         r = run_ours(args, rank, world, device)
+        sweep = run_sweep(args, device) if (world == 1 and not args.no_sweep) else None
         if rank == 0:
+            w = synth.WORKLOADS[args.workload]
             line = {
-                "metric": "quantize+encode / decode GB/s of bf16 input vs B200 HBM peak; MSE at bps",
-                "value": round(r["value"], 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 4), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": {"workload": args.workload, "rows": 4096, "cols": 4096, "dtype_in": "bf16",
-                           "points": "E8,D4,A2,Z x 3,4,5 bps", "step": "12 x (hq_quantize + hq_dequantize bf16)",
-                           "l2": "flushed (256 MiB write) before every timed kernel; kernels timed alone",
-                           "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU"},
+                "metric": METRIC, "value": round(r["value"], 2), "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 4),
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic",
+                "config": {"workload": args.workload, "matrices": w["n"], "rows": w["rows"], "cols": w["cols"],
+                           "dtype_in": "bf16", "distribution": "Student-t nu=5, std 0.02", "seed": w["seed"],
+                           "points": "E8 at 3 and 4 bps",
+                           "step": "per rate: hq_quantize of every matrix, then hq_dequantize of every stream to bf16",
+                           "l2": "inputs larger than L2 (8.6 GB per rate); no flush",
+                           "parallelism": (f"{world} ranks, matrices partitioned in contiguous blocks"
+                                           if world > 1 else "single GPU")},
                 "quantize_encode_gbs": round(r["enc_gbs"], 2), "decode_gbs": round(r["dec_gbs"], 2),
                 "roofline": r["roofline"], "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": r["launches"],
-                "points": r["per_point"],
+                "points": r["per_point"], "global_stream": r["global_stream"],
             }
+            if sweep is not None:
+                line["rate_sweep_4096"] = sweep
             if not args.no_cpu_baseline and world == 1:   # the oracle is timed at N = 1 only
                 line["cpu_baseline"] = cpu_baseline(args.workload)
             print(json.dumps(line), flush=True)

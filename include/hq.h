@@ -272,6 +272,18 @@ HQ_API int hq_quantize_static(const void *x, int64_t rows, int64_t cols, int64_t
                               uint32_t *d_stream, uint64_t cap_words, uint64_t *d_offsets, hq_stats *d_stats,
                               void *cuda_stream);
 
+/* ------------------------------------------------------------- several GPUs */
+
+/* Add base to count chunk offsets (device uint64, 8-byte aligned), in place.
+ * The coding path shards into independent tensors with no exchange: each GPU
+ * codes its share into its own streams and offsets.  To read the shards as one
+ * global stream, each GPU moves its offsets by the global word index at which
+ * its part starts (the sum of the word counts of the GPUs before it, one gather
+ * of 8 bytes per GPU).  The pages describe a single-device method; this is the
+ * only step that several GPUs add.  count 0 is a no-op.  HQ_EINVAL for a null or
+ * misaligned pointer; asynchronous on cuda_stream. */
+HQ_API int hq_offsets_add(uint64_t *d_offsets, uint64_t count, uint64_t base, void *cuda_stream);
+
 /* ----------------------------------------------------------------- rate targeting */
 
 /* The rate of a quantize call, without its stream.  The pages state that alpha

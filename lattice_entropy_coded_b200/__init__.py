@@ -103,6 +103,7 @@ EXPORTS = {
     "hq_quantize_static": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.POINTER(hq_params), C.c_void_p,
                                      C.c_uint64, C.c_void_p, C.c_void_p, C.c_void_p]),
     "hq_haar_rotation": (C.c_int, [C.c_uint64, C.c_void_p, C.c_void_p]),
+    "hq_offsets_add": (C.c_int, [C.c_void_p, C.c_uint64, C.c_uint64, C.c_void_p]),
 }
 
 
@@ -251,6 +252,13 @@ def hq_haar_rotation(seed: int, out: torch.Tensor | None = None, cuda_stream=Non
     assert out.dtype == torch.float32 and out.is_contiguous() and tuple(out.shape) == (128, 128)
     _check(_lib.hq_haar_rotation(int(seed) & (2**64 - 1), _ptr(out), _stream(cuda_stream)), "hq_haar_rotation")
     return out
+
+
+def hq_offsets_add(offsets: torch.Tensor, base: int, cuda_stream=None) -> int:
+    """offsets (int64 / uint64 words of a stream's chunk offsets, on the device) += base, in place."""
+    assert offsets.dtype == torch.int64 and offsets.is_contiguous()
+    return _check(_lib.hq_offsets_add(_ptr(offsets), offsets.numel(), int(base), _stream(cuda_stream)),
+                  "hq_offsets_add")
 
 
 def hq_debug_set_encode_path(path: int) -> int:

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libhq.so")
 SOURCES = ["hq_api.cu", "hq_encode.cu", "hq_decode.cu", "hq_consume.cu", "hq_static.cu", "hq_debug.cu",
-           "hq_rot_encode.cu", "hq_rot_decode.cu", "hq_haar.cu"]
+           "hq_rot_encode.cu", "hq_rot_decode.cu", "hq_haar.cu", "hq_shard.cu"]
 HEADERS = ["hq_internal.h", "hq_device.cuh", "hq_encode.cuh", "hq_decode.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -89,13 +89,19 @@ def weight_set_elems(layers: int = 8) -> int:
     return layers * sum(r * c for _, r, c in LAYER_SHAPES)
 
 
-def student_t(n: int, rows: int, cols: int, seed: int, device="cpu", nu: int = 5, std: float = WEIGHT_STD):
-    """Yields n bf16 matrices, entries Student-t(nu) * std / sqrt(nu / (nu - 2)) (so std = `std`).
+STUDENT_T_STRIDE = 1_000_003   # matrix i of a set is drawn from seed + i * STUDENT_T_STRIDE
+
+
+def student_t(n: int, rows: int, cols: int, seed: int, device="cpu", nu: int = 5, std: float = WEIGHT_STD,
+              first: int = 0):
+    """Yields n bf16 matrices (numbers first .. first + n - 1 of the set), entries
+    Student-t(nu) * std / sqrt(nu / (nu - 2)) (so std = `std`).  Each matrix has its
+    own generator, so any part of the set can be drawn alone (one rank's share).
 
     t = N / sqrt(chi2_nu / nu) with chi2_nu a sum of nu squared standard normals."""
-    g = _gen(seed, device)
     scale = std / math.sqrt(nu / (nu - 2.0))
-    for _ in range(n):
+    for i in range(first, first + n):
+        g = _gen(seed + i * STUDENT_T_STRIDE, device)
         z = torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32)
         chi2 = torch.zeros_like(z)
         for _ in range(nu):

@@ -1,7 +1,8 @@
 """bench.py's reference arm on CPU: one JSON line with the contract's keys.
 
 The reference arm times the CPU oracle on a bounded sample of the default workload
-(there is no other reference implementation), so it runs without a GPU."""
+(the 64 x 8192 x 8192 Student-t set; there is no other reference implementation),
+so it runs without a GPU."""
 import json
 import os
 import subprocess
@@ -22,7 +23,7 @@ def test_reference_arm_prints_one_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["higher_is_better"] is True
     assert d["steps"] == 1 and d["warmup"] >= 3 and d["value"] > 0
-    assert d["config"]["workload"] == "weight_4096x4096_rate_sweep"
+    assert d["config"]["workload"] == "student_t_64x8192x8192_e8"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     e = d["e2e"]

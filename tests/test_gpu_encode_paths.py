@@ -90,7 +90,7 @@ def test_stats_are_replaced_not_accumulated(path):
     words = torch.empty(bound, dtype=torch.int32, device="cuda")
     offs = torch.empty(nch + 1, dtype=torch.int64, device="cuda")
     ws = torch.empty(hq.hq_workspace_bytes(nch), dtype=torch.uint8, device="cuda")
-    st = torch.full((32,), 0xFF, dtype=torch.uint8, device="cuda")
+    st = torch.full((hq.STATS_BYTES,), 0xFF, dtype=torch.uint8, device="cuda")
     for _ in range(2):
         hq.hq_quantize(x, params, words, offs, st, ws)
         got = hq.read_stats(st)

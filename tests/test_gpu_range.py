@@ -95,7 +95,7 @@ def test_kv_running_range(rot):
     K, _ = synth.kv(3, 341, seed=4)
     seed, alpha, k = 6, 9.0, 2
     Q = ORot.haar_rotation(seed) if rot else None
-    cache = hq.KVCache(3, 341, hq.make_params("E8", 1.0, k, seed, 1), bits_per_scalar=16.0, max_appends=4,
+    cache = hq.KVCache(3, 341, hq.make_params("E8", 1.0, k, seed, 1), bits_per_scalar=64.0, max_appends=4,
                        max_append_tokens=300, rotation=torch.from_numpy(Q).cuda() if rot else None)
     mx, ov = 0, 0
     t0 = 0
