@@ -431,6 +431,23 @@ __device__ __forceinline__ void round_symbols_rolled(const EncodeArgs &a, const 
 template <bool KSMALL>
 __device__ __forceinline__ void put_rem(uint32_t *dst, const uint32_t (&z)[32], int k, bool store) {
     if (k == 0) return;
+    if (KSMALL && (k & (k - 1)) == 0) {
+        // k in {1, 2, 4}: 32 / k remainders fill a word exactly.  Each symbol's k low bits
+        // enter at the top of the word by one funnel shift, (z : acc) >> k, so that when the
+        // word is full its first symbol sits in the lowest bits; full words are stored.
+        uint32_t acc = 0;
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            acc = __funnelshift_r(acc, z[i], k);
+            if (store) {
+                if (i == 7 && k == 4) dst[0] = acc;
+                if (i == 15 && k >= 2) dst[k / 2 - 1] = acc;
+                if (i == 23 && k == 4) dst[2] = acc;
+                if (i == 31) dst[k - 1] = acc;
+            }
+        }
+        return;
+    }
     const uint32_t mask = (1u << k) - 1u;
     unsigned long long acc = 0;
     uint32_t nb = 0, w = 0;
@@ -503,13 +520,10 @@ __device__ __forceinline__ void put_rem_mixed(uint32_t *rem, uint32_t lb, const 
     }
 }
 
-// Unary terminators of 8 symbols with quotients q[0..7], starting at bit pos of
-// `un` (zeroed shared words).  A group whose codes fit in 32 bits is built in a
-// register (last symbol first) and ORed in with at most two shared atomics.
-__device__ __forceinline__ uint32_t unary_group_shared(uint32_t *un, uint32_t pos, const uint32_t (&q)[8]) {
-    uint32_t ug = 8;
-#pragma unroll
-    for (int i = 0; i < 8; i++) ug += q[i];
+// Unary terminators of 8 symbols with quotients q[0..7] (ug = 8 + their sum bits in all),
+// starting at bit pos of `un` (zeroed shared words).  A group whose codes fit in 32 bits is
+// built in a register (last symbol first) and ORed in with at most two shared atomics.
+__device__ __forceinline__ void unary_group_bits(uint32_t *un, uint32_t pos, const uint32_t (&q)[8], uint32_t ug) {
     if (ug <= 32u) {
         uint32_t acc = 0;
 #pragma unroll
@@ -529,6 +543,13 @@ __device__ __forceinline__ uint32_t unary_group_shared(uint32_t *un, uint32_t po
             p += 1;
         }
     }
+}
+// The same, summing the group's bits; returns them.
+__device__ __forceinline__ uint32_t unary_group_shared(uint32_t *un, uint32_t pos, const uint32_t (&q)[8]) {
+    uint32_t ug = 8;
+#pragma unroll
+    for (int i = 0; i < 8; i++) ug += q[i];
+    unary_group_bits(un, pos, q, ug);
     return ug;
 }
 
@@ -592,6 +613,40 @@ __device__ __noinline__ void encode_chunk_global(const EncodeArgs &a, const Chun
     }
 }
 
+// Copy a chunk's n stage words to stream[start, start + n), dropping words at or past
+// cap_words: the words before the stream's first 16-byte boundary one per lane, then
+// groups of four words as one 16-byte store per lane, then the last few words.  Whole
+// warp.  ZERO: also clear the stage words [0, n) (forms that reuse a stage unzeroed).
+template <bool ZERO>
+__device__ __forceinline__ void copy_stage_out(const EncodeArgs &a, uint32_t *stage, unsigned long long start,
+                                               uint32_t n, int lane) {
+    const unsigned long long cap = a.cap_words;
+    uint32_t *g = a.stream + start;
+    const uint32_t head = min(n, (uint32_t)((16u - ((uint32_t)(uintptr_t)g & 15u)) & 15u) >> 2);
+    if ((uint32_t)lane < head && start + lane < cap) g[lane] = stage[lane];
+    const uint32_t groups = (n - head) >> 2;
+    uint4 *g4 = reinterpret_cast<uint4 *>(g + head);
+    for (uint32_t q = lane; q < groups; q += 32) {
+        const uint32_t s = head + 4 * q;
+        const uint4 v = make_uint4(stage[s], stage[s + 1], stage[s + 2], stage[s + 3]);
+        if (start + s + 4 <= cap) {
+            g4[q] = v;
+        } else {
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                if (start + s + j < cap) g[s + j] = w[j];
+        }
+    }
+    const uint32_t t = head + 4 * groups + (uint32_t)lane;
+    if (t < n && start + t < cap) g[t] = stage[t];
+    if (ZERO) {
+        __syncwarp();
+        uint4 *s4 = reinterpret_cast<uint4 *>(stage);
+        for (uint32_t i = lane; i < (n + 3) >> 2; i += 32) s4[i] = make_uint4(0, 0, 0, 0);
+    }
+}
+
 // A chunk that has been encoded into a stage and waits for its offset.
 struct Pending {
     unsigned long long c, total;
@@ -619,8 +674,7 @@ __device__ __forceinline__ void finish_chunk_warp(const EncodeArgs &a, const Pen
         if (p.c == 0 && a.row) *a.row = a.row_val;
     }
     if (!p.range_bad && !p.overflow) {
-        for (uint32_t i = lane; i < (uint32_t)p.total; i += 32)
-            if (start + i < a.cap_words) a.stream[start + i] = stage[i];
+        copy_stage_out<false>(a, stage, start, (uint32_t)p.total, lane);
     } else if (!p.range_bad) {
         uint32_t *g = a.stream + start;
         const unsigned long long room = (start < a.cap_words) ? a.cap_words - start : 0ull;
@@ -718,12 +772,19 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             round_symbols<LAT, DITHER>(a, cur, raw, lane, sign_tab, z, cbits, rkey);
             rng.add<LAT>(rkey, z, cbits);
             const bool valid = cur.valid;
-            uint32_t usum = 0, lor = 0;
+            // the quotients of the lane's 4 groups of 8 symbols and their sums (the unary bits)
+            uint32_t qg[4][8], gsum[4], lor = 0;
 #pragma unroll
-            for (int i = 0; i < 32; i++) {
-                usum += z[i] >> sym_k<N>(i, k, kl);
-                lor |= z[i];
+            for (int g = 0; g < 4; g++) {
+                gsum[g] = 8u;
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    qg[g][i] = z[8 * g + i] >> sym_k<N>(i, k, kl);
+                    gsum[g] += qg[g][i];
+                    lor |= z[8 * g + i];
+                }
             }
+            const uint32_t usum = (gsum[0] + gsum[1]) + (gsum[2] + gsum[3]) - 32u;
             zor |= lor;
             const uint32_t ub = valid ? usum + 32u : 0u;
             uint32_t incl = ub;
@@ -749,10 +810,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
                     uint32_t pos = urun + incl - ub;
 #pragma unroll
                     for (int g = 0; g < 4; g++) {
-                        uint32_t qg[8];
-#pragma unroll
-                        for (int i = 0; i < 8; i++) qg[i] = z[8 * g + i] >> sym_k<N>(i, k, kl);
-                        pos += unary_group_shared(un, pos, qg);
+                        unary_group_bits(un, pos, qg[g], gsum[g]);
+                        pos += gsum[g];
                     }
                 }
             }
@@ -822,11 +881,7 @@ __device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending 
         if (p.c == 0 && a.row) *a.row = a.row_val;
     }
     if (!p.range_bad && !p.overflow) {
-        for (uint32_t i = lane; i < (uint32_t)p.total; i += 32) {
-            const uint32_t v = stage[i];
-            stage[i] = 0u;
-            if (start + i < a.cap_words) a.stream[start + i] = v;
-        }
+        copy_stage_out<true>(a, stage, start, (uint32_t)p.total, lane);
     } else if (!p.range_bad) {
         uint32_t *g = a.stream + start;
         const unsigned long long room = (start < a.cap_words) ? a.cap_words - start : 0ull;
