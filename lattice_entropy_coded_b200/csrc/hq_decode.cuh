@@ -100,17 +100,19 @@ __device__ __noinline__ uint32_t unary_slow(const uint32_t *un, uint32_t nu, uin
 // quotient is a count-leading-zeros, else the slow path.
 template <bool STAGED>
 __device__ __forceinline__ void unary4(const uint32_t *un, uint32_t nu, uint32_t &bp, bool &ok, uint32_t *q) {
-    uint32_t w = __brev(fetch32<STAGED>(un, nu, bp));
+    const uint32_t w = __brev(fetch32<STAGED>(un, nu, bp));
     if (__popc(w) >= 4) {
-        uint32_t used = 4;
+        // quotient i is the count of leading zeros after the first s_i bits, s_i = the
+        // bits of the codewords before it (each quotient plus its terminator); s_i < 32
+        // for i < 4 since the window holds four terminators
+        uint32_t s = 0;
 #pragma unroll
         for (int i = 0; i < 4; i++) {
-            const uint32_t t = __clz(w);
+            const uint32_t t = __clz(w << s);
             q[i] = t;
-            used += t;
-            w = (w << t) << 1;
+            s += t + 1u;
         }
-        bp += used;
+        bp += s;
     } else {
         uint32_t tmp[4];
         bp = unary_slow(un, nu, bp, &ok, tmp);

@@ -428,8 +428,9 @@ template <> struct Lattice<HQ_A2> {
 // arithmetic (for B up to the rounding of v - 1).  Over both candidates the
 // estimates differ from the reading's fp32 sequential-fma distances / 4 by at most
 // 19.01u (E_A + E_B) + u sum|v| + 10u (u = 2^-24; terms: the reading's rounded
-// residuals and 8-step fma chain, 10.01u E each; this estimate's fma chain and two
-// roundings, 9u E + u each; the rounding of v - 1 in candidate B, u (sum|v| + 8)).
+// residuals and 8-step fma chain, 10.01u E each; this estimate's sum of squares (two
+// 4-step fma chains over alternate coordinates and their sum) and two roundings, at
+// most 9u E + u each; the rounding of v - 1 in candidate B, u (sum|v| + 8)).
 // The margin below, 2^-18 (E_A + E_B + 4) + 2^-21 sum|v| = 64u (E_A + E_B) + 256u
 // + 8u sum|v|, is at least 3.3 times that bound.  Outside the margin the estimate
 // decides; inside it (near-ties, exact ties, huge inputs) the reading's own
@@ -470,33 +471,42 @@ template <> struct Lattice<HQ_E8> {
         return acc;
     }
     // D8 coordinates m of the nearest point (after the winner's parity fix); returns the coset bit.
+    //
+    // The two candidates' halved inputs are y_A = v / 2 and y_B = fl((v - 1) / 2), formed
+    // here for two coordinates at a time as y_A = v * 0.5 and y_B = y_A - 0.5: halving is
+    // exact and rounding commutes with it, so fl(y_A - 0.5) = fl(v - 1) / 2 bit for bit.
     __device__ static __forceinline__ uint32_t nearest_d8(const float (&v)[8], int32_t (&m)[8]) {
-        const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
+        const float2 M2 = make_float2(kRoundMagic, kRoundMagic), H2 = make_float2(0.5f, 0.5f);
         uint32_t ta[8], tb[8];
         float ra[8], rb[8];
-        float2 S = make_float2(0.0f, 0.0f);
+        float2 SA = make_float2(0.0f, 0.0f), SB = make_float2(0.0f, 0.0f);
         float ma = 0.0f, mb = 0.0f, sv = 0.0f;
         uint32_t pa = 0, pb = 0;
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const float2 y = f2_mul(make_float2(v[i], __fsub_rn(v[i], 1.0f)), make_float2(0.5f, 0.5f));
-            const float2 t = f2_add(y, M2);
-            const float2 f = f2_sub(t, M2);
-            const float2 r = f2_sub(y, f);
-            ta[i] = __float_as_uint(t.x);
-            tb[i] = __float_as_uint(t.y);
-            ra[i] = r.x;
-            rb[i] = r.y;
-            pa ^= ta[i];
-            pb ^= tb[i];
-            S = f2_fma(r, r, S);
-            ma = fmaxf(ma, fabsf(r.x));
-            mb = fmaxf(mb, fabsf(r.y));
-            sv = __fadd_rn(sv, fabsf(v[i]));
+        for (int j = 0; j < 4; j++) {
+            const float2 ya = f2_mul(make_float2(v[2 * j], v[2 * j + 1]), H2);
+            const float2 yb = f2_sub(ya, H2);
+            const float2 tA = f2_add(ya, M2), tB = f2_add(yb, M2);
+            const float2 rA = f2_sub(ya, f2_sub(tA, M2)), rB = f2_sub(yb, f2_sub(tB, M2));
+            ta[2 * j] = __float_as_uint(tA.x);
+            ta[2 * j + 1] = __float_as_uint(tA.y);
+            tb[2 * j] = __float_as_uint(tB.x);
+            tb[2 * j + 1] = __float_as_uint(tB.y);
+            ra[2 * j] = rA.x;
+            ra[2 * j + 1] = rA.y;
+            rb[2 * j] = rB.x;
+            rb[2 * j + 1] = rB.y;
+            pa ^= ta[2 * j] ^ ta[2 * j + 1];
+            pb ^= tb[2 * j] ^ tb[2 * j + 1];
+            SA = f2_fma(rA, rA, SA);
+            SB = f2_fma(rB, rB, SB);
+            ma = fmaxf(ma, fmaxf(fabsf(rA.x), fabsf(rA.y)));
+            mb = fmaxf(mb, fmaxf(fabsf(rB.x), fabsf(rB.y)));
+            sv = __fadd_rn(__fadd_rn(sv, fabsf(v[2 * j])), fabsf(v[2 * j + 1]));
         }
         const float adja = (pa & 1u) ? __fmaf_rn(-2.0f, ma, 1.0f) : 0.0f;
         const float adjb = (pb & 1u) ? __fmaf_rn(-2.0f, mb, 1.0f) : 0.0f;
-        const float2 E = f2_add(S, make_float2(adja, adjb));
+        const float2 E = make_float2(__fadd_rn(__fadd_rn(SA.x, SA.y), adja), __fadd_rn(__fadd_rn(SB.x, SB.y), adjb));
         const float diff = __fsub_rn(E.x, E.y);
         const float margin =
             __fmaf_rn(0x1p-21f, sv, __fmul_rn(0x1p-18f, __fadd_rn(__fadd_rn(E.x, E.y), 4.0f)));

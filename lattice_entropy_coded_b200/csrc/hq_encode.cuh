@@ -653,13 +653,14 @@ struct Pending {
     bool overflow, range_bad;
 };
 
+// `first`: lookback_peek(a.lookback, p.c), loaded earlier so that its latency overlaps work.
 template <int LAT, bool DITHER>
 __device__ __forceinline__ void finish_chunk_warp(const EncodeArgs &a, const Pending &p, uint32_t *stage,
-                                                  const uint32_t *sign_tab, unsigned long long base, uint32_t &status) {
+                                                  const uint32_t *sign_tab, unsigned long long base, uint32_t &status,
+                                                  unsigned long long first) {
     const int lane = threadIdx.x & 31;
     bool to = false;
-    const unsigned long long excl =
-        lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to, lookback_peek(a.lookback, p.c));
+    const unsigned long long excl = lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to, first);
     if (to) status |= HQ_ST_TIMEOUT;
     const unsigned long long start = base + excl;
     if (lane == 0) {
@@ -824,7 +825,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         lookback_publish(a.lookback, c, total);
 
         // the previous chunk's predecessors have had a whole chunk's time to publish
-        if (have_pend) finish_chunk_warp<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
+        if (have_pend)
+            finish_chunk_warp<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status,
+                                           lookback_peek(a.lookback, pend.c));
         pend.c = c;
         pend.total = total;
         pend.overflow = overflow;
@@ -833,7 +836,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         c = cn;
         buf ^= 1;
     }
-    if (have_pend) finish_chunk_warp<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status);
+    if (have_pend)
+        finish_chunk_warp<LAT, DITHER>(a, pend, stages + (buf ^ 1) * kStageWords, sign_tab, base, status,
+                                       lookback_peek(a.lookback, pend.c));
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 
     stats_add_warp<LAT>(a, status, zor_all, payload, rng);
