@@ -5,19 +5,19 @@
 Default workload: the large weight stream -- 64 bf16 matrices of 8192 x 8192
 (4.29 G elements, 8.6 GB) drawn Student-t (nu = 5) scaled to std 0.02, seed 4,
 E8 at 3 and 4 bits per scalar (alpha and Rice k from tests/golden/rate_points.json),
-all resident in HBM.  One step = for each of the two rates, hq_quantize
-(quantize + encode) of every matrix, then hq_dequantize of every stream back to
-bf16: the whole weights path over the whole set.  Inputs (8.6 GB per rate) are
-far larger than the 126 MB L2, so nothing is flushed; launches run back to back
-on one stream, each bracketed by CUDA events.
+all resident in HBM.  One step = for each of the two rates, one hq_quantize_batch
+launch (quantize + encode of every matrix of the set) and one hq_dequantize_batch
+launch (every stream back to bf16): the whole weights path over the whole set.
+Inputs (8.6 GB per rate) are far larger than the 126 MB L2, so nothing is
+flushed; launches run back to back on one stream, each bracketed by CUDA events.
 
 metric: GB/s of bf16 input through quantize+encode and decode.  value = the
 round trip: input bytes of both rates / device time of the K steps (events
 around all of them); each direction is also reported, with MSE and bits per
 scalar per rate.  The roofline object is the dominant kernel's (the E8 encoder
-at 4 bps): algorithmic bytes per launch (2 B/element in + stream words and
-offsets out) / its mean event-timed launch duration, against the measured HBM
-copy bandwidth.
+at 4 bps, one launch over the set): algorithmic bytes per launch (2 B/element
+in + stream words and offsets out) / its mean event-timed launch duration,
+against the measured HBM copy bandwidth.
 
 Under torchrun (N > 1) the 64 matrices are partitioned across ranks in
 contiguous blocks (lattice_entropy_coded_b200.shard): each rank codes only its
@@ -187,7 +187,8 @@ def _events(n: int = 2):
 
 def run_ours(args, rank: int, world: int, device: torch.device):
     """The large weight stream: this rank's share of the 64 Student-t matrices, E8 at 3 and
-    4 bps; quantize+encode every matrix, then decode every stream, for each rate."""
+    4 bps.  Per rate one hq_quantize_batch launch codes every matrix of the share and one
+    hq_dequantize_batch launch decodes every stream back to bf16."""
     import lattice_entropy_coded_b200 as hq
     from lattice_entropy_coded_b200 import shard
     assert hq.hq_device_check() == hq.HQ_OK, "needs an sm_100 (B200) device"
@@ -195,30 +196,37 @@ def run_ours(args, rank: int, world: int, device: torch.device):
     assert w["kind"] == "student_t", "the default bench workload is the Student-t matrix set"
     rows, cols, seed = w["rows"], w["cols"], w["seed"]
     lo, hi = shard.shard_range(w["n"], world, rank)
-    mats = list(synth.student_t(hi - lo, rows, cols, seed, device=device, first=lo))
-    n_mat, elems = len(mats), rows * cols
+    n_mat, elems = hi - lo, rows * cols
+    mats = torch.empty(n_mat, rows, cols, dtype=torch.bfloat16, device=device)
+    for i, m in enumerate(synth.student_t(n_mat, rows, cols, seed, device=device, first=lo)):
+        mats[i].copy_(m)
     pts = rate_points()[args.workload]["points"]
     stream = torch.cuda.current_stream(device)
-    codecs = [[hq.Codec(rows, cols, hq.make_params(p["lattice"], p["alpha"], p["k"], seed, 0),
-                        cap_words=int(elems * (p["bps"] + 3.0) / 32) + 8192, device=device) for _ in mats]
-              for p in pts]
-    outs = [torch.empty(rows, cols, dtype=torch.bfloat16, device=device) for _ in mats]
-    per_step = 2 * len(pts) * n_mat          # launches of our kernels per step (one encode, one decode each)
+    params = [hq.make_params(p["lattice"], p["alpha"], p["k"], seed, 0) for p in pts]
+    caps = [int(elems * (p["bps"] + 3.0) / 32) + 8192 for p in pts]
+    nch = hq.hq_stream_bound(rows, cols, params[0])[1]
+    words = [torch.empty(n_mat, c, dtype=torch.int32, device=device) for c in caps]
+    offsets = [torch.empty(n_mat, nch + 1, dtype=torch.int64, device=device) for _ in pts]
+    stats = [torch.zeros(n_mat, hq.STATS_BYTES, dtype=torch.uint8, device=device) for _ in pts]
+    dstats = torch.zeros(n_mat, hq.STATS_BYTES, dtype=torch.uint8, device=device)
+    ws = torch.empty(hq.hq_batch_workspace_bytes(n_mat, nch), dtype=torch.uint8, device=device)
+    outs = torch.empty(n_mat, rows, cols, dtype=torch.bfloat16, device=device)
+    per_step = 2 * len(pts)          # launches of our kernels per step: one batched encode, one batched decode
+
+    def encode(pi):
+        hq.hq_quantize_batch(mats, params[pi], words[pi], offsets[pi], stats[pi], ws)
+
+    def decode(pi):
+        hq.hq_dequantize_batch(words[pi], caps[pi], offsets[pi], rows, cols, params[pi], outs, dstats)
 
     def one_step(evs):
-        j = 0
         for pi in range(len(pts)):
-            comps = []
-            for i, m in enumerate(mats):
-                evs[j][0].record(stream)
-                comps.append(codecs[pi][i].quantize(m))
-                evs[j][1].record(stream)
-                j += 1
-            for i in range(n_mat):
-                evs[j][0].record(stream)
-                codecs[pi][i].dequantize(comps[i], outs[i])
-                evs[j][1].record(stream)
-                j += 1
+            evs[2 * pi][0].record(stream)
+            encode(pi)
+            evs[2 * pi][1].record(stream)
+            evs[2 * pi + 1][0].record(stream)
+            decode(pi)
+            evs[2 * pi + 1][1].record(stream)
 
     warm = [_events() for _ in range(per_step)]
     for _ in range(args.warmup):
@@ -238,147 +246,155 @@ def run_ours(args, rank: int, world: int, device: torch.device):
     if world > 1:
         torch.distributed.barrier()
     step_ms_local = t0.elapsed_time(t1) / args.steps
-    # launch times [step, point, encode/decode, matrix]
-    ms = np.array([[a.elapsed_time(b) for a, b in evs] for evs in timed]).reshape(args.steps, len(pts), 2, n_mat)
+    # launch times [step, point, encode/decode]
+    ms = np.array([[a.elapsed_time(b) for a, b in evs] for evs in timed]).reshape(args.steps, len(pts), 2)
 
     # per rate (outside the timed region): stats, stream size, MSE of the bf16 reconstruction
     peak, peak_kind = measured_peaks()
     per_point, alg_launch = [], []
+    var = float(sum(float(mats[i].double().var()) for i in range(n_mat)) / n_mat)
     for pi, p in enumerate(pts):
-        stats = [hq.read_stats(c.stats) for c in codecs[pi]]
-        assert all(st["status"] == 0 for st in stats), (p, stats)
-        words = [int(c.offsets[-1].item()) for c in codecs[pi]]
-        se = 0.0
-        for i, m in enumerate(mats):
-            codecs[pi][i].dequantize(codecs[pi][i].quantize(m), outs[i])
-            se += float((outs[i].double() - m.double()).pow_(2).sum())
-        var = sum(float(m.double().var()) for m in mats) / n_mat
-        nch = codecs[pi][0].n_chunks
-        alg = [2.0 * elems + 4.0 * wd + 8.0 * (nch + 1) for wd in words]
+        encode(pi)
+        decode(pi)
+        st = [hq.read_stats(stats[pi][i]) for i in range(n_mat)]
+        assert all(x["status"] == 0 for x in st), (p, st)
+        assert all(hq.read_stats(dstats[i])["status"] == 0 for i in range(n_mat))
+        wds = [int(v) for v in offsets[pi][:, -1].cpu()]
+        se = sum(float((outs[i].double() - mats[i].double()).pow_(2).sum()) for i in range(n_mat))
+        alg = 2.0 * elems * n_mat + 4.0 * sum(wds) + 8.0 * n_mat * (nch + 1)
         alg_launch.append(alg)
-        enc = ms[:, pi, 0, :].mean(0)          # per matrix, mean over steps
-        dec = ms[:, pi, 1, :].mean(0)
-        tot = reduce_sum([float(sum(st["payload_bits"] for st in stats)), float(sum(words)), se,
+        enc, dec = float(ms[:, pi, 0].mean()), float(ms[:, pi, 1].mean())
+        tot = reduce_sum([float(sum(x["payload_bits"] for x in st)), float(sum(wds)), se,
                           float(n_mat * (nch + 1)), float(n_mat)], device)
         n_all = tot[4] * elems
         per_point.append(dict(
             lattice=p["lattice"], bps_target=p["bps"], k=p["k"], alpha=p["alpha"],
             bps_payload=tot[0] / n_all, bps_stream=tot[1] * 32.0 / n_all,
             bps_total=(tot[1] * 32.0 + 64.0 * tot[3]) / n_all, mse=tot[2] / n_all, d_over_sigma2=tot[2] / n_all / var,
-            max_abs_code=int(reduce_max([float(max(st["max_abs_code"] for st in stats))], device)[0]),
-            int8_overflow_count=int(reduce_sum([float(sum(st["int8_overflow_count"] for st in stats))], device)[0]),
-            encode_ms_per_matrix=float(enc.mean()), decode_ms_per_matrix=float(dec.mean()),
-            encode_gbs_per_gpu=2.0 * elems / (float(enc.mean()) * 1e6),
-            decode_gbs_per_gpu=2.0 * elems / (float(dec.mean()) * 1e6),
-            encode_hbm_frac=float(np.mean(alg)) / (float(enc.mean()) * 1e6) / peak,
-            decode_hbm_frac=float(np.mean(alg)) / (float(dec.mean()) * 1e6) / peak))
+            max_abs_code=int(reduce_max([float(max(x["max_abs_code"] for x in st))], device)[0]),
+            int8_overflow_count=int(reduce_sum([float(sum(x["int8_overflow_count"] for x in st))], device)[0]),
+            encode_ms_per_launch=enc, decode_ms_per_launch=dec, matrices_per_launch=n_mat,
+            encode_gbs_per_gpu=2.0 * elems * n_mat / (enc * 1e6), decode_gbs_per_gpu=2.0 * elems * n_mat / (dec * 1e6),
+            encode_hbm_frac=alg / (enc * 1e6) / peak, decode_hbm_frac=alg / (dec * 1e6) / peak))
 
     # the whole job: every rank's bytes over the slowest rank's time
-    step_ms, enc_ms, dec_ms = reduce_max([step_ms_local, float(ms[:, :, 0, :].sum() / args.steps),
-                                          float(ms[:, :, 1, :].sum() / args.steps)], device)
+    step_ms, enc_ms, dec_ms = reduce_max([step_ms_local, float(ms[:, :, 0].sum() / args.steps),
+                                          float(ms[:, :, 1].sum() / args.steps)], device)
     bytes_step = reduce_sum([2.0 * elems * n_mat * len(pts)], device)[0]
     value = job_gbs(bytes_step, step_ms)
 
-    # roofline of the dominant kernel: the E8 encoder at 4 bps
+    # roofline of the dominant kernel: the E8 encoder at 4 bps, one launch over the share
     e4 = [i for i, p in enumerate(pts) if p["bps"] == 4.0][0]
-    enc4 = ms[:, e4, 0, :]
-    launch_ms = float(enc4.mean())
-    alg4 = float(np.mean(alg_launch[e4]))
+    launch_ms = float(ms[:, e4, 0].mean())
+    alg4 = alg_launch[e4]
     achieved = alg4 / (launch_ms * 1e6)
     clk = clk.summary()
     prof = profiled_encode()
     sm_mhz = clk["sm_mhz"] or 1965.0
     issue_peak = SM_COUNT * SMSP_PER_SM * sm_mhz * 1e6 / 1e9          # G warp-instructions / s
+    launch_elems = elems * n_mat
     roofline = {
-        "kernel": "hq::encode_kernel<E8> (per-warp form), one 8192 x 8192 matrix at 4 bps",
+        "kernel": f"hq::encode_kernel<E8> (per-warp form), one hq_quantize_batch launch over {n_mat} matrices of "
+                  f"{rows} x {cols} at 4 bps",
         "bound": "hbm", "unit": "GB/s", "achieved": round(achieved, 1), "peak": peak,
         "frac": round(achieved / peak, 4),
         "peak_kind": ("of measured: MEASURED_PEAKS.json hbm_gbs (copy bandwidth)" if peak_kind == "measured"
                       else "of fallback 6.65 TB/s"),
         "algorithmic_bytes_per_launch": round(alg4, 1),
-        "launch_ms": round(launch_ms, 5), "launches_averaged": int(enc4.size),
-        "traffic": None if prof is None else prof["dram_bytes_per_launch"],
+        "launch_ms": round(launch_ms, 4), "launches_averaged": int(args.steps),
+        "traffic": None if prof is None else round(prof["dram_bytes_per_element"] * launch_elems, 1),
         "traffic_source": None if prof is None else os.path.relpath(PROFILE_ENCODE, ROOT),
         "issue": (None if prof is None else {
             "warp_inst_per_element": prof["warp_inst_per_element"],
-            "achieved_ginst_s": round(prof["warp_inst_per_element"] * elems / (launch_ms * 1e6), 1),
+            "achieved_ginst_s": round(prof["warp_inst_per_element"] * launch_elems / (launch_ms * 1e6), 1),
             "peak_ginst_s": round(issue_peak, 1),
-            "frac": round(prof["warp_inst_per_element"] * elems / (launch_ms * 1e6) / issue_peak, 4),
+            "frac": round(prof["warp_inst_per_element"] * launch_elems / (launch_ms * 1e6) / issue_peak, 4),
             "peak_kind": f"{SM_COUNT} SMs x {SMSP_PER_SM} schedulers x 1 warp-instruction/cycle at the sampled "
                          f"{sm_mhz:.0f} MHz"}),
-        "decoder": {"kernel": "hq::decode_kernel<E8> at 4 bps",
-                    "achieved": round(alg4 / (float(ms[:, e4, 1, :].mean()) * 1e6), 1),
-                    "frac": round(alg4 / (float(ms[:, e4, 1, :].mean()) * 1e6) / peak, 4)},
+        "decoder": {"kernel": f"hq::decode_kernel<E8> at 4 bps, one hq_dequantize_batch launch over {n_mat} matrices",
+                    "achieved": round(alg4 / (float(ms[:, e4, 1].mean()) * 1e6), 1),
+                    "frac": round(alg4 / (float(ms[:, e4, 1].mean()) * 1e6) / peak, 4)},
     }
 
     # one global stream index over the ranks' parts (outside the timed region)
-    words4 = sum(int(c.offsets[-1].item()) for c in codecs[e4])
+    words4 = int(offsets[e4][:, -1].sum().item())
     gbase, gtotal = shard.global_base(words4, device=device)
 
-    e2e = run_e2e(args, hq, codecs, pts, mats, outs, device, stream)
+    e2e = run_e2e(args, hq, mats, outs, params, caps, pts, device, stream)
     return dict(value=value, enc_gbs=job_gbs(bytes_step, enc_ms), dec_gbs=job_gbs(bytes_step, dec_ms),
                 ms_per_step=step_ms, per_point=per_point, roofline=roofline, clocks=clk, e2e=e2e,
                 launches=per_step * args.steps, matrices=(lo, hi), global_stream={"rank_base_words": gbase,
                                                                                    "total_words_4bps": gtotal})
 
 
-def run_e2e(args, hq, codecs, pts, mats, outs, device, stream):
-    """The same step through the C ABI from host memory: every step copies each matrix in
-    from pinned host memory, quantizes it at both rates and decodes the streams (the
-    reconstruction stays on the device, where its consumer runs), and copies every stream
-    (its exact words, read from the call's stats), offsets and stats block back to pinned
-    host memory.  Host-to-device copies run on their own stream, device-to-host copies on
-    another, so matrix i's copies overlap the coding of its neighbours."""
-    n_mat = len(mats)
-    rows, cols = mats[0].shape
-    host_x = []
-    for m in mats:
-        h = torch.empty(rows, cols, dtype=torch.bfloat16, pin_memory=True)
-        h.copy_(m)
-        host_x.append(h)
-    host_w = [[torch.empty(c.cap_words, dtype=torch.int32, pin_memory=True) for c in row] for row in codecs]
-    host_off = [[torch.empty(c.n_chunks + 1, dtype=torch.int64, pin_memory=True) for c in row] for row in codecs]
-    host_st = [[torch.empty(hq.STATS_BYTES, dtype=torch.uint8, pin_memory=True) for _ in row] for row in codecs]
-    dec_st = [hq.stats_tensor(device) for _ in mats]
-    host_dst = [torch.empty(hq.STATS_BYTES, dtype=torch.uint8, pin_memory=True) for _ in mats]
+E2E_GROUP = 8   # matrices per launch in the end-to-end run: coding group j overlaps copying group j + 1
+
+
+def run_e2e(args, hq, mats, outs, params, caps, pts, device, stream):
+    """The same step through the C ABI from host memory: every step copies the matrices in
+    from pinned host memory, in groups of E2E_GROUP; each group is coded at both rates by
+    hq_quantize_batch and decoded by hq_dequantize_batch (the reconstruction stays on the
+    device, where its consumer runs), and every stream (its exact words, read from its stats),
+    offsets and stats block goes back to pinned host memory.  Host-to-device copies run on
+    their own stream, device-to-host copies on another, so a group's copies overlap the
+    coding of its neighbours."""
+    n_mat, rows, cols = mats.shape
+    nch = hq.hq_stream_bound(rows, cols, params[0])[1]
+    groups = [(g, min(n_mat, g + E2E_GROUP)) for g in range(0, n_mat, E2E_GROUP)]
+    host_x = torch.empty(n_mat, rows, cols, dtype=torch.bfloat16, pin_memory=True)
+    host_x.copy_(mats)
+    wbufs = [[torch.empty(hi - lo, c, dtype=torch.int32, device=device) for (lo, hi) in groups] for c in caps]
+    obufs = [[torch.empty(hi - lo, nch + 1, dtype=torch.int64, device=device) for (lo, hi) in groups] for _ in pts]
+    sbufs = [[torch.zeros(hi - lo, hq.STATS_BYTES, dtype=torch.uint8, device=device) for (lo, hi) in groups]
+             for _ in pts]
+    dbufs = [torch.zeros(hi - lo, hq.STATS_BYTES, dtype=torch.uint8, device=device) for (lo, hi) in groups]
+    ws = torch.empty(hq.hq_batch_workspace_bytes(E2E_GROUP, nch), dtype=torch.uint8, device=device)
+    host_w = [[torch.empty(hi - lo, c, dtype=torch.int32, pin_memory=True) for (lo, hi) in groups] for c in caps]
+    host_o = [[torch.empty(hi - lo, nch + 1, dtype=torch.int64, pin_memory=True) for (lo, hi) in groups] for _ in pts]
+    host_s = [[torch.empty(hi - lo, hq.STATS_BYTES, dtype=torch.uint8, pin_memory=True) for (lo, hi) in groups]
+              for _ in pts]
+    host_d = [torch.empty(hi - lo, hq.STATS_BYTES, dtype=torch.uint8, pin_memory=True) for (lo, hi) in groups]
     h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    landed = [torch.cuda.Event() for _ in mats]
-    coded = [[torch.cuda.Event() for _ in mats] for _ in pts]
-    small = [[torch.cuda.Event() for _ in mats] for _ in pts]
+    landed = [torch.cuda.Event() for _ in groups]
+    coded = [[torch.cuda.Event() for _ in groups] for _ in pts]
+    small = [[torch.cuda.Event() for _ in groups] for _ in pts]
     counts = {"h2d": 0, "d2h": 0}
 
     def step():
         counts["h2d"] = counts["d2h"] = 0
         h2d.wait_stream(stream)            # the previous step's coding has read the inputs
-        for i in range(n_mat):
+        for gi, (lo, hi) in enumerate(groups):
             with torch.cuda.stream(h2d):
-                mats[i].copy_(host_x[i], non_blocking=True)
-                landed[i].record(h2d)
-            counts["h2d"] += 2 * rows * cols
+                mats[lo:hi].copy_(host_x[lo:hi], non_blocking=True)
+                landed[gi].record(h2d)
+            counts["h2d"] += 2 * rows * cols * (hi - lo)
         d2h.wait_stream(stream)
-        for i in range(n_mat):
-            stream.wait_event(landed[i])
+        for gi, (lo, hi) in enumerate(groups):
+            stream.wait_event(landed[gi])
             for pi in range(len(pts)):
-                comp = codecs[pi][i].quantize(mats[i])
-                coded[pi][i].record(stream)
-                codecs[pi][i].dequantize(comp, outs[i], dec_st[i])
+                hq.hq_quantize_batch(mats[lo:hi], params[pi], wbufs[pi][gi], obufs[pi][gi], sbufs[pi][gi], ws)
+                coded[pi][gi].record(stream)
+                hq.hq_dequantize_batch(wbufs[pi][gi], caps[pi], obufs[pi][gi], rows, cols, params[pi], outs[lo:hi],
+                                       dbufs[gi])
                 with torch.cuda.stream(d2h):
-                    d2h.wait_event(coded[pi][i])
-                    host_st[pi][i].copy_(codecs[pi][i].stats, non_blocking=True)
-                    host_off[pi][i].copy_(codecs[pi][i].offsets, non_blocking=True)
-                    small[pi][i].record(d2h)
+                    d2h.wait_event(coded[pi][gi])
+                    host_s[pi][gi].copy_(sbufs[pi][gi], non_blocking=True)
+                    host_o[pi][gi].copy_(obufs[pi][gi], non_blocking=True)
+                    small[pi][gi].record(d2h)
             with torch.cuda.stream(d2h):
                 d2h.wait_stream(stream)
-                host_dst[i].copy_(dec_st[i], non_blocking=True)
+                host_d[gi].copy_(dbufs[gi], non_blocking=True)
         # the host reads each stream's size as soon as its stats land, then fetches exactly its words
-        for i in range(n_mat):
+        for gi, (lo, hi) in enumerate(groups):
             for pi in range(len(pts)):
-                small[pi][i].synchronize()
-                nw = hq.read_stats(host_st[pi][i])["stream_words"]
-                with torch.cuda.stream(d2h):
-                    host_w[pi][i][:nw].copy_(codecs[pi][i].words[:nw], non_blocking=True)
-                counts["d2h"] += 4 * nw + 8 * (codecs[pi][i].n_chunks + 1) + hq.STATS_BYTES
-            counts["d2h"] += hq.STATS_BYTES
+                small[pi][gi].synchronize()
+                for i in range(hi - lo):
+                    nw = hq.read_stats(host_s[pi][gi][i])["stream_words"]
+                    with torch.cuda.stream(d2h):
+                        host_w[pi][gi][i, :nw].copy_(wbufs[pi][gi][i, :nw], non_blocking=True)
+                    counts["d2h"] += 4 * nw
+                counts["d2h"] += (hi - lo) * (8 * (nch + 1) + hq.STATS_BYTES)
+            counts["d2h"] += (hi - lo) * hq.STATS_BYTES
         stream.wait_stream(d2h)            # the step ends when its copies have landed
 
     for _ in range(max(1, min(args.warmup, 2))):
@@ -396,20 +412,23 @@ def run_e2e(args, hq, codecs, pts, mats, outs, device, stream):
     torch.cuda.synchronize(device)
     ms = reduce_max([t0.elapsed_time(t1)], device)[0]
     for pi in range(len(pts)):
-        for i in range(n_mat):
-            assert hq.read_stats(host_st[pi][i])["status"] == 0
-    for i in range(n_mat):
-        assert hq.read_stats(host_dst[i])["status"] == 0
+        for gi in range(len(groups)):
+            for i in range(groups[gi][1] - groups[gi][0]):
+                assert hq.read_stats(host_s[pi][gi][i])["status"] == 0
+    for gi in range(len(groups)):
+        for i in range(groups[gi][1] - groups[gi][0]):
+            assert hq.read_stats(host_d[gi][i])["status"] == 0
     # the streams that came back are the device's
-    assert torch.equal(host_w[-1][0][:int(host_off[-1][0][-1])].to(device),
-                       codecs[-1][0].words[:int(host_off[-1][0][-1])])
+    nw0 = int(host_o[-1][0][0, -1])
+    assert torch.equal(host_w[-1][0][0, :nw0].to(device), wbufs[-1][0][0, :nw0])
     bytes_step = reduce_sum([2.0 * rows * cols * n_mat * len(pts), float(counts["h2d"]), float(counts["d2h"])],
                             device)
     return {"value": round(job_gbs(bytes_step[0] * steps, ms), 3), "unit": "GB/s",
             "h2d_bytes_per_step": int(bytes_step[1]), "d2h_bytes_per_step": int(bytes_step[2]),
             "steps": steps, "ms_per_step": round(ms / steps, 3),
-            "step": "H2D of every matrix from pinned host memory, hq_quantize at both rates, hq_dequantize "
-                    "to bf16 on the device, D2H of every stream's words, offsets and stats"}
+            "step": f"H2D of every matrix from pinned host memory in groups of {E2E_GROUP}; per group "
+                    "hq_quantize_batch at both rates and hq_dequantize_batch to bf16 on the device; D2H of every "
+                    "stream's words, offsets and stats"}
 
 
 def run_sweep(args, device: torch.device):
@@ -1084,7 +1103,8 @@ def main():
                 "config": {"workload": args.workload, "matrices": w["n"], "rows": w["rows"], "cols": w["cols"],
                            "dtype_in": "bf16", "distribution": "Student-t nu=5, std 0.02", "seed": w["seed"],
                            "points": "E8 at 3 and 4 bps",
-                           "step": "per rate: hq_quantize of every matrix, then hq_dequantize of every stream to bf16",
+                           "step": "per rate: one hq_quantize_batch launch over every matrix, then one "
+                                   "hq_dequantize_batch launch over every stream (to bf16)",
                            "l2": "inputs larger than L2 (8.6 GB per rate); no flush",
                            "parallelism": (f"{world} ranks, matrices partitioned in contiguous blocks"
                                            if world > 1 else "single GPU")},

@@ -218,6 +218,37 @@ HQ_API int hq_dequantize(const uint32_t *d_stream, uint64_t stream_words, const 
                   int64_t cols, const hq_params *p, void *out, int out_dtype, int64_t ld, hq_stats *d_stats,
                   void *cuda_stream);
 
+/* A set of equally shaped matrices in one launch (a strided batch), for coding a
+ * model's weight set in bulk.  Item i of `batch`:
+ *   input    x + i * x_stride (elements; x_stride % 8 == 0 and >= (rows - 1) * ld + cols),
+ *   stream   d_stream + i * stream_stride (words; stream_stride >= cap_words, cap_words
+ *            each; any stride: the items' streams need no alignment of their own),
+ *   offsets  d_offsets + i * (n_chunks + 1),
+ *   stats    d_stats + i (or d_stats NULL).
+ * Each item's stream, offsets and stats are exactly what hq_quantize of that matrix alone
+ * would write; one launch codes all of them, which removes the start-up and the partly
+ * idle last wave that each separate launch has.  workspace >= hq_batch_workspace_bytes
+ * (batch, n_chunks) with n_chunks the chunks of one matrix.  batch 0 writes nothing;
+ * batch 1 is hq_quantize.  HQ_EUNSUPPORTED when batch * n_chunks reaches 2^31.  Errors
+ * otherwise as hq_quantize; asynchronous on cuda_stream.  No counterpart in the paper:
+ * the pages code each tensor on its own, and the batch only changes how the work is
+ * launched. */
+HQ_API int hq_batch_workspace_bytes(int64_t batch, uint64_t n_chunks, size_t *bytes);
+HQ_API int hq_quantize_batch(const void *x, int64_t batch, int64_t x_stride, int64_t rows, int64_t cols, int64_t ld,
+                             const hq_params *p, uint32_t *d_stream, uint64_t stream_stride, uint64_t cap_words,
+                             uint64_t *d_offsets, hq_stats *d_stats, void *workspace, size_t ws_bytes,
+                             void *cuda_stream);
+
+/* The inverse of hq_quantize_batch: item i's stream (stream_words words, checked against
+ * its offsets) at d_stream + i * stream_stride, offsets at d_offsets + i * (n_chunks + 1),
+ * output at out + i * out_stride elements (out_stride % 8 == 0 for bf16, % 4 for fp32,
+ * >= (rows - 1) * ld + cols), stats d_stats + i (HQ_ST_CORRUPT per item).  Each item's
+ * output is exactly hq_dequantize's.  batch 1 is hq_dequantize. */
+HQ_API int hq_dequantize_batch(const uint32_t *d_stream, uint64_t stream_stride, uint64_t stream_words,
+                               const uint64_t *d_offsets, int64_t batch, int64_t rows, int64_t cols,
+                               const hq_params *p, void *out, int out_dtype, int64_t ld, int64_t out_stride,
+                               hq_stats *d_stats, void *cuda_stream);
+
 /* Decode fused into its consumer: y = W x for a compressed matrix W, without
  * writing W to memory.  The pages name the cost of the variable-length format at
  * inference ("Results": decode adds latency on an H100); here each decoded

@@ -104,6 +104,13 @@ EXPORTS = {
                                      C.c_uint64, C.c_void_p, C.c_void_p, C.c_void_p]),
     "hq_haar_rotation": (C.c_int, [C.c_uint64, C.c_void_p, C.c_void_p]),
     "hq_offsets_add": (C.c_int, [C.c_void_p, C.c_uint64, C.c_uint64, C.c_void_p]),
+    "hq_batch_workspace_bytes": (C.c_int, [C.c_int64, C.c_uint64, C.POINTER(C.c_size_t)]),
+    "hq_quantize_batch": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.c_int64, C.c_int64,
+                                    C.POINTER(hq_params), C.c_void_p, C.c_uint64, C.c_uint64, C.c_void_p, C.c_void_p,
+                                    C.c_void_p, C.c_size_t, C.c_void_p]),
+    "hq_dequantize_batch": (C.c_int, [C.c_void_p, C.c_uint64, C.c_uint64, C.c_void_p, C.c_int64, C.c_int64,
+                                      C.c_int64, C.POINTER(hq_params), C.c_void_p, C.c_int, C.c_int64, C.c_int64,
+                                      C.c_void_p, C.c_void_p]),
 }
 
 
@@ -296,6 +303,40 @@ def hq_quantize(x: torch.Tensor, params: hq_params, stream: torch.Tensor, offset
     return _check(_lib.hq_quantize(_ptr(x), rows, cols, ld, C.byref(params), _ptr(stream), stream.numel(),
                                    _ptr(offsets), _ptr(stats), _ptr(workspace), workspace.numel(),
                                    _stream(cuda_stream)), "hq_quantize")
+
+
+def hq_batch_workspace_bytes(batch: int, n_chunks: int) -> int:
+    b = C.c_size_t()
+    _check(_lib.hq_batch_workspace_bytes(batch, n_chunks, C.byref(b)), "hq_batch_workspace_bytes")
+    return int(b.value)
+
+
+def hq_quantize_batch(x: torch.Tensor, params: hq_params, stream: torch.Tensor, offsets: torch.Tensor,
+                      stats: torch.Tensor | None, workspace: torch.Tensor, cap_words: int | None = None,
+                      cuda_stream=None) -> int:
+    """x: bf16 [batch, rows, cols] (row stride x.stride(1), item stride x.stride(0));
+    stream: int32 [batch, S] words (item i's stream is row i, cap_words <= S words);
+    offsets: int64 [batch, n_chunks + 1]; stats: uint8 [batch, STATS_BYTES] or None."""
+    B, rows, cols = x.shape
+    assert stream.dim() == 2 and stream.shape[0] == B and stream.stride(1) == 1
+    cap = stream.shape[1] if cap_words is None else cap_words
+    return _check(_lib.hq_quantize_batch(_ptr(x), B, x.stride(0), rows, cols, x.stride(1), C.byref(params),
+                                         _ptr(stream), stream.stride(0), cap, _ptr(offsets), _ptr(stats),
+                                         _ptr(workspace), workspace.numel(), _stream(cuda_stream)),
+                  "hq_quantize_batch")
+
+
+def hq_dequantize_batch(stream: torch.Tensor, stream_words: int, offsets: torch.Tensor, rows: int, cols: int,
+                        params: hq_params, out: torch.Tensor, stats: torch.Tensor | None = None,
+                        cuda_stream=None) -> int:
+    """stream: int32 [batch, S]; offsets: int64 [batch, n_chunks + 1]; out: bf16 or fp32
+    [batch, rows, cols] (row stride out.stride(1), item stride out.stride(0))."""
+    B = out.shape[0]
+    assert out.dtype in (torch.float32, torch.bfloat16)
+    dt = 1 if out.dtype == torch.float32 else 0
+    return _check(_lib.hq_dequantize_batch(_ptr(stream), stream.stride(0), stream_words, _ptr(offsets), B, rows,
+                                           cols, C.byref(params), _ptr(out), dt, out.stride(1), out.stride(0),
+                                           _ptr(stats), _stream(cuda_stream)), "hq_dequantize_batch")
 
 
 def hq_quantize_static(x: torch.Tensor, params: hq_params, stream: torch.Tensor, offsets: torch.Tensor,

@@ -206,6 +206,120 @@ int hq_dequantize(const uint32_t *d_stream, uint64_t stream_words, const uint64_
     return cuda_rc(launch_decode(p->lattice, p->dither, a, s));
 }
 
+int hq_batch_workspace_bytes(int64_t batch, uint64_t n_chunks, size_t *bytes) {
+    if (!bytes || batch < 0) return HQ_EINVAL;
+    if (n_chunks && (uint64_t)batch > (UINT64_C(1) << 40) / n_chunks) return HQ_EUNSUPPORTED;
+    const size_t b = encode_scratch_bytes((uint64_t)batch * n_chunks, batch > 1 ? (uint64_t)batch : 1u);
+    *bytes = (b + 255) & ~(size_t)255;
+    return HQ_OK;
+}
+
+int hq_quantize_batch(const void *x, int64_t batch, int64_t x_stride, int64_t rows, int64_t cols, int64_t ld,
+                      const hq_params *p, uint32_t *d_stream, uint64_t stream_stride, uint64_t cap_words,
+                      uint64_t *d_offsets, hq_stats *d_stats, void *workspace, size_t ws_bytes, void *cuda_stream) {
+    int rc = check_weight_params(p);
+    if (rc) return rc;
+    if ((rc = check_matrix(rows, cols))) return rc;
+    if (batch < 0) return HQ_EINVAL;
+    if (batch == 1)
+        return hq_quantize(x, rows, cols, ld, p, d_stream, cap_words, d_offsets, d_stats, workspace, ws_bytes,
+                           cuda_stream);
+    const uint64_t nch = chunks_of(rows, cols);
+    // chunk tickets are 32-bit counters: the whole launch stays well below 2^32 chunks
+    if (batch > 0 && nch > 0 && (uint64_t)batch > (UINT64_C(1) << 31) / nch) return HQ_EUNSUPPORTED;
+    if (batch == 0) return HQ_OK;
+    if (!d_offsets || !aligned(d_offsets, 8)) return HQ_EINVAL;
+    if (d_stats && !aligned(d_stats, 8)) return HQ_EINVAL;
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    if (nch == 0) {
+        if (d_stats && cudaMemsetAsync(d_stats, 0, (size_t)batch * sizeof(hq_stats), s) != cudaSuccess)
+            return HQ_ECUDA;
+        // offsets[i * 1] = 0 for every item: each item's single entry
+        return cuda_rc(cudaMemsetAsync(d_offsets, 0, (size_t)batch * sizeof(uint64_t), s));
+    }
+    if (!x || !aligned(x, 16) || ld < cols || ld % 8) return HQ_EINVAL;
+    if (x_stride < 0 || x_stride % 8 || x_stride < (rows - 1) * ld + cols) return HQ_EINVAL;
+    if (!d_stream || !aligned(d_stream, 4) || stream_stride < cap_words) return HQ_EINVAL;
+    size_t need = 0;
+    if ((rc = hq_batch_workspace_bytes(batch, nch, &need))) return rc;
+    if (!workspace || !aligned(workspace, 8) || ws_bytes < need) return HQ_EINVAL;
+
+    EncodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = (const uint16_t *)x;
+    a.map.kv = 0;
+    a.map.rows = rows;
+    a.map.cols = cols;
+    a.map.ld = ld;
+    a.n_chunks = (uint64_t)batch * nch;
+    a.chunk_base = 0;
+    a.c_scale = scale_fwd(p->alpha);
+    a.k = p->rice_k;
+    a.k_last = k_last_of(*p);
+    a.seed = p->seed;
+    a.stream = d_stream;
+    a.cap_words = cap_words;
+    a.offsets = d_offsets;
+    a.stats = d_stats;
+    a.stats_add = 0;
+    set_scratch(a, workspace, a.n_chunks);
+    a.tcols = (int)(cols / kTile);
+    a.spin_limit = g_spin_limit;
+    a.batch = (uint64_t)batch;
+    a.item_chunks = nch;
+    a.item_stream_stride = stream_stride;
+    a.item_x_stride = x_stride;
+    return cuda_rc(launch_encode(p->lattice, p->dither, a, s));
+}
+
+int hq_dequantize_batch(const uint32_t *d_stream, uint64_t stream_stride, uint64_t stream_words,
+                        const uint64_t *d_offsets, int64_t batch, int64_t rows, int64_t cols, const hq_params *p,
+                        void *out, int out_dtype, int64_t ld, int64_t out_stride, hq_stats *d_stats, void *cuda_stream) {
+    int rc = check_weight_params(p);
+    if (rc) return rc;
+    if ((rc = check_matrix(rows, cols))) return rc;
+    if (batch < 0) return HQ_EINVAL;
+    if (batch == 1)
+        return hq_dequantize(d_stream, stream_words, d_offsets, rows, cols, p, out, out_dtype, ld, d_stats,
+                             cuda_stream);
+    if (out_dtype != 0 && out_dtype != 1) return HQ_EINVAL;
+    if (d_stats && !aligned(d_stats, 8)) return HQ_EINVAL;
+    const uint64_t nch = chunks_of(rows, cols);
+    if (batch > 0 && nch > 0 && (uint64_t)batch > (UINT64_C(1) << 40) / nch) return HQ_EUNSUPPORTED;
+    if (batch == 0) return HQ_OK;
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    if (d_stats && cudaMemsetAsync(d_stats, 0, (size_t)batch * sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;
+    if (nch == 0) return HQ_OK;
+    if (!d_stream || !aligned(d_stream, 4) || !d_offsets || !aligned(d_offsets, 8)) return HQ_EINVAL;
+    if (stream_stride < stream_words) return HQ_EINVAL;
+    if (!out || !aligned(out, 16) || ld < cols || ld % (out_dtype ? 4 : 8)) return HQ_EINVAL;
+    if (out_stride < 0 || out_stride % (out_dtype ? 4 : 8) || out_stride < (rows - 1) * ld + cols) return HQ_EINVAL;
+
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.stream = d_stream;
+    a.stream_words = stream_words;
+    a.offsets = d_offsets;
+    a.map.kv = 0;
+    a.map.rows = rows;
+    a.map.cols = cols;
+    a.n_chunks = (uint64_t)batch * nch;
+    a.e_scale = scale_inv(p->alpha);
+    a.k = p->rice_k;
+    a.k_last = k_last_of(*p);
+    a.seed = p->seed;
+    a.out = out;
+    a.out_fp32 = out_dtype;
+    a.out_ld = ld;
+    a.stats = d_stats;
+    a.tcols = (int)(cols / kTile);
+    a.batch = (uint64_t)batch;
+    a.item_chunks = nch;
+    a.item_stream_stride = stream_stride;
+    a.item_out_stride = out_stride;
+    return cuda_rc(launch_decode(p->lattice, p->dither, a, s));
+}
+
 int hq_gemv_workspace_bytes(int64_t rows, int64_t cols, size_t *bytes) {
     if (!bytes) return HQ_EINVAL;
     int rc = check_matrix(rows, cols);

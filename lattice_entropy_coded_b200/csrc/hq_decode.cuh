@@ -190,8 +190,11 @@ struct ChunkOut {
     float e_scale;
     long long row0, h, tok_base, tok0;
     int tc0, tpr;
+    long long out_off;   // elements from out to this chunk's matrix (a batch item; 0 otherwise)
 
-    __device__ __forceinline__ void init(const DecodeArgs &a, unsigned long long c) {
+    // c: the chunk's index within its matrix; item: its batch item (weights only)
+    __device__ __forceinline__ void init(const DecodeArgs &a, unsigned long long c, unsigned long long item = 0) {
+        out_off = (long long)item * a.item_out_stride;
         if (KV) {
             // the append that holds global chunk c (binary search on first_chunk)
             unsigned long long lo = 0, hi = a.n_appends - 1;
@@ -249,23 +252,31 @@ struct ChunkOut {
         tcol = tc;
         e0 = (unsigned long long)(r * a.map.cols + (long long)tc * kTile);
         pos = r * tpr + tc;
-        if (a.out) dst = (char *)a.out + (size_t)(r * a.out_ld + (long long)tc * kTile) * esz;
+        if (a.out) dst = (char *)a.out + (size_t)(out_off + r * a.out_ld + (long long)tc * kTile) * esz;
         return true;
     }
 };
 
-// Valid word range of chunk c, or nw = 0 if the offsets are not consistent.
+// Valid word range of chunk c, or nw = 0 if the offsets are not consistent; src is the
+// chunk's first word.  In a strided batch, c is split into its item and its index there.
 struct ChunkWords {
     unsigned long long w0, nw;
     bool ok;
+    const uint32_t *src;
+    unsigned long long item, local;
 };
 
 __device__ __forceinline__ ChunkWords chunk_words(const DecodeArgs &a, unsigned long long c) {
     ChunkWords r;
-    r.w0 = a.offsets[c];
-    const unsigned long long w1 = a.offsets[c + 1];
+    r.item = 0;
+    r.local = c;
+    if (a.batch > 1) divmod_u64(c, a.item_chunks, r.item, r.local);
+    const uint64_t *offs = a.offsets + r.item * (a.batch > 1 ? a.item_chunks + 1 : 0ull);
+    r.w0 = offs[r.local];
+    const unsigned long long w1 = offs[r.local + 1];
     r.ok = r.w0 <= w1 && w1 <= a.stream_words;
     r.nw = r.ok ? w1 - r.w0 : 0ull;
+    r.src = a.stream + r.item * a.item_stream_stride + r.w0;
     return r;
 }
 
@@ -274,7 +285,7 @@ __device__ __forceinline__ ChunkWords chunk_words(const DecodeArgs &a, unsigned 
 __device__ __forceinline__ void stage_chunk(const DecodeArgs &a, const ChunkWords &cw, uint32_t *stage, int lane) {
     if (cw.nw <= (unsigned long long)kStageWords) {
         const uint32_t n = (uint32_t)cw.nw;
-        const uint32_t *src = a.stream + cw.w0;
+        const uint32_t *src = cw.src;
         for (uint32_t i = lane; i < n; i += 32) {
             const unsigned sa = (unsigned)__cvta_generic_to_shared(stage + i);
             asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(src + i) : "memory");
@@ -539,7 +550,7 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
     unsigned long long v = (ROT || lg) ? (unsigned long long)warp * gridDim.x + blockIdx.x
                                        : (unsigned long long)blockIdx.x * W + warp;
     int buf = 0;
-    ChunkWords cw = {0, 0, false};
+    ChunkWords cw = {0, 0, false, nullptr, 0, 0};
     if ((v >> lg) < a.n_chunks) {
         cw = chunk_words(a, v >> lg);
         stage_chunk(a, cw, stages, lane);
@@ -547,7 +558,7 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
     for (; (v >> lg) < a.n_chunks; v += nwarps, buf ^= 1) {
         // start bringing in the next chunk while this one is decoded
         const unsigned long long cn = (v + nwarps) >> lg;
-        ChunkWords cwn = {0, 0, false};
+        ChunkWords cwn = {0, 0, false, nullptr, 0, 0};
         if (cn < a.n_chunks) {
             cwn = chunk_words(a, cn);
             stage_chunk(a, cwn, stages + (buf ^ 1) * kStageSlot, lane);
@@ -560,7 +571,7 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
         const unsigned long long c = v >> lg;
         const int r0 = (int)(v & ((1u << lg) - 1u)) << (2 - lg), r1 = r0 + (kRoundsPerChunk >> lg);
         ChunkOut<KV> geo;
-        geo.init(a, c);
+        geo.init(a, cw.local, cw.item);
         const int ntiles = geo.ntiles;
         const uint32_t nsym = (uint32_t)ntiles * kTile, nseg = 4u * (uint32_t)ntiles;
         const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * ntiles + 31) / 32u : 0u;
@@ -578,12 +589,18 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
             bad = decode_rounds<LAT, DITHER, KV, KSMALL, true, MODE, ROT, MIXED>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab,
                                                                           rot_s, r0, r1, lane);
         } else {
-            const uint32_t *src = a.stream + cw.w0;
+            const uint32_t *src = cw.src;
             ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
             bad = decode_rounds<LAT, DITHER, KV, KSMALL, false, MODE, ROT, MIXED>(a, geo, src, ok, nc, nr, nu, startbit,
                                                                            sign_tab, rot_s, r0, r1, lane);
         }
-        if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) status |= HQ_ST_CORRUPT;
+        if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) {
+            if (a.batch > 1) {
+                if (lane == 0 && a.stats) atomicOr(&a.stats[cw.item].status, HQ_ST_CORRUPT);
+            } else {
+                status |= HQ_ST_CORRUPT;
+            }
+        }
         cw = cwn;
         __syncwarp();
     }

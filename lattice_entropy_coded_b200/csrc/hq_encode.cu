@@ -61,6 +61,8 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     }
     if (mode == 4 && a.n_chunks > (unsigned long long)kTinyMaxChunks) mode = 1;
     if (mixed && mode == 3) mode = 2;
+    const bool batched = a.batch > 1;
+    if (batched) mode = 1;   // a strided batch runs the per-warp form, which keeps per-item state
     if (mode == 4) {
         // a one-token KV append (one tile per chunk) with a single Rice parameter
         if (a.map.kv && a.map.tokens == 1 && !mixed) return launch_tok_t<LAT, DITHER>(a, s);
@@ -68,7 +70,9 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     }
     // the multi-CTA forms share the workspace: look-back words, ticket, done counter and
     // stats accumulator, cleared by one memset
-    if ((e = cudaMemsetAsync(a.lookback, 0, encode_scratch_bytes(a.n_chunks), s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.lookback, 0, encode_scratch_bytes(a.n_chunks, batched ? a.batch : 1), s)) !=
+        cudaSuccess)
+        return e;
     if (mode == 3) {
         const size_t smem =
             (size_t)(a.tcols * kSignWords + 2 * kStageWords) * sizeof(uint32_t) + sizeof(WideCtl);

@@ -58,10 +58,11 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
 // inclusive prefix.  A chunk publishes its count as soon as it is encoded and
 // resolves its offset later, so waits are short.
 
-// Publish chunk c's word count (chunk 0 publishes its inclusive prefix).
+// Publish chunk c's word count (the first chunk of a stream, `first`, publishes its
+// inclusive prefix: the walk-back of later chunks stops there).
 __device__ __forceinline__ void lookback_publish(unsigned long long *lb, unsigned long long c,
-                                                 unsigned long long agg) {
-    if ((threadIdx.x & 31) == 0) st_relaxed_u64(lb + c, (c == 0 ? kFlagInc : kFlagAgg) | agg);
+                                                 unsigned long long agg, bool first) {
+    if ((threadIdx.x & 31) == 0) st_relaxed_u64(lb + c, (first ? kFlagInc : kFlagAgg) | agg);
 }
 
 // The look-back word of predecessor c - 1 - lane (INC with value 0 before chunk 0):
@@ -77,9 +78,10 @@ __device__ __forceinline__ unsigned long long lookback_peek(const unsigned long 
 // calls it.  Bounded: gives up after spin_limit polls.
 __device__ __noinline__ unsigned long long lookback_resolve(unsigned long long *lb, unsigned long long c,
                                                             unsigned long long agg, uint32_t spin_limit,
-                                                            bool &timed_out, unsigned long long first) {
+                                                            bool &timed_out, unsigned long long first,
+                                                            bool stream_first) {
     const int lane = threadIdx.x & 31;
-    if (c == 0) return 0;
+    if (stream_first) return 0;
     unsigned long long excl = 0;
     long long pos = (long long)c - 1;
     uint32_t spins = 0;
@@ -127,21 +129,23 @@ struct CodeRange {
 // replacing them (hq_quantize) or adding to them (a KV cache's running stats).
 template <int LAT>
 __device__ __forceinline__ void stats_add_warp(const EncodeArgs &a, uint32_t status, uint32_t zor_all,
-                                               unsigned long long payload, const CodeRange &rng) {
+                                               unsigned long long payload, const CodeRange &rng,
+                                               unsigned long long item = 0) {
     status = __reduce_or_sync(0xffffffffu, status);
     zor_all = __reduce_or_sync(0xffffffffu, zor_all);
     const uint32_t key = __reduce_max_sync(0xffffffffu, rng.key);
     const uint32_t ovf = __reduce_add_sync(0xffffffffu, rng.ovf);
     if ((threadIdx.x & 31) == 0) {
-        if (status) atomicOr(&a.acc->status, status);
-        if (zor_all) atomicOr(&a.acc->max_symbol, zor_all);
-        if (payload) atomicAdd((unsigned long long *)&a.acc->payload_bits, payload);
-        if (key) atomicMax(&a.acc->max_abs_code, code_abs_of_key<LAT>(key));
-        if (ovf) atomicAdd((unsigned long long *)&a.acc->int8_overflow_count, (unsigned long long)ovf);
+        hq_stats *acc = a.acc + item;
+        if (status) atomicOr(&acc->status, status);
+        if (zor_all) atomicOr(&acc->max_symbol, zor_all);
+        if (payload) atomicAdd((unsigned long long *)&acc->payload_bits, payload);
+        if (key) atomicMax(&acc->max_abs_code, code_abs_of_key<LAT>(key));
+        if (ovf) atomicAdd((unsigned long long *)&acc->int8_overflow_count, (unsigned long long)ovf);
     }
 }
 
-// Whole CTA calls it once, at its end.
+// Whole CTA calls it once, at its end.  The last CTA moves every item's accumulator.
 __device__ __forceinline__ void stats_finish_cta(const EncodeArgs &a) {
     __syncthreads();
     if (threadIdx.x != 0) return;
@@ -149,31 +153,47 @@ __device__ __forceinline__ void stats_finish_cta(const EncodeArgs &a) {
     if (atomicAdd(a.done, 1u) != gridDim.x - 1) return;
     __threadfence();
     if (!a.stats) return;
-    const uint32_t st = ld_relaxed_u32(&a.acc->status), mx = ld_relaxed_u32(&a.acc->max_symbol);
-    const unsigned long long pb = ld_relaxed_u64((const unsigned long long *)&a.acc->payload_bits);
-    const unsigned long long sw = ld_relaxed_u64((const unsigned long long *)&a.acc->stream_words);
-    const uint32_t am = ld_relaxed_u32(&a.acc->max_abs_code);
-    const unsigned long long ov = ld_relaxed_u64((const unsigned long long *)&a.acc->int8_overflow_count);
-    if (a.stats_add) {
-        if (st) atomicOr(&a.stats->status, st);
-        if (mx) atomicOr(&a.stats->max_symbol, mx);
-        if (pb) atomicAdd((unsigned long long *)&a.stats->payload_bits, pb);
-        if (am) atomicMax(&a.stats->max_abs_code, am);
-        if (ov) atomicAdd((unsigned long long *)&a.stats->int8_overflow_count, ov);
-    } else {
-        a.stats->status = st;
-        a.stats->max_symbol = mx;
-        a.stats->payload_bits = pb;
-        a.stats->max_abs_code = am;
-        a.stats->reserved = 0u;
-        a.stats->int8_overflow_count = ov;
+    const unsigned long long items = a.batch > 1 ? a.batch : 1ull;
+    for (unsigned long long i = 0; i < items; i++) {
+        const hq_stats *acc = a.acc + i;
+        hq_stats *out = a.stats + i;
+        const uint32_t st = ld_relaxed_u32(&acc->status), mx = ld_relaxed_u32(&acc->max_symbol);
+        const unsigned long long pb = ld_relaxed_u64((const unsigned long long *)&acc->payload_bits);
+        const unsigned long long sw = ld_relaxed_u64((const unsigned long long *)&acc->stream_words);
+        const uint32_t am = ld_relaxed_u32(&acc->max_abs_code);
+        const unsigned long long ov = ld_relaxed_u64((const unsigned long long *)&acc->int8_overflow_count);
+        if (a.stats_add) {
+            if (st) atomicOr(&out->status, st);
+            if (mx) atomicOr(&out->max_symbol, mx);
+            if (pb) atomicAdd((unsigned long long *)&out->payload_bits, pb);
+            if (am) atomicMax(&out->max_abs_code, am);
+            if (ov) atomicAdd((unsigned long long *)&out->int8_overflow_count, ov);
+        } else {
+            out->status = st;
+            out->max_symbol = mx;
+            out->payload_bits = pb;
+            out->max_abs_code = am;
+            out->reserved = 0u;
+            out->int8_overflow_count = ov;
+        }
+        out->stream_words = sw;
     }
-    a.stats->stream_words = sw;
+}
+
+// The item of a strided batch that chunk c belongs to, and c's index within it.
+struct ItemChunk {
+    unsigned long long item, local;
+};
+__device__ __forceinline__ ItemChunk item_chunk(const EncodeArgs &a, unsigned long long c) {
+    ItemChunk r{0ull, c};
+    if (a.batch > 1) divmod_u64(c, a.item_chunks, r.item, r.local);
+    return r;
 }
 
 // Where the tiles of one chunk are (computed once per chunk).
 struct ChunkGeo {
     int ntiles;
+    long long xoff;   // elements from x to this chunk's matrix (a batch item; 0 otherwise)
     // weights: tile ti of the chunk is row row0 + (tc0 + ti) / tpr, tile column (tc0 + ti) % tpr
     long long row0;
     int tc0, tpr;
@@ -181,6 +201,7 @@ struct ChunkGeo {
     long long h, tok_base;
 
     __device__ __forceinline__ void init(const TileMap &m, unsigned long long c) {
+        xoff = 0;
         if (m.kv) {
             const long long cph = (m.tokens + 31) / 32;
             unsigned long long hq_, rq;
@@ -218,7 +239,7 @@ struct ChunkGeo {
             r += d;
             tc -= d * tpr;
         }
-        src = x + r * m.ld + (long long)tc * kTile;
+        src = x + xoff + r * m.ld + (long long)tc * kTile;
         tcol = tc;
         e0 = (unsigned long long)(r * m.cols + (long long)tc * kTile);
         return true;
@@ -618,10 +639,10 @@ __device__ __noinline__ void encode_chunk_global(const EncodeArgs &a, const Chun
 // groups of four words as one 16-byte store per lane, then the last few words.  Whole
 // warp.  ZERO: also clear the stage words [0, n) (forms that reuse a stage unzeroed).
 template <bool ZERO>
-__device__ __forceinline__ void copy_stage_out(const EncodeArgs &a, uint32_t *stage, unsigned long long start,
-                                               uint32_t n, int lane) {
+__device__ __forceinline__ void copy_stage_out(const EncodeArgs &a, uint32_t *stream, uint32_t *stage,
+                                               unsigned long long start, uint32_t n, int lane) {
     const unsigned long long cap = a.cap_words;
-    uint32_t *g = a.stream + start;
+    uint32_t *g = stream + start;
     const uint32_t head = min(n, (uint32_t)((16u - ((uint32_t)(uintptr_t)g & 15u)) & 15u) >> 2);
     if ((uint32_t)lane < head && start + lane < cap) g[lane] = stage[lane];
     const uint32_t groups = (n - head) >> 2;
@@ -651,40 +672,51 @@ __device__ __forceinline__ void copy_stage_out(const EncodeArgs &a, uint32_t *st
 struct Pending {
     unsigned long long c, total;
     bool overflow, range_bad;
+    unsigned long long item, local;   // batch item and the chunk's index in it (0 and c unbatched)
 };
 
 // `first`: lookback_peek(a.lookback, p.c), loaded earlier so that its latency overlaps work.
+// A batch item's stream is its own: its chunk offsets, tail and stream size are written
+// into the item's entries, and its capacity and look-back timeout bits go straight to its
+// accumulator.
 template <int LAT, bool DITHER>
 __device__ __forceinline__ void finish_chunk_warp(const EncodeArgs &a, const Pending &p, uint32_t *stage,
                                                   const uint32_t *sign_tab, unsigned long long base, uint32_t &status,
                                                   unsigned long long first) {
     const int lane = threadIdx.x & 31;
+    const bool batched = a.batch > 1;
+    const unsigned long long nloc = batched ? a.item_chunks : a.n_chunks;
+    uint64_t *offs = batched ? a.offsets + p.item * (a.item_chunks + 1) : a.offsets + a.chunk_base;
+    uint32_t *stream = a.stream + (batched ? p.item * a.item_stream_stride : 0ull);
     bool to = false;
-    const unsigned long long excl = lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to, first);
-    if (to) status |= HQ_ST_TIMEOUT;
+    const unsigned long long excl = lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to, first, p.local == 0);
+    uint32_t st = to ? HQ_ST_TIMEOUT : 0u;
     const unsigned long long start = base + excl;
     if (lane == 0) {
-        a.offsets[a.chunk_base + p.c] = start;
-        if (p.c + 1 == a.n_chunks) {
+        offs[p.local] = start;
+        if (p.local + 1 == nloc) {
             const unsigned long long end = start + p.total;
-            a.offsets[a.chunk_base + a.n_chunks] = end;
+            offs[nloc] = end;
             if (a.tail_out) *a.tail_out = end;
-            a.acc->stream_words = end;
-            if (end > a.cap_words) status |= HQ_ST_CAPACITY;
+            a.acc[p.item].stream_words = end;
+            if (end > a.cap_words) st |= HQ_ST_CAPACITY;
         }
-        if (p.c == 0 && a.row) *a.row = a.row_val;
+        if (p.local == 0 && a.row) *a.row = a.row_val;
+        if (batched && st) atomicOr(&a.acc[p.item].status, st);
     }
+    if (!batched) status |= st;
     if (!p.range_bad && !p.overflow) {
-        copy_stage_out<false>(a, stage, start, (uint32_t)p.total, lane);
+        copy_stage_out<false>(a, stream, stage, start, (uint32_t)p.total, lane);
     } else if (!p.range_bad) {
-        uint32_t *g = a.stream + start;
+        uint32_t *g = stream + start;
         const unsigned long long room = (start < a.cap_words) ? a.cap_words - start : 0ull;
         for (unsigned long long i = lane; i < p.total; i += 32)
             if (i < room) g[i] = 0u;
         __syncwarp();
         __threadfence_block();
         ChunkGeo geo;
-        geo.init(a.map, p.c);
+        geo.init(a.map, p.local);
+        geo.xoff = (long long)p.item * a.item_x_stride;
         const uint32_t nc = (LAT == HQ_E8) ? (uint32_t)(16 * geo.ntiles + 31) / 32u : 0u;
         const uint32_t nr = ((uint32_t)geo.ntiles * tile_rem_bits<Lattice<LAT>::N>(a.k, a.k_last) + 31u) >> 5;
         encode_chunk_global<LAT, DITHER, false>(a, geo, sign_tab, nullptr, g, room, nc, nr);
@@ -725,17 +757,31 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
 
     unsigned long long c = take_ticket(a);
     if (c < a.n_chunks) {
+        const ItemChunk ic = item_chunk(a, c);
         ChunkGeo g0;
-        g0.init(a.map, c);
+        g0.init(a.map, ic.local);
+        g0.xoff = (long long)ic.item * a.item_x_stride;
         prefetch_round(a, g0, 0, lane, slot);
     }
     Pending pend;
     bool have_pend = false;
     int buf = 0;
+    // a batch's stats are gathered per item: the warp's running figures belong to item
+    // cur_item and are added to its accumulator when the warp moves to another item
+    unsigned long long cur_item = 0;
     while (c < a.n_chunks) {
         const unsigned long long cn = take_ticket(a);
+        const ItemChunk ic = item_chunk(a, c);
+        if (ic.item != cur_item) {
+            stats_add_warp<LAT>(a, status, zor_all, payload, rng, cur_item);
+            status = zor_all = 0;
+            payload = 0;
+            rng = CodeRange();
+            cur_item = ic.item;
+        }
         ChunkGeo geo;
-        geo.init(a.map, c);
+        geo.init(a.map, ic.local);
+        geo.xoff = (long long)ic.item * a.item_x_stride;
         uint32_t *stage = stages + buf * kStageWords;
 
         const int ntiles = geo.ntiles;
@@ -764,8 +810,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             if (r + 1 < nrounds) {
                 prefetch_round(a, geo, r + 1, lane, slot);
             } else if (cn < a.n_chunks) {
+                const ItemChunk icn = item_chunk(a, cn);
                 ChunkGeo gn;
-                gn.init(a.map, cn);
+                gn.init(a.map, icn.local);
+                gn.xoff = (long long)icn.item * a.item_x_stride;
                 prefetch_round(a, gn, 0, lane, slot);
             }
 
@@ -822,7 +870,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         if (range_bad) status |= HQ_ST_RANGE;
         const unsigned long long total = nc + nr + ((unsigned long long)urun + 31) / 32;
         payload += urun + (unsigned long long)rbits + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
-        lookback_publish(a.lookback, c, total);
+        lookback_publish(a.lookback, c, total, ic.local == 0);
 
         // the previous chunk's predecessors have had a whole chunk's time to publish
         if (have_pend)
@@ -832,6 +880,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         pend.total = total;
         pend.overflow = overflow;
         pend.range_bad = range_bad;
+        pend.item = ic.item;
+        pend.local = ic.local;
         have_pend = true;
         c = cn;
         buf ^= 1;
@@ -841,7 +891,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
                                        lookback_peek(a.lookback, pend.c));
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 
-    stats_add_warp<LAT>(a, status, zor_all, payload, rng);
+    stats_add_warp<LAT>(a, status, zor_all, payload, rng, cur_item);
     stats_finish_cta(a);
 }
 
@@ -871,7 +921,7 @@ __device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending 
                                              uint32_t &status, unsigned long long first) {
     const int lane = threadIdx.x & 31;
     bool to = false;
-    const unsigned long long excl = lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to, first);
+    const unsigned long long excl = lookback_resolve(a.lookback, p.c, p.total, a.spin_limit, to, first, p.c == 0);
     if (to) status |= HQ_ST_TIMEOUT;
     const unsigned long long start = base + excl;
     if (lane == 0) {
@@ -886,7 +936,7 @@ __device__ __forceinline__ void finish_chunk(const EncodeArgs &a, const Pending 
         if (p.c == 0 && a.row) *a.row = a.row_val;
     }
     if (!p.range_bad && !p.overflow) {
-        copy_stage_out<true>(a, stage, start, (uint32_t)p.total, lane);
+        copy_stage_out<true>(a, a.stream, stage, start, (uint32_t)p.total, lane);
     } else if (!p.range_bad) {
         uint32_t *g = a.stream + start;
         const unsigned long long room = (start < a.cap_words) ? a.cap_words - start : 0ull;
@@ -1056,7 +1106,7 @@ __global__ void __launch_bounds__((ROT ? kRotGroups : kGroups) * kGroupWarps * 3
                 }
             }
             if (w == 0) {
-                lookback_publish(a.lookback, c, total);
+                lookback_publish(a.lookback, c, total, c == 0);
                 if (range_bad) status |= HQ_ST_RANGE;
                 if (lane == 0) payload += U + (unsigned long long)rbits + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
             }
@@ -1308,7 +1358,7 @@ __global__ void __launch_bounds__(kWideWarps * 32, 1) encode_kernel_wide(const E
                 }
             }
             if (w == 0) {
-                lookback_publish(a.lookback, c, total);
+                lookback_publish(a.lookback, c, total, c == 0);
                 if (range_bad) status |= HQ_ST_RANGE;
                 if (lane == 0) payload += U + (unsigned long long)nr * 32 + ((LAT == HQ_E8) ? 16ull * ntiles : 0ull);
             }

@@ -23,8 +23,11 @@ constexpr uint32_t kSpinLimit = 1u << 22;   // look-back polls before giving up 
 constexpr uint32_t kMaxUnaryBits = 1u << 31; // chunks with more unary bits are outside the supported range
 
 // Encoder workspace of n chunks: look-back words [0, 8n), ticket at 8n, done counter at
-// 8n + 4, stats accumulator at 8n + 8; all cleared by one memset of encode_scratch_bytes(n).
-inline size_t encode_scratch_bytes(uint64_t n_chunks) { return (size_t)n_chunks * 8 + 8 + sizeof(hq_stats); }
+// 8n + 4, stats accumulator at 8n + 8 (one per item of a batch); all cleared by one memset
+// of encode_scratch_bytes(n, items).
+inline size_t encode_scratch_bytes(uint64_t n_chunks, uint64_t items = 1) {
+    return (size_t)n_chunks * 8 + 8 + (size_t)items * sizeof(hq_stats);
+}
 
 // Salts xor-ed into the seed: "SIGN" for the sign diagonal, "DITH" for the dither.
 constexpr uint64_t kSignSalt = 0x5349474Eull;
@@ -64,6 +67,13 @@ struct EncodeArgs {
     int tcols;                // tile columns in the sign table (cols / 128, or 1 for KV)
     uint32_t spin_limit;
     const float *rot;         // KV: the dense rotation Q (128 x 128 fp32, row-major) or null (sign diagonal, H_128)
+    // A strided batch (hq_quantize_batch; 0 or 1: one matrix): item i of `batch` equally
+    // shaped matrices is chunks [i item_chunks, (i + 1) item_chunks) of the launch; its input
+    // starts i item_x_stride elements after x, its stream i item_stream_stride words after
+    // stream (cap_words each), its offsets i (item_chunks + 1) entries after offsets, its
+    // stats and workspace accumulator i entries after stats and acc.  The per-warp form only.
+    uint64_t batch, item_chunks, item_stream_stride;
+    int64_t item_x_stride;
 };
 
 struct DecodeArgs {
@@ -90,6 +100,13 @@ struct DecodeArgs {
     float *res;               // gemv: one partial per tile [rows * tcols]; scores: [heads * group, out_ld]
     int group;                // scores: query heads per KV head
     const float *rot;         // KV: the dense rotation Q, or null
+    // A strided batch (hq_dequantize_batch; 0 or 1: one matrix): chunk c of the launch is
+    // chunk c mod item_chunks of item c / item_chunks, whose stream starts i item_stream_stride
+    // words after stream (stream_words each), offsets i (item_chunks + 1) entries after
+    // offsets, output i item_out_stride elements after out, stats i entries after stats.
+    // Stored tiles only.
+    uint64_t batch, item_chunks, item_stream_stride;
+    int64_t item_out_stride;
 };
 
 // Decoder outputs: the tile itself, its dot product with x, or its dot products with queries.

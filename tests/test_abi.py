@@ -205,6 +205,29 @@ def test_static_entry_point_applies_the_same_checks():
     assert lib.hq_quantize_static(None, 32, 128, 128, C.byref(p), None, 0, None, None, None) == hq.HQ_EUNSUPPORTED
 
 
+def test_batch_entry_points_check_their_arguments():
+    """Strided batches: sizes and argument errors, all before any device work (null pointers only)."""
+    import lattice_entropy_coded_b200 as hq
+    lib = hq._lib
+    p = hq.make_params("E8", 300.0, 2)
+    assert hq.hq_batch_workspace_bytes(64, 16384) >= 64 * 16384 * 8 + 8 + 64 * hq.STATS_BYTES
+    assert hq.hq_batch_workspace_bytes(64, 16384) % 256 == 0
+    assert hq.hq_batch_workspace_bytes(0, 16384) >= 8
+    q = lambda *a: lib.hq_quantize_batch(*a)
+    # batch < 0; batch * chunks beyond 2^31; batch 0 is a no-op
+    assert q(None, -1, 0, 32, 128, 128, C.byref(p), None, 0, 0, None, None, None, 0, None) == hq.HQ_EINVAL
+    assert q(None, 1 << 30, 0, 4096, 4096, 4096, C.byref(p), None, 0, 0, None, None, None, 0,
+             None) == hq.HQ_EUNSUPPORTED
+    assert q(None, 0, 0, 32, 128, 128, C.byref(p), None, 0, 0, None, None, None, 0, None) == hq.HQ_OK
+    # batch >= 2 with null buffers or strides that overlap the items
+    assert q(None, 2, 4096, 32, 128, 128, C.byref(p), None, 100, 100, None, None, None, 0, None) == hq.HQ_EINVAL
+    d = lambda *a: lib.hq_dequantize_batch(*a)
+    assert d(None, 0, 0, None, -1, 32, 128, C.byref(p), None, 0, 128, 4096, None, None) == hq.HQ_EINVAL
+    assert d(None, 0, 0, None, 0, 32, 128, C.byref(p), None, 0, 128, 4096, None, None) == hq.HQ_OK
+    assert d(None, 10, 5, None, 3, 32, 128, C.byref(p), None, 0, 128, 4096, None, None) == hq.HQ_EINVAL
+    assert d(None, 10, 5, None, 3, 32, 128, C.byref(p), None, 2, 128, 4096, None, None) == hq.HQ_EINVAL
+
+
 def test_binding_fails_loudly_without_the_library(tmp_path):
     """The binding has no fallback: a missing libhq.so is an import error."""
     import subprocess
