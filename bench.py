@@ -999,6 +999,54 @@ def run_case(args):
                                           "bf16_gemv": 2.0 * n + 2.0 * cols}}), flush=True)
 
 
+def run_case_batch(args):
+    """Matrices 0..B-1 of the Student-t set (R x C corners) coded by one hq_quantize_batch
+    launch and decoded by one hq_dequantize_batch launch, back to back, no L2 flush: the case
+    the ncu captures of the benchmark's batched launches run on."""
+    import lattice_entropy_coded_b200 as hq
+    rows, cols = (int(v) for v in args.case.lower().split("x"))
+    B = args.case_batch
+    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    seed = w["seed"]
+    p = [q for q in rate_points()[DEFAULT_WORKLOAD]["points"] if q["bps"] == args.bps][0]
+    device = torch.device("cuda", 0)
+    x = torch.empty(B, rows, cols, dtype=torch.bfloat16, device=device)
+    for i, m in enumerate(synth.student_t(B, w["rows"], w["cols"], seed, device=device)):
+        x[i].copy_(m[:rows, :cols])
+    params = hq.make_params(p["lattice"], p["alpha"], p["k"], seed, 0)
+    n = rows * cols
+    cap = int(n * (p["bps"] + 3.0) / 32) + 8192
+    nch = hq.hq_stream_bound(rows, cols, params)[1]
+    words = torch.empty(B, cap, dtype=torch.int32, device=device)
+    offs = torch.empty(B, nch + 1, dtype=torch.int64, device=device)
+    st = torch.zeros(B, hq.STATS_BYTES, dtype=torch.uint8, device=device)
+    ws = torch.empty(hq.hq_batch_workspace_bytes(B, nch), dtype=torch.uint8, device=device)
+    out = torch.empty(B, rows, cols, dtype=torch.bfloat16, device=device)
+    ev = []
+    for i in range(args.warmup + args.steps):
+        a, b, c = _events(3)
+        a.record()
+        hq.hq_quantize_batch(x, params, words, offs, st, ws)
+        b.record()
+        hq.hq_dequantize_batch(words, cap, offs, rows, cols, params, out)
+        c.record()
+        if i >= args.warmup:
+            ev.append((a, b, c))
+    torch.cuda.synchronize()
+    stats = [hq.read_stats(st[i]) for i in range(B)]
+    enc = float(np.median([a.elapsed_time(b) for a, b, _ in ev]))
+    dec = float(np.median([b.elapsed_time(c) for _, b, c in ev]))
+    wds = int(offs[:, -1].sum().item())
+    alg = 2.0 * n * B + 4.0 * wds + 8.0 * B * (nch + 1)
+    peak, _ = measured_peaks()
+    print(json.dumps({"case": f"{B} x {args.case}", "data": "student_t", "lattice": p["lattice"], "bps": p["bps"],
+                      "status": max(s_["status"] for s_ in stats),
+                      "bps_payload": sum(s_["payload_bits"] for s_ in stats) / (n * B),
+                      "enc_ms": enc, "dec_ms": dec, "elements": n * B, "alg_bytes": alg,
+                      "enc_gbs_in": 2.0 * n * B / enc / 1e6, "dec_gbs_in": 2.0 * n * B / dec / 1e6,
+                      "enc_frac": alg / enc / 1e6 / peak, "dec_frac": alg / dec / 1e6 / peak}), flush=True)
+
+
 def run_token_case(args):
     """One-token KV appends, as a decode step makes them: 8 heads, E8 with dither at the K 2.0 bps
     point of the 8-head KV workload; 128 appends replayed from a CUDA graph, then the same appends
@@ -1058,6 +1106,9 @@ def main():
     ap.add_argument("--case", default=None, help="RxC: time one matrix (profiling case)")
     ap.add_argument("--case-data", default="weight", choices=["weight", "student_t"],
                     help="--case input: the sweep's Gaussian weights, or matrix 0 of the Student-t set")
+    ap.add_argument("--case-batch", type=int, default=0,
+                    help="with --case-data student_t: code matrices 0..B-1 of the set with one batched "
+                         "launch each way (hq_quantize_batch / hq_dequantize_batch) instead of one matrix")
     ap.add_argument("--token-case", action="store_true", help="time one-token KV appends (profiling case)")
     ap.add_argument("--lattice", default="E8")
     ap.add_argument("--bps", type=float, default=4.0)
@@ -1065,7 +1116,10 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.case:
-        run_case(args)
+        if args.case_batch:
+            run_case_batch(args)
+        else:
+            run_case(args)
         return
     if args.token_case:
         run_token_case(args)

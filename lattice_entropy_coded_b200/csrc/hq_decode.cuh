@@ -434,7 +434,7 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
                             m[i] = unzigzag(imad(qv[bb * N + i], (N > 1 && i == N - 1) ? pkl : pk, rv[bb * N + i]));
                         L::reinsert(m, (coset >> b) & 1u, qq);
                     }
-                    L::point(qq, p);
+                    decoded_point<LAT>(qq, p);
                     if (DITHER) {
                         float d[N];
                         dither_block<LAT>(a.seed, eq + (unsigned long long)(8 * g + bb * N), d);
@@ -568,7 +568,6 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
         }
         __syncwarp();
 
-        const unsigned long long c = v >> lg;
         const int r0 = (int)(v & ((1u << lg) - 1u)) << (2 - lg), r1 = r0 + (kRoundsPerChunk >> lg);
         ChunkOut<KV> geo;
         geo.init(a, cw.local, cw.item);

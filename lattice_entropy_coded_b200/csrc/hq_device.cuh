@@ -583,6 +583,28 @@ __device__ __forceinline__ void e8_codes_from_symbols(const uint32_t (&z)[8], ui
     q[7] = (int32_t)((t7 << 1) | (x & 2u) | c);
 }
 
+// ------------------------------------------------------------------ decoded points
+// fp32 value of an integer code q with -2^22 <= q < 2^22, without the conversion pipe:
+// 1.5 * 2^23 + q has spacing 1 there, so its bit pattern is that of the constant plus q
+// and subtracting the constant is exact.
+__device__ __forceinline__ float small_int_float(int32_t q) {
+    return __fsub_rn(__int_as_float(q + kRoundMagicBits), kRoundMagic);
+}
+// The lattice point of decoded codes (Lattice<LAT>::point), for codes rebuilt from
+// symbols below 2^22 (the encoder flags larger ones): every coordinate except E8's last,
+// whose code (4 m_7' + 2 p + c) may reach 2^23, is in small_int_float's range.
+template <int LAT>
+__device__ __forceinline__ void decoded_point(const int32_t (&q)[Lattice<LAT>::N], float (&p)[Lattice<LAT>::N]) {
+    if constexpr (LAT == HQ_A2) {
+        p[0] = __fmul_rn(small_int_float(q[0]), 0.5f);
+        p[1] = __fmul_rn(small_int_float(q[1]), HQ_SQRT3_2);
+    } else {
+        constexpr int N = Lattice<LAT>::N;
+#pragma unroll
+        for (int i = 0; i < N; i++) p[i] = (LAT == HQ_E8 && i == N - 1) ? (float)q[i] : small_int_float(q[i]);
+    }
+}
+
 // ------------------------------------------------------------------ integer range of the codes
 // The pages store the embedding's integers in 8 bits, with alpha chosen so that they fit
 // (explainer pages, "Methodology" 2, the integer implementation); the encoders report the
@@ -604,7 +626,7 @@ __device__ __forceinline__ uint32_t key_int8_limit() {
 // bits in cbits, bit b for block b), rebuilt from the symbols.  The rare path: taken only when
 // a key reached key_int8_limit.
 template <int LAT, int S>
-__device__ __forceinline__ uint32_t int8_overflow(const uint32_t (&z)[S], uint32_t cbits) {
+__device__ __noinline__ uint32_t int8_overflow(const uint32_t (&z)[S], uint32_t cbits) {
     constexpr int N = Lattice<LAT>::N;
     uint32_t n = 0;
 #pragma unroll
