@@ -131,3 +131,30 @@ def test_decode_leaves_range_zero():
     hq.hq_dequantize(g["words_t"], g["cap"], g["offsets_t"], 64, 512, p, out, st)
     torch.cuda.synchronize()
     assert _rng(hq.read_stats(st)) == (0, 0)
+
+
+@pytest.mark.parametrize("lat,alpha,dither", [("E8", 3000.0, 0), ("E8", 314.15, 1), ("D4", 2000.0, 0),
+                                              ("A2", 2500.0, 1), ("Z", 700.0, 0)])
+def test_max_symbol_is_the_or_of_all_symbols(path, lat, alpha, dither):
+    """hq_stats.max_symbol is the bitwise OR of every zigzag symbol of the call (its bit
+    length bounds them all, the figure hq_stream_bound's max_abs_symbol takes): every chunk
+    of the oracle's stream decoded back to codes, each lattice block stripped to its symbols
+    by the oracle, and the OR taken."""
+    hq = _hq()
+    L = O.LATTICES[lat]
+    n = O.DIM[L]
+    for rows, cols in ((37, 384), (64, 1024)):
+        x = synth.weight(rows, cols, seed=33)
+        p = hq.make_params(lat, alpha, 3, 9, dither)
+        g = gpu_quantize(x.cuda(), p)
+        s, off, _ = O.quantize(x, L, alpha, 3, 9, dither)
+        want = 0
+        for c in range(O.n_chunks(rows, cols)):
+            nt = min(32, rows * cols // 128 - 32 * c)
+            q = O.decode_chunk(L, 3, s[int(off[c]):int(off[c + 1])], nt)
+            for b in range(q.size // n):
+                m, _ = O.strip(L, q[b * n:(b + 1) * n])
+                for v in m:
+                    want |= O.zigzag(int(v))
+        assert g["stats"]["status"] == 0
+        assert g["stats"]["max_symbol"] == want, (rows, cols, g["stats"]["max_symbol"], want)
