@@ -95,12 +95,18 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
         const size_t smem =
             (size_t)(a.tcols * kSignWords + kWarpsPerCta * 2 * kStageWords + kWarpsPerCta * 32 * kInSlotWords) *
             sizeof(uint32_t);
+        // weights whose rows hold whole rounds (cols a multiple of 8 tiles): every round is one
+        // 2 KB run of x, 16-byte aligned (x, ld and the item stride are checked at the API),
+        // brought in by one bulk copy
+        const bool bulk = !mixed && !a.map.kv && a.map.cols % (kTilesPerRound * kTile) == 0 &&
+                          ((uintptr_t)a.x & 15u) == 0 && a.map.ld % 8 == 0 && (a.batch <= 1 || a.item_x_stride % 8 == 0);
         auto kern = mixed ? encode_kernel<LAT, DITHER, false, true>
+                    : bulk ? (small ? encode_kernel<LAT, DITHER, true, false, true>
+                                    : encode_kernel<LAT, DITHER, false, false, true>)
                     : small ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
-        static LaunchPlan plans[3];
-        if ((e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem,
-                                                        (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid)) !=
-            cudaSuccess)
+        static LaunchPlan plans[5];
+        if ((e = plans[mixed ? 2 : (small ? 1 : 0) + (bulk ? 3 : 0)].grid(
+                 kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid)) != cudaSuccess)
             return e;
         kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     }

@@ -276,6 +276,39 @@ __device__ __forceinline__ void prefetch_round(const EncodeArgs &a, const ChunkG
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
+// Bulk form of the per-warp kernel's input (BULK: weights whose rows hold whole rounds):
+// the round's 8 tiles are one 2 KB run of x, copied by a single cp.async.bulk issued by
+// lane 0 into the warp's buffer and completed on the warp's mbarrier (transaction count
+// 2048 bytes).  Lane l then reads bytes [64 l, 64 l + 64): its quarter l % 4 of tile l / 4,
+// as in the per-lane form.
+constexpr uint32_t kRoundBytes = kTilesPerRound * kTile * 2;
+
+__device__ __forceinline__ void bulk_prefetch_round(const EncodeArgs &a, const ChunkGeo &geo, int r, uint32_t buf,
+                                                    uint32_t mb) {
+    const uint16_t *src = nullptr;
+    int tcol;
+    unsigned long long e0;
+    geo.tile(a.map, a.x, r * kTilesPerRound, src, tcol, e0);
+    // the buffer was last read through the generic proxy (ordered by the caller's __syncwarp)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(kRoundBytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(buf), "l"(src), "r"(kRoundBytes), "r"(mb) : "memory");
+}
+
+// Wait for the phase of parity `phase` of mbarrier mb to complete; false after `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint32_t mb, uint32_t phase, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; i++) {
+        uint32_t done;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(done) : "r"(mb), "r"(phase) : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
 __device__ __forceinline__ void round_input(const EncodeArgs &a, const ChunkGeo &geo, int r, int lane,
                                             RoundInput &in) {
     const uint16_t *src = nullptr;
@@ -732,9 +765,11 @@ __device__ __forceinline__ unsigned long long take_ticket(const EncodeArgs &a) {
 
 // Throughput form: persistent CTAs of kWarpsPerCta warps, each warp encoding whole
 // chunks (4 rounds of 8 tiles) taken by ticket, with a two-chunk stage pipeline.
+// BULK: each round's input arrives by one bulk copy (bulk_prefetch_round); otherwise
+// each lane copies its own 64 bytes (prefetch_round).
 // MIXED: the last symbol of each block has its own Rice parameter (a.k_last != a.k),
 // so lanes' remainder runs are not word-aligned (put_rem_mixed).
-template <int LAT, bool DITHER, bool KSMALL, bool MIXED = false>
+template <int LAT, bool DITHER, bool KSMALL, bool MIXED = false, bool BULK = false>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *sign_tab = smem;                                        // tcols * kSignWords
@@ -743,7 +778,18 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t *stages = stage_all + warp * 2 * kStageWords;
     uint32_t *slot = in_all + (warp * 32 + lane) * kInSlotWords;
+    // bulk form: the warp's 2 KB round buffer and its mbarrier (inside the warp's slots)
+    uint32_t *wbuf = in_all + warp * 32 * kInSlotWords;
+    const uint32_t wbuf_s = (uint32_t)__cvta_generic_to_shared(wbuf);
+    const uint32_t mb = wbuf_s + kRoundBytes;
+    constexpr bool bulk = BULK;
+    const uint32_t *rd = bulk ? wbuf + 16 * lane : slot;
+    uint32_t phase = 0;
 
+    if (bulk && lane == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mb) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     build_sign_table(sign_tab, a.tcols, a.seed);
     __syncthreads();
 
@@ -761,7 +807,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
         ChunkGeo g0;
         g0.init(a.map, ic.local);
         g0.xoff = (long long)ic.item * a.item_x_stride;
-        prefetch_round(a, g0, 0, lane, slot);
+        if (bulk) {
+            if (lane == 0) bulk_prefetch_round(a, g0, 0, wbuf_s, mb);
+        } else {
+            prefetch_round(a, g0, 0, lane, slot);
+        }
     }
     Pending pend;
     bool have_pend = false;
@@ -803,11 +853,31 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             // start the copy of the next round's
             RoundInput cur;
             round_input(a, geo, r, lane, cur);
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            if (bulk) {
+                // a wait that gives up flags the call and waits once more (bounded) for the copy
+                if (!mbar_wait(mb, phase, a.spin_limit)) {
+                    status |= HQ_ST_TIMEOUT;
+                    mbar_wait(mb, phase, a.spin_limit);
+                }
+                phase ^= 1u;
+            } else {
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+            }
             uint4 raw[4];
 #pragma unroll
-            for (int j = 0; j < 4; j++) raw[j] = *reinterpret_cast<const uint4 *>(slot + 4 * j);
-            if (r + 1 < nrounds) {
+            for (int j = 0; j < 4; j++) raw[j] = *reinterpret_cast<const uint4 *>(rd + 4 * j);
+            if (bulk) {
+                __syncwarp();   // every lane has its bytes before the buffer is refilled
+                if (r + 1 < nrounds) {
+                    if (lane == 0) bulk_prefetch_round(a, geo, r + 1, wbuf_s, mb);
+                } else if (cn < a.n_chunks) {
+                    const ItemChunk icn = item_chunk(a, cn);
+                    ChunkGeo gn;
+                    gn.init(a.map, icn.local);
+                    gn.xoff = (long long)icn.item * a.item_x_stride;
+                    if (lane == 0) bulk_prefetch_round(a, gn, 0, wbuf_s, mb);
+                }
+            } else if (r + 1 < nrounds) {
                 prefetch_round(a, geo, r + 1, lane, slot);
             } else if (cn < a.n_chunks) {
                 const ItemChunk icn = item_chunk(a, cn);

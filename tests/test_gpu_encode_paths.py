@@ -4,7 +4,9 @@ The encoder has a per-warp form (a warp encodes whole chunks; used for large
 launches), a grouped form (four warps share a chunk), a wide form (sixteen warps
 share a chunk) and a single-CTA form (one CTA for a launch of at most 32 chunks,
 such as a KV append of a few tokens; forced on a larger launch, the per-warp form
-runs).  By default the size decides;
+runs).  The per-warp form takes its input by one bulk copy per round where the
+rows hold whole rounds (cols a multiple of 1024: the 4096 and 65536 column cases)
+and by per-lane copies otherwise (384 columns, strided rows).  By default the size decides;
 here each form is forced in turn on the cases that exercise its control flow:
 ragged last chunks, every Rice parameter, strided rows, exact ties, chunks too
 large for the shared stage, capacity overflow, bounded look-back waits, KV
