@@ -200,9 +200,11 @@ struct ChunkGeo {
     // kv: head h, tokens tok_base + ti
     long long h, tok_base;
 
+    // KV false: the caller knows the map is a weights matrix (the KV branch is compiled out)
+    template <bool KV = true>
     __device__ __forceinline__ void init(const TileMap &m, unsigned long long c) {
         xoff = 0;
-        if (m.kv) {
+        if (KV && m.kv) {
             const long long cph = (m.tokens + 31) / 32;
             unsigned long long hq_, rq;
             divmod_u64(c, (unsigned long long)cph, hq_, rq);
@@ -222,10 +224,11 @@ struct ChunkGeo {
         }
     }
     // Tile ti (< 32) of the chunk: first element, sign-table column, dither counter of its element 0.
+    template <bool KV = true>
     __device__ __forceinline__ bool tile(const TileMap &m, const uint16_t *x, int ti, const uint16_t *&src,
                                          int &tcol, unsigned long long &e0) const {
         if (ti >= ntiles) return false;
-        if (m.kv) {
+        if (KV && m.kv) {
             long long tok = tok_base + ti;
             src = x + h * m.ld_head + tok * m.ld_tok;
             tcol = 0;
@@ -288,7 +291,7 @@ __device__ __forceinline__ void bulk_prefetch_round(const EncodeArgs &a, const C
     const uint16_t *src = nullptr;
     int tcol;
     unsigned long long e0;
-    geo.tile(a.map, a.x, r * kTilesPerRound, src, tcol, e0);
+    geo.tile<false>(a.map, a.x, r * kTilesPerRound, src, tcol, e0);
     // the buffer was last read through the generic proxy (ordered by the caller's __syncwarp)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(kRoundBytes) : "memory");
@@ -309,12 +312,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mb, uint32_t phase, uint32_t 
     return false;
 }
 
+template <bool KV = true>
 __device__ __forceinline__ void round_input(const EncodeArgs &a, const ChunkGeo &geo, int r, int lane,
                                             RoundInput &in) {
     const uint16_t *src = nullptr;
     in.tcol = 0;
     in.e0 = 0;
-    in.valid = geo.tile(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, in.tcol, in.e0);
+    in.valid = geo.template tile<KV>(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, in.tcol, in.e0);
 }
 
 // The transform of one round for one lane: D x -> H_128 (with the three partner
@@ -805,7 +809,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     if (c < a.n_chunks) {
         const ItemChunk ic = item_chunk(a, c);
         ChunkGeo g0;
-        g0.init(a.map, ic.local);
+        g0.init<!BULK>(a.map, ic.local);
         g0.xoff = (long long)ic.item * a.item_x_stride;
         if (bulk) {
             if (lane == 0) bulk_prefetch_round(a, g0, 0, wbuf_s, mb);
@@ -830,7 +834,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             cur_item = ic.item;
         }
         ChunkGeo geo;
-        geo.init(a.map, ic.local);
+        geo.init<!BULK>(a.map, ic.local);
         geo.xoff = (long long)ic.item * a.item_x_stride;
         uint32_t *stage = stages + buf * kStageWords;
 
@@ -852,7 +856,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             // this round's bytes are arriving in the lane's slot; take them, then
             // start the copy of the next round's
             RoundInput cur;
-            round_input(a, geo, r, lane, cur);
+            round_input<!BULK>(a, geo, r, lane, cur);
             if (bulk) {
                 // a wait that gives up flags the call and waits once more (bounded) for the copy
                 if (!mbar_wait(mb, phase, a.spin_limit)) {
@@ -873,7 +877,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
                 } else if (cn < a.n_chunks) {
                     const ItemChunk icn = item_chunk(a, cn);
                     ChunkGeo gn;
-                    gn.init(a.map, icn.local);
+                    gn.init<!BULK>(a.map, icn.local);
                     gn.xoff = (long long)icn.item * a.item_x_stride;
                     if (lane == 0) bulk_prefetch_round(a, gn, 0, wbuf_s, mb);
                 }
@@ -882,7 +886,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             } else if (cn < a.n_chunks) {
                 const ItemChunk icn = item_chunk(a, cn);
                 ChunkGeo gn;
-                gn.init(a.map, icn.local);
+                gn.init<!BULK>(a.map, icn.local);
                 gn.xoff = (long long)icn.item * a.item_x_stride;
                 prefetch_round(a, gn, 0, lane, slot);
             }
