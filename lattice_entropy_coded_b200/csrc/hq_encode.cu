@@ -97,8 +97,10 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
             sizeof(uint32_t);
         // weights whose rows hold whole rounds (cols a multiple of 8 tiles): every round is one
         // 2 KB run of x, 16-byte aligned (x, ld and the item stride are checked at the API),
-        // brought in by one bulk copy
+        // brought in by one bulk copy.  Fewer than 2^27 chunks (more than device memory holds)
+        // keep that kernel's chunk arithmetic 32-bit.
         const bool bulk = !mixed && !a.map.kv && a.map.cols % (kTilesPerRound * kTile) == 0 &&
+                          a.n_chunks < (1ull << 27) &&
                           ((uintptr_t)a.x & 15u) == 0 && a.map.ld % 8 == 0 && (a.batch <= 1 || a.item_x_stride % 8 == 0);
         auto kern = mixed ? encode_kernel<LAT, DITHER, false, true>
                     : bulk ? (small ? encode_kernel<LAT, DITHER, true, false, true>

@@ -184,9 +184,19 @@ __device__ __forceinline__ void stats_finish_cta(const EncodeArgs &a) {
 struct ItemChunk {
     unsigned long long item, local;
 };
+// NARROW: the launch has fewer than 2^27 chunks (32-bit divisions suffice).
+template <bool NARROW = false>
 __device__ __forceinline__ ItemChunk item_chunk(const EncodeArgs &a, unsigned long long c) {
     ItemChunk r{0ull, c};
-    if (a.batch > 1) divmod_u64(c, a.item_chunks, r.item, r.local);
+    if (a.batch > 1) {
+        if (NARROW) {
+            const uint32_t q = (uint32_t)c / (uint32_t)a.item_chunks;
+            r.item = q;
+            r.local = (uint32_t)c - q * (uint32_t)a.item_chunks;
+        } else {
+            divmod_u64(c, a.item_chunks, r.item, r.local);
+        }
+    }
     return r;
 }
 
@@ -200,8 +210,9 @@ struct ChunkGeo {
     // kv: head h, tokens tok_base + ti
     long long h, tok_base;
 
-    // KV false: the caller knows the map is a weights matrix (the KV branch is compiled out)
-    template <bool KV = true>
+    // KV false: the caller knows the map is a weights matrix (the KV branch is compiled out);
+    // NARROW: c < 2^27, so the chunk's first tile 32 c fits 32 bits
+    template <bool KV = true, bool NARROW = false>
     __device__ __forceinline__ void init(const TileMap &m, unsigned long long c) {
         xoff = 0;
         if (KV && m.kv) {
@@ -217,10 +228,16 @@ struct ChunkGeo {
             long long t0 = (long long)c * 32;
             long long all = m.rows * (long long)tpr;
             ntiles = (int)((all - t0) < 32 ? (all - t0) : 32);
-            unsigned long long rq, cq;
-            divmod_u64((unsigned long long)t0, (unsigned long long)tpr, rq, cq);
-            row0 = (long long)rq;
-            tc0 = (int)cq;
+            if (NARROW) {
+                const uint32_t rq = (uint32_t)t0 / (uint32_t)tpr;
+                row0 = rq;
+                tc0 = (int)((uint32_t)t0 - rq * (uint32_t)tpr);
+            } else {
+                unsigned long long rq, cq;
+                divmod_u64((unsigned long long)t0, (unsigned long long)tpr, rq, cq);
+                row0 = (long long)rq;
+                tc0 = (int)cq;
+            }
         }
     }
     // Tile ti (< 32) of the chunk: first element, sign-table column, dither counter of its element 0.
@@ -807,9 +824,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
 
     unsigned long long c = take_ticket(a);
     if (c < a.n_chunks) {
-        const ItemChunk ic = item_chunk(a, c);
+        const ItemChunk ic = item_chunk<BULK>(a, c);
         ChunkGeo g0;
-        g0.init<!BULK>(a.map, ic.local);
+        g0.init<!BULK, BULK>(a.map, ic.local);
         g0.xoff = (long long)ic.item * a.item_x_stride;
         if (bulk) {
             if (lane == 0) bulk_prefetch_round(a, g0, 0, wbuf_s, mb);
@@ -825,7 +842,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     unsigned long long cur_item = 0;
     while (c < a.n_chunks) {
         const unsigned long long cn = take_ticket(a);
-        const ItemChunk ic = item_chunk(a, c);
+        const ItemChunk ic = item_chunk<BULK>(a, c);
         if (ic.item != cur_item) {
             stats_add_warp<LAT>(a, status, zor_all, payload, rng, cur_item);
             status = zor_all = 0;
@@ -834,7 +851,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             cur_item = ic.item;
         }
         ChunkGeo geo;
-        geo.init<!BULK>(a.map, ic.local);
+        geo.init<!BULK, BULK>(a.map, ic.local);
         geo.xoff = (long long)ic.item * a.item_x_stride;
         uint32_t *stage = stages + buf * kStageWords;
 
@@ -875,18 +892,18 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
                 if (r + 1 < nrounds) {
                     if (lane == 0) bulk_prefetch_round(a, geo, r + 1, wbuf_s, mb);
                 } else if (cn < a.n_chunks) {
-                    const ItemChunk icn = item_chunk(a, cn);
+                    const ItemChunk icn = item_chunk<BULK>(a, cn);
                     ChunkGeo gn;
-                    gn.init<!BULK>(a.map, icn.local);
+                    gn.init<!BULK, BULK>(a.map, icn.local);
                     gn.xoff = (long long)icn.item * a.item_x_stride;
                     if (lane == 0) bulk_prefetch_round(a, gn, 0, wbuf_s, mb);
                 }
             } else if (r + 1 < nrounds) {
                 prefetch_round(a, geo, r + 1, lane, slot);
             } else if (cn < a.n_chunks) {
-                const ItemChunk icn = item_chunk(a, cn);
+                const ItemChunk icn = item_chunk<BULK>(a, cn);
                 ChunkGeo gn;
-                gn.init<!BULK>(a.map, icn.local);
+                gn.init<!BULK, BULK>(a.map, icn.local);
                 gn.xoff = (long long)icn.item * a.item_x_stride;
                 prefetch_round(a, gn, 0, lane, slot);
             }
