@@ -29,7 +29,9 @@
  *  - bf16 tensors are little-endian IEEE bfloat16, 16-byte aligned, with
  *    element strides that are multiples of 8 elements (16 bytes).
  *  - A tile is 128 consecutive elements of a row; a chunk is 32 consecutive
- *    tiles (4096 elements).  Weights: tiles in row-major order of an R x C
+ *    tiles (4096 elements).  A weights matrix (or a strided batch of them, per
+ *    launch) has at most 2^27 chunks (2^39 elements, more than device memory
+ *    holds); larger requests return HQ_EUNSUPPORTED.  Weights: tiles in row-major order of an R x C
  *    matrix (C % 128 == 0), chunk c = tiles [32c, 32c+32).  KV cache: per
  *    append of T tokens and H heads, ceil(T/32) chunks per head, head-major;
  *    one tile = one token's 128-dim head vector.
@@ -243,7 +245,8 @@ HQ_API int hq_quantize_batch(const void *x, int64_t batch, int64_t x_stride, int
  * its offsets) at d_stream + i * stream_stride, offsets at d_offsets + i * (n_chunks + 1),
  * output at out + i * out_stride elements (out_stride % 8 == 0 for bf16, % 4 for fp32,
  * >= (rows - 1) * ld + cols), stats d_stats + i (HQ_ST_CORRUPT per item).  Each item's
- * output is exactly hq_dequantize's.  batch 1 is hq_dequantize. */
+ * output is exactly hq_dequantize's.  batch 1 is hq_dequantize.  HQ_EUNSUPPORTED when
+ * batch * n_chunks exceeds 2^27. */
 HQ_API int hq_dequantize_batch(const uint32_t *d_stream, uint64_t stream_stride, uint64_t stream_words,
                                const uint64_t *d_offsets, int64_t batch, int64_t rows, int64_t cols,
                                const hq_params *p, void *out, int out_dtype, int64_t ld, int64_t out_stride,

@@ -49,7 +49,8 @@ int check_weight_params(const hq_params *p) {
 int check_matrix(int64_t rows, int64_t cols) {
     if (rows < 0 || cols < 0 || cols % kTile) return HQ_EINVAL;
     if (cols > kMaxCols) return HQ_EUNSUPPORTED;
-    if (rows > 0 && cols > 0 && rows > (INT64_C(1) << 40) / cols) return HQ_EUNSUPPORTED;
+    // at most 2^39 elements (2^27 chunks): the weights decoder's chunk arithmetic is 32-bit
+    if (rows > 0 && cols > 0 && rows > (INT64_C(1) << 39) / cols) return HQ_EUNSUPPORTED;
     return HQ_OK;
 }
 
@@ -285,7 +286,7 @@ int hq_dequantize_batch(const uint32_t *d_stream, uint64_t stream_stride, uint64
     if (out_dtype != 0 && out_dtype != 1) return HQ_EINVAL;
     if (d_stats && !aligned(d_stats, 8)) return HQ_EINVAL;
     const uint64_t nch = chunks_of(rows, cols);
-    if (batch > 0 && nch > 0 && (uint64_t)batch > (UINT64_C(1) << 40) / nch) return HQ_EUNSUPPORTED;
+    if (batch > 0 && nch > 0 && (uint64_t)batch > (UINT64_C(1) << 27) / nch) return HQ_EUNSUPPORTED;
     if (batch == 0) return HQ_OK;
     cudaStream_t s = (cudaStream_t)cuda_stream;
     if (d_stats && cudaMemsetAsync(d_stats, 0, (size_t)batch * sizeof(hq_stats), s) != cudaSuccess) return HQ_ECUDA;

@@ -213,13 +213,13 @@ struct ChunkOut {
             ntiles = (int)(left < 32 ? left : 32);
             e_scale = row.scale_inv;
         } else {
+            // a weights launch has at most 2^27 chunks (the API's limit): 32 c fits 32 bits
             tpr = (int)(a.map.cols / kTile);
             const long long t0 = (long long)c * 32, all = a.map.rows * (long long)tpr;
             ntiles = (int)((all - t0) < 32 ? (all - t0) : 32);
-            unsigned long long rq, cq;
-            divmod_u64((unsigned long long)t0, (unsigned long long)tpr, rq, cq);
-            row0 = (long long)rq;
-            tc0 = (int)cq;
+            const uint32_t rq = (uint32_t)t0 / (uint32_t)tpr;
+            row0 = rq;
+            tc0 = (int)((uint32_t)t0 - rq * (uint32_t)tpr);
             e_scale = a.e_scale;
         }
     }
@@ -270,7 +270,12 @@ __device__ __forceinline__ ChunkWords chunk_words(const DecodeArgs &a, unsigned 
     ChunkWords r;
     r.item = 0;
     r.local = c;
-    if (a.batch > 1) divmod_u64(c, a.item_chunks, r.item, r.local);
+    if (a.batch > 1) {
+        // a strided batch has at most 2^27 chunks in all (the API's limit)
+        const uint32_t q = (uint32_t)c / (uint32_t)a.item_chunks;
+        r.item = q;
+        r.local = (uint32_t)c - q * (uint32_t)a.item_chunks;
+    }
     const uint64_t *offs = a.offsets + r.item * (a.batch > 1 ? a.item_chunks + 1 : 0ull);
     r.w0 = offs[r.local];
     const unsigned long long w1 = offs[r.local + 1];
