@@ -836,7 +836,11 @@ def run_bulk(args):
         flush = (torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
                  if 2 * n < L2_FLUSH_BYTES else None)
         res = []
-        for p in pts:
+        if not w.get("dk_last") and len(mats) > 1:
+            # a set of matrices: equally shaped ones coded by one hq_quantize_batch launch and decoded
+            # by one hq_dequantize_batch launch each way, as a model's weights would be
+            out["points"] = [weight_set_batched(hq, mats, p, w["seed"], args, device, peak) for p in pts]
+        for p in (pts if "points" not in out else []):
             params = hq.make_params(p["lattice"], p["alpha"], p["k"], w["seed"], 0, dk_last=p.get("dk_last", 0))
             codecs = [hq.Codec(m.shape[0], m.shape[1], params, device=device,
                                cap_words=int(m.numel() * (p["bps"] + 3.0) / 32) + 8192) for m in mats]
@@ -876,7 +880,8 @@ def run_bulk(args):
                             **({"dk_last": p["dk_last"]} if "dk_last" in p else {})))
             del codecs, outs, comps
             torch.cuda.empty_cache()
-        out["points"] = res
+        if res:
+            out["points"] = res
         if w["kind"] == "student_t":
             out["calibration"] = calibrate_set(hq, mats, pts, w["seed"])
     if args.oracle:
@@ -887,6 +892,65 @@ def run_bulk(args):
         if w["kind"] == "weight":
             out["oracle"]["single_thread"] = oracle_workload(wl, 1, pts=pts if w.get("dk_last") else None)
     print(json.dumps(out), flush=True)
+
+
+def weight_set_batched(hq, mats, p, seed, args, device, peak):
+    """One operating point over a set of matrices, grouped by shape: per group one
+    hq_quantize_batch launch (all groups between one pair of events), then one
+    hq_dequantize_batch launch per group back to bf16.  Inputs resident; the set is
+    larger than L2."""
+    params = hq.make_params(p["lattice"], p["alpha"], p["k"], seed, 0)
+    groups = {}
+    for m in mats:
+        groups.setdefault(tuple(m.shape), []).append(m)
+    gs = []
+    for (rows, cols), ms in groups.items():
+        x = torch.stack(ms)
+        B = x.shape[0]
+        cap = int(rows * cols * (p["bps"] + 3.0) / 32) + 8192
+        _, nch = hq.hq_stream_bound(rows, cols, params)
+        gs.append(dict(x=x, rows=rows, cols=cols, cap=cap, nch=nch,
+                       words=torch.empty(B, cap, dtype=torch.int32, device=device),
+                       offs=torch.empty(B, nch + 1, dtype=torch.int64, device=device),
+                       st=torch.zeros(B, hq.STATS_BYTES, dtype=torch.uint8, device=device),
+                       dst=torch.zeros(B, hq.STATS_BYTES, dtype=torch.uint8, device=device),
+                       ws=torch.empty(hq.hq_batch_workspace_bytes(B, nch), dtype=torch.uint8, device=device),
+                       out=torch.empty_like(x)))
+    del groups
+    enc_ms, dec_ms = [], []
+    for it in range(args.warmup + args.steps):
+        e0, e1 = _events()
+        e0.record()
+        for g in gs:
+            hq.hq_quantize_batch(g["x"], params, g["words"], g["offs"], g["st"], g["ws"], cap_words=g["cap"])
+        e1.record()
+        d0, d1 = _events()
+        d0.record()
+        for g in gs:
+            hq.hq_dequantize_batch(g["words"], g["cap"], g["offs"], g["rows"], g["cols"], params, g["out"], g["dst"])
+        d1.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            enc_ms.append(e0.elapsed_time(e1))
+            dec_ms.append(d0.elapsed_time(d1))
+    n = sum(g["x"].numel() for g in gs)
+    stats = [hq.read_stats(g["st"][i]) for g in gs for i in range(g["x"].shape[0])]
+    dstat = max(hq.read_stats(g["dst"][i])["status"] for g in gs for i in range(g["x"].shape[0]))
+    words = sum(int(g["offs"][:, -1].sum().item()) for g in gs)
+    nch = sum(g["x"].shape[0] * (g["nch"] + 1) for g in gs)
+    se = sum(float(((g["out"].double() - g["x"].double()) ** 2).sum()) for g in gs)
+    var = sum(float(m.double().var()) * m.numel() for m in mats) / n
+    em, dm = float(np.median(enc_ms)), float(np.median(dec_ms))
+    alg = 2.0 * n + 4.0 * words + 8.0 * nch
+    return dict(lattice=p["lattice"], bps_target=p["bps"], k=p["k"], alpha=p["alpha"],
+                status=max(st["status"] for st in stats) | dstat,
+                bps_payload=sum(st["payload_bits"] for st in stats) / n, bps_stream=words * 32.0 / n,
+                mse=se / n, d_over_sigma2=se / n / var, matrices=len(mats), elements=n,
+                launches_per_direction=len(gs), shapes=[[g["x"].shape[0], g["rows"], g["cols"]] for g in gs],
+                max_abs_code=max(st["max_abs_code"] for st in stats),
+                int8_overflow_count=sum(st["int8_overflow_count"] for st in stats),
+                encode_ms=em, decode_ms=dm, encode_gbs=2.0 * n / (em * 1e6), decode_gbs=2.0 * n / (dm * 1e6),
+                encode_hbm_frac=alg / (em * 1e6) / peak, decode_hbm_frac=alg / (dm * 1e6) / peak)
 
 
 def calibrate_set(hq, mats, pts, seed):
