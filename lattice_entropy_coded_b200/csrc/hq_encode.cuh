@@ -119,7 +119,14 @@ struct CodeRange {
     template <int LAT, int S>
     __device__ __forceinline__ void add(uint32_t rkey, const uint32_t (&z)[S], uint32_t cbits) {
         key = max(key, rkey);
-        if (rkey >= key_int8_limit<LAT>()) ovf += int8_overflow<LAT, S>(z, cbits);
+        if (rkey >= key_int8_limit<LAT>()) {
+            // the out-of-line recount takes its symbols from memory: copy them there only on this
+            // rare path, so that z itself stays in registers every round
+            uint32_t zc[S];
+#pragma unroll
+            for (int i = 0; i < S; i++) zc[i] = z[i];
+            ovf += int8_overflow<LAT, S>(zc, cbits);
+        }
     }
 };
 

@@ -21,3 +21,9 @@ def test_readme_python_example_runs():
     assert abs(env["cal"]["bps"] - 4.0) <= 0.002
     assert env["s"].shape == (32, 256) and bool(torch.isfinite(env["s"]).all())
     assert hq.read_stats(env["rcache"].stats)["status"] == 0 and env["rcache"].tokens == 256
+    # the batch decodes to what single calls give
+    Ws, Ws_hat, p = env["Ws"], env["Ws_hat"], env["p"]
+    one = hq.Codec(1024, 4096, p)
+    ref = one.dequantize(one.quantize(Ws[5]), torch.empty_like(Ws[5]))
+    torch.cuda.synchronize()
+    assert torch.equal(Ws_hat[5], ref)
