@@ -487,17 +487,24 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
                 }
             }
         } else if (dst) {
-            const uint32_t es = ROT ? 0u : sign_tab[tcol * kSignWords + q];
+            // a bad tile is stored as +0: its values zeroed and no sign flipped (rare, so a
+            // branch rather than a select per word)
+            uint32_t es = ROT ? 0u : sign_tab[tcol * kSignWords + q];
+            if (tile_bad) {
+                es = 0u;
+#pragma unroll
+                for (int j = 0; j < 16; j++) v[j] = make_float2(0.0f, 0.0f);
+            }
             if (a.out_fp32) {
                 uint4 *o = reinterpret_cast<uint4 *>(dst) + 8 * q;
 #pragma unroll
                 for (int j = 0; j < 8; j++) {
                     const uint32_t m0 = sign_pair_mask(es, 2 * j), m1 = sign_pair_mask(es, 2 * j + 1);
                     uint4 w;
-                    w.x = tile_bad ? 0u : __float_as_uint(v[2 * j].x) ^ (m0 << 16);
-                    w.y = tile_bad ? 0u : __float_as_uint(v[2 * j].y) ^ (m0 & 0x80000000u);
-                    w.z = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].x) ^ (m1 << 16);
-                    w.w = tile_bad ? 0u : __float_as_uint(v[2 * j + 1].y) ^ (m1 & 0x80000000u);
+                    w.x = __float_as_uint(v[2 * j].x) ^ (m0 << 16);
+                    w.y = __float_as_uint(v[2 * j].y) ^ (m0 & 0x80000000u);
+                    w.z = __float_as_uint(v[2 * j + 1].x) ^ (m1 << 16);
+                    w.w = __float_as_uint(v[2 * j + 1].y) ^ (m1 & 0x80000000u);
                     o[j] = w;
                 }
             } else {
@@ -508,7 +515,7 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
 #pragma unroll
                     for (int u2 = 0; u2 < 4; u2++) {
                         __nv_bfloat162 hb = __floats2bfloat162_rn(v[4 * j + u2].x, v[4 * j + u2].y);
-                        pk[u2] = tile_bad ? 0u : (*reinterpret_cast<uint32_t *>(&hb) ^ sign_pair_mask(es, 4 * j + u2));
+                        pk[u2] = *reinterpret_cast<uint32_t *>(&hb) ^ sign_pair_mask(es, 4 * j + u2);
                     }
                     o[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
