@@ -20,11 +20,22 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
     const bool small = a.k <= 4, mixed = a.k_last != a.k;
     auto kern = mixed ? decode_kernel<LAT, DITHER, KV, false, kStoreTiles, false, true>
                 : small ? decode_kernel<LAT, DITHER, KV, true, kStoreTiles> : decode_kernel<LAT, DITHER, KV, false, kStoreTiles>;
-    static LaunchPlan plans[3];
+    int plan_i = mixed ? 2 : small ? 1 : 0;
+    if constexpr (LAT == HQ_E8 && !DITHER && !KV) {
+        // E8 weights at the common rates (k = 1 .. 4): the Rice parameter compiled in
+        if (!mixed && a.k >= 1 && a.k <= 4) {
+            plan_i = 2 + a.k;
+            kern = a.k == 1   ? decode_kernel<LAT, DITHER, KV, true, kStoreTiles, false, false, 1>
+                   : a.k == 2 ? decode_kernel<LAT, DITHER, KV, true, kStoreTiles, false, false, 2>
+                   : a.k == 3 ? decode_kernel<LAT, DITHER, KV, true, kStoreTiles, false, false, 3>
+                              : decode_kernel<LAT, DITHER, KV, true, kStoreTiles, false, false, 4>;
+        }
+    }
+    static LaunchPlan plans[7];
     unsigned grid = 0;
     // at most one CTA per round (the kernel deals rounds to CTAs first)
-    cudaError_t e = plans[mixed ? 2 : small ? 1 : 0].grid(kern, kWarpsPerCta * 32, smem,
-                                                           (unsigned long long)kRoundsPerChunk * a.n_chunks, grid);
+    cudaError_t e = plans[plan_i].grid(kern, kWarpsPerCta * 32, smem, (unsigned long long)kRoundsPerChunk * a.n_chunks,
+                                       grid);
     if (e != cudaSuccess) return e;
     kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     return cudaGetLastError();

@@ -369,14 +369,14 @@ __device__ __forceinline__ float tile_sum(float acc) {
 // Rounds [r0, r1) of one chunk, reading its planes from `src` (a stage when STAGED).
 // ROT: the dense KV rotation's inverse (rot_s: its shared form) in place of H_128
 // and the sign diagonal.
-template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED, int MODE, bool ROT, bool MIXED>
+template <int LAT, bool DITHER, bool KV, bool KSMALL, bool STAGED, int MODE, bool ROT, bool MIXED, int KC = -1>
 __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOut<KV> &geo, const uint32_t *src,
                                               bool ok, uint32_t nc, uint32_t nr, uint32_t nu,
                                               const uint32_t *startbit, const uint32_t *sign_tab,
                                               const float *rot_s, int r0, int r1, int lane) {
     using L = Lattice<LAT>;
     constexpr int N = L::N;
-    const int k = a.k, kl = a.k_last;
+    const int k = KC >= 0 ? KC : a.k, kl = KC >= 0 ? KC : a.k_last;
     const int q = lane & 3;
     const uint32_t *un = src + nc + nr;
     const float2 e2 = make_float2(geo.e_scale, geo.e_scale);
@@ -530,7 +530,8 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
 // dense rotation one CTA of kRotDecodeWarps warps, whose shared form of Q^T and per-warp
 // rotation buffers (rot_smem_bytes) come first.
 // MIXED: the last symbol of each block has its own Rice parameter (a.k_last != a.k).
-template <int LAT, bool DITHER, bool KV, bool KSMALL, int MODE, bool ROT = false, bool MIXED = false>
+// KC >= 0: the Rice parameter is KC (= a.k = a.k_last), fixed at compile time.
+template <int LAT, bool DITHER, bool KV, bool KSMALL, int MODE, bool ROT = false, bool MIXED = false, int KC = -1>
 __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, ROT ? 1 : ((DITHER || MIXED) ? 2 : 3))
     decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
@@ -550,7 +551,7 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
         build_sign_table(sign_tab, a.tcols, a.seed);
     __syncthreads();
 
-    const int k = a.k;
+    const int k = KC >= 0 ? KC : a.k;
     uint32_t status = 0;
     // Which rounds this warp decodes: m = 2^lg = 1, 2 or 4 warps share a chunk, 4 / m
     // rounds each, with m as large as the launch's chunks leave warps for.  The warp's
@@ -597,12 +598,12 @@ __global__ void __launch_bounds__((ROT ? kRotDecodeWarps : kWarpsPerCta) * 32, R
         if (staged) {
             const uint32_t *src = stages + buf * kStageSlot;
             ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
-            bad = decode_rounds<LAT, DITHER, KV, KSMALL, true, MODE, ROT, MIXED>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab,
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, true, MODE, ROT, MIXED, KC>(a, geo, src, ok, nc, nr, nu, startbit, sign_tab,
                                                                           rot_s, r0, r1, lane);
         } else {
             const uint32_t *src = cw.src;
             ok = find_segment_starts(src + nc + nr, nu, nsym, nseg, ok, startbit, lane);
-            bad = decode_rounds<LAT, DITHER, KV, KSMALL, false, MODE, ROT, MIXED>(a, geo, src, ok, nc, nr, nu, startbit,
+            bad = decode_rounds<LAT, DITHER, KV, KSMALL, false, MODE, ROT, MIXED, KC>(a, geo, src, ok, nc, nr, nu, startbit,
                                                                            sign_tab, rot_s, r0, r1, lane);
         }
         if (__any_sync(0xffffffffu, bad || (!ok && ntiles > 0))) {

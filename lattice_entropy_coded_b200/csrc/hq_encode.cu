@@ -106,9 +106,20 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
                     : bulk ? (small ? encode_kernel<LAT, DITHER, true, false, true>
                                     : encode_kernel<LAT, DITHER, false, false, true>)
                     : small ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
-        static LaunchPlan plans[5];
-        if ((e = plans[mixed ? 2 : (small ? 1 : 0) + (bulk ? 3 : 0)].grid(
-                 kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta, grid)) != cudaSuccess)
+        int plan_i = mixed ? 2 : (small ? 1 : 0) + (bulk ? 3 : 0);
+        if constexpr (LAT == HQ_E8 && !DITHER) {
+            // E8 weights at the common rates (k = 1 .. 4): the Rice parameter compiled in
+            if (bulk && a.k >= 1 && a.k <= 4) {
+                plan_i = 4 + a.k;
+                kern = a.k == 1   ? encode_kernel<LAT, DITHER, true, false, true, 1>
+                       : a.k == 2 ? encode_kernel<LAT, DITHER, true, false, true, 2>
+                       : a.k == 3 ? encode_kernel<LAT, DITHER, true, false, true, 3>
+                                  : encode_kernel<LAT, DITHER, true, false, true, 4>;
+            }
+        }
+        static LaunchPlan plans[9];
+        if ((e = plans[plan_i].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta,
+                                    grid)) != cudaSuccess)
             return e;
         kern<<<grid, kWarpsPerCta * 32, smem, s>>>(a);
     }

@@ -797,7 +797,8 @@ __device__ __forceinline__ unsigned long long take_ticket(const EncodeArgs &a) {
 // each lane copies its own 64 bytes (prefetch_round).
 // MIXED: the last symbol of each block has its own Rice parameter (a.k_last != a.k),
 // so lanes' remainder runs are not word-aligned (put_rem_mixed).
-template <int LAT, bool DITHER, bool KSMALL, bool MIXED = false, bool BULK = false>
+// KC >= 0: the Rice parameter is KC (= a.k = a.k_last), fixed at compile time.
+template <int LAT, bool DITHER, bool KSMALL, bool MIXED = false, bool BULK = false, int KC = -1>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *sign_tab = smem;                                        // tcols * kSignWords
@@ -822,7 +823,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     __syncthreads();
 
     constexpr int N = Lattice<LAT>::N;
-    const int k = a.k, kl = a.k_last;
+    const int k = KC >= 0 ? KC : a.k, kl = KC >= 0 ? KC : a.k_last;
     const uint32_t lane_bits = 4u * group_rem_bits<N>(k, kl);   // remainder bits of a lane's 32 symbols
     const unsigned long long base = a.base_ptr ? *a.base_ptr : 0ull;
     uint32_t status = 0, zor_all = 0;

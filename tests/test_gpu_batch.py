@@ -12,7 +12,7 @@ import torch
 
 import oracle as O
 import synth
-from hqtest import u16
+from hqtest import rate_points, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -136,3 +136,52 @@ def test_batch_flags_per_item():
     hq.hq_dequantize(w0, cap, o0, rows, cols, params, ref)
     torch.cuda.synchronize()
     assert torch.equal(out[0], ref)
+
+
+def test_student_t_set_as_benched():
+    """The benchmark's launch configuration at its full size: all 64 Student-t matrices of
+    8192 x 8192 (seed 4) coded by one hq_quantize_batch launch and decoded to bf16 by one
+    hq_dequantize_batch launch, at each of the set's operating points (E8 3 and 4 bps).  In
+    items 0, 37 and 63, sampled chunks (and each item's last) are compared word for word with
+    the oracle, which computes any chunk from its row alone, and their bf16 reconstructions
+    with the oracle's; every item's offsets increase and end at its stats' stream_words, with
+    status 0 in both directions."""
+    hq = _hq()
+    B, R, Cc, seed = 64, 8192, 8192, 4
+    x = torch.empty(B, R, Cc, dtype=torch.bfloat16, device="cuda")
+    for i, m in enumerate(synth.student_t(B, R, Cc, seed, device="cuda")):
+        x[i].copy_(m)
+    out = torch.empty_like(x)
+    rng = np.random.default_rng(64)
+    for p in rate_points()["student_t_64x8192x8192_e8"]["points"]:
+        params = hq.make_params("E8", p["alpha"], p["k"], seed, 0)
+        cap = int(R * Cc * (p["bps"] + 3.0) / 32) + 8192            # the bench's capacity
+        _, nch = hq.hq_stream_bound(R, Cc, params)
+        words = torch.empty(B, cap, dtype=torch.int32, device="cuda")
+        offs = torch.empty(B, nch + 1, dtype=torch.int64, device="cuda")
+        st = torch.zeros(B, hq.STATS_BYTES, dtype=torch.uint8, device="cuda")
+        dst = torch.zeros(B, hq.STATS_BYTES, dtype=torch.uint8, device="cuda")
+        ws = torch.empty(hq.hq_batch_workspace_bytes(B, nch), dtype=torch.uint8, device="cuda")
+        hq.hq_quantize_batch(x, params, words, offs, st, ws, cap_words=cap)
+        hq.hq_dequantize_batch(words, cap, offs, R, Cc, params, out, dst)
+        torch.cuda.synchronize()
+        offs_c = offs.cpu().numpy().view(np.uint64)
+        for i in range(B):
+            s = hq.read_stats(st[i])
+            assert s["status"] == 0 and hq.read_stats(dst[i])["status"] == 0, i
+            assert s["stream_words"] == int(offs_c[i, -1]) <= cap
+            assert offs_c[i, 0] == 0 and np.all(np.diff(offs_c[i].astype(np.int64)) > 0)
+        for i in (0, 37, 63):
+            wi = words[i].cpu().numpy().view(np.uint32)
+            for c in [int(v) for v in rng.integers(0, nch, 3)] + [nch - 1]:
+                r, h = divmod(c, 2)                  # 64 tiles per row: chunk c is half h of row r
+                row = x[i, r:r + 1].cpu()
+                ref_w, ref_off, _ = O.quantize(u16(row), O.E8, p["alpha"], p["k"], seed, 0, h, h + 1)
+                a, b = int(offs_c[i, c]), int(offs_c[i, c + 1])
+                assert np.array_equal(wi[a:b], ref_w), (p["bps"], i, c)
+                ref_y = O.dequantize(ref_w, ref_off, 1, Cc, O.E8, p["alpha"], p["k"], seed, 0, False, h, h + 1)
+                got = u16(out[i, r:r + 1])
+                assert np.array_equal(got[0, 4096 * h:4096 * (h + 1)], ref_y[0, 4096 * h:4096 * (h + 1)]), (i, c)
+        del words, offs, ws
+    del x, out
+    torch.cuda.empty_cache()
