@@ -23,12 +23,13 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
     int plan_i = mixed ? 2 : small ? 1 : 0;
     if constexpr (LAT == HQ_E8 && !DITHER && !KV) {
         // E8 weights at the common rates (k = 1 .. 4): the Rice parameter compiled in
-        if (!mixed && a.k >= 1 && a.k <= 4) {
+        // (to bf16, the fp32 store compiled out)
+        if (!mixed && !a.out_fp32 && a.k >= 1 && a.k <= 4) {
             plan_i = 2 + a.k;
-            kern = a.k == 1   ? decode_kernel<LAT, DITHER, KV, true, kStoreTiles, false, false, 1>
-                   : a.k == 2 ? decode_kernel<LAT, DITHER, KV, true, kStoreTiles, false, false, 2>
-                   : a.k == 3 ? decode_kernel<LAT, DITHER, KV, true, kStoreTiles, false, false, 3>
-                              : decode_kernel<LAT, DITHER, KV, true, kStoreTiles, false, false, 4>;
+            kern = a.k == 1   ? decode_kernel<LAT, DITHER, KV, true, kStoreBf16, false, false, 1>
+                   : a.k == 2 ? decode_kernel<LAT, DITHER, KV, true, kStoreBf16, false, false, 2>
+                   : a.k == 3 ? decode_kernel<LAT, DITHER, KV, true, kStoreBf16, false, false, 3>
+                              : decode_kernel<LAT, DITHER, KV, true, kStoreBf16, false, false, 4>;
         }
     }
     static LaunchPlan plans[7];

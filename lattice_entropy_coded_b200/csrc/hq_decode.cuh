@@ -226,12 +226,13 @@ struct ChunkOut {
     // Tile ti of the chunk: destination of its element 0 (null if not stored), sign
     // column, dither counter of element 0, and its position for dot-product outputs
     // (weights: row * tiles per row + tile column; KV: the token, or -1 past len).
+    template <int MODE = kStoreTiles>
     __device__ __forceinline__ bool tile(const DecodeArgs &a, int ti, char *&dst, int &tcol,
                                          unsigned long long &e0, long long &pos) const {
         dst = nullptr;
         pos = -1;
         if (ti >= ntiles) return false;
-        const size_t esz = a.out_fp32 ? 4 : 2;
+        const size_t esz = (MODE != kStoreBf16 && a.out_fp32) ? 4 : 2;
         if (KV) {
             const long long gt = tok0 + tok_base + ti;
             tcol = 0;
@@ -390,7 +391,7 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
         int tcol = 0;
         unsigned long long e0 = 0;
         long long pos = -1;
-        const bool valid = geo.tile(a, r * kTilesPerRound + (lane >> 2), dst, tcol, e0, pos);
+        const bool valid = geo.template tile<MODE>(a, r * kTilesPerRound + (lane >> 2), dst, tcol, e0, pos);
         const uint32_t segi = 32u * r + lane;
         float2 v[16];
         bool lane_ok = ok;
@@ -466,7 +467,7 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
         // a tile is written as zeros unless all four of its lanes decoded
         const unsigned bad_lanes = __ballot_sync(0xffffffffu, valid && !lane_ok);
         const bool tile_bad = (bad_lanes >> (lane & ~3)) & 0xFu;
-        if constexpr (MODE != kStoreTiles) {
+        if constexpr (MODE == kGemvPartials || MODE == kKvScores) {
             // the tile as hq_dequantize stores it in bf16, then dot products with the vector(s)
             const uint32_t es = ROT ? 0u : sign_tab[tcol * kSignWords + q];
             uint32_t w[16];
@@ -495,7 +496,7 @@ __device__ __forceinline__ bool decode_rounds(const DecodeArgs &a, const ChunkOu
 #pragma unroll
                 for (int j = 0; j < 16; j++) v[j] = make_float2(0.0f, 0.0f);
             }
-            if (a.out_fp32) {
+            if (MODE != kStoreBf16 && a.out_fp32) {
                 uint4 *o = reinterpret_cast<uint4 *>(dst) + 8 * q;
 #pragma unroll
                 for (int j = 0; j < 8; j++) {

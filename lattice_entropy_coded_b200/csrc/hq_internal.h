@@ -110,7 +110,9 @@ struct DecodeArgs {
 };
 
 // Decoder outputs: the tile itself, its dot product with x, or its dot products with queries.
-enum DecodeMode { kStoreTiles = 0, kGemvPartials = 1, kKvScores = 2 };
+// kStoreTiles stores bf16 or fp32 (DecodeArgs::out_fp32); kStoreBf16 stores bf16 only
+// (the fp32 store compiled out).
+enum DecodeMode { kStoreTiles = 0, kGemvPartials = 1, kKvScores = 2, kStoreBf16 = 3 };
 
 // Persistent-grid size of one kernel on the current device: SM count x resident CTAs per SM at
 // `smem` dynamic shared bytes, capped at `want` CTAs.  The shared-memory attribute and the
