@@ -32,7 +32,14 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
                               : decode_kernel<LAT, DITHER, KV, true, kStoreBf16, false, false, 4>;
         }
     }
-    static LaunchPlan plans[7];
+    if constexpr (LAT == HQ_E8 && DITHER && KV) {
+        // a KV cache read to bf16 at k = 0 (the KV caches' rates near 2 bits): k compiled in
+        if (!mixed && !a.out_fp32 && a.k == 0) {
+            plan_i = 7;
+            kern = decode_kernel<LAT, DITHER, KV, true, kStoreBf16, false, false, 0>;
+        }
+    }
+    static LaunchPlan plans[8];
     unsigned grid = 0;
     // at most one CTA per round (the kernel deals rounds to CTAs first)
     cudaError_t e = plans[plan_i].grid(kern, kWarpsPerCta * 32, smem, (unsigned long long)kRoundsPerChunk * a.n_chunks,

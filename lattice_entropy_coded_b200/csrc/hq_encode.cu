@@ -117,7 +117,20 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
                                   : encode_kernel<LAT, DITHER, true, false, true, 4>;
             }
         }
-        static LaunchPlan plans[9];
+        if (a.map.kv && !mixed) {
+            // a KV append (a prefill, or many tokens): the weights tile map compiled out, and for
+            // E8 with dither at k = 0 (the KV caches' rates near 2 bits) the Rice parameter too
+            plan_i = 9 + (small ? 1 : 0);
+            kern = small ? encode_kernel<LAT, DITHER, true, false, false, -1, true>
+                         : encode_kernel<LAT, DITHER, false, false, false, -1, true>;
+            if constexpr (LAT == HQ_E8 && DITHER) {
+                if (a.k == 0) {
+                    plan_i = 11;
+                    kern = encode_kernel<LAT, DITHER, true, false, false, 0, true>;
+                }
+            }
+        }
+        static LaunchPlan plans[12];
         if ((e = plans[plan_i].grid(kern, kWarpsPerCta * 32, smem, (a.n_chunks + kWarpsPerCta - 1) / kWarpsPerCta,
                                     grid)) != cudaSuccess)
             return e;

@@ -207,6 +207,10 @@ __device__ __forceinline__ ItemChunk item_chunk(const EncodeArgs &a, unsigned lo
     return r;
 }
 
+// Which tile maps a kernel handles: both (chosen at run time by TileMap::kv), or one known
+// at compile time (the other's code compiled out).
+constexpr int kMapAny = 0, kMapWeights = 1, kMapKv = 2;
+
 // Where the tiles of one chunk are (computed once per chunk).
 struct ChunkGeo {
     int ntiles;
@@ -217,12 +221,12 @@ struct ChunkGeo {
     // kv: head h, tokens tok_base + ti
     long long h, tok_base;
 
-    // KV false: the caller knows the map is a weights matrix (the KV branch is compiled out);
+    // MAP: kMapAny, or the map the caller knows it has (kMapWeights, kMapKv);
     // NARROW: c < 2^27, so the chunk's first tile 32 c fits 32 bits
-    template <bool KV = true, bool NARROW = false>
+    template <int MAP = kMapAny, bool NARROW = false>
     __device__ __forceinline__ void init(const TileMap &m, unsigned long long c) {
         xoff = 0;
-        if (KV && m.kv) {
+        if (MAP == kMapKv || (MAP == kMapAny && m.kv)) {
             const long long cph = (m.tokens + 31) / 32;
             unsigned long long hq_, rq;
             divmod_u64(c, (unsigned long long)cph, hq_, rq);
@@ -248,11 +252,11 @@ struct ChunkGeo {
         }
     }
     // Tile ti (< 32) of the chunk: first element, sign-table column, dither counter of its element 0.
-    template <bool KV = true>
+    template <int MAP = kMapAny>
     __device__ __forceinline__ bool tile(const TileMap &m, const uint16_t *x, int ti, const uint16_t *&src,
                                          int &tcol, unsigned long long &e0) const {
         if (ti >= ntiles) return false;
-        if (KV && m.kv) {
+        if (MAP == kMapKv || (MAP == kMapAny && m.kv)) {
             long long tok = tok_base + ti;
             src = x + h * m.ld_head + tok * m.ld_tok;
             tcol = 0;
@@ -287,12 +291,13 @@ struct RoundInput {
 constexpr int kInSlotWords = 20;     // per-lane input slot of the per-warp kernel (80 B)
 constexpr int kGroupSlotWords = 36;  // grouped kernel: the slot also parks the 32 symbols (144 B)
 
+template <int MAP = kMapAny>
 __device__ __forceinline__ void prefetch_round(const EncodeArgs &a, const ChunkGeo &geo, int r, int lane,
                                                uint32_t *slot) {
     const uint16_t *src = nullptr;
     int tcol;
     unsigned long long e0;
-    if (geo.tile(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, tcol, e0)) {
+    if (geo.template tile<MAP>(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, tcol, e0)) {
         const uint16_t *g = src + 32 * (lane & 3);
 #pragma unroll
         for (int j = 0; j < 4; j++) {
@@ -315,7 +320,7 @@ __device__ __forceinline__ void bulk_prefetch_round(const EncodeArgs &a, const C
     const uint16_t *src = nullptr;
     int tcol;
     unsigned long long e0;
-    geo.tile<false>(a.map, a.x, r * kTilesPerRound, src, tcol, e0);
+    geo.tile<kMapWeights>(a.map, a.x, r * kTilesPerRound, src, tcol, e0);
     // the buffer was last read through the generic proxy (ordered by the caller's __syncwarp)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(kRoundBytes) : "memory");
@@ -336,13 +341,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mb, uint32_t phase, uint32_t 
     return false;
 }
 
-template <bool KV = true>
+template <int MAP = kMapAny>
 __device__ __forceinline__ void round_input(const EncodeArgs &a, const ChunkGeo &geo, int r, int lane,
                                             RoundInput &in) {
     const uint16_t *src = nullptr;
     in.tcol = 0;
     in.e0 = 0;
-    in.valid = geo.template tile<KV>(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, in.tcol, in.e0);
+    in.valid = geo.template tile<MAP>(a.map, a.x, r * kTilesPerRound + (lane >> 2), src, in.tcol, in.e0);
 }
 
 // The transform of one round for one lane: D x -> H_128 (with the three partner
@@ -798,8 +803,10 @@ __device__ __forceinline__ unsigned long long take_ticket(const EncodeArgs &a) {
 // MIXED: the last symbol of each block has its own Rice parameter (a.k_last != a.k),
 // so lanes' remainder runs are not word-aligned (put_rem_mixed).
 // KC >= 0: the Rice parameter is KC (= a.k = a.k_last), fixed at compile time.
-template <int LAT, bool DITHER, bool KSMALL, bool MIXED = false, bool BULK = false, int KC = -1>
+// KVONLY: the launch is a KV append (the weights tile map compiled out).
+template <int LAT, bool DITHER, bool KSMALL, bool MIXED = false, bool BULK = false, int KC = -1, bool KVONLY = false>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const EncodeArgs a) {
+    constexpr int MAP = BULK ? kMapWeights : KVONLY ? kMapKv : kMapAny;
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *sign_tab = smem;                                        // tcols * kSignWords
     uint32_t *stage_all = smem + a.tcols * kSignWords;                // warps * 2 * kStageWords
@@ -834,12 +841,12 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
     if (c < a.n_chunks) {
         const ItemChunk ic = item_chunk<BULK>(a, c);
         ChunkGeo g0;
-        g0.init<!BULK, BULK>(a.map, ic.local);
+        g0.init<MAP, BULK>(a.map, ic.local);
         g0.xoff = (long long)ic.item * a.item_x_stride;
         if (bulk) {
             if (lane == 0) bulk_prefetch_round(a, g0, 0, wbuf_s, mb);
         } else {
-            prefetch_round(a, g0, 0, lane, slot);
+            prefetch_round<MAP>(a, g0, 0, lane, slot);
         }
     }
     Pending pend;
@@ -859,7 +866,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             cur_item = ic.item;
         }
         ChunkGeo geo;
-        geo.init<!BULK, BULK>(a.map, ic.local);
+        geo.init<MAP, BULK>(a.map, ic.local);
         geo.xoff = (long long)ic.item * a.item_x_stride;
         uint32_t *stage = stages + buf * kStageWords;
 
@@ -881,7 +888,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             // this round's bytes are arriving in the lane's slot; take them, then
             // start the copy of the next round's
             RoundInput cur;
-            round_input<!BULK>(a, geo, r, lane, cur);
+            round_input<MAP>(a, geo, r, lane, cur);
             if (bulk) {
                 // a wait that gives up flags the call and waits once more (bounded) for the copy
                 if (!mbar_wait(mb, phase, a.spin_limit)) {
@@ -902,18 +909,18 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
                 } else if (cn < a.n_chunks) {
                     const ItemChunk icn = item_chunk<BULK>(a, cn);
                     ChunkGeo gn;
-                    gn.init<!BULK, BULK>(a.map, icn.local);
+                    gn.init<MAP, BULK>(a.map, icn.local);
                     gn.xoff = (long long)icn.item * a.item_x_stride;
                     if (lane == 0) bulk_prefetch_round(a, gn, 0, wbuf_s, mb);
                 }
             } else if (r + 1 < nrounds) {
-                prefetch_round(a, geo, r + 1, lane, slot);
+                prefetch_round<MAP>(a, geo, r + 1, lane, slot);
             } else if (cn < a.n_chunks) {
                 const ItemChunk icn = item_chunk<BULK>(a, cn);
                 ChunkGeo gn;
-                gn.init<!BULK, BULK>(a.map, icn.local);
+                gn.init<MAP, BULK>(a.map, icn.local);
                 gn.xoff = (long long)icn.item * a.item_x_stride;
-                prefetch_round(a, gn, 0, lane, slot);
+                prefetch_round<MAP>(a, gn, 0, lane, slot);
             }
 
             uint32_t z[32], cbits, rkey;
