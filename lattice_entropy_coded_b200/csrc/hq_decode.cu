@@ -21,7 +21,7 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
     auto kern = mixed ? decode_kernel<LAT, DITHER, KV, false, kStoreTiles, false, true>
                 : small ? decode_kernel<LAT, DITHER, KV, true, kStoreTiles> : decode_kernel<LAT, DITHER, KV, false, kStoreTiles>;
     int plan_i = mixed ? 2 : small ? 1 : 0;
-    if constexpr (LAT == HQ_E8 && !DITHER && !KV) {
+    if constexpr (LAT == HQ_E8 && !KV) {
         // E8 weights at the common rates (k = 1 .. 4): the Rice parameter compiled in
         // (to bf16, the fp32 store compiled out)
         if (!mixed && !a.out_fp32 && a.k >= 1 && a.k <= 4) {

@@ -107,7 +107,7 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
                                     : encode_kernel<LAT, DITHER, false, false, true>)
                     : small ? encode_kernel<LAT, DITHER, true> : encode_kernel<LAT, DITHER, false>;
         int plan_i = mixed ? 2 : (small ? 1 : 0) + (bulk ? 3 : 0);
-        if constexpr (LAT == HQ_E8 && !DITHER) {
+        if constexpr (LAT == HQ_E8) {
             // E8 weights at the common rates (k = 1 .. 4): the Rice parameter compiled in
             if (bulk && a.k >= 1 && a.k <= 4) {
                 plan_i = 4 + a.k;
