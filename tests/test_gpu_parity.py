@@ -68,6 +68,23 @@ def test_every_rice_parameter(k):
     _roundtrip(x, O.E8, 300.0 * 2 ** (k - 2) if k < 8 else 300.0, k, seed=7)
 
 
+@pytest.mark.parametrize("k", [1, 2, 3, 4])
+@pytest.mark.parametrize("dither", [0, 1])
+def test_rice_parameter_compiled_in(k, dither):
+    """E8 weights at k = 1 .. 4 with rows that hold whole rounds (cols a multiple of 1024), forced
+    onto the per-warp form: the bulk-input encoder and the bf16 decoder instantiations with k
+    compiled in (with and without dither), and at k = 0 the runtime-k ones, against the oracle."""
+    hq = _hq()
+    hq.hq_debug_set_encode_path(1)
+    try:
+        x = synth.weight(40, 2048, seed=11)
+        _roundtrip(x, O.E8, 300.0 * 2 ** (k - 2), k, seed=7, dither=dither)
+        if k == 1:
+            _roundtrip(x, O.E8, 40.0, 0, seed=7, dither=dither)
+    finally:
+        hq.hq_debug_set_encode_path(0)
+
+
 def test_strided_rows():
     x = synth.weight(33, 256, seed=4)
     _roundtrip(x, O.E8, 300.0, 2, seed=5, ld=512)
