@@ -65,6 +65,10 @@ def test_kv_appends(path, lat):
     P.test_kv_appends_bit_exact(lat)
 
 
+def test_kv_appends_k0(path):
+    P.test_kv_appends_k0_bit_exact()
+
+
 def test_many_chunks_per_worker(path):
     """4096 x 4096 (4096 chunks): every group or warp encodes several chunks in turn."""
     import lattice_entropy_coded_b200 as hq

@@ -199,6 +199,20 @@ def test_kv_appends_bit_exact(lat):
     _kv_case(4, [256, 100, 1, 31, 312], O.LATTICES[lat], 0.5, 1, seed=77, dither=1, source=K)
 
 
+def test_kv_appends_k0_bit_exact():
+    """E8 with dither at k = 0 (the caches' rates near 2 bits): the KV-only encoder and the bf16
+    read decoder with k compiled in, and a prefill-sized append (one launch of 2048 tokens)."""
+    K, _ = synth.kv(4, 2700, seed=3)
+    cache = _kv_case(4, [256, 100, 1, 31, 312, 2000], O.E8, 0.17, 0, seed=78, dither=1, source=K)
+    # the bf16 read is the round-to-nearest-even of the fp32 read (checked against the oracle above)
+    y32 = torch.empty(4, 2700, 128, device="cuda")
+    y16 = torch.empty(4, 2700, 128, dtype=torch.bfloat16, device="cuda")
+    cache.read(y32)
+    cache.read(y16)
+    torch.cuda.synchronize()
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
 def test_kv_config3_full_size():
     """8 heads x 32768 tokens, appends of 256 tokens, E8 with dither at the calibrated 2.0 bps point."""
     K, V = synth.kv(8, 32768, seed=2)
