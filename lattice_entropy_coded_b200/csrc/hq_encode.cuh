@@ -328,9 +328,10 @@ __device__ __forceinline__ void bulk_prefetch_round(const EncodeArgs &a, const C
                  ::"r"(buf), "l"(src), "r"(kRoundBytes), "r"(mb) : "memory");
 }
 
-// Polls of a round's bulk-copy wait before it gives up: its own bound, far above any copy's
-// latency (seconds), and not the look-back's (which tests lower to one poll): a CTA must not
-// end while a copy into its shared memory is in flight.
+// Polls of a round's bulk-copy wait before it gives up: at least this many, far above any copy's
+// latency (seconds), whatever the look-back's limit (which tests lower to one poll): a CTA must
+// not end while a copy into its shared memory is in flight.  (Taken as spin_limit | this, a run-time
+// value: a compile-time bound made the kernel about 1 % slower.)
 constexpr uint32_t kBulkWaitPolls = 1u << 24;
 
 // Wait for the phase of parity `phase` of mbarrier mb to complete; false after `limit` polls.
@@ -896,9 +897,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2) encode_kernel(const Enco
             round_input<MAP>(a, geo, r, lane, cur);
             if (bulk) {
                 // a wait that gives up flags the call and waits once more (bounded) for the copy
-                if (!mbar_wait(mb, phase, kBulkWaitPolls)) {
+                if (!mbar_wait(mb, phase, a.spin_limit | kBulkWaitPolls)) {
                     status |= HQ_ST_TIMEOUT;
-                    mbar_wait(mb, phase, kBulkWaitPolls);
+                    mbar_wait(mb, phase, a.spin_limit | kBulkWaitPolls);
                 }
                 phase ^= 1u;
             } else {
