@@ -101,17 +101,19 @@ __device__ __noinline__ uint32_t unary_slow(const uint32_t *un, uint32_t nu, uin
 template <bool STAGED>
 __device__ __forceinline__ void unary4(const uint32_t *un, uint32_t nu, uint32_t &bp, bool &ok, uint32_t *q) {
     const uint32_t w = __brev(fetch32<STAGED>(un, nu, bp));
-    if (__popc(w) >= 4) {
-        // quotient i is the count of leading zeros after the first s_i bits, s_i = the
-        // bits of the codewords before it (each quotient plus its terminator); s_i < 32
-        // for i < 4 since the window holds four terminators
-        uint32_t s = 0;
+    // quotient i is the count of leading zeros after the first s_i bits, s_i = the bits of
+    // the codewords before it (each quotient plus its terminator).  The shift saturates at 32
+    // (w << 32 = 0, clz 32), so a window with fewer than 4 terminators ends with s > 32:
+    // the check comes after the counts, with no population count first.
+    uint32_t s = 0, t[4];
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const uint32_t t = __clz(w << s);
-            q[i] = t;
-            s += t + 1u;
-        }
+    for (int i = 0; i < 4; i++) {
+        t[i] = __clz(__funnelshift_lc(0u, w, s));
+        s += t[i] + 1u;
+    }
+    if (s <= 32u) {
+#pragma unroll
+        for (int i = 0; i < 4; i++) q[i] = t[i];
         bp += s;
     } else {
         uint32_t tmp[4];
